@@ -1,0 +1,323 @@
+"""MonarchAttention forward pass in float64 on the CPU: the oracle.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the CPU-baseline
+leg of the benchmark use this file.  It is deliberately plain and slow: numpy
+float64, one step of the method per function, no blocking or fusion beyond
+what the method itself states.  Library primitives (matmul, einsum, exp, log)
+serve as steps.
+
+Parity status: every function below is pinned by ``tests/test_oracle_pins.py``
+against dense softmax attention, closed forms, invariants and brute force.
+The one thing left unpinned is the ViT-B objective table printed in the
+MonarchAttention OpenReview discussion (f(M) = 418, 937, 940, 940 for T = 0..3):
+it needs trained ViT-B weights and ImageNet images, so that table is
+"parity unpinned".
+
+Notation (one head)
+-------------------
+N = b1 * b2 tokens.  Token n = l * b2 + i with l in [b1] (the chunk) and
+i in [b2] (the position inside the chunk); keys are n' = k * b2 + j likewise.
+For a (f, h, w) video latent flattened row-major, the aligned block sizes
+(b1, b2) = (f h, w) give l = (f, h) and i = w (MonarchRT summary, "Key claims":
+the six aligned configurations).
+
+Logits S[(l,i),(k,j)] = sc * q_(l,i) . k_(k,j) with sc = 1 / sqrt(d).
+
+Monarch matrix M = P L P^T R with L, R block diagonal (MonarchRT summary,
+"Method" (1)).  Entry by entry:
+
+    M[(l,i),(k,j)] = L_i[l,k] * R_k[i,j]
+
+Tiled Monarch (MonarchRT summary, "Key claims" and "Method" (2), Theorem 4.1):
+every (i,k) block is cut into c1 x c2 sub-tiles, each independently rank one.
+With p(l) in [c1] the contiguous row group of l and q(j) in [c2] the
+contiguous column group of j:
+
+    M[(l,i),(k,j)] = L_i[l,(k,q(j))] * R_{k,p(l)}[i,j]
+
+Constraints (OpenReview discussion, response to reviewer nTcP: L and R are
+kept positive, "Alternating Maximization with Constraints"): each row of L_i
+lies on the simplex over the b1*c2 pairs (k,q); each row of R_{k,p} lies on the
+simplex separately inside every column group q.  Then M >= 0 and every row of
+M sums to one.  c1 = c2 = 1 is the untiled model.
+
+Softmax variational objective (MonarchAttention AI summary, "Approach";
+OpenReview discussion, f(M) of eq. (6)):
+
+    f(M) = sum over rows of  <M_row, S_row> + H(M_row),   H(m) = -sum m ln m
+
+Over row-stochastic M >= 0 its maximiser is softmax(S) row by row.  For the
+Monarch model the row entropy splits as
+
+    H(M_(l,i)) = H(L_i[l,:]) + sum_{k,q} L_i[l,(k,q)] Hs_{k,p(l),q,i}
+
+with Hs_{k,p,q,i} = H(R_{k,p}[i, j in q]).  Writing
+Kt_{k,p,q,i} = sum_{j in q} R_{k,p}[i,j] k_(k,j):
+
+    f = sum_{l,i} [ sum_{k,q} L_i[l,(k,q)] (sc q_(l,i).Kt_{k,p(l),q,i} + Hs_{k,p(l),q,i})
+                    + H(L_i[l,:]) ]
+
+Alternating maximisation.  With L fixed the objective is concave in R and with
+R fixed concave in L (OpenReview discussion, response to reviewer nTcP on
+concavity); each sub-problem splits into independent entropy-regularised
+linear problems on simplices, whose maximiser is a softmax:
+
+  R-update, for every (k, p, q, i):
+      c  = sum_{l in p} L_i[l,(k,q)]
+      Qt = sum_{l in p} L_i[l,(k,q)] q_(l,i) / c          (the aggregated query)
+      R_{k,p}[i, j in q] = softmax_{j in q}( sc Qt . k_(k,j) )
+  L-update, for every (l, i):
+      L_i[l,(k,q)] = softmax_{(k,q)}( sc q_(l,i).Kt_{k,p(l),q,i} + Hs_{k,p(l),q,i} )
+
+Output without forming the N x N matrix (MonarchRT summary, "Method" (3);
+MonarchAttention abstract: Theta(N sqrt(N) d) compute, Theta(N d) I/O):
+
+    O_(l,i) = sum_{k,q} L_i[l,(k,q)] Y_{k,p(l),q,i},   Y_{k,p,q,i} = sum_{j in q} R_{k,p}[i,j] v_(k,j)
+
+Readings where the pages are silent:
+  * L starts uniform, 1 / (b1 c2); R starts uniform inside every column group.
+  * One step is an R-update followed by an L-update; T = 0 returns the
+    uniform initial Monarch matrix; the output uses the last L and R.
+  * Uneven groups: sizes differ by at most one, larger groups first.
+  * If c == 0 (underflow) the aggregated query is 0 (that R row then is
+    uniform and carries zero weight in M).
+  * Natural logarithm, 0 ln 0 = 0, softmax is max-subtracted.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+# ----------------------------------------------------------------------------
+# helpers
+# ----------------------------------------------------------------------------
+def groups(n: int, c: int):
+    """Split range(n) into c contiguous (start, end) groups.
+
+    Sizes differ by at most one, the larger groups first (945 rows in two
+    groups give 473 and 472).
+    """
+    if not (1 <= c <= n):
+        raise ValueError(f"need 1 <= c <= n, got c={c}, n={n}")
+    base, extra = divmod(n, c)
+    out, s = [], 0
+    for g in range(c):
+        z = base + (1 if g < extra else 0)
+        out.append((s, s + z))
+        s += z
+    return out
+
+
+def _xlogx(p):
+    """p ln p with 0 ln 0 = 0."""
+    pos = p > 0
+    return np.where(pos, p * np.log(np.where(pos, p, 1.0)), 0.0)
+
+
+def _softmax_last(s):
+    m = s.max(axis=-1, keepdims=True)
+    e = np.exp(s - m)
+    return e / e.sum(axis=-1, keepdims=True)
+
+
+def as_heads(x, b1: int, b2: int):
+    """(..., N, d) -> float64 (G, b1, b2, d) with token n = l*b2 + i."""
+    x = np.asarray(x, dtype=np.float64)
+    *lead, N, d = x.shape
+    if N != b1 * b2:
+        raise ValueError(f"N={N} != b1*b2={b1 * b2}")
+    return x.reshape(-1, b1, b2, d), tuple(lead)
+
+
+# ----------------------------------------------------------------------------
+# the two factors
+# ----------------------------------------------------------------------------
+class RFactor:
+    """R_{k,p}[i,j] for all chunks k and row groups p, with its contractions.
+
+    ``R`` has shape (G, b1[k], c1[p], b2[i], b2[j]); inside every column group
+    q the entries of a row sum to one.  From it:
+      Kt (G, b1[k], c1[p], c2[q], b2[i], d) = sum_{j in q} R k_(k,j)
+      Y  (same)                             = sum_{j in q} R v_(k,j)
+      Hs (G, b1[k], c1[p], c2[q], b2[i])    = entropy of R over j in q
+    """
+
+    def __init__(self, R, k, v, cols):
+        self.R = R
+        G, b1, c1, b2, _ = R.shape
+        c2 = len(cols)
+        d, dv = k.shape[-1], v.shape[-1]
+        self.Kt = np.empty((G, b1, c1, c2, b2, d))
+        self.Y = np.empty((G, b1, c1, c2, b2, dv))
+        self.Hs = np.empty((G, b1, c1, c2, b2))
+        for qi, (j0, j1) in enumerate(cols):
+            Rq = R[..., j0:j1]                               # (G, k, p, i, j in q)
+            self.Kt[:, :, :, qi] = Rq @ k[:, :, None, j0:j1]  # (G, k, p, i, d)
+            self.Y[:, :, :, qi] = Rq @ v[:, :, None, j0:j1]
+            self.Hs[:, :, :, qi] = -_xlogx(Rq).sum(axis=-1)
+
+    @classmethod
+    def uniform(cls, k, v, rows, cols):
+        G, b1, b2, _ = k.shape
+        R = np.zeros((G, b1, len(rows), b2, b2))
+        for j0, j1 in cols:
+            R[..., j0:j1] = 1.0 / (j1 - j0)
+        return cls(R, k, v, cols)
+
+
+class LFactor:
+    """L_i[l,(k,q)] for every position i, produced one block at a time.
+
+    ``block(i)`` returns an array of shape (G, b1[l], b1[k], c2[q]) whose rows
+    sum to one over (k, q).  The factor is either uniform, an explicit array
+    of shape (G, b2[i], b1[l], b1[k], c2[q]), or the L-update of an RFactor.
+    """
+
+    def __init__(self, G, b1, b2, rows, cols, *, arr=None, q=None, rf=None, sc=None):
+        self.G, self.b1, self.b2 = G, b1, b2
+        self.rows, self.cols = rows, cols
+        self.arr, self.q, self.rf, self.sc = arr, q, rf, sc
+
+    @classmethod
+    def uniform(cls, G, b1, b2, rows, cols):
+        return cls(G, b1, b2, rows, cols)
+
+    @classmethod
+    def explicit(cls, arr, rows, cols):
+        G, b2, b1, _, _ = arr.shape
+        return cls(G, b1, b2, rows, cols, arr=arr)
+
+    def logits(self, i):
+        """sc q_(l,i).Kt_{k,p(l),q,i} + Hs_{k,p(l),q,i}, shape (G, l, k, q)."""
+        rf, q = self.rf, self.q
+        out = np.empty((self.G, self.b1, self.b1, len(self.cols)))
+        for pi, (l0, l1) in enumerate(self.rows):
+            Kt = rf.Kt[:, :, pi, :, i, :]                     # (G, k, q, d)
+            Hs = rf.Hs[:, :, pi, :, i]                        # (G, k, q)
+            out[:, l0:l1] = self.sc * np.einsum("gld,gkqd->glkq", q[:, l0:l1, i], Kt) \
+                + Hs[:, None]
+        return out
+
+    def block(self, i):
+        c2 = len(self.cols)
+        if self.arr is not None:
+            return self.arr[:, i]
+        if self.rf is None:
+            return np.full((self.G, self.b1, self.b1, c2), 1.0 / (self.b1 * c2))
+        s = self.logits(i)
+        flat = s.reshape(self.G, self.b1, self.b1 * c2)
+        return _softmax_last(flat).reshape(s.shape)
+
+    def materialise(self):
+        return np.stack([self.block(i) for i in range(self.b2)], axis=1)
+
+
+# ----------------------------------------------------------------------------
+# the steps
+# ----------------------------------------------------------------------------
+def r_update(q, k, v, L: LFactor, rows, cols, sc) -> RFactor:
+    """Exact maximiser of f over R with L fixed (a softmax per (k, p, q, i))."""
+    G, b1, b2, d = q.shape
+    c1, c2 = len(rows), len(cols)
+    Qt = np.zeros((G, b1, c1, c2, b2, d))                    # [k, p, q, i]
+    for i in range(b2):
+        Lb = L.block(i)                                      # (G, l, k, q)
+        for pi, (l0, l1) in enumerate(rows):
+            Lp = Lb[:, l0:l1]
+            c = Lp.sum(axis=1)                               # (G, k, q)
+            num = np.einsum("glkq,gld->gkqd", Lp, q[:, l0:l1, i], optimize=True)
+            safe = np.where(c > 0, c, 1.0)
+            Qt[:, :, pi, :, i] = np.where((c > 0)[..., None], num / safe[..., None], 0.0)
+    R = np.empty((G, b1, c1, b2, b2))
+    for pi in range(c1):
+        for qi, (j0, j1) in enumerate(cols):
+            s = sc * (Qt[:, :, pi, qi] @ np.swapaxes(k[:, :, j0:j1], -1, -2))  # (G, k, i, j)
+            R[:, :, pi, :, j0:j1] = _softmax_last(s)
+    return RFactor(R, k, v, cols)
+
+
+def l_update(q, rf: RFactor, rows, cols, sc) -> LFactor:
+    """Exact maximiser of f over L with R fixed (a softmax per row (l, i))."""
+    G, b1, b2, _ = q.shape
+    return LFactor(G, b1, b2, rows, cols, q=q, rf=rf, sc=sc)
+
+
+def output(L: LFactor, rf: RFactor, rows):
+    """O_(l,i) = sum_{k,q} L_i[l,(k,q)] Y_{k,p(l),q,i}; shape (G, b1, b2, d)."""
+    G, b1, _, _, b2, dv = rf.Y.shape
+    O = np.empty((G, b1, b2, dv))
+    for i in range(b2):
+        Lb = L.block(i)
+        for pi, (l0, l1) in enumerate(rows):
+            O[:, l0:l1, i] = np.einsum("glkq,gkqd->gld", Lb[:, l0:l1], rf.Y[:, :, pi, :, i],
+                                       optimize=True)
+    return O
+
+
+def objective(q, L: LFactor, rf: RFactor, rows, sc):
+    """f(M) of the factored Monarch matrix, per head (shape (G,))."""
+    G = q.shape[0]
+    f = np.zeros(G)
+    for i in range(q.shape[2]):
+        Lb = L.block(i)
+        for pi, (l0, l1) in enumerate(rows):
+            lin = sc * np.einsum("gld,gkqd->glkq", q[:, l0:l1, i], rf.Kt[:, :, pi, :, i]) \
+                + rf.Hs[:, :, pi, :, i][:, None]
+            Lp = Lb[:, l0:l1]
+            f += (Lp * lin).sum(axis=(1, 2, 3)) - _xlogx(Lp).sum(axis=(1, 2, 3))
+    return f
+
+
+def materialise(L: LFactor, rf: RFactor, rows, cols):
+    """Dense M (G, N, N) with M[(l,i),(k,j)] = L_i[l,(k,q(j))] R_{k,p(l)}[i,j]."""
+    G, b1, _, b2, _ = rf.R.shape
+    M = np.zeros((G, b1, b2, b1, b2))
+    for i in range(b2):
+        Lb = L.block(i)
+        for pi, (l0, l1) in enumerate(rows):
+            for qi, (j0, j1) in enumerate(cols):
+                M[:, l0:l1, i, :, j0:j1] = Lb[:, l0:l1, :, qi][..., None] \
+                    * rf.R[:, :, pi, i, j0:j1][:, None]
+    return M.reshape(G, b1 * b2, b1 * b2)
+
+
+def dense_logits(q, k):
+    """S = q k^T / sqrt(d) for (G, b1, b2, d) inputs, shape (G, N, N)."""
+    G, b1, b2, d = q.shape
+    qf = q.reshape(G, b1 * b2, d)
+    kf = k.reshape(G, b1 * b2, d)
+    return (qf @ np.swapaxes(kf, -1, -2)) / np.sqrt(d)
+
+
+def objective_dense(M, S):
+    """f(M) = sum M o S - sum M ln M per head, straight from the definition."""
+    return (M * S).sum(axis=(1, 2)) - _xlogx(M).sum(axis=(1, 2))
+
+
+# ----------------------------------------------------------------------------
+# the forward pass
+# ----------------------------------------------------------------------------
+def monarch_attention(q, k, v, b1, b2, T, c1=1, c2=1, return_state=False):
+    """MonarchAttention forward: T alternating steps, then O = M V.
+
+    q, k, v: arrays (..., N, d) with N = b1*b2 (any float dtype; read as
+    float64).  Returns O (..., N, d) in float64; with ``return_state`` also
+    the final (L, R) factors and the head-major inputs.
+    """
+    qh, lead = as_heads(q, b1, b2)
+    kh, _ = as_heads(k, b1, b2)
+    vh, _ = as_heads(v, b1, b2)
+    if T < 0:
+        raise ValueError("T must be >= 0")
+    G, _, _, d = qh.shape
+    sc = 1.0 / np.sqrt(d)
+    rows, cols = groups(b1, c1), groups(b2, c2)
+    L = LFactor.uniform(G, b1, b2, rows, cols)
+    rf = RFactor.uniform(kh, vh, rows, cols)
+    for _ in range(T):
+        rf = r_update(qh, kh, vh, L, rows, cols, sc)
+        L = l_update(qh, rf, rows, cols, sc)
+    O = output(L, rf, rows).reshape(*lead, b1 * b2, vh.shape[-1])
+    if return_state:
+        return O, dict(L=L, R=rf, q=qh, k=kh, v=vh, rows=rows, cols=cols, sc=sc)
+    return O
