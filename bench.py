@@ -1,0 +1,472 @@
+#!/usr/bin/env python
+"""Benchmark of the MonarchAttention forward pass on B200; prints ONE JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl native|reference]
+
+A step is one full forward call (every kernel of the path) over one batch of
+synthetic inputs already resident in device memory.  Inputs rotate over
+several copies whose total exceeds the 126 MB L2 several times, so every step
+reads its Q/K/V from HBM.  Multi-GPU runs (torchrun, one rank per GPU) give
+every rank its own batch (independent heads: weak scaling, no collective on
+the data path) and report the max over ranks of the device time.
+
+Keys beyond the base contract: "e2e" (the same metric through the host-buffer
+C-ABI call, copies included), "roofline" (dominant kernel, CUDA events taken
+live in this run), "cpu_baseline" (the float64 oracle on the host cores, on a
+bounded sample), "clocks" (SM clock and throttle reasons sampled while the
+timed calls run), "gpu_launches" (kernels launched in the timed region).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from structured_sub_quadratic_b200.inputs import WORKLOADS, Workload, make_inputs  # noqa: E402
+
+METRIC = "MonarchAttention fwd ms/call & TFLOP/s at 1 B200; % tensor-pipe/HBM roofline"
+UNIT = "TFLOP/s"
+L2_BYTES = 126 * 2 ** 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# FP32 FFMA peak of the SIMT kernels: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz.
+ALU_FP32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work model
+# ---------------------------------------------------------------------------
+def alg_flops(wl: Workload) -> float:
+    """2 N d [(2T+1) c1 b2 + 2T c2 b1] per head: T R-updates (logits + R K),
+    Y = R V once, T L-updates (logits + aggregation or output)."""
+    N, d, T = wl.N, wl.d, wl.T
+    return wl.heads * 2.0 * N * d * ((2 * T + 1) * wl.c1 * wl.b2 + 2 * T * wl.c2 * wl.b1)
+
+
+def elt_bytes(wl: Workload) -> int:
+    return 4 if wl.dtype == torch.float32 else 2
+
+
+def alg_bytes(wl: Workload) -> float:
+    """Q, K, V read once and O written once: 4 N d elements per head."""
+    return wl.heads * 4.0 * wl.N * wl.d * elt_bytes(wl)
+
+
+def kernel_work(name: str, wl: Workload):
+    """(FLOPs, HBM bytes) one launch of kernel `name` does algorithmically on wl.
+
+    Intermediates (aggregated queries, Kt, Y, entropies) are counted at the
+    width the kernel stores them (fp32 on the SIMT path, bf16 on the
+    tensor-core path); Q/K/V/O at the input width.
+    """
+    G, N, d, b1, b2, c1, c2 = wl.heads, wl.N, wl.d, wl.b1, wl.b2, wl.c1, wl.c2
+    e = elt_bytes(wl)
+    w = 4 if name.startswith("simt") else 2
+    io = G * N * d * e
+    inter = G * N * c1 * c2 * d * w            # one of Kt or Y
+    if name.endswith("init_qt"):
+        return G * N * d, io + G * c1 * b2 * d * w
+    if name.endswith("r_update"):
+        # logits + R K (+ R V on the last step): the last-step launch is timed
+        fl = G * b1 * c1 * b2 * b2 * d * 2 * 3
+        return fl, 2 * io + 2 * inter + G * N * c1 * c2 * 4
+    if name.endswith("l_output"):
+        fl = G * N * b1 * c2 * d * 4
+        return fl, io + 2 * inter + G * N * c1 * c2 * 4 + io
+    if name.endswith("l_stats"):
+        return G * N * b1 * c2 * d * 2, io + inter
+    if name.endswith("l_aggregate"):
+        return G * N * b1 * c2 * d * 4, io + inter + G * N * c1 * c2 * d * w
+    return 0, 0
+
+
+def kernel_bound(name: str):
+    return "alu" if name.startswith("simt") else None
+
+
+# ---------------------------------------------------------------------------
+# distributed helpers (also exercised by the gloo tests)
+# ---------------------------------------------------------------------------
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def reduce_max(x: float, device) -> float:
+    """Max of a scalar over all ranks (identity without a process group)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def job_value(units_per_rank: float, world: int, seconds: float) -> float:
+    """Whole-job throughput: work of all ranks divided by the slowest rank's time."""
+    return units_per_rank * world / seconds
+
+
+# ---------------------------------------------------------------------------
+# measurement helpers
+# ---------------------------------------------------------------------------
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+REASON_BITS = {
+    0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+    0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+    0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+}
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML on a thread."""
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.period = period_s
+        self.samples = []
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            bus = torch.cuda.get_device_properties(device_index).pci_bus_id
+            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.nv = pynvml
+            self.ok = True
+        except Exception as exc:  # NVML missing: report, do not guess
+            self.err = repr(exc)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((mhz, reasons))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": self.err}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        mask = 0
+        for _, r in self.samples:
+            mask |= r
+        reasons = [n for b, n in REASON_BITS.items() if mask & b and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples),
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.samples)}
+
+
+def traffic_for(kernel: str, workload: str):
+    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, or
+    None when the kernel source changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    for line in open(path):
+        f = line.split()
+        if len(f) < 4 or f[0].startswith("#") or f[0] != kernel or f[1] != workload:
+            continue
+        kv = dict(x.split("=", 1) for x in f[2:] if "=" in x)
+        src = os.path.join(ROOT, "structured_sub_quadratic_b200", "csrc", kv.get("src", ""))
+        if not os.path.exists(src):
+            return None
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if sha != kv.get("sha"):
+            return None
+        return float(kv["bytes"])
+    return None
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def oracle_sample(wl: Workload, budget_s: float, heads_per_run: int):
+    """Time the float64 oracle on `heads_per_run` heads of wl, repeatedly,
+    for about budget_s seconds; returns (TFLOP/s, seconds, heads done)."""
+    from oracle import monarch_attention
+    q, k, v = make_inputs(wl)
+    hs = slice(0, heads_per_run)
+    qn, kn, vn = (x.reshape(wl.heads, wl.N, wl.d)[hs].double().numpy() for x in (q, k, v))
+    per_head = alg_flops(wl) / wl.heads
+    done, t0 = 0, time.perf_counter()
+    while True:
+        monarch_attention(qn, kn, vn, wl.b1, wl.b2, wl.T, wl.c1, wl.c2)
+        done += heads_per_run
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return per_head * done / el / 1e12, el, done
+
+
+def heads_for_budget(wl: Workload, target_s: float) -> int:
+    """Heads of wl the oracle processes in about target_s (first estimate from one head)."""
+    from oracle import monarch_attention
+    q, k, v = make_inputs(Workload(**{**wl.__dict__, "B": 1, "H": 1}))
+    t0 = time.perf_counter()
+    monarch_attention(q.double().numpy(), k.double().numpy(), v.double().numpy(),
+                      wl.b1, wl.b2, wl.T, wl.c1, wl.c2)
+    one = time.perf_counter() - t0
+    return max(1, min(wl.heads, int(target_s / max(one, 1e-3))))
+
+
+# ---------------------------------------------------------------------------
+# arms
+# ---------------------------------------------------------------------------
+def run_reference(args, wl):
+    """The oracle as the reference arm, on the host cores (rank 0 only)."""
+    rank, _, world = dist_env()
+    if rank != 0:
+        return 0
+    per_step_heads = heads_for_budget(wl, 0.5)
+    per_head = alg_flops(wl) / wl.heads
+    from oracle import monarch_attention
+    q, k, v = make_inputs(wl)
+    qn, kn, vn = (x.reshape(wl.heads, wl.N, wl.d)[:per_step_heads].double().numpy()
+                  for x in (q, k, v))
+    for _ in range(args.warmup):
+        monarch_attention(qn, kn, vn, wl.b1, wl.b2, wl.T, wl.c1, wl.c2)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        monarch_attention(qn, kn, vn, wl.b1, wl.b2, wl.T, wl.c1, wl.c2)
+    el = time.perf_counter() - t0
+    value = per_head * per_step_heads * args.steps / el / 1e12
+    sample = (f"{per_step_heads} of {wl.heads} heads of the workload per step "
+              f"(float64 numpy oracle)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(wl, None),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(wl: Workload, l2_note):
+    cfg = {"workload": wl.name, "B": wl.B, "H": wl.H, "N": wl.N, "b1": wl.b1, "b2": wl.b2,
+           "d": wl.d, "T": wl.T, "c1": wl.c1, "c2": wl.c2, "inputs": wl.kind, "seed": wl.seed}
+    if wl.latent:
+        cfg["latent_fhw"] = list(wl.latent)
+    if l2_note:
+        cfg["l2"] = l2_note
+    return cfg
+
+
+def run_native(args, wl):
+    from structured_sub_quadratic_b200 import api
+    rank, local_rank, world = dist_env()
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", device_id=device,
+                                timeout=datetime.timedelta(seconds=300))
+    api.load_library()
+    stream = torch.cuda.current_stream(device)
+
+    # rotating device-resident input sets, together several times the L2
+    io_in = 3 * wl.heads * wl.N * wl.d * elt_bytes(wl)
+    n_sets = max(1, min(16, math.ceil(4 * L2_BYTES / io_in)))
+    sets = []
+    for s in range(n_sets):
+        w = Workload(**{**wl.__dict__, "seed": wl.seed + 1000 * rank + s})
+        q, k, v = (x.to(device) for x in make_inputs(w))
+        sets.append((q, k, v, torch.empty_like(q)))
+    l2_note = (f"inputs rotate over {n_sets} device-resident sets "
+               f"({n_sets * io_in / 2**20:.0f} MiB of Q/K/V > 126 MiB L2)")
+
+    def step(s):
+        q, k, v, o = sets[s % n_sets]
+        api.monarch_attn_fwd(q, k, v, wl.b1, wl.b2, wl.T, wl.c1, wl.c2, out=o, stream=stream)
+
+    for s in range(args.warmup):
+        step(s)
+    torch.cuda.synchronize(device)
+    api.check(stream)
+    launches_per_call = api.last_launches()
+
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        barrier(device)
+        torch.cuda.synchronize(device)
+        ev0.record(stream)
+        for s in range(args.steps):
+            step(s)
+        ev1.record(stream)
+        torch.cuda.synchronize(device)
+        barrier(device)
+        ms_local = ev0.elapsed_time(ev1)
+        # keep the same calls running for >= 1 s so the sampler sees the load
+        t_end = time.perf_counter() + max(0.0, 1.0 - ms_local / 1e3)
+        s = 0
+        while time.perf_counter() < t_end:
+            for _ in range(20):
+                step(s)
+                s += 1
+            torch.cuda.synchronize(device)
+    api.check(stream)
+    ms = reduce_max(ms_local, device)
+    flops = alg_flops(wl)
+    value = job_value(flops, world, ms / 1e3) / 1e12
+
+    # per-kernel device time (CUDA events around every launch, same stream)
+    api.timing_read()
+    api.timing_enable(True)
+    for s in range(args.steps):
+        step(s)
+    torch.cuda.synchronize(device)
+    per_kernel = api.timing_read()
+    api.timing_enable(False)
+    roofline = None
+    peaks, peak_src = load_peaks()
+    if per_kernel:
+        name, (tot_ms, n) = max(per_kernel.items(), key=lambda kv: kv[1][0])
+        avg_s = tot_ms / n / 1e3
+        fl, by = kernel_work(name, wl)
+        t_mem = by / (peaks["hbm_gbs"] * 1e9)
+        if kernel_bound(name) == "alu":
+            t_cmp, peak_c, bound_c = fl / (ALU_FP32_TFLOPS * 1e12), ALU_FP32_TFLOPS, "alu"
+        else:
+            t_cmp, peak_c, bound_c = fl / (peaks["bf16_tflops"] * 1e12), peaks["bf16_tflops"], \
+                "tensor"
+        if t_mem >= t_cmp:
+            roofline = {"bound": "hbm", "achieved": by / avg_s / 1e9, "peak": peaks["hbm_gbs"],
+                        "unit": "GB/s"}
+        else:
+            roofline = {"bound": bound_c, "achieved": fl / avg_s / 1e12, "peak": peak_c,
+                        "unit": "TFLOP/s"}
+        roofline["frac"] = roofline["achieved"] / roofline["peak"]
+        roofline["traffic"] = traffic_for(name, args.workload)
+        roofline["kernel"] = name
+        roofline["kernel_ms"] = tot_ms / n
+        roofline["peak_source"] = ("derived: 148 SMs x 128 FP32 lanes x 2 x 1.965 GHz"
+                                   if roofline["bound"] == "alu" else f"{peak_src} (burst)")
+        roofline["kernels"] = {k: {"ms": t / c, "launches_per_call": c / args.steps,
+                                   "share": t / sum(x[0] for x in per_kernel.values())}
+                               for k, (t, c) in per_kernel.items()}
+
+    # end to end through the host-buffer C-ABI call, copies inside the timed region
+    q, k, v, _ = sets[0]
+    qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
+    oh = torch.empty_like(qh).pin_memory()
+    e2e_steps = max(1, min(args.steps, 50))
+    api.monarch_attn_fwd_host(qh, kh, vh, oh, wl.b1, wl.b2, wl.T, wl.c1, wl.c2, stream=stream)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    ev0.record(stream)
+    for _ in range(e2e_steps):
+        api.monarch_attn_fwd_host(qh, kh, vh, oh, wl.b1, wl.b2, wl.T, wl.c1, wl.c2,
+                                  stream=stream)
+    ev1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    e2e_ms = reduce_max(ev0.elapsed_time(ev1) / e2e_steps, device)
+    e2e_value = job_value(flops, world, e2e_ms / 1e3) / 1e12
+    io_elt = wl.heads * wl.N * wl.d * elt_bytes(wl)
+
+    cpu_baseline = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        nh = heads_for_budget(wl, 2.0)
+        val, el, done = oracle_sample(wl, args.cpu_seconds, nh)
+        cpu_baseline = {"value": val, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                        "sample": f"{done} heads of the workload ({nh} per oracle call, "
+                                  f"{el:.1f} s, float64 numpy)"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if wl.dtype == torch.bfloat16 else "f32",
+        "data": "synthetic", "config": workload_config(wl, l2_note),
+        "clocks": clk.summary(),
+        "e2e": {"value": e2e_value, "unit": UNIT, "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": 3 * io_elt, "d2h_bytes_per_step": io_elt},
+        "gpu_launches": launches_per_call * args.steps,
+        "roofline": roofline,
+        "cpu_baseline": cpu_baseline,
+        "path_hbm_frac": (alg_bytes(wl) / (ms / args.steps / 1e3) / 1e9) / peaks["hbm_gbs"],
+        "path_tensor_frac": (flops / (ms / args.steps / 1e3) / 1e12) / peaks["bf16_tflops"],
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        barrier(device)
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="480p", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    wl = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    return run_native(args, wl)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

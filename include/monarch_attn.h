@@ -1,0 +1,152 @@
+/*
+ * monarch_attn.h -- C ABI of the MonarchAttention forward pass on B200 (sm_100a).
+ *
+ * What it computes (one head; the library loops over B*H independent heads):
+ *
+ *   MonarchAttention replaces softmax(Q K^T / sqrt(d)) V by M V, where M is a
+ *   Monarch matrix M = P L P^T R with block-diagonal L and R (MonarchRT
+ *   summary, "Method" (1)) found by T steps of alternating maximisation of
+ *   the softmax variational objective  f(M) = <M, Q K^T / sqrt(d)> + H(M)
+ *   over block rank-one factors (MonarchAttention AI summary, "Approach";
+ *   OpenReview discussion of MonarchAttention, eq. (6) and "Alternating
+ *   Maximization with Constraints").  M V is applied without forming the
+ *   N x N matrix; compute is Theta(N sqrt(N) d) and I/O Theta(N d)
+ *   (MonarchAttention abstract).  The tiled variant cuts every Monarch block
+ *   into c1 x c2 independently rank-one sub-tiles (MonarchRT summary,
+ *   "Key claims", Theorem 4.1; "Method" (2)).
+ *
+ *   Token n = l*b2 + i (l in [b1] the chunk, i in [b2] the position in the
+ *   chunk).  For a (f,h,w) video latent flattened row-major, (b1,b2) = (f*h, w)
+ *   is the aligned (fh,w) layout (MonarchRT summary, "Key claims").
+ *   Row groups p of l and column groups q of j are contiguous, sizes
+ *   differing by at most one, larger groups first.
+ *   One step = R-update then L-update; the initial L and R are uniform;
+ *   T = 0 returns the uniform Monarch matrix applied to V.
+ *
+ * Layout: q, k, v, out are contiguous row-major (B, H, N, d) with
+ *   N = b1*b2, i.e. element (b, h, n, x) at ((b*H + h)*N + n)*d + x.
+ *
+ * Ownership: the caller owns q, k, v, out.  `out` must not overlap any input.
+ *   Device pointers must be 16-byte aligned.  The library owns one cached
+ *   device workspace per device (allocated on first use, grown on demand,
+ *   freed by monarch_attn_release_workspace); calls on one device that may
+ *   overlap on the GPU must be ordered on one stream, because they share it.
+ *
+ * Semantics: asynchronous on `stream` (host-buffer variant excepted).
+ *   Deterministic: no atomics in any reduction.
+ *
+ * Errors: every entry point returns 0 on success or a negative status:
+ *   MONARCH_ERR_INVALID_ARG  null/misaligned pointer, B,H,b1,b2 < 1, T < 0,
+ *                            c1 not in [1,b1], c2 not in [1,b2], size overflow.
+ *   MONARCH_ERR_UNSUPPORTED  d not in [1, 256] (d a multiple of 8 on the
+ *                            tensor-core path, which otherwise falls back).
+ *   MONARCH_ERR_CUDA         a CUDA launch, copy or allocation failed (the
+ *                            CUDA error string is kept, see strerror).
+ *   MONARCH_ERR_DEVICE_TIMEOUT a bounded device wait expired; the kernel
+ *                            stopped and the context stays usable.  Reported
+ *                            by monarch_attn_check() (and by the host-buffer
+ *                            entry point, which checks before returning).
+ *   MONARCH_ERR_NO_MEMORY    the workspace could not be allocated.
+ */
+#ifndef MONARCH_ATTN_H
+#define MONARCH_ATTN_H
+
+#include <stddef.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define MONARCH_API __attribute__((visibility("default")))
+#else
+#define MONARCH_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MONARCH_OK                  0
+#define MONARCH_ERR_INVALID_ARG    -1
+#define MONARCH_ERR_UNSUPPORTED    -2
+#define MONARCH_ERR_CUDA           -3
+#define MONARCH_ERR_DEVICE_TIMEOUT -4
+#define MONARCH_ERR_NO_MEMORY      -5
+
+#define MONARCH_DTYPE_BF16 0
+#define MONARCH_DTYPE_F32  1
+
+/* Kernel path selection (process-wide): AUTO uses the tcgen05 tensor-core
+ * kernels where the shape allows and the SIMT kernels elsewhere; SIMT forces
+ * the SIMT kernels everywhere (used to cross-check the two). */
+#define MONARCH_PATH_AUTO 0
+#define MONARCH_PATH_SIMT 1
+
+/* Forward pass, bf16 in/out, fp32 accumulation.
+ * q, k, v, out: device pointers to __nv_bfloat16, (B, H, N, d), N = b1*b2.
+ * (Pages: MonarchAttention abstract and AI summary "Approach"; MonarchRT
+ * summary "Method" (2)-(3) for c1, c2 > 1.) */
+MONARCH_API int monarch_attn_fwd(const void* q, const void* k, const void* v, void* out,
+                     int B, int H, int b1, int b2, int d, int T, int c1, int c2,
+                     cudaStream_t stream);
+
+/* Same computation with float32 in/out and float32 arithmetic throughout
+ * (no TF32). */
+MONARCH_API int monarch_attn_fwd_f32(const float* q, const float* k, const float* v, float* out,
+                         int B, int H, int b1, int b2, int d, int T, int c1, int c2,
+                         cudaStream_t stream);
+
+/* Same computation on HOST buffers (dtype MONARCH_DTYPE_BF16 or _F32).
+ * Copies q, k, v to cached device staging buffers on `stream`, runs the
+ * forward pass, copies the result into out_host and synchronises `stream`
+ * before returning.  Pinned host memory gives full PCIe/C2C bandwidth;
+ * pageable memory works but is slower. */
+MONARCH_API int monarch_attn_fwd_host(int dtype, const void* q_host, const void* k_host,
+                          const void* v_host, void* out_host,
+                          int B, int H, int b1, int b2, int d, int T, int c1, int c2,
+                          cudaStream_t stream);
+
+/* Bytes of device workspace a call with these arguments uses (0 on invalid
+ * arguments).  dtype is MONARCH_DTYPE_BF16 or MONARCH_DTYPE_F32. */
+MONARCH_API size_t monarch_attn_workspace_bytes(int B, int H, int b1, int b2, int d, int T,
+                                    int c1, int c2, int dtype);
+
+/* Free the cached workspace and staging buffers of every device.  Must not
+ * be called while a forward pass is still running on the GPU. */
+MONARCH_API void monarch_attn_release_workspace(void);
+
+/* Synchronise `stream` and report a device-side failure (a bounded wait that
+ * expired) recorded since the last check; clears the flag. */
+MONARCH_API int monarch_attn_check(cudaStream_t stream);
+
+/* Human-readable text for a status code (includes the last CUDA error text
+ * for MONARCH_ERR_CUDA). */
+MONARCH_API const char* monarch_attn_strerror(int status);
+
+/* Select MONARCH_PATH_AUTO or MONARCH_PATH_SIMT; returns the previous path. */
+MONARCH_API int monarch_attn_set_path(int path);
+
+/* Number of kernels the most recent forward call on this host thread
+ * launched (for launch accounting in benchmarks). */
+MONARCH_API int monarch_attn_last_launches(void);
+
+/* Per-kernel timing (a profiling aid; off by default).  While enabled, every
+ * kernel a forward call launches is bracketed by two CUDA events recorded on
+ * the call's stream.  Returns the previous setting. */
+MONARCH_API int monarch_attn_timing_enable(int enable);
+
+/* Synchronise on the recorded events and report, per kernel name, the summed
+ * device milliseconds and launch count since the previous read (which this
+ * read clears).  Up to max_kernels entries are written: names as
+ * NUL-terminated strings of at most name_len bytes at names + i*name_len,
+ * ms_total[i], launches[i].  Returns the number of distinct kernels, or a
+ * negative status. */
+MONARCH_API int monarch_attn_timing_read(int max_kernels, char* names, int name_len,
+                                         double* ms_total, long* launches);
+
+/* Library version, (major << 16) | minor. */
+MONARCH_API int monarch_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MONARCH_ATTN_H */

@@ -192,10 +192,11 @@ class LFactor:
         rf, q = self.rf, self.q
         out = np.empty((self.G, self.b1, self.b1, len(self.cols)))
         for pi, (l0, l1) in enumerate(self.rows):
-            Kt = rf.Kt[:, :, pi, :, i, :]                     # (G, k, q, d)
-            Hs = rf.Hs[:, :, pi, :, i]                        # (G, k, q)
-            out[:, l0:l1] = self.sc * np.einsum("gld,gkqd->glkq", q[:, l0:l1, i], Kt) \
-                + Hs[:, None]
+            nk = self.b1 * len(self.cols)
+            Kt = rf.Kt[:, :, pi, :, i, :].reshape(self.G, nk, -1)   # (G, (k,q), d)
+            Hs = rf.Hs[:, :, pi, :, i].reshape(self.G, 1, nk)       # (G, 1, (k,q))
+            s = self.sc * (q[:, l0:l1, i] @ np.swapaxes(Kt, -1, -2)) + Hs
+            out[:, l0:l1] = s.reshape(self.G, l1 - l0, self.b1, len(self.cols))
         return out
 
     def block(self, i):
@@ -248,9 +249,10 @@ def output(L: LFactor, rf: RFactor, rows):
     O = np.empty((G, b1, b2, dv))
     for i in range(b2):
         Lb = L.block(i)
+        nk = Lb.shape[2] * Lb.shape[3]
         for pi, (l0, l1) in enumerate(rows):
-            O[:, l0:l1, i] = np.einsum("glkq,gkqd->gld", Lb[:, l0:l1], rf.Y[:, :, pi, :, i],
-                                       optimize=True)
+            Lp = Lb[:, l0:l1].reshape(G, l1 - l0, nk)                # (G, l, (k,q))
+            O[:, l0:l1, i] = Lp @ rf.Y[:, :, pi, :, i].reshape(G, nk, dv)
     return O
 
 
@@ -261,10 +263,12 @@ def objective(q, L: LFactor, rf: RFactor, rows, sc):
     for i in range(q.shape[2]):
         Lb = L.block(i)
         for pi, (l0, l1) in enumerate(rows):
-            lin = sc * np.einsum("gld,gkqd->glkq", q[:, l0:l1, i], rf.Kt[:, :, pi, :, i]) \
-                + rf.Hs[:, :, pi, :, i][:, None]
-            Lp = Lb[:, l0:l1]
-            f += (Lp * lin).sum(axis=(1, 2, 3)) - _xlogx(Lp).sum(axis=(1, 2, 3))
+            nk = Lb.shape[2] * Lb.shape[3]
+            Kt = rf.Kt[:, :, pi, :, i].reshape(G, nk, -1)
+            lin = sc * (q[:, l0:l1, i] @ np.swapaxes(Kt, -1, -2)) \
+                + rf.Hs[:, :, pi, :, i].reshape(G, 1, nk)
+            Lp = Lb[:, l0:l1].reshape(G, l1 - l0, nk)
+            f += (Lp * lin).sum(axis=(1, 2)) - _xlogx(Lp).sum(axis=(1, 2))
     return f
 
 

@@ -1,0 +1,317 @@
+// C ABI of the MonarchAttention forward pass (declared in include/monarch_attn.h).
+//
+// This file validates arguments, owns the per-device workspace cache and the
+// device status word, and dispatches to the kernels: the tcgen05 tensor-core
+// path for the bf16 shapes it supports, the SIMT path for everything else.
+#include "monarch_attn.h"
+
+#include <atomic>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "simt_kernels.cuh"
+#include "tc_path.cuh"
+
+namespace {
+
+using monarch::Problem;
+
+constexpr int kMaxDevices = 64;
+constexpr size_t kAlign = 256;
+
+struct DevBuf {
+  void* ptr = nullptr;
+  size_t bytes = 0;
+};
+
+std::mutex g_mu;                // workspace and status words
+std::mutex g_stage_mu;          // held for a whole host-buffer call
+DevBuf g_ws[kMaxDevices];      // kernel workspace
+DevBuf g_stage[kMaxDevices];   // staging for the host-buffer entry point
+int* g_status[kMaxDevices];    // device status word (bounded-wait timeouts)
+std::atomic<int> g_path{MONARCH_PATH_AUTO};
+thread_local int t_launches = 0;
+thread_local char t_err[256] = "";
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+int record_cuda(cudaError_t e) {
+  std::snprintf(t_err, sizeof(t_err), "CUDA error: %s", cudaGetErrorString(e));
+  return MONARCH_ERR_CUDA;
+}
+
+bool mul_ok(size_t a, size_t b, size_t* out) {
+  if (a != 0 && b > SIZE_MAX / a) return false;
+  *out = a * b;
+  return true;
+}
+
+int validate(int B, int H, int b1, int b2, int d, int T, int c1, int c2) {
+  if (B < 1 || H < 1 || b1 < 1 || b2 < 1 || T < 0) return MONARCH_ERR_INVALID_ARG;
+  if (c1 < 1 || c1 > b1 || c2 < 1 || c2 > b2) return MONARCH_ERR_INVALID_ARG;
+  if (d < 1 || d > 256) return MONARCH_ERR_UNSUPPORTED;
+  size_t n;
+  if (!mul_ok((size_t)B, (size_t)H, &n) || !mul_ok(n, (size_t)b1, &n) ||
+      !mul_ok(n, (size_t)b2, &n) || !mul_ok(n, (size_t)d, &n) || !mul_ok(n, (size_t)c1, &n) ||
+      !mul_ok(n, (size_t)c2, &n) || n > ((size_t)1 << 40))
+    return MONARCH_ERR_INVALID_ARG;
+  if ((long long)B * H > (1LL << 30)) return MONARCH_ERR_INVALID_ARG;
+  return MONARCH_OK;
+}
+
+bool aligned16(const void* p) { return p != nullptr && ((uintptr_t)p & 15u) == 0; }
+
+Problem make_problem(int B, int H, int b1, int b2, int d, int T, int c1, int c2) {
+  Problem pb;
+  pb.G = B * H;
+  pb.b1 = b1;
+  pb.b2 = b2;
+  pb.d = d;
+  pb.T = T;
+  pb.c1 = c1;
+  pb.c2 = c2;
+  pb.sc = 1.0f / sqrtf((float)d);
+  return pb;
+}
+
+// Workspace of one call: the tensor-core path's if it takes the shape, else
+// the SIMT path's (fp32 pieces, each 256-byte aligned).
+struct Plan {
+  bool tc = false;
+  size_t bytes = 0;
+  monarch::SimtWorkspaceSizes simt{};
+};
+
+Plan make_plan(const Problem& pb, int dtype) {
+  Plan pl;
+  if (dtype == MONARCH_DTYPE_BF16 && g_path.load() == MONARCH_PATH_AUTO &&
+      monarch::tc_supports(pb)) {
+    pl.tc = true;
+    pl.bytes = monarch::tc_workspace_bytes(pb);
+    return pl;
+  }
+  pl.simt = monarch::simt_workspace_sizes(pb);
+  const size_t* f = &pl.simt.qt0;
+  for (int t = 0; t < 7; ++t) pl.bytes += align_up(f[t] * sizeof(float));
+  return pl;
+}
+
+monarch::SimtWorkspace carve_simt(const Plan& pl, char* base) {
+  monarch::SimtWorkspace ws;
+  float** dst = &ws.qt0;
+  const size_t* f = &pl.simt.qt0;
+  size_t off = 0;
+  for (int t = 0; t < 7; ++t) {
+    dst[t] = f[t] ? reinterpret_cast<float*>(base + off) : nullptr;
+    off += align_up(f[t] * sizeof(float));
+  }
+  return ws;
+}
+
+int current_device(int* dev) {
+  cudaError_t e = cudaGetDevice(dev);
+  if (e != cudaSuccess) return record_cuda(e);
+  if (*dev < 0 || *dev >= kMaxDevices) return MONARCH_ERR_UNSUPPORTED;
+  return MONARCH_OK;
+}
+
+// Grow-only cached device buffer.  cudaFree synchronises the device, so a
+// buffer still used by an earlier call is never freed under it.
+int ensure(DevBuf& b, size_t bytes) {
+  if (bytes <= b.bytes) return MONARCH_OK;
+  if (b.ptr) {
+    cudaError_t e = cudaFree(b.ptr);
+    b.ptr = nullptr;
+    b.bytes = 0;
+    if (e != cudaSuccess) return record_cuda(e);
+  }
+  cudaError_t e = cudaMalloc(&b.ptr, bytes);
+  if (e != cudaSuccess) {
+    b.ptr = nullptr;
+    cudaGetLastError();
+    std::snprintf(t_err, sizeof(t_err), "workspace allocation of %zu bytes failed: %s", bytes,
+                  cudaGetErrorString(e));
+    return MONARCH_ERR_NO_MEMORY;
+  }
+  b.bytes = bytes;
+  return MONARCH_OK;
+}
+
+int ensure_status(int dev) {
+  if (g_status[dev]) return MONARCH_OK;
+  int* p = nullptr;
+  cudaError_t e = cudaMalloc(&p, kAlign);
+  if (e != cudaSuccess) return record_cuda(e);
+  e = cudaMemset(p, 0, kAlign);
+  if (e != cudaSuccess) {
+    cudaFree(p);
+    return record_cuda(e);
+  }
+  g_status[dev] = p;
+  return MONARCH_OK;
+}
+
+template <typename TIn>
+int forward_device(const TIn* q, const TIn* k, const TIn* v, TIn* out, int B, int H, int b1,
+                   int b2, int d, int T, int c1, int c2, cudaStream_t stream, int dtype) {
+  t_launches = 0;
+  int st = validate(B, H, b1, b2, d, T, c1, c2);
+  if (st != MONARCH_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return MONARCH_ERR_INVALID_ARG;
+  const Problem pb = make_problem(B, H, b1, b2, d, T, c1, c2);
+  const size_t bytes_io = (size_t)pb.G * b1 * b2 * d * sizeof(TIn);
+  const char* o0 = reinterpret_cast<const char*>(out);
+  for (const void* in : {(const void*)q, (const void*)k, (const void*)v}) {
+    const char* i0 = reinterpret_cast<const char*>(in);
+    if (o0 < i0 + bytes_io && i0 < o0 + bytes_io) return MONARCH_ERR_INVALID_ARG;
+  }
+  int dev;
+  if ((st = current_device(&dev)) != MONARCH_OK) return st;
+  const Plan pl = make_plan(pb, dtype);
+  std::lock_guard<std::mutex> lock(g_mu);
+  if ((st = ensure_status(dev)) != MONARCH_OK) return st;
+  if ((st = ensure(g_ws[dev], pl.bytes ? pl.bytes : kAlign)) != MONARCH_OK) return st;
+  cudaError_t e;
+  if (pl.tc) {
+    e = monarch::tc_forward(reinterpret_cast<const monarch::bf16*>(q),
+                            reinterpret_cast<const monarch::bf16*>(k),
+                            reinterpret_cast<const monarch::bf16*>(v),
+                            reinterpret_cast<monarch::bf16*>(out), pb,
+                            static_cast<char*>(g_ws[dev].ptr), g_status[dev], stream,
+                            &t_launches);
+  } else {
+    const monarch::SimtWorkspace ws = carve_simt(pl, static_cast<char*>(g_ws[dev].ptr));
+    e = monarch::simt_forward<TIn>(q, k, v, out, pb, ws, stream, &t_launches);
+  }
+  if (e != cudaSuccess) return record_cuda(e);
+  return MONARCH_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int monarch_attn_fwd(const void* q, const void* k, const void* v, void* out, int B, int H,
+                     int b1, int b2, int d, int T, int c1, int c2, cudaStream_t stream) {
+  using monarch::bf16;
+  return forward_device<bf16>(static_cast<const bf16*>(q), static_cast<const bf16*>(k),
+                              static_cast<const bf16*>(v), static_cast<bf16*>(out), B, H, b1, b2,
+                              d, T, c1, c2, stream, MONARCH_DTYPE_BF16);
+}
+
+int monarch_attn_fwd_f32(const float* q, const float* k, const float* v, float* out, int B,
+                         int H, int b1, int b2, int d, int T, int c1, int c2,
+                         cudaStream_t stream) {
+  return forward_device<float>(q, k, v, out, B, H, b1, b2, d, T, c1, c2, stream,
+                               MONARCH_DTYPE_F32);
+}
+
+int monarch_attn_fwd_host(int dtype, const void* q_host, const void* k_host, const void* v_host,
+                          void* out_host, int B, int H, int b1, int b2, int d, int T, int c1,
+                          int c2, cudaStream_t stream) {
+  if (dtype != MONARCH_DTYPE_BF16 && dtype != MONARCH_DTYPE_F32) return MONARCH_ERR_INVALID_ARG;
+  if (!q_host || !k_host || !v_host || !out_host) return MONARCH_ERR_INVALID_ARG;
+  int st = validate(B, H, b1, b2, d, T, c1, c2);
+  if (st != MONARCH_OK) return st;
+  const size_t elt = dtype == MONARCH_DTYPE_BF16 ? 2 : 4;
+  const size_t n = (size_t)B * H * b1 * b2 * d * elt;
+  const size_t slot = align_up(n);
+  int dev;
+  if ((st = current_device(&dev)) != MONARCH_OK) return st;
+  std::lock_guard<std::mutex> stage_lock(g_stage_mu);
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if ((st = ensure(g_stage[dev], 4 * slot)) != MONARCH_OK) return st;
+  }
+  char* base = static_cast<char*>(g_stage[dev].ptr);
+  char *dq = base, *dk = base + slot, *dv = base + 2 * slot, *dout = base + 3 * slot;
+  cudaError_t e;
+  if ((e = cudaMemcpyAsync(dq, q_host, n, cudaMemcpyHostToDevice, stream)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(dk, k_host, n, cudaMemcpyHostToDevice, stream)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(dv, v_host, n, cudaMemcpyHostToDevice, stream)) != cudaSuccess)
+    return record_cuda(e);
+  st = dtype == MONARCH_DTYPE_BF16
+           ? monarch_attn_fwd(dq, dk, dv, dout, B, H, b1, b2, d, T, c1, c2, stream)
+           : monarch_attn_fwd_f32(reinterpret_cast<float*>(dq), reinterpret_cast<float*>(dk),
+                                  reinterpret_cast<float*>(dv), reinterpret_cast<float*>(dout), B,
+                                  H, b1, b2, d, T, c1, c2, stream);
+  if (st != MONARCH_OK) return st;
+  if ((e = cudaMemcpyAsync(out_host, dout, n, cudaMemcpyDeviceToHost, stream)) != cudaSuccess)
+    return record_cuda(e);
+  return monarch_attn_check(stream);
+}
+
+size_t monarch_attn_workspace_bytes(int B, int H, int b1, int b2, int d, int T, int c1, int c2,
+                                    int dtype) {
+  if (validate(B, H, b1, b2, d, T, c1, c2) != MONARCH_OK) return 0;
+  if (dtype != MONARCH_DTYPE_BF16 && dtype != MONARCH_DTYPE_F32) return 0;
+  return make_plan(make_problem(B, H, b1, b2, d, T, c1, c2), dtype).bytes;
+}
+
+void monarch_attn_release_workspace(void) {
+  std::lock_guard<std::mutex> stage_lock(g_stage_mu);
+  std::lock_guard<std::mutex> lock(g_mu);
+  int cur = 0;
+  cudaGetDevice(&cur);
+  for (int dev = 0; dev < kMaxDevices; ++dev) {
+    if (!g_ws[dev].ptr && !g_stage[dev].ptr && !g_status[dev]) continue;
+    cudaSetDevice(dev);
+    if (g_ws[dev].ptr) cudaFree(g_ws[dev].ptr);
+    if (g_stage[dev].ptr) cudaFree(g_stage[dev].ptr);
+    if (g_status[dev]) cudaFree(g_status[dev]);
+    g_ws[dev] = DevBuf();
+    g_stage[dev] = DevBuf();
+    g_status[dev] = nullptr;
+  }
+  cudaSetDevice(cur);
+}
+
+int monarch_attn_check(cudaStream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return record_cuda(e);
+  int dev;
+  int st = current_device(&dev);
+  if (st != MONARCH_OK) return st;
+  int* p;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    p = g_status[dev];
+  }
+  if (!p) return MONARCH_OK;
+  int flag = 0;
+  if ((e = cudaMemcpy(&flag, p, sizeof(int), cudaMemcpyDeviceToHost)) != cudaSuccess)
+    return record_cuda(e);
+  if (flag) {
+    if ((e = cudaMemset(p, 0, sizeof(int))) != cudaSuccess) return record_cuda(e);
+    return MONARCH_ERR_DEVICE_TIMEOUT;
+  }
+  return MONARCH_OK;
+}
+
+const char* monarch_attn_strerror(int status) {
+  switch (status) {
+    case MONARCH_OK: return "ok";
+    case MONARCH_ERR_INVALID_ARG:
+      return "invalid argument (null or misaligned pointer, overlapping output, or a size out "
+             "of range)";
+    case MONARCH_ERR_UNSUPPORTED: return "unsupported shape (d must be in [1, 256])";
+    case MONARCH_ERR_CUDA: return t_err[0] ? t_err : "CUDA error";
+    case MONARCH_ERR_DEVICE_TIMEOUT:
+      return "a bounded device wait expired; the kernel stopped early and its output is invalid";
+    case MONARCH_ERR_NO_MEMORY: return t_err[0] ? t_err : "workspace allocation failed";
+    default: return "unknown status";
+  }
+}
+
+int monarch_attn_set_path(int path) {
+  if (path != MONARCH_PATH_AUTO && path != MONARCH_PATH_SIMT) return -1;
+  return g_path.exchange(path);
+}
+
+int monarch_attn_last_launches(void) { return t_launches; }
+
+int monarch_attn_version(void) { return (0 << 16) | 1; }
+
+}  // extern "C"

@@ -1,0 +1,35 @@
+// Host-side interface of the SIMT (general-shape) MonarchAttention kernels.
+#pragma once
+
+#include <algorithm>
+#include <stddef.h>
+
+#include "common.cuh"
+
+namespace monarch {
+
+// Element strides of the aggregated-query buffer read by the R-update:
+// qt row (g, k, p, q, i) starts at g*g_ + k*k_ + p*p_ + q*q_ + i*i_.
+// Step one reads the uniform-L means Qt0[g][p][i] (k and q strides 0).
+struct QtStrides {
+  long g, k, p, q, i;
+};
+
+// fp32 workspace pieces (element counts), see simt_kernels.cu for layouts.
+struct SimtWorkspaceSizes {
+  size_t qt0, qt, kt, y, hs, lse, ybar;
+};
+
+struct SimtWorkspace {
+  float *qt0, *qt, *kt, *y, *hs, *lse, *ybar;
+};
+
+SimtWorkspaceSizes simt_workspace_sizes(const Problem& pb);
+
+// Runs the whole forward pass on `stream`; adds the number of kernels it
+// launched to *launches.
+template <typename TIn>
+cudaError_t simt_forward(const TIn* q, const TIn* k, const TIn* v, TIn* out, const Problem& pb,
+                         const SimtWorkspace& ws, cudaStream_t stream, int* launches);
+
+}  // namespace monarch

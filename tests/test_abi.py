@@ -1,0 +1,92 @@
+"""The C-ABI library builds, loads and exports every symbol its header
+declares; argument validation answers without touching the GPU.  CPU only:
+no forward pass is run here."""
+import re
+import subprocess
+
+import pytest
+
+from structured_sub_quadratic_b200 import _build, api
+
+HEADER = _build.os.path.join(_build.INCLUDE, "monarch_attn.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return set(re.findall(r"^MONARCH_API\s+[\w\s\*]+?\b(monarch_attn_\w+)\s*\(", text, re.M))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    _build.build()
+    return api.load_library()
+
+
+def test_header_and_binding_agree():
+    syms = declared_symbols()
+    assert len(syms) >= 10
+    assert syms == set(api.SIGNATURES)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", _build.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT\s+(monarch_attn_\w+)$", out, re.M))
+    assert declared_symbols() <= exported
+    for name in declared_symbols():
+        assert getattr(lib, name) is not None
+
+
+def test_library_targets_sm100a_only():
+    out = subprocess.run(["cuobjdump", "--list-elf", _build.LIB_PATH], capture_output=True,
+                         text=True)
+    if out.returncode != 0:
+        pytest.skip("cuobjdump unavailable")
+    archs = set(re.findall(r"sm_(\d+a?)", out.stdout))
+    assert archs == {"100a"}
+
+
+def test_version_and_strerror(lib):
+    assert lib.monarch_attn_version() >= 1
+    for st in (0, -1, -2, -3, -4, -5, 7):
+        assert lib.monarch_attn_strerror(st)
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((0, 1, 4, 4, 64, 1, 1, 1), api.MONARCH_ERR_INVALID_ARG),     # B < 1
+    ((1, 1, 0, 4, 64, 1, 1, 1), api.MONARCH_ERR_INVALID_ARG),     # b1 < 1
+    ((1, 1, 4, 4, 64, -1, 1, 1), api.MONARCH_ERR_INVALID_ARG),    # T < 0
+    ((1, 1, 4, 4, 64, 1, 5, 1), api.MONARCH_ERR_INVALID_ARG),     # c1 > b1
+    ((1, 1, 4, 4, 64, 1, 1, 0), api.MONARCH_ERR_INVALID_ARG),     # c2 < 1
+    ((1, 1, 4, 4, 512, 1, 1, 1), api.MONARCH_ERR_UNSUPPORTED),    # d > 256
+])
+def test_invalid_arguments_are_rejected_before_any_launch(lib, args, expect):
+    # valid-looking (aligned, non-null) fake pointers: validation fails first
+    p = 1 << 20
+    assert lib.monarch_attn_fwd(p, 2 * p, 3 * p, 4 * p, *args, None) == expect
+    assert lib.monarch_attn_workspace_bytes(*args, 0) == 0
+
+
+def test_null_misaligned_and_overlapping_pointers_are_rejected(lib):
+    p = 1 << 20
+    sizes = (1, 1, 4, 4, 64, 1, 1, 1)
+    assert lib.monarch_attn_fwd(None, p, p, p, *sizes, None) == api.MONARCH_ERR_INVALID_ARG
+    assert lib.monarch_attn_fwd(p + 2, 2 * p, 3 * p, 4 * p, *sizes, None) == \
+        api.MONARCH_ERR_INVALID_ARG
+    # out overlapping q (16*64*2 bytes of q starting at p)
+    assert lib.monarch_attn_fwd(p, 2 * p, 3 * p, p + 256, *sizes, None) == \
+        api.MONARCH_ERR_INVALID_ARG
+    assert lib.monarch_attn_fwd_host(9, p, p, p, p, *sizes, None) == api.MONARCH_ERR_INVALID_ARG
+
+
+def test_workspace_bytes_scale_with_shape(lib):
+    w1 = lib.monarch_attn_workspace_bytes(1, 12, 90, 52, 128, 1, 1, 1, 0)
+    w2 = lib.monarch_attn_workspace_bytes(2, 12, 90, 52, 128, 1, 1, 1, 0)
+    w3 = lib.monarch_attn_workspace_bytes(1, 12, 90, 52, 128, 2, 1, 1, 0)
+    assert 0 < w1 < w2 and w1 < w3
+
+
+def test_path_switch_round_trips(lib):
+    prev = lib.monarch_attn_set_path(api.PATH_SIMT)
+    assert lib.monarch_attn_set_path(prev) == api.PATH_SIMT
+    assert lib.monarch_attn_set_path(7) == -1
