@@ -20,13 +20,13 @@ from __future__ import annotations
 
 import argparse
 import datetime
+import faulthandler
 import hashlib
 import json
 import math
 import os
 import statistics
 import sys
-import threading
 import time
 
 import torch
@@ -35,6 +35,14 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from structured_sub_quadratic_b200.inputs import WORKLOADS, Workload, make_inputs  # noqa: E402
+
+faulthandler.enable()
+
+
+def log(msg):
+    """Progress marker on stderr (stdout carries only the JSON line)."""
+    print(f"[bench] {msg}", file=sys.stderr, flush=True)
+
 
 METRIC = "MonarchAttention fwd ms/call & TFLOP/s at 1 B200; % tensor-pipe/HBM roofline"
 UNIT = "TFLOP/s"
@@ -139,65 +147,78 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-REASON_BITS = {
-    0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
-    0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
-    0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
-}
+SMI_FIELDS = ["pci.bus_id", "clocks.sm", "clocks.max.sm", "power.draw",
+              "clocks_event_reasons.active", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+REASON_COLS = {"clocks_event_reasons.hw_slowdown": "hw_slowdown",
+               "clocks_event_reasons.hw_thermal_slowdown": "hw_thermal_slowdown",
+               "clocks_event_reasons.sw_thermal_slowdown": "sw_thermal_slowdown",
+               "clocks_event_reasons.sw_power_cap": "sw_power_cap"}
 
 
 class ClockSampler:
-    """Samples SM clock and clock-event reasons through NVML on a thread."""
+    """Samples SM clock and throttle reasons with `nvidia-smi -lms` while the
+    timed calls run, keeping the rows of this process's GPU (matched by PCI
+    bus id, since nvidia-smi numbers GPUs differently from CUDA)."""
 
-    def __init__(self, device_index: int, period_s: float = 0.02):
-        self.period = period_s
-        self.samples = []
-        self.ok = False
-        self._stop = threading.Event()
+    def __init__(self, device_index: int, period_ms: int = 100, enabled: bool = True):
+        self.period_ms = period_ms
+        self.enabled = enabled
+        self.err = "clock sampling disabled" if not enabled else None
+        self.rows = []
         try:
-            import pynvml
-            pynvml.nvmlInit()
-            bus = torch.cuda.get_device_properties(device_index).pci_bus_id
-            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
-            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
-            self.nv = pynvml
-            self.ok = True
-        except Exception as exc:  # NVML missing: report, do not guess
-            self.err = repr(exc)
-
-    def _run(self):
-        nv = self.nv
-        while not self._stop.is_set():
-            try:
-                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
-                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                self.samples.append((mhz, reasons))
-            except Exception:
-                pass
-            time.sleep(self.period)
+            pr = torch.cuda.get_device_properties(device_index)
+            self.bus = f"{int(pr.pci_bus_id):02X}:{int(pr.pci_device_id):02X}.0"  # "1B:00.0"
+        except Exception as exc:
+            self.enabled, self.err = False, repr(exc)
 
     def __enter__(self):
-        if self.ok:
-            self.t = threading.Thread(target=self._run, daemon=True)
-            self.t.start()
+        import subprocess
+        import tempfile
+        if not self.enabled:
+            return self
+        self.tmp = tempfile.TemporaryFile(mode="w+")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + ",".join(SMI_FIELDS), "--format=csv,noheader",
+                 "-lms", str(self.period_ms)], stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except Exception as exc:
+            self.enabled, self.err = False, repr(exc)
         return self
 
     def __exit__(self, *a):
-        if self.ok:
-            self._stop.set()
-            self.t.join()
+        if not self.enabled:
+            return
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=10)
+        except Exception:
+            self.proc.kill()
+        self.tmp.seek(0)
+        for line in self.tmp:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) == len(SMI_FIELDS) and f[0].upper().endswith(self.bus):
+                self.rows.append(dict(zip(SMI_FIELDS, f)))
+        self.tmp.close()
 
     def summary(self):
-        if not self.ok:
+        if not self.enabled:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": self.err}
-        if not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
-        mask = 0
-        for _, r in self.samples:
-            mask |= r
-        reasons = [n for b, n in REASON_BITS.items() if mask & b and n != "gpu_idle"]
-        return {"sm_mhz": statistics.median(m for m, _ in self.samples),
-                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.samples)}
+        def num(x):
+            try:
+                return float(x.split()[0])
+            except Exception:
+                return None
+        mhz = [num(r["clocks.sm"]) for r in self.rows if num(r["clocks.sm"])]
+        reasons = sorted({name for r in self.rows for col, name in REASON_COLS.items()
+                          if r[col].lower() == "active"})
+        return {"sm_mhz": statistics.median(mhz) if mhz else None,
+                "sm_max_mhz": num(self.rows[0]["clocks.max.sm"]) if self.rows else None,
+                "reasons": reasons, "samples": len(self.rows),
+                "power_w_max": max((num(r["power.draw"]) or 0) for r in self.rows)
+                if self.rows else None,
+                "window": "the timed calls plus the same calls repeated to >= 1 s"}
 
 
 def traffic_for(kernel: str, workload: str):
@@ -317,6 +338,7 @@ def run_native(args, wl):
                                 timeout=datetime.timedelta(seconds=300))
     api.load_library()
     stream = torch.cuda.current_stream(device)
+    log("library loaded")
 
     # rotating device-resident input sets, together several times the L2
     io_in = 3 * wl.heads * wl.N * wl.d * elt_bytes(wl)
@@ -333,14 +355,16 @@ def run_native(args, wl):
         q, k, v, o = sets[s % n_sets]
         api.monarch_attn_fwd(q, k, v, wl.b1, wl.b2, wl.T, wl.c1, wl.c2, out=o, stream=stream)
 
+    log(f"{n_sets} input sets on device")
     for s in range(args.warmup):
         step(s)
     torch.cuda.synchronize(device)
     api.check(stream)
+    log("warm-up done")
     launches_per_call = api.last_launches()
 
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local_rank) as clk:
+    with ClockSampler(local_rank, enabled=not args.no_clocks) as clk:
         barrier(device)
         torch.cuda.synchronize(device)
         ev0.record(stream)
@@ -359,9 +383,10 @@ def run_native(args, wl):
                 s += 1
             torch.cuda.synchronize(device)
     api.check(stream)
+    log(f"timed region done: {ms_local:.3f} ms; clocks {clk.summary()}")
     ms = reduce_max(ms_local, device)
     flops = alg_flops(wl)
-    value = job_value(flops, world, ms / 1e3) / 1e12
+    value = job_value(flops * args.steps, world, ms / 1e3) / 1e12
 
     # per-kernel device time (CUDA events around every launch, same stream)
     api.timing_read()
@@ -371,6 +396,7 @@ def run_native(args, wl):
     torch.cuda.synchronize(device)
     per_kernel = api.timing_read()
     api.timing_enable(False)
+    log(f"per-kernel timing: {per_kernel}")
     roofline = None
     peaks, peak_src = load_peaks()
     if per_kernel:
@@ -416,11 +442,13 @@ def run_native(args, wl):
     barrier(device)
     e2e_ms = reduce_max(ev0.elapsed_time(ev1) / e2e_steps, device)
     e2e_value = job_value(flops, world, e2e_ms / 1e3) / 1e12
+    log(f"e2e done: {e2e_ms:.3f} ms/step")
     io_elt = wl.heads * wl.N * wl.d * elt_bytes(wl)
 
     cpu_baseline = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         nh = heads_for_budget(wl, 2.0)
+        log(f"cpu baseline: {nh} heads per oracle call")
         val, el, done = oracle_sample(wl, args.cpu_seconds, nh)
         cpu_baseline = {"value": val, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                         "sample": f"{done} heads of the workload ({nh} per oracle call, "
@@ -459,6 +487,7 @@ def main(argv=None):
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true", help="skip the NVML clock sampler")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -99,13 +99,20 @@ Plan make_plan(const Problem& pb, int dtype) {
 
 monarch::SimtWorkspace carve_simt(const Plan& pl, char* base) {
   monarch::SimtWorkspace ws;
-  float** dst = &ws.qt0;
+  void* dst[7];
   const size_t* f = &pl.simt.qt0;
   size_t off = 0;
   for (int t = 0; t < 7; ++t) {
-    dst[t] = f[t] ? reinterpret_cast<float*>(base + off) : nullptr;
+    dst[t] = f[t] ? static_cast<void*>(base + off) : nullptr;
     off += align_up(f[t] * sizeof(float));
   }
+  ws.qt0 = static_cast<float*>(dst[0]);
+  ws.qt = static_cast<float*>(dst[1]);
+  ws.kt = dst[2];
+  ws.y = dst[3];
+  ws.hs = static_cast<float*>(dst[4]);
+  ws.lse = static_cast<float*>(dst[5]);
+  ws.ybar = static_cast<float*>(dst[6]);
   return ws;
 }
 
@@ -183,7 +190,7 @@ int forward_device(const TIn* q, const TIn* k, const TIn* v, TIn* out, int B, in
                             &t_launches);
   } else {
     const monarch::SimtWorkspace ws = carve_simt(pl, static_cast<char*>(g_ws[dev].ptr));
-    e = monarch::simt_forward<TIn>(q, k, v, out, pb, ws, stream, &t_launches);
+    e = monarch::simt_forward<TIn, float>(q, k, v, out, pb, ws, stream, &t_launches);
   }
   if (e != cudaSuccess) return record_cuda(e);
   return MONARCH_OK;

@@ -15,7 +15,7 @@
 //             non-final: Qt_{k,p,q,i} = sum_{l in p} L q_(l,i) / sum_{l in p} L
 //             final:     O_(l,i) = sum_(k,q) L Y_{k,p(l),q,i}
 //
-// Workspace layouts (fp32):
+// Workspace layouts (fp32 unless noted; Kt and Y are fp32 or bf16, TW):
 //   Qt0 [G][c1][b2][d]           Qt [G][b1 k][c1][c2][b2][d]
 //   Kt, Y [G][b2 i][c1 p][b1 k][c2 q][d]   Hs [G][b2][c1][b1][c2]
 //   lse [G][b2 i][b1 l]          Ybar [G][d]
@@ -52,11 +52,11 @@ __global__ void init_qt_kernel(const TIn* __restrict__ Q, float* __restrict__ qt
 }
 
 // One block per (g, k); one warp per R row (p, q, i).
-template <typename TIn, int DV>
+template <typename TIn, typename TW, int DV>
 __global__ void __launch_bounds__(kThreads)
 r_update_kernel(const TIn* __restrict__ K, const TIn* __restrict__ V,
-                const float* __restrict__ qt, QtStrides st, float* __restrict__ kt,
-                float* __restrict__ y, float* __restrict__ hs, Problem pb, int write_y) {
+                const float* __restrict__ qt, QtStrides st, TW* __restrict__ kt,
+                TW* __restrict__ y, float* __restrict__ hs, Problem pb, int write_y) {
   extern __shared__ float smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int d = pb.d, b1 = pb.b1, b2 = pb.b2, c1 = pb.c1, c2 = pb.c2;
@@ -110,8 +110,8 @@ r_update_kernel(const TIn* __restrict__ K, const TIn* __restrict__ V,
     for (int u = 0; u < DV; ++u) {
       const int x = lane + 32 * u;
       if (x < d) {
-        kt[orow * d + x] = ak[u] * inv;
-        if (write_y) y[orow * d + x] = av[u] * inv;
+        kt[orow * d + x] = from_f32<TW>(ak[u] * inv);
+        if (write_y) y[orow * d + x] = from_f32<TW>(av[u] * inv);
       }
     }
     if (lane == 0) hs[orow] = logf(z) - t * inv;
@@ -121,10 +121,10 @@ r_update_kernel(const TIn* __restrict__ K, const TIn* __restrict__ V,
 
 // One warp per query row (g, i, l).  MODE 0 writes O, MODE 1 writes the
 // row's log-sum-exp (used by the aggregation of a non-final L-update).
-template <typename TIn, int DV, int MODE>
+template <typename TIn, typename TW, int DV, int MODE>
 __global__ void __launch_bounds__(kThreads)
-l_rows_kernel(const TIn* __restrict__ Q, const float* __restrict__ kt,
-              const float* __restrict__ y, const float* __restrict__ hs, TIn* __restrict__ O,
+l_rows_kernel(const TIn* __restrict__ Q, const TW* __restrict__ kt,
+              const TW* __restrict__ y, const float* __restrict__ hs, TIn* __restrict__ O,
               float* __restrict__ lse, Problem pb) {
   extern __shared__ float smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -161,11 +161,11 @@ l_rows_kernel(const TIn* __restrict__ Q, const float* __restrict__ kt,
       const int nj = min(32, nk - kb);
       for (int jj = 0; jj < nj; ++jj) {
         const float ej = __shfl_sync(0xffffffffu, e, jj);
-        const float* yr = y + (kbase + kb + jj) * d;
+        const TW* yr = y + (kbase + kb + jj) * d;
 #pragma unroll
         for (int u = 0; u < DV; ++u) {
           const int x = lane + 32 * u;
-          if (x < d) ao[u] = fmaf(ej, yr[x], ao[u]);
+          if (x < d) ao[u] = fmaf(ej, to_f32(yr[x]), ao[u]);
         }
       }
     }
@@ -186,9 +186,9 @@ l_rows_kernel(const TIn* __restrict__ Q, const float* __restrict__ kt,
 
 // Non-final L-update, aggregation side: one warp per key (g, i, p, k, q)
 // sums the normalised L column over the rows l of group p.
-template <typename TIn, int DV>
+template <typename TIn, typename TW, int DV>
 __global__ void __launch_bounds__(kThreads)
-l_aggregate_kernel(const TIn* __restrict__ Q, const float* __restrict__ kt,
+l_aggregate_kernel(const TIn* __restrict__ Q, const TW* __restrict__ kt,
                    const float* __restrict__ hs, const float* __restrict__ lse,
                    float* __restrict__ qt, Problem pb) {
   extern __shared__ float smem[];
@@ -207,7 +207,7 @@ l_aggregate_kernel(const TIn* __restrict__ Q, const float* __restrict__ kt,
   const int k = kk / c2, q = kk % c2;
   const long key = ((g * b2 + i) * c1 + p) * (long)nk + kk;
   float* sk = smem + warp * d;
-  for (int x = lane; x < d; x += 32) sk[x] = kt[key * d + x] * pb.sc;
+  for (int x = lane; x < d; x += 32) sk[x] = to_f32(kt[key * d + x]) * pb.sc;
   __syncwarp();
   const float bias = hs[key];
   const int l0 = group_start(b1, c1, p), l1 = group_start(b1, c1, p + 1);
@@ -279,9 +279,11 @@ __global__ void broadcast_kernel(const float* __restrict__ ybar, TIn* __restrict
 
 inline unsigned blocks_for(long n, int threads) { return (unsigned)((n + threads - 1) / threads); }
 
-template <typename TIn, int DV>
+template <typename TIn, typename TW, int DV>
 cudaError_t run(const TIn* q, const TIn* k, const TIn* v, TIn* out, const Problem& pb,
-                const SimtWorkspace& ws, cudaStream_t stream, int* launches) {
+                const SimtWorkspace& ws, cudaStream_t stream, int* launches, bool final_output) {
+  TW* kt = static_cast<TW*>(ws.kt);
+  TW* yw = static_cast<TW*>(ws.y);
   const int G = pb.G, b1 = pb.b1, b2 = pb.b2, c1 = pb.c1, c2 = pb.c2, d = pb.d;
   const size_t shm = (size_t)kWarps * d * sizeof(float);
   cudaError_t err;
@@ -307,22 +309,24 @@ cudaError_t run(const TIn* q, const TIn* k, const TIn* v, TIn* out, const Proble
   for (int t = 1; t <= pb.T; ++t) {
     const bool last = (t == pb.T);
     MONARCH_LAUNCH("simt_r_update",
-                   (r_update_kernel<TIn, DV><<<(unsigned)((long)G * b1), kThreads, shm, stream>>>(
-                       k, v, t == 1 ? ws.qt0 : ws.qt, t == 1 ? s0 : s1, ws.kt, ws.y, ws.hs, pb,
-                       last ? 1 : 0)));
+                   (r_update_kernel<TIn, TW, DV><<<(unsigned)((long)G * b1), kThreads, shm,
+                                                   stream>>>(k, v, t == 1 ? ws.qt0 : ws.qt,
+                                                             t == 1 ? s0 : s1, kt, yw, ws.hs, pb,
+                                                             last ? 1 : 0)));
     const unsigned nrow_blocks = (unsigned)((long)G * b2 * ((b1 + kWarps - 1) / kWarps));
     if (last) {
-      MONARCH_LAUNCH("simt_l_output",
-                     (l_rows_kernel<TIn, DV, 0><<<nrow_blocks, kThreads, shm, stream>>>(
-                         q, ws.kt, ws.y, ws.hs, out, nullptr, pb)));
+      if (final_output)
+        MONARCH_LAUNCH("simt_l_output",
+                       (l_rows_kernel<TIn, TW, DV, 0><<<nrow_blocks, kThreads, shm, stream>>>(
+                           q, kt, yw, ws.hs, out, nullptr, pb)));
     } else {
       MONARCH_LAUNCH("simt_l_stats",
-                     (l_rows_kernel<TIn, DV, 1><<<nrow_blocks, kThreads, shm, stream>>>(
-                         q, ws.kt, ws.y, ws.hs, nullptr, ws.lse, pb)));
+                     (l_rows_kernel<TIn, TW, DV, 1><<<nrow_blocks, kThreads, shm, stream>>>(
+                         q, kt, yw, ws.hs, nullptr, ws.lse, pb)));
       const unsigned nagg = (unsigned)((long)G * b2 * c1 * ((b1 * c2 + kWarps - 1) / kWarps));
       MONARCH_LAUNCH("simt_l_aggregate",
-                     (l_aggregate_kernel<TIn, DV><<<nagg, kThreads, shm, stream>>>(
-                         q, ws.kt, ws.hs, ws.lse, ws.qt, pb)));
+                     (l_aggregate_kernel<TIn, TW, DV><<<nagg, kThreads, shm, stream>>>(
+                         q, kt, ws.hs, ws.lse, ws.qt, pb)));
     }
   }
 #undef MONARCH_LAUNCH
@@ -344,18 +348,23 @@ SimtWorkspaceSizes simt_workspace_sizes(const Problem& pb) {
   return s;
 }
 
-template <typename TIn>
+template <typename TIn, typename TW>
 cudaError_t simt_forward(const TIn* q, const TIn* k, const TIn* v, TIn* out, const Problem& pb,
-                         const SimtWorkspace& ws, cudaStream_t stream, int* launches) {
-  if (pb.d <= 32) return run<TIn, 1>(q, k, v, out, pb, ws, stream, launches);
-  if (pb.d <= 64) return run<TIn, 2>(q, k, v, out, pb, ws, stream, launches);
-  if (pb.d <= 128) return run<TIn, 4>(q, k, v, out, pb, ws, stream, launches);
-  return run<TIn, 8>(q, k, v, out, pb, ws, stream, launches);
+                         const SimtWorkspace& ws, cudaStream_t stream, int* launches,
+                         bool final_output) {
+  if (pb.d <= 32) return run<TIn, TW, 1>(q, k, v, out, pb, ws, stream, launches, final_output);
+  if (pb.d <= 64) return run<TIn, TW, 2>(q, k, v, out, pb, ws, stream, launches, final_output);
+  if (pb.d <= 128) return run<TIn, TW, 4>(q, k, v, out, pb, ws, stream, launches, final_output);
+  return run<TIn, TW, 8>(q, k, v, out, pb, ws, stream, launches, final_output);
 }
 
-template cudaError_t simt_forward<float>(const float*, const float*, const float*, float*,
-                                         const Problem&, const SimtWorkspace&, cudaStream_t, int*);
-template cudaError_t simt_forward<bf16>(const bf16*, const bf16*, const bf16*, bf16*,
-                                        const Problem&, const SimtWorkspace&, cudaStream_t, int*);
+#define MONARCH_INSTANTIATE(TIn, TW)                                                        \
+  template cudaError_t simt_forward<TIn, TW>(const TIn*, const TIn*, const TIn*, TIn*,      \
+                                             const Problem&, const SimtWorkspace&,          \
+                                             cudaStream_t, int*, bool);
+MONARCH_INSTANTIATE(float, float)
+MONARCH_INSTANTIATE(bf16, float)
+MONARCH_INSTANTIATE(bf16, bf16)
+#undef MONARCH_INSTANTIATE
 
 }  // namespace monarch

@@ -15,21 +15,27 @@ struct QtStrides {
   long g, k, p, q, i;
 };
 
-// fp32 workspace pieces (element counts), see simt_kernels.cu for layouts.
+// Workspace pieces (element counts), see simt_kernels.cu for layouts.  Kt
+// and Y hold TW elements (fp32 or bf16), everything else fp32.
 struct SimtWorkspaceSizes {
   size_t qt0, qt, kt, y, hs, lse, ybar;
 };
 
 struct SimtWorkspace {
-  float *qt0, *qt, *kt, *y, *hs, *lse, *ybar;
+  float *qt0, *qt;
+  void *kt, *y;
+  float *hs, *lse, *ybar;
 };
 
 SimtWorkspaceSizes simt_workspace_sizes(const Problem& pb);
 
-// Runs the whole forward pass on `stream`; adds the number of kernels it
-// launched to *launches.
-template <typename TIn>
+// Runs the forward pass on `stream` with TW-typed Kt/Y intermediates; adds
+// the number of kernels it launched to *launches.  With final_output false
+// it stops after the last R-update (Kt, Y, Hs written), leaving the final
+// L-update and output to the caller.
+template <typename TIn, typename TW>
 cudaError_t simt_forward(const TIn* q, const TIn* k, const TIn* v, TIn* out, const Problem& pb,
-                         const SimtWorkspace& ws, cudaStream_t stream, int* launches);
+                         const SimtWorkspace& ws, cudaStream_t stream, int* launches,
+                         bool final_output = true);
 
 }  // namespace monarch
