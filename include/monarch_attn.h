@@ -47,6 +47,8 @@
  *                            by monarch_attn_check() (and by the host-buffer
  *                            entry point, which checks before returning).
  *   MONARCH_ERR_NO_MEMORY    the workspace could not be allocated.
+ *   MONARCH_ERR_SCRATCH_LIMIT the shape needs more scratch than the static
+ *                            array of monarch_attn_fwd_noalloc holds.
  */
 #ifndef MONARCH_ATTN_H
 #define MONARCH_ATTN_H
@@ -70,6 +72,7 @@ extern "C" {
 #define MONARCH_ERR_CUDA           -3
 #define MONARCH_ERR_DEVICE_TIMEOUT -4
 #define MONARCH_ERR_NO_MEMORY      -5
+#define MONARCH_ERR_SCRATCH_LIMIT  -6
 
 #define MONARCH_DTYPE_BF16 0
 #define MONARCH_DTYPE_F32  1
@@ -103,6 +106,34 @@ MONARCH_API int monarch_attn_fwd_host(int dtype, const void* q_host, const void*
                           const void* v_host, void* out_host,
                           int B, int H, int b1, int b2, int d, int T, int c1, int c2,
                           cudaStream_t stream);
+
+/* Forward pass, bf16, that allocates nothing.  The pages have no
+ * counterpart of this entry point: it is for callers that cannot allocate
+ * device memory when they call, such as a real-time frame loop (cudaMalloc
+ * and cudaFree can synchronise the device and stall a frame past its
+ * deadline) or a host framework that reserves all device memory for its own
+ * pool and leaves a plugin no room for a cache of its own.
+ *
+ * Arguments, layout and result are those of monarch_attn_fwd, for the shapes
+ * its tensor-core path takes (d = 64 or 128, T >= 1; any other shape returns
+ * MONARCH_ERR_UNSUPPORTED).  The caller still passes q, k, v and out.
+ *
+ * Scratch: one static device array of 64 MiB (67108864 bytes) on every
+ * device that loads this library, held until the process exits.  A shape
+ * whose scratch (monarch_attn_workspace_bytes(..., MONARCH_DTYPE_BF16) on the
+ * default path) exceeds it returns MONARCH_ERR_SCRATCH_LIMIT.  The first call
+ * on a device looks up the array's device address and clears its status word
+ * (a synchronous memset), so make that first call before any stream capture.
+ * Every call on a device shares the array and leaves the last call's contents
+ * in it; the kernels write each scratch entry before they read it.  Calls
+ * that overlap on the GPU (other streams, or unordered host threads) race on
+ * the array: order them on one stream.  No cudaMalloc, cudaFree or other
+ * allocating routine is called.  A bounded device wait that expires (the
+ * kernel stops early and out is invalid) is recorded in the array's own
+ * status word, which this entry point does not report back. */
+MONARCH_API int monarch_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out,
+                                         int B, int H, int b1, int b2, int d, int T, int c1,
+                                         int c2, cudaStream_t stream);
 
 /* Bytes of device workspace a call with these arguments uses (0 on invalid
  * arguments).  dtype is MONARCH_DTYPE_BF16 or MONARCH_DTYPE_F32. */

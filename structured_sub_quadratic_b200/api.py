@@ -20,6 +20,7 @@ MONARCH_ERR_UNSUPPORTED = -2
 MONARCH_ERR_CUDA = -3
 MONARCH_ERR_DEVICE_TIMEOUT = -4
 MONARCH_ERR_NO_MEMORY = -5
+MONARCH_ERR_SCRATCH_LIMIT = -6
 DTYPE_BF16 = 0
 DTYPE_F32 = 1
 PATH_AUTO = 0
@@ -32,6 +33,7 @@ SIGNATURES = {
     "monarch_attn_fwd": (_I, [_P, _P, _P, _P, *_SIZES, _P]),
     "monarch_attn_fwd_f32": (_I, [_P, _P, _P, _P, *_SIZES, _P]),
     "monarch_attn_fwd_host": (_I, [_I, _P, _P, _P, _P, *_SIZES, _P]),
+    "monarch_attn_fwd_noalloc": (_I, [_P, _P, _P, _P, *_SIZES, _P]),
     "monarch_attn_workspace_bytes": (_Z, [*_SIZES, _I]),
     "monarch_attn_release_workspace": (None, []),
     "monarch_attn_check": (_I, [_P]),
@@ -114,6 +116,30 @@ def monarch_attn_fwd(q, k, v, b1, b2, T, c1=1, c2=1, out=None, stream=None):
         raise ValueError(f"unsupported dtype {q.dtype}")
     _check(fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
               B, H, b1, b2, d, T, c1, c2, _stream_ptr(stream)))
+    return out
+
+
+def monarch_attn_fwd_noalloc(q, k, v, b1, b2, T, c1=1, c2=1, out=None, stream=None):
+    """bf16 forward pass that allocates no device memory inside the library.
+
+    For callers that cannot allocate when they call (a real-time frame loop
+    that must not stall on cudaMalloc/cudaFree, or a host that reserves all
+    device memory for its own pool).  Scratch is a static 64 MiB device array
+    shared by all calls on a device; calls that overlap on the GPU race on
+    it, so keep them on one stream.  Pass ``out`` to avoid the one
+    allocation this wrapper would otherwise make through torch.
+    """
+    lib = load_library()
+    B, H, d = _dims(q, b1, b2)
+    for t in (q, k, v):
+        if t.shape != q.shape or t.dtype != torch.bfloat16 or not t.is_cuda \
+                or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous bf16 CUDA tensors of one shape")
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib.monarch_attn_fwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                        out.data_ptr(), B, H, b1, b2, d, T, c1, c2,
+                                        _stream_ptr(stream)))
     return out
 
 

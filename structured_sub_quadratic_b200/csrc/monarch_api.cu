@@ -308,6 +308,9 @@ const char* monarch_attn_strerror(int status) {
     case MONARCH_ERR_DEVICE_TIMEOUT:
       return "a bounded device wait expired; the kernel stopped early and its output is invalid";
     case MONARCH_ERR_NO_MEMORY: return t_err[0] ? t_err : "workspace allocation failed";
+    case MONARCH_ERR_SCRATCH_LIMIT:
+      return "the shape needs more scratch than the 64 MiB static array of "
+             "monarch_attn_fwd_noalloc holds";
     default: return "unknown status";
   }
 }
