@@ -26,6 +26,8 @@
 
 #include <math.h>
 
+#include <type_traits>
+
 namespace monarch {
 
 namespace {
@@ -347,6 +349,55 @@ SimtWorkspaceSizes simt_workspace_sizes(const Problem& pb) {
   s.ybar = pb.T == 0 ? G * d : 0;
   return s;
 }
+
+template <typename TIn, typename TW>
+cudaError_t simt_r_update(const TIn* k, const TIn* v, const float* qt, const QtStrides& st,
+                          TW* kt, TW* y, float* hs, const Problem& pb, bool write_y,
+                          cudaStream_t stream, int* launches) {
+  const size_t shm = (size_t)kWarps * pb.d * sizeof(float);
+  const unsigned nb = (unsigned)((long)pb.G * pb.b1);
+  auto go = [&](auto dv) {
+    constexpr int DV = decltype(dv)::value;
+    return timed_launch("simt_r_update", stream, launches, [&] {
+      r_update_kernel<TIn, TW, DV><<<nb, kThreads, shm, stream>>>(k, v, qt, st, kt, y, hs, pb,
+                                                                  write_y ? 1 : 0);
+    });
+  };
+  if (pb.d <= 32) return go(std::integral_constant<int, 1>());
+  if (pb.d <= 64) return go(std::integral_constant<int, 2>());
+  if (pb.d <= 128) return go(std::integral_constant<int, 4>());
+  return go(std::integral_constant<int, 8>());
+}
+
+template <typename TIn, typename TW>
+cudaError_t simt_l_update(const TIn* q, const TW* kt, const float* hs, float* lse, float* qt,
+                          const Problem& pb, cudaStream_t stream, int* launches) {
+  const size_t shm = (size_t)kWarps * pb.d * sizeof(float);
+  const int G = pb.G, b1 = pb.b1, b2 = pb.b2, c1 = pb.c1, c2 = pb.c2;
+  const unsigned nrow_blocks = (unsigned)((long)G * b2 * ((b1 + kWarps - 1) / kWarps));
+  const unsigned nagg = (unsigned)((long)G * b2 * c1 * ((b1 * c2 + kWarps - 1) / kWarps));
+  auto go = [&](auto dv) {
+    constexpr int DV = decltype(dv)::value;
+    cudaError_t e = timed_launch("simt_l_stats", stream, launches, [&] {
+      l_rows_kernel<TIn, TW, DV, 1><<<nrow_blocks, kThreads, shm, stream>>>(
+          q, kt, (const TW*)nullptr, hs, (TIn*)nullptr, lse, pb);
+    });
+    if (e != cudaSuccess) return e;
+    return timed_launch("simt_l_aggregate", stream, launches, [&] {
+      l_aggregate_kernel<TIn, TW, DV><<<nagg, kThreads, shm, stream>>>(q, kt, hs, lse, qt, pb);
+    });
+  };
+  if (pb.d <= 32) return go(std::integral_constant<int, 1>());
+  if (pb.d <= 64) return go(std::integral_constant<int, 2>());
+  if (pb.d <= 128) return go(std::integral_constant<int, 4>());
+  return go(std::integral_constant<int, 8>());
+}
+
+template cudaError_t simt_r_update<bf16, bf16>(const bf16*, const bf16*, const float*,
+                                               const QtStrides&, bf16*, bf16*, float*,
+                                               const Problem&, bool, cudaStream_t, int*);
+template cudaError_t simt_l_update<bf16, bf16>(const bf16*, const bf16*, const float*, float*,
+                                               float*, const Problem&, cudaStream_t, int*);
 
 template <typename TIn, typename TW>
 cudaError_t simt_forward(const TIn* q, const TIn* k, const TIn* v, TIn* out, const Problem& pb,

@@ -38,4 +38,17 @@ cudaError_t simt_forward(const TIn* q, const TIn* k, const TIn* v, TIn* out, con
                          const SimtWorkspace& ws, cudaStream_t stream, int* launches,
                          bool final_output = true);
 
+// Single steps, for paths that run the other steps elsewhere.
+// R-update of one step: qt rows addressed by `st`; writes Kt, Hs (and Y).
+template <typename TIn, typename TW>
+cudaError_t simt_r_update(const TIn* k, const TIn* v, const float* qt, const QtStrides& st,
+                          TW* kt, TW* y, float* hs, const Problem& pb, bool write_y,
+                          cudaStream_t stream, int* launches);
+
+// Non-final L-update: row log-sum-exps, then the aggregated queries
+// Qt [G][b1 k][c1][c2][b2 i][d] (fp32) of the next step.
+template <typename TIn, typename TW>
+cudaError_t simt_l_update(const TIn* q, const TW* kt, const float* hs, float* lse, float* qt,
+                          const Problem& pb, cudaStream_t stream, int* launches);
+
 }  // namespace monarch

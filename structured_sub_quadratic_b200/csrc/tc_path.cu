@@ -19,8 +19,8 @@
 // The running max is only raised when a tile's max exceeds it by more than
 // 2^8 (exact result, fewer rescales of the TMEM accumulator).
 //
-// The earlier steps (initial aggregated queries, R-updates, non-final
-// L-updates) currently run on the SIMT kernels writing bf16 Kt and Y.
+// Step one (aggregated queries under the uniform L, R-update) also runs on
+// the tensor cores; later steps of T >= 2 run on the SIMT kernels.
 #include "tc_path.cuh"
 
 #include <cudaTypedefs.h>
@@ -328,6 +328,269 @@ __global__ void __launch_bounds__(kThreadsKO)
 }
 
 // ---------------------------------------------------------------------------
+// Step-one aggregated queries under the uniform initial L (bf16):
+// Qt0[g][p][i][:] = mean_{l in p} q_(l,i).  One block per (g, p, i); 16-byte
+// column chunks x row lanes, reduced through shared memory.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256)
+    init_qt_bf16_kernel(const bf16* __restrict__ q, bf16* __restrict__ qt0, int b1, int b2,
+                        int c1) {
+  constexpr int CH = D / 8;
+  constexpr int LANES = 256 / CH;
+  __shared__ float red[LANES][D];
+  int bid = blockIdx.x;
+  const int i = bid % b2;
+  bid /= b2;
+  const int p = bid % c1;
+  const long g = bid / c1;
+  const int l0 = group_start(b1, c1, p), l1 = group_start(b1, c1, p + 1);
+  const int ch = threadIdx.x % CH, lane = threadIdx.x / CH;
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  for (int l = l0 + lane; l < l1; l += LANES) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(q + ((g * b1 + l) * b2 + i) * D) + ch);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      acc[2 * e] += __uint_as_float(w[e] << 16);
+      acc[2 * e + 1] += __uint_as_float(w[e] & 0xffff0000u);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) red[lane][ch * 8 + e] = acc[e];
+  __syncthreads();
+  if (threadIdx.x < D) {
+    float sum = 0.f;
+#pragma unroll 4
+    for (int ln = 0; ln < LANES; ++ln) sum += red[ln][threadIdx.x];
+    qt0[((g * c1 + p) * b2 + i) * D + threadIdx.x] = __float2bfloat16_rn(sum / (float)(l1 - l0));
+  }
+}
+
+// ---------------------------------------------------------------------------
+// R-update of step one on the tensor cores.  One CTA per (g, k, p): the b2
+// aggregated queries Qt0_{p,i} (rows, <= 128) against the b2 keys of chunk k:
+//   S = Qt0 K_k^T / sqrt(d)                      128 x bk in TMEM
+//   per column group q: R = softmax_{j in q}(S), Hs = entropy of R
+//   [Kt | Y] = R [K_k | V_k]                      one N = 2d MMA chain
+// The same K tile is the K-major B operand of the first product and the
+// MN-major B operand of the second; [K | V] sit side by side in shared
+// memory so their four 64-column blocks are one MN-major operand.  The
+// output accumulator reuses the TMEM columns of S (S is in registers by
+// then), so a CTA holds 2d columns.
+// ---------------------------------------------------------------------------
+struct KRArgs {
+  bf16* kt;   // [G][b2][c1][b1][c2][d]
+  bf16* y;
+  float* hs;  // [G][b2][c1][b1][c2]
+  int b1, b2, c1, c2, bk, write_y;
+  float sc_log2;
+  int* status;
+};
+
+template <int D>
+struct KRLayout {
+  int kv_box, q_off, k_off, v_off, p_off, bar_off, bytes;
+  __host__ __device__ explicit KRLayout(int bk) {
+    kv_box = bk * 128;
+    q_off = 0;
+    k_off = D / 64 * kRows * 128;
+    v_off = k_off + D / 64 * kv_box;
+    p_off = v_off + D / 64 * kv_box;
+    bar_off = p_off + ((bk + 63) / 64) * kRows * 128;
+    bytes = bar_off + 64;
+  }
+  static constexpr uint32_t kTmemCols = 2 * D;  // >= bk for bk <= 128
+};
+
+template <int D, int BKMAX>
+__global__ void __launch_bounds__(128)
+    kr_kernel(const __grid_constant__ CUtensorMap tm_qt, const __grid_constant__ CUtensorMap tm_k,
+              const __grid_constant__ CUtensorMap tm_v, KRArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int tid = threadIdx.x, warp = tid >> 5;
+  if (smem_u32(smem) & 1023u) {
+    if (tid == 0) atomicExch(a.status, 2);
+    return;
+  }
+  const KRLayout<D> L(a.bk);
+  int bid = blockIdx.x;
+  const int p = bid % a.c1;
+  bid /= a.c1;
+  const int k = bid % a.b1;
+  const int g = bid / a.b1;
+  const int bk = a.bk;
+
+  uint8_t* sQ = smem + L.q_off;
+  uint8_t* sK = smem + L.k_off;
+  uint8_t* sV = smem + L.v_off;
+  uint8_t* sP = smem + L.p_off;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar_off);
+  uint64_t* load_full = bars + 0;
+  uint64_t* s_full = bars + 1;
+  uint64_t* o_full = bars + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 4);
+
+  if (tid == 0) {
+    mbar_init(load_full, 1);
+    mbar_init(s_full, 1);
+    mbar_init(o_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, KRLayout<D>::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+
+  bool load_waited = false;
+  int mma_issued = 0;  // commits outstanding on s_full / o_full, for the abort drain
+  if (tid == 0) {
+    tma_prefetch_desc(&tm_qt);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    mbar_arrive_expect_tx(load_full, D / 64 * (kRows * 128 + 2 * L.kv_box));
+    const int qrow = (g * a.c1 + p) * a.b2;
+    const int krow = (g * a.b1 + k) * a.b2;
+#pragma unroll
+    for (int c = 0; c < D / 64; ++c) {
+      tma_load_2d(sQ + c * kRows * 128, &tm_qt, load_full, c * 64, qrow);
+      tma_load_2d(sK + c * L.kv_box, &tm_k, load_full, c * 64, krow);
+      tma_load_2d(sV + c * L.kv_box, &tm_v, load_full, c * 64, krow);
+    }
+    load_waited = mbar_wait(load_full, 0, abort_flag, a.status);
+    if (load_waited) {
+      tc_fence_after();
+      const uint32_t qb = smem_u32(sQ), kb = smem_u32(sK);
+      const uint32_t idesc = idesc_bf16(kRows, bk, false);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint64_t ad = desc_kmajor(qb + (kk >> 2) * (kRows * 128) + (kk & 3) * 32);
+        const uint64_t bd = desc_kmajor(kb + (kk >> 2) * L.kv_box + (kk & 3) * 32);
+        mma_bf16_ss(tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
+      }
+      mma_commit(s_full);
+      mma_issued = 1;
+    }
+  }
+  bool ok = mbar_wait(s_full, 0, abort_flag, a.status);
+  ok = __all_sync(0xffffffffu, ok);
+  float sv[BKMAX];
+  if (ok) {
+    tc_fence_after();
+#pragma unroll
+    for (int c = 0; c < BKMAX / 32; ++c) {
+      float t[32];
+      tmem_ld32(tmem + lane_off + c * 32, t);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) sv[c * 32 + e] = t[e] * a.sc_log2;
+    }
+    tmem_wait_ld();
+  }
+  const int r = tid;  // row = position i
+  const bool row_valid = r < a.b2;
+  for (int q = 0; q < a.c2; ++q) {
+    const int j0 = group_start(a.b2, a.c2, q), j1 = group_start(a.b2, a.c2, q + 1);
+    float m2 = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < BKMAX; ++j)
+      if (j >= j0 && j < j1) m2 = fmaxf(m2, sv[j]);
+    float z = 0.f, t2 = 0.f;
+    if (ok) {
+#pragma unroll
+      for (int u = 0; u < BKMAX / 8; ++u) {
+        if (u * 8 >= bk) break;
+        float e8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int j = u * 8 + e;
+          const float x = (j >= j0 && j < j1) ? ex2(sv[j] - m2) : 0.f;
+          e8[e] = __bfloat162float(__float2bfloat16_rn(x));
+          z += e8[e];
+          t2 += (j >= j0 && j < j1) ? e8[e] * (sv[j] - m2) : 0.f;
+        }
+        uint4 pk;
+        pk.x = pack_bf16x2(e8[0], e8[1]);
+        pk.y = pack_bf16x2(e8[2], e8[3]);
+        pk.z = pack_bf16x2(e8[4], e8[5]);
+        pk.w = pack_bf16x2(e8[6], e8[7]);
+        const int chunk = u >> 3, unit = u & 7;
+        *reinterpret_cast<uint4*>(sP + chunk * (kRows * 128) + r * 128 +
+                                  ((unit ^ (r & 7)) << 4)) = pk;
+      }
+      fence_proxy_async_smem();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (*abort_flag) break;
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t pb = smem_u32(sP), kb = smem_u32(sK);
+      const uint32_t idesc = idesc_bf16(kRows, 2 * D, true);
+      for (int kk = 0; kk < bk / 16; ++kk) {
+        const uint64_t ad = desc_kmajor(pb + (kk >> 2) * (kRows * 128) + (kk & 3) * 32);
+        const uint64_t bd = desc_mnmajor(kb + kk * 16 * 128, L.kv_box);
+        mma_bf16_ss(tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
+      }
+      mma_commit(o_full);
+      ++mma_issued;
+    }
+    ok = mbar_wait(o_full, q & 1, abort_flag, a.status);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+      tc_fence_after();
+      const float inv = 1.f / z;
+      const long orow = ((((long)g * a.b2 + r) * a.c1 + p) * a.b1 + k) * a.c2 + q;
+#pragma unroll 1
+      for (int half = 0; half < (a.write_y ? 2 : 1); ++half) {
+        bf16* dst = (half == 0 ? a.kt : a.y) + orow * D;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          float t[32];
+          tmem_ld32(tmem + lane_off + half * D + c * 32, t);
+          tmem_wait_ld();
+          if (row_valid) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              uint4 pk;
+              pk.x = pack_bf16x2(t[8 * u + 0] * inv, t[8 * u + 1] * inv);
+              pk.y = pack_bf16x2(t[8 * u + 2] * inv, t[8 * u + 3] * inv);
+              pk.z = pack_bf16x2(t[8 * u + 4] * inv, t[8 * u + 5] * inv);
+              pk.w = pack_bf16x2(t[8 * u + 6] * inv, t[8 * u + 7] * inv);
+              *reinterpret_cast<uint4*>(dst + c * 32 + 8 * u) = pk;
+            }
+          }
+        }
+      }
+      // entropy of the R row: ln z - sum e (s - m) / z, with s - m in log2 units
+      if (row_valid) a.hs[orow] = logf(z) - t2 * 0.69314718055994531f * inv;
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (*abort_flag) break;
+  }
+  if (tid == 0 && *abort_flag) {
+    if (!load_waited) drain(load_full, 0);
+    if (mma_issued >= 1) drain(s_full, 0);
+    if (mma_issued >= 2) drain(o_full, (mma_issued - 2) & 1);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, KRLayout<D>::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -401,6 +664,66 @@ cudaError_t launch_ko(const bf16* q, const bf16* kt, const bf16* y, const float*
   });
 }
 
+template <int D, int BKMAX>
+cudaError_t launch_kr(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, bf16* y, float* hs,
+                      const Problem& pb, int bk, int* status, cudaStream_t stream,
+                      int* launches) {
+  const KRLayout<D> L(bk);
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(kr_kernel<D, BKMAX>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    KRLayout<D>(BKMAX).bytes);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  CUtensorMap tq, tk, tv;
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)pb.G * pb.c1 * pb.b2};
+    const cuuint64_t str[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64, kRows};
+    if (!make_map(&tq, qt0, 2, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)pb.G * pb.b1 * pb.b2};
+    const cuuint64_t str[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)bk};
+    if (!make_map(&tk, k, 2, dims, str, box)) return cudaErrorInvalidValue;
+    if (!make_map(&tv, v, 2, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  KRArgs a;
+  a.kt = kt;
+  a.y = y;
+  a.hs = hs;
+  a.b1 = pb.b1;
+  a.b2 = pb.b2;
+  a.c1 = pb.c1;
+  a.c2 = pb.c2;
+  a.bk = bk;
+  a.write_y = pb.T == 1 ? 1 : 0;
+  a.sc_log2 = kLog2e * pb.sc;
+  a.status = status;
+  const long blocks = (long)pb.G * pb.b1 * pb.c1;
+  return timed_launch("tc_r_update", stream, launches, [&] {
+    kr_kernel<D, BKMAX><<<(unsigned)blocks, 128, L.bytes, stream>>>(tq, tk, tv, a);
+  });
+}
+
+// Step one: aggregated queries under the uniform L, then the R-update.
+template <int D>
+cudaError_t launch_r_step1(const bf16* q, const bf16* k, const bf16* v, bf16* qt0, bf16* kt,
+                           bf16* y, float* hs, const Problem& pb, int* status,
+                           cudaStream_t stream, int* launches) {
+  cudaError_t e = timed_launch("tc_init_qt", stream, launches, [&] {
+    init_qt_bf16_kernel<D><<<(unsigned)((long)pb.G * pb.c1 * pb.b2), 256, 0, stream>>>(
+        q, qt0, pb.b1, pb.b2, pb.c1);
+  });
+  if (e != cudaSuccess) return e;
+  const int bk = (pb.b2 + 15) / 16 * 16;
+  if (bk <= 64) return launch_kr<D, 64>(qt0, k, v, kt, y, hs, pb, bk, status, stream, launches);
+  return launch_kr<D, 128>(qt0, k, v, kt, y, hs, pb, bk, status, stream, launches);
+}
+
 constexpr size_t kAlign = 256;
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
@@ -431,7 +754,7 @@ SimtWorkspace carve(const Problem& pb, char* base, size_t* total) {
 
 bool tc_supports(const Problem& pb) {
   if (pb.d != 64 && pb.d != 128) return false;
-  if (pb.T < 1) return false;
+  if (pb.T < 1 || pb.b2 > 128) return false;  // R-side tile: b2 keys <= 128 rows
   const long key_rows = (long)pb.G * pb.b2 * pb.c1 * pb.b1 * pb.c2;
   if (key_rows + 256 >= (1L << 31) || (long)pb.G * pb.b1 >= (1L << 31)) return false;
   return encode_fn() != nullptr;
@@ -446,10 +769,23 @@ size_t tc_workspace_bytes(const Problem& pb) {
 cudaError_t tc_forward(const bf16* q, const bf16* k, const bf16* v, bf16* out, const Problem& pb,
                        char* ws_base, int* status, cudaStream_t stream, int* launches) {
   const SimtWorkspace ws = carve(pb, ws_base, nullptr);
-  cudaError_t e = simt_forward<bf16, bf16>(q, k, v, out, pb, ws, stream, launches, false);
+  bf16* kt = static_cast<bf16*>(ws.kt);
+  bf16* y = static_cast<bf16*>(ws.y);
+  bf16* qt0 = reinterpret_cast<bf16*>(ws.qt0);
+  cudaError_t e = pb.d == 128 ? launch_r_step1<128>(q, k, v, qt0, kt, y, ws.hs, pb, status, stream,
+                                                    launches)
+                              : launch_r_step1<64>(q, k, v, qt0, kt, y, ws.hs, pb, status, stream,
+                                                   launches);
   if (e != cudaSuccess) return e;
-  const bf16* kt = static_cast<const bf16*>(ws.kt);
-  const bf16* y = static_cast<const bf16*>(ws.y);
+  const QtStrides s1 = {(long)pb.b1 * pb.c1 * pb.c2 * pb.b2 * pb.d,
+                        (long)pb.c1 * pb.c2 * pb.b2 * pb.d, (long)pb.c2 * pb.b2 * pb.d,
+                        (long)pb.b2 * pb.d, (long)pb.d};
+  for (int t = 2; t <= pb.T; ++t) {
+    e = simt_l_update<bf16, bf16>(q, kt, ws.hs, ws.lse, ws.qt, pb, stream, launches);
+    if (e != cudaSuccess) return e;
+    e = simt_r_update<bf16, bf16>(k, v, ws.qt, s1, kt, y, ws.hs, pb, t == pb.T, stream, launches);
+    if (e != cudaSuccess) return e;
+  }
   if (pb.d == 128) return launch_ko<128, 64>(q, kt, y, ws.hs, out, pb, status, stream, launches);
   return launch_ko<64, 64>(q, kt, y, ws.hs, out, pb, status, stream, launches);
 }
