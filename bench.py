@@ -487,11 +487,15 @@ def main(argv=None):
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-clocks", action="store_true", help="skip the NVML clock sampler")
+    ap.add_argument("--no-clocks", action="store_true", help="skip the clock sampler")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="override H (profiling a smaller case of the same shape)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     wl = WORKLOADS[args.workload]
+    if args.heads is not None:
+        wl = Workload(**{**wl.__dict__, "H": args.heads, "name": f"{wl.name} [H={args.heads}]"})
     if args.impl == "reference":
         return run_reference(args, wl)
     return run_native(args, wl)

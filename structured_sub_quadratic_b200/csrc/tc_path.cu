@@ -44,34 +44,27 @@ constexpr float kLog2e = 1.4426950408889634f;
 template <int D, int NK>
 struct KOLayout {
   static constexpr int kQBytes = D / 64 * kRows * 128;
-  static constexpr int kKtBytes = D / 64 * NK * 128;
-  static constexpr int kStageBytes = 2 * kKtBytes;  // Kt then Y
+  static constexpr int kTileBytes = D / 64 * NK * 128;  // one Kt or Y tile
+  static constexpr int kStageBytes = 2 * kTileBytes;      // Kt then Y
   static constexpr int kStages = 2;
   static constexpr int kPBytes = NK / 64 * kRows * 128;
   static constexpr int kStageOff = kQBytes;
   static constexpr int kPOff = kStageOff + kStages * kStageBytes;
-  static constexpr int kBiasOff = kPOff + kPBytes;             // float [2][NK]
-  static constexpr int kBarOff = kBiasOff + 2 * NK * 4;         // 8 x u64
-  static constexpr int kBytes = kBarOff + 8 * 8;
-  static constexpr int kAlloc = kBytes;  // the dynamic buffer is declared 1024-B aligned
-  static constexpr uint32_t kTmemCols = (D + NK <= 128) ? 128u : (D + NK <= 256 ? 256u : 512u);
-  static_assert(D % 64 == 0 && NK % 64 == 0, "tile sizes");
+  static constexpr int kBiasOff = kPOff + kPBytes;  // float [kStages][NK]
+  static constexpr int kBarOff = kBiasOff + kStages * NK * 4;
+  static constexpr int kBytes = kBarOff + 16 * 8;
+  // At most two CTAs per SM (their TMEM use is 2 x 256 columns).
+  static constexpr int kAlloc = kBytes > 100 * 1024 ? kBytes : 100 * 1024;
+  static constexpr uint32_t kTmemCols = 256;  // O: D columns, S: two buffers of NK
+  static_assert(D % 64 == 0 && NK % 64 == 0 && D + 2 * NK <= 256, "tile sizes");
 };
 
 struct KOArgs {
   const float* hs;  // [G][b2][c1][nk]
   bf16* out;        // (G, N, d)
-  int b1, b2, c1, nk, row_tiles;
+  int b1, b2, c1, nk, row_tiles, n_items;
   float sc_log2;    // log2(e) / sqrt(d)
   int* status;
-};
-
-// Thread-0 bookkeeping of asynchronous work in flight, so that an aborted
-// CTA can drain it (bounded) before releasing TMEM.
-struct InFlight {
-  int kv_issued = 0, kv_waited = 0;
-  int s_issued = 0, pv_issued = 0;
-  bool q_waited = false;
 };
 
 __device__ __forceinline__ void drain(uint64_t* bar, uint32_t parity) {
@@ -81,56 +74,86 @@ __device__ __forceinline__ void drain(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// Work item = one 128-row query tile of one (g, i, p).  Returns false for
+// tiles past the end of the row group (possible when groups differ in size).
+struct KOItem {
+  int g, i, p, row0, nrows, nt;
+  long key_row0;
+};
+
+template <int NK>
+__device__ __forceinline__ bool ko_decode(const KOArgs& a, int item, KOItem& it) {
+  int bid = item;
+  const int rt = bid % a.row_tiles;
+  bid /= a.row_tiles;
+  it.p = bid % a.c1;
+  bid /= a.c1;
+  it.i = bid % a.b2;
+  it.g = bid / a.b2;
+  const int l0 = group_start(a.b1, a.c1, it.p), l1 = group_start(a.b1, a.c1, it.p + 1);
+  it.row0 = l0 + rt * kRows;
+  if (it.row0 >= l1) return false;
+  it.nrows = min(kRows, l1 - it.row0);
+  it.key_row0 = ((long)(it.g * a.b2 + it.i) * a.c1 + it.p) * a.nk;
+  it.nt = (a.nk + NK - 1) / NK;
+  return true;
+}
+
+// Persistent, warp-specialised L-update + output.  Warp 0 loads (TMA for Q,
+// Kt, Y; plain loads for the entropy bias), warp 1 issues the tcgen05.mma
+// instructions from one thread, warps 2-5 own the 128 rows (TMEM lanes) for
+// the online softmax and the epilogue.  mbarriers hand tiles between roles:
+//   q_full/q_empty      Q tile (one per item)
+//   kv_full/kv_empty    two-stage Kt/Y ring (global tile counter T)
+//   s_full/s_empty      two S buffers in TMEM
+//   p_full              P of tile T written to shared memory
+//   pv_done             O += P Y of tile T complete (P buffer free, O stable)
+//   o_empty             epilogue has read O (next item may overwrite it)
 template <int D, int NK>
-__global__ void __launch_bounds__(kThreadsKO)
+__global__ void __launch_bounds__(192, 2)
     ko_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kt,
               const __grid_constant__ CUtensorMap tm_y, KOArgs a) {
   using L = KOLayout<D, NK>;
   extern __shared__ __align__(1024) uint8_t smem[];
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (smem_u32(smem) & 1023u) {  // swizzled tiles need 1024-B alignment: report, never fault
     if (tid == 0) atomicExch(a.status, 2);
     return;
   }
-
-  int bid = blockIdx.x;
-  const int rt = bid % a.row_tiles;
-  bid /= a.row_tiles;
-  const int p = bid % a.c1;
-  bid /= a.c1;
-  const int i = bid % a.b2;
-  const int g = bid / a.b2;
-  const int l0 = group_start(a.b1, a.c1, p), l1 = group_start(a.b1, a.c1, p + 1);
-  const int row0 = l0 + rt * kRows;
-  if (row0 >= l1) return;  // whole CTA past the group: uniform, before any sync
-  const int nrows = min(kRows, l1 - row0);
-  const long key_row0 = ((long)(g * a.b2 + i) * a.c1 + p) * a.nk;
-  const int nt = (a.nk + NK - 1) / NK;
-
   uint8_t* sQ = smem;
   uint8_t* sP = smem + L::kPOff;
   float* sBias = reinterpret_cast<float*>(smem + L::kBiasOff);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
   uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;  // two stages
-  uint64_t* s_full = bars + 3;
-  uint64_t* pv_done = bars + 4;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 5);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 6);
+  uint64_t* q_empty = bars + 1;
+  uint64_t* kv_full = bars + 2;   // [2]
+  uint64_t* kv_empty = bars + 4;  // [2]
+  uint64_t* s_full = bars + 6;    // [2]
+  uint64_t* s_empty = bars + 8;   // [2]
+  uint64_t* p_full = bars + 10;
+  uint64_t* pv_done = bars + 11;
+  uint64_t* o_empty = bars + 12;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 14);
   auto sKt = [&](int st) { return smem + L::kStageOff + st * L::kStageBytes; };
-  auto sY = [&](int st) { return smem + L::kStageOff + st * L::kStageBytes + L::kKtBytes; };
+  auto sY = [&](int st) { return smem + L::kStageOff + st * L::kStageBytes + L::kTileBytes; };
 
   if (tid == 0) {
     mbar_init(q_full, 1);
-    mbar_init(kv_full, 1);
-    mbar_init(kv_full + 1, 1);
-    mbar_init(s_full, 1);
+    mbar_init(q_empty, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(kv_full + s, 32);
+      mbar_init(kv_empty + s, 1);
+      mbar_init(s_full + s, 1);
+      mbar_init(s_empty + s, 128);
+    }
+    mbar_init(p_full, 128);
     mbar_init(pv_done, 1);
+    mbar_init(o_empty, 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (tid < NK) sBias[tid] = tid < a.nk ? a.hs[key_row0 + tid] * kLog2e : 0.f;
-  if (warp == 0) {
+  if (warp == 1) {
     tmem_alloc(tmem_slot, L::kTmemCols);
     tmem_relinquish();
   }
@@ -138,190 +161,259 @@ __global__ void __launch_bounds__(kThreadsKO)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tmem_o = tmem;      // columns [0, D): output accumulator
-  const uint32_t tmem_s = tmem + D;  // columns [D, D + NK): logits tile
-  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t tmem_o = tmem;  // columns [0, D)
+  auto tmem_s = [&](int sb) { return tmem + D + sb * NK; };
 
-  InFlight fl;
-  auto issue_kv = [&](int j) {
-    const int st = j & 1;
-    mbar_arrive_expect_tx(kv_full + st, L::kStageBytes);
-    const int y = static_cast<int>(key_row0 + (long)j * NK);
-#pragma unroll
-    for (int c = 0; c < D / 64; ++c) {
-      tma_load_2d(sKt(st) + c * NK * 128, &tm_kt, kv_full + st, c * 64, y);
-      tma_load_2d(sY(st) + c * NK * 128, &tm_y, kv_full + st, c * 64, y);
+  if (warp == 0) {
+    // ------------------------------ producer ------------------------------
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_kt);
+      tma_prefetch_desc(&tm_y);
     }
-    ++fl.kv_issued;
-  };
-  if (tid == 0) {
-    tma_prefetch_desc(&tm_q);
-    tma_prefetch_desc(&tm_kt);
-    tma_prefetch_desc(&tm_y);
-    mbar_arrive_expect_tx(q_full, L::kQBytes);
+    int n = 0, last_q = -1;
+    long T = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
+      KOItem it;
+      if (!ko_decode<NK>(a, item, it)) continue;
+      if (n >= 1) ok = mbar_wait(q_empty, (n - 1) & 1, abort_flag, a.status);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(q_full, L::kQBytes);
 #pragma unroll
-    for (int c = 0; c < D / 64; ++c)
-      tma_load_3d(sQ + c * kRows * 128, &tm_q, q_full, c * 64, i, g * a.b1 + row0);
-    issue_kv(0);
-    if (nt > 1) issue_kv(1);
-  }
-
-  const uint32_t idesc_s = idesc_bf16(kRows, NK, false);
-  const uint32_t idesc_o = idesc_bf16(kRows, D, true);
-  const int row = tid;
-  float m_run = -INFINITY, l_run = 0.f;
-
-  for (int j = 0; j < nt; ++j) {
-    const int st = j & 1;
-    // ---- S = Q Kt^T (one thread issues) ----
-    if (tid == 0) {
-      bool w = mbar_wait(kv_full + st, (j >> 1) & 1, abort_flag, a.status);
-      if (w) ++fl.kv_waited;
-      if (w && j == 0) {
-        w = mbar_wait(q_full, 0, abort_flag, a.status);
-        fl.q_waited = w;
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(sQ + c * kRows * 128, &tm_q, q_full, c * 64, it.i, it.g * a.b1 + it.row0);
       }
-      if (w) {
+      last_q = n;
+      for (int j = 0; j < it.nt; ++j, ++T) {
+        const int st = (int)(T & 1);
+        if (T >= 2) ok = mbar_wait(kv_empty + st, ((T >> 1) - 1) & 1, abort_flag, a.status);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        float* bias = sBias + st * NK;
+        for (int e = lane; e < NK; e += 32) {
+          const int col = j * NK + e;
+          bias[e] = col < a.nk ? __ldg(a.hs + it.key_row0 + col) * kLog2e : 0.f;
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(kv_full + st, L::kStageBytes);
+          const int y = static_cast<int>(it.key_row0 + (long)j * NK);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_2d(sKt(st) + c * NK * 128, &tm_kt, kv_full + st, c * 64, y);
+            tma_load_2d(sY(st) + c * NK * 128, &tm_y, kv_full + st, c * 64, y);
+          }
+        } else {
+          mbar_arrive(kv_full + st);
+        }
+      }
+      ++n;
+    }
+    if (lane == 0 && *abort_flag) {  // drain the loads this warp issued (bounded)
+      if (last_q >= 0) drain(q_full, last_q & 1);
+      for (long t = (T >= 2 ? T - 2 : 0); t < T; ++t) drain(kv_full + (t & 1), (t >> 1) & 1);
+    }
+  } else if (warp == 1) {
+    // -------------------------------- MMA ---------------------------------
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_bf16(kRows, NK, false);
+      const uint32_t idesc_o = idesc_bf16(kRows, D, true);
+      int n = 0;
+      long T = 0, last_s = -1, last_pv = -1;
+      bool ok = true;
+      auto issue_pv = [&](long Tp, bool first, int item_n) -> bool {
+        if (!mbar_wait(p_full, Tp & 1, abort_flag, a.status)) return false;
+        if (first && item_n >= 1 && !mbar_wait(o_empty, (item_n - 1) & 1, abort_flag, a.status))
+          return false;
         tc_fence_after();
-        const uint32_t qb = smem_u32(sQ), kb = smem_u32(sKt(st));
+        const int st = (int)(Tp & 1);
+        const uint32_t pb = smem_u32(sP), yb = smem_u32(sY(st));
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t ad = desc_kmajor(qb + (kk >> 2) * (kRows * 128) + (kk & 3) * 32);
-          const uint64_t bd = desc_kmajor(kb + (kk >> 2) * (NK * 128) + (kk & 3) * 32);
-          mma_bf16_ss(tmem_s, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < NK / 16; ++kk) {
+          const uint64_t ad = desc_kmajor(pb + (kk >> 2) * (kRows * 128) + (kk & 3) * 32);
+          const uint64_t bd = desc_mnmajor(yb + kk * 16 * 128, NK * 128);
+          mma_bf16_ss(tmem_o, ad, bd, idesc_o, (!first || kk > 0) ? 1u : 0u);
         }
-        mma_commit(s_full);
-        ++fl.s_issued;
+        mma_commit(kv_empty + st);
+        mma_commit(pv_done);
+        last_pv = Tp;
+        return true;
+      };
+      for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
+        KOItem it;
+        if (!ko_decode<NK>(a, item, it)) continue;
+        ok = mbar_wait(q_full, n & 1, abort_flag, a.status);
+        const long T0 = T;
+        for (int j = 0; j < it.nt && ok; ++j, ++T) {
+          const int st = (int)(T & 1);
+          ok = mbar_wait(kv_full + st, (T >> 1) & 1, abort_flag, a.status);
+          if (ok && T >= 2) ok = mbar_wait(s_empty + st, ((T >> 1) - 1) & 1, abort_flag, a.status);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t qb = smem_u32(sQ), kb = smem_u32(sKt(st));
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t ad = desc_kmajor(qb + (kk >> 2) * (kRows * 128) + (kk & 3) * 32);
+            const uint64_t bd = desc_kmajor(kb + (kk >> 2) * (NK * 128) + (kk & 3) * 32);
+            mma_bf16_ss(tmem_s(st), ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(s_full + st);
+          last_s = T;
+          if (j == it.nt - 1) mma_commit(q_empty);
+          if (j >= 1) ok = issue_pv(T - 1, j == 1, n);
+        }
+        if (ok) ok = issue_pv(T0 + it.nt - 1, it.nt == 1, n);
+        ++n;
+      }
+      if (*abort_flag) {  // drain this thread's MMAs (bounded)
+        if (last_s >= 0) drain(s_full + (last_s & 1), (last_s >> 1) & 1);
+        if (last_pv >= 0) drain(pv_done, last_pv & 1);
       }
     }
-    bool ok = mbar_wait(s_full, j & 1, abort_flag, a.status);
-    ok = __all_sync(0xffffffffu, ok);
-
-    // ---- softmax of this row's NK logits ----
-    float sv[NK];
-    float alpha = 1.f;
-    bool resc = false;
-    if (ok) {
-      tc_fence_after();
+    __syncwarp();
+  } else {
+    // ------------------------- softmax + epilogue --------------------------
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;  // TMEM lane == tile row
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    long T = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
+      KOItem it;
+      if (!ko_decode<NK>(a, item, it)) continue;
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int j = 0; j < it.nt; ++j, ++T) {
+        const int sb = (int)(T & 1);
+        ok = mbar_wait(s_full + sb, (T >> 1) & 1, abort_flag, a.status);
+        if (ok) ok = mbar_wait(kv_full + sb, (T >> 1) & 1, abort_flag, a.status);  // bias
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        float sv[NK];
+        tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < NK / 32; ++c) {
-        float t[32];
-        tmem_ld32(tmem_s + lane_off + c * 32, t);
+        for (int c = 0; c < NK / 32; ++c) {
+          float t[32];
+          tmem_ld32(tmem_s(sb) + lane_off + c * 32, t);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) sv[c * 32 + e] = t[e];
-      }
-      tmem_wait_ld();
-      const float* bias = sBias + st * NK;
-      const int valid = a.nk - j * NK;
-      float mt = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < NK; ++c) {
-        sv[c] = c < valid ? fmaf(sv[c], a.sc_log2, bias[c]) : -INFINITY;
-        mt = fmaxf(mt, sv[c]);
-      }
-      if (mt > m_run + 8.f) {  // first tile, or the max grew by more than 2^8
-        alpha = ex2(m_run - mt);
-        resc = j > 0;
-        m_run = mt;
-      }
-      float ls = 0.f;
-#pragma unroll
-      for (int c = 0; c < NK; ++c) {
-        sv[c] = ex2(sv[c] - m_run);
-        ls += sv[c];
-      }
-      l_run = l_run * alpha + ls;
-    }
-    // ---- previous P V done: P buffer free, O stable, its stage free ----
-    if (ok && j > 0) ok = mbar_wait(pv_done, (j - 1) & 1, abort_flag, a.status);
-    ok = __all_sync(0xffffffffu, ok);
-    if (ok && tid == 0 && j >= 1 && j + 1 < nt) issue_kv(j + 1);
-    if (ok && __any_sync(0xffffffffu, resc)) {
-      tc_fence_after();
-#pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        float t[32];
-        tmem_ld32(tmem_o + lane_off + c * 32, t);
+          for (int e = 0; e < 32; ++e) sv[c * 32 + e] = t[e];
+        }
         tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(s_empty + sb);
+        const float* bias = sBias + sb * NK;
+        const int valid = a.nk - j * NK;
+        // logits in log2 units; 4 partial maxima / sums break the serial chains
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        if (valid >= NK) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) t[e] *= alpha;
-        tmem_st32(tmem_o + lane_off + c * 32, t);
-      }
-      tmem_wait_st();
-    }
-    if (ok) {
-      // P row -> shared memory, K-major with 128-byte swizzle
+          for (int c = 0; c < NK; ++c) {
+            sv[c] = fmaf(sv[c], a.sc_log2, bias[c]);
+            mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
+          }
+        } else {
 #pragma unroll
-      for (int u = 0; u < NK / 8; ++u) {
-        uint4 pk;
-        pk.x = pack_bf16x2(sv[8 * u + 0], sv[8 * u + 1]);
-        pk.y = pack_bf16x2(sv[8 * u + 2], sv[8 * u + 3]);
-        pk.z = pack_bf16x2(sv[8 * u + 4], sv[8 * u + 5]);
-        pk.w = pack_bf16x2(sv[8 * u + 6], sv[8 * u + 7]);
-        const int chunk = u >> 3, unit = u & 7;
-        *reinterpret_cast<uint4*>(sP + chunk * (kRows * 128) + row * 128 +
-                                  ((unit ^ (row & 7)) << 4)) = pk;
-      }
-      fence_proxy_async_smem();
-    }
-    if (tid < NK && j + 1 < nt) {
-      const int col = (j + 1) * NK + tid;
-      sBias[((j + 1) & 1) * NK + tid] = col < a.nk ? a.hs[key_row0 + col] * kLog2e : 0.f;
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (*abort_flag) break;  // read after the barrier: uniform across the CTA
-    // ---- O += P Y ----
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t pb = smem_u32(sP), yb = smem_u32(sY(st));
-#pragma unroll
-      for (int kk = 0; kk < NK / 16; ++kk) {
-        const uint64_t ad = desc_kmajor(pb + (kk >> 2) * (kRows * 128) + (kk & 3) * 32);
-        const uint64_t bd = desc_mnmajor(yb + kk * 16 * 128, NK * 128);
-        mma_bf16_ss(tmem_o, ad, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
-      }
-      mma_commit(pv_done);
-      ++fl.pv_issued;
-    }
-  }
-
-  // ---- epilogue: O / l -> global ----
-  bool ok = !*abort_flag && mbar_wait(pv_done, (nt - 1) & 1, abort_flag, a.status);
-  ok = __all_sync(0xffffffffu, ok);
-  if (ok) {
-    tc_fence_after();
-    const float inv = 1.f / l_run;
-    const bool valid = row < nrows;
-    bf16* orow = a.out + (((long)g * a.b1 + row0 + row) * a.b2 + i) * D;
-#pragma unroll 1
-    for (int c = 0; c < D / 32; ++c) {
-      float t[32];
-      tmem_ld32(tmem_o + lane_off + c * 32, t);
-      tmem_wait_ld();
-      if (valid) {
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          uint4 pk;
-          pk.x = pack_bf16x2(t[8 * u + 0] * inv, t[8 * u + 1] * inv);
-          pk.y = pack_bf16x2(t[8 * u + 2] * inv, t[8 * u + 3] * inv);
-          pk.z = pack_bf16x2(t[8 * u + 4] * inv, t[8 * u + 5] * inv);
-          pk.w = pack_bf16x2(t[8 * u + 6] * inv, t[8 * u + 7] * inv);
-          *reinterpret_cast<uint4*>(orow + c * 32 + 8 * u) = pk;
+          for (int c = 0; c < NK; ++c) {
+            sv[c] = c < valid ? fmaf(sv[c], a.sc_log2, bias[c]) : -INFINITY;
+            mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
+          }
         }
+        const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        float alpha = 1.f;
+        bool resc = false;
+        if (mt > m_run + 8.f) {  // first tile, or the max grew by more than 2^8
+          alpha = ex2(m_run - mt);
+          resc = j > 0;
+          m_run = mt;
+        }
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < NK; ++c) {
+          sv[c] = ex2(sv[c] - m_run);
+          ls[c & 3] += sv[c];
+        }
+        l_run = l_run * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
+        // P buffer free and O stable once the previous tile's P Y is done
+        if (T >= 1) ok = mbar_wait(pv_done, (T - 1) & 1, abort_flag, a.status);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        if (__any_sync(0xffffffffu, resc)) {
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            float t[32];
+            tmem_ld32(tmem_o + lane_off + c * 32, t);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) t[e] *= alpha;
+            tmem_st32(tmem_o + lane_off + c * 32, t);
+          }
+          tmem_wait_st();
+        }
+#pragma unroll
+        for (int u = 0; u < NK / 8; ++u) {
+          uint4 pk;
+          pk.x = pack_bf16x2(sv[8 * u + 0], sv[8 * u + 1]);
+          pk.y = pack_bf16x2(sv[8 * u + 2], sv[8 * u + 3]);
+          pk.z = pack_bf16x2(sv[8 * u + 4], sv[8 * u + 5]);
+          pk.w = pack_bf16x2(sv[8 * u + 6], sv[8 * u + 7]);
+          const int chunk = u >> 3, unit = u & 7;
+          *reinterpret_cast<uint4*>(sP + chunk * (kRows * 128) + row * 128 +
+                                    ((unit ^ (row & 7)) << 4)) = pk;
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(p_full);
       }
+      if (!ok) break;
+      // ---- epilogue: O / l -> global rows ----
+      ok = mbar_wait(pv_done, (T - 1) & 1, abort_flag, a.status);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const float inv = 1.f / l_run;
+      // Rows go out through shared memory (the P buffer is free now): each
+      // thread stages its row, then 8 threads write one row's 128-byte half,
+      // so global stores are whole sectors.
+      const int srow = tid - 64;  // 0..127 over the four softmax warps
+#pragma unroll 1
+      for (int h = 0; h < D / 64; ++h) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          float t[32];
+          tmem_ld32(tmem_o + lane_off + h * 64 + c * 32, t);
+          tmem_wait_ld();
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            uint4 pk;
+            pk.x = pack_bf16x2(t[8 * u + 0] * inv, t[8 * u + 1] * inv);
+            pk.y = pack_bf16x2(t[8 * u + 2] * inv, t[8 * u + 3] * inv);
+            pk.z = pack_bf16x2(t[8 * u + 4] * inv, t[8 * u + 5] * inv);
+            pk.w = pack_bf16x2(t[8 * u + 6] * inv, t[8 * u + 7] * inv);
+            const int unit = c * 4 + u;
+            *reinterpret_cast<uint4*>(sP + row * 128 + ((unit ^ (row & 7)) << 4)) = pk;
+          }
+        }
+        named_barrier(1, 128);
+#pragma unroll
+        for (int pass = 0; pass < kRows / 16; ++pass) {
+          const int r = pass * 16 + (srow >> 3), unit = srow & 7;
+          if (r < it.nrows) {
+            const uint4 v4 = *reinterpret_cast<const uint4*>(sP + r * 128 + ((unit ^ (r & 7)) << 4));
+            bf16* dst = a.out + (((long)it.g * a.b1 + it.row0 + r) * a.b2 + it.i) * D + h * 64;
+            *reinterpret_cast<uint4*>(dst + unit * 8) = v4;
+          }
+        }
+        named_barrier(1, 128);
+      }
+      tc_fence_before();
+      mbar_arrive(o_empty);
     }
-  }
-  // ---- aborted: drain what is still in flight (bounded) before freeing TMEM ----
-  if (tid == 0 && *abort_flag) {
-    if (!fl.q_waited) drain(q_full, 0);
-    for (int j = fl.kv_waited; j < fl.kv_issued; ++j) drain(kv_full + (j & 1), (j >> 1) & 1);
-    if (fl.s_issued > 0) drain(s_full, (fl.s_issued - 1) & 1);
-    if (fl.pv_issued > 0) drain(pv_done, (fl.pv_issued - 1) & 1);
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, L::kTmemCols);
   }
@@ -371,63 +463,60 @@ __global__ void __launch_bounds__(256)
 
 // ---------------------------------------------------------------------------
 // R-update of step one on the tensor cores.  One CTA per (g, k, p): the b2
-// aggregated queries Qt0_{p,i} (rows, <= 128) against the b2 keys of chunk k:
-//   S = Qt0 K_k^T / sqrt(d)                      128 x bk in TMEM
-//   per column group q: R = softmax_{j in q}(S), Hs = entropy of R
-//   [Kt | Y] = R [K_k | V_k]                      one N = 2d MMA chain
-// The same K tile is the K-major B operand of the first product and the
-// MN-major B operand of the second; [K | V] sit side by side in shared
-// memory so their four 64-column blocks are one MN-major operand.  The
-// output accumulator reuses the TMEM columns of S (S is in registers by
-// then), so a CTA holds 2d columns.
+// aggregated queries Qt0_{p,i} (rows, <= 128) against the keys of chunk k,
+// one column group q at a time:
+//   S_q = Qt0 K_q^T / sqrt(d)            128 x NQ in TMEM (K_q: keys j in q)
+//   R = softmax_j(S_q), Hs = entropy      one TMEM lane (row) per thread
+//   [Kt | Y] = R [K_q | V_q]               one N = 2d MMA chain
+// K_q and V_q of every group are separate TMA boxes (any start row), laid
+// side by side so that [K_q | V_q] is one MN-major operand; K_q alone is the
+// K-major operand of S_q.  The output accumulator reuses the TMEM columns of
+// S_q (S_q is in registers by then), so a CTA holds 2d columns.
 // ---------------------------------------------------------------------------
 struct KRArgs {
   bf16* kt;   // [G][b2][c1][b1][c2][d]
   bf16* y;
   float* hs;  // [G][b2][c1][b1][c2]
-  int b1, b2, c1, c2, bk, write_y;
+  int b1, b2, c1, c2, write_y;
   float sc_log2;
   int* status;
 };
 
-template <int D>
+template <int D, int NQ>
 struct KRLayout {
-  int kv_box, q_off, k_off, v_off, p_off, bar_off, bytes;
-  __host__ __device__ explicit KRLayout(int bk) {
-    kv_box = bk * 128;
-    q_off = 0;
-    k_off = D / 64 * kRows * 128;
-    v_off = k_off + D / 64 * kv_box;
-    p_off = v_off + D / 64 * kv_box;
-    bar_off = p_off + ((bk + 63) / 64) * kRows * 128;
-    bytes = bar_off + 64;
-  }
-  static constexpr uint32_t kTmemCols = 2 * D;  // >= bk for bk <= 128
+  static constexpr int kBox = NQ * 128;                    // one 64-column box of NQ rows
+  static constexpr int kGroupBytes = 2 * (D / 64) * kBox;  // K_q then V_q
+  static constexpr int kQOff = 0;
+  static constexpr int kKVOff = D / 64 * kRows * 128;
+  static constexpr int kPBytes = (NQ + 63) / 64 * kRows * 128;
+  __host__ __device__ static constexpr int p_off(int c2) { return kKVOff + c2 * kGroupBytes; }
+  __host__ __device__ static constexpr int bar_off(int c2) { return p_off(c2) + kPBytes; }
+  __host__ __device__ static constexpr int bytes(int c2) { return bar_off(c2) + 64; }
+  static constexpr uint32_t kTmemCols = 2 * D;  // O (2d columns); S_q uses the first NQ
+  static_assert(NQ % 16 == 0 && NQ <= 128 && NQ <= 2 * D, "group tile");
 };
 
-template <int D, int BKMAX>
+template <int D, int NQ>
 __global__ void __launch_bounds__(128)
     kr_kernel(const __grid_constant__ CUtensorMap tm_qt, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, KRArgs a) {
+  using L = KRLayout<D, NQ>;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5;
   if (smem_u32(smem) & 1023u) {
     if (tid == 0) atomicExch(a.status, 2);
     return;
   }
-  const KRLayout<D> L(a.bk);
   int bid = blockIdx.x;
   const int p = bid % a.c1;
   bid /= a.c1;
   const int k = bid % a.b1;
   const int g = bid / a.b1;
-  const int bk = a.bk;
 
-  uint8_t* sQ = smem + L.q_off;
-  uint8_t* sK = smem + L.k_off;
-  uint8_t* sV = smem + L.v_off;
-  uint8_t* sP = smem + L.p_off;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar_off);
+  uint8_t* sQ = smem + L::kQOff;
+  auto sK = [&](int q) { return smem + L::kKVOff + q * L::kGroupBytes; };
+  uint8_t* sP = smem + L::p_off(a.c2);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::bar_off(a.c2));
   uint64_t* load_full = bars + 0;
   uint64_t* s_full = bars + 1;
   uint64_t* o_full = bars + 2;
@@ -442,7 +531,7 @@ __global__ void __launch_bounds__(128)
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(tmem_slot, KRLayout<D>::kTmemCols);
+    tmem_alloc(tmem_slot, L::kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -452,76 +541,82 @@ __global__ void __launch_bounds__(128)
   const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
 
   bool load_waited = false;
-  int mma_issued = 0;  // commits outstanding on s_full / o_full, for the abort drain
+  int s_issued = 0, o_issued = 0;
+  auto issue_s = [&](int q) {
+    tc_fence_after();
+    const uint32_t qb = smem_u32(sQ), kb = smem_u32(sK(q));
+    const uint32_t idesc = idesc_bf16(kRows, NQ, false);
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint64_t ad = desc_kmajor(qb + (kk >> 2) * (kRows * 128) + (kk & 3) * 32);
+      const uint64_t bd = desc_kmajor(kb + (kk >> 2) * L::kBox + (kk & 3) * 32);
+      mma_bf16_ss(tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
+    }
+    mma_commit(s_full);
+    ++s_issued;
+  };
   if (tid == 0) {
     tma_prefetch_desc(&tm_qt);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
-    mbar_arrive_expect_tx(load_full, D / 64 * (kRows * 128 + 2 * L.kv_box));
+    mbar_arrive_expect_tx(load_full, D / 64 * kRows * 128 + a.c2 * L::kGroupBytes);
     const int qrow = (g * a.c1 + p) * a.b2;
-    const int krow = (g * a.b1 + k) * a.b2;
 #pragma unroll
-    for (int c = 0; c < D / 64; ++c) {
-      tma_load_2d(sQ + c * kRows * 128, &tm_qt, load_full, c * 64, qrow);
-      tma_load_2d(sK + c * L.kv_box, &tm_k, load_full, c * 64, krow);
-      tma_load_2d(sV + c * L.kv_box, &tm_v, load_full, c * 64, krow);
+    for (int c = 0; c < D / 64; ++c) tma_load_2d(sQ + c * kRows * 128, &tm_qt, load_full, c * 64, qrow);
+    for (int q = 0; q < a.c2; ++q) {
+      const int krow = (g * a.b1 + k) * a.b2 + group_start(a.b2, a.c2, q);
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        tma_load_2d(sK(q) + c * L::kBox, &tm_k, load_full, c * 64, krow);
+        tma_load_2d(sK(q) + (D / 64 + c) * L::kBox, &tm_v, load_full, c * 64, krow);
+      }
     }
     load_waited = mbar_wait(load_full, 0, abort_flag, a.status);
-    if (load_waited) {
-      tc_fence_after();
-      const uint32_t qb = smem_u32(sQ), kb = smem_u32(sK);
-      const uint32_t idesc = idesc_bf16(kRows, bk, false);
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint64_t ad = desc_kmajor(qb + (kk >> 2) * (kRows * 128) + (kk & 3) * 32);
-        const uint64_t bd = desc_kmajor(kb + (kk >> 2) * L.kv_box + (kk & 3) * 32);
-        mma_bf16_ss(tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
-      }
-      mma_commit(s_full);
-      mma_issued = 1;
-    }
-  }
-  bool ok = mbar_wait(s_full, 0, abort_flag, a.status);
-  ok = __all_sync(0xffffffffu, ok);
-  float sv[BKMAX];
-  if (ok) {
-    tc_fence_after();
-#pragma unroll
-    for (int c = 0; c < BKMAX / 32; ++c) {
-      float t[32];
-      tmem_ld32(tmem + lane_off + c * 32, t);
-#pragma unroll
-      for (int e = 0; e < 32; ++e) sv[c * 32 + e] = t[e] * a.sc_log2;
-    }
-    tmem_wait_ld();
+    if (load_waited) issue_s(0);
   }
   const int r = tid;  // row = position i
   const bool row_valid = r < a.b2;
   for (int q = 0; q < a.c2; ++q) {
-    const int j0 = group_start(a.b2, a.c2, q), j1 = group_start(a.b2, a.c2, q + 1);
-    float m2 = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < BKMAX; ++j)
-      if (j >= j0 && j < j1) m2 = fmaxf(m2, sv[j]);
+    const int nq = group_start(a.b2, a.c2, q + 1) - group_start(a.b2, a.c2, q);
+    bool ok = mbar_wait(s_full, q & 1, abort_flag, a.status);
+    ok = __all_sync(0xffffffffu, ok);
     float z = 0.f, t2 = 0.f;
     if (ok) {
+      tc_fence_after();
+      float sv[NQ];
 #pragma unroll
-      for (int u = 0; u < BKMAX / 8; ++u) {
-        if (u * 8 >= bk) break;
-        float e8[8];
+      for (int c = 0; c < NQ / 16; ++c) {
+        float t[16];
+        tmem_ld16(tmem + lane_off + c * 16, t);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int j = u * 8 + e;
-          const float x = (j >= j0 && j < j1) ? ex2(sv[j] - m2) : 0.f;
-          e8[e] = __bfloat162float(__float2bfloat16_rn(x));
-          z += e8[e];
-          t2 += (j >= j0 && j < j1) ? e8[e] * (sv[j] - m2) : 0.f;
-        }
+        for (int e = 0; e < 16; ++e) sv[c * 16 + e] = t[e];
+      }
+      tmem_wait_ld();
+      // logits in log2 units; 4 partial maxima and sums break the serial chains
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int j = 0; j < NQ; ++j) {
+        sv[j] = j < nq ? sv[j] * a.sc_log2 : -INFINITY;
+        mx[j & 3] = fmaxf(mx[j & 3], sv[j]);
+      }
+      const float m2 = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      float zs[4] = {0.f, 0.f, 0.f, 0.f}, ts[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int j = 0; j < NQ; ++j) {
+        const float d2 = sv[j] - m2;  // -inf for j >= nq
+        sv[j] = ex2(d2);
+        zs[j & 3] += sv[j];
+        ts[j & 3] += j < nq ? sv[j] * d2 : 0.f;
+      }
+      z = (zs[0] + zs[1]) + (zs[2] + zs[3]);
+      t2 = (ts[0] + ts[1]) + (ts[2] + ts[3]);
+#pragma unroll
+      for (int u = 0; u < NQ / 8; ++u) {
         uint4 pk;
-        pk.x = pack_bf16x2(e8[0], e8[1]);
-        pk.y = pack_bf16x2(e8[2], e8[3]);
-        pk.z = pack_bf16x2(e8[4], e8[5]);
-        pk.w = pack_bf16x2(e8[6], e8[7]);
+        pk.x = pack_bf16x2(sv[8 * u + 0], sv[8 * u + 1]);
+        pk.y = pack_bf16x2(sv[8 * u + 2], sv[8 * u + 3]);
+        pk.z = pack_bf16x2(sv[8 * u + 4], sv[8 * u + 5]);
+        pk.w = pack_bf16x2(sv[8 * u + 6], sv[8 * u + 7]);
         const int chunk = u >> 3, unit = u & 7;
         *reinterpret_cast<uint4*>(sP + chunk * (kRows * 128) + r * 128 +
                                   ((unit ^ (r & 7)) << 4)) = pk;
@@ -533,60 +628,79 @@ __global__ void __launch_bounds__(128)
     if (*abort_flag) break;
     if (tid == 0) {
       tc_fence_after();
-      const uint32_t pb = smem_u32(sP), kb = smem_u32(sK);
+      const uint32_t pb = smem_u32(sP), kb = smem_u32(sK(q));
       const uint32_t idesc = idesc_bf16(kRows, 2 * D, true);
-      for (int kk = 0; kk < bk / 16; ++kk) {
+#pragma unroll
+      for (int kk = 0; kk < NQ / 16; ++kk) {
         const uint64_t ad = desc_kmajor(pb + (kk >> 2) * (kRows * 128) + (kk & 3) * 32);
-        const uint64_t bd = desc_mnmajor(kb + kk * 16 * 128, L.kv_box);
+        const uint64_t bd = desc_mnmajor(kb + kk * 16 * 128, L::kBox);
         mma_bf16_ss(tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
       }
       mma_commit(o_full);
-      ++mma_issued;
+      ++o_issued;
     }
     ok = mbar_wait(o_full, q & 1, abort_flag, a.status);
     ok = __all_sync(0xffffffffu, ok);
     if (ok) {
       tc_fence_after();
       const float inv = 1.f / z;
-      const long orow = ((((long)g * a.b2 + r) * a.c1 + p) * a.b1 + k) * a.c2 + q;
+      // Rows (positions i, b2*c1*b1*c2*d elements apart) go out through the
+      // P buffer (free once [Kt | Y] is complete; the Qt0 tile must survive
+      // for the next group): 64 columns at a time, each thread stages its
+      // row, then 8 threads write one row's 128 bytes as whole sectors.
+      const int nblk = (a.write_y ? 2 : 1) * (D / 64);
 #pragma unroll 1
-      for (int half = 0; half < (a.write_y ? 2 : 1); ++half) {
-        bf16* dst = (half == 0 ? a.kt : a.y) + orow * D;
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          float t[32];
-          tmem_ld32(tmem + lane_off + half * D + c * 32, t);
-          tmem_wait_ld();
-          if (row_valid) {
+      for (int cb = 0; cb < nblk; ++cb) {
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              uint4 pk;
-              pk.x = pack_bf16x2(t[8 * u + 0] * inv, t[8 * u + 1] * inv);
-              pk.y = pack_bf16x2(t[8 * u + 2] * inv, t[8 * u + 3] * inv);
-              pk.z = pack_bf16x2(t[8 * u + 4] * inv, t[8 * u + 5] * inv);
-              pk.w = pack_bf16x2(t[8 * u + 6] * inv, t[8 * u + 7] * inv);
-              *reinterpret_cast<uint4*>(dst + c * 32 + 8 * u) = pk;
-            }
+        for (int c = 0; c < 2; ++c) {
+          float t[32];
+          tmem_ld32(tmem + lane_off + cb * 64 + c * 32, t);
+          tmem_wait_ld();
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            uint4 pk;
+            pk.x = pack_bf16x2(t[8 * u + 0] * inv, t[8 * u + 1] * inv);
+            pk.y = pack_bf16x2(t[8 * u + 2] * inv, t[8 * u + 3] * inv);
+            pk.z = pack_bf16x2(t[8 * u + 4] * inv, t[8 * u + 5] * inv);
+            pk.w = pack_bf16x2(t[8 * u + 6] * inv, t[8 * u + 7] * inv);
+            const int unit = c * 4 + u;
+            *reinterpret_cast<uint4*>(sP + r * 128 + ((unit ^ (r & 7)) << 4)) = pk;
           }
         }
+        __syncthreads();
+        bf16* base = (cb < D / 64 ? a.kt : a.y) + (cb % (D / 64)) * 64;
+#pragma unroll
+        for (int pass = 0; pass < kRows / 16; ++pass) {
+          const int rr = pass * 16 + (tid >> 3), unit = tid & 7;
+          if (rr < a.b2) {
+            const uint4 v4 = *reinterpret_cast<const uint4*>(sP + rr * 128 + ((unit ^ (rr & 7)) << 4));
+            const long orr = ((((long)g * a.b2 + rr) * a.c1 + p) * a.b1 + k) * a.c2 + q;
+            *reinterpret_cast<uint4*>(base + orr * D + unit * 8) = v4;
+          }
+        }
+        __syncthreads();
       }
       // entropy of the R row: ln z - sum e (s - m) / z, with s - m in log2 units
-      if (row_valid) a.hs[orow] = logf(z) - t2 * 0.69314718055994531f * inv;
+      if (row_valid) {
+        const long orow = ((((long)g * a.b2 + r) * a.c1 + p) * a.b1 + k) * a.c2 + q;
+        a.hs[orow] = logf(z) - t2 * 0.69314718055994531f * inv;
+      }
     }
     tc_fence_before();
     __syncthreads();
     if (*abort_flag) break;
+    if (tid == 0 && q + 1 < a.c2) issue_s(q + 1);
   }
   if (tid == 0 && *abort_flag) {
     if (!load_waited) drain(load_full, 0);
-    if (mma_issued >= 1) drain(s_full, 0);
-    if (mma_issued >= 2) drain(o_full, (mma_issued - 2) & 1);
+    if (s_issued > 0) drain(s_full, (s_issued - 1) & 1);
+    if (o_issued > 0) drain(o_full, (o_issued - 1) & 1);
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, KRLayout<D>::kTmemCols);
+    tmem_dealloc(tmem, L::kTmemCols);
   }
 }
 
@@ -620,6 +734,18 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+int num_sms() {
+  static int n = 0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+      n = 148;
+  });
+  return n;
+}
+
 template <int D, int NK>
 cudaError_t launch_ko(const bf16* q, const bf16* kt, const bf16* y, const float* hs, bf16* out,
                       const Problem& pb, int* status, cudaStream_t stream, int* launches) {
@@ -629,6 +755,9 @@ cudaError_t launch_ko(const bf16* q, const bf16* kt, const bf16* y, const float*
   std::call_once(attr_once, [] {
     attr_err = cudaFuncSetAttribute(ko_kernel<D, NK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     L::kAlloc);
+    if (attr_err == cudaSuccess)
+      attr_err = cudaFuncSetAttribute(ko_kernel<D, NK>,
+                                      cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   });
   if (attr_err != cudaSuccess) return attr_err;
   const int nk = pb.b1 * pb.c2;
@@ -656,27 +785,33 @@ cudaError_t launch_ko(const bf16* q, const bf16* kt, const bf16* y, const float*
   a.c1 = pb.c1;
   a.nk = nk;
   a.row_tiles = (gmax + kRows - 1) / kRows;
+  const long items = (long)pb.G * pb.b2 * pb.c1 * a.row_tiles;
+  if (items >= (1L << 31)) return cudaErrorInvalidValue;
+  a.n_items = (int)items;
   a.sc_log2 = kLog2e * pb.sc;
   a.status = status;
-  const long blocks = (long)pb.G * pb.b2 * pb.c1 * a.row_tiles;
+  const int grid = (int)std::min<long>(items, 2L * num_sms());
   return timed_launch("tc_l_output", stream, launches, [&] {
-    ko_kernel<D, NK><<<(unsigned)blocks, kThreadsKO, L::kAlloc, stream>>>(tq, tk, tyv, a);
+    ko_kernel<D, NK><<<grid, 192, L::kAlloc, stream>>>(tq, tk, tyv, a);
   });
 }
 
-template <int D, int BKMAX>
+template <int D, int NQ>
 cudaError_t launch_kr(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, bf16* y, float* hs,
-                      const Problem& pb, int bk, int* status, cudaStream_t stream,
-                      int* launches) {
-  const KRLayout<D> L(bk);
+                      const Problem& pb, int* status, cudaStream_t stream, int* launches) {
+  using L = KRLayout<D, NQ>;
+  constexpr int kMaxBytes = L::bytes(256 / NQ);
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(kr_kernel<D, BKMAX>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    KRLayout<D>(BKMAX).bytes);
+    attr_err = cudaFuncSetAttribute(kr_kernel<D, NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    kMaxBytes);
+    if (attr_err == cudaSuccess)
+      attr_err = cudaFuncSetAttribute(kr_kernel<D, NQ>,
+                                      cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   });
   if (attr_err != cudaSuccess) return attr_err;
+  if (L::bytes(pb.c2) > kMaxBytes) return cudaErrorInvalidValue;
   CUtensorMap tq, tk, tv;
   {
     const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)pb.G * pb.c1 * pb.b2};
@@ -687,7 +822,7 @@ cudaError_t launch_kr(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, b
   {
     const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)pb.G * pb.b1 * pb.b2};
     const cuuint64_t str[1] = {(cuuint64_t)D * 2};
-    const cuuint32_t box[2] = {64, (cuuint32_t)bk};
+    const cuuint32_t box[2] = {64, (cuuint32_t)NQ};
     if (!make_map(&tk, k, 2, dims, str, box)) return cudaErrorInvalidValue;
     if (!make_map(&tv, v, 2, dims, str, box)) return cudaErrorInvalidValue;
   }
@@ -699,14 +834,39 @@ cudaError_t launch_kr(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, b
   a.b2 = pb.b2;
   a.c1 = pb.c1;
   a.c2 = pb.c2;
-  a.bk = bk;
   a.write_y = pb.T == 1 ? 1 : 0;
   a.sc_log2 = kLog2e * pb.sc;
   a.status = status;
   const long blocks = (long)pb.G * pb.b1 * pb.c1;
   return timed_launch("tc_r_update", stream, launches, [&] {
-    kr_kernel<D, BKMAX><<<(unsigned)blocks, 128, L.bytes, stream>>>(tq, tk, tv, a);
+    kr_kernel<D, NQ><<<(unsigned)blocks, 128, L::bytes(pb.c2), stream>>>(tq, tk, tv, a);
   });
+}
+
+// Column-group tile width: the largest group (ceil(b2 / c2) keys) rounded up
+// to 16, the K step of one tcgen05.mma.
+inline int kr_group_tile(const Problem& pb) {
+  return ((pb.b2 + pb.c2 - 1) / pb.c2 + 15) / 16 * 16;
+}
+
+template <int D>
+cudaError_t dispatch_kr(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, bf16* y,
+                        float* hs, const Problem& pb, int* status, cudaStream_t stream,
+                        int* launches) {
+  switch (kr_group_tile(pb)) {
+#define MONARCH_KR_CASE(NQ) \
+  case NQ: return launch_kr<D, NQ>(qt0, k, v, kt, y, hs, pb, status, stream, launches);
+    MONARCH_KR_CASE(16)
+    MONARCH_KR_CASE(32)
+    MONARCH_KR_CASE(48)
+    MONARCH_KR_CASE(64)
+    MONARCH_KR_CASE(80)
+    MONARCH_KR_CASE(96)
+    MONARCH_KR_CASE(112)
+    MONARCH_KR_CASE(128)
+#undef MONARCH_KR_CASE
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 // Step one: aggregated queries under the uniform L, then the R-update.
@@ -719,9 +879,7 @@ cudaError_t launch_r_step1(const bf16* q, const bf16* k, const bf16* v, bf16* qt
         q, qt0, pb.b1, pb.b2, pb.c1);
   });
   if (e != cudaSuccess) return e;
-  const int bk = (pb.b2 + 15) / 16 * 16;
-  if (bk <= 64) return launch_kr<D, 64>(qt0, k, v, kt, y, hs, pb, bk, status, stream, launches);
-  return launch_kr<D, 128>(qt0, k, v, kt, y, hs, pb, bk, status, stream, launches);
+  return dispatch_kr<D>(qt0, k, v, kt, y, hs, pb, status, stream, launches);
 }
 
 constexpr size_t kAlign = 256;
@@ -754,7 +912,9 @@ SimtWorkspace carve(const Problem& pb, char* base, size_t* total) {
 
 bool tc_supports(const Problem& pb) {
   if (pb.d != 64 && pb.d != 128) return false;
-  if (pb.T < 1 || pb.b2 > 128) return false;  // R-side tile: b2 keys <= 128 rows
+  if (pb.T < 1 || pb.b2 > 128) return false;  // R-side tile: b2 queries <= 128 rows
+  const int nq = ((pb.b2 + pb.c2 - 1) / pb.c2 + 15) / 16 * 16;
+  if (nq > 2 * pb.d || pb.c2 * nq > 256) return false;  // TMEM columns, shared memory
   const long key_rows = (long)pb.G * pb.b2 * pb.c1 * pb.b1 * pb.c2;
   if (key_rows + 256 >= (1L << 31) || (long)pb.G * pb.b1 >= (1L << 31)) return false;
   return encode_fn() != nullptr;
