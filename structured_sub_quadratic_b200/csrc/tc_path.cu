@@ -45,14 +45,13 @@ template <int D, int NK>
 struct KOLayout {
   static constexpr int kQBytes = D / 64 * kRows * 128;
   static constexpr int kTileBytes = D / 64 * NK * 128;  // one Kt or Y tile
-  static constexpr int kStageBytes = 2 * kTileBytes;      // Kt then Y
-  static constexpr int kStages = 2;
   static constexpr int kPBytes = NK / 64 * kRows * 128;
-  static constexpr int kStageOff = kQBytes;
-  static constexpr int kPOff = kStageOff + kStages * kStageBytes;
-  static constexpr int kBiasOff = kPOff + kPBytes;  // float [kStages][NK]
-  static constexpr int kBarOff = kBiasOff + kStages * NK * 4;
-  static constexpr int kBytes = kBarOff + 16 * 8;
+  static constexpr int kKtOff = kQBytes;                 // Kt ring, 2 slots
+  static constexpr int kYOff = kKtOff + 2 * kTileBytes;   // Y ring, 2 slots
+  static constexpr int kPOff = kYOff + 2 * kTileBytes;
+  static constexpr int kBiasOff = kPOff + kPBytes;        // float [2][NK]
+  static constexpr int kBarOff = kBiasOff + 2 * NK * 4;
+  static constexpr int kBytes = kBarOff + 24 * 8;
   // At most two CTAs per SM (their TMEM use is 2 x 256 columns).
   static constexpr int kAlloc = kBytes > 100 * 1024 ? kBytes : 100 * 1024;
   static constexpr uint32_t kTmemCols = 256;  // O: D columns, S: two buffers of NK
@@ -99,18 +98,22 @@ __device__ __forceinline__ bool ko_decode(const KOArgs& a, int item, KOItem& it)
   return true;
 }
 
-// Persistent, warp-specialised L-update + output.  Warp 0 loads (TMA for Q,
-// Kt, Y; plain loads for the entropy bias), warp 1 issues the tcgen05.mma
-// instructions from one thread, warps 2-5 own the 128 rows (TMEM lanes) for
-// the online softmax and the epilogue.  mbarriers hand tiles between roles:
-//   q_full/q_empty      Q tile (one per item)
-//   kv_full/kv_empty    two-stage Kt/Y ring (global tile counter T)
-//   s_full/s_empty      two S buffers in TMEM
-//   p_full              P of tile T written to shared memory
-//   pv_done             O += P Y of tile T complete (P buffer free, O stable)
-//   o_empty             epilogue has read O (next item may overwrite it)
+// Persistent, warp-specialised L-update + output.  Warp 0 loads Q, Kt
+// (TMA) and the entropy bias (plain loads), warp 6 loads Y (TMA), warp 1
+// issues the tcgen05.mma instructions from one thread, warps 2-5 own the 128
+// rows (TMEM lanes) for the online softmax and the epilogue.  Kt and Y have
+// separate two-slot rings: a Kt slot is recycled as soon as its S tile is
+// computed, a Y slot once its P Y product is, so each load is issued about
+// two tiles before it is needed.  mbarriers hand tiles between roles:
+//   q_full/q_empty          Q tile (one per item)
+//   kt_full/kt_empty        Kt ring          y_full/y_empty   Y ring
+//   bias_full/bias_empty    bias ring        s_full/s_empty   S buffers in TMEM
+//   p_full                  P of tile T written to shared memory
+//   pv_done                 O += P Y of tile T complete (P buffer free, O stable)
+//   o_empty                 epilogue has read O (next item may overwrite it)
+// All counters run over the tiles T of every item this CTA processes.
 template <int D, int NK>
-__global__ void __launch_bounds__(192, 2)
+__global__ void __launch_bounds__(224, 2)
     ko_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kt,
               const __grid_constant__ CUtensorMap tm_y, KOArgs a) {
   using L = KOLayout<D, NK>;
@@ -126,26 +129,34 @@ __global__ void __launch_bounds__(192, 2)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
-  uint64_t* kv_full = bars + 2;   // [2]
-  uint64_t* kv_empty = bars + 4;  // [2]
-  uint64_t* s_full = bars + 6;    // [2]
-  uint64_t* s_empty = bars + 8;   // [2]
-  uint64_t* p_full = bars + 10;
-  uint64_t* pv_done = bars + 11;
-  uint64_t* o_empty = bars + 12;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 14);
-  auto sKt = [&](int st) { return smem + L::kStageOff + st * L::kStageBytes; };
-  auto sY = [&](int st) { return smem + L::kStageOff + st * L::kStageBytes + L::kTileBytes; };
+  uint64_t* kt_full = bars + 2;      // [2]
+  uint64_t* kt_empty = bars + 4;     // [2]
+  uint64_t* y_full = bars + 6;       // [2]
+  uint64_t* y_empty = bars + 8;      // [2]
+  uint64_t* s_full = bars + 10;      // [2]
+  uint64_t* s_empty = bars + 12;     // [2]
+  uint64_t* bias_full = bars + 14;   // [2]
+  uint64_t* bias_empty = bars + 16;  // [2]
+  uint64_t* p_full = bars + 18;
+  uint64_t* pv_done = bars + 19;
+  uint64_t* o_empty = bars + 20;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 21);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 22);
+  auto sKt = [&](int st) { return smem + L::kKtOff + st * L::kTileBytes; };
+  auto sY = [&](int st) { return smem + L::kYOff + st * L::kTileBytes; };
 
   if (tid == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(kv_full + s, 32);
-      mbar_init(kv_empty + s, 1);
+      mbar_init(kt_full + s, 1);
+      mbar_init(kt_empty + s, 1);
+      mbar_init(y_full + s, 1);
+      mbar_init(y_empty + s, 1);
       mbar_init(s_full + s, 1);
       mbar_init(s_empty + s, 128);
+      mbar_init(bias_full + s, 32);
+      mbar_init(bias_empty + s, 128);
     }
     mbar_init(p_full, 128);
     mbar_init(pv_done, 1);
@@ -165,11 +176,10 @@ __global__ void __launch_bounds__(192, 2)
   auto tmem_s = [&](int sb) { return tmem + D + sb * NK; };
 
   if (warp == 0) {
-    // ------------------------------ producer ------------------------------
+    // ------------------------ producer: Q, Kt, bias ------------------------
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_kt);
-      tma_prefetch_desc(&tm_y);
     }
     int n = 0, last_q = -1;
     long T = 0;
@@ -189,32 +199,56 @@ __global__ void __launch_bounds__(192, 2)
       last_q = n;
       for (int j = 0; j < it.nt; ++j, ++T) {
         const int st = (int)(T & 1);
-        if (T >= 2) ok = mbar_wait(kv_empty + st, ((T >> 1) - 1) & 1, abort_flag, a.status);
+        if (T >= 2) {
+          ok = mbar_wait(kt_empty + st, ((T >> 1) - 1) & 1, abort_flag, a.status);
+          if (ok) ok = mbar_wait(bias_empty + st, ((T >> 1) - 1) & 1, abort_flag, a.status);
+        }
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(kt_full + st, L::kTileBytes);
+          const int y = static_cast<int>(it.key_row0 + (long)j * NK);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_2d(sKt(st) + c * NK * 128, &tm_kt, kt_full + st, c * 64, y);
+        }
         float* bias = sBias + st * NK;
         for (int e = lane; e < NK; e += 32) {
           const int col = j * NK + e;
           bias[e] = col < a.nk ? __ldg(a.hs + it.key_row0 + col) * kLog2e : 0.f;
         }
-        if (lane == 0) {
-          mbar_arrive_expect_tx(kv_full + st, L::kStageBytes);
-          const int y = static_cast<int>(it.key_row0 + (long)j * NK);
-#pragma unroll
-          for (int c = 0; c < D / 64; ++c) {
-            tma_load_2d(sKt(st) + c * NK * 128, &tm_kt, kv_full + st, c * 64, y);
-            tma_load_2d(sY(st) + c * NK * 128, &tm_y, kv_full + st, c * 64, y);
-          }
-        } else {
-          mbar_arrive(kv_full + st);
-        }
+        mbar_arrive(bias_full + st);
       }
       ++n;
     }
     if (lane == 0 && *abort_flag) {  // drain the loads this warp issued (bounded)
       if (last_q >= 0) drain(q_full, last_q & 1);
-      for (long t = (T >= 2 ? T - 2 : 0); t < T; ++t) drain(kv_full + (t & 1), (t >> 1) & 1);
+      for (long t = (T >= 2 ? T - 2 : 0); t < T; ++t) drain(kt_full + (t & 1), (t >> 1) & 1);
     }
+  } else if (warp == 6) {
+    // ---------------------------- producer: Y -----------------------------
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_y);
+      long T = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
+        KOItem it;
+        if (!ko_decode<NK>(a, item, it)) continue;
+        for (int j = 0; j < it.nt; ++j, ++T) {
+          const int st = (int)(T & 1);
+          if (T >= 2) ok = mbar_wait(y_empty + st, ((T >> 1) - 1) & 1, abort_flag, a.status);
+          if (!ok) break;
+          mbar_arrive_expect_tx(y_full + st, L::kTileBytes);
+          const int y = static_cast<int>(it.key_row0 + (long)j * NK);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_2d(sY(st) + c * NK * 128, &tm_y, y_full + st, c * 64, y);
+        }
+      }
+      if (*abort_flag)
+        for (long t = (T >= 2 ? T - 2 : 0); t < T; ++t) drain(y_full + (t & 1), (t >> 1) & 1);
+    }
+    __syncwarp();
   } else if (warp == 1) {
     // -------------------------------- MMA ---------------------------------
     if (lane == 0) {
@@ -224,11 +258,12 @@ __global__ void __launch_bounds__(192, 2)
       long T = 0, last_s = -1, last_pv = -1;
       bool ok = true;
       auto issue_pv = [&](long Tp, bool first, int item_n) -> bool {
+        const int st = (int)(Tp & 1);
         if (!mbar_wait(p_full, Tp & 1, abort_flag, a.status)) return false;
+        if (!mbar_wait(y_full + st, (Tp >> 1) & 1, abort_flag, a.status)) return false;
         if (first && item_n >= 1 && !mbar_wait(o_empty, (item_n - 1) & 1, abort_flag, a.status))
           return false;
         tc_fence_after();
-        const int st = (int)(Tp & 1);
         const uint32_t pb = smem_u32(sP), yb = smem_u32(sY(st));
 #pragma unroll
         for (int kk = 0; kk < NK / 16; ++kk) {
@@ -236,7 +271,7 @@ __global__ void __launch_bounds__(192, 2)
           const uint64_t bd = desc_mnmajor(yb + kk * 16 * 128, NK * 128);
           mma_bf16_ss(tmem_o, ad, bd, idesc_o, (!first || kk > 0) ? 1u : 0u);
         }
-        mma_commit(kv_empty + st);
+        mma_commit(y_empty + st);
         mma_commit(pv_done);
         last_pv = Tp;
         return true;
@@ -248,7 +283,7 @@ __global__ void __launch_bounds__(192, 2)
         const long T0 = T;
         for (int j = 0; j < it.nt && ok; ++j, ++T) {
           const int st = (int)(T & 1);
-          ok = mbar_wait(kv_full + st, (T >> 1) & 1, abort_flag, a.status);
+          ok = mbar_wait(kt_full + st, (T >> 1) & 1, abort_flag, a.status);
           if (ok && T >= 2) ok = mbar_wait(s_empty + st, ((T >> 1) - 1) & 1, abort_flag, a.status);
           if (!ok) break;
           tc_fence_after();
@@ -260,6 +295,7 @@ __global__ void __launch_bounds__(192, 2)
             mma_bf16_ss(tmem_s(st), ad, bd, idesc_s, kk > 0 ? 1u : 0u);
           }
           mma_commit(s_full + st);
+          mma_commit(kt_empty + st);
           last_s = T;
           if (j == it.nt - 1) mma_commit(q_empty);
           if (j >= 1) ok = issue_pv(T - 1, j == 1, n);
@@ -287,7 +323,7 @@ __global__ void __launch_bounds__(192, 2)
       for (int j = 0; j < it.nt; ++j, ++T) {
         const int sb = (int)(T & 1);
         ok = mbar_wait(s_full + sb, (T >> 1) & 1, abort_flag, a.status);
-        if (ok) ok = mbar_wait(kv_full + sb, (T >> 1) & 1, abort_flag, a.status);  // bias
+        if (ok) ok = mbar_wait(bias_full + sb, (T >> 1) & 1, abort_flag, a.status);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         float sv[NK];
@@ -300,8 +336,6 @@ __global__ void __launch_bounds__(192, 2)
           for (int e = 0; e < 32; ++e) sv[c * 32 + e] = t[e];
         }
         tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(s_empty + sb);
         const float* bias = sBias + sb * NK;
         const int valid = a.nk - j * NK;
         // logits in log2 units; 4 partial maxima / sums break the serial chains
@@ -319,6 +353,9 @@ __global__ void __launch_bounds__(192, 2)
             mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
           }
         }
+        tc_fence_before();
+        mbar_arrive(s_empty + sb);
+        mbar_arrive(bias_empty + sb);
         const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
         float alpha = 1.f;
         bool resc = false;
@@ -792,7 +829,7 @@ cudaError_t launch_ko(const bf16* q, const bf16* kt, const bf16* y, const float*
   a.status = status;
   const int grid = (int)std::min<long>(items, 2L * num_sms());
   return timed_launch("tc_l_output", stream, launches, [&] {
-    ko_kernel<D, NK><<<grid, 192, L::kAlloc, stream>>>(tq, tk, tyv, a);
+    ko_kernel<D, NK><<<grid, 224, L::kAlloc, stream>>>(tq, tk, tyv, a);
   });
 }
 
