@@ -26,6 +26,7 @@
 #include <cudaTypedefs.h>
 
 #include <mutex>
+#include <utility>
 
 #include "simt_kernels.cuh"
 #include "tc_ptx.cuh"
@@ -123,6 +124,7 @@ __global__ void __launch_bounds__(224, 2)
     if (tid == 0) atomicExch(a.status, 2);
     return;
   }
+  pdl_launch_dependents();
   uint8_t* sQ = smem;
   uint8_t* sP = smem + L::kPOff;
   float* sBias = reinterpret_cast<float*>(smem + L::kBiasOff);
@@ -196,6 +198,7 @@ __global__ void __launch_bounds__(224, 2)
         for (int c = 0; c < D / 64; ++c)
           tma_load_3d(sQ + c * kRows * 128, &tm_q, q_full, c * 64, it.i, it.g * a.b1 + it.row0);
       }
+      if (n == 0) pdl_wait();  // Kt, Hs come from the previous kernel
       last_q = n;
       for (int j = 0; j < it.nt; ++j, ++T) {
         const int st = (int)(T & 1);
@@ -229,6 +232,7 @@ __global__ void __launch_bounds__(224, 2)
     // ---------------------------- producer: Y -----------------------------
     if (lane == 0) {
       tma_prefetch_desc(&tm_y);
+      pdl_wait();  // Y comes from the previous kernel
       long T = 0;
       bool ok = true;
       for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
@@ -462,24 +466,28 @@ __global__ void __launch_bounds__(224, 2)
 // column chunks x row lanes, reduced through shared memory.
 // ---------------------------------------------------------------------------
 template <int D>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(512)
     init_qt_bf16_kernel(const bf16* __restrict__ q, bf16* __restrict__ qt0, int b1, int b2,
                         int c1) {
-  constexpr int CH = D / 8;
-  constexpr int LANES = 256 / CH;
-  __shared__ float red[LANES][D];
+  constexpr int CH = D / 8;          // 16-byte chunks per row
+  constexpr int LANES = 512 / CH;    // rows summed in parallel
+  __shared__ float red[LANES][D + 1];
   int bid = blockIdx.x;
   const int i = bid % b2;
   bid /= b2;
   const int p = bid % c1;
   const long g = bid / c1;
   const int l0 = group_start(b1, c1, p), l1 = group_start(b1, c1, p + 1);
+  pdl_launch_dependents();
   const int ch = threadIdx.x % CH, lane = threadIdx.x / CH;
   float acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  const uint4* base = reinterpret_cast<const uint4*>(q + (g * b1 * b2 + i) * D) + ch;
+  const long row_stride = (long)b2 * D / 8;  // in uint4
+#pragma unroll 4
   for (int l = l0 + lane; l < l1; l += LANES) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(q + ((g * b1 + l) * b2 + i) * D) + ch);
+    const uint4 u = __ldg(base + l * row_stride);
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -492,7 +500,7 @@ __global__ void __launch_bounds__(256)
   __syncthreads();
   if (threadIdx.x < D) {
     float sum = 0.f;
-#pragma unroll 4
+#pragma unroll 8
     for (int ln = 0; ln < LANES; ++ln) sum += red[ln][threadIdx.x];
     qt0[((g * c1 + p) * b2 + i) * D + threadIdx.x] = __float2bfloat16_rn(sum / (float)(l1 - l0));
   }
@@ -526,8 +534,10 @@ struct KRLayout {
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = D / 64 * kRows * 128;
   static constexpr int kPBytes = (NQ + 63) / 64 * kRows * 128;
+  static constexpr int kStageBytes = kRows * 128;  // one 64-column staging block
   __host__ __device__ static constexpr int p_off(int c2) { return kKVOff + c2 * kGroupBytes; }
-  __host__ __device__ static constexpr int bar_off(int c2) { return p_off(c2) + kPBytes; }
+  __host__ __device__ static constexpr int stage_off(int c2) { return p_off(c2) + kPBytes; }
+  __host__ __device__ static constexpr int bar_off(int c2) { return stage_off(c2) + kStageBytes; }
   __host__ __device__ static constexpr int bytes(int c2) { return bar_off(c2) + 64; }
   static constexpr uint32_t kTmemCols = 2 * D;  // O (2d columns); S_q uses the first NQ
   static_assert(NQ % 16 == 0 && NQ <= 128 && NQ <= 2 * D, "group tile");
@@ -536,7 +546,8 @@ struct KRLayout {
 template <int D, int NQ>
 __global__ void __launch_bounds__(128)
     kr_kernel(const __grid_constant__ CUtensorMap tm_qt, const __grid_constant__ CUtensorMap tm_k,
-              const __grid_constant__ CUtensorMap tm_v, KRArgs a) {
+              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kt,
+              const __grid_constant__ CUtensorMap tm_y, KRArgs a) {
   using L = KRLayout<D, NQ>;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -553,6 +564,7 @@ __global__ void __launch_bounds__(128)
   uint8_t* sQ = smem + L::kQOff;
   auto sK = [&](int q) { return smem + L::kKVOff + q * L::kGroupBytes; };
   uint8_t* sP = smem + L::p_off(a.c2);
+  uint8_t* sStage[2] = {sP, smem + L::stage_off(a.c2)};  // P is free once [Kt | Y] is done
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::bar_off(a.c2));
   uint64_t* load_full = bars + 0;
   uint64_t* s_full = bars + 1;
@@ -577,6 +589,7 @@ __global__ void __launch_bounds__(128)
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
 
+  pdl_launch_dependents();
   bool load_waited = false;
   int s_issued = 0, o_issued = 0;
   auto issue_s = [&](int q) {
@@ -597,9 +610,6 @@ __global__ void __launch_bounds__(128)
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
     mbar_arrive_expect_tx(load_full, D / 64 * kRows * 128 + a.c2 * L::kGroupBytes);
-    const int qrow = (g * a.c1 + p) * a.b2;
-#pragma unroll
-    for (int c = 0; c < D / 64; ++c) tma_load_2d(sQ + c * kRows * 128, &tm_qt, load_full, c * 64, qrow);
     for (int q = 0; q < a.c2; ++q) {
       const int krow = (g * a.b1 + k) * a.b2 + group_start(a.b2, a.c2, q);
 #pragma unroll
@@ -608,6 +618,10 @@ __global__ void __launch_bounds__(128)
         tma_load_2d(sK(q) + (D / 64 + c) * L::kBox, &tm_v, load_full, c * 64, krow);
       }
     }
+    pdl_wait();  // Qt0 comes from the previous kernel
+    const int qrow = (g * a.c1 + p) * a.b2;
+#pragma unroll
+    for (int c = 0; c < D / 64; ++c) tma_load_2d(sQ + c * kRows * 128, &tm_qt, load_full, c * 64, qrow);
     load_waited = mbar_wait(load_full, 0, abort_flag, a.status);
     if (load_waited) issue_s(0);
   }
@@ -681,13 +695,19 @@ __global__ void __launch_bounds__(128)
     if (ok) {
       tc_fence_after();
       const float inv = 1.f / z;
-      // Rows (positions i, b2*c1*b1*c2*d elements apart) go out through the
-      // P buffer (free once [Kt | Y] is complete; the Qt0 tile must survive
-      // for the next group): 64 columns at a time, each thread stages its
-      // row, then 8 threads write one row's 128 bytes as whole sectors.
+      // The b2 rows of this (g, p, k, q) are positions i of the position-major
+      // Kt/Y layout: one 3-D TMA box {64 columns, 1, b2 rows}.  Each 64-column
+      // block is staged (swizzled) in one of two buffers and handed to a TMA
+      // bulk store; a buffer is refilled once its previous store has read it.
       const int nblk = (a.write_y ? 2 : 1) * (D / 64);
+      const int ycoord = (p * a.b1 + k) * a.c2 + q;
 #pragma unroll 1
       for (int cb = 0; cb < nblk; ++cb) {
+        uint8_t* buf = sStage[cb & 1];
+        if (cb >= 2) {
+          if (tid == 0) bulk_wait_read<1>();
+          __syncthreads();
+        }
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           float t[32];
@@ -701,22 +721,18 @@ __global__ void __launch_bounds__(128)
             pk.z = pack_bf16x2(t[8 * u + 4] * inv, t[8 * u + 5] * inv);
             pk.w = pack_bf16x2(t[8 * u + 6] * inv, t[8 * u + 7] * inv);
             const int unit = c * 4 + u;
-            *reinterpret_cast<uint4*>(sP + r * 128 + ((unit ^ (r & 7)) << 4)) = pk;
+            *reinterpret_cast<uint4*>(buf + r * 128 + ((unit ^ (r & 7)) << 4)) = pk;
           }
         }
+        fence_proxy_async_smem();
         __syncthreads();
-        bf16* base = (cb < D / 64 ? a.kt : a.y) + (cb % (D / 64)) * 64;
-#pragma unroll
-        for (int pass = 0; pass < kRows / 16; ++pass) {
-          const int rr = pass * 16 + (tid >> 3), unit = tid & 7;
-          if (rr < a.b2) {
-            const uint4 v4 = *reinterpret_cast<const uint4*>(sP + rr * 128 + ((unit ^ (rr & 7)) << 4));
-            const long orr = ((((long)g * a.b2 + rr) * a.c1 + p) * a.b1 + k) * a.c2 + q;
-            *reinterpret_cast<uint4*>(base + orr * D + unit * 8) = v4;
-          }
+        if (tid == 0) {
+          tma_store_3d(cb < D / 64 ? &tm_kt : &tm_y, buf, (cb % (D / 64)) * 64, ycoord, g * a.b2);
+          bulk_commit();
         }
-        __syncthreads();
       }
+      // the staging buffers (P among them) are reused by the next group
+      if (tid == 0) bulk_wait_read<0>();
       // entropy of the R row: ln z - sum e (s - m) / z, with s - m in log2 units
       if (row_valid) {
         const long orow = ((((long)g * a.b2 + r) * a.c1 + p) * a.b1 + k) * a.c2 + q;
@@ -733,11 +749,331 @@ __global__ void __launch_bounds__(128)
     if (s_issued > 0) drain(s_full, (s_issued - 1) & 1);
     if (o_issued > 0) drain(o_full, (o_issued - 1) & 1);
   }
+  if (tid == 0) bulk_wait<0>();  // stores done reading shared memory before the CTA exits
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Persistent R-update (step one) for column-group tiles NQ <= 64.  One CTA
+// per SM walks a contiguous range of items (g, p, k), each split into c2
+// sub-items (one per column group q).  Warp 0 loads (Qt0 once per (g, p),
+// K_q / V_q through a three-slot ring), warp 1 issues the MMAs, and two
+// warpgroups (warps 2-5 and 6-9) take alternate sub-items: softmax, then
+// the Kt / Y rows through double-buffered TMA bulk stores.  Each warpgroup
+// owns one 2d-column TMEM slot in which S is later overwritten by
+// [Kt | Y], so sub-item n+1's S and softmax overlap sub-item n's stores.
+// Barriers (sub-item counter n over the CTA's items):
+//   q_full / q_empty       Qt0 tile        kv_full / kv_empty   K/V ring
+//   s_full[w] / o_full[w]  S / [Kt | Y] of warpgroup w's slot complete
+//   p_full[w]              P written       tmem_free[w]         slot read out
+// ---------------------------------------------------------------------------
+template <int D, int NQ>
+struct KR2Layout {
+  static constexpr int kBox = NQ * 128;
+  static constexpr int kKVBytes = 2 * (D / 64) * kBox;  // K_q then V_q
+  static constexpr int kKVSlots = 3;
+  static constexpr int kQOff = 0;
+  static constexpr int kKVOff = D / 64 * kRows * 128;
+  static constexpr int kPOff = kKVOff + kKVSlots * kKVBytes;     // [2] x 16 KB
+  static constexpr int kStageOff = kPOff + 2 * kRows * 128;      // [2 wg][2] x 16 KB
+  static constexpr int kBarOff = kStageOff + 4 * kRows * 128;
+  static constexpr int kBytes = kBarOff + 32 * 8;
+  static_assert(NQ % 16 == 0 && NQ <= 64, "group tile");
+  static_assert(kBytes <= 227 * 1024, "shared memory");
+};
+
+struct KR2Args {
+  float* hs;
+  int b1, b2, c1, c2, n_items, write_y;
+  float sc_log2;
+  int* status;
+};
+
+struct KR2Sub {
+  int g, p, k, q, gp;
+};
+
+__device__ __forceinline__ KR2Sub kr2_sub(const KR2Args& a, long n_sub) {
+  KR2Sub s;
+  const int item = (int)(n_sub / a.c2);
+  s.q = (int)(n_sub % a.c2);
+  s.k = item % a.b1;
+  s.gp = item / a.b1;  // g * c1 + p
+  s.p = s.gp % a.c1;
+  s.g = s.gp / a.c1;
+  return s;
+}
+
+template <int D, int NQ>
+__global__ void __launch_bounds__(320, 1)
+    kr2_kernel(const __grid_constant__ CUtensorMap tm_qt, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kt,
+               const __grid_constant__ CUtensorMap tm_y, KR2Args a) {
+  using L = KR2Layout<D, NQ>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (smem_u32(smem) & 1023u) {
+    if (tid == 0) atomicExch(a.status, 2);
+    return;
+  }
+  pdl_launch_dependents();
+  // this CTA's sub-items [s0, s1)
+  const long n_sub = (long)a.n_items * a.c2;
+  const long s0 = n_sub * blockIdx.x / gridDim.x, s1 = n_sub * (blockIdx.x + 1) / gridDim.x;
+
+  uint8_t* sQ = smem + L::kQOff;
+  auto sKV = [&](int sl) { return smem + L::kKVOff + sl * L::kKVBytes; };
+  auto sP = [&](int w) { return smem + L::kPOff + w * kRows * 128; };
+  auto sStage = [&](int w, int b) { return smem + L::kStageOff + (w * 2 + b) * kRows * 128; };
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* q_full = bars + 0;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* kv_full = bars + 2;    // [3]
+  uint64_t* kv_empty = bars + 5;   // [3]
+  uint64_t* s_full = bars + 8;     // [2]
+  uint64_t* o_full = bars + 10;    // [2]
+  uint64_t* p_full = bars + 12;    // [2]
+  uint64_t* tmem_free = bars + 14; // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 17);
+
+  if (tid == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int i = 0; i < 3; ++i) {
+      mbar_init(kv_full + i, 1);
+      mbar_init(kv_empty + i, 1);
+    }
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(s_full + w, 1);
+      mbar_init(o_full + w, 1);
+      mbar_init(p_full + w, 128);
+      mbar_init(tmem_free + w, 128);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------ producer ------------------------------
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_qt);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      int cur_gp = -1, nq_loads = 0;
+      bool ok = true;
+      long last_kv = -1;
+      for (long n = s0; n < s1 && ok; ++n) {
+        const KR2Sub sb = kr2_sub(a, n);
+        const long u = n - s0;
+        const int sl = (int)(u % 3);
+        if (u >= 3) ok = mbar_wait(kv_empty + sl, ((u / 3) - 1) & 1, abort_flag, a.status);
+        if (!ok) break;
+        const int krow = (sb.g * a.b1 + sb.k) * a.b2 + group_start(a.b2, a.c2, sb.q);
+        mbar_arrive_expect_tx(kv_full + sl, L::kKVBytes);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_2d(sKV(sl) + c * L::kBox, &tm_k, kv_full + sl, c * 64, krow);
+          tma_load_2d(sKV(sl) + (D / 64 + c) * L::kBox, &tm_v, kv_full + sl, c * 64, krow);
+        }
+        last_kv = u;
+        if (sb.gp != cur_gp) {
+          if (nq_loads == 0) pdl_wait();  // Qt0 comes from the previous kernel
+          if (nq_loads >= 1) ok = mbar_wait(q_empty, (nq_loads - 1) & 1, abort_flag, a.status);
+          if (!ok) break;
+          mbar_arrive_expect_tx(q_full, D / 64 * kRows * 128);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_2d(sQ + c * kRows * 128, &tm_qt, q_full, c * 64, sb.gp * a.b2);
+          cur_gp = sb.gp;
+          ++nq_loads;
+        }
+      }
+      if (*abort_flag) {
+        if (nq_loads >= 1) drain(q_full, (nq_loads - 1) & 1);
+        for (long u = (last_kv >= 2 ? last_kv - 2 : 0); u <= last_kv; ++u) drain(kv_full + u % 3, (u / 3) & 1);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // -------------------------------- MMA ---------------------------------
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_bf16(kRows, NQ, false);
+      const uint32_t idesc_o = idesc_bf16(kRows, 2 * D, true);
+      int cur_gp = -1, nq_loads = 0;
+      bool ok = true;
+      long last_s = -1, last_o = -1;
+      auto issue_pv = [&](long u) -> bool {
+        const int w = (int)(u & 1);
+        if (!mbar_wait(p_full + w, (u >> 1) & 1, abort_flag, a.status)) return false;
+        tc_fence_after();
+        const uint32_t pb = smem_u32(sP(w)), kb = smem_u32(sKV((int)(u % 3)));
+#pragma unroll
+        for (int kk = 0; kk < NQ / 16; ++kk) {
+          const uint64_t ad = desc_kmajor(pb + (kk & 3) * 32);
+          const uint64_t bd = desc_mnmajor(kb + kk * 16 * 128, L::kBox);
+          mma_bf16_ss(tmem + w * 256, ad, bd, idesc_o, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(o_full + w);
+        mma_commit(kv_empty + (int)(u % 3));
+        last_o = u;
+        return true;
+      };
+      for (long n = s0; n < s1 && ok; ++n) {
+        const KR2Sub sb = kr2_sub(a, n);
+        const long u = n - s0;
+        const int w = (int)(u & 1), sl = (int)(u % 3);
+        if (sb.gp != cur_gp) {
+          ok = mbar_wait(q_full, nq_loads & 1, abort_flag, a.status);
+          cur_gp = sb.gp;
+          ++nq_loads;
+        }
+        if (ok) ok = mbar_wait(kv_full + sl, (u / 3) & 1, abort_flag, a.status);
+        if (ok && u >= 2) ok = mbar_wait(tmem_free + w, ((u >> 1) - 1) & 1, abort_flag, a.status);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t qb = smem_u32(sQ), kb = smem_u32(sKV(sl));
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t ad = desc_kmajor(qb + (kk >> 2) * (kRows * 128) + (kk & 3) * 32);
+          const uint64_t bd = desc_kmajor(kb + (kk >> 2) * L::kBox + (kk & 3) * 32);
+          mma_bf16_ss(tmem + w * 256, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(s_full + w);
+        last_s = u;
+        if (n + 1 >= s1 || kr2_sub(a, n + 1).gp != cur_gp) mma_commit(q_empty);
+        if (u >= 1) ok = issue_pv(u - 1);
+      }
+      if (ok && s1 > s0) ok = issue_pv(s1 - 1 - s0);
+      if (*abort_flag) {
+        if (last_s >= 0) drain(s_full + (last_s & 1), (last_s >> 1) & 1);
+        if (last_o >= 0) drain(o_full + (last_o & 1), (last_o >> 1) & 1);
+      }
+    }
+    __syncwarp();
+  } else {
+    // -------------------- softmax + epilogue (two warpgroups) --------------------
+    const int w = (warp - 2) >> 2;            // warpgroup 0: warps 2-5, 1: warps 6-9
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;           // TMEM lane == row == position i
+    const int wtid = tid - 64 - w * 128;      // 0..127 inside the warpgroup
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t tslot = tmem + w * 256;
+    const bool leader = wtid == 0;
+    int nst = 0;  // stores issued by this warpgroup; buffer nst & 1
+    bool ok = true;
+    for (long n = s0 + w; n < s1 && ok; n += 2) {
+      const KR2Sub sb = kr2_sub(a, n);
+      const long u = n - s0;
+      const int nq = group_start(a.b2, a.c2, sb.q + 1) - group_start(a.b2, a.c2, sb.q);
+      ok = mbar_wait(s_full + w, (u >> 1) & 1, abort_flag, a.status);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      float sv[NQ];
+#pragma unroll
+      for (int c = 0; c < NQ / 16; ++c) {
+        float t[16];
+        tmem_ld16(tslot + lane_off + c * 16, t);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) sv[c * 16 + e] = t[e];
+      }
+      tmem_wait_ld();
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int j = 0; j < NQ; ++j) {
+        sv[j] = j < nq ? sv[j] * a.sc_log2 : -INFINITY;
+        mx[j & 3] = fmaxf(mx[j & 3], sv[j]);
+      }
+      const float m2 = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      float zs[4] = {0.f, 0.f, 0.f, 0.f}, ts[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int j = 0; j < NQ; ++j) {
+        const float d2 = sv[j] - m2;
+        sv[j] = ex2(d2);
+        zs[j & 3] += sv[j];
+        ts[j & 3] += j < nq ? sv[j] * d2 : 0.f;
+      }
+      const float z = (zs[0] + zs[1]) + (zs[2] + zs[3]);
+      const float t2 = (ts[0] + ts[1]) + (ts[2] + ts[3]);
+      uint8_t* pbuf = sP(w);
+#pragma unroll
+      for (int uu = 0; uu < NQ / 8; ++uu) {
+        uint4 pk;
+        pk.x = pack_bf16x2(sv[8 * uu + 0], sv[8 * uu + 1]);
+        pk.y = pack_bf16x2(sv[8 * uu + 2], sv[8 * uu + 3]);
+        pk.z = pack_bf16x2(sv[8 * uu + 4], sv[8 * uu + 5]);
+        pk.w = pack_bf16x2(sv[8 * uu + 6], sv[8 * uu + 7]);
+        *reinterpret_cast<uint4*>(pbuf + r * 128 + ((uu ^ (r & 7)) << 4)) = pk;
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(p_full + w);
+      ok = mbar_wait(o_full + w, (u >> 1) & 1, abort_flag, a.status);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const float inv = 1.f / z;
+      const int nblk = (a.write_y ? 2 : 1) * (D / 64);
+      const int ycoord = (sb.p * a.b1 + sb.k) * a.c2 + sb.q;
+#pragma unroll 1
+      for (int cb = 0; cb < nblk; ++cb, ++nst) {
+        uint8_t* buf = sStage(w, nst & 1);
+        if (leader) bulk_wait_read<1>();  // the store that last used buf has read it
+        named_barrier(1 + w, 128);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          float t[32];
+          tmem_ld32(tslot + lane_off + cb * 64 + c * 32, t);
+          tmem_wait_ld();
+#pragma unroll
+          for (int uu = 0; uu < 4; ++uu) {
+            uint4 pk;
+            pk.x = pack_bf16x2(t[8 * uu + 0] * inv, t[8 * uu + 1] * inv);
+            pk.y = pack_bf16x2(t[8 * uu + 2] * inv, t[8 * uu + 3] * inv);
+            pk.z = pack_bf16x2(t[8 * uu + 4] * inv, t[8 * uu + 5] * inv);
+            pk.w = pack_bf16x2(t[8 * uu + 6] * inv, t[8 * uu + 7] * inv);
+            const int unit = c * 4 + uu;
+            *reinterpret_cast<uint4*>(buf + r * 128 + ((unit ^ (r & 7)) << 4)) = pk;
+          }
+        }
+        if (cb == nblk - 1) {  // slot fully read out: the MMA may reuse it
+          tc_fence_before();
+          mbar_arrive(tmem_free + w);
+        }
+        fence_proxy_async_smem();
+        named_barrier(1 + w, 128);
+        if (leader) {
+          tma_store_3d(cb < D / 64 ? &tm_kt : &tm_y, buf, (cb % (D / 64)) * 64, ycoord,
+                       sb.g * a.b2);
+          bulk_commit();
+        }
+      }
+      if (r < a.b2) {
+        const long orow = ((((long)sb.g * a.b2 + r) * a.c1 + sb.p) * a.b1 + sb.k) * a.c2 + sb.q;
+        a.hs[orow] = logf(z) - t2 * 0.69314718055994531f * inv;
+      }
+    }
+    if (leader) bulk_wait<0>();  // stores done reading shared memory before exit
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -769,6 +1105,25 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Launch with programmatic stream serialisation: the kernel may start while
+// the previous kernel of the stream finishes; it calls pdl_wait() before it
+// reads anything that kernel wrote.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 int num_sms() {
@@ -829,7 +1184,7 @@ cudaError_t launch_ko(const bf16* q, const bf16* kt, const bf16* y, const float*
   a.status = status;
   const int grid = (int)std::min<long>(items, 2L * num_sms());
   return timed_launch("tc_l_output", stream, launches, [&] {
-    ko_kernel<D, NK><<<grid, 224, L::kAlloc, stream>>>(tq, tk, tyv, a);
+    return launch_pdl(ko_kernel<D, NK>, dim3(grid), dim3(224), L::kAlloc, stream, tq, tk, tyv, a);
   });
 }
 
@@ -863,6 +1218,16 @@ cudaError_t launch_kr(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, b
     if (!make_map(&tk, k, 2, dims, str, box)) return cudaErrorInvalidValue;
     if (!make_map(&tv, v, 2, dims, str, box)) return cudaErrorInvalidValue;
   }
+  CUtensorMap tkt, tyy;
+  {
+    // Kt / Y [G][b2 i][c1 p][b1 k][c2 q][d] viewed as (d, c1*b1*c2, G*b2)
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)pb.c1 * pb.b1 * pb.c2,
+                                (cuuint64_t)pb.G * pb.b2};
+    const cuuint64_t str[2] = {(cuuint64_t)D * 2, (cuuint64_t)pb.c1 * pb.b1 * pb.c2 * D * 2};
+    const cuuint32_t box[3] = {64, 1, (cuuint32_t)pb.b2};
+    if (!make_map(&tkt, kt, 3, dims, str, box)) return cudaErrorInvalidValue;
+    if (!make_map(&tyy, y, 3, dims, str, box)) return cudaErrorInvalidValue;
+  }
   KRArgs a;
   a.kt = kt;
   a.y = y;
@@ -876,7 +1241,61 @@ cudaError_t launch_kr(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, b
   a.status = status;
   const long blocks = (long)pb.G * pb.b1 * pb.c1;
   return timed_launch("tc_r_update", stream, launches, [&] {
-    kr_kernel<D, NQ><<<(unsigned)blocks, 128, L::bytes(pb.c2), stream>>>(tq, tk, tv, a);
+    return launch_pdl(kr_kernel<D, NQ>, dim3((unsigned)blocks), dim3(128), L::bytes(pb.c2), stream, tq,
+               tk, tv, tkt, tyy, a);
+  });
+}
+
+template <int D, int NQ>
+cudaError_t launch_kr2(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, bf16* y,
+                       float* hs, const Problem& pb, int* status, cudaStream_t stream,
+                       int* launches) {
+  using L = KR2Layout<D, NQ>;
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(kr2_kernel<D, NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    L::kBytes);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  CUtensorMap tq, tk, tv, tkt, tyy;
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)pb.G * pb.c1 * pb.b2};
+    const cuuint64_t str[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64, kRows};
+    if (!make_map(&tq, qt0, 2, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)pb.G * pb.b1 * pb.b2};
+    const cuuint64_t str[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)NQ};
+    if (!make_map(&tk, k, 2, dims, str, box)) return cudaErrorInvalidValue;
+    if (!make_map(&tv, v, 2, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)pb.c1 * pb.b1 * pb.c2,
+                                (cuuint64_t)pb.G * pb.b2};
+    const cuuint64_t str[2] = {(cuuint64_t)D * 2, (cuuint64_t)pb.c1 * pb.b1 * pb.c2 * D * 2};
+    const cuuint32_t box[3] = {64, 1, (cuuint32_t)pb.b2};
+    if (!make_map(&tkt, kt, 3, dims, str, box)) return cudaErrorInvalidValue;
+    if (!make_map(&tyy, y, 3, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  KR2Args a;
+  a.hs = hs;
+  a.b1 = pb.b1;
+  a.b2 = pb.b2;
+  a.c1 = pb.c1;
+  a.c2 = pb.c2;
+  const long items = (long)pb.G * pb.c1 * pb.b1;
+  if (items * pb.c2 >= (1L << 31)) return cudaErrorInvalidValue;
+  a.n_items = (int)items;
+  a.write_y = pb.T == 1 ? 1 : 0;
+  a.sc_log2 = kLog2e * pb.sc;
+  a.status = status;
+  const int grid = (int)std::min<long>(items * pb.c2, num_sms());
+  return timed_launch("tc_r_update", stream, launches, [&] {
+    return launch_pdl(kr2_kernel<D, NQ>, dim3(grid), dim3(320), L::kBytes, stream, tq, tk, tv,
+                      tkt, tyy, a);
   });
 }
 
@@ -891,17 +1310,20 @@ cudaError_t dispatch_kr(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt,
                         float* hs, const Problem& pb, int* status, cudaStream_t stream,
                         int* launches) {
   switch (kr_group_tile(pb)) {
+#define MONARCH_KR2_CASE(NQ) \
+  case NQ: return launch_kr2<D, NQ>(qt0, k, v, kt, y, hs, pb, status, stream, launches);
 #define MONARCH_KR_CASE(NQ) \
   case NQ: return launch_kr<D, NQ>(qt0, k, v, kt, y, hs, pb, status, stream, launches);
-    MONARCH_KR_CASE(16)
-    MONARCH_KR_CASE(32)
-    MONARCH_KR_CASE(48)
-    MONARCH_KR_CASE(64)
+    MONARCH_KR2_CASE(16)
+    MONARCH_KR2_CASE(32)
+    MONARCH_KR2_CASE(48)
+    MONARCH_KR2_CASE(64)
     MONARCH_KR_CASE(80)
     MONARCH_KR_CASE(96)
     MONARCH_KR_CASE(112)
     MONARCH_KR_CASE(128)
 #undef MONARCH_KR_CASE
+#undef MONARCH_KR2_CASE
     default: return cudaErrorInvalidValue;
   }
 }
@@ -912,7 +1334,7 @@ cudaError_t launch_r_step1(const bf16* q, const bf16* k, const bf16* v, bf16* qt
                            bf16* y, float* hs, const Problem& pb, int* status,
                            cudaStream_t stream, int* launches) {
   cudaError_t e = timed_launch("tc_init_qt", stream, launches, [&] {
-    init_qt_bf16_kernel<D><<<(unsigned)((long)pb.G * pb.c1 * pb.b2), 256, 0, stream>>>(
+    init_qt_bf16_kernel<D><<<(unsigned)((long)pb.G * pb.c1 * pb.b2), 512, 0, stream>>>(
         q, qt0, pb.b1, pb.b2, pb.c1);
   });
   if (e != cudaSuccess) return e;

@@ -4,6 +4,8 @@
 
 #include <cuda_runtime.h>
 
+#include <type_traits>
+
 namespace monarch {
 
 bool timing_enabled();
@@ -23,11 +25,19 @@ class KernelTimer {
 
 // Launch `f` (a lambda that performs one <<<>>> launch), timing it when
 // enabled, checking the launch error and counting it in *launches.
+// `f` may return the launch's cudaError_t (cudaLaunchKernelEx) or nothing
+// (a <<<>>> launch, checked with cudaGetLastError).
 template <typename F>
 cudaError_t timed_launch(const char* name, cudaStream_t stream, int* launches, F&& f) {
   KernelTimer t(name, stream);
-  f();
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e;
+  if constexpr (std::is_same<decltype(f()), cudaError_t>::value) {
+    e = f();
+    if (e == cudaSuccess) e = cudaGetLastError();
+  } else {
+    f();
+    e = cudaGetLastError();
+  }
   t.stop();
   if (e == cudaSuccess) ++*launches;
   return e;
