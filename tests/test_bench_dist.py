@@ -1,0 +1,66 @@
+"""Multi-rank host logic of bench.py on CPU: world size 2 over gloo.
+
+The forward pass shards into independent heads, so ranks share no data; the
+only cross-rank step is the timing reduction (max over ranks) and the
+whole-job throughput computed from it.
+"""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        dev = torch.device("cpu")
+        assert bench.dist_env() == (rank, rank, world)
+        # rank r "took" 10 + r milliseconds: everyone must see the slowest
+        t = bench.reduce_max(10.0 + rank, dev)
+        bench.barrier(dev)
+        value = bench.job_value(100.0, world, t / 1e3)
+        out[rank] = (t, value)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2])
+def test_reduce_max_and_job_value_over_gloo(world):
+    port = _free_port()
+    out = mp.Manager().dict()
+    mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
+    assert sorted(out.keys()) == list(range(world))
+    for rank in range(world):
+        t, value = out[rank]
+        assert t == 10.0 + (world - 1)
+        assert value == pytest.approx(100.0 * world / (t / 1e3))
+
+
+def test_single_process_helpers_are_identity():
+    dev = torch.device("cpu")
+    assert bench.reduce_max(3.5, dev) == 3.5
+    bench.barrier(dev)  # no process group: no-op
+    assert bench.job_value(10.0, 1, 2.0) == 5.0
+
+
+def test_work_model_matches_the_flop_formula():
+    from structured_sub_quadratic_b200.inputs import WORKLOADS
+    wl = WORKLOADS["480p"]
+    # 2 N d [(2T+1) c1 b2 + 2T c2 b1] per head, 12 heads
+    assert bench.alg_flops(wl) == 12 * 2 * 4680 * 128 * (3 * 52 + 2 * 90)
+    assert bench.alg_bytes(wl) == 12 * 4 * 4680 * 128 * 2
+    fl, by = bench.kernel_work("tc_l_output", wl)
+    assert fl == 12 * 4680 * 90 * 128 * 4 and by > 0
