@@ -932,32 +932,37 @@ __global__ void __launch_bounds__(320, 1)
         last_o = u;
         return true;
       };
-      for (long n = s0; n < s1 && ok; ++n) {
-        const KR2Sub sb = kr2_sub(a, n);
-        const long u = n - s0;
-        const int w = (int)(u & 1), sl = (int)(u % 3);
-        if (sb.gp != cur_gp) {
-          ok = mbar_wait(q_full, nq_loads & 1, abort_flag, a.status);
-          cur_gp = sb.gp;
-          ++nq_loads;
-        }
-        if (ok) ok = mbar_wait(kv_full + sl, (u / 3) & 1, abort_flag, a.status);
-        if (ok && u >= 2) ok = mbar_wait(tmem_free + w, ((u >> 1) - 1) & 1, abort_flag, a.status);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t qb = smem_u32(sQ), kb = smem_u32(sKV(sl));
+      // Sub-items go in pairs, one per warpgroup: both S products first, then
+      // both [Kt | Y] products, so that neither warpgroup's product waits
+      // behind the other's epilogue.
+      for (long nb = s0; nb < s1 && ok; nb += 2) {
+        const long ne = nb + 2 < s1 ? nb + 2 : s1;
+        for (long n = nb; n < ne && ok; ++n) {
+          const KR2Sub sb = kr2_sub(a, n);
+          const long u = n - s0;
+          const int w = (int)(u & 1), sl = (int)(u % 3);
+          if (sb.gp != cur_gp) {
+            ok = mbar_wait(q_full, nq_loads & 1, abort_flag, a.status);
+            cur_gp = sb.gp;
+            ++nq_loads;
+          }
+          if (ok) ok = mbar_wait(kv_full + sl, (u / 3) & 1, abort_flag, a.status);
+          if (ok && u >= 2) ok = mbar_wait(tmem_free + w, ((u >> 1) - 1) & 1, abort_flag, a.status);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t qb = smem_u32(sQ), kb = smem_u32(sKV(sl));
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t ad = desc_kmajor(qb + (kk >> 2) * (kRows * 128) + (kk & 3) * 32);
-          const uint64_t bd = desc_kmajor(kb + (kk >> 2) * L::kBox + (kk & 3) * 32);
-          mma_bf16_ss(tmem + w * 256, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t ad = desc_kmajor(qb + (kk >> 2) * (kRows * 128) + (kk & 3) * 32);
+            const uint64_t bd = desc_kmajor(kb + (kk >> 2) * L::kBox + (kk & 3) * 32);
+            mma_bf16_ss(tmem + w * 256, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(s_full + w);
+          last_s = u;
+          if (n + 1 >= s1 || kr2_sub(a, n + 1).gp != cur_gp) mma_commit(q_empty);
         }
-        mma_commit(s_full + w);
-        last_s = u;
-        if (n + 1 >= s1 || kr2_sub(a, n + 1).gp != cur_gp) mma_commit(q_empty);
-        if (u >= 1) ok = issue_pv(u - 1);
+        for (long n = nb; n < ne && ok; ++n) ok = issue_pv(n - s0);
       }
-      if (ok && s1 > s0) ok = issue_pv(s1 - 1 - s0);
       if (*abort_flag) {
         if (last_s >= 0) drain(s_full + (last_s & 1), (last_s >> 1) & 1);
         if (last_o >= 0) drain(o_full + (last_o & 1), (last_o >> 1) & 1);
