@@ -40,6 +40,8 @@ using namespace tc;
 
 constexpr int kRows = 128;  // query rows per CTA = UMMA M = TMEM lanes
 constexpr float kLog2e = 1.4426950408889634f;
+// Lazy rescale threshold of the output kernel: 8 in log2 units (a factor 2^8).
+constexpr float kRescaleNat = 8.f * 0.69314718055994531f;
 
 template <int D, int NK>
 struct KOLayout {
@@ -62,7 +64,7 @@ struct KOArgs {
   const float* hs;  // [G][b2][c1][nk]
   bf16* out;        // (G, N, d)
   int b1, b2, c1, nk, row_tiles, n_items;
-  float sc_log2;    // log2(e) / sqrt(d)
+  float sc;         // 1 / sqrt(d)
   int* status;
 };
 
@@ -98,10 +100,10 @@ __device__ __forceinline__ bool ko_decode(const KOArgs& a, int item, KOItem& it)
   return true;
 }
 
-// Persistent, warp-specialised L-update + output.  Warp 0 loads Q, Kt
-// (TMA) and the entropy bias (plain loads), warp 6 loads Y (TMA), warp 1
-// issues the tcgen05.mma instructions from one thread, warps 2-5 own the 128
-// rows (TMEM lanes) for the online softmax and the epilogue.  Kt and Y have
+// Persistent, warp-specialised L-update + output.  Warp 0 loads Q, Kt, Y
+// (TMA) and the entropy bias (plain loads), warp 1 issues the tcgen05.mma
+// instructions from one thread, warps 2-5 own the 128 rows (TMEM lanes) for
+// the online softmax and the epilogue.  Kt and Y have
 // separate two-slot rings: a Kt slot is recycled as soon as its S tile is
 // computed, a Y slot once its P Y product is, so each load is issued about
 // two tiles before it is needed.  mbarriers hand tiles between roles:
@@ -113,7 +115,7 @@ __device__ __forceinline__ bool ko_decode(const KOArgs& a, int item, KOItem& it)
 //   o_empty                 epilogue has read O (next item may overwrite it)
 // All counters run over the tiles T of every item this CTA processes.
 template <int D, int NK>
-__global__ void __launch_bounds__(224, 2)
+__global__ void __launch_bounds__(192, 2)
     ko_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kt,
               const __grid_constant__ CUtensorMap tm_y, KOArgs a) {
   using L = KOLayout<D, NK>;
@@ -176,82 +178,114 @@ __global__ void __launch_bounds__(224, 2)
   const uint32_t tmem_o = tmem;  // columns [0, D)
   auto tmem_s = [&](int sb) { return tmem + D + sb * NK; };
 
+  auto first_item = [&](int item, KOItem& it) {
+    for (; item < a.n_items; item += gridDim.x)
+      if (ko_decode<NK>(a, item, it)) return item;
+    return a.n_items;
+  };
   if (warp == 0) {
-    // ------------------------ producer: Q, Kt, bias ------------------------
+    // ------------------- producer: Q, Kt + bias, Y (event-driven) -------------------
+    // Two cursors walk the tiles: Kt (with the bias, and Q at an item's first
+    // tile) and Y; each load is issued as soon as its slot is free.  Lane 0
+    // probes the barriers and issues TMA; all lanes copy the bias.
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_kt);
+      tma_prefetch_desc(&tm_y);
     }
-    int n = 0, last_q = -1;
-    long T = 0;
-    bool ok = true;
-    for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
-      KOItem it;
-      if (!ko_decode<NK>(a, item, it)) continue;
-      if (n >= 1) ok = mbar_wait(q_empty, (n - 1) & 1, abort_flag, a.status);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(q_full, L::kQBytes);
+    KOItem kit, yit;
+    int k_item = first_item(blockIdx.x, kit), y_item = first_item(blockIdx.x, yit);
+    int k_j = 0, k_n = 0, y_j = 0;
+    long Tk = 0, Ty = 0;
+    bool ok = true, waited = false;
+    unsigned long long idle_since = global_ns();
+    while ((k_item < a.n_items || y_item < a.n_items) && ok) {
+      bool progressed = false;
+      if (k_item < a.n_items) {
+        const int st = (int)(Tk & 1);
+        int ready = 0;
+        if (lane == 0)
+          ready = (k_j > 0 || k_n == 0 || mbar_test(q_empty, (k_n - 1) & 1)) &&
+                  (Tk < 2 || (mbar_test(kt_empty + st, ((Tk >> 1) - 1) & 1) &&
+                              mbar_test(bias_empty + st, ((Tk >> 1) - 1) & 1)));
+        if (__shfl_sync(0xffffffffu, ready, 0)) {
+          if (lane == 0 && k_j == 0) {
+            mbar_arrive_expect_tx(q_full, L::kQBytes);
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(sQ + c * kRows * 128, &tm_q, q_full, c * 64, it.i, it.g * a.b1 + it.row0);
-      }
-      if (n == 0) pdl_wait();  // Kt, Hs come from the previous kernel
-      last_q = n;
-      for (int j = 0; j < it.nt; ++j, ++T) {
-        const int st = (int)(T & 1);
-        if (T >= 2) {
-          ok = mbar_wait(kt_empty + st, ((T >> 1) - 1) & 1, abort_flag, a.status);
-          if (ok) ok = mbar_wait(bias_empty + st, ((T >> 1) - 1) & 1, abort_flag, a.status);
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_3d(sQ + c * kRows * 128, &tm_q, q_full, c * 64, kit.i,
+                          kit.g * a.b1 + kit.row0);
+          }
+          if (!waited) {  // Kt, Y and the bias come from the previous kernel
+            pdl_wait();
+            waited = true;
+          }
+          const int y = static_cast<int>(kit.key_row0 + (long)k_j * NK);
+          if (lane == 0) {
+            mbar_arrive_expect_tx(kt_full + st, L::kTileBytes);
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_2d(sKt(st) + c * NK * 128, &tm_kt, kt_full + st, c * 64, y);
+          }
+          // the tile's entropy bias, copied asynchronously (columns past nk
+          // are left stale; the softmax masks them)
+          float* bias = sBias + st * NK;
+          for (int e = lane; e < NK; e += 32) {
+            const int col = k_j * NK + e;
+            if (col < a.nk) cp_async_4(bias + e, a.hs + kit.key_row0 + col);
+          }
+          cp_async_arrive_noinc(bias_full + st);
+          ++Tk;
+          if (++k_j == kit.nt) {
+            k_j = 0;
+            ++k_n;
+            k_item = first_item(k_item + gridDim.x, kit);
+          }
+          progressed = true;
         }
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
+      }
+      if (y_item < a.n_items && Ty < Tk) {
+        const int st = (int)(Ty & 1);
+        int ready = 0;
+        if (lane == 0) ready = Ty < 2 || mbar_test(y_empty + st, ((Ty >> 1) - 1) & 1);
+        if (__shfl_sync(0xffffffffu, ready, 0)) {
+          if (lane == 0) {
+            mbar_arrive_expect_tx(y_full + st, L::kTileBytes);
+            const int y = static_cast<int>(yit.key_row0 + (long)y_j * NK);
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_2d(sY(st) + c * NK * 128, &tm_y, y_full + st, c * 64, y);
+          }
+          ++Ty;
+          if (++y_j == yit.nt) {
+            y_j = 0;
+            y_item = first_item(y_item + gridDim.x, yit);
+          }
+          progressed = true;
+        }
+      }
+      if (progressed) {
+        idle_since = global_ns();
+      } else {
+        __nanosleep(32);
+        int bad = 0;
         if (lane == 0) {
-          mbar_arrive_expect_tx(kt_full + st, L::kTileBytes);
-          const int y = static_cast<int>(it.key_row0 + (long)j * NK);
-#pragma unroll
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_2d(sKt(st) + c * NK * 128, &tm_kt, kt_full + st, c * 64, y);
+          if (*abort_flag) {
+            bad = 1;
+          } else if (global_ns() - idle_since > kWaitLimitNs) {
+            *abort_flag = 1;
+            atomicExch(a.status, 1);
+            bad = 1;
+          }
         }
-        float* bias = sBias + st * NK;
-        for (int e = lane; e < NK; e += 32) {
-          const int col = j * NK + e;
-          bias[e] = col < a.nk ? __ldg(a.hs + it.key_row0 + col) * kLog2e : 0.f;
-        }
-        mbar_arrive(bias_full + st);
+        ok = !__shfl_sync(0xffffffffu, bad, 0);
       }
-      ++n;
     }
     if (lane == 0 && *abort_flag) {  // drain the loads this warp issued (bounded)
-      if (last_q >= 0) drain(q_full, last_q & 1);
-      for (long t = (T >= 2 ? T - 2 : 0); t < T; ++t) drain(kt_full + (t & 1), (t >> 1) & 1);
+      if (k_n >= 1 || k_j > 0) drain(q_full, (k_j > 0 ? k_n : k_n - 1) & 1);
+      for (long t = (Tk >= 2 ? Tk - 2 : 0); t < Tk; ++t) drain(kt_full + (t & 1), (t >> 1) & 1);
+      for (long t = (Ty >= 2 ? Ty - 2 : 0); t < Ty; ++t) drain(y_full + (t & 1), (t >> 1) & 1);
     }
-  } else if (warp == 6) {
-    // ---------------------------- producer: Y -----------------------------
-    if (lane == 0) {
-      tma_prefetch_desc(&tm_y);
-      pdl_wait();  // Y comes from the previous kernel
-      long T = 0;
-      bool ok = true;
-      for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
-        KOItem it;
-        if (!ko_decode<NK>(a, item, it)) continue;
-        for (int j = 0; j < it.nt; ++j, ++T) {
-          const int st = (int)(T & 1);
-          if (T >= 2) ok = mbar_wait(y_empty + st, ((T >> 1) - 1) & 1, abort_flag, a.status);
-          if (!ok) break;
-          mbar_arrive_expect_tx(y_full + st, L::kTileBytes);
-          const int y = static_cast<int>(it.key_row0 + (long)j * NK);
-#pragma unroll
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_2d(sY(st) + c * NK * 128, &tm_y, y_full + st, c * 64, y);
-        }
-      }
-      if (*abort_flag)
-        for (long t = (T >= 2 ? T - 2 : 0); t < T; ++t) drain(y_full + (t & 1), (t >> 1) & 1);
-    }
-    __syncwarp();
   } else if (warp == 1) {
     // -------------------------------- MMA ---------------------------------
     if (lane == 0) {
@@ -266,11 +300,6 @@ __global__ void __launch_bounds__(224, 2)
                      dy1 = desc_mnmajor(smem_u32(sY(1)), NK * 128);
       // Event-driven issue over two cursors (next S tile, next P Y tile):
       // whichever has its inputs ready goes out first.
-      auto first_item = [&](int item, KOItem& it) {
-        for (; item < a.n_items; item += gridDim.x)
-          if (ko_decode<NK>(a, item, it)) return item;
-        return a.n_items;
-      };
       KOItem sit, pit;
       int s_item = first_item(blockIdx.x, sit), p_item = first_item(blockIdx.x, pit);
       int s_j = 0, s_n = 0, p_j = 0, p_n = 0;
@@ -369,18 +398,19 @@ __global__ void __launch_bounds__(224, 2)
         tmem_wait_ld();
         const float* bias = sBias + sb * NK;
         const int valid = a.nk - j * NK;
-        // logits in log2 units; 4 partial maxima / sums break the serial chains
+        // logits sc q.Kt + Hs (natural units); 4 partial maxima / sums break
+        // the serial chains
         float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         if (valid >= NK) {
 #pragma unroll
           for (int c = 0; c < NK; ++c) {
-            sv[c] = fmaf(sv[c], a.sc_log2, bias[c]);
+            sv[c] = fmaf(sv[c], a.sc, bias[c]);
             mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
           }
         } else {
 #pragma unroll
           for (int c = 0; c < NK; ++c) {
-            sv[c] = c < valid ? fmaf(sv[c], a.sc_log2, bias[c]) : -INFINITY;
+            sv[c] = c < valid ? fmaf(sv[c], a.sc, bias[c]) : -INFINITY;
             mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
           }
         }
@@ -390,15 +420,16 @@ __global__ void __launch_bounds__(224, 2)
         const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
         float alpha = 1.f;
         bool resc = false;
-        if (mt > m_run + 8.f) {  // first tile, or the max grew by more than 2^8
-          alpha = ex2(m_run - mt);
+        if (mt > m_run + kRescaleNat) {  // first tile, or the max grew by more than 2^8
+          alpha = ex2((m_run - mt) * kLog2e);
           resc = j > 0;
           m_run = mt;
         }
+        const float neg_m2 = -m_run * kLog2e;
         float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int c = 0; c < NK; ++c) {
-          sv[c] = ex2(sv[c] - m_run);
+          sv[c] = ex2(fmaf(sv[c], kLog2e, neg_m2));
           ls[c & 3] += sv[c];
         }
         l_run = l_run * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
@@ -1296,11 +1327,11 @@ cudaError_t launch_ko(const bf16* q, const bf16* kt, const bf16* y, const float*
   const long items = (long)pb.G * pb.b2 * pb.c1 * a.row_tiles;
   if (items >= (1L << 31)) return cudaErrorInvalidValue;
   a.n_items = (int)items;
-  a.sc_log2 = kLog2e * pb.sc;
+  a.sc = pb.sc;
   a.status = status;
   const int grid = (int)std::min<long>(items, 2L * num_sms());
   return timed_launch("tc_l_output", stream, launches, [&] {
-    return launch_pdl(ko_kernel<D, NK>, dim3(grid), dim3(224), L::kAlloc, stream, tq, tk, tyv, a);
+    return launch_pdl(ko_kernel<D, NK>, dim3(grid), dim3(192), L::kAlloc, stream, tq, tk, tyv, a);
   });
 }
 

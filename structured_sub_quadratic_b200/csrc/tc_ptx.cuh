@@ -145,6 +145,22 @@ __device__ __forceinline__ void bulk_wait() {
   asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// 4-byte asynchronous copy global -> shared (cp.async); completion is
+// signalled through cp_async_arrive_noinc on an mbarrier whose expected
+// count includes this thread.
+__device__ __forceinline__ void cp_async_4(void* dst_smem, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst_smem)),
+               "l"(src)
+               : "memory");
+}
+
+// One arrival on `bar` once all of this thread's earlier cp.async copies
+// have completed (the expected count is not raised).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
 // Make generic-proxy writes to shared memory visible to the async proxy
 // (tcgen05.mma operand reads, TMA).
 __device__ __forceinline__ void fence_proxy_async_smem() {
