@@ -173,6 +173,14 @@ MONARCH_API int monarch_attn_timing_enable(int enable);
 MONARCH_API int monarch_attn_timing_read(int max_kernels, char* names, int name_len,
                                          double* ms_total, long* launches);
 
+/* Self-test of the device-timeout path (not part of the method): launches
+ * one CTA on `stream` that waits on a barrier nothing arrives on; after
+ * limit_ns nanoseconds (at most 10 s) the wait gives up, records the timeout
+ * in the device status word and the kernel returns normally, leaving the
+ * context usable.  A following monarch_attn_check() returns
+ * MONARCH_ERR_DEVICE_TIMEOUT.  Returns MONARCH_OK once launched. */
+MONARCH_API int monarch_attn_selftest_timeout(unsigned long long limit_ns, cudaStream_t stream);
+
 /* Library version, (major << 16) | minor. */
 MONARCH_API int monarch_attn_version(void);
 

@@ -41,6 +41,7 @@ SIGNATURES = {
     "monarch_attn_set_path": (_I, [_I]),
     "monarch_attn_last_launches": (_I, []),
     "monarch_attn_version": (_I, []),
+    "monarch_attn_selftest_timeout": (_I, [ctypes.c_ulonglong, _P]),
     "monarch_attn_timing_enable": (_I, [_I]),
     "monarch_attn_timing_read": (_I, [_I, ctypes.c_char_p, _I,
                                       ctypes.POINTER(ctypes.c_double),
@@ -198,3 +199,8 @@ def timing_read(max_kernels: int = 32):
         raw = names.raw[s * name_len:(s + 1) * name_len]
         out[raw.split(b"\0", 1)[0].decode()] = (ms[s], cnt[s])
     return out
+
+
+def selftest_timeout(limit_ns: int, stream=None):
+    """Launch the bounded-wait self-test (see the header); check() then reports it."""
+    _check(load_library().monarch_attn_selftest_timeout(limit_ns, _stream_ptr(stream)))

@@ -322,6 +322,21 @@ int monarch_attn_set_path(int path) {
 
 int monarch_attn_last_launches(void) { return t_launches; }
 
+int monarch_attn_selftest_timeout(unsigned long long limit_ns, cudaStream_t stream) {
+  if (limit_ns > 10ull * 1000000000ull) return MONARCH_ERR_INVALID_ARG;
+  int dev;
+  int st = current_device(&dev);
+  if (st != MONARCH_OK) return st;
+  int* status;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if ((st = ensure_status(dev)) != MONARCH_OK) return st;
+    status = g_status[dev];
+  }
+  cudaError_t e = monarch::tc_selftest_timeout(status, limit_ns, stream);
+  return e == cudaSuccess ? MONARCH_OK : record_cuda(e);
+}
+
 int monarch_attn_version(void) { return (0 << 16) | 1; }
 
 }  // extern "C"

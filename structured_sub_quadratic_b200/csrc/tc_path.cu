@@ -1182,6 +1182,23 @@ __global__ void __launch_bounds__(320, 1)
 }
 
 // ---------------------------------------------------------------------------
+// Self-test of the bounded-wait path: one CTA waits on an mbarrier that
+// nothing ever arrives on, gives up after limit_ns, records the timeout in
+// the status word and returns normally.
+// ---------------------------------------------------------------------------
+__global__ void selftest_timeout_kernel(int* status, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_word;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_word = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  (void)mbar_wait(&bar, 0, &abort_word, status, limit_ns);
+}
+
+// ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -1518,6 +1535,11 @@ SimtWorkspace carve(const Problem& pb, char* base, size_t* total) {
 }
 
 }  // namespace
+
+cudaError_t tc_selftest_timeout(int* status, unsigned long long limit_ns, cudaStream_t stream) {
+  selftest_timeout_kernel<<<1, 32, 0, stream>>>(status, limit_ns);
+  return cudaGetLastError();
+}
 
 bool tc_supports(const Problem& pb) {
   if (pb.d != 64 && pb.d != 128) return false;

@@ -19,4 +19,8 @@ size_t tc_workspace_bytes(const Problem& pb);
 cudaError_t tc_forward(const bf16* q, const bf16* k, const bf16* v, bf16* out, const Problem& pb,
                        char* ws, int* status, cudaStream_t stream, int* launches);
 
+// Launches one CTA whose bounded wait must expire after limit_ns and set the
+// status word (exercises the timeout path without any fault).
+cudaError_t tc_selftest_timeout(int* status, unsigned long long limit_ns, cudaStream_t stream);
+
 }  // namespace monarch

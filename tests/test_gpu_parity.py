@@ -124,3 +124,18 @@ def test_simt_and_default_paths_agree(cuda_lib):
     finally:
         cuda_lib.set_path(prev)
     assert_parity(O_auto, O_simt, v, wl.dtype)
+
+
+def test_bounded_wait_timeout_is_reported_and_context_survives(cuda_lib):
+    """A device wait that nothing satisfies gives up after its limit, sets the
+    status word and returns; the host reads MONARCH_ERR_DEVICE_TIMEOUT once,
+    and the context keeps running forward passes."""
+    cuda_lib.check()  # clean slate
+    cuda_lib.selftest_timeout(20_000_000)  # 20 ms
+    with pytest.raises(cuda_lib.MonarchError) as exc:
+        cuda_lib.check()
+    assert exc.value.status == cuda_lib.MONARCH_ERR_DEVICE_TIMEOUT
+    cuda_lib.check()  # the flag was cleared by the read
+    q, k, v = iid_qkv(1, 2, 64, 64, torch.bfloat16, seed=9)
+    O = gpu_forward(cuda_lib, q, k, v, 8, 8, 1)
+    assert_parity(O, oracle_forward(q, k, v, 8, 8, 1), v, torch.bfloat16)
