@@ -109,9 +109,12 @@ __device__ __forceinline__ bool ko_decode(const KOArgs& a, int item, KOItem& it)
 // two tiles before it is needed.  mbarriers hand tiles between roles:
 //   q_full/q_empty          Q tile (one per item)
 //   kt_full/kt_empty        Kt ring          y_full/y_empty   Y ring
-//   bias_full/bias_empty    bias ring        s_full/s_empty   S buffers in TMEM
-//   p_full                  P of tile T written to shared memory
-//   pv_done                 O += P Y of tile T complete (P buffer free, O stable)
+//   bias_full/bias_empty    bias ring        s_full[2]        S tile in TMEM buffer
+//   p_full[2]               P of the tile written over its S (TMEM, bf16 pairs)
+//   pv_done[2]              O += P Y of the tile complete (its S/P buffer free,
+//                           O stable)
+// P never leaves the tensor memory: the softmax overwrites its S tile with P
+// and the P Y product reads A from TMEM, so S and P are double-buffered.
 //   o_empty                 epilogue has read O (next item may overwrite it)
 // All counters run over the tiles T of every item this CTA processes.
 template <int D, int NK>
@@ -137,11 +140,10 @@ __global__ void __launch_bounds__(192, 2)
   uint64_t* y_full = bars + 6;       // [2]
   uint64_t* y_empty = bars + 8;      // [2]
   uint64_t* s_full = bars + 10;      // [2]
-  uint64_t* s_empty = bars + 12;     // [2]
+  uint64_t* pv_done = bars + 12;     // [2]
   uint64_t* bias_full = bars + 14;   // [2]
   uint64_t* bias_empty = bars + 16;  // [2]
-  uint64_t* p_full = bars + 18;
-  uint64_t* pv_done = bars + 19;
+  uint64_t* p_full = bars + 18;      // [2]
   uint64_t* o_empty = bars + 20;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 21);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 22);
@@ -157,12 +159,11 @@ __global__ void __launch_bounds__(192, 2)
       mbar_init(y_full + s, 1);
       mbar_init(y_empty + s, 1);
       mbar_init(s_full + s, 1);
-      mbar_init(s_empty + s, 128);
+      mbar_init(pv_done + s, 1);
+      mbar_init(p_full + s, 128);
       mbar_init(bias_full + s, 32);
       mbar_init(bias_empty + s, 128);
     }
-    mbar_init(p_full, 128);
-    mbar_init(pv_done, 1);
     mbar_init(o_empty, 128);
     *abort_flag = 0;
     fence_mbar_init();
@@ -294,7 +295,7 @@ __global__ void __launch_bounds__(192, 2)
       long last_s = -1, last_pv = -1;
       bool ok = true;
       // Base descriptors, built once; each MMA adds a compile-time offset.
-      const uint64_t dq = desc_kmajor(smem_u32(sQ)), dp = desc_kmajor(smem_u32(sP));
+      const uint64_t dq = desc_kmajor(smem_u32(sQ));
       const uint64_t dkt0 = desc_kmajor(smem_u32(sKt(0))), dkt1 = desc_kmajor(smem_u32(sKt(1)));
       const uint64_t dy0 = desc_mnmajor(smem_u32(sY(0)), NK * 128),
                      dy1 = desc_mnmajor(smem_u32(sY(1)), NK * 128);
@@ -310,7 +311,7 @@ __global__ void __launch_bounds__(192, 2)
         if (s_item < a.n_items) {
           const int st = (int)(Ts & 1);
           if ((s_j > 0 || mbar_test(q_full, s_n & 1)) && mbar_test(kt_full + st, (Ts >> 1) & 1) &&
-              (Ts < 2 || mbar_test(s_empty + st, ((Ts >> 1) - 1) & 1))) {
+              (Ts < 2 || mbar_test(pv_done + st, ((Ts >> 1) - 1) & 1))) {
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk)
@@ -333,16 +334,15 @@ __global__ void __launch_bounds__(192, 2)
         }
         if (Tp < Ts) {
           const int st = (int)(Tp & 1);
-          if (mbar_test(p_full, Tp & 1) && mbar_test(y_full + st, (Tp >> 1) & 1) &&
+          if (mbar_test(p_full + st, (Tp >> 1) & 1) && mbar_test(y_full + st, (Tp >> 1) & 1) &&
               (p_j > 0 || p_n == 0 || mbar_test(o_empty, (p_n - 1) & 1))) {
             tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < NK / 16; ++kk)
-              mma_bf16_ss(tmem_o, dp + (((kk >> 2) * (kRows * 128) + (kk & 3) * 32) >> 4),
-                          (st ? dy1 : dy0) + ((kk * 16 * 128) >> 4), idesc_o,
-                          (p_j > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < NK / 16; ++kk)  // A = P from TMEM: 8 columns per 16 keys
+              mma_bf16_ts(tmem_o, tmem_s(st) + kk * 8, (st ? dy1 : dy0) + ((kk * 16 * 128) >> 4),
+                          idesc_o, (p_j > 0 || kk > 0) ? 1u : 0u);
             mma_commit(y_empty + st);
-            mma_commit(pv_done);
+            mma_commit(pv_done + st);
             last_pv = Tp;
             ++Tp;
             if (++p_j == pit.nt) {
@@ -365,7 +365,7 @@ __global__ void __launch_bounds__(192, 2)
       }
       if (*abort_flag) {  // drain this thread's MMAs (bounded)
         if (last_s >= 0) drain(s_full + (last_s & 1), (last_s >> 1) & 1);
-        if (last_pv >= 0) drain(pv_done, last_pv & 1);
+        if (last_pv >= 0) drain(pv_done + (last_pv & 1), (last_pv >> 1) & 1);
       }
     }
     __syncwarp();
@@ -414,8 +414,6 @@ __global__ void __launch_bounds__(192, 2)
             mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
           }
         }
-        tc_fence_before();
-        mbar_arrive(s_empty + sb);
         mbar_arrive(bias_empty + sb);
         const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
         float alpha = 1.f;
@@ -433,11 +431,11 @@ __global__ void __launch_bounds__(192, 2)
           ls[c & 3] += sv[c];
         }
         l_run = l_run * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
-        // P buffer free and O stable once the previous tile's P Y is done
-        if (T >= 1) ok = mbar_wait(pv_done, (T - 1) & 1, abort_flag, a.status);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
         if (__any_sync(0xffffffffu, resc)) {
+          // O is stable once the previous tile's P Y is done
+          ok = mbar_wait(pv_done + ((T - 1) & 1), ((T - 1) >> 1) & 1, abort_flag, a.status);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
           tc_fence_after();
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
@@ -450,24 +448,21 @@ __global__ void __launch_bounds__(192, 2)
           }
           tmem_wait_st();
         }
+        // P (bf16 pairs) over the first NK/2 columns of this tile's S buffer
 #pragma unroll
-        for (int u = 0; u < NK / 8; ++u) {
-          uint4 pk;
-          pk.x = pack_bf16x2(sv[8 * u + 0], sv[8 * u + 1]);
-          pk.y = pack_bf16x2(sv[8 * u + 2], sv[8 * u + 3]);
-          pk.z = pack_bf16x2(sv[8 * u + 4], sv[8 * u + 5]);
-          pk.w = pack_bf16x2(sv[8 * u + 6], sv[8 * u + 7]);
-          const int chunk = u >> 3, unit = u & 7;
-          *reinterpret_cast<uint4*>(sP + chunk * (kRows * 128) + row * 128 +
-                                    ((unit ^ (row & 7)) << 4)) = pk;
+        for (int c = 0; c < NK / 32; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(sv[c * 32 + 2 * e], sv[c * 32 + 2 * e + 1]);
+          tmem_st16(tmem_s(sb) + lane_off + c * 16, pk);
         }
-        fence_proxy_async_smem();
+        tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(p_full);
+        mbar_arrive(p_full + sb);
       }
       if (!ok) break;
       // ---- epilogue: O / l -> global rows ----
-      ok = mbar_wait(pv_done, (T - 1) & 1, abort_flag, a.status);
+      ok = mbar_wait(pv_done + ((T - 1) & 1), ((T - 1) >> 1) & 1, abort_flag, a.status);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
