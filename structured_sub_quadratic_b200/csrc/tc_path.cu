@@ -514,6 +514,313 @@ __global__ void __launch_bounds__(192, 2)
 }
 
 // ---------------------------------------------------------------------------
+// L-update + output when every row's keys fit one tile (nk = b1*c2 <= NK <=
+// 128): the softmax is exact in two passes over the S tile (max, then
+// exponentials), so there is no running max and no rescaling of O.  Each
+// ring has one slot; S of the next item goes out as soon as the previous
+// P Y product has consumed its P (which overwrites S in TMEM), so it
+// overlaps the previous item's epilogue.  Warp roles as in ko_kernel; items
+// are walked in order, so every barrier's phase is the item counter n.
+//   q_full/q_empty, kt_full/kt_empty, y_full/y_empty   operand slots
+//   bias_full/bias_empty   entropy bias      s_full   S ready
+//   p_full                 P written         pv_done  O = P Y complete
+//   o_empty                epilogue has read O
+// ---------------------------------------------------------------------------
+template <int D, int NK>
+struct KO1Layout {
+  static constexpr int kQBytes = D / 64 * kRows * 128;
+  static constexpr int kTileBytes = D / 64 * NK * 128;  // Kt or Y
+  static constexpr int kKtOff = kQBytes;
+  static constexpr int kYOff = kKtOff + kTileBytes;
+  static constexpr int kPOff = kYOff + kTileBytes;      // epilogue staging, 128 rows x 128 B
+  static constexpr int kBiasOff = kPOff + kRows * 128;
+  static constexpr int kBarOff = kBiasOff + NK * 4;
+  static constexpr int kBytes = kBarOff + 16 * 8;
+  static constexpr int kAlloc = kBytes > 100 * 1024 ? kBytes : 100 * 1024;  // <= 2 CTAs / SM
+  static constexpr uint32_t kTmemCols = 256;  // O: D columns, S: NK columns
+  static_assert(D % 64 == 0 && NK % 64 == 0 && NK <= 128 && D + NK <= 256, "tile sizes");
+  static_assert(2 * (kAlloc + 1024) <= 233472, "two CTAs per SM");
+};
+
+template <int D, int NK>
+__global__ void __launch_bounds__(192, 2)
+    ko1_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kt,
+               const __grid_constant__ CUtensorMap tm_y, KOArgs a) {
+  using L = KO1Layout<D, NK>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (smem_u32(smem) & 1023u) {
+    if (tid == 0) atomicExch(a.status, 2);
+    return;
+  }
+  pdl_launch_dependents();
+  uint8_t* sQ = smem;
+  uint8_t* sKt = smem + L::kKtOff;
+  uint8_t* sY = smem + L::kYOff;
+  uint8_t* sP = smem + L::kPOff;
+  float* sBias = reinterpret_cast<float*>(smem + L::kBiasOff);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* q_full = bars + 0;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* kt_full = bars + 2;
+  uint64_t* kt_empty = bars + 3;
+  uint64_t* y_full = bars + 4;
+  uint64_t* y_empty = bars + 5;
+  uint64_t* s_full = bars + 6;
+  uint64_t* p_full = bars + 7;
+  uint64_t* pv_done = bars + 8;
+  uint64_t* bias_full = bars + 9;
+  uint64_t* bias_empty = bars + 10;
+  uint64_t* o_empty = bars + 11;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 13);
+
+  if (tid == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    mbar_init(kt_full, 1);
+    mbar_init(kt_empty, 1);
+    mbar_init(y_full, 1);
+    mbar_init(y_empty, 1);
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 128);
+    mbar_init(pv_done, 1);
+    mbar_init(bias_full, 32);
+    mbar_init(bias_empty, 128);
+    mbar_init(o_empty, 128);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem_o = tmem;      // columns [0, D)
+  const uint32_t tmem_s = tmem + D;  // columns [D, D + NK); P (bf16 pairs) over its first NK/2
+
+  if (warp == 0) {
+    // ------------------------- producer: Q, Kt + bias, Y -------------------------
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_kt);
+      tma_prefetch_desc(&tm_y);
+    }
+    bool ok = true;
+    long n = 0;
+    for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
+      KOItem it;
+      if (!ko_decode<NK>(a, item, it)) continue;
+      if (lane == 0) {
+        if (n >= 1) ok = mbar_wait(q_empty, (n - 1) & 1, abort_flag, a.status);
+        if (ok) {
+          mbar_arrive_expect_tx(q_full, L::kQBytes);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(sQ + c * kRows * 128, &tm_q, q_full, c * 64, it.i, it.g * a.b1 + it.row0);
+        }
+      }
+      if (n == 0) pdl_wait();  // Kt, Y and the bias come from the previous kernel
+      if (lane == 0) {
+        if (ok && n >= 1) ok = mbar_wait(kt_empty, (n - 1) & 1, abort_flag, a.status);
+        if (ok) {
+          mbar_arrive_expect_tx(kt_full, L::kTileBytes);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_2d(sKt + c * NK * 128, &tm_kt, kt_full, c * 64, (int)it.key_row0);
+        }
+        if (ok && n >= 1) ok = mbar_wait(bias_empty, (n - 1) & 1, abort_flag, a.status);
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      // the entropy bias of the item's nk keys (columns past nk stay stale; masked)
+      for (int e = lane; e < a.nk; e += 32) cp_async_4(sBias + e, a.hs + it.key_row0 + e);
+      cp_async_arrive_noinc(bias_full);
+      if (lane == 0) {
+        if (n >= 1) ok = mbar_wait(y_empty, (n - 1) & 1, abort_flag, a.status);
+        if (ok) {
+          mbar_arrive_expect_tx(y_full, L::kTileBytes);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_2d(sY + c * NK * 128, &tm_y, y_full, c * 64, (int)it.key_row0);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      ++n;
+    }
+    if (lane == 0 && *abort_flag && n >= 1) {  // drain this warp's loads (bounded)
+      drain(q_full, (n - 1) & 1);
+      drain(kt_full, (n - 1) & 1);
+      drain(y_full, (n - 1) & 1);
+    }
+  } else if (warp == 1) {
+    // -------------------------------- MMA ---------------------------------
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_bf16(kRows, NK, false);
+      const uint32_t idesc_o = idesc_bf16(kRows, D, true);
+      const uint64_t dq = desc_kmajor(smem_u32(sQ));
+      const uint64_t dkt = desc_kmajor(smem_u32(sKt));
+      const uint64_t dy = desc_mnmajor(smem_u32(sY), NK * 128);
+      const int kk_pv = (a.nk + 15) / 16;  // P Y over the valid keys only
+      bool ok = true;
+      long n = 0, issued_s = 0, issued_pv = 0;
+      for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
+        KOItem it;
+        if (!ko_decode<NK>(a, item, it)) continue;
+        ok = mbar_wait(q_full, n & 1, abort_flag, a.status) &&
+             mbar_wait(kt_full, n & 1, abort_flag, a.status) &&
+             (n == 0 || mbar_wait(pv_done, (n - 1) & 1, abort_flag, a.status));
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_bf16_ss(tmem_s, dq + (((kk >> 2) * (kRows * 128) + (kk & 3) * 32) >> 4),
+                      dkt + (((kk >> 2) * (NK * 128) + (kk & 3) * 32) >> 4), idesc_s,
+                      kk > 0 ? 1u : 0u);
+        mma_commit(s_full);
+        mma_commit(kt_empty);
+        mma_commit(q_empty);
+        issued_s = n + 1;
+        ok = mbar_wait(p_full, n & 1, abort_flag, a.status) &&
+             mbar_wait(y_full, n & 1, abort_flag, a.status) &&
+             (n == 0 || mbar_wait(o_empty, (n - 1) & 1, abort_flag, a.status));
+        if (!ok) break;
+        tc_fence_after();
+        for (int kk = 0; kk < kk_pv; ++kk)  // A = P from TMEM: 8 columns per 16 keys
+          mma_bf16_ts(tmem_o, tmem_s + kk * 8, dy + ((kk * 16 * 128) >> 4), idesc_o,
+                      kk > 0 ? 1u : 0u);
+        mma_commit(pv_done);
+        mma_commit(y_empty);
+        issued_pv = n + 1;
+        ++n;
+      }
+      if (*abort_flag) {  // drain this thread's MMAs (bounded)
+        if (issued_s > 0) drain(s_full, (issued_s - 1) & 1);
+        if (issued_pv > 0) drain(pv_done, (issued_pv - 1) & 1);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------- softmax + epilogue --------------------------
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;  // TMEM lane == tile row
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const int nch = (a.nk + 31) / 32;  // 32-column chunks holding valid keys
+    const float sc = a.sc;
+    bool ok = true;
+    long n = 0;
+    for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
+      KOItem it;
+      if (!ko_decode<NK>(a, item, it)) continue;
+      ok = mbar_wait(s_full, n & 1, abort_flag, a.status);
+      if (ok) ok = mbar_wait(bias_full, n & 1, abort_flag, a.status);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      // pass 1: row max of sc q.Kt + Hs over the valid keys
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int c = 0; c < NK / 32; ++c) {
+        if (c < nch) {
+          float t[32];
+          tmem_ld32(tmem_s + lane_off + c * 32, t);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int col = c * 32 + e;
+            const float v = col < a.nk ? fmaf(t[e], sc, sBias[col]) : -INFINITY;
+            mx[e & 3] = fmaxf(mx[e & 3], v);
+          }
+        }
+      }
+      const float m = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      const float neg_m2 = -m * kLog2e;
+      // pass 2: P = exp(S - m) as bf16 pairs over the first columns of S (a
+      // chunk's P lands in columns already read), and the row sum
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int c = 0; c < NK / 32; ++c) {
+        if (c < nch) {
+          float t[32];
+          tmem_ld32(tmem_s + lane_off + c * 32, t);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int col = c * 32 + e;
+            const float v = col < a.nk ? fmaf(t[e], sc, sBias[col]) : -INFINITY;
+            t[e] = ex2(fmaf(v, kLog2e, neg_m2));
+            ls[e & 3] += t[e];
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(t[2 * e], t[2 * e + 1]);
+          tmem_st16(tmem_s + lane_off + c * 16, pk);
+        }
+      }
+      mbar_arrive(bias_empty);
+      const float l_row = (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_full);
+      // ---- epilogue: O / l -> global rows ----
+      ok = mbar_wait(pv_done, n & 1, abort_flag, a.status);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const float inv = 1.f / l_row;
+      // Rows go out through shared memory: each thread stages its row, then 8
+      // threads write one row's 128-byte half, so global stores are whole
+      // sectors.
+      const int srow = tid - 64;  // 0..127 over the four softmax warps
+#pragma unroll 1
+      for (int h = 0; h < D / 64; ++h) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          float t[32];
+          tmem_ld32(tmem_o + lane_off + h * 64 + c * 32, t);
+          tmem_wait_ld();
+          if (h == D / 64 - 1 && c == 1) {  // O fully read: the next P Y may overwrite it
+            tc_fence_before();
+            mbar_arrive(o_empty);
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            uint4 pk;
+            pk.x = pack_bf16x2(t[8 * u + 0] * inv, t[8 * u + 1] * inv);
+            pk.y = pack_bf16x2(t[8 * u + 2] * inv, t[8 * u + 3] * inv);
+            pk.z = pack_bf16x2(t[8 * u + 4] * inv, t[8 * u + 5] * inv);
+            pk.w = pack_bf16x2(t[8 * u + 6] * inv, t[8 * u + 7] * inv);
+            const int unit = c * 4 + u;
+            *reinterpret_cast<uint4*>(sP + row * 128 + ((unit ^ (row & 7)) << 4)) = pk;
+          }
+        }
+        named_barrier(1, 128);
+#pragma unroll
+        for (int pass = 0; pass < kRows / 16; ++pass) {
+          const int r = pass * 16 + (srow >> 3), unit = srow & 7;
+          if (r < it.nrows) {
+            const uint4 v4 = *reinterpret_cast<const uint4*>(sP + r * 128 + ((unit ^ (r & 7)) << 4));
+            bf16* dst = a.out + (((long)it.g * a.b1 + it.row0 + r) * a.b2 + it.i) * D + h * 64;
+            *reinterpret_cast<uint4*>(dst + unit * 8) = v4;
+          }
+        }
+        named_barrier(1, 128);
+      }
+      ++n;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Step-one aggregated queries under the uniform initial L (bf16):
 // Qt0[g][p][i][:] = mean_{l in p} q_(l,i).  One block per (g, p, i); 16-byte
 // column chunks x row lanes, reduced through shared memory.
@@ -813,29 +1120,48 @@ __global__ void __launch_bounds__(128)
 
 // ---------------------------------------------------------------------------
 // Persistent R-update (step one) for column-group tiles NQ <= 64.  One CTA
-// per SM walks a contiguous range of items (g, p, k), each split into c2
-// sub-items (one per column group q).  Warp 0 loads (Qt0 once per (g, p),
-// K_q / V_q through a three-slot ring), warp 1 issues the MMAs, and two
-// warpgroups (warps 2-5 and 6-9) take alternate sub-items: softmax (R is
-// normalised before the MMA), then the Kt / Y rows through double-buffered
-// TMA bulk stores.  Each warpgroup
-// owns one 2d-column TMEM slot in which S is later overwritten by
-// [Kt | Y], so sub-item n+1's S and softmax overlap sub-item n's stores.
-// Barriers (sub-item counter n over the CTA's items):
+// per SM walks a contiguous range of sub-items (g, p, k, q): one item (g, p, k)
+// is split into c2 sub-items, one per column group q.  Warp 0 loads (Qt0, and
+// K_q / V_q through a ring of slots), warp 1 issues the MMAs, and two
+// warpgroups (warps 2-5 and 6-9) take alternate tiles: softmax (R is
+// normalised before the MMA), then the Kt / Y rows through TMA bulk stores.
+// Each warpgroup owns one 2d-column TMEM slot in which S is later
+// overwritten by [Kt | Y], so tile t+1's S and softmax overlap tile t's
+// stores.
+//
+// Paired tiles (PAIR, b2 <= 64): the b2 positions of one sub-item fill only
+// half of the 128 TMEM lanes, so a tile carries two consecutive sub-items A
+// and B.  Rows 0-63 of the A operand hold sub-item A's aggregated queries and
+// rows 64-127 sub-item B's; the key operand stacks A's NQ keys over B's, so S
+// is 128 x 2NQ and rows 0-63 use its first NQ columns, rows 64-127 its last
+// NQ.  P is block diagonal ([R_A 0; 0 R_B]), so one product with the stacked
+// [K | V] of both sub-items gives [Kt | Y] of A in rows 0-63 and of B in rows
+// 64-127.  Each warp then stores its own 32 rows with a 4-D TMA box (rows
+// clipped at b2), staging in its own rows of the P buffer, which is dead once
+// the product is done.
+//
+// Barriers (tile counter t over the CTA's tiles):
 //   q_full / q_empty       Qt0 tile        kv_full / kv_empty   K/V ring
 //   s_full[w] / o_full[w]  S / [Kt | Y] of warpgroup w's slot complete
 //   p_full[w]              P written       tmem_free[w]         slot read out
 // ---------------------------------------------------------------------------
-template <int D, int NQ>
+template <int D, int NQ, bool PAIR>
 struct KR2Layout {
-  static constexpr int kBox = NQ * 128;
-  static constexpr int kKVBytes = 2 * (D / 64) * kBox;  // K_q then V_q
-  static constexpr int kKVSlots = 3;
+  static constexpr int kHalves = PAIR ? 2 : 1;             // sub-items per tile
+  static constexpr int kKeys = kHalves * NQ;               // N of S, K-extent of [K | V]
+  static constexpr int kBox = NQ * 128;                    // one TMA box: NQ keys x 64 columns
+  static constexpr int kBlk = kKeys * 128;                 // one 64-column block of K or V
+  static constexpr int kKVBytes = 2 * (D / 64) * kBlk;     // K blocks, then V blocks
+  static constexpr int kKVSlots = PAIR ? 2 : 3;
+  // P (K-major, 64-key chunks of 128 rows); paired tiles keep two chunks so
+  // that each warp finds two 4 KB staging buffers in its own rows.
+  static constexpr int kPBytes = (PAIR ? 2 : (kKeys + 63) / 64) * kRows * 128;
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = D / 64 * kRows * 128;
-  static constexpr int kPOff = kKVOff + kKVSlots * kKVBytes;     // [2] x 16 KB
-  static constexpr int kStageOff = kPOff + 2 * kRows * 128;      // [2 wg][2] x 16 KB
-  static constexpr int kBarOff = kStageOff + 4 * kRows * 128;
+  static constexpr int kPOff = kKVOff + kKVSlots * kKVBytes;       // [2 wg]
+  static constexpr int kStageOff = kPOff + 2 * kPBytes;            // [2 wg][2] x 16 KB
+  static constexpr int kStageBytes = PAIR ? 0 : 4 * kRows * 128;
+  static constexpr int kBarOff = kStageOff + kStageBytes;
   static constexpr int kBytes = kBarOff + 32 * 8;
   static_assert(NQ % 16 == 0 && NQ <= 64, "group tile");
   static_assert(kBytes <= 227 * 1024, "shared memory");
@@ -865,12 +1191,33 @@ __device__ __forceinline__ KR2Sub kr2_sub(const KR2Args& a, long n_sub) {
   return s;
 }
 
-template <int D, int NQ>
+// Next sub-item in (gp, k, q) order.
+__device__ __forceinline__ void kr2_next(const KR2Args& a, KR2Sub& s) {
+  if (++s.q == a.c2) {
+    s.q = 0;
+    if (++s.k == a.b1) {
+      s.k = 0;
+      ++s.gp;
+      s.p = s.gp % a.c1;
+      s.g = s.gp / a.c1;
+    }
+  }
+}
+
+// Which aggregated-query rows a tile needs: (gp of its first sub-item, gp of
+// its last); a change of key means a new Qt0 load.
+__device__ __forceinline__ long kr2_qkey(int gp_a, int gp_b) {
+  return ((long)gp_a << 32) | (unsigned)gp_b;
+}
+
+template <int D, int NQ, bool PAIR>
 __global__ void __launch_bounds__(320, 1)
     kr2_kernel(const __grid_constant__ CUtensorMap tm_qt, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kt,
                const __grid_constant__ CUtensorMap tm_y, KR2Args a) {
-  using L = KR2Layout<D, NQ>;
+  using L = KR2Layout<D, NQ, PAIR>;
+  constexpr int H = L::kHalves;
+  constexpr int kSlots = L::kKVSlots;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (smem_u32(smem) & 1023u) {
@@ -878,19 +1225,22 @@ __global__ void __launch_bounds__(320, 1)
     return;
   }
   pdl_launch_dependents();
-  // this CTA's sub-items [s0, s1)
+  // this CTA's tiles: H consecutive sub-items each, sub-items [s0, s1)
   const long n_sub = (long)a.n_items * a.c2;
-  const long s0 = n_sub * blockIdx.x / gridDim.x, s1 = n_sub * (blockIdx.x + 1) / gridDim.x;
+  const long n_units = (n_sub + H - 1) / H;
+  const long s0 = n_units * blockIdx.x / gridDim.x * H;
+  const long s1 = min(n_units * (blockIdx.x + 1) / gridDim.x * H, n_sub);
+  const long ntiles = (s1 - s0 + H - 1) / H;
 
   uint8_t* sQ = smem + L::kQOff;
   auto sKV = [&](int sl) { return smem + L::kKVOff + sl * L::kKVBytes; };
-  auto sP = [&](int w) { return smem + L::kPOff + w * kRows * 128; };
+  auto sP = [&](int w) { return smem + L::kPOff + w * L::kPBytes; };
   auto sStage = [&](int w, int b) { return smem + L::kStageOff + (w * 2 + b) * kRows * 128; };
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
-  uint64_t* kv_full = bars + 2;    // [3]
-  uint64_t* kv_empty = bars + 5;   // [3]
+  uint64_t* kv_full = bars + 2;    // [kSlots]
+  uint64_t* kv_empty = bars + 5;   // [kSlots]
   uint64_t* s_full = bars + 8;     // [2]
   uint64_t* o_full = bars + 10;    // [2]
   uint64_t* p_full = bars + 12;    // [2]
@@ -901,7 +1251,7 @@ __global__ void __launch_bounds__(320, 1)
   if (tid == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
-    for (int i = 0; i < 3; ++i) {
+    for (int i = 0; i < kSlots; ++i) {
       mbar_init(kv_full + i, 1);
       mbar_init(kv_empty + i, 1);
     }
@@ -929,55 +1279,77 @@ __global__ void __launch_bounds__(320, 1)
       tma_prefetch_desc(&tm_qt);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      int cur_gp = -1, nq_loads = 0;
+      long cur_key = -1;
+      int nq_loads = 0;
       bool ok = true;
       long last_kv = -1;
-      for (long n = s0; n < s1 && ok; ++n) {
-        const KR2Sub sb = kr2_sub(a, n);
-        const long u = n - s0;
-        const int sl = (int)(u % 3);
-        if (u >= 3) ok = mbar_wait(kv_empty + sl, ((u / 3) - 1) & 1, abort_flag, a.status);
+      KR2Sub cur = kr2_sub(a, s0);
+      for (long t = 0; t < ntiles && ok; ++t) {
+        const int sl = (int)(t % kSlots);
+        const int nh = (int)min((long)H, s1 - (s0 + t * H));
+        if (t >= kSlots) ok = mbar_wait(kv_empty + sl, ((t / kSlots) - 1) & 1, abort_flag, a.status);
         if (!ok) break;
-        const int krow = (sb.g * a.b1 + sb.k) * a.b2 + group_start(a.b2, a.c2, sb.q);
-        mbar_arrive_expect_tx(kv_full + sl, L::kKVBytes);
+        mbar_arrive_expect_tx(kv_full + sl, H * 2 * (D / 64) * L::kBox);
+        const int gp_a = cur.gp;
+        int gp_b = gp_a, krow = 0;
+        for (int h = 0; h < H; ++h) {
+          // An absent second half (odd count, last tile) repeats the first:
+          // finite keys that its zero rows of P weigh by zero.
+          if (h < nh) {
+            krow = (cur.g * a.b1 + cur.k) * a.b2 + group_start(a.b2, a.c2, cur.q);
+            gp_b = cur.gp;
+            kr2_next(a, cur);
+          }
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          tma_load_2d(sKV(sl) + c * L::kBox, &tm_k, kv_full + sl, c * 64, krow);
-          tma_load_2d(sKV(sl) + (D / 64 + c) * L::kBox, &tm_v, kv_full + sl, c * 64, krow);
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_2d(sKV(sl) + c * L::kBlk + h * L::kBox, &tm_k, kv_full + sl, c * 64, krow);
+            tma_load_2d(sKV(sl) + (D / 64 + c) * L::kBlk + h * L::kBox, &tm_v, kv_full + sl, c * 64,
+                        krow);
+          }
         }
-        last_kv = u;
-        if (sb.gp != cur_gp) {
+        last_kv = t;
+        const long key = kr2_qkey(gp_a, gp_b);
+        if (key != cur_key) {
           if (nq_loads == 0) pdl_wait();  // Qt0 comes from the previous kernel
-          if (nq_loads >= 1) ok = mbar_wait(q_empty, (nq_loads - 1) & 1, abort_flag, a.status);
+          if (ok && nq_loads >= 1) ok = mbar_wait(q_empty, (nq_loads - 1) & 1, abort_flag, a.status);
           if (!ok) break;
           mbar_arrive_expect_tx(q_full, D / 64 * kRows * 128);
+          if (PAIR) {
 #pragma unroll
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_2d(sQ + c * kRows * 128, &tm_qt, q_full, c * 64, sb.gp * a.b2);
-          cur_gp = sb.gp;
+            for (int c = 0; c < D / 64; ++c) {
+              tma_load_2d(sQ + c * kRows * 128, &tm_qt, q_full, c * 64, gp_a * a.b2);
+              tma_load_2d(sQ + c * kRows * 128 + 64 * 128, &tm_qt, q_full, c * 64, gp_b * a.b2);
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_2d(sQ + c * kRows * 128, &tm_qt, q_full, c * 64, gp_a * a.b2);
+          }
+          cur_key = key;
           ++nq_loads;
         }
       }
       if (*abort_flag) {
         if (nq_loads >= 1) drain(q_full, (nq_loads - 1) & 1);
-        for (long u = (last_kv >= 2 ? last_kv - 2 : 0); u <= last_kv; ++u) drain(kv_full + u % 3, (u / 3) & 1);
+        for (long t = (last_kv >= kSlots - 1 ? last_kv - (kSlots - 1) : 0); t <= last_kv; ++t)
+          drain(kv_full + t % kSlots, (t / kSlots) & 1);
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     // -------------------------------- MMA ---------------------------------
     if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16(kRows, NQ, false);
+      const uint32_t idesc_s = idesc_bf16(kRows, L::kKeys, false);
       const uint32_t idesc_o = idesc_bf16(kRows, 2 * D, true);
       // Base descriptors, built once; each MMA adds a compile-time offset
       // (in 16-byte units) to the start-address field.  The issuing thread
       // shares its scheduler with softmax warps, so its path is kept short.
       const uint64_t dq = desc_kmajor(smem_u32(sQ));
       const uint64_t dk0 = desc_kmajor(smem_u32(sKV(0))), dk1 = desc_kmajor(smem_u32(sKV(1))),
-                     dk2 = desc_kmajor(smem_u32(sKV(2)));
-      const uint64_t dkv0 = desc_mnmajor(smem_u32(sKV(0)), L::kBox),
-                     dkv1 = desc_mnmajor(smem_u32(sKV(1)), L::kBox),
-                     dkv2 = desc_mnmajor(smem_u32(sKV(2)), L::kBox);
+                     dk2 = desc_kmajor(smem_u32(sKV(kSlots > 2 ? 2 : 1)));
+      const uint64_t dkv0 = desc_mnmajor(smem_u32(sKV(0)), L::kBlk),
+                     dkv1 = desc_mnmajor(smem_u32(sKV(1)), L::kBlk),
+                     dkv2 = desc_mnmajor(smem_u32(sKV(kSlots > 2 ? 2 : 1)), L::kBlk);
       const uint64_t dp0 = desc_kmajor(smem_u32(sP(0))), dp1 = desc_kmajor(smem_u32(sP(1)));
       auto pick3 = [](int i, uint64_t x0, uint64_t x1, uint64_t x2) {
         return i == 0 ? x0 : (i == 1 ? x1 : x2);
@@ -985,64 +1357,67 @@ __global__ void __launch_bounds__(320, 1)
       int nq_loads = 0;
       bool ok = true;
       long last_s = -1, last_o = -1;
-      // Event-driven issue: S of the next sub-item and [Kt | Y] of the oldest
+      // Event-driven issue: S of the next tile and [Kt | Y] of the oldest
       // pending one go out as soon as their inputs are ready, in whichever
       // order that happens, so one warpgroup's epilogue never holds back the
-      // other warpgroup's product.  The sub-item (q, k, gp) is walked
-      // incrementally.
-      const long nloc = s1 - s0;
-      long us = 0, up = 0;
+      // other warpgroup's product.  The sub-items are walked incrementally.
+      long ts = 0, tp = 0;
       KR2Sub cur = kr2_sub(a, s0);
-      int cur_gp = -1;
+      long cur_key = -1;
+      // key of tile ts (and the walker moved to tile ts + 1)
+      auto tile_key = [&](long t) {
+        const int nh = (int)min((long)H, s1 - (s0 + t * H));
+        const int gp_a = cur.gp;
+        int gp_b = gp_a;
+        for (int h = 0; h < nh; ++h) {
+          gp_b = cur.gp;
+          kr2_next(a, cur);
+        }
+        return kr2_qkey(gp_a, gp_b);
+      };
+      long key = ntiles > 0 ? tile_key(0) : -1;
       unsigned long long idle_since = global_ns();
-      while (up < nloc && ok) {
+      while (tp < ntiles && ok) {
         bool progressed = false;
-        if (us < nloc) {
-          const int w = (int)(us & 1), sl = (int)(us % 3);
+        if (ts < ntiles) {
+          const int w = (int)(ts & 1), sl = (int)(ts % kSlots);
           bool ready = true;
-          if (cur.gp != cur_gp) {
+          if (key != cur_key) {
             ready = mbar_test(q_full, nq_loads & 1);
             if (ready) {
-              cur_gp = cur.gp;
+              cur_key = key;
               ++nq_loads;
             }
           }
-          if (ready && mbar_test(kv_full + sl, (us / 3) & 1) &&
-              (us < 2 || mbar_test(tmem_free + w, ((us >> 1) - 1) & 1))) {
+          if (ready && mbar_test(kv_full + sl, (ts / kSlots) & 1) &&
+              (ts < 2 || mbar_test(tmem_free + w, ((ts >> 1) - 1) & 1))) {
             tc_fence_after();
             const uint64_t dks = pick3(sl, dk0, dk1, dk2);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk)
               mma_bf16_ss(tmem + w * 256, dq + (((kk >> 2) * (kRows * 128) + (kk & 3) * 32) >> 4),
-                          dks + (((kk >> 2) * L::kBox + (kk & 3) * 32) >> 4), idesc_s,
+                          dks + (((kk >> 2) * L::kBlk + (kk & 3) * 32) >> 4), idesc_s,
                           kk > 0 ? 1u : 0u);
             mma_commit(s_full + w);
-            last_s = us;
-            // advance (q, k, gp); release Qt0 after its last S
-            if (++cur.q == a.c2) {
-              cur.q = 0;
-              if (++cur.k == a.b1) {
-                cur.k = 0;
-                ++cur.gp;
-              }
-            }
-            ++us;
-            if (us >= nloc || cur.gp != cur_gp) mma_commit(q_empty);
+            last_s = ts;
+            ++ts;
+            key = ts < ntiles ? tile_key(ts) : -1;
+            if (key != cur_key) mma_commit(q_empty);  // Qt0 rows no longer needed
             progressed = true;
           }
         }
-        if (up < us && mbar_test(p_full + (int)(up & 1), (up >> 1) & 1)) {
-          const int w = (int)(up & 1), sl = (int)(up % 3);
+        if (tp < ts && mbar_test(p_full + (int)(tp & 1), (tp >> 1) & 1)) {
+          const int w = (int)(tp & 1), sl = (int)(tp % kSlots);
           tc_fence_after();
           const uint64_t dps = w == 0 ? dp0 : dp1, dkvs = pick3(sl, dkv0, dkv1, dkv2);
 #pragma unroll
-          for (int kk = 0; kk < NQ / 16; ++kk)
-            mma_bf16_ss(tmem + w * 256, dps + (((kk & 3) * 32) >> 4),
+          for (int kk = 0; kk < L::kKeys / 16; ++kk)
+            mma_bf16_ss(tmem + w * 256, dps + (((kk >> 2) * (kRows * 128) + (kk & 3) * 32) >> 4),
                         dkvs + ((kk * 16 * 128) >> 4), idesc_o, kk > 0 ? 1u : 0u);
           mma_commit(o_full + w);
           mma_commit(kv_empty + sl);
-          last_o = up;
-          ++up;
+          last_o = tp;
+          ++tp;
           progressed = true;
         }
         if (progressed) {
@@ -1065,28 +1440,31 @@ __global__ void __launch_bounds__(320, 1)
     // -------------------- softmax + epilogue (two warpgroups) --------------------
     const int w = (warp - 2) >> 2;            // warpgroup 0: warps 2-5, 1: warps 6-9
     const int quad = warp & 3;
-    const int r = quad * 32 + lane;           // TMEM lane == row == position i
+    const int r = quad * 32 + lane;           // TMEM lane == tile row
+    const int h = PAIR ? (quad >> 1) : 0;     // which sub-item of the tile (warp-uniform)
+    const int i = PAIR ? (r & 63) : r;        // position of this row
     const int wtid = tid - 64 - w * 128;      // 0..127 inside the warpgroup
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t tslot = tmem + w * 256;
     const bool leader = wtid == 0;
-    int nst = 0;  // stores issued by this warpgroup; buffer nst & 1
+    int nst = 0;  // unpaired tiles: stores issued by this warpgroup; buffer nst & 1
     bool ok = true;
-    for (long n = s0 + w; n < s1 && ok; n += 2) {
-      const KR2Sub sb = kr2_sub(a, n);
-      const long u = n - s0;
+    for (long t = w; t < ntiles && ok; t += 2) {
+      const long n = s0 + t * H + h;
+      const bool have = n < s1;  // warp-uniform
+      const KR2Sub sb = kr2_sub(a, have ? n : s0 + t * H);
       const int nq = group_start(a.b2, a.c2, sb.q + 1) - group_start(a.b2, a.c2, sb.q);
-      ok = mbar_wait(s_full + w, (u >> 1) & 1, abort_flag, a.status);
+      ok = mbar_wait(s_full + w, (t >> 1) & 1, abort_flag, a.status);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
       float sv[NQ];
 #pragma unroll
       for (int c = 0; c < NQ / 16; ++c) {
-        float t[16];
-        tmem_ld16(tslot + lane_off + c * 16, t);
+        float tt[16];
+        tmem_ld16(tslot + lane_off + h * NQ + c * 16, tt);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) sv[c * 16 + e] = t[e];
+        for (int e = 0; e < 16; ++e) sv[c * 16 + e] = tt[e];
       }
       tmem_wait_ld();
       float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -1096,19 +1474,29 @@ __global__ void __launch_bounds__(320, 1)
         mx[j & 3] = fmaxf(mx[j & 3], sv[j]);
       }
       const float m2 = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-      float zs[4] = {0.f, 0.f, 0.f, 0.f}, ts[4] = {0.f, 0.f, 0.f, 0.f};
+      float zs[4] = {0.f, 0.f, 0.f, 0.f}, ts2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int j = 0; j < NQ; ++j) {
         const float d2 = sv[j] - m2;
         sv[j] = ex2(d2);
         zs[j & 3] += sv[j];
-        ts[j & 3] += j < nq ? sv[j] * d2 : 0.f;
+        ts2[j & 3] += j < nq ? sv[j] * d2 : 0.f;
       }
       const float z = (zs[0] + zs[1]) + (zs[2] + zs[3]);
-      const float t2 = (ts[0] + ts[1]) + (ts[2] + ts[3]);
-      const float inv = 1.f / z;
+      const float t2 = (ts2[0] + ts2[1]) + (ts2[2] + ts2[3]);
+      const float inv = have ? 1.f / z : 0.f;  // an absent sub-item contributes P = 0
       uint8_t* pbuf = sP(w);
-      // P holds R itself (normalised), so [Kt | Y] comes out of the MMA final
+      if (PAIR) {  // this warp's rows of P were the previous tile's staging: stores must have read them
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+      }
+      // P holds R itself (normalised), so [Kt | Y] comes out of the MMA final.
+      // Paired tiles: this row's R in its own half of the columns, zeros in
+      // the other half.
+      auto p_unit = [&](int u) {  // 16-byte unit u (keys 8u .. 8u+7) of this row of P
+        return reinterpret_cast<uint4*>(pbuf + (u >> 3) * (kRows * 128) + r * 128 +
+                                        (((u & 7) ^ (r & 7)) << 4));
+      };
 #pragma unroll
       for (int uu = 0; uu < NQ / 8; ++uu) {
         uint4 pk;
@@ -1116,57 +1504,102 @@ __global__ void __launch_bounds__(320, 1)
         pk.y = pack_bf16x2(sv[8 * uu + 2] * inv, sv[8 * uu + 3] * inv);
         pk.z = pack_bf16x2(sv[8 * uu + 4] * inv, sv[8 * uu + 5] * inv);
         pk.w = pack_bf16x2(sv[8 * uu + 6] * inv, sv[8 * uu + 7] * inv);
-        *reinterpret_cast<uint4*>(pbuf + r * 128 + ((uu ^ (r & 7)) << 4)) = pk;
+        *p_unit(uu + h * (NQ / 8)) = pk;
+        if (PAIR) *p_unit(uu + (1 - h) * (NQ / 8)) = make_uint4(0u, 0u, 0u, 0u);
       }
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(p_full + w);
-      ok = mbar_wait(o_full + w, (u >> 1) & 1, abort_flag, a.status);
+      ok = mbar_wait(o_full + w, (t >> 1) & 1, abort_flag, a.status);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      // The b2 rows of this (g, p, k, q) are positions i of the position-major
-      // Kt/Y layout: one 3-D TMA box {64 columns, 1, b2 rows}.  Each 64-column
-      // block is staged (swizzled) in one of two buffers and handed to a TMA
-      // bulk store; a buffer is refilled once its previous store has read it.
       const int nblk = (a.write_y ? 2 : 1) * (D / 64);
       const int ycoord = (sb.p * a.b1 + sb.k) * a.c2 + sb.q;
-      const bool row_ok = r < a.b2;
-      const long orow_w = ((((long)sb.g * a.b2 + r) * a.c1 + sb.p) * a.b1 + sb.k) * a.c2 + sb.q;
-#pragma unroll 1
-      for (int cb = 0; cb < nblk; ++cb, ++nst) {
-        uint8_t* buf = sStage(w, nst & 1);
-        float ta[32], tb[32];
-        tmem_ld32(tslot + lane_off + cb * 64, ta);
-        tmem_ld32(tslot + lane_off + cb * 64 + 32, tb);
-        if (leader) bulk_wait_read<1>();  // the store that last used buf has read it
-        named_barrier(1 + w, 128);
-        tmem_wait_ld();
-        if (cb == nblk - 1) {  // slot fully read out: the MMA may reuse it
+      const bool row_ok = have && i < a.b2;
+      const long orow_w = ((((long)sb.g * a.b2 + i) * a.c1 + sb.p) * a.b1 + sb.k) * a.c2 + sb.q;
+      if constexpr (PAIR) {
+        // Each warp stores its own 32 rows (positions i0 .. i0 + 31 of its
+        // sub-item) through a 4-D box clipped at b2, staging in its own rows
+        // of the P buffer (two 4 KB buffers, one per 64-key chunk).
+        const int i0 = (quad & 1) * 32;
+        const bool store = have && i0 < a.b2;  // warp-uniform
+        if (!store) {
           tc_fence_before();
           mbar_arrive(tmem_free + w);
-        }
+        } else {
+#pragma unroll 1
+          for (int cb = 0; cb < nblk; ++cb) {
+            uint8_t* buf = pbuf + (cb & 1) * (kRows * 128) + quad * 32 * 128;
+            float ta[32], tb[32];
+            tmem_ld32(tslot + lane_off + cb * 64, ta);
+            tmem_ld32(tslot + lane_off + cb * 64 + 32, tb);
+            if (cb >= 2 && lane == 0) bulk_wait_read<1>();  // store of block cb-2 has read buf
+            __syncwarp();
+            tmem_wait_ld();
+            if (cb == nblk - 1) {  // slot fully read out: the MMA may reuse it
+              tc_fence_before();
+              mbar_arrive(tmem_free + w);
+            }
 #pragma unroll
-        for (int uu = 0; uu < 8; ++uu) {
-          const float* v = uu < 4 ? ta + 8 * uu : tb + 8 * (uu - 4);
-          uint4 pk;
-          pk.x = pack_bf16x2(v[0], v[1]);
-          pk.y = pack_bf16x2(v[2], v[3]);
-          pk.z = pack_bf16x2(v[4], v[5]);
-          pk.w = pack_bf16x2(v[6], v[7]);
-          *reinterpret_cast<uint4*>(buf + r * 128 + ((uu ^ (r & 7)) << 4)) = pk;
+            for (int uu = 0; uu < 8; ++uu) {
+              const float* v = uu < 4 ? ta + 8 * uu : tb + 8 * (uu - 4);
+              uint4 pk;
+              pk.x = pack_bf16x2(v[0], v[1]);
+              pk.y = pack_bf16x2(v[2], v[3]);
+              pk.z = pack_bf16x2(v[4], v[5]);
+              pk.w = pack_bf16x2(v[6], v[7]);
+              *reinterpret_cast<uint4*>(buf + lane * 128 + ((uu ^ (lane & 7)) << 4)) = pk;
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_4d(cb < D / 64 ? &tm_kt : &tm_y, buf, (cb % (D / 64)) * 64, ycoord, i0,
+                           sb.g);
+              bulk_commit();
+            }
+          }
         }
-        fence_proxy_async_smem();
-        named_barrier(1 + w, 128);
-        if (leader) {
-          tma_store_3d(cb < D / 64 ? &tm_kt : &tm_y, buf, (cb % (D / 64)) * 64, ycoord,
-                       sb.g * a.b2);
-          bulk_commit();
+      } else {
+        // The b2 rows of this (g, p, k, q) are positions i of the position-major
+        // Kt/Y layout: one 3-D TMA box {64 columns, 1, b2 rows}.  Each 64-column
+        // block is staged (swizzled) in one of two buffers and handed to a TMA
+        // bulk store; a buffer is refilled once its previous store has read it.
+#pragma unroll 1
+        for (int cb = 0; cb < nblk; ++cb, ++nst) {
+          uint8_t* buf = sStage(w, nst & 1);
+          float ta[32], tb[32];
+          tmem_ld32(tslot + lane_off + cb * 64, ta);
+          tmem_ld32(tslot + lane_off + cb * 64 + 32, tb);
+          if (leader) bulk_wait_read<1>();  // the store that last used buf has read it
+          named_barrier(1 + w, 128);
+          tmem_wait_ld();
+          if (cb == nblk - 1) {  // slot fully read out: the MMA may reuse it
+            tc_fence_before();
+            mbar_arrive(tmem_free + w);
+          }
+#pragma unroll
+          for (int uu = 0; uu < 8; ++uu) {
+            const float* v = uu < 4 ? ta + 8 * uu : tb + 8 * (uu - 4);
+            uint4 pk;
+            pk.x = pack_bf16x2(v[0], v[1]);
+            pk.y = pack_bf16x2(v[2], v[3]);
+            pk.z = pack_bf16x2(v[4], v[5]);
+            pk.w = pack_bf16x2(v[6], v[7]);
+            *reinterpret_cast<uint4*>(buf + r * 128 + ((uu ^ (r & 7)) << 4)) = pk;
+          }
+          fence_proxy_async_smem();
+          named_barrier(1 + w, 128);
+          if (leader) {
+            tma_store_3d(cb < D / 64 ? &tm_kt : &tm_y, buf, (cb % (D / 64)) * 64, ycoord,
+                         sb.g * a.b2);
+            bulk_commit();
+          }
         }
       }
-      if (row_ok) a.hs[orow_w] = logf(z) - t2 * 0.69314718055994531f * inv;
+      if (row_ok) a.hs[orow_w] = logf(z) - t2 * 0.69314718055994531f / z;
     }
-    if (leader) bulk_wait<0>();  // stores done reading shared memory before exit
+    if (PAIR ? lane == 0 : leader) bulk_wait<0>();  // stores done reading shared memory before exit
   }
   tc_fence_before();
   __syncthreads();
@@ -1217,8 +1650,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 struct MapKey {
   const void* base;
   int rank;
-  cuuint64_t dims[3], str[2];
-  cuuint32_t box[3];
+  cuuint64_t dims[4], str[3];
+  cuuint32_t box[4];
   bool operator==(const MapKey& o) const {
     if (base != o.base || rank != o.rank) return false;
     for (int i = 0; i < rank; ++i)
@@ -1235,6 +1668,7 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims
   static MapKey keys[64];
   static CUtensorMap maps[64];
   static int used = 0, next = 0;
+  if (rank < 1 || rank > 4) return false;
   MapKey key = {};
   key.base = base;
   key.rank = rank;
@@ -1347,6 +1781,67 @@ cudaError_t launch_ko(const bf16* q, const bf16* kt, const bf16* y, const float*
   });
 }
 
+template <int D, int NK>
+cudaError_t launch_ko1(const bf16* q, const bf16* kt, const bf16* y, const float* hs, bf16* out,
+                       const Problem& pb, int* status, cudaStream_t stream, int* launches) {
+  using L = KO1Layout<D, NK>;
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(ko1_kernel<D, NK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    L::kAlloc);
+    if (attr_err == cudaSuccess)
+      attr_err = cudaFuncSetAttribute(ko1_kernel<D, NK>,
+                                      cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  const int nk = pb.b1 * pb.c2;
+  if (nk > NK) return cudaErrorInvalidValue;
+  const long key_rows = (long)pb.G * pb.b2 * pb.c1 * nk;
+  CUtensorMap tq, tk, tyv;
+  {
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)pb.b2, (cuuint64_t)pb.G * pb.b1};
+    const cuuint64_t str[2] = {(cuuint64_t)D * 2, (cuuint64_t)pb.b2 * D * 2};
+    const cuuint32_t box[3] = {64, 1, kRows};
+    if (!make_map(&tq, q, 3, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)key_rows};
+    const cuuint64_t str[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64, NK};
+    if (!make_map(&tk, kt, 2, dims, str, box)) return cudaErrorInvalidValue;
+    if (!make_map(&tyv, y, 2, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  const int gmax = (pb.b1 + pb.c1 - 1) / pb.c1;
+  KOArgs a;
+  a.hs = hs;
+  a.out = out;
+  a.b1 = pb.b1;
+  a.b2 = pb.b2;
+  a.c1 = pb.c1;
+  a.nk = nk;
+  a.row_tiles = (gmax + kRows - 1) / kRows;
+  const long items = (long)pb.G * pb.b2 * pb.c1 * a.row_tiles;
+  if (items >= (1L << 31)) return cudaErrorInvalidValue;
+  a.n_items = (int)items;
+  a.sc = pb.sc;
+  a.status = status;
+  const int grid = (int)std::min<long>(items, 2L * num_sms());
+  return timed_launch("tc_l_output", stream, launches, [&] {
+    return launch_pdl(ko1_kernel<D, NK>, dim3(grid), dim3(192), L::kAlloc, stream, tq, tk, tyv, a);
+  });
+}
+
+// Output kernel by key count: one key tile per row when b1*c2 <= 64, else
+// the online-softmax kernel over 64-key tiles.
+template <int D>
+cudaError_t dispatch_ko(const bf16* q, const bf16* kt, const bf16* y, const float* hs, bf16* out,
+                        const Problem& pb, int* status, cudaStream_t stream, int* launches) {
+  const int nk = pb.b1 * pb.c2;
+  if (nk <= 64) return launch_ko1<D, 64>(q, kt, y, hs, out, pb, status, stream, launches);
+  return launch_ko<D, 64>(q, kt, y, hs, out, pb, status, stream, launches);
+}
+
 template <int D, int NQ>
 cudaError_t launch_kr(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, bf16* y, float* hs,
                       const Problem& pb, int* status, cudaStream_t stream, int* launches) {
@@ -1405,23 +1900,24 @@ cudaError_t launch_kr(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, b
   });
 }
 
-template <int D, int NQ>
+template <int D, int NQ, bool PAIR>
 cudaError_t launch_kr2(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, bf16* y,
                        float* hs, const Problem& pb, int* status, cudaStream_t stream,
                        int* launches) {
-  using L = KR2Layout<D, NQ>;
+  using L = KR2Layout<D, NQ, PAIR>;
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(kr2_kernel<D, NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    L::kBytes);
+    attr_err = cudaFuncSetAttribute(kr2_kernel<D, NQ, PAIR>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
   });
   if (attr_err != cudaSuccess) return attr_err;
   CUtensorMap tq, tk, tv, tkt, tyy;
   {
+    // paired tiles load each sub-item's b2 (<= 64) query rows as a 64-row box
     const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)pb.G * pb.c1 * pb.b2};
     const cuuint64_t str[1] = {(cuuint64_t)D * 2};
-    const cuuint32_t box[2] = {64, kRows};
+    const cuuint32_t box[2] = {64, PAIR ? 64u : (cuuint32_t)kRows};
     if (!make_map(&tq, qt0, 2, dims, str, box)) return cudaErrorInvalidValue;
   }
   {
@@ -1431,11 +1927,19 @@ cudaError_t launch_kr2(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, 
     if (!make_map(&tk, k, 2, dims, str, box)) return cudaErrorInvalidValue;
     if (!make_map(&tv, v, 2, dims, str, box)) return cudaErrorInvalidValue;
   }
-  {
-    // Kt / Y [G][b2 i][c1 p][b1 k][c2 q][d] viewed as (d, c1*b1*c2, G*b2)
-    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)pb.c1 * pb.b1 * pb.c2,
-                                (cuuint64_t)pb.G * pb.b2};
-    const cuuint64_t str[2] = {(cuuint64_t)D * 2, (cuuint64_t)pb.c1 * pb.b1 * pb.c2 * D * 2};
+  const cuuint64_t ny = (cuuint64_t)pb.c1 * pb.b1 * pb.c2;
+  if (PAIR) {
+    // Kt / Y [G][b2 i][c1 p][b1 k][c2 q][d] viewed as (d, c1*b1*c2, b2, G);
+    // one warp's box is {64 columns, 1, 32 positions, 1}, clipped at b2
+    const cuuint64_t dims[4] = {(cuuint64_t)D, ny, (cuuint64_t)pb.b2, (cuuint64_t)pb.G};
+    const cuuint64_t str[3] = {(cuuint64_t)D * 2, ny * D * 2, ny * pb.b2 * D * 2};
+    const cuuint32_t box[4] = {64, 1, 32, 1};
+    if (!make_map(&tkt, kt, 4, dims, str, box)) return cudaErrorInvalidValue;
+    if (!make_map(&tyy, y, 4, dims, str, box)) return cudaErrorInvalidValue;
+  } else {
+    // Kt / Y viewed as (d, c1*b1*c2, G*b2); one box holds the b2 positions
+    const cuuint64_t dims[3] = {(cuuint64_t)D, ny, (cuuint64_t)pb.G * pb.b2};
+    const cuuint64_t str[2] = {(cuuint64_t)D * 2, ny * D * 2};
     const cuuint32_t box[3] = {64, 1, (cuuint32_t)pb.b2};
     if (!make_map(&tkt, kt, 3, dims, str, box)) return cudaErrorInvalidValue;
     if (!make_map(&tyy, y, 3, dims, str, box)) return cudaErrorInvalidValue;
@@ -1454,10 +1958,11 @@ cudaError_t launch_kr2(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, 
   a.write_y = pb.T == 1 ? 1 : 0;
   a.sc_log2 = kLog2e * pb.sc;
   a.status = status;
-  const int grid = (int)std::min<long>(items * pb.c2, num_sms());
+  const long units = (items * pb.c2 + L::kHalves - 1) / L::kHalves;
+  const int grid = (int)std::min<long>(units, num_sms());
   return timed_launch("tc_r_update", stream, launches, [&] {
-    return launch_pdl(kr2_kernel<D, NQ>, dim3(grid), dim3(320), L::kBytes, stream, tq, tk, tv,
-                      tkt, tyy, a);
+    return launch_pdl(kr2_kernel<D, NQ, PAIR>, dim3(grid), dim3(320), L::kBytes, stream, tq, tk,
+                      tv, tkt, tyy, a);
   });
 }
 
@@ -1467,13 +1972,24 @@ inline int kr_group_tile(const Problem& pb) {
   return ((pb.b2 + pb.c2 - 1) / pb.c2 + 15) / 16 * 16;
 }
 
+// Step one: aggregated queries under the uniform L, then the R-update (the
+// persistent kernel for column groups of <= 64 keys, the per-item kernel for
+// wider ones).
 template <int D>
-cudaError_t dispatch_kr(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, bf16* y,
-                        float* hs, const Problem& pb, int* status, cudaStream_t stream,
-                        int* launches) {
+cudaError_t launch_r_step1(const bf16* q, const bf16* k, const bf16* v, bf16* qt0, bf16* kt,
+                           bf16* y, float* hs, const Problem& pb, int* status,
+                           cudaStream_t stream, int* launches) {
+  cudaError_t e = timed_launch("tc_init_qt", stream, launches, [&] {
+    init_qt_bf16_kernel<D><<<(unsigned)((long)pb.G * pb.c1 * pb.b2), 512, 0, stream>>>(
+        q, qt0, pb.b1, pb.b2, pb.c1);
+  });
+  if (e != cudaSuccess) return e;
   switch (kr_group_tile(pb)) {
-#define MONARCH_KR2_CASE(NQ) \
-  case NQ: return launch_kr2<D, NQ>(qt0, k, v, kt, y, hs, pb, status, stream, launches);
+#define MONARCH_KR2_CASE(NQ)                                                               \
+  case NQ:                                                                                 \
+    return pb.b2 <= 64                                                                     \
+               ? launch_kr2<D, NQ, true>(qt0, k, v, kt, y, hs, pb, status, stream, launches) \
+               : launch_kr2<D, NQ, false>(qt0, k, v, kt, y, hs, pb, status, stream, launches);
 #define MONARCH_KR_CASE(NQ) \
   case NQ: return launch_kr<D, NQ>(qt0, k, v, kt, y, hs, pb, status, stream, launches);
     MONARCH_KR2_CASE(16)
@@ -1488,19 +2004,6 @@ cudaError_t dispatch_kr(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt,
 #undef MONARCH_KR2_CASE
     default: return cudaErrorInvalidValue;
   }
-}
-
-// Step one: aggregated queries under the uniform L, then the R-update.
-template <int D>
-cudaError_t launch_r_step1(const bf16* q, const bf16* k, const bf16* v, bf16* qt0, bf16* kt,
-                           bf16* y, float* hs, const Problem& pb, int* status,
-                           cudaStream_t stream, int* launches) {
-  cudaError_t e = timed_launch("tc_init_qt", stream, launches, [&] {
-    init_qt_bf16_kernel<D><<<(unsigned)((long)pb.G * pb.c1 * pb.b2), 512, 0, stream>>>(
-        q, qt0, pb.b1, pb.b2, pb.c1);
-  });
-  if (e != cudaSuccess) return e;
-  return dispatch_kr<D>(qt0, k, v, kt, y, hs, pb, status, stream, launches);
 }
 
 constexpr size_t kAlign = 256;
@@ -1572,8 +2075,8 @@ cudaError_t tc_forward(const bf16* q, const bf16* k, const bf16* v, bf16* out, c
     e = simt_r_update<bf16, bf16>(k, v, ws.qt, s1, kt, y, ws.hs, pb, t == pb.T, stream, launches);
     if (e != cudaSuccess) return e;
   }
-  if (pb.d == 128) return launch_ko<128, 64>(q, kt, y, ws.hs, out, pb, status, stream, launches);
-  return launch_ko<64, 64>(q, kt, y, ws.hs, out, pb, status, stream, launches);
+  if (pb.d == 128) return dispatch_ko<128>(q, kt, y, ws.hs, out, pb, status, stream, launches);
+  return dispatch_ko<64>(q, kt, y, ws.hs, out, pb, status, stream, launches);
 }
 
 }  // namespace monarch

@@ -71,6 +71,9 @@ EDGE = [
     (1, 1, 100, 3, 32, 2, 2, 1),     # long L rows
     (1, 2, 7, 7, 64, 0, 1, 3),       # T = 0 with uneven column groups
     (1, 1, 4, 70, 64, 1, 1, 3),      # long R rows in groups
+    (1, 2, 200, 8, 64, 1, 1, 1),     # more than 128 keys per L row: multi-tile output kernel
+    (1, 1, 70, 20, 128, 2, 2, 2),    # 140 keys per L row in row groups, two steps
+    (1, 1, 45, 64, 128, 1, 1, 1),    # paired R tiles with 64 positions, odd sub-item count
 ]
 
 
