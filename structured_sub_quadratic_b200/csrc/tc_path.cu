@@ -822,31 +822,38 @@ __global__ void __launch_bounds__(192, 2)
 
 // ---------------------------------------------------------------------------
 // Step-one aggregated queries under the uniform initial L (bf16):
-// Qt0[g][p][i][:] = mean_{l in p} q_(l,i).  One block per (g, p, i); 16-byte
-// column chunks x row lanes, reduced through shared memory.
+// Qt0[g][p][i][:] = mean_{l in p} q_(l,i).  One block per (g, p, i): 16-byte
+// column chunks x row lanes, every row load of a thread in flight at once;
+// the row lanes are summed in a fixed order (warp shuffles, then the 8 warps
+// through shared memory).  Launched with programmatic stream serialisation:
+// its blocks may be scheduled while the previous kernel of the stream
+// finishes, but they wait for it before reading q (which may be that
+// kernel's output) and only then let the next kernel launch, so every later
+// kernel of the call (which reads K and V early) runs after all earlier work.
 // ---------------------------------------------------------------------------
 template <int D>
-__global__ void __launch_bounds__(512)
+__global__ void __launch_bounds__(256)
     init_qt_bf16_kernel(const bf16* __restrict__ q, bf16* __restrict__ qt0, int b1, int b2,
                         int c1) {
-  constexpr int CH = D / 8;          // 16-byte chunks per row
-  constexpr int LANES = 512 / CH;    // rows summed in parallel
-  __shared__ float red[LANES][D + 1];
+  constexpr int CH = D / 8;        // 16-byte chunks per row
+  constexpr int RL = 256 / CH;     // row lanes
+  __shared__ float red[8][D];
   int bid = blockIdx.x;
   const int i = bid % b2;
   bid /= b2;
   const int p = bid % c1;
   const long g = bid / c1;
   const int l0 = group_start(b1, c1, p), l1 = group_start(b1, c1, p + 1);
+  pdl_wait();
   pdl_launch_dependents();
-  const int ch = threadIdx.x % CH, lane = threadIdx.x / CH;
+  const int ch = threadIdx.x % CH, rl = threadIdx.x / CH, lane = threadIdx.x & 31;
   float acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
   const uint4* base = reinterpret_cast<const uint4*>(q + (g * b1 * b2 + i) * D) + ch;
   const long row_stride = (long)b2 * D / 8;  // in uint4
-#pragma unroll 4
-  for (int l = l0 + lane; l < l1; l += LANES) {
+#pragma unroll 8
+  for (int l = l0 + rl; l < l1; l += RL) {
     const uint4 u = __ldg(base + l * row_stride);
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -856,12 +863,19 @@ __global__ void __launch_bounds__(512)
     }
   }
 #pragma unroll
-  for (int e = 0; e < 8; ++e) red[lane][ch * 8 + e] = acc[e];
+  for (int e = 0; e < 8; ++e) {
+#pragma unroll
+    for (int o = CH; o < 32; o <<= 1) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
+  }
+  if (lane < CH) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) red[threadIdx.x >> 5][ch * 8 + e] = acc[e];
+  }
   __syncthreads();
   if (threadIdx.x < D) {
     float sum = 0.f;
-#pragma unroll 8
-    for (int ln = 0; ln < LANES; ++ln) sum += red[ln][threadIdx.x];
+#pragma unroll
+    for (int w8 = 0; w8 < 8; ++w8) sum += red[w8][threadIdx.x];
     qt0[((g * c1 + p) * b2 + i) * D + threadIdx.x] = __float2bfloat16_rn(sum / (float)(l1 - l0));
   }
 }
@@ -1980,8 +1994,8 @@ cudaError_t launch_r_step1(const bf16* q, const bf16* k, const bf16* v, bf16* qt
                            bf16* y, float* hs, const Problem& pb, int* status,
                            cudaStream_t stream, int* launches) {
   cudaError_t e = timed_launch("tc_init_qt", stream, launches, [&] {
-    init_qt_bf16_kernel<D><<<(unsigned)((long)pb.G * pb.c1 * pb.b2), 512, 0, stream>>>(
-        q, qt0, pb.b1, pb.b2, pb.c1);
+    return launch_pdl(init_qt_bf16_kernel<D>, dim3((unsigned)((long)pb.G * pb.c1 * pb.b2)),
+                      dim3(256), 0, stream, q, qt0, pb.b1, pb.b2, pb.c1);
   });
   if (e != cudaSuccess) return e;
   switch (kr_group_tile(pb)) {

@@ -142,3 +142,21 @@ def test_bounded_wait_timeout_is_reported_and_context_survives(cuda_lib):
     q, k, v = iid_qkv(1, 2, 64, 64, torch.bfloat16, seed=9)
     O = gpu_forward(cuda_lib, q, k, v, 8, 8, 1)
     assert_parity(O, oracle_forward(q, k, v, 8, 8, 1), v, torch.bfloat16)
+
+
+def test_back_to_back_calls_consume_previous_output(cuda_lib):
+    """Stream ordering across calls: the next call's queries (then keys) are
+    the previous call's output, issued without a host synchronisation, so an
+    early start of any kernel of the second call would read stale rows."""
+    wl = WORKLOADS["480p"]
+    q, k, v = make_inputs(wl)
+    qd, kd, vd = (x.cuda() for x in (q, k, v))
+    o1 = cuda_lib.monarch_attn_fwd(qd, kd, vd, wl.b1, wl.b2, wl.T)
+    o2 = cuda_lib.monarch_attn_fwd(o1, kd, vd, wl.b1, wl.b2, wl.T)
+    o3 = cuda_lib.monarch_attn_fwd(qd, o2, vd, wl.b1, wl.b2, wl.T)
+    cuda_lib.check()
+    o1c, o2c = o1.cpu(), o2.cpu()
+    assert_parity(o2.double().cpu().numpy(), oracle_forward(o1c, k, v, wl.b1, wl.b2, wl.T), v,
+                  wl.dtype)
+    assert_parity(o3.double().cpu().numpy(), oracle_forward(q, o2c, v, wl.b1, wl.b2, wl.T), v,
+                  wl.dtype)
