@@ -4,9 +4,9 @@
 // 5th-generation tensor cores: for every (head g, position i, row group p)
 // it is an attention of the |p| queries q_(l,i) against the b1*c2 keys
 // Kt_{k,p,q,i} with a per-key bias Hs and values Y
-// (MonarchAttention OpenReview discussion: the intermediate steps are
-// FlashAttention-like calls; MonarchRT summary, "Method" (3): the N x N
-// matrix is never formed):
+// (MonarchAttention OpenReview discussion, author response on the kernels:
+// each intermediate step is a fused attention-style call; MonarchRT
+// summary, "Method" (3): the N x N matrix is never formed):
 //
 //   S = q Kt^T / sqrt(d) + Hs          128 x NK tile, accumulated in TMEM
 //   L = softmax over (k, q) of S        online, one TMEM lane (row) per thread
