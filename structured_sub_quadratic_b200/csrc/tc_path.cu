@@ -337,10 +337,14 @@ __global__ void __launch_bounds__(192, 2)
           if (mbar_test(p_full + st, (Tp >> 1) & 1) && mbar_test(y_full + st, (Tp >> 1) & 1) &&
               (p_j > 0 || p_n == 0 || mbar_test(o_empty, (p_n - 1) & 1))) {
             tc_fence_after();
+            // A = P from TMEM, 8 columns per 16 keys; a partial last tile
+            // only over its valid keys (the rest of its P is not written)
+            const int kk_n = min(NK / 16, (a.nk - p_j * NK + 15) / 16);
 #pragma unroll
-            for (int kk = 0; kk < NK / 16; ++kk)  // A = P from TMEM: 8 columns per 16 keys
-              mma_bf16_ts(tmem_o, tmem_s(st) + kk * 8, (st ? dy1 : dy0) + ((kk * 16 * 128) >> 4),
-                          idesc_o, (p_j > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < NK / 16; ++kk)
+              if (kk < kk_n)
+                mma_bf16_ts(tmem_o, tmem_s(st) + kk * 8, (st ? dy1 : dy0) + ((kk * 16 * 128) >> 4),
+                            idesc_o, (p_j > 0 || kk > 0) ? 1u : 0u);
             mma_commit(y_empty + st);
             mma_commit(pv_done + st);
             last_pv = Tp;
@@ -388,16 +392,24 @@ __global__ void __launch_bounds__(192, 2)
         if (!ok) break;
         float sv[NK];
         tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < NK / 32; ++c) {
-          float t[32];
-          tmem_ld32(tmem_s(sb) + lane_off + c * 32, t);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) sv[c * 32 + e] = t[e];
-        }
-        tmem_wait_ld();
         const float* bias = sBias + sb * NK;
         const int valid = a.nk - j * NK;
+        // a last tile with at most NK/2 valid keys is handled at half width
+        // (its other columns are neither read nor written)
+        const bool half = valid <= NK / 2;
+#pragma unroll
+        for (int c = 0; c < NK / 32; ++c) {
+          if (c == 0 || !half) {
+            float t[32];
+            tmem_ld32(tmem_s(sb) + lane_off + c * 32, t);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) sv[c * 32 + e] = t[e];
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) sv[c * 32 + e] = -INFINITY;
+          }
+        }
+        tmem_wait_ld();
         // logits sc q.Kt + Hs (natural units); 4 partial maxima / sums break
         // the serial chains
         float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -410,8 +422,10 @@ __global__ void __launch_bounds__(192, 2)
         } else {
 #pragma unroll
           for (int c = 0; c < NK; ++c) {
-            sv[c] = c < valid ? fmaf(sv[c], a.sc, bias[c]) : -INFINITY;
-            mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
+            if (c < NK / 2 || !half) {
+              sv[c] = c < valid ? fmaf(sv[c], a.sc, bias[c]) : -INFINITY;
+              mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
+            }
           }
         }
         mbar_arrive(bias_empty + sb);
@@ -427,8 +441,10 @@ __global__ void __launch_bounds__(192, 2)
         float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int c = 0; c < NK; ++c) {
-          sv[c] = ex2(fmaf(sv[c], kLog2e, neg_m2));
-          ls[c & 3] += sv[c];
+          if (c < NK / 2 || !half) {
+            sv[c] = ex2(fmaf(sv[c], kLog2e, neg_m2));
+            ls[c & 3] += sv[c];
+          }
         }
         l_run = l_run * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
         if (__any_sync(0xffffffffu, resc)) {
@@ -451,10 +467,13 @@ __global__ void __launch_bounds__(192, 2)
         // P (bf16 pairs) over the first NK/2 columns of this tile's S buffer
 #pragma unroll
         for (int c = 0; c < NK / 32; ++c) {
-          uint32_t pk[16];
+          if (c == 0 || !half) {
+            uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(sv[c * 32 + 2 * e], sv[c * 32 + 2 * e + 1]);
-          tmem_st16(tmem_s(sb) + lane_off + c * 16, pk);
+            for (int e = 0; e < 16; ++e)
+              pk[e] = pack_bf16x2(sv[c * 32 + 2 * e], sv[c * 32 + 2 * e + 1]);
+            tmem_st16(tmem_s(sb) + lane_off + c * 16, pk);
+          }
         }
         tmem_wait_st();
         tc_fence_before();
