@@ -100,6 +100,55 @@ __device__ __forceinline__ bool ko_decode(const KOArgs& a, int item, KOItem& it)
   return true;
 }
 
+// Epilogue of the output kernels (four softmax warps, thread = tile row):
+// O / l from TMEM to the rows' global memory.  TMEM loads run one 32-column
+// unit ahead of the staging; each 64-column half is staged (swizzled) in
+// sP, then 8 threads write one row's 128-byte half, so global stores are
+// whole sectors.  o_empty is arrived on as soon as the last TMEM load of O
+// has landed, so the next item's P Y may start while the rows go out.
+template <int D>
+__device__ __forceinline__ void ko_epilogue(uint32_t tmem_o, uint32_t lane_off, int row, float inv,
+                                            uint8_t* sP, bf16* out_rows, long row_stride,
+                                            int nrows, uint64_t* o_empty) {
+  const int srow = threadIdx.x - 64;  // 0..127 over the four softmax warps
+  float rs[2][32];
+  tmem_ld32(tmem_o + lane_off, rs[0]);
+#pragma unroll
+  for (int u = 0; u < D / 32; ++u) {
+    const int h = u >> 1, c = u & 1;
+    tmem_wait_ld();  // unit u is in registers
+    if (u == D / 32 - 1) {  // O fully read: the next P Y may overwrite it
+      tc_fence_before();
+      mbar_arrive(o_empty);
+    } else {
+      tmem_ld32(tmem_o + lane_off + (u + 1) * 32, rs[(u + 1) & 1]);
+    }
+#pragma unroll
+    for (int uu = 0; uu < 4; ++uu) {
+      const float* t = rs[u & 1] + 8 * uu;
+      uint4 pk;
+      pk.x = pack_bf16x2(t[0] * inv, t[1] * inv);
+      pk.y = pack_bf16x2(t[2] * inv, t[3] * inv);
+      pk.z = pack_bf16x2(t[4] * inv, t[5] * inv);
+      pk.w = pack_bf16x2(t[6] * inv, t[7] * inv);
+      const int unit = c * 4 + uu;
+      *reinterpret_cast<uint4*>(sP + row * 128 + ((unit ^ (row & 7)) << 4)) = pk;
+    }
+    if (c == 1) {
+      named_barrier(1, 128);
+#pragma unroll
+      for (int pass = 0; pass < kRows / 16; ++pass) {
+        const int r = pass * 16 + (srow >> 3), unit = srow & 7;
+        if (r < nrows) {
+          const uint4 v4 = *reinterpret_cast<const uint4*>(sP + r * 128 + ((unit ^ (r & 7)) << 4));
+          *reinterpret_cast<uint4*>(out_rows + r * row_stride + h * 64 + unit * 8) = v4;
+        }
+      }
+      named_barrier(1, 128);
+    }
+  }
+}
+
 // Persistent, warp-specialised L-update + output.  Warp 0 loads Q, Kt, Y
 // (TMA) and the entropy bias (plain loads), warp 1 issues the tcgen05.mma
 // instructions from one thread, warps 2-5 own the 128 rows (TMEM lanes) for
@@ -485,43 +534,9 @@ __global__ void __launch_bounds__(192, 2)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const float inv = 1.f / l_run;
-      // Rows go out through shared memory (the P buffer is free now): each
-      // thread stages its row, then 8 threads write one row's 128-byte half,
-      // so global stores are whole sectors.
-      const int srow = tid - 64;  // 0..127 over the four softmax warps
-#pragma unroll 1
-      for (int h = 0; h < D / 64; ++h) {
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          float t[32];
-          tmem_ld32(tmem_o + lane_off + h * 64 + c * 32, t);
-          tmem_wait_ld();
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            uint4 pk;
-            pk.x = pack_bf16x2(t[8 * u + 0] * inv, t[8 * u + 1] * inv);
-            pk.y = pack_bf16x2(t[8 * u + 2] * inv, t[8 * u + 3] * inv);
-            pk.z = pack_bf16x2(t[8 * u + 4] * inv, t[8 * u + 5] * inv);
-            pk.w = pack_bf16x2(t[8 * u + 6] * inv, t[8 * u + 7] * inv);
-            const int unit = c * 4 + u;
-            *reinterpret_cast<uint4*>(sP + row * 128 + ((unit ^ (row & 7)) << 4)) = pk;
-          }
-        }
-        named_barrier(1, 128);
-#pragma unroll
-        for (int pass = 0; pass < kRows / 16; ++pass) {
-          const int r = pass * 16 + (srow >> 3), unit = srow & 7;
-          if (r < it.nrows) {
-            const uint4 v4 = *reinterpret_cast<const uint4*>(sP + r * 128 + ((unit ^ (r & 7)) << 4));
-            bf16* dst = a.out + (((long)it.g * a.b1 + it.row0 + r) * a.b2 + it.i) * D + h * 64;
-            *reinterpret_cast<uint4*>(dst + unit * 8) = v4;
-          }
-        }
-        named_barrier(1, 128);
-      }
-      tc_fence_before();
-      mbar_arrive(o_empty);
+      ko_epilogue<D>(tmem_o, lane_off, row, 1.f / l_run, sP,
+                     a.out + (((long)it.g * a.b1 + it.row0) * a.b2 + it.i) * D, (long)a.b2 * D,
+                     it.nrows, o_empty);
     }
   }
   tc_fence_before();
@@ -789,45 +804,9 @@ __global__ void __launch_bounds__(192, 2)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const float inv = 1.f / l_row;
-      // Rows go out through shared memory: each thread stages its row, then 8
-      // threads write one row's 128-byte half, so global stores are whole
-      // sectors.
-      const int srow = tid - 64;  // 0..127 over the four softmax warps
-#pragma unroll 1
-      for (int h = 0; h < D / 64; ++h) {
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          float t[32];
-          tmem_ld32(tmem_o + lane_off + h * 64 + c * 32, t);
-          tmem_wait_ld();
-          if (h == D / 64 - 1 && c == 1) {  // O fully read: the next P Y may overwrite it
-            tc_fence_before();
-            mbar_arrive(o_empty);
-          }
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            uint4 pk;
-            pk.x = pack_bf16x2(t[8 * u + 0] * inv, t[8 * u + 1] * inv);
-            pk.y = pack_bf16x2(t[8 * u + 2] * inv, t[8 * u + 3] * inv);
-            pk.z = pack_bf16x2(t[8 * u + 4] * inv, t[8 * u + 5] * inv);
-            pk.w = pack_bf16x2(t[8 * u + 6] * inv, t[8 * u + 7] * inv);
-            const int unit = c * 4 + u;
-            *reinterpret_cast<uint4*>(sP + row * 128 + ((unit ^ (row & 7)) << 4)) = pk;
-          }
-        }
-        named_barrier(1, 128);
-#pragma unroll
-        for (int pass = 0; pass < kRows / 16; ++pass) {
-          const int r = pass * 16 + (srow >> 3), unit = srow & 7;
-          if (r < it.nrows) {
-            const uint4 v4 = *reinterpret_cast<const uint4*>(sP + r * 128 + ((unit ^ (r & 7)) << 4));
-            bf16* dst = a.out + (((long)it.g * a.b1 + it.row0 + r) * a.b2 + it.i) * D + h * 64;
-            *reinterpret_cast<uint4*>(dst + unit * 8) = v4;
-          }
-        }
-        named_barrier(1, 128);
-      }
+      ko_epilogue<D>(tmem_o, lane_off, row, 1.f / l_row, sP,
+                     a.out + (((long)it.g * a.b1 + it.row0) * a.b2 + it.i) * D, (long)a.b2 * D,
+                     it.nrows, o_empty);
       ++n;
     }
   }
@@ -1561,35 +1540,47 @@ __global__ void __launch_bounds__(320, 1)
           tc_fence_before();
           mbar_arrive(tmem_free + w);
         } else {
-#pragma unroll 1
-          for (int cb = 0; cb < nblk; ++cb) {
-            uint8_t* buf = pbuf + (cb & 1) * (kRows * 128) + quad * 32 * 128;
-            float ta[32], tb[32];
-            tmem_ld32(tslot + lane_off + cb * 64, ta);
-            tmem_ld32(tslot + lane_off + cb * 64 + 32, tb);
-            if (cb >= 2 && lane == 0) bulk_wait_read<1>();  // store of block cb-2 has read buf
-            __syncwarp();
-            tmem_wait_ld();
-            if (cb == nblk - 1) {  // slot fully read out: the MMA may reuse it
-              tc_fence_before();
-              mbar_arrive(tmem_free + w);
-            }
+          // TMEM loads run one 32-column unit ahead of the staging: unit
+          // u + 1 is in flight while unit u is packed into its 64-column
+          // block's staging rows; a block goes out once both halves are in.
+          float rs[2][32];
+          tmem_ld32(tslot + lane_off, rs[0]);
 #pragma unroll
-            for (int uu = 0; uu < 8; ++uu) {
-              const float* v = uu < 4 ? ta + 8 * uu : tb + 8 * (uu - 4);
-              uint4 pk;
-              pk.x = pack_bf16x2(v[0], v[1]);
-              pk.y = pack_bf16x2(v[2], v[3]);
-              pk.z = pack_bf16x2(v[4], v[5]);
-              pk.w = pack_bf16x2(v[6], v[7]);
-              *reinterpret_cast<uint4*>(buf + lane * 128 + ((uu ^ (lane & 7)) << 4)) = pk;
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-              tma_store_4d(cb < D / 64 ? &tm_kt : &tm_y, buf, (cb % (D / 64)) * 64, ycoord, i0,
-                           sb.g);
-              bulk_commit();
+          for (int u = 0; u < 4 * (D / 64); ++u) {
+            if (u < 2 * nblk) {
+              const int cb = u >> 1, hf = u & 1;
+              tmem_wait_ld();  // unit u is in registers
+              if (u == 2 * nblk - 1) {  // slot fully read out: the MMA may reuse it
+                tc_fence_before();
+                mbar_arrive(tmem_free + w);
+              } else {
+                tmem_ld32(tslot + lane_off + (u + 1) * 32, rs[(u + 1) & 1]);
+              }
+              uint8_t* buf = pbuf + (cb & 1) * (kRows * 128) + quad * 32 * 128;
+              if (hf == 0) {
+                if (cb >= 2 && lane == 0) bulk_wait_read<1>();  // store of block cb-2 has read buf
+                __syncwarp();
+              }
+#pragma unroll
+              for (int uu = 0; uu < 4; ++uu) {
+                const float* v = rs[u & 1] + 8 * uu;
+                uint4 pk;
+                pk.x = pack_bf16x2(v[0], v[1]);
+                pk.y = pack_bf16x2(v[2], v[3]);
+                pk.z = pack_bf16x2(v[4], v[5]);
+                pk.w = pack_bf16x2(v[6], v[7]);
+                const int chunk = hf * 4 + uu;
+                *reinterpret_cast<uint4*>(buf + lane * 128 + ((chunk ^ (lane & 7)) << 4)) = pk;
+              }
+              if (hf == 1) {
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                  tma_store_4d(cb < D / 64 ? &tm_kt : &tm_y, buf, (cb % (D / 64)) * 64, ycoord,
+                               i0, sb.g);
+                  bulk_commit();
+                }
+              }
             }
           }
         }
