@@ -94,6 +94,8 @@ def kernel_work(name: str, wl: Workload):
         return fl, io + 2 * inter + G * N * c1 * c2 * 4 + io
     if name.endswith("l_stats"):
         return G * N * b1 * c2 * d * 2, io + inter
+    if name == "permute_rows":  # aligned video layouts: q, k, v in, or the output back
+        return 0, 2 * io * 2  # averaged over the two launches of a call (3 + 1 tensors)
     if name.endswith("l_aggregate"):
         return G * N * b1 * c2 * d * 4, io + inter + G * N * c1 * c2 * d * w
     return 0, 0
@@ -317,11 +319,14 @@ def run_reference(args, wl):
     return 0
 
 
-def workload_config(wl: Workload, l2_note):
+def workload_config(wl: Workload, l2_note, layout=None):
     cfg = {"workload": wl.name, "B": wl.B, "H": wl.H, "N": wl.N, "b1": wl.b1, "b2": wl.b2,
            "d": wl.d, "T": wl.T, "c1": wl.c1, "c2": wl.c2, "inputs": wl.kind, "seed": wl.seed}
     if wl.latent:
         cfg["latent_fhw"] = list(wl.latent)
+    if layout:
+        cfg["layout"] = f"({layout})"
+
     if l2_note:
         cfg["l2"] = l2_note
     return cfg
@@ -353,7 +358,11 @@ def run_native(args, wl):
 
     def step(s):
         q, k, v, o = sets[s % n_sets]
-        api.monarch_attn_fwd(q, k, v, wl.b1, wl.b2, wl.T, wl.c1, wl.c2, out=o, stream=stream)
+        if args.layout:
+            api.monarch_attn_fwd_video(q, k, v, *wl.latent, args.layout, wl.T, wl.c1, wl.c2,
+                                       out=o, stream=stream)
+        else:
+            api.monarch_attn_fwd(q, k, v, wl.b1, wl.b2, wl.T, wl.c1, wl.c2, out=o, stream=stream)
 
     log(f"{n_sets} input sets on device")
     for s in range(args.warmup):
@@ -425,18 +434,32 @@ def run_native(args, wl):
                                    "share": t / sum(x[0] for x in per_kernel.values())}
                                for k, (t, c) in per_kernel.items()}
 
-    # end to end through the host-buffer C-ABI call, copies inside the timed region
-    q, k, v, _ = sets[0]
+    # end to end through the public API with host buffers, copies inside the timed region:
+    # the host-buffer C-ABI call, or (aligned video layouts) pinned-host copies around the
+    # video-layout call
+    q, k, v, o = sets[0]
     qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
     oh = torch.empty_like(qh).pin_memory()
     e2e_steps = max(1, min(args.steps, 50))
-    api.monarch_attn_fwd_host(qh, kh, vh, oh, wl.b1, wl.b2, wl.T, wl.c1, wl.c2, stream=stream)
+
+    def e2e_call():
+        if args.layout:
+            for dst, src in ((q, qh), (k, kh), (v, vh)):
+                dst.copy_(src, non_blocking=True)
+            api.monarch_attn_fwd_video(q, k, v, *wl.latent, args.layout, wl.T, wl.c1, wl.c2,
+                                       out=o, stream=stream)
+            oh.copy_(o, non_blocking=True)
+            torch.cuda.current_stream(device).synchronize()
+        else:
+            api.monarch_attn_fwd_host(qh, kh, vh, oh, wl.b1, wl.b2, wl.T, wl.c1, wl.c2,
+                                      stream=stream)
+
+    e2e_call()
     barrier(device)
     torch.cuda.synchronize(device)
     ev0.record(stream)
     for _ in range(e2e_steps):
-        api.monarch_attn_fwd_host(qh, kh, vh, oh, wl.b1, wl.b2, wl.T, wl.c1, wl.c2,
-                                  stream=stream)
+        e2e_call()
     ev1.record(stream)
     torch.cuda.synchronize(device)
     barrier(device)
@@ -459,7 +482,7 @@ def run_native(args, wl):
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if wl.dtype == torch.bfloat16 else "f32",
-        "data": "synthetic", "config": workload_config(wl, l2_note),
+        "data": "synthetic", "config": workload_config(wl, l2_note, args.layout),
         "clocks": clk.summary(),
         "e2e": {"value": e2e_value, "unit": UNIT, "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": 3 * io_elt, "d2h_bytes_per_step": io_elt},
@@ -488,6 +511,10 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true", help="skip the clock sampler")
+    ap.add_argument("--layout", default=None,
+                    choices=["fh,w", "w,fh", "f,hw", "hw,f", "fw,h", "h,fw"],
+                    help="video workloads: aligned block layout of the latent (raster-order "
+                         "inputs through the video-layout entry point)")
     ap.add_argument("--heads", type=int, default=None,
                     help="override H (profiling a smaller case of the same shape)")
     args = ap.parse_args(argv)
@@ -496,6 +523,14 @@ def main(argv=None):
     wl = WORKLOADS[args.workload]
     if args.heads is not None:
         wl = Workload(**{**wl.__dict__, "H": args.heads, "name": f"{wl.name} [H={args.heads}]"})
+    if args.layout:
+        if not wl.latent:
+            ap.error("--layout needs a video workload (480p or 720p)")
+        size = dict(zip("fhw", wl.latent))
+        rows, cols = args.layout.split(",")
+        b1 = math.prod(size[a] for a in rows)
+        wl = Workload(**{**wl.__dict__, "b1": b1, "b2": wl.N // b1,
+                         "name": f"{wl.name} blocks ({args.layout})=({b1},{wl.N // b1})"})
     if args.impl == "reference":
         return run_reference(args, wl)
     return run_native(args, wl)

@@ -135,6 +135,39 @@ MONARCH_API int monarch_attn_fwd_noalloc(const void* q, const void* k, const voi
                                          int B, int H, int b1, int b2, int d, int T, int c1,
                                          int c2, cudaStream_t stream);
 
+/* Aligned block layouts of a video latent with f frames of h x w tokens,
+ * stored in raster order (token n = (t*h + y)*w + x for frame t, row y,
+ * column x).  A layout names the axes that form the Monarch row index l
+ * (first) and the position index i (second); b1 is the product of the first
+ * group's sizes, b2 of the second's (MonarchRT summary, "Key claims" and
+ * "Method": block sizes aligned with the latent's (f, h, w) axes).  Inside a
+ * group the axes keep the order written. */
+#define MONARCH_LAYOUT_FH_W 0  /* l = (f, h), i = w:      b1 = f*h, b2 = w   */
+#define MONARCH_LAYOUT_W_FH 1  /* l = w,      i = (f, h): b1 = w,   b2 = f*h */
+#define MONARCH_LAYOUT_F_HW 2  /* l = f,      i = (h, w): b1 = f,   b2 = h*w */
+#define MONARCH_LAYOUT_HW_F 3  /* l = (h, w), i = f:      b1 = h*w, b2 = f   */
+#define MONARCH_LAYOUT_FW_H 4  /* l = (f, w), i = h:      b1 = f*w, b2 = h   */
+#define MONARCH_LAYOUT_H_FW 5  /* l = h,      i = (f, w): b1 = h,   b2 = f*w */
+
+/* Forward pass on a video latent in one of the aligned layouts above.
+ * q, k, v, out: device pointers (B, H, N, d) in raster token order,
+ * N = f*h*w, dtype MONARCH_DTYPE_BF16 (__nv_bfloat16) or MONARCH_DTYPE_F32.
+ * The result is monarch_attn_fwd / _f32 applied to the tokens reordered
+ * into the layout's Monarch order (token l*b2 + i), with the output put back
+ * into raster order.  (fh, w) and (f, hw) are already in Monarch order and
+ * run directly; the other four layouts gather q, k, v into a cached device
+ * buffer of 4*B*H*N*d elements (allocated on first use, grown on demand,
+ * freed by monarch_attn_release_workspace) and scatter the output back: one
+ * extra read and write of each tensor.  The gather uses a table of N raster
+ * indices per (f, h, w, layout) and device, built and uploaded with a
+ * synchronous copy on its first use and kept until
+ * monarch_attn_release_workspace.  Otherwise asynchronous on `stream`; errors
+ * as for monarch_attn_fwd, plus MONARCH_ERR_INVALID_ARG for an unknown
+ * layout. */
+MONARCH_API int monarch_attn_fwd_video(int dtype, const void* q, const void* k, const void* v,
+                                       void* out, int B, int H, int f, int h, int w, int layout,
+                                       int d, int T, int c1, int c2, cudaStream_t stream);
+
 /* Bytes of device workspace a call with these arguments uses (0 on invalid
  * arguments).  dtype is MONARCH_DTYPE_BF16 or MONARCH_DTYPE_F32. */
 MONARCH_API size_t monarch_attn_workspace_bytes(int B, int H, int b1, int b2, int d, int T,

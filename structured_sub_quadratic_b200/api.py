@@ -25,6 +25,7 @@ DTYPE_BF16 = 0
 DTYPE_F32 = 1
 PATH_AUTO = 0
 PATH_SIMT = 1
+LAYOUTS = {"fh,w": 0, "w,fh": 1, "f,hw": 2, "hw,f": 3, "fw,h": 4, "h,fw": 5}
 
 # Every symbol the header declares, with its ctypes signature.
 _I, _P, _Z = ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t
@@ -34,6 +35,8 @@ SIGNATURES = {
     "monarch_attn_fwd_f32": (_I, [_P, _P, _P, _P, *_SIZES, _P]),
     "monarch_attn_fwd_host": (_I, [_I, _P, _P, _P, _P, *_SIZES, _P]),
     "monarch_attn_fwd_noalloc": (_I, [_P, _P, _P, _P, *_SIZES, _P]),
+    "monarch_attn_fwd_video": (_I, [_I, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I,
+                                    _I, _P]),
     "monarch_attn_workspace_bytes": (_Z, [*_SIZES, _I]),
     "monarch_attn_release_workspace": (None, []),
     "monarch_attn_check": (_I, [_P]),
@@ -141,6 +144,42 @@ def monarch_attn_fwd_noalloc(q, k, v, b1, b2, T, c1=1, c2=1, out=None, stream=No
     _check(lib.monarch_attn_fwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(),
                                         out.data_ptr(), B, H, b1, b2, d, T, c1, c2,
                                         _stream_ptr(stream)))
+    return out
+
+
+def video_blocks(f, h, w, layout):
+    """(b1, b2) of an aligned layout name such as "w,fh" (see LAYOUTS)."""
+    size = {"f": f, "h": h, "w": w}
+    rows, cols = layout.split(",")
+    b1 = 1
+    for a in rows:
+        b1 *= size[a]
+    b2 = 1
+    for a in cols:
+        b2 *= size[a]
+    return b1, b2
+
+
+def monarch_attn_fwd_video(q, k, v, f, h, w, layout, T, c1=1, c2=1, out=None, stream=None):
+    """Forward pass on a video latent (B, H, f*h*w, d) in raster token order,
+    with the Monarch blocks aligned to ``layout`` (a key of LAYOUTS)."""
+    lib = load_library()
+    if layout not in LAYOUTS:
+        raise ValueError(f"unknown layout {layout!r}; expected one of {sorted(LAYOUTS)}")
+    if q.dim() != 4 or q.shape[2] != f * h * w:
+        raise ValueError("expected (B, H, f*h*w, d) tensors")
+    B, H, _, d = q.shape
+    for t in (q, k, v):
+        if t.shape != q.shape or t.dtype != q.dtype or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous CUDA tensors of one shape and dtype")
+    dtype = {torch.bfloat16: DTYPE_BF16, torch.float32: DTYPE_F32}.get(q.dtype)
+    if dtype is None:
+        raise ValueError(f"unsupported dtype {q.dtype}")
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib.monarch_attn_fwd_video(dtype, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                      out.data_ptr(), B, H, f, h, w, LAYOUTS[layout], d, T, c1,
+                                      c2, _stream_ptr(stream)))
     return out
 
 

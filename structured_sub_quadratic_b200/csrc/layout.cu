@@ -1,0 +1,96 @@
+// Row permutation between raster and Monarch token order.
+#include "layout.cuh"
+
+#include <cstdint>
+
+#include "timing.cuh"
+
+namespace monarch {
+namespace {
+
+// One thread per unit of a row; consecutive threads cover consecutive units
+// of one row, so each row moves as one contiguous read and one contiguous
+// write.  UNITS > 0 fixes the units per row at compile time (a shift).
+// Up to three tensors per launch (blockIdx.y picks the pair).
+struct RowPairs {
+  const void* src[3];
+  void* dst[3];
+};
+
+template <typename U, int UNITS>
+__global__ void __launch_bounds__(256)
+    permute_rows_kernel(RowPairs pairs, const int* __restrict__ table, long total, int N,
+                        int units_rt, bool to_monarch) {
+  const int units = UNITS > 0 ? UNITS : units_rt;
+  const U* __restrict__ src = static_cast<const U*>(pairs.src[blockIdx.y]);
+  U* __restrict__ dst = static_cast<U*>(pairs.dst[blockIdx.y]);
+  for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (long)gridDim.x * blockDim.x) {
+    const long row = idx / units;
+    const int c = (int)(idx - row * units);
+    const long g = row / N;
+    const int m = (int)(row - g * N);
+    const long n = __ldg(table + m);
+    const long mi = (g * N + m) * units + c, ni = (g * N + n) * units + c;
+    if (to_monarch)
+      dst[mi] = src[ni];
+    else
+      dst[ni] = src[mi];
+  }
+}
+
+template <typename U, int UNITS>
+cudaError_t launch(const RowPairs& pairs, int npairs, const int* table, long G, int N,
+                   int row_bytes, bool to_monarch, cudaStream_t stream, int* launches) {
+  const int units = row_bytes / (int)sizeof(U);
+  const long total = G * N * (long)units;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long want = (total + 255) / 256;
+  const int grid = (int)(want < 16L * sms ? want : 16L * sms);
+  return timed_launch("permute_rows", stream, launches, [&] {
+    permute_rows_kernel<U, UNITS><<<dim3(grid, npairs), 256, 0, stream>>>(pairs, table, total, N,
+                                                                          units, to_monarch);
+  });
+}
+
+}  // namespace
+
+void video_perm_table(const VideoPerm& vp, int* table) {
+  int m = 0;
+  for (int x0 = 0; x0 < vp.s[0]; ++x0)
+    for (int x1 = 0; x1 < vp.s[1]; ++x1)
+      for (int x2 = 0; x2 < vp.s[2]; ++x2)
+        table[m++] = (int)(x0 * vp.t[0] + x1 * vp.t[1] + x2 * vp.t[2]);
+}
+
+cudaError_t permute_rows(const void* const* src, void* const* dst, int n, const int* table,
+                         long G, int N, int row_bytes, bool to_monarch, cudaStream_t stream,
+                         int* launches) {
+  if (n < 1 || n > 3 || G < 1 || N < 1 || row_bytes < 1) return cudaErrorInvalidValue;
+  RowPairs pairs = {};
+  uintptr_t a = static_cast<uintptr_t>(row_bytes);
+  for (int i = 0; i < n; ++i) {
+    pairs.src[i] = src[i];
+    pairs.dst[i] = dst[i];
+    a |= reinterpret_cast<uintptr_t>(src[i]) | reinterpret_cast<uintptr_t>(dst[i]);
+  }
+#define MONARCH_PERMUTE(U, UNITS) \
+  return launch<U, UNITS>(pairs, n, table, G, N, row_bytes, to_monarch, stream, launches)
+  if (a % 16 == 0) {
+    switch (row_bytes / 16) {  // d = 64 / 128 in bf16 or fp32
+      case 8: MONARCH_PERMUTE(uint4, 8);
+      case 16: MONARCH_PERMUTE(uint4, 16);
+      case 32: MONARCH_PERMUTE(uint4, 32);
+      default: MONARCH_PERMUTE(uint4, 0);
+    }
+  }
+  if (a % 8 == 0) MONARCH_PERMUTE(uint2, 0);
+  if (a % 4 == 0) MONARCH_PERMUTE(uint32_t, 0);
+  if (a % 2 == 0) MONARCH_PERMUTE(uint16_t, 0);
+  MONARCH_PERMUTE(uint8_t, 0);
+#undef MONARCH_PERMUTE
+}
+
+}  // namespace monarch

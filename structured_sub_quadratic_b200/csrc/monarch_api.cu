@@ -9,7 +9,9 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
+#include "layout.cuh"
 #include "simt_kernels.cuh"
 #include "tc_path.cuh"
 
@@ -27,8 +29,18 @@ struct DevBuf {
 
 std::mutex g_mu;                // workspace and status words
 std::mutex g_stage_mu;          // held for a whole host-buffer call
+std::mutex g_layout_mu;         // held for a whole video-layout call
 DevBuf g_ws[kMaxDevices];      // kernel workspace
 DevBuf g_stage[kMaxDevices];   // staging for the host-buffer entry point
+DevBuf g_layout[kMaxDevices];  // reordered q, k, v and output of the video-layout entry point
+
+// Raster index tables of the video layouts used so far, per device (uploaded
+// once per (f, h, w, layout); guarded by g_layout_mu).
+struct PermTable {
+  int f, h, w, layout;
+  int* dev_table;
+};
+std::vector<PermTable> g_tables[kMaxDevices];
 int* g_status[kMaxDevices];    // device status word (bounded-wait timeouts)
 std::atomic<int> g_path{MONARCH_PATH_AUTO};
 thread_local int t_launches = 0;
@@ -250,6 +262,88 @@ int monarch_attn_fwd_host(int dtype, const void* q_host, const void* k_host, con
   return monarch_attn_check(stream);
 }
 
+int monarch_attn_fwd_video(int dtype, const void* q, const void* k, const void* v, void* out,
+                           int B, int H, int f, int h, int w, int layout, int d, int T, int c1,
+                           int c2, cudaStream_t stream) {
+  if (dtype != MONARCH_DTYPE_BF16 && dtype != MONARCH_DTYPE_F32) return MONARCH_ERR_INVALID_ARG;
+  if (layout < MONARCH_LAYOUT_FH_W || layout > MONARCH_LAYOUT_H_FW) return MONARCH_ERR_INVALID_ARG;
+  if (f < 1 || h < 1 || w < 1 || (long long)f * h * w > (1LL << 30)) return MONARCH_ERR_INVALID_ARG;
+  // axes in Monarch order (sizes, raster strides in tokens) and the row-group size b1
+  const long hw = (long)h * w;
+  monarch::VideoPerm vp;
+  long b1 = 0;
+  auto axes = [&](int s0, long t0, int s1, long t1, int s2, long t2, long rows) {
+    vp.s[0] = s0; vp.t[0] = t0;
+    vp.s[1] = s1; vp.t[1] = t1;
+    vp.s[2] = s2; vp.t[2] = t2;
+    b1 = rows;
+  };
+  switch (layout) {
+    case MONARCH_LAYOUT_FH_W: axes(f, hw, h, w, w, 1, (long)f * h); break;
+    case MONARCH_LAYOUT_W_FH: axes(w, 1, f, hw, h, w, w); break;
+    case MONARCH_LAYOUT_F_HW: axes(f, hw, h, w, w, 1, f); break;
+    case MONARCH_LAYOUT_HW_F: axes(h, w, w, 1, f, hw, hw); break;
+    case MONARCH_LAYOUT_FW_H: axes(f, hw, w, 1, h, w, (long)f * w); break;
+    default: axes(h, w, f, hw, w, 1, h); break;  // MONARCH_LAYOUT_H_FW
+  }
+  const int N = (int)((long)f * hw), rows = (int)b1, cols = N / rows;
+  int st = validate(B, H, rows, cols, d, T, c1, c2);
+  if (st != MONARCH_OK) return st;
+  auto fwd = [&](const void* a, const void* b, const void* c, void* o) {
+    return dtype == MONARCH_DTYPE_BF16
+               ? monarch_attn_fwd(a, b, c, o, B, H, rows, cols, d, T, c1, c2, stream)
+               : monarch_attn_fwd_f32(static_cast<const float*>(a), static_cast<const float*>(b),
+                                      static_cast<const float*>(c), static_cast<float*>(o), B, H,
+                                      rows, cols, d, T, c1, c2, stream);
+  };
+  if (layout == MONARCH_LAYOUT_FH_W || layout == MONARCH_LAYOUT_F_HW) return fwd(q, k, v, out);
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return MONARCH_ERR_INVALID_ARG;
+  const int row_bytes = d * (dtype == MONARCH_DTYPE_BF16 ? 2 : 4);
+  const size_t slot = align_up((size_t)B * H * N * row_bytes);
+  int dev;
+  if ((st = current_device(&dev)) != MONARCH_OK) return st;
+  std::lock_guard<std::mutex> layout_lock(g_layout_mu);
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if ((st = ensure(g_layout[dev], 4 * slot)) != MONARCH_OK) return st;
+  }
+  char* base = static_cast<char*>(g_layout[dev].ptr);
+  char *dq = base, *dk = base + slot, *dv = base + 2 * slot, *dout = base + 3 * slot;
+  const int* table = nullptr;
+  for (const PermTable& t : g_tables[dev])
+    if (t.f == f && t.h == h && t.w == w && t.layout == layout) table = t.dev_table;
+  cudaError_t e;
+  if (!table) {  // first use of this latent and layout on this device: build and upload
+    std::vector<int> host(N);
+    monarch::video_perm_table(vp, host.data());
+    int* p = nullptr;
+    if ((e = cudaMalloc(&p, sizeof(int) * N)) != cudaSuccess) return record_cuda(e);
+    if ((e = cudaMemcpy(p, host.data(), sizeof(int) * N, cudaMemcpyHostToDevice)) !=
+        cudaSuccess) {
+      cudaFree(p);
+      return record_cuda(e);
+    }
+    g_tables[dev].push_back({f, h, w, layout, p});
+    table = p;
+  }
+  const long G = (long)B * H;
+  int perm_launches = 0;
+  const void* in_src[3] = {q, k, v};
+  void* in_dst[3] = {dq, dk, dv};
+  if ((e = monarch::permute_rows(in_src, in_dst, 3, table, G, N, row_bytes, true, stream,
+                                 &perm_launches)) != cudaSuccess)
+    return record_cuda(e);
+  if ((st = fwd(dq, dk, dv, dout)) != MONARCH_OK) return st;
+  const void* out_src[1] = {dout};
+  void* out_dst[1] = {out};
+  if ((e = monarch::permute_rows(out_src, out_dst, 1, table, G, N, row_bytes, false, stream,
+                                 &perm_launches)) != cudaSuccess)
+    return record_cuda(e);
+  t_launches += perm_launches;
+  return MONARCH_OK;
+}
+
 size_t monarch_attn_workspace_bytes(int B, int H, int b1, int b2, int d, int T, int c1, int c2,
                                     int dtype) {
   if (validate(B, H, b1, b2, d, T, c1, c2) != MONARCH_OK) return 0;
@@ -258,18 +352,25 @@ size_t monarch_attn_workspace_bytes(int B, int H, int b1, int b2, int d, int T, 
 }
 
 void monarch_attn_release_workspace(void) {
+  std::lock_guard<std::mutex> layout_lock(g_layout_mu);
   std::lock_guard<std::mutex> stage_lock(g_stage_mu);
   std::lock_guard<std::mutex> lock(g_mu);
   int cur = 0;
   cudaGetDevice(&cur);
   for (int dev = 0; dev < kMaxDevices; ++dev) {
-    if (!g_ws[dev].ptr && !g_stage[dev].ptr && !g_status[dev]) continue;
+    if (!g_ws[dev].ptr && !g_stage[dev].ptr && !g_layout[dev].ptr && g_tables[dev].empty() &&
+        !g_status[dev])
+      continue;
     cudaSetDevice(dev);
     if (g_ws[dev].ptr) cudaFree(g_ws[dev].ptr);
     if (g_stage[dev].ptr) cudaFree(g_stage[dev].ptr);
+    if (g_layout[dev].ptr) cudaFree(g_layout[dev].ptr);
+    for (PermTable& t : g_tables[dev]) cudaFree(t.dev_table);
+    g_tables[dev].clear();
     if (g_status[dev]) cudaFree(g_status[dev]);
     g_ws[dev] = DevBuf();
     g_stage[dev] = DevBuf();
+    g_layout[dev] = DevBuf();
     g_status[dev] = nullptr;
   }
   cudaSetDevice(cur);

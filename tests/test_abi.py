@@ -90,3 +90,23 @@ def test_path_switch_round_trips(lib):
     prev = lib.monarch_attn_set_path(api.PATH_SIMT)
     assert lib.monarch_attn_set_path(prev) == api.PATH_SIMT
     assert lib.monarch_attn_set_path(7) == -1
+
+
+@pytest.mark.parametrize("dtype,f,h,w,layout,expect", [
+    (api.DTYPE_BF16, 2, 3, 4, 6, api.MONARCH_ERR_INVALID_ARG),    # unknown layout
+    (api.DTYPE_BF16, 2, 3, 4, -1, api.MONARCH_ERR_INVALID_ARG),   # unknown layout
+    (7, 2, 3, 4, 1, api.MONARCH_ERR_INVALID_ARG),                 # unknown dtype
+    (api.DTYPE_BF16, 0, 3, 4, 1, api.MONARCH_ERR_INVALID_ARG),    # empty latent
+    (api.DTYPE_F32, 2, 3, 4, 1, api.MONARCH_ERR_INVALID_ARG),     # null pointers (after the shape)
+])
+def test_video_layout_entry_validates_before_any_launch(lib, dtype, f, h, w, layout, expect):
+    st = lib.monarch_attn_fwd_video(dtype, None, None, None, None, 1, 1, f, h, w, layout, 64, 1,
+                                    1, 1, None)
+    assert st == expect
+
+
+def test_video_blocks_of_each_layout():
+    f, h, w = 3, 30, 52
+    got = {name: api.video_blocks(f, h, w, name) for name in api.LAYOUTS}
+    assert got == {"fh,w": (90, 52), "w,fh": (52, 90), "f,hw": (3, 1560), "hw,f": (1560, 3),
+                   "fw,h": (156, 30), "h,fw": (30, 156)}

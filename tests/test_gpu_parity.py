@@ -160,3 +160,44 @@ def test_back_to_back_calls_consume_previous_output(cuda_lib):
                   wl.dtype)
     assert_parity(o3.double().cpu().numpy(), oracle_forward(q, o2c, v, wl.b1, wl.b2, wl.T), v,
                   wl.dtype)
+
+
+# Aligned video layouts: Monarch token m is raster token perm[m], with the
+# latent's (f, h, w) axes taken in the layout's order.
+LAYOUT_AXES = {"fh,w": (0, 1, 2), "w,fh": (2, 0, 1), "f,hw": (0, 1, 2), "hw,f": (1, 2, 0),
+               "fw,h": (0, 2, 1), "h,fw": (1, 0, 2)}
+
+
+def layout_oracle(q, k, v, latent, layout, T, c1=1, c2=1):
+    f, h, w = latent
+    perm = np.arange(f * h * w).reshape(f, h, w).transpose(LAYOUT_AXES[layout]).reshape(-1)
+    sizes = [latent[a] for a in LAYOUT_AXES[layout]]
+    split = 2 if layout in ("fh,w", "hw,f", "fw,h") else 1
+    b1 = int(np.prod(sizes[:split]))
+    ref_m = oracle_forward(q[..., perm, :], k[..., perm, :], v[..., perm, :], b1,
+                           f * h * w // b1, T, c1, c2)
+    ref = np.empty_like(ref_m)
+    ref[..., perm, :] = ref_m
+    return ref
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("layout", list(LAYOUT_AXES))
+def test_video_layouts_match_the_permuted_oracle(cuda_lib, dtype, layout):
+    latent = (2, 6, 8)
+    q, k, v = video_qkv(1, 2, latent, 64, dtype, seed=11)
+    O = cuda_lib.monarch_attn_fwd_video(q.cuda(), k.cuda(), v.cuda(), *latent, layout, 1)
+    cuda_lib.check()
+    assert_parity(O.double().cpu().numpy(), layout_oracle(q, k, v, latent, layout, 1), v, dtype)
+
+
+@pytest.mark.parametrize("layout,T,c", [("w,fh", 1, 1), ("hw,f", 1, 1), ("h,fw", 2, 2)])
+def test_video_layouts_on_the_480p_latent(cuda_lib, layout, T, c):
+    """The 480p latent (3, 30, 52), two heads, bf16: (w,fh) is 52 x 90 blocks
+    (wide column groups), (hw,f) 1560 x 3 (long L rows), (h,fw) tiled."""
+    latent = (3, 30, 52)
+    q, k, v = video_qkv(1, 2, latent, 128, torch.bfloat16, seed=12)
+    O = cuda_lib.monarch_attn_fwd_video(q.cuda(), k.cuda(), v.cuda(), *latent, layout, T, c, c)
+    cuda_lib.check()
+    assert_parity(O.double().cpu().numpy(), layout_oracle(q, k, v, latent, layout, T, c, c), v,
+                  torch.bfloat16)
