@@ -94,6 +94,8 @@ def kernel_work(name: str, wl: Workload):
         return fl, io + 2 * inter + G * N * c1 * c2 * 4 + io
     if name.endswith("l_stats"):
         return G * N * b1 * c2 * d * 2, io + inter
+    if name == "small_head":  # the whole forward pass of small heads in one kernel
+        return alg_flops(wl), alg_bytes(wl)
     if name == "permute_rows":  # aligned video layouts: q, k, v in, or the output back
         return 0, 2 * io * 2  # averaged over the two launches of a call (3 + 1 tensors)
     if name.endswith("l_aggregate"):

@@ -13,6 +13,7 @@
 
 #include "layout.cuh"
 #include "simt_kernels.cuh"
+#include "small_head.cuh"
 #include "tc_path.cuh"
 
 namespace {
@@ -87,9 +88,12 @@ Problem make_problem(int B, int H, int b1, int b2, int d, int T, int c1, int c2)
   return pb;
 }
 
-// Workspace of one call: the tensor-core path's if it takes the shape, else
-// the SIMT path's (fp32 pieces, each 256-byte aligned).
+// Workspace of one call: none for the one-CTA-per-head kernel (small untiled
+// heads with T >= 2, whose later steps would otherwise run on the SIMT
+// kernels), the tensor-core path's if it takes the shape, else the SIMT
+// path's (fp32 pieces, each 256-byte aligned).
 struct Plan {
+  bool small = false;
   bool tc = false;
   size_t bytes = 0;
   monarch::SimtWorkspaceSizes simt{};
@@ -97,6 +101,11 @@ struct Plan {
 
 Plan make_plan(const Problem& pb, int dtype) {
   Plan pl;
+  if (dtype == MONARCH_DTYPE_BF16 && g_path.load() == MONARCH_PATH_AUTO && pb.T >= 2 &&
+      monarch::small_head_supports(pb)) {
+    pl.small = true;
+    return pl;
+  }
   if (dtype == MONARCH_DTYPE_BF16 && g_path.load() == MONARCH_PATH_AUTO &&
       monarch::tc_supports(pb)) {
     pl.tc = true;
@@ -193,7 +202,12 @@ int forward_device(const TIn* q, const TIn* k, const TIn* v, TIn* out, int B, in
   if ((st = ensure_status(dev)) != MONARCH_OK) return st;
   if ((st = ensure(g_ws[dev], pl.bytes ? pl.bytes : kAlign)) != MONARCH_OK) return st;
   cudaError_t e;
-  if (pl.tc) {
+  if (pl.small) {
+    e = monarch::small_head_forward(reinterpret_cast<const monarch::bf16*>(q),
+                                    reinterpret_cast<const monarch::bf16*>(k),
+                                    reinterpret_cast<const monarch::bf16*>(v),
+                                    reinterpret_cast<monarch::bf16*>(out), pb, stream, &t_launches);
+  } else if (pl.tc) {
     e = monarch::tc_forward(reinterpret_cast<const monarch::bf16*>(q),
                             reinterpret_cast<const monarch::bf16*>(k),
                             reinterpret_cast<const monarch::bf16*>(v),

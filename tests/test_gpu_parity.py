@@ -74,6 +74,10 @@ EDGE = [
     (1, 2, 200, 8, 64, 1, 1, 1),     # more than 128 keys per L row: multi-tile output kernel
     (1, 1, 70, 20, 128, 2, 2, 2),    # 140 keys per L row in row groups, two steps
     (1, 1, 45, 64, 128, 1, 1, 1),    # paired R tiles with 64 positions, odd sub-item count
+    (2, 3, 5, 7, 64, 2, 1, 1),       # small head kept in shared memory, two steps
+    (1, 2, 16, 13, 64, 3, 1, 1),     # largest small-head blocks, three steps
+    (1, 1, 1, 9, 64, 2, 1, 1),       # small head, one row block
+    (1, 1, 12, 1, 64, 2, 1, 1),      # small head, one position
 ]
 
 
