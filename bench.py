@@ -104,7 +104,8 @@ def kernel_work(name: str, wl: Workload):
 
 
 def kernel_bound(name: str):
-    return "alu" if name.startswith("simt") else None
+    # FP32 SIMT arithmetic: the generic kernels and the one-CTA-per-head kernel
+    return "alu" if name.startswith("simt") or name == "small_head" else None
 
 
 # ---------------------------------------------------------------------------
