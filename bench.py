@@ -104,8 +104,7 @@ def kernel_work(name: str, wl: Workload):
 
 
 def kernel_bound(name: str):
-    # FP32 SIMT arithmetic: the generic kernels and the one-CTA-per-head kernel
-    return "alu" if name.startswith("simt") or name == "small_head" else None
+    return "alu" if name.startswith("simt") else None
 
 
 # ---------------------------------------------------------------------------
