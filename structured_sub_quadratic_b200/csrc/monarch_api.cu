@@ -1,8 +1,10 @@
 // C ABI of the MonarchAttention forward pass (declared in include/monarch_attn.h).
 //
 // This file validates arguments, owns the per-device workspace cache and the
-// device status word, and dispatches to the kernels: the tcgen05 tensor-core
-// path for the bf16 shapes it supports, the SIMT path for everything else.
+// device status word, and dispatches to the kernels: the one-CTA-per-head
+// kernel for small untiled bf16 heads with T >= 2, the tcgen05 tensor-core
+// path for the other bf16 shapes it supports, the SIMT path for everything
+// else.  The video-layout entry point reorders tokens around a forward call.
 #include "monarch_attn.h"
 
 #include <atomic>
