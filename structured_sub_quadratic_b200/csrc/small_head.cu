@@ -14,9 +14,11 @@
 //   L-update  warp i:  S = sc q_(.,i) Kt_i^T + Hs_i (rows l, columns k),
 //             L = softmax_k; non-final: Qt_{k,i} = L^T q_(.,i) / column sums
 //             of L; final: O_(l,i) = L Y_i
-// Kt, Y, Qt and P are stored as bf16 (as on the tensor-core path), softmax
-// statistics and Hs in fp32.  bf16 rows are padded to 144 bytes so that the
-// 8 row groups of a fragment load hit different shared-memory banks.
+// Kt, Y, Qt, P and L are stored as bf16 (as on the tensor-core path),
+// softmax statistics and Hs in fp32.  Fragments come from shared memory by
+// ldmatrix (transposed where the operand is stored k-major); bf16 rows are
+// padded to 144 bytes (L tiles to 48) so that the 8 rows of each 8 x 8
+// matrix hit different banks.
 #include "small_head.cuh"
 
 #include <mutex>
@@ -35,17 +37,25 @@ constexpr int kWarps = 16;     // one per chunk k (R-update) or position i (L-up
 constexpr int kThreads = kWarps * 32;
 constexpr float kLog2e = 1.4426950408889634f;
 
+constexpr int kPL = 24;         // L tile row pitch (bf16): 48-byte rows, conflict-free ldmatrix
+
 constexpr size_t smem_bytes(int n) {
-  // Qs, Ks, Vs, Kt, Ys, Qt (bf16 rows), Hs, L tiles [16 positions][16][16] fp32
-  return (size_t)n * (6 * kPB * 2 + 4) + (size_t)kMaxB * kMaxB * kMaxB * 4;
+  // Qs, Ks, Vs, Kt, Ys, Qt (bf16 rows), Hs, L tiles [16 positions][16 l][kPL] bf16
+  return (size_t)n * 6 * kPB * 2 + (size_t)((n + 3) & ~3) * 4 + (size_t)kMaxB * kMaxB * kPL * 2;
 }
 
-__device__ __forceinline__ uint32_t ld32(const bf16* p) {
-  return *reinterpret_cast<const uint32_t*>(p);
+// Four 8 x 8 bf16 matrices from shared memory (lane l gives the address of
+// row l % 8 of matrix l / 8); .trans delivers each matrix transposed.
+__device__ __forceinline__ void ldsm4(uint32_t (&r)[4], const bf16* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(tc::smem_u32(p)));
 }
 
-__device__ __forceinline__ uint32_t pack2(bf16 lo, bf16 hi) {
-  return (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
+__device__ __forceinline__ void ldsm4_t(uint32_t (&r)[4], const bf16* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(tc::smem_u32(p)));
 }
 
 // D += A B for one m16n8k16 tile (A 16 x 16 row-major, B 16 x 8 column-major).
@@ -122,10 +132,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   bf16* Ys = Kt + N * kPB;
   bf16* Qt = Ys + N * kPB;                   // rows (k, i): k * b2 + i
   float* Hs = reinterpret_cast<float*>(Qt + N * kPB);  // (i, k)
-  float* Ls = Hs + N;                        // [position i][l][k] L tiles
+  bf16* Ls = reinterpret_cast<bf16*>(Hs + ((N + 3) & ~3));  // [position i][l][k], pitch kPL
   const long gh = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
+  // ldmatrix lane roles: matrix mi = lane / 8, row lr = lane % 8
+  const int mi = lane >> 3, lr = lane & 7;
 
   // q, k, v of the head into shared memory (16-byte chunks)
   {
@@ -160,21 +172,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- R-update: warp kk, rows i (positions), columns j (keys of chunk kk) ----
     if (warp < b1) {
       const int kk = warp;
-      const int i0 = min(g, b2 - 1), i1 = min(g + 8, b2 - 1);  // clamped rows (results unused)
-      const bf16* qa = Qt + (kk * b2 + i0) * kPB;
-      const bf16* qb = Qt + (kk * b2 + i1) * kPB;
       const bf16* kr = Ks + kk * b2 * kPB;
       const bf16* vr = Vs + kk * b2 * kPB;
+      // A rows i (clamped; their results are unused), B rows j (keys, clamped and masked)
+      const bf16* a_src = Qt + (kk * b2 + min(lr + (mi & 1) * 8, b2 - 1)) * kPB + (mi >> 1) * 8;
+      const bf16* b_src = kr + min(lr + (mi >> 1) * 8, b2 - 1) * kPB + (mi & 1) * 8;
       float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
       for (int ks = 0; ks < kD / 16; ++ks) {
-        const int c = ks * 16 + 2 * t;
-        const uint32_t a[4] = {ld32(qa + c), ld32(qb + c), ld32(qa + c + 8), ld32(qb + c + 8)};
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          const bf16* krow = kr + min(nt * 8 + g, b2 - 1) * kPB;
-          mma16816(s[nt], a, ld32(krow + c), ld32(krow + c + 8));
-        }
+        uint32_t a[4], b[4];
+        ldsm4(a, a_src + ks * 16);
+        ldsm4(b, b_src + ks * 16);
+        mma16816(s[0], a, b[0], b[1]);
+        mma16816(s[1], a, b[2], b[3]);
       }
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
@@ -188,30 +198,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       uint32_t pa[4];
       acc_to_a(s, pa);  // R (rows i, k-dim j)
-      // B[j][c] = k_(kk,j)[c]: rows j = 2t, 2t+1 (+8), column c = nt*8 + g
-      const int j0 = min(2 * t, b2 - 1), j1 = min(2 * t + 1, b2 - 1);
-      const int j2 = min(2 * t + 8, b2 - 1), j3 = min(2 * t + 9, b2 - 1);
+      // B[j][c] = k_(kk,j)[c] (stored j-major): transposed ldmatrix, two 8-column tiles per load
+      const int jb = min(lr + (mi & 1) * 8, b2 - 1);
 #pragma unroll
-      for (int nt = 0; nt < kD / 8; ++nt) {
-        const int c = nt * 8 + g;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        mma16816(acc, pa, pack2(kr[j0 * kPB + c], kr[j1 * kPB + c]),
-                 pack2(kr[j2 * kPB + c], kr[j3 * kPB + c]));
-        const int cc = nt * 8 + 2 * t;
-        if (g < b2)
-          *reinterpret_cast<uint32_t*>(Kt + (g * b1 + kk) * kPB + cc) = tc::pack_bf16x2(acc[0], acc[1]);
-        if (g + 8 < b2)
-          *reinterpret_cast<uint32_t*>(Kt + ((g + 8) * b1 + kk) * kPB + cc) =
-              tc::pack_bf16x2(acc[2], acc[3]);
+      for (int cb = 0; cb < kD / 16; ++cb) {
+        const int coff = cb * 16 + (mi >> 1) * 8;
+        uint32_t b[4];
+        ldsm4_t(b, kr + jb * kPB + coff);
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        mma16816(acc[0], pa, b[0], b[1]);
+        mma16816(acc[1], pa, b[2], b[3]);
+        float ay[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
         if (last) {
-          float ay[4] = {0.f, 0.f, 0.f, 0.f};
-          mma16816(ay, pa, pack2(vr[j0 * kPB + c], vr[j1 * kPB + c]),
-                   pack2(vr[j2 * kPB + c], vr[j3 * kPB + c]));
-          if (g < b2)
-            *reinterpret_cast<uint32_t*>(Ys + (g * b1 + kk) * kPB + cc) = tc::pack_bf16x2(ay[0], ay[1]);
-          if (g + 8 < b2)
-            *reinterpret_cast<uint32_t*>(Ys + ((g + 8) * b1 + kk) * kPB + cc) =
-                tc::pack_bf16x2(ay[2], ay[3]);
+          ldsm4_t(b, vr + jb * kPB + coff);
+          mma16816(ay[0], pa, b[0], b[1]);
+          mma16816(ay[1], pa, b[2], b[3]);
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int cc = cb * 16 + h * 8 + 2 * t;
+          if (g < b2) {
+            *reinterpret_cast<uint32_t*>(Kt + (g * b1 + kk) * kPB + cc) =
+                tc::pack_bf16x2(acc[h][0], acc[h][1]);
+            if (last)
+              *reinterpret_cast<uint32_t*>(Ys + (g * b1 + kk) * kPB + cc) =
+                  tc::pack_bf16x2(ay[h][0], ay[h][1]);
+          }
+          if (g + 8 < b2) {
+            *reinterpret_cast<uint32_t*>(Kt + ((g + 8) * b1 + kk) * kPB + cc) =
+                tc::pack_bf16x2(acc[h][2], acc[h][3]);
+            if (last)
+              *reinterpret_cast<uint32_t*>(Ys + ((g + 8) * b1 + kk) * kPB + cc) =
+                  tc::pack_bf16x2(ay[h][2], ay[h][3]);
+          }
         }
       }
     }
@@ -219,20 +238,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- L-update: warp i, rows l, columns k ----
     if (warp < b2) {
       const int i = warp;
-      const int l0 = min(g, b1 - 1), l1 = min(g + 8, b1 - 1);
-      const bf16* qa = Qs + (l0 * b2 + i) * kPB;
-      const bf16* qb = Qs + (l1 * b2 + i) * kPB;
       const bf16* ktr = Kt + i * b1 * kPB;
+      // A rows l (query rows of position i, clamped), B rows k (Kt rows, clamped and masked)
+      const bf16* a_src = Qs + (min(lr + (mi & 1) * 8, b1 - 1) * b2 + i) * kPB + (mi >> 1) * 8;
+      const bf16* b_src = ktr + min(lr + (mi >> 1) * 8, b1 - 1) * kPB + (mi & 1) * 8;
       float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
       for (int ks = 0; ks < kD / 16; ++ks) {
-        const int c = ks * 16 + 2 * t;
-        const uint32_t a[4] = {ld32(qa + c), ld32(qb + c), ld32(qa + c + 8), ld32(qb + c + 8)};
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          const bf16* krow = ktr + min(nt * 8 + g, b1 - 1) * kPB;
-          mma16816(s[nt], a, ld32(krow + c), ld32(krow + c + 8));
-        }
+        uint32_t a[4], b[4];
+        ldsm4(a, a_src + ks * 16);
+        ldsm4(b, b_src + ks * 16);
+        mma16816(s[0], a, b[0], b[1]);
+        mma16816(s[1], a, b[2], b[3]);
       }
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
@@ -244,66 +261,70 @@ __global__ void __launch_bounds__(kThreads, 1)
       float ent[2];
       quad_softmax(s, b1, t, ent);
       if (!last) {
-        // L (rows l >= b1 zeroed) to this position's tile, then Qt = L^T q / colsum(L)
-        float* Lt = Ls + i * kMaxB * kMaxB;
+        // L (bf16; rows l >= b1 zeroed) to this position's tile, then
+        // Qt = L^T q / column sums of L
+        bf16* Lt = Ls + i * kMaxB * kPL;
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int row = g + 8 * (e >> 1), col = nt * 8 + 2 * t + (e & 1);
-            Lt[row * kMaxB + col] = row < b1 ? s[nt][e] : 0.f;
+          for (int h = 0; h < 2; ++h) {
+            const int row = g + 8 * h, col = nt * 8 + 2 * t;
+            *reinterpret_cast<uint32_t*>(Lt + row * kPL + col) =
+                row < b1 ? tc::pack_bf16x2(s[nt][2 * h], s[nt][2 * h + 1]) : 0u;
           }
         __syncwarp();
-        // A = L^T: rows k = g, g+8; k-dim l = 2t, 2t+1 (+8)
+        // A = L^T (rows k, k-dim l) from the l-major tile: transposed ldmatrix
         uint32_t a[4];
-        {
-          auto lk = [&](int l, int kk) { return __float2bfloat16_rn(Lt[l * kMaxB + kk]); };
-          a[0] = pack2(lk(2 * t, g), lk(2 * t + 1, g));
-          a[1] = pack2(lk(2 * t, g + 8), lk(2 * t + 1, g + 8));
-          a[2] = pack2(lk(2 * t + 8, g), lk(2 * t + 9, g));
-          a[3] = pack2(lk(2 * t + 8, g + 8), lk(2 * t + 9, g + 8));
-        }
-        float cs0 = 0.f, cs1 = 0.f;  // column sums for k = g, g + 8
+        ldsm4_t(a, Lt + (lr + (mi >> 1) * 8) * kPL + (mi & 1) * 8);
+        float cs0 = 0.f, cs1 = 0.f;  // column sums for k = g, g + 8 (of the bf16 weights)
         for (int l = 0; l < b1; ++l) {
-          cs0 += Lt[l * kMaxB + g];
-          cs1 += Lt[l * kMaxB + g + 8];
+          cs0 += __bfloat162float(Lt[l * kPL + g]);
+          cs1 += __bfloat162float(Lt[l * kPL + g + 8]);
         }
         const float inv0 = cs0 > 0.f ? 1.f / cs0 : 0.f, inv1 = cs1 > 0.f ? 1.f / cs1 : 0.f;
-        // B[l][c] = q_(l,i)[c]: rows l = 2t, 2t+1 (+8), column c = nt*8 + g
-        const int r0 = min(2 * t, b1 - 1) * b2 + i, r1 = min(2 * t + 1, b1 - 1) * b2 + i;
-        const int r2 = min(2 * t + 8, b1 - 1) * b2 + i, r3 = min(2 * t + 9, b1 - 1) * b2 + i;
+        // B[l][c] = q_(l,i)[c] (stored l-major): transposed ldmatrix; rows l >= b1 clamped
+        // (their A weights are 0)
+        const bf16* qb_src = Qs + (min(lr + (mi & 1) * 8, b1 - 1) * b2 + i) * kPB + (mi >> 1) * 8;
 #pragma unroll
-        for (int nt = 0; nt < kD / 8; ++nt) {
-          const int c = nt * 8 + g;
-          float acc[4] = {0.f, 0.f, 0.f, 0.f};
-          mma16816(acc, a, pack2(Qs[r0 * kPB + c], Qs[r1 * kPB + c]),
-                   pack2(Qs[r2 * kPB + c], Qs[r3 * kPB + c]));
-          const int cc = nt * 8 + 2 * t;
-          if (g < b1)
-            *reinterpret_cast<uint32_t*>(Qt + (g * b2 + i) * kPB + cc) =
-                tc::pack_bf16x2(acc[0] * inv0, acc[1] * inv0);
-          if (g + 8 < b1)
-            *reinterpret_cast<uint32_t*>(Qt + ((g + 8) * b2 + i) * kPB + cc) =
-                tc::pack_bf16x2(acc[2] * inv1, acc[3] * inv1);
+        for (int cb = 0; cb < kD / 16; ++cb) {
+          uint32_t b[4];
+          ldsm4_t(b, qb_src + cb * 16);
+          float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+          mma16816(acc[0], a, b[0], b[1]);
+          mma16816(acc[1], a, b[2], b[3]);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int cc = cb * 16 + h * 8 + 2 * t;
+            if (g < b1)
+              *reinterpret_cast<uint32_t*>(Qt + (g * b2 + i) * kPB + cc) =
+                  tc::pack_bf16x2(acc[h][0] * inv0, acc[h][1] * inv0);
+            if (g + 8 < b1)
+              *reinterpret_cast<uint32_t*>(Qt + ((g + 8) * b2 + i) * kPB + cc) =
+                  tc::pack_bf16x2(acc[h][2] * inv1, acc[h][3] * inv1);
+          }
         }
       } else {
-        // O_(l,i) = L Y_i: A = L (rows l, k-dim k), B[k][c] = Y_{i,k}[c]
+        // O_(l,i) = L Y_i: A = L (rows l, k-dim k), B[k][c] = Y_{i,k}[c] (stored
+        // k-major): transposed ldmatrix; rows k >= b1 clamped (their L weights are 0)
         uint32_t a[4];
         acc_to_a(s, a);
-        const bf16* yr = Ys + i * b1 * kPB;
-        const int k0 = min(2 * t, b1 - 1), k1 = min(2 * t + 1, b1 - 1);
-        const int k2 = min(2 * t + 8, b1 - 1), k3 = min(2 * t + 9, b1 - 1);
+        const bf16* y_src = Ys + (i * b1 + min(lr + (mi & 1) * 8, b1 - 1)) * kPB + (mi >> 1) * 8;
         bf16* orow0 = out + (gh * N + g * b2 + i) * kD;
         bf16* orow1 = out + (gh * N + (g + 8) * b2 + i) * kD;
 #pragma unroll
-        for (int nt = 0; nt < kD / 8; ++nt) {
-          const int c = nt * 8 + g;
-          float acc[4] = {0.f, 0.f, 0.f, 0.f};
-          mma16816(acc, a, pack2(yr[k0 * kPB + c], yr[k1 * kPB + c]),
-                   pack2(yr[k2 * kPB + c], yr[k3 * kPB + c]));
-          const int cc = nt * 8 + 2 * t;
-          if (g < b1) *reinterpret_cast<uint32_t*>(orow0 + cc) = tc::pack_bf16x2(acc[0], acc[1]);
-          if (g + 8 < b1) *reinterpret_cast<uint32_t*>(orow1 + cc) = tc::pack_bf16x2(acc[2], acc[3]);
+        for (int cb = 0; cb < kD / 16; ++cb) {
+          uint32_t b[4];
+          ldsm4_t(b, y_src + cb * 16);
+          float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+          mma16816(acc[0], a, b[0], b[1]);
+          mma16816(acc[1], a, b[2], b[3]);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int cc = cb * 16 + h * 8 + 2 * t;
+            if (g < b1) *reinterpret_cast<uint32_t*>(orow0 + cc) = tc::pack_bf16x2(acc[h][0], acc[h][1]);
+            if (g + 8 < b1)
+              *reinterpret_cast<uint32_t*>(orow1 + cc) = tc::pack_bf16x2(acc[h][2], acc[h][3]);
+          }
         }
       }
     }
