@@ -493,6 +493,8 @@ def run_native(args, wl):
         "cpu_baseline": cpu_baseline,
         "path_hbm_frac": (alg_bytes(wl) / (ms / args.steps / 1e3) / 1e9) / peaks["hbm_gbs"],
         "path_tensor_frac": (flops / (ms / args.steps / 1e3) / 1e12) / peaks["bf16_tflops"],
+        # dense softmax attention on the same shape: 4 N^2 d FLOPs per head
+        "dense_equiv_tflops": wl.heads * 4.0 * wl.N * wl.N * wl.d / (ms / args.steps / 1e3) / 1e12,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -71,7 +71,7 @@ extern "C" {
 #define MONARCH_ERR_UNSUPPORTED    -2
 #define MONARCH_ERR_CUDA           -3
 #define MONARCH_ERR_DEVICE_TIMEOUT -4
-#define MONARCH_ERR_NO_MEMORY      -5
+#define MONARCH_ERR_NO_MEMORY      -5  /* also forced by MONARCH_ATTN_FAIL_ALLOC=1 (see below) */
 #define MONARCH_ERR_SCRATCH_LIMIT  -6
 
 #define MONARCH_DTYPE_BF16 0
@@ -172,6 +172,12 @@ MONARCH_API int monarch_attn_fwd_video(int dtype, const void* q, const void* k, 
  * arguments).  dtype is MONARCH_DTYPE_BF16 or MONARCH_DTYPE_F32. */
 MONARCH_API size_t monarch_attn_workspace_bytes(int B, int H, int b1, int b2, int d, int T,
                                     int c1, int c2, int dtype);
+
+/* Fault injection for tests: while the environment variable
+ * MONARCH_ATTN_FAIL_ALLOC is "1", every device allocation the library would
+ * make for its workspace or staging buffers fails with
+ * MONARCH_ERR_NO_MEMORY before any device call (calls whose cached buffers
+ * are already large enough are unaffected). */
 
 /* Free the cached workspace and staging buffers of every device.  Must not
  * be called while a forward pass is still running on the GPU. */

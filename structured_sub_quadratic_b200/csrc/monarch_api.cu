@@ -9,6 +9,7 @@
 
 #include <atomic>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -146,10 +147,24 @@ int current_device(int* dev) {
   return MONARCH_OK;
 }
 
+// Host-side fault injection: with MONARCH_ATTN_FAIL_ALLOC=1 in the
+// environment every workspace or staging allocation the library attempts
+// fails as if cudaMalloc had run out of memory (no device call is made).
+bool alloc_failure_injected() {
+  const char* e = std::getenv("MONARCH_ATTN_FAIL_ALLOC");
+  return e != nullptr && e[0] == '1';
+}
+
 // Grow-only cached device buffer.  cudaFree synchronises the device, so a
 // buffer still used by an earlier call is never freed under it.
 int ensure(DevBuf& b, size_t bytes) {
   if (bytes <= b.bytes) return MONARCH_OK;
+  if (alloc_failure_injected()) {
+    std::snprintf(t_err, sizeof(t_err),
+                  "workspace allocation of %zu bytes failed (injected by MONARCH_ATTN_FAIL_ALLOC)",
+                  bytes);
+    return MONARCH_ERR_NO_MEMORY;
+  }
   if (b.ptr) {
     cudaError_t e = cudaFree(b.ptr);
     b.ptr = nullptr;

@@ -205,3 +205,20 @@ def test_video_layouts_on_the_480p_latent(cuda_lib, layout, T, c):
     cuda_lib.check()
     assert_parity(O.double().cpu().numpy(), layout_oracle(q, k, v, latent, layout, T, c, c), v,
                   torch.bfloat16)
+
+
+def test_injected_allocation_failure_is_reported_and_recovers(cuda_lib, monkeypatch):
+    """Host-side fault injection: with MONARCH_ATTN_FAIL_ALLOC=1 the workspace
+    allocation of a call fails with MONARCH_ERR_NO_MEMORY (no device call);
+    without it the next call allocates and runs."""
+    q, k, v = iid_qkv(1, 2, 64, 64, torch.bfloat16, seed=13)
+    qd, kd, vd = (x.cuda() for x in (q, k, v))
+    torch.cuda.synchronize()
+    cuda_lib.release_workspace()
+    monkeypatch.setenv("MONARCH_ATTN_FAIL_ALLOC", "1")
+    with pytest.raises(cuda_lib.MonarchError) as exc:
+        cuda_lib.monarch_attn_fwd(qd, kd, vd, 8, 8, 1)
+    assert exc.value.status == cuda_lib.MONARCH_ERR_NO_MEMORY
+    monkeypatch.delenv("MONARCH_ATTN_FAIL_ALLOC")
+    O = gpu_forward(cuda_lib, q, k, v, 8, 8, 1)
+    assert_parity(O, oracle_forward(q, k, v, 8, 8, 1), v, torch.bfloat16)
