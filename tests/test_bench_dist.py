@@ -64,3 +64,21 @@ def test_work_model_matches_the_flop_formula():
     assert bench.alg_bytes(wl) == 12 * 4 * 4680 * 128 * 2
     fl, by = bench.kernel_work("tc_l_output", wl)
     assert fl == 12 * 4680 * 90 * 128 * 4 and by > 0
+
+
+def test_reference_arm_times_the_oracle_on_the_host(capsys):
+    """bench.py --impl reference: the float64 oracle on the host cores, one JSON line."""
+    import json
+    assert bench.main(["--impl", "reference", "--workload", "tiny", "--steps", "1",
+                       "--warmup", "3"]) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+@pytest.mark.parametrize("argv", [["--workload", "vit", "--layout", "w,fh"],
+                                  ["--warmup", "2"]])
+def test_bench_rejects_invalid_options(argv):
+    with pytest.raises(SystemExit):
+        bench.main(argv)
