@@ -77,12 +77,6 @@ extern "C" {
 #define MONARCH_DTYPE_BF16 0
 #define MONARCH_DTYPE_F32  1
 
-/* Kernel path selection (process-wide): AUTO uses the tcgen05 tensor-core
- * kernels where the shape allows and the SIMT kernels elsewhere; SIMT forces
- * the SIMT kernels everywhere (used to cross-check the two). */
-#define MONARCH_PATH_AUTO 0
-#define MONARCH_PATH_SIMT 1
-
 /* Forward pass, bf16 in/out, fp32 accumulation.
  * q, k, v, out: device pointers to __nv_bfloat16, (B, H, N, d), N = b1*b2.
  * (Pages: MonarchAttention abstract and AI summary "Approach"; MonarchRT
@@ -114,23 +108,33 @@ MONARCH_API int monarch_attn_fwd_host(int dtype, const void* q_host, const void*
  * deadline) or a host framework that reserves all device memory for its own
  * pool and leaves a plugin no room for a cache of its own.
  *
- * Arguments, layout and result are those of monarch_attn_fwd, for the shapes
- * its tensor-core path takes (d = 64 or 128, T >= 1; any other shape returns
- * MONARCH_ERR_UNSUPPORTED).  The caller still passes q, k, v and out.
+ * Arguments, layout and result are those of monarch_attn_fwd, and it runs
+ * the same kernels, so the output is bit-identical to monarch_attn_fwd's on
+ * the same inputs.  Only the shapes those kernels take run here (d = 64 or
+ * 128, T >= 1, b2 <= 128 and column groups of <= 128 keys; small untiled
+ * heads with T >= 2 need no scratch at all); any other shape returns
+ * MONARCH_ERR_UNSUPPORTED.  The caller still passes q, k, v and out.
  *
  * Scratch: one static device array of 64 MiB (67108864 bytes) on every
  * device that loads this library, held until the process exits.  A shape
- * whose scratch (monarch_attn_workspace_bytes(..., MONARCH_DTYPE_BF16) on the
- * default path) exceeds it returns MONARCH_ERR_SCRATCH_LIMIT.  The first call
- * on a device looks up the array's device address and clears its status word
- * (a synchronous memset), so make that first call before any stream capture.
- * Every call on a device shares the array and leaves the last call's contents
- * in it; the kernels write each scratch entry before they read it.  Calls
- * that overlap on the GPU (other streams, or unordered host threads) race on
- * the array: order them on one stream.  No cudaMalloc, cudaFree or other
- * allocating routine is called.  A bounded device wait that expires (the
- * kernel stops early and out is invalid) is recorded in the array's own
- * status word, which this entry point does not report back. */
+ * whose scratch (monarch_attn_workspace_bytes(..., MONARCH_DTYPE_BF16))
+ * exceeds it returns MONARCH_ERR_SCRATCH_LIMIT (the 720p config does).
+ * CUDA loads device code lazily by default: the first call on a device
+ * looks up the array's device address, which loads it there and commits the
+ * 64 MiB, so make that first call at initialisation, while device memory is
+ * still free and before any stream capture.  Later calls of a shape that
+ * already ran on the device neither allocate nor change the device's free
+ * memory (the first call of another shape may make CUDA load the code of
+ * kernels not run before).  Every call on a device shares the
+ * array and leaves the last call's contents in it; the kernels write every
+ * scratch entry before they read it.  Calls that overlap on the GPU (other
+ * streams, or unordered host threads) race on the array: order them on one
+ * stream.  No cudaMalloc, cudaFree or other allocating routine is called.
+ *
+ * A bounded device wait that expires (the kernel stops early and out is
+ * invalid) sets the library's device status word, which is a static device
+ * variable too: monarch_attn_check() reports it as
+ * MONARCH_ERR_DEVICE_TIMEOUT and clears it. */
 MONARCH_API int monarch_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out,
                                          int B, int H, int b1, int b2, int d, int T, int c1,
                                          int c2, cudaStream_t stream);
@@ -184,15 +188,14 @@ MONARCH_API size_t monarch_attn_workspace_bytes(int B, int H, int b1, int b2, in
 MONARCH_API void monarch_attn_release_workspace(void);
 
 /* Synchronise `stream` and report a device-side failure (a bounded wait that
- * expired) recorded since the last check; clears the flag. */
+ * expired, in any entry point) recorded on the current device since the
+ * last check; clears the flag.  The flag is a static device variable: this
+ * call reads it with a 4-byte copy and allocates nothing. */
 MONARCH_API int monarch_attn_check(cudaStream_t stream);
 
 /* Human-readable text for a status code (includes the last CUDA error text
  * for MONARCH_ERR_CUDA). */
 MONARCH_API const char* monarch_attn_strerror(int status);
-
-/* Select MONARCH_PATH_AUTO or MONARCH_PATH_SIMT; returns the previous path. */
-MONARCH_API int monarch_attn_set_path(int path);
 
 /* Number of kernels the most recent forward call on this host thread
  * launched (for launch accounting in benchmarks). */

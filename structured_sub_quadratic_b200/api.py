@@ -23,8 +23,6 @@ MONARCH_ERR_NO_MEMORY = -5
 MONARCH_ERR_SCRATCH_LIMIT = -6
 DTYPE_BF16 = 0
 DTYPE_F32 = 1
-PATH_AUTO = 0
-PATH_SIMT = 1
 LAYOUTS = {"fh,w": 0, "w,fh": 1, "f,hw": 2, "hw,f": 3, "fw,h": 4, "h,fw": 5}
 
 # Every symbol the header declares, with its ctypes signature.
@@ -41,7 +39,6 @@ SIGNATURES = {
     "monarch_attn_release_workspace": (None, []),
     "monarch_attn_check": (_I, [_P]),
     "monarch_attn_strerror": (ctypes.c_char_p, [_I]),
-    "monarch_attn_set_path": (_I, [_I]),
     "monarch_attn_last_launches": (_I, []),
     "monarch_attn_version": (_I, []),
     "monarch_attn_selftest_timeout": (_I, [ctypes.c_ulonglong, _P]),
@@ -128,10 +125,13 @@ def monarch_attn_fwd_noalloc(q, k, v, b1, b2, T, c1=1, c2=1, out=None, stream=No
 
     For callers that cannot allocate when they call (a real-time frame loop
     that must not stall on cudaMalloc/cudaFree, or a host that reserves all
-    device memory for its own pool).  Scratch is a static 64 MiB device array
-    shared by all calls on a device; calls that overlap on the GPU race on
-    it, so keep them on one stream.  Pass ``out`` to avoid the one
-    allocation this wrapper would otherwise make through torch.
+    device memory for its own pool).  It runs the kernels of
+    ``monarch_attn_fwd`` and returns bit-identical results.  Scratch is a
+    static 64 MiB device array shared by all calls on a device, committed at
+    the first call on that device (make it at initialisation); calls that
+    overlap on the GPU race on it, so keep them on one stream.  Pass ``out``
+    to avoid the one allocation this wrapper would otherwise make through
+    torch.
     """
     lib = load_library()
     B, H, d = _dims(q, b1, b2)
@@ -208,10 +208,6 @@ def release_workspace():
 
 def check(stream=None):
     _check(load_library().monarch_attn_check(_stream_ptr(stream)))
-
-
-def set_path(path: int) -> int:
-    return load_library().monarch_attn_set_path(path)
 
 
 def last_launches() -> int:

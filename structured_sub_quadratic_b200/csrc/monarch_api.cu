@@ -7,17 +7,23 @@
 // else.  The video-layout entry point reorders tokens around a forward call.
 #include "monarch_attn.h"
 
-#include <atomic>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <vector>
 
+#include "entry.cuh"
 #include "layout.cuh"
 #include "simt_kernels.cuh"
 #include "small_head.cuh"
 #include "tc_path.cuh"
+
+// Status word of every entry point on a device: a bounded device wait that
+// expires sets it (no kernel traps).  A static device variable, so neither
+// entry point allocates for it; each device that loads the library holds
+// its own copy, zero at load time.
+static __device__ __align__(256) int g_status_word;
 
 namespace {
 
@@ -45,8 +51,7 @@ struct PermTable {
   int* dev_table;
 };
 std::vector<PermTable> g_tables[kMaxDevices];
-int* g_status[kMaxDevices];    // device status word (bounded-wait timeouts)
-std::atomic<int> g_path{MONARCH_PATH_AUTO};
+int* g_status[kMaxDevices];    // resolved address of g_status_word on each device
 thread_local int t_launches = 0;
 thread_local char t_err[256] = "";
 
@@ -63,33 +68,7 @@ bool mul_ok(size_t a, size_t b, size_t* out) {
   return true;
 }
 
-int validate(int B, int H, int b1, int b2, int d, int T, int c1, int c2) {
-  if (B < 1 || H < 1 || b1 < 1 || b2 < 1 || T < 0) return MONARCH_ERR_INVALID_ARG;
-  if (c1 < 1 || c1 > b1 || c2 < 1 || c2 > b2) return MONARCH_ERR_INVALID_ARG;
-  if (d < 1 || d > 256) return MONARCH_ERR_UNSUPPORTED;
-  size_t n;
-  if (!mul_ok((size_t)B, (size_t)H, &n) || !mul_ok(n, (size_t)b1, &n) ||
-      !mul_ok(n, (size_t)b2, &n) || !mul_ok(n, (size_t)d, &n) || !mul_ok(n, (size_t)c1, &n) ||
-      !mul_ok(n, (size_t)c2, &n) || n > ((size_t)1 << 40))
-    return MONARCH_ERR_INVALID_ARG;
-  if ((long long)B * H > (1LL << 30)) return MONARCH_ERR_INVALID_ARG;
-  return MONARCH_OK;
-}
-
 bool aligned16(const void* p) { return p != nullptr && ((uintptr_t)p & 15u) == 0; }
-
-Problem make_problem(int B, int H, int b1, int b2, int d, int T, int c1, int c2) {
-  Problem pb;
-  pb.G = B * H;
-  pb.b1 = b1;
-  pb.b2 = b2;
-  pb.d = d;
-  pb.T = T;
-  pb.c1 = c1;
-  pb.c2 = c2;
-  pb.sc = 1.0f / sqrtf((float)d);
-  return pb;
-}
 
 // Workspace of one call: none for the one-CTA-per-head kernel (small untiled
 // heads with T >= 2, whose later steps would otherwise run on the SIMT
@@ -104,16 +83,18 @@ struct Plan {
 
 Plan make_plan(const Problem& pb, int dtype) {
   Plan pl;
-  if (dtype == MONARCH_DTYPE_BF16 && g_path.load() == MONARCH_PATH_AUTO && pb.T >= 2 &&
-      monarch::small_head_supports(pb)) {
-    pl.small = true;
-    return pl;
-  }
-  if (dtype == MONARCH_DTYPE_BF16 && g_path.load() == MONARCH_PATH_AUTO &&
-      monarch::tc_supports(pb)) {
-    pl.tc = true;
-    pl.bytes = monarch::tc_workspace_bytes(pb);
-    return pl;
+  if (dtype == MONARCH_DTYPE_BF16) {
+    switch (monarch::choose_bf16_kernels(pb)) {
+      case monarch::Bf16Kernels::kSmallHead:
+        pl.small = true;
+        return pl;
+      case monarch::Bf16Kernels::kTensorCore:
+        pl.tc = true;
+        pl.bytes = monarch::tc_workspace_bytes(pb);
+        return pl;
+      case monarch::Bf16Kernels::kSimt:
+        break;
+    }
   }
   pl.simt = monarch::simt_workspace_sizes(pb);
   const size_t* f = &pl.simt.qt0;
@@ -183,17 +164,15 @@ int ensure(DevBuf& b, size_t bytes) {
   return MONARCH_OK;
 }
 
-int ensure_status(int dev) {
-  if (g_status[dev]) return MONARCH_OK;
-  int* p = nullptr;
-  cudaError_t e = cudaMalloc(&p, kAlign);
-  if (e != cudaSuccess) return record_cuda(e);
-  e = cudaMemset(p, 0, kAlign);
-  if (e != cudaSuccess) {
-    cudaFree(p);
-    return record_cuda(e);
+// Device address of g_status_word on `dev` (current), resolved once.  g_mu held.
+int status_word_locked(int dev, int** out) {
+  if (!g_status[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_status_word);
+    if (e != cudaSuccess) return record_cuda(e);
+    g_status[dev] = static_cast<int*>(p);
   }
-  g_status[dev] = p;
+  *out = g_status[dev];
   return MONARCH_OK;
 }
 
@@ -201,11 +180,11 @@ template <typename TIn>
 int forward_device(const TIn* q, const TIn* k, const TIn* v, TIn* out, int B, int H, int b1,
                    int b2, int d, int T, int c1, int c2, cudaStream_t stream, int dtype) {
   t_launches = 0;
-  int st = validate(B, H, b1, b2, d, T, c1, c2);
+  int st = monarch::validate_args(B, H, b1, b2, d, T, c1, c2);
   if (st != MONARCH_OK) return st;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
     return MONARCH_ERR_INVALID_ARG;
-  const Problem pb = make_problem(B, H, b1, b2, d, T, c1, c2);
+  const Problem pb = monarch::make_problem(B, H, b1, b2, d, T, c1, c2);
   const size_t bytes_io = (size_t)pb.G * b1 * b2 * d * sizeof(TIn);
   const char* o0 = reinterpret_cast<const char*>(out);
   for (const void* in : {(const void*)q, (const void*)k, (const void*)v}) {
@@ -216,7 +195,8 @@ int forward_device(const TIn* q, const TIn* k, const TIn* v, TIn* out, int B, in
   if ((st = current_device(&dev)) != MONARCH_OK) return st;
   const Plan pl = make_plan(pb, dtype);
   std::lock_guard<std::mutex> lock(g_mu);
-  if ((st = ensure_status(dev)) != MONARCH_OK) return st;
+  int* status = nullptr;
+  if ((st = status_word_locked(dev, &status)) != MONARCH_OK) return st;
   if ((st = ensure(g_ws[dev], pl.bytes ? pl.bytes : kAlign)) != MONARCH_OK) return st;
   cudaError_t e;
   if (pl.small) {
@@ -229,7 +209,7 @@ int forward_device(const TIn* q, const TIn* k, const TIn* v, TIn* out, int B, in
                             reinterpret_cast<const monarch::bf16*>(k),
                             reinterpret_cast<const monarch::bf16*>(v),
                             reinterpret_cast<monarch::bf16*>(out), pb,
-                            static_cast<char*>(g_ws[dev].ptr), g_status[dev], stream,
+                            static_cast<char*>(g_ws[dev].ptr), status, stream,
                             &t_launches);
   } else {
     const monarch::SimtWorkspace ws = carve_simt(pl, static_cast<char*>(g_ws[dev].ptr));
@@ -240,6 +220,50 @@ int forward_device(const TIn* q, const TIn* k, const TIn* v, TIn* out, int B, in
 }
 
 }  // namespace
+
+namespace monarch {
+
+int validate_args(int B, int H, int b1, int b2, int d, int T, int c1, int c2) {
+  if (B < 1 || H < 1 || b1 < 1 || b2 < 1 || T < 0) return MONARCH_ERR_INVALID_ARG;
+  if (c1 < 1 || c1 > b1 || c2 < 1 || c2 > b2) return MONARCH_ERR_INVALID_ARG;
+  if (d < 1 || d > 256) return MONARCH_ERR_UNSUPPORTED;
+  size_t n;
+  if (!mul_ok((size_t)B, (size_t)H, &n) || !mul_ok(n, (size_t)b1, &n) ||
+      !mul_ok(n, (size_t)b2, &n) || !mul_ok(n, (size_t)d, &n) || !mul_ok(n, (size_t)c1, &n) ||
+      !mul_ok(n, (size_t)c2, &n) || n > ((size_t)1 << 40))
+    return MONARCH_ERR_INVALID_ARG;
+  if ((long long)B * H > (1LL << 30)) return MONARCH_ERR_INVALID_ARG;
+  return MONARCH_OK;
+}
+
+Problem make_problem(int B, int H, int b1, int b2, int d, int T, int c1, int c2) {
+  Problem pb;
+  pb.G = B * H;
+  pb.b1 = b1;
+  pb.b2 = b2;
+  pb.d = d;
+  pb.T = T;
+  pb.c1 = c1;
+  pb.c2 = c2;
+  pb.sc = 1.0f / sqrtf((float)d);
+  return pb;
+}
+
+Bf16Kernels choose_bf16_kernels(const Problem& pb) {
+  // Small untiled heads with T >= 2 keep every step in one CTA (their later
+  // steps would otherwise run on the SIMT kernels).
+  if (pb.T >= 2 && small_head_supports(pb)) return Bf16Kernels::kSmallHead;
+  if (tc_supports(pb)) return Bf16Kernels::kTensorCore;
+  return Bf16Kernels::kSimt;
+}
+
+int device_status_word(int dev, int** out) {
+  if (dev < 0 || dev >= kMaxDevices) return MONARCH_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mu);
+  return status_word_locked(dev, out);
+}
+
+}  // namespace monarch
 
 extern "C" {
 
@@ -263,7 +287,7 @@ int monarch_attn_fwd_host(int dtype, const void* q_host, const void* k_host, con
                           int c2, cudaStream_t stream) {
   if (dtype != MONARCH_DTYPE_BF16 && dtype != MONARCH_DTYPE_F32) return MONARCH_ERR_INVALID_ARG;
   if (!q_host || !k_host || !v_host || !out_host) return MONARCH_ERR_INVALID_ARG;
-  int st = validate(B, H, b1, b2, d, T, c1, c2);
+  int st = monarch::validate_args(B, H, b1, b2, d, T, c1, c2);
   if (st != MONARCH_OK) return st;
   const size_t elt = dtype == MONARCH_DTYPE_BF16 ? 2 : 4;
   const size_t n = (size_t)B * H * b1 * b2 * d * elt;
@@ -318,7 +342,7 @@ int monarch_attn_fwd_video(int dtype, const void* q, const void* k, const void* 
     default: axes(h, w, f, hw, w, 1, h); break;  // MONARCH_LAYOUT_H_FW
   }
   const int N = (int)((long)f * hw), rows = (int)b1, cols = N / rows;
-  int st = validate(B, H, rows, cols, d, T, c1, c2);
+  int st = monarch::validate_args(B, H, rows, cols, d, T, c1, c2);
   if (st != MONARCH_OK) return st;
   auto fwd = [&](const void* a, const void* b, const void* c, void* o) {
     return dtype == MONARCH_DTYPE_BF16
@@ -377,9 +401,9 @@ int monarch_attn_fwd_video(int dtype, const void* q, const void* k, const void* 
 
 size_t monarch_attn_workspace_bytes(int B, int H, int b1, int b2, int d, int T, int c1, int c2,
                                     int dtype) {
-  if (validate(B, H, b1, b2, d, T, c1, c2) != MONARCH_OK) return 0;
+  if (monarch::validate_args(B, H, b1, b2, d, T, c1, c2) != MONARCH_OK) return 0;
   if (dtype != MONARCH_DTYPE_BF16 && dtype != MONARCH_DTYPE_F32) return 0;
-  return make_plan(make_problem(B, H, b1, b2, d, T, c1, c2), dtype).bytes;
+  return make_plan(monarch::make_problem(B, H, b1, b2, d, T, c1, c2), dtype).bytes;
 }
 
 void monarch_attn_release_workspace(void) {
@@ -389,8 +413,7 @@ void monarch_attn_release_workspace(void) {
   int cur = 0;
   cudaGetDevice(&cur);
   for (int dev = 0; dev < kMaxDevices; ++dev) {
-    if (!g_ws[dev].ptr && !g_stage[dev].ptr && !g_layout[dev].ptr && g_tables[dev].empty() &&
-        !g_status[dev])
+    if (!g_ws[dev].ptr && !g_stage[dev].ptr && !g_layout[dev].ptr && g_tables[dev].empty())
       continue;
     cudaSetDevice(dev);
     if (g_ws[dev].ptr) cudaFree(g_ws[dev].ptr);
@@ -398,11 +421,9 @@ void monarch_attn_release_workspace(void) {
     if (g_layout[dev].ptr) cudaFree(g_layout[dev].ptr);
     for (PermTable& t : g_tables[dev]) cudaFree(t.dev_table);
     g_tables[dev].clear();
-    if (g_status[dev]) cudaFree(g_status[dev]);
     g_ws[dev] = DevBuf();
     g_stage[dev] = DevBuf();
     g_layout[dev] = DevBuf();
-    g_status[dev] = nullptr;
   }
   cudaSetDevice(cur);
 }
@@ -416,9 +437,8 @@ int monarch_attn_check(cudaStream_t stream) {
   int* p;
   {
     std::lock_guard<std::mutex> lock(g_mu);
-    p = g_status[dev];
+    if ((st = status_word_locked(dev, &p)) != MONARCH_OK) return st;
   }
-  if (!p) return MONARCH_OK;
   int flag = 0;
   if ((e = cudaMemcpy(&flag, p, sizeof(int), cudaMemcpyDeviceToHost)) != cudaSuccess)
     return record_cuda(e);
@@ -447,11 +467,6 @@ const char* monarch_attn_strerror(int status) {
   }
 }
 
-int monarch_attn_set_path(int path) {
-  if (path != MONARCH_PATH_AUTO && path != MONARCH_PATH_SIMT) return -1;
-  return g_path.exchange(path);
-}
-
 int monarch_attn_last_launches(void) { return t_launches; }
 
 int monarch_attn_selftest_timeout(unsigned long long limit_ns, cudaStream_t stream) {
@@ -462,13 +477,12 @@ int monarch_attn_selftest_timeout(unsigned long long limit_ns, cudaStream_t stre
   int* status;
   {
     std::lock_guard<std::mutex> lock(g_mu);
-    if ((st = ensure_status(dev)) != MONARCH_OK) return st;
-    status = g_status[dev];
+    if ((st = status_word_locked(dev, &status)) != MONARCH_OK) return st;
   }
   cudaError_t e = monarch::tc_selftest_timeout(status, limit_ns, stream);
   return e == cudaSuccess ? MONARCH_OK : record_cuda(e);
 }
 
-int monarch_attn_version(void) { return (0 << 16) | 1; }
+int monarch_attn_version(void) { return (0 << 16) | 2; }
 
 }  // extern "C"

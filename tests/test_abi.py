@@ -37,13 +37,12 @@ def test_library_exports_every_declared_symbol(lib):
         assert getattr(lib, name) is not None
 
 
-def test_library_targets_sm100a_only():
-    out = subprocess.run(["cuobjdump", "--list-elf", _build.LIB_PATH], capture_output=True,
-                         text=True)
-    if out.returncode != 0:
-        pytest.skip("cuobjdump unavailable")
-    archs = set(re.findall(r"sm_(\d+a?)", out.stdout))
-    assert archs == {"100a"}
+def test_library_is_built_for_sm100a_only():
+    """The build compiles every source for sm_100a and nothing else."""
+    arch = _build.ARCH
+    assert arch == ["-gencode", "arch=compute_100a,code=sm_100a"]
+    flags = " ".join(_build.NVCC_FLAGS)
+    assert "-arch" not in flags and "-gencode" not in flags
 
 
 def test_version_and_strerror(lib):
@@ -86,12 +85,6 @@ def test_workspace_bytes_scale_with_shape(lib):
     assert 0 < w1 < w2 and w1 < w3
 
 
-def test_path_switch_round_trips(lib):
-    prev = lib.monarch_attn_set_path(api.PATH_SIMT)
-    assert lib.monarch_attn_set_path(prev) == api.PATH_SIMT
-    assert lib.monarch_attn_set_path(7) == -1
-
-
 @pytest.mark.parametrize("dtype,f,h,w,layout,expect", [
     (api.DTYPE_BF16, 2, 3, 4, 6, api.MONARCH_ERR_INVALID_ARG),    # unknown layout
     (api.DTYPE_BF16, 2, 3, 4, -1, api.MONARCH_ERR_INVALID_ARG),   # unknown layout
@@ -110,3 +103,18 @@ def test_video_blocks_of_each_layout():
     got = {name: api.video_blocks(f, h, w, name) for name in api.LAYOUTS}
     assert got == {"fh,w": (90, 52), "w,fh": (52, 90), "f,hw": (3, 1560), "hw,f": (1560, 3),
                    "fw,h": (156, 30), "h,fw": (30, 156)}
+
+
+@pytest.mark.parametrize("d,T,expect", [
+    (96, 1, api.MONARCH_ERR_UNSUPPORTED),     # d outside {64, 128}: checked before sizes
+    (0, 1, api.MONARCH_ERR_UNSUPPORTED),
+    (-5, 1, api.MONARCH_ERR_UNSUPPORTED),
+    (256, 1, api.MONARCH_ERR_UNSUPPORTED),
+    (64, -1, api.MONARCH_ERR_INVALID_ARG),
+])
+def test_noalloc_entry_validates_before_any_launch(lib, d, T, expect):
+    p = 1 << 20
+    assert lib.monarch_attn_fwd_noalloc(p, 2 * p, 3 * p, 4 * p, 1, 1, 4, 4, d, T, 1, 1,
+                                        None) == expect
+    assert lib.monarch_attn_fwd_noalloc(None, p, p, p, 1, 1, 4, 4, 64, 1, 1, 1, None) == \
+        api.MONARCH_ERR_INVALID_ARG

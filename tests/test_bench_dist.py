@@ -82,3 +82,25 @@ def test_reference_arm_times_the_oracle_on_the_host(capsys):
 def test_bench_rejects_invalid_options(argv):
     with pytest.raises(SystemExit):
         bench.main(argv)
+
+
+def test_roofline_uses_algorithmic_work_not_intermediates():
+    """The roofline of a kernel divides its share of the method's own work (Q/K/V/O
+    bytes, or its FLOPs) by its event time; Kt/Y intermediates are not counted."""
+    from structured_sub_quadratic_b200.inputs import WORKLOADS
+    peaks = {"hbm_gbs": 6458.1, "bf16_tflops": 1672.0, "bf16_tflops_sustained": 1408.0}
+    wl = WORKLOADS["480p"]
+    # R-update at 480p: K and V read once, 2 * 12 * 4680 * 128 * 2 bytes, HBM bound
+    r = bench.roofline_for("tc_r_update", 0.0230128, 1, wl, peaks, "measured", 29064192.0)
+    kv = 2 * 12 * 4680 * 128 * 2
+    assert r["bound"] == "hbm" and r["algorithmic_bytes"] == kv
+    assert r["frac"] == pytest.approx(kv / 23.0128e-6 / 1e9 / 6458.1)
+    assert r["frac"] == pytest.approx(0.1935, abs=1e-3)
+    assert r["traffic_over_algorithmic"] == pytest.approx(29064192.0 / kv)
+    # output kernel at 720p: 4 |p| b1 c2 d FLOPs per (g, i, p), tensor bound, sustained peak
+    wl = WORKLOADS["720p"]
+    r = bench.roofline_for("tc_l_output", 1.1126, 1, wl, peaks, "measured", None)
+    fl = 12 * 75600 * 945 * 2 * 128 * 4
+    assert r["bound"] == "tensor" and r["algorithmic_flops"] == fl
+    assert r["frac"] == pytest.approx(fl / 1.1126e-3 / 1e12 / 1408.0)
+    assert r["traffic_over_algorithmic"] is None
