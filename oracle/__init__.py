@@ -9,6 +9,7 @@ from .monarch_ref import (  # noqa: F401
     LFactor,
     RFactor,
     dense_logits,
+    group_valid,
     groups,
     materialise,
     monarch_attention,
@@ -17,4 +18,5 @@ from .monarch_ref import (  # noqa: F401
     output,
     r_update,
     l_update,
+    token_mask,
 )

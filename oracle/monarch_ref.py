@@ -74,6 +74,20 @@ MonarchAttention abstract: Theta(N sqrt(N) d) compute, Theta(N d) I/O):
 
     O_(l,i) = sum_{k,q} L_i[l,(k,q)] Y_{k,p(l),q,i},   Y_{k,p,q,i} = sum_{j in q} R_{k,p}[i,j] v_(k,j)
 
+Padding (OpenReview discussion, author response on choosing block sizes:
+m is the ceiling of N / b, and for ViT's N = 197 the pad tokens go before the
+class token): a sequence of N_real < b1 * b2 tokens is padded to b1 * b2,
+with the pad tokens before the real ones (pre-padding) or after them.  The
+pages do not say how pad tokens enter the softmaxes; the reading taken here
+keeps the objective over the real tokens only:
+  * a pad key gets zero R weight (R rows are softmaxes over the real keys of
+    each column group);
+  * a column group (k, q) with no real key gets zero L weight (L rows are
+    softmaxes over the pairs (k, q) that hold a real key);
+  * pad query rows are left out of the aggregated queries and of the
+    objective, and their outputs are dropped.
+With no pad tokens every mask is all true and nothing changes.
+
 Readings where the pages are silent:
   * L starts uniform, 1 / (b1 c2); R starts uniform inside every column group.
   * One step is an R-update followed by an L-update; T = 0 returns the
@@ -114,10 +128,35 @@ def _xlogx(p):
     return np.where(pos, p * np.log(np.where(pos, p, 1.0)), 0.0)
 
 
-def _softmax_last(s):
-    m = s.max(axis=-1, keepdims=True)
-    e = np.exp(s - m)
-    return e / e.sum(axis=-1, keepdims=True)
+def _masked_softmax_last(s, mask):
+    """softmax over the last axis restricted to mask (broadcast to s); entries
+    outside the mask are 0, and a row with no entry inside it is all 0."""
+    mask = np.broadcast_to(mask, s.shape)
+    sm = np.where(mask, s, -np.inf)
+    m = sm.max(axis=-1, keepdims=True)
+    m = np.where(np.isfinite(m), m, 0.0)
+    e = np.where(mask, np.exp(sm - m), 0.0)
+    z = e.sum(axis=-1, keepdims=True)
+    return np.where(z > 0, e / np.where(z > 0, z, 1.0), 0.0)
+
+
+def token_mask(b1: int, b2: int, n_pad: int = 0, pad_front: bool = True):
+    """(b1, b2) bool: True where token l*b2 + i is real.  The n_pad pad tokens
+    come first (pre-padding) or last."""
+    N = b1 * b2
+    if not (0 <= n_pad < N):
+        raise ValueError(f"need 0 <= n_pad < b1*b2, got {n_pad}")
+    m = np.zeros(N, dtype=bool)
+    if pad_front:
+        m[n_pad:] = True
+    else:
+        m[:N - n_pad] = True
+    return m.reshape(b1, b2)
+
+
+def group_valid(real, cols):
+    """(b1, c2) bool: column group q of chunk k holds at least one real key."""
+    return np.stack([real[:, j0:j1].any(axis=1) for j0, j1 in cols], axis=1)
 
 
 def as_heads(x, b1: int, b2: int):
@@ -136,17 +175,22 @@ class RFactor:
     """R_{k,p}[i,j] for all chunks k and row groups p, with its contractions.
 
     ``R`` has shape (G, b1[k], c1[p], b2[i], b2[j]); inside every column group
-    q the entries of a row sum to one.  From it:
+    q the entries of a row sum to one (all zero for a group with no real
+    key).  From it:
       Kt (G, b1[k], c1[p], c2[q], b2[i], d) = sum_{j in q} R k_(k,j)
       Y  (same)                             = sum_{j in q} R v_(k,j)
       Hs (G, b1[k], c1[p], c2[q], b2[i])    = entropy of R over j in q
+      valid (b1[k], c2[q])                  = group q of chunk k holds a real key
     """
 
-    def __init__(self, R, k, v, cols):
+    def __init__(self, R, k, v, cols, real=None):
         self.R = R
         G, b1, c1, b2, _ = R.shape
         c2 = len(cols)
         d, dv = k.shape[-1], v.shape[-1]
+        if real is None:
+            real = np.ones((b1, b2), dtype=bool)
+        self.valid = group_valid(real, cols)
         self.Kt = np.empty((G, b1, c1, c2, b2, d))
         self.Y = np.empty((G, b1, c1, c2, b2, dv))
         self.Hs = np.empty((G, b1, c1, c2, b2))
@@ -157,35 +201,48 @@ class RFactor:
             self.Hs[:, :, :, qi] = -_xlogx(Rq).sum(axis=-1)
 
     @classmethod
-    def uniform(cls, k, v, rows, cols):
+    def uniform(cls, k, v, rows, cols, real=None):
+        """R uniform over the real keys of every column group."""
         G, b1, b2, _ = k.shape
+        if real is None:
+            real = np.ones((b1, b2), dtype=bool)
         R = np.zeros((G, b1, len(rows), b2, b2))
         for j0, j1 in cols:
-            R[..., j0:j1] = 1.0 / (j1 - j0)
-        return cls(R, k, v, cols)
+            w = real[:, j0:j1].astype(np.float64)            # (k, j in q)
+            cnt = w.sum(axis=1, keepdims=True)
+            w = np.where(cnt > 0, w / np.where(cnt > 0, cnt, 1.0), 0.0)
+            R[..., j0:j1] = w[None, :, None, None, :]
+        return cls(R, k, v, cols, real)
 
 
 class LFactor:
     """L_i[l,(k,q)] for every position i, produced one block at a time.
 
     ``block(i)`` returns an array of shape (G, b1[l], b1[k], c2[q]) whose rows
-    sum to one over (k, q).  The factor is either uniform, an explicit array
-    of shape (G, b2[i], b1[l], b1[k], c2[q]), or the L-update of an RFactor.
+    sum to one over the valid pairs (k, q), those whose column group holds a
+    real key, and are zero on the others.  The factor is either uniform, an
+    explicit array of shape (G, b2[i], b1[l], b1[k], c2[q]), or the L-update
+    of an RFactor.
     """
 
-    def __init__(self, G, b1, b2, rows, cols, *, arr=None, q=None, rf=None, sc=None):
+    def __init__(self, G, b1, b2, rows, cols, *, arr=None, q=None, rf=None, sc=None,
+                 valid=None):
         self.G, self.b1, self.b2 = G, b1, b2
         self.rows, self.cols = rows, cols
         self.arr, self.q, self.rf, self.sc = arr, q, rf, sc
+        if valid is None:
+            valid = rf.valid if rf is not None else np.ones((b1, len(cols)), dtype=bool)
+        self.valid = valid
 
     @classmethod
-    def uniform(cls, G, b1, b2, rows, cols):
-        return cls(G, b1, b2, rows, cols)
+    def uniform(cls, G, b1, b2, rows, cols, valid=None):
+        """L uniform over the valid pairs (k, q)."""
+        return cls(G, b1, b2, rows, cols, valid=valid)
 
     @classmethod
-    def explicit(cls, arr, rows, cols):
+    def explicit(cls, arr, rows, cols, valid=None):
         G, b2, b1, _, _ = arr.shape
-        return cls(G, b1, b2, rows, cols, arr=arr)
+        return cls(G, b1, b2, rows, cols, arr=arr, valid=valid)
 
     def logits(self, i):
         """sc q_(l,i).Kt_{k,p(l),q,i} + Hs_{k,p(l),q,i}, shape (G, l, k, q)."""
@@ -204,10 +261,11 @@ class LFactor:
         if self.arr is not None:
             return self.arr[:, i]
         if self.rf is None:
-            return np.full((self.G, self.b1, self.b1, c2), 1.0 / (self.b1 * c2))
+            w = self.valid / self.valid.sum()
+            return np.broadcast_to(w, (self.G, self.b1, self.b1, c2)).copy()
         s = self.logits(i)
         flat = s.reshape(self.G, self.b1, self.b1 * c2)
-        return _softmax_last(flat).reshape(s.shape)
+        return _masked_softmax_last(flat, self.valid.reshape(-1)).reshape(s.shape)
 
     def materialise(self):
         return np.stack([self.block(i) for i in range(self.b2)], axis=1)
@@ -216,15 +274,20 @@ class LFactor:
 # ----------------------------------------------------------------------------
 # the steps
 # ----------------------------------------------------------------------------
-def r_update(q, k, v, L: LFactor, rows, cols, sc) -> RFactor:
-    """Exact maximiser of f over R with L fixed (a softmax per (k, p, q, i))."""
+def r_update(q, k, v, L: LFactor, rows, cols, sc, real=None) -> RFactor:
+    """Exact maximiser of f over R with L fixed (a softmax per (k, p, q, i)).
+
+    ``real`` (b1, b2) marks the real tokens: pad rows l are left out of the
+    aggregated queries and pad keys get zero weight."""
     G, b1, b2, d = q.shape
     c1, c2 = len(rows), len(cols)
+    if real is None:
+        real = np.ones((b1, b2), dtype=bool)
     Qt = np.zeros((G, b1, c1, c2, b2, d))                    # [k, p, q, i]
     for i in range(b2):
         Lb = L.block(i)                                      # (G, l, k, q)
         for pi, (l0, l1) in enumerate(rows):
-            Lp = Lb[:, l0:l1]
+            Lp = Lb[:, l0:l1] * real[l0:l1, i][None, :, None, None]
             c = Lp.sum(axis=1)                               # (G, k, q)
             num = np.einsum("glkq,gld->gkqd", Lp, q[:, l0:l1, i], optimize=True)
             safe = np.where(c > 0, c, 1.0)
@@ -233,8 +296,8 @@ def r_update(q, k, v, L: LFactor, rows, cols, sc) -> RFactor:
     for pi in range(c1):
         for qi, (j0, j1) in enumerate(cols):
             s = sc * (Qt[:, :, pi, qi] @ np.swapaxes(k[:, :, j0:j1], -1, -2))  # (G, k, i, j)
-            R[:, :, pi, :, j0:j1] = _softmax_last(s)
-    return RFactor(R, k, v, cols)
+            R[:, :, pi, :, j0:j1] = _masked_softmax_last(s, real[None, :, None, j0:j1])
+    return RFactor(R, k, v, cols, real)
 
 
 def l_update(q, rf: RFactor, rows, cols, sc) -> LFactor:
@@ -256,9 +319,11 @@ def output(L: LFactor, rf: RFactor, rows):
     return O
 
 
-def objective(q, L: LFactor, rf: RFactor, rows, sc):
-    """f(M) of the factored Monarch matrix, per head (shape (G,))."""
+def objective(q, L: LFactor, rf: RFactor, rows, sc, real=None):
+    """f(M) of the factored Monarch matrix over the real rows, per head (shape (G,))."""
     G = q.shape[0]
+    if real is None:
+        real = np.ones(q.shape[1:3], dtype=bool)
     f = np.zeros(G)
     for i in range(q.shape[2]):
         Lb = L.block(i)
@@ -268,7 +333,8 @@ def objective(q, L: LFactor, rf: RFactor, rows, sc):
             lin = sc * (q[:, l0:l1, i] @ np.swapaxes(Kt, -1, -2)) \
                 + rf.Hs[:, :, pi, :, i].reshape(G, 1, nk)
             Lp = Lb[:, l0:l1].reshape(G, l1 - l0, nk)
-            f += (Lp * lin).sum(axis=(1, 2)) - _xlogx(Lp).sum(axis=(1, 2))
+            rw = real[l0:l1, i][None, :, None]
+            f += (rw * (Lp * lin - _xlogx(Lp))).sum(axis=(1, 2))
     return f
 
 
@@ -301,27 +367,41 @@ def objective_dense(M, S):
 # ----------------------------------------------------------------------------
 # the forward pass
 # ----------------------------------------------------------------------------
-def monarch_attention(q, k, v, b1, b2, T, c1=1, c2=1, return_state=False):
+def monarch_attention(q, k, v, b1, b2, T, c1=1, c2=1, return_state=False, n_pad=0,
+                      pad_front=True):
     """MonarchAttention forward: T alternating steps, then O = M V.
 
-    q, k, v: arrays (..., N, d) with N = b1*b2 (any float dtype; read as
-    float64).  Returns O (..., N, d) in float64; with ``return_state`` also
-    the final (L, R) factors and the head-major inputs.
+    q, k, v: arrays (..., N_real, d) with N_real = b1*b2 - n_pad (any float
+    dtype; read as float64).  The n_pad pad tokens are placed before the real
+    tokens (``pad_front``) or after them.  Returns O (..., N_real, d) in
+    float64, the real tokens' rows; with ``return_state`` also the final
+    (L, R) factors, the head-major padded inputs and the real-token mask.
     """
-    qh, lead = as_heads(q, b1, b2)
-    kh, _ = as_heads(k, b1, b2)
-    vh, _ = as_heads(v, b1, b2)
+    real = token_mask(b1, b2, n_pad, pad_front)
+    qa, ka, va = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
+    *lead, n_in, d = qa.shape
+    if n_in != b1 * b2 - n_pad:
+        raise ValueError(f"N={n_in} != b1*b2 - n_pad = {b1 * b2 - n_pad}")
     if T < 0:
         raise ValueError("T must be >= 0")
-    G, _, _, d = qh.shape
+
+    def padded(x):
+        x = x.reshape(-1, n_in, x.shape[-1])
+        out = np.zeros((x.shape[0], b1 * b2, x.shape[-1]))
+        out[:, real.reshape(-1)] = x
+        return out.reshape(-1, b1, b2, x.shape[-1])
+
+    qh, kh, vh = padded(qa), padded(ka), padded(va)
+    G = qh.shape[0]
     sc = 1.0 / np.sqrt(d)
     rows, cols = groups(b1, c1), groups(b2, c2)
-    L = LFactor.uniform(G, b1, b2, rows, cols)
-    rf = RFactor.uniform(kh, vh, rows, cols)
+    L = LFactor.uniform(G, b1, b2, rows, cols, valid=group_valid(real, cols))
+    rf = RFactor.uniform(kh, vh, rows, cols, real)
     for _ in range(T):
-        rf = r_update(qh, kh, vh, L, rows, cols, sc)
+        rf = r_update(qh, kh, vh, L, rows, cols, sc, real)
         L = l_update(qh, rf, rows, cols, sc)
-    O = output(L, rf, rows).reshape(*lead, b1 * b2, vh.shape[-1])
+    O = output(L, rf, rows).reshape(G, b1 * b2, vh.shape[-1])[:, real.reshape(-1)]
+    O = O.reshape(*lead, n_in, vh.shape[-1])
     if return_state:
-        return O, dict(L=L, R=rf, q=qh, k=kh, v=vh, rows=rows, cols=cols, sc=sc)
+        return O, dict(L=L, R=rf, q=qh, k=kh, v=vh, rows=rows, cols=cols, sc=sc, real=real)
     return O

@@ -821,7 +821,7 @@ __global__ void __launch_bounds__(192, 2)
 // ---------------------------------------------------------------------------
 // Step-one aggregated queries under the uniform initial L (bf16):
 // Qt0[g][p][i][:] = mean_{l in p} q_(l,i).  One block per (g, p, i): 16-byte
-// column chunks x row lanes, every row load of a thread in flight at once;
+// column chunks x row lanes, up to eight row loads of a thread in flight at once;
 // the row lanes are summed in a fixed order (warp shuffles, then the 8 warps
 // through shared memory).  Launched with programmatic stream serialisation:
 // its blocks may be scheduled while the previous kernel of the stream
@@ -850,14 +850,24 @@ __global__ void __launch_bounds__(256)
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
   const uint4* base = reinterpret_cast<const uint4*>(q + (g * b1 * b2 + i) * D) + ch;
   const long row_stride = (long)b2 * D / 8;  // in uint4
-#pragma unroll 8
-  for (int l = l0 + rl; l < l1; l += RL) {
-    const uint4 u = __ldg(base + l * row_stride);
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  // Rounds of U predicated loads, all issued before any is summed, so a
+  // short group (a few rows per lane) still has every load in flight.
+  constexpr int U = 8;
+  for (int l = l0 + rl; l < l1; l += U * RL) {
+    uint4 u[U];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      acc[2 * e] += __uint_as_float(w[e] << 16);
-      acc[2 * e + 1] += __uint_as_float(w[e] & 0xffff0000u);
+    for (int t = 0; t < U; ++t) {
+      const int lt = l + t * RL;
+      u[t] = lt < l1 ? __ldg(base + lt * row_stride) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int t = 0; t < U; ++t) {
+      const uint32_t w[4] = {u[t].x, u[t].y, u[t].z, u[t].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        acc[2 * e] += __uint_as_float(w[e] << 16);
+        acc[2 * e + 1] += __uint_as_float(w[e] & 0xffff0000u);
+      }
     }
   }
 #pragma unroll
