@@ -172,6 +172,30 @@ MONARCH_API int monarch_attn_fwd_video(int dtype, const void* q, const void* k, 
                                        void* out, int B, int H, int f, int h, int w, int layout,
                                        int d, int T, int c1, int c2, cudaStream_t stream);
 
+/* Forward pass on n_real <= b1*b2 tokens per head, padded to the b1*b2
+ * grid (MonarchAttention OpenReview discussion, author response on choosing
+ * block sizes: the chunk count is the ceiling of N over the block size, and
+ * ViT's 197 tokens are pre-padded).  The n_pad = b1*b2 - n_real pad tokens
+ * sit before the real ones (pad_front = 1, pre-padding) or after them
+ * (pad_front = 0).  The objective is taken over the real tokens only: pad
+ * keys get zero R weight, a column group without a real key zero L weight,
+ * and pad query rows are left out of the aggregations.
+ *
+ * dtype: MONARCH_DTYPE_BF16 (__nv_bfloat16) or MONARCH_DTYPE_F32.
+ * q, k, v, out: device pointers, (B, H, n_real, d) contiguous, real tokens
+ * only.  Small untiled bf16 heads (b1, b2 <= 16, d = 64, T >= 2) run in
+ * place; other shapes copy q, k, v into a cached device buffer of
+ * 4*B*H*b1*b2*d elements in grid order (allocated on first use, grown on
+ * demand, freed by monarch_attn_release_workspace), run the masked forward
+ * pass there and copy the real output rows back.  n_real = b1*b2 is
+ * monarch_attn_fwd / _f32.  Asynchronous on `stream`.  Errors as for
+ * monarch_attn_fwd, plus MONARCH_ERR_INVALID_ARG for n_real outside
+ * [1, b1*b2], pad_front not 0 or 1, or an unknown dtype. */
+MONARCH_API int monarch_attn_fwd_padded(int dtype, const void* q, const void* k, const void* v,
+                                        void* out, int B, int H, int n_real, int b1, int b2,
+                                        int pad_front, int d, int T, int c1, int c2,
+                                        cudaStream_t stream);
+
 /* Bytes of device workspace a call with these arguments uses (0 on invalid
  * arguments).  dtype is MONARCH_DTYPE_BF16 or MONARCH_DTYPE_F32. */
 MONARCH_API size_t monarch_attn_workspace_bytes(int B, int H, int b1, int b2, int d, int T,

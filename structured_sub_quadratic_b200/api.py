@@ -35,6 +35,8 @@ SIGNATURES = {
     "monarch_attn_fwd_noalloc": (_I, [_P, _P, _P, _P, *_SIZES, _P]),
     "monarch_attn_fwd_video": (_I, [_I, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I,
                                     _I, _P]),
+    "monarch_attn_fwd_padded": (_I, [_I, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I,
+                                     _I, _P]),
     "monarch_attn_workspace_bytes": (_Z, [*_SIZES, _I]),
     "monarch_attn_release_workspace": (None, []),
     "monarch_attn_check": (_I, [_P]),
@@ -144,6 +146,30 @@ def monarch_attn_fwd_noalloc(q, k, v, b1, b2, T, c1=1, c2=1, out=None, stream=No
     _check(lib.monarch_attn_fwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(),
                                         out.data_ptr(), B, H, b1, b2, d, T, c1, c2,
                                         _stream_ptr(stream)))
+    return out
+
+
+def monarch_attn_fwd_padded(q, k, v, b1, b2, T, c1=1, c2=1, pad_front=True, out=None,
+                            stream=None):
+    """Forward pass on (B, H, n_real, d) tensors with n_real <= b1*b2: the
+    sequence is padded to the b1*b2 grid with the pad tokens before the real
+    ones (``pad_front``, pre-padding) or after them; the objective covers the
+    real tokens only.  Returns ``out`` (B, H, n_real, d)."""
+    lib = load_library()
+    if q.dim() != 4:
+        raise ValueError("expected (B, H, n_real, d) tensors")
+    B, H, n_real, d = q.shape
+    for t in (q, k, v):
+        if t.shape != q.shape or t.dtype != q.dtype or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous CUDA tensors of one shape and dtype")
+    dtype = {torch.bfloat16: DTYPE_BF16, torch.float32: DTYPE_F32}.get(q.dtype)
+    if dtype is None:
+        raise ValueError(f"unsupported dtype {q.dtype}")
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib.monarch_attn_fwd_padded(dtype, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                       out.data_ptr(), B, H, n_real, b1, b2,
+                                       1 if pad_front else 0, d, T, c1, c2, _stream_ptr(stream)))
     return out
 
 

@@ -14,11 +14,36 @@ typedef __nv_bfloat16 bf16;
 // Token n = l*b2 + i.  Row groups p of l in [b1] (c1 of them) and column
 // groups q of j in [b2] (c2 of them) are contiguous, sizes differing by at
 // most one with the larger groups first.
+//
+// Padding: a sequence of fewer than b1*b2 tokens sits on the b1*b2 grid with
+// its real tokens at [real_lo, real_hi) (pad tokens before and/or after).
+// Pad keys get zero R weight, a column group with no real key zero L
+// weight (its entropy bias is -inf), and pad query rows are left out of the
+// aggregations; unpadded problems have real_lo = 0, real_hi = b1*b2.
 // ---------------------------------------------------------------------------
 struct Problem {
   int G, b1, b2, d, T, c1, c2;
   float sc;  // 1/sqrt(d)
+  int real_lo, real_hi;
 };
+
+__host__ __device__ __forceinline__ bool is_real(const Problem& pb, long m) {
+  return m >= pb.real_lo && m < pb.real_hi;
+}
+
+__host__ __device__ __forceinline__ bool is_padded(const Problem& pb) {
+  return pb.real_lo != 0 || pb.real_hi != pb.b1 * pb.b2;
+}
+
+// The rows l in [l0, l1) whose token l*b2 + i is real: [*lr0, *lr1).
+__host__ __device__ __forceinline__ void real_rows(const Problem& pb, int i, int l0, int l1,
+                                                   int* lr0, int* lr1) {
+  const int a = pb.real_lo > i ? (pb.real_lo - i + pb.b2 - 1) / pb.b2 : 0;
+  const int b = pb.real_hi > i ? (pb.real_hi - i + pb.b2 - 1) / pb.b2 : 0;
+  *lr0 = a > l0 ? a : l0;
+  *lr1 = b < l1 ? b : l1;
+  if (*lr1 < *lr0) *lr1 = *lr0;
+}
 
 __host__ __device__ __forceinline__ int group_start(int n, int c, int g) {
   const int base = n / c, extra = n % c;

@@ -55,6 +55,51 @@ cudaError_t launch(const RowPairs& pairs, int npairs, const int* table, long G, 
   });
 }
 
+// Padding copies: one thread per unit of a destination row.
+template <typename U>
+__global__ void __launch_bounds__(256)
+    pad_rows_kernel(RowPairs pairs, long total, int rows_dst, int N, int n_src, int real_lo,
+                    int units, bool to_grid) {
+  const U* __restrict__ src = static_cast<const U*>(pairs.src[blockIdx.y]);
+  U* __restrict__ dst = static_cast<U*>(pairs.dst[blockIdx.y]);
+  for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (long)gridDim.x * blockDim.x) {
+    const long row = idx / units;
+    const int c = (int)(idx - row * units);
+    const long g = row / rows_dst;
+    const int r = (int)(row - g * rows_dst);
+    if (to_grid) {  // r is a grid row
+      const int rs = r - real_lo;
+      U val;
+      if (rs >= 0 && rs < n_src) {
+        val = src[(g * n_src + rs) * units + c];
+      } else {
+        memset(&val, 0, sizeof(U));
+      }
+      dst[idx] = val;
+    } else {  // r is a real row
+      dst[idx] = src[(g * N + r + real_lo) * units + c];
+    }
+  }
+}
+
+template <typename U>
+cudaError_t launch_pad(const RowPairs& pairs, int npairs, long G, int N, int n_src, int real_lo,
+                       int row_bytes, bool to_grid, cudaStream_t stream, int* launches) {
+  const int units = row_bytes / (int)sizeof(U);
+  const int rows_dst = to_grid ? N : n_src;
+  const long total = G * rows_dst * (long)units;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long want = (total + 255) / 256;
+  const int grid = (int)(want < 16L * sms ? want : 16L * sms);
+  return timed_launch("pad_rows", stream, launches, [&] {
+    pad_rows_kernel<U><<<dim3(grid, npairs), 256, 0, stream>>>(pairs, total, rows_dst, N, n_src,
+                                                               real_lo, units, to_grid);
+  });
+}
+
 }  // namespace
 
 void video_perm_table(const VideoPerm& vp, int* table) {
@@ -91,6 +136,29 @@ cudaError_t permute_rows(const void* const* src, void* const* dst, int n, const 
   if (a % 2 == 0) MONARCH_PERMUTE(uint16_t, 0);
   MONARCH_PERMUTE(uint8_t, 0);
 #undef MONARCH_PERMUTE
+}
+
+cudaError_t pad_rows(const void* const* src, void* const* dst, int n, long G, int N, int n_src,
+                     int real_lo, int row_bytes, bool to_grid, cudaStream_t stream,
+                     int* launches) {
+  if (n < 1 || n > 3 || G < 1 || N < 1 || n_src < 1 || real_lo < 0 || real_lo + n_src > N ||
+      row_bytes < 1)
+    return cudaErrorInvalidValue;
+  RowPairs pairs = {};
+  uintptr_t a = static_cast<uintptr_t>(row_bytes);
+  for (int i = 0; i < n; ++i) {
+    pairs.src[i] = src[i];
+    pairs.dst[i] = dst[i];
+    a |= reinterpret_cast<uintptr_t>(src[i]) | reinterpret_cast<uintptr_t>(dst[i]);
+  }
+#define MONARCH_PAD(U) \
+  return launch_pad<U>(pairs, n, G, N, n_src, real_lo, row_bytes, to_grid, stream, launches)
+  if (a % 16 == 0) MONARCH_PAD(uint4);
+  if (a % 8 == 0) MONARCH_PAD(uint2);
+  if (a % 4 == 0) MONARCH_PAD(uint32_t);
+  if (a % 2 == 0) MONARCH_PAD(uint16_t);
+  MONARCH_PAD(uint8_t);
+#undef MONARCH_PAD
 }
 
 }  // namespace monarch

@@ -28,4 +28,14 @@ cudaError_t permute_rows(const void* const* src, void* const* dst, int n, const 
                          long G, int N, int row_bytes, bool to_monarch, cudaStream_t stream,
                          int* launches);
 
+// Padding: for each of the n (1-3) tensor pairs, in one launch.  to_grid:
+// dst holds G blocks of N rows and src G blocks of n_src rows; dst row m of
+// a block = src row m - real_lo of the same block when that is in
+// [0, n_src), zeros otherwise.  !to_grid: the reverse, dst (n_src rows per
+// block) row r = src (N rows per block) row r + real_lo.  Rows move in the
+// widest unit that divides row_bytes and every base address.
+cudaError_t pad_rows(const void* const* src, void* const* dst, int n, long G, int N, int n_src,
+                     int real_lo, int row_bytes, bool to_grid, cudaStream_t stream,
+                     int* launches);
+
 }  // namespace monarch

@@ -40,9 +40,11 @@ struct DevBuf {
 std::mutex g_mu;                // workspace and status words
 std::mutex g_stage_mu;          // held for a whole host-buffer call
 std::mutex g_layout_mu;         // held for a whole video-layout call
+std::mutex g_pad_mu;            // held for a whole padded call
 DevBuf g_ws[kMaxDevices];      // kernel workspace
 DevBuf g_stage[kMaxDevices];   // staging for the host-buffer entry point
 DevBuf g_layout[kMaxDevices];  // reordered q, k, v and output of the video-layout entry point
+DevBuf g_pad[kMaxDevices];     // padded q, k, v and output of the padded entry point
 
 // Raster index tables of the video layouts used so far, per device (uploaded
 // once per (f, h, w, layout); guarded by g_layout_mu).
@@ -176,15 +178,22 @@ int status_word_locked(int dev, int** out) {
   return MONARCH_OK;
 }
 
+// real_lo, real_hi: the real tokens of the b1*b2 grid (padding; the default
+// is every token).  q, k, v, out always hold whole grids here.
 template <typename TIn>
 int forward_device(const TIn* q, const TIn* k, const TIn* v, TIn* out, int B, int H, int b1,
-                   int b2, int d, int T, int c1, int c2, cudaStream_t stream, int dtype) {
+                   int b2, int d, int T, int c1, int c2, cudaStream_t stream, int dtype,
+                   int real_lo = 0, int real_hi = -1) {
   t_launches = 0;
   int st = monarch::validate_args(B, H, b1, b2, d, T, c1, c2);
   if (st != MONARCH_OK) return st;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
     return MONARCH_ERR_INVALID_ARG;
-  const Problem pb = monarch::make_problem(B, H, b1, b2, d, T, c1, c2);
+  Problem pb = monarch::make_problem(B, H, b1, b2, d, T, c1, c2);
+  if (real_hi >= 0) {
+    pb.real_lo = real_lo;
+    pb.real_hi = real_hi;
+  }
   const size_t bytes_io = (size_t)pb.G * b1 * b2 * d * sizeof(TIn);
   const char* o0 = reinterpret_cast<const char*>(out);
   for (const void* in : {(const void*)q, (const void*)k, (const void*)v}) {
@@ -246,6 +255,8 @@ Problem make_problem(int B, int H, int b1, int b2, int d, int T, int c1, int c2)
   pb.c1 = c1;
   pb.c2 = c2;
   pb.sc = 1.0f / sqrtf((float)d);
+  pb.real_lo = 0;
+  pb.real_hi = b1 * b2;
   return pb;
 }
 
@@ -399,6 +410,83 @@ int monarch_attn_fwd_video(int dtype, const void* q, const void* k, const void* 
   return MONARCH_OK;
 }
 
+int monarch_attn_fwd_padded(int dtype, const void* q, const void* k, const void* v, void* out,
+                            int B, int H, int n_real, int b1, int b2, int pad_front, int d, int T,
+                            int c1, int c2, cudaStream_t stream) {
+  t_launches = 0;
+  if (dtype != MONARCH_DTYPE_BF16 && dtype != MONARCH_DTYPE_F32) return MONARCH_ERR_INVALID_ARG;
+  if (pad_front != 0 && pad_front != 1) return MONARCH_ERR_INVALID_ARG;
+  int st = monarch::validate_args(B, H, b1, b2, d, T, c1, c2);
+  if (st != MONARCH_OK) return st;
+  const int N = b1 * b2;
+  if (n_real < 1 || n_real > N) return MONARCH_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return MONARCH_ERR_INVALID_ARG;
+  using monarch::bf16;
+  if (n_real == N)
+    return dtype == MONARCH_DTYPE_BF16
+               ? monarch_attn_fwd(q, k, v, out, B, H, b1, b2, d, T, c1, c2, stream)
+               : monarch_attn_fwd_f32(static_cast<const float*>(q), static_cast<const float*>(k),
+                                      static_cast<const float*>(v), static_cast<float*>(out), B,
+                                      H, b1, b2, d, T, c1, c2, stream);
+  const int real_lo = pad_front ? N - n_real : 0;
+  Problem pb = monarch::make_problem(B, H, b1, b2, d, T, c1, c2);
+  pb.real_lo = real_lo;
+  pb.real_hi = real_lo + n_real;
+  const int row_bytes = d * (dtype == MONARCH_DTYPE_BF16 ? 2 : 4);
+  const size_t bytes_io = (size_t)pb.G * n_real * row_bytes;
+  const char* o0 = static_cast<const char*>(out);
+  for (const void* in : {q, k, v}) {
+    const char* i0 = static_cast<const char*>(in);
+    if (o0 < i0 + bytes_io && i0 < o0 + bytes_io) return MONARCH_ERR_INVALID_ARG;
+  }
+  int dev;
+  if ((st = current_device(&dev)) != MONARCH_OK) return st;
+  if (dtype == MONARCH_DTYPE_BF16 &&
+      monarch::choose_bf16_kernels(pb) == monarch::Bf16Kernels::kSmallHead) {
+    // small heads: the kernel reads and writes the real rows in place
+    const cudaError_t e = monarch::small_head_forward(
+        static_cast<const bf16*>(q), static_cast<const bf16*>(k), static_cast<const bf16*>(v),
+        static_cast<bf16*>(out), pb, stream, &t_launches);
+    return e == cudaSuccess ? MONARCH_OK : record_cuda(e);
+  }
+  // every other kernel works on whole grids: pad q, k, v into a cached
+  // buffer, run the masked forward pass, copy the real output rows back
+  const size_t slot = align_up((size_t)pb.G * N * row_bytes);
+  std::lock_guard<std::mutex> pad_lock(g_pad_mu);
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if ((st = ensure(g_pad[dev], 4 * slot)) != MONARCH_OK) return st;
+  }
+  char* base = static_cast<char*>(g_pad[dev].ptr);
+  char *dq = base, *dk = base + slot, *dv = base + 2 * slot, *dout = base + 3 * slot;
+  int pad_launches = 0;
+  const void* in_src[3] = {q, k, v};
+  void* in_dst[3] = {dq, dk, dv};
+  cudaError_t e = monarch::pad_rows(in_src, in_dst, 3, pb.G, N, n_real, real_lo, row_bytes, true,
+                                    stream, &pad_launches);
+  if (e != cudaSuccess) return record_cuda(e);
+  st = dtype == MONARCH_DTYPE_BF16
+           ? forward_device<bf16>(reinterpret_cast<const bf16*>(dq),
+                                  reinterpret_cast<const bf16*>(dk),
+                                  reinterpret_cast<const bf16*>(dv), reinterpret_cast<bf16*>(dout),
+                                  B, H, b1, b2, d, T, c1, c2, stream, MONARCH_DTYPE_BF16,
+                                  pb.real_lo, pb.real_hi)
+           : forward_device<float>(reinterpret_cast<const float*>(dq),
+                                   reinterpret_cast<const float*>(dk),
+                                   reinterpret_cast<const float*>(dv),
+                                   reinterpret_cast<float*>(dout), B, H, b1, b2, d, T, c1, c2,
+                                   stream, MONARCH_DTYPE_F32, pb.real_lo, pb.real_hi);
+  if (st != MONARCH_OK) return st;
+  const void* out_src[1] = {dout};
+  void* out_dst[1] = {out};
+  e = monarch::pad_rows(out_src, out_dst, 1, pb.G, N, n_real, real_lo, row_bytes, false, stream,
+                        &pad_launches);
+  if (e != cudaSuccess) return record_cuda(e);
+  t_launches += pad_launches;
+  return MONARCH_OK;
+}
+
 size_t monarch_attn_workspace_bytes(int B, int H, int b1, int b2, int d, int T, int c1, int c2,
                                     int dtype) {
   if (monarch::validate_args(B, H, b1, b2, d, T, c1, c2) != MONARCH_OK) return 0;
@@ -407,23 +495,27 @@ size_t monarch_attn_workspace_bytes(int B, int H, int b1, int b2, int d, int T, 
 }
 
 void monarch_attn_release_workspace(void) {
+  std::lock_guard<std::mutex> pad_lock(g_pad_mu);
   std::lock_guard<std::mutex> layout_lock(g_layout_mu);
   std::lock_guard<std::mutex> stage_lock(g_stage_mu);
   std::lock_guard<std::mutex> lock(g_mu);
   int cur = 0;
   cudaGetDevice(&cur);
   for (int dev = 0; dev < kMaxDevices; ++dev) {
-    if (!g_ws[dev].ptr && !g_stage[dev].ptr && !g_layout[dev].ptr && g_tables[dev].empty())
+    if (!g_ws[dev].ptr && !g_stage[dev].ptr && !g_layout[dev].ptr && !g_pad[dev].ptr &&
+        g_tables[dev].empty())
       continue;
     cudaSetDevice(dev);
     if (g_ws[dev].ptr) cudaFree(g_ws[dev].ptr);
     if (g_stage[dev].ptr) cudaFree(g_stage[dev].ptr);
     if (g_layout[dev].ptr) cudaFree(g_layout[dev].ptr);
+    if (g_pad[dev].ptr) cudaFree(g_pad[dev].ptr);
     for (PermTable& t : g_tables[dev]) cudaFree(t.dev_table);
     g_tables[dev].clear();
     g_ws[dev] = DevBuf();
     g_stage[dev] = DevBuf();
     g_layout[dev] = DevBuf();
+    g_pad[dev] = DevBuf();
   }
   cudaSetDevice(cur);
 }

@@ -46,11 +46,12 @@ __global__ void init_qt_kernel(const TIn* __restrict__ Q, float* __restrict__ qt
   r /= pb.b2;
   const int p = (int)(r % pb.c1);
   const long g = r / pb.c1;
-  const int l0 = group_start(pb.b1, pb.c1, p), l1 = group_start(pb.b1, pb.c1, p + 1);
+  int l0 = group_start(pb.b1, pb.c1, p), l1 = group_start(pb.b1, pb.c1, p + 1);
+  real_rows(pb, i, l0, l1, &l0, &l1);  // the group's real rows at position i
   const TIn* base = Q + (g * pb.b1 * pb.b2 + i) * (long)pb.d + x;
   float s = 0.f;
   for (int l = l0; l < l1; ++l) s += to_f32(base[(long)l * pb.b2 * pb.d]);
-  qt0[tid] = s / (float)(l1 - l0);
+  qt0[tid] = l1 > l0 ? s / (float)(l1 - l0) : 0.f;
 }
 
 // One block per (g, k); one warp per R row (p, q, i).
@@ -80,11 +81,11 @@ r_update_kernel(const TIn* __restrict__ K, const TIn* __restrict__ V,
     for (int u = 0; u < DV; ++u) ak[u] = av[u] = 0.f;
     for (int jb = j0; jb < j1; jb += 32) {
       const int j = jb + lane;
-      const bool valid = j < j1;
+      const bool valid = j < j1 && is_real(pb, (long)k * b2 + j);  // pad keys: zero weight
       const float s = valid ? dot_row(sq, Kk + (long)j * d, d) : -INFINITY;
       const float mn = fmaxf(m, warp_max(s));
       const float alpha = (m == -INFINITY) ? 0.f : expf(m - mn);
-      const float e = valid ? expf(s - mn) : 0.f;
+      const float e = valid ? expf(s - mn) : 0.f;  // valid implies mn finite
       t = (m == -INFINITY) ? 0.f : alpha * (t + z * (m - mn));
       z = z * alpha + warp_sum(e);
       t += warp_sum(valid ? e * (s - mn) : 0.f);
@@ -106,7 +107,9 @@ r_update_kernel(const TIn* __restrict__ K, const TIn* __restrict__ V,
       }
       m = mn;
     }
-    const float inv = 1.f / z;
+    // a group without a real key: Kt = Y = 0 and an entropy bias of -inf,
+    // which gives it zero weight in the L-update
+    const float inv = z > 0.f ? 1.f / z : 0.f;
     const long orow = (((g * b2 + i) * c1 + p) * b1 + k) * (long)c2 + q;
 #pragma unroll
     for (int u = 0; u < DV; ++u) {
@@ -116,7 +119,7 @@ r_update_kernel(const TIn* __restrict__ K, const TIn* __restrict__ V,
         if (write_y) y[orow * d + x] = from_f32<TW>(av[u] * inv);
       }
     }
-    if (lane == 0) hs[orow] = logf(z) - t * inv;
+    if (lane == 0) hs[orow] = z > 0.f ? logf(z) - t * inv : -INFINITY;
     __syncwarp();
   }
 }
@@ -138,6 +141,7 @@ l_rows_kernel(const TIn* __restrict__ Q, const TW* __restrict__ kt,
   const long g = r / b2;
   const int l = lb * kWarps + warp;
   if (l >= b1) return;
+  if (!is_real(pb, (long)l * b2 + i)) return;  // pad query rows: no output, no statistics
   const int p = group_of(b1, c1, l);
   float* sq = smem + warp * d;
   const TIn* qrow = Q + ((g * b1 + l) * b2 + i) * (long)d;
@@ -155,7 +159,8 @@ l_rows_kernel(const TIn* __restrict__ Q, const TW* __restrict__ kt,
     const float s = valid ? dot_row(sq, kt + (kbase + kk) * d, d) + hs[kbase + kk] : -INFINITY;
     const float mn = fmaxf(m, warp_max(s));
     const float alpha = (m == -INFINITY) ? 0.f : expf(m - mn);
-    const float e = valid ? expf(s - mn) : 0.f;
+    // keys of a group without a real key have s = -inf (so does a whole block of them)
+    const float e = s > -INFINITY ? expf(s - mn) : 0.f;
     z = z * alpha + warp_sum(e);
     if (MODE == 0) {
 #pragma unroll
@@ -220,7 +225,7 @@ l_aggregate_kernel(const TIn* __restrict__ Q, const TW* __restrict__ kt,
   for (int u = 0; u < DV; ++u) acc[u] = 0.f;
   for (int lb = l0; lb < l1; lb += 32) {
     const int l = lb + lane;
-    const bool valid = l < l1;
+    const bool valid = l < l1 && is_real(pb, (long)l * b2 + i);  // pad rows: zero weight
     float P = 0.f;
     if (valid) {
       const float s = dot_row(sk, Q + ((g * b1 + l) * b2 + i) * (long)d, d) + bias - lse_i[l];
@@ -249,21 +254,32 @@ l_aggregate_kernel(const TIn* __restrict__ Q, const TW* __restrict__ kt,
 
 // T = 0: every row of M is the uniform Monarch row, so O is the same for all
 // tokens of a head: sum over (k, q) of mean_{j in q} v_(k,j) / (b1 c2).
+// With padding, the means run over the real keys and the groups with at
+// least one real key.
 template <typename TIn>
 __global__ void ybar_kernel(const TIn* __restrict__ V, float* __restrict__ ybar, Problem pb) {
   const long g = blockIdx.x;
   const int d = pb.d, b1 = pb.b1, b2 = pb.b2, c2 = pb.c2;
   for (int x = threadIdx.x; x < d; x += blockDim.x) {
     float acc = 0.f;
+    int groups_used = 0;
     for (int k = 0; k < b1; ++k) {
       for (int q = 0; q < c2; ++q) {
         const int j0 = group_start(b2, c2, q), j1 = group_start(b2, c2, q + 1);
         float s = 0.f;
-        for (int j = j0; j < j1; ++j) s += to_f32(V[((g * b1 + k) * b2 + j) * (long)d + x]);
-        acc += s / (float)(j1 - j0);
+        int n = 0;
+        for (int j = j0; j < j1; ++j) {
+          if (!is_real(pb, (long)k * b2 + j)) continue;
+          s += to_f32(V[((g * b1 + k) * b2 + j) * (long)d + x]);
+          ++n;
+        }
+        if (n > 0) {
+          acc += s / (float)n;
+          ++groups_used;
+        }
       }
     }
-    ybar[g * d + x] = acc / (float)(b1 * c2);
+    ybar[g * d + x] = acc / (float)groups_used;
   }
 }
 

@@ -69,10 +69,13 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
 }
 
 // Row softmax over the 16 columns of a 16 x 16 accumulator pair s[2][4]
-// (this thread: rows g and g+8, columns nt*8 + 2t + {0, 1}); columns >= n
-// are masked.  On return s holds the normalised weights; lnz/dot get, per
-// row half h, ln z and sum_j w_j (s_j - m) (for the entropy).
-__device__ __forceinline__ void quad_softmax(float (&s)[2][4], int n, int t, float (&ent)[2]) {
+// (this thread: rows g and g+8, columns nt*8 + 2t + {0, 1}); columns outside
+// [c_lo, c_hi) are masked, and so are columns already -inf.  On return s
+// holds the normalised weights (all 0 in a row with every column masked);
+// ent gets, per row half h, the entropy ln z - sum_j w_j (s_j - m) / z
+// (-inf for such a row).
+__device__ __forceinline__ void quad_softmax(float (&s)[2][4], int c_lo, int c_hi, int t,
+                                             float (&ent)[2]) {
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     float m = -INFINITY;
@@ -81,11 +84,12 @@ __device__ __forceinline__ void quad_softmax(float (&s)[2][4], int n, int t, flo
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int col = nt * 8 + 2 * t + e;
-        if (col >= n) s[nt][2 * h + e] = -INFINITY;
+        if (col < c_lo || col >= c_hi) s[nt][2 * h + e] = -INFINITY;
         m = fmaxf(m, s[nt][2 * h + e]);
       }
     m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
     m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+    if (m == -INFINITY) m = 0.f;  // every column masked: all weights 0
     float z = 0.f, dot = 0.f;
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
@@ -101,12 +105,12 @@ __device__ __forceinline__ void quad_softmax(float (&s)[2][4], int n, int t, flo
     z += __shfl_xor_sync(0xffffffffu, z, 2);
     dot += __shfl_xor_sync(0xffffffffu, dot, 1);
     dot += __shfl_xor_sync(0xffffffffu, dot, 2);
-    const float inv = 1.f / z;
+    const float inv = z > 0.f ? 1.f / z : 0.f;
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int e = 0; e < 2; ++e) s[nt][2 * h + e] *= inv;
-    ent[h] = __logf(z) - dot * inv;
+    ent[h] = z > 0.f ? __logf(z) - dot * inv : -INFINITY;
   }
 }
 
@@ -119,12 +123,16 @@ __device__ __forceinline__ void acc_to_a(const float (&s)[2][4], uint32_t (&a)[4
   a[3] = tc::pack_bf16x2(s[1][2], s[1][3]);
 }
 
+// Padding: the head's real tokens are grid tokens [real_lo, real_hi); q, k, v
+// and out hold only those rows (real_hi - real_lo per head), pad rows are
+// zero in shared memory and are masked in every softmax and aggregation.
 __global__ void __launch_bounds__(kThreads, 1)
     small_head_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
                       const bf16* __restrict__ v, bf16* __restrict__ out, int b1, int b2, int T,
-                      float sc) {
+                      float sc, int real_lo, int real_hi) {
   extern __shared__ __align__(16) uint8_t smem[];
   const int N = b1 * b2;
+  const int n_src = real_hi - real_lo;  // rows per head in q, k, v, out
   bf16* Qs = reinterpret_cast<bf16*>(smem);  // token rows l * b2 + i
   bf16* Ks = Qs + N * kPB;
   bf16* Vs = Ks + N * kPB;
@@ -139,30 +147,39 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ldmatrix lane roles: matrix mi = lane / 8, row lr = lane % 8
   const int mi = lane >> 3, lr = lane & 7;
 
-  // q, k, v of the head into shared memory (16-byte chunks)
+  // q, k, v of the head into shared memory (16-byte chunks); pad rows are zero
   {
-    const uint4* gq = reinterpret_cast<const uint4*>(q + gh * N * kD);
-    const uint4* gk = reinterpret_cast<const uint4*>(k + gh * N * kD);
-    const uint4* gv = reinterpret_cast<const uint4*>(v + gh * N * kD);
+    const uint4* gq = reinterpret_cast<const uint4*>(q + gh * n_src * kD);
+    const uint4* gk = reinterpret_cast<const uint4*>(k + gh * n_src * kD);
+    const uint4* gv = reinterpret_cast<const uint4*>(v + gh * n_src * kD);
     for (int x = tid; x < N * (kD / 8); x += kThreads) {
       const int r = x / (kD / 8), c = x % (kD / 8);
       const int so = r * kPB + c * 8;
-      *reinterpret_cast<uint4*>(Qs + so) = __ldg(gq + x);
-      *reinterpret_cast<uint4*>(Ks + so) = __ldg(gk + x);
-      *reinterpret_cast<uint4*>(Vs + so) = __ldg(gv + x);
+      const bool real = r >= real_lo && r < real_hi;
+      const int xs = (r - real_lo) * (kD / 8) + c;
+      const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+      *reinterpret_cast<uint4*>(Qs + so) = real ? __ldg(gq + xs) : zero;
+      *reinterpret_cast<uint4*>(Ks + so) = real ? __ldg(gk + xs) : zero;
+      *reinterpret_cast<uint4*>(Vs + so) = real ? __ldg(gv + xs) : zero;
     }
   }
   __syncthreads();
-  // step-one aggregated queries (uniform L): every row (k, i) gets mean_l q_(l,i)
+  // step-one aggregated queries (uniform L): every row (k, i) gets the mean of
+  // the real q_(l,i) (0 if position i has none)
   for (int x = tid; x < b2 * (kD / 2); x += kThreads) {
     const int i = x / (kD / 2), c = (x % (kD / 2)) * 2;
     float s0 = 0.f, s1 = 0.f;
+    int nl = 0;
     for (int l = 0; l < b1; ++l) {
+      if (l * b2 + i < real_lo || l * b2 + i >= real_hi) continue;
       const __nv_bfloat162 p = *reinterpret_cast<const __nv_bfloat162*>(Qs + (l * b2 + i) * kPB + c);
       s0 += __low2float(p);
       s1 += __high2float(p);
+      ++nl;
     }
-    const uint32_t m = tc::pack_bf16x2(s0 / (float)b1, s1 / (float)b1);
+    const float inv_n = nl > 0 ? 1.f / (float)nl : 0.f;
+    const uint32_t m = nl == b1 ? tc::pack_bf16x2(s0 / (float)b1, s1 / (float)b1)
+                                : tc::pack_bf16x2(s0 * inv_n, s1 * inv_n);
     for (int kk = 0; kk < b1; ++kk) *reinterpret_cast<uint32_t*>(Qt + (kk * b2 + i) * kPB + c) = m;
   }
   __syncthreads();
@@ -190,8 +207,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) s[nt][e] *= sc;
+      // real keys of chunk kk: j in [j_lo, j_hi)
+      const int j_lo = min(max(real_lo - kk * b2, 0), b2);
+      const int j_hi = max(min(real_hi - kk * b2, b2), j_lo);
       float ent[2];
-      quad_softmax(s, b2, t, ent);
+      quad_softmax(s, j_lo, j_hi, t, ent);
       if (t == 0) {
         if (g < b2) Hs[g * b1 + kk] = ent[0];
         if (g + 8 < b2) Hs[(g + 8) * b1 + kk] = ent[1];
@@ -259,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           s[nt][e] = fmaf(s[nt][e], sc, Hs[i * b1 + col]);
         }
       float ent[2];
-      quad_softmax(s, b1, t, ent);
+      quad_softmax(s, 0, b1, t, ent);  // chunks without a real key carry Hs = -inf
       if (!last) {
         // L (bf16; rows l >= b1 zeroed) to this position's tile, then
         // Qt = L^T q / column sums of L
@@ -269,8 +289,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const int row = g + 8 * h, col = nt * 8 + 2 * t;
+            const bool real = row < b1 && row * b2 + i >= real_lo && row * b2 + i < real_hi;
             *reinterpret_cast<uint32_t*>(Lt + row * kPL + col) =
-                row < b1 ? tc::pack_bf16x2(s[nt][2 * h], s[nt][2 * h + 1]) : 0u;
+                real ? tc::pack_bf16x2(s[nt][2 * h], s[nt][2 * h + 1]) : 0u;
           }
         __syncwarp();
         // A = L^T (rows k, k-dim l) from the l-major tile: transposed ldmatrix
@@ -309,8 +330,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t a[4];
         acc_to_a(s, a);
         const bf16* y_src = Ys + (i * b1 + min(lr + (mi & 1) * 8, b1 - 1)) * kPB + (mi >> 1) * 8;
-        bf16* orow0 = out + (gh * N + g * b2 + i) * kD;
-        bf16* orow1 = out + (gh * N + (g + 8) * b2 + i) * kD;
+        // only real rows are written, to their row in the unpadded output
+        const int m0 = g * b2 + i, m1 = (g + 8) * b2 + i;
+        const bool w0 = g < b1 && m0 >= real_lo && m0 < real_hi;
+        const bool w1 = g + 8 < b1 && m1 >= real_lo && m1 < real_hi;
+        bf16* orow0 = out + (gh * n_src + (m0 - real_lo)) * kD;
+        bf16* orow1 = out + (gh * n_src + (m1 - real_lo)) * kD;
 #pragma unroll
         for (int cb = 0; cb < kD / 16; ++cb) {
           uint32_t b[4];
@@ -321,9 +346,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const int cc = cb * 16 + h * 8 + 2 * t;
-            if (g < b1) *reinterpret_cast<uint32_t*>(orow0 + cc) = tc::pack_bf16x2(acc[h][0], acc[h][1]);
-            if (g + 8 < b1)
-              *reinterpret_cast<uint32_t*>(orow1 + cc) = tc::pack_bf16x2(acc[h][2], acc[h][3]);
+            if (w0) *reinterpret_cast<uint32_t*>(orow0 + cc) = tc::pack_bf16x2(acc[h][0], acc[h][1]);
+            if (w1) *reinterpret_cast<uint32_t*>(orow1 + cc) = tc::pack_bf16x2(acc[h][2], acc[h][3]);
           }
         }
       }
@@ -351,7 +375,8 @@ cudaError_t small_head_forward(const bf16* q, const bf16* k, const bf16* v, bf16
   if (!small_head_supports(pb)) return cudaErrorInvalidValue;
   const size_t smem = smem_bytes(pb.b1 * pb.b2);
   return timed_launch("small_head", stream, launches, [&] {
-    small_head_kernel<<<pb.G, kThreads, smem, stream>>>(q, k, v, out, pb.b1, pb.b2, pb.T, pb.sc);
+    small_head_kernel<<<pb.G, kThreads, smem, stream>>>(q, k, v, out, pb.b1, pb.b2, pb.T, pb.sc,
+                                                         pb.real_lo, pb.real_hi);
   });
 }
 

@@ -486,7 +486,8 @@ __global__ void __launch_bounds__(192, 2)
           resc = j > 0;
           m_run = mt;
         }
-        const float neg_m2 = -m_run * kLog2e;
+        // every key seen so far masked (groups without a real key): weights 0
+        const float neg_m2 = m_run > -INFINITY ? -m_run * kLog2e : 0.f;
         float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int c = 0; c < NK; ++c) {
@@ -821,7 +822,7 @@ __global__ void __launch_bounds__(192, 2)
 // ---------------------------------------------------------------------------
 // Step-one aggregated queries under the uniform initial L (bf16):
 // Qt0[g][p][i][:] = mean_{l in p} q_(l,i).  One block per (g, p, i): 16-byte
-// column chunks x row lanes, up to eight row loads of a thread in flight at once;
+// column chunks x row lanes, every row load of a thread in flight at once;
 // the row lanes are summed in a fixed order (warp shuffles, then the 8 warps
 // through shared memory).  Launched with programmatic stream serialisation:
 // its blocks may be scheduled while the previous kernel of the stream
@@ -831,17 +832,18 @@ __global__ void __launch_bounds__(192, 2)
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256)
-    init_qt_bf16_kernel(const bf16* __restrict__ q, bf16* __restrict__ qt0, int b1, int b2,
-                        int c1) {
+    init_qt_bf16_kernel(const bf16* __restrict__ q, bf16* __restrict__ qt0, Problem pb) {
   constexpr int CH = D / 8;        // 16-byte chunks per row
   constexpr int RL = 256 / CH;     // row lanes
   __shared__ float red[8][D];
+  const int b1 = pb.b1, b2 = pb.b2, c1 = pb.c1;
   int bid = blockIdx.x;
   const int i = bid % b2;
   bid /= b2;
   const int p = bid % c1;
   const long g = bid / c1;
-  const int l0 = group_start(b1, c1, p), l1 = group_start(b1, c1, p + 1);
+  int l0 = group_start(b1, c1, p), l1 = group_start(b1, c1, p + 1);
+  real_rows(pb, i, l0, l1, &l0, &l1);  // the group's real rows at position i
   pdl_wait();
   pdl_launch_dependents();
   const int ch = threadIdx.x % CH, rl = threadIdx.x / CH, lane = threadIdx.x & 31;
@@ -850,24 +852,14 @@ __global__ void __launch_bounds__(256)
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
   const uint4* base = reinterpret_cast<const uint4*>(q + (g * b1 * b2 + i) * D) + ch;
   const long row_stride = (long)b2 * D / 8;  // in uint4
-  // Rounds of U predicated loads, all issued before any is summed, so a
-  // short group (a few rows per lane) still has every load in flight.
-  constexpr int U = 8;
-  for (int l = l0 + rl; l < l1; l += U * RL) {
-    uint4 u[U];
+#pragma unroll 8
+  for (int l = l0 + rl; l < l1; l += RL) {
+    const uint4 u = __ldg(base + l * row_stride);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-    for (int t = 0; t < U; ++t) {
-      const int lt = l + t * RL;
-      u[t] = lt < l1 ? __ldg(base + lt * row_stride) : make_uint4(0u, 0u, 0u, 0u);
-    }
-#pragma unroll
-    for (int t = 0; t < U; ++t) {
-      const uint32_t w[4] = {u[t].x, u[t].y, u[t].z, u[t].w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        acc[2 * e] += __uint_as_float(w[e] << 16);
-        acc[2 * e + 1] += __uint_as_float(w[e] & 0xffff0000u);
-      }
+    for (int e = 0; e < 4; ++e) {
+      acc[2 * e] += __uint_as_float(w[e] << 16);
+      acc[2 * e + 1] += __uint_as_float(w[e] & 0xffff0000u);
     }
   }
 #pragma unroll
@@ -884,7 +876,8 @@ __global__ void __launch_bounds__(256)
     float sum = 0.f;
 #pragma unroll
     for (int w8 = 0; w8 < 8; ++w8) sum += red[w8][threadIdx.x];
-    qt0[((g * c1 + p) * b2 + i) * D + threadIdx.x] = __float2bfloat16_rn(sum / (float)(l1 - l0));
+    qt0[((g * c1 + p) * b2 + i) * D + threadIdx.x] =
+        __float2bfloat16_rn(l1 > l0 ? sum / (float)(l1 - l0) : 0.f);
   }
 }
 
@@ -907,7 +900,62 @@ struct KRArgs {
   int b1, b2, c1, c2, write_y;
   float sc_log2;
   int* status;
+  int real_lo, real_hi;  // real tokens (padding): keys outside get zero weight
 };
+
+// Keys [*j_lo, *j_hi) of the nq keys of column group q (first key js) of
+// chunk k are real; an empty range marks a group without a real key.
+__device__ __forceinline__ void real_keys(int real_lo, int real_hi, int b2, int k, int js, int nq,
+                                          int* j_lo, int* j_hi) {
+  const long first = (long)k * b2 + js;
+  *j_lo = (int)max(0L, min((long)nq, real_lo - first));
+  *j_hi = (int)max((long)*j_lo, min((long)nq, real_hi - first));
+}
+
+// Softmax of one R row held as NQ raw logits in sv (this thread's TMEM lane):
+// columns [jlo, jhi) are the group's real keys (nq of them without padding).
+// On return sv holds exp2(s - m) in log2 units (0 outside the real keys),
+// z their sum and t2 = sum exp2(s - m) (s - m), the entropy's numerator.  A
+// group without a real key gets all zeros and z = 0.  The unpadded case
+// (jlo = 0, jhi = nq: warp-uniform) keeps the single bound check.
+template <int NQ>
+__device__ __forceinline__ void r_row_softmax(float (&sv)[NQ], float sc_log2, int jlo, int jhi,
+                                              int nq, float& z, float& t2) {
+  float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+  float zs[4] = {0.f, 0.f, 0.f, 0.f}, ts[4] = {0.f, 0.f, 0.f, 0.f};
+  if (jlo == 0 && jhi == nq) {
+#pragma unroll
+    for (int j = 0; j < NQ; ++j) {
+      sv[j] = j < nq ? sv[j] * sc_log2 : -INFINITY;
+      mx[j & 3] = fmaxf(mx[j & 3], sv[j]);
+    }
+    const float m2 = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+#pragma unroll
+    for (int j = 0; j < NQ; ++j) {
+      const float d2 = sv[j] - m2;  // -inf for j >= nq
+      sv[j] = ex2(d2);
+      zs[j & 3] += sv[j];
+      ts[j & 3] += j < nq ? sv[j] * d2 : 0.f;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < NQ; ++j) {
+      sv[j] = (j >= jlo && j < jhi) ? sv[j] * sc_log2 : -INFINITY;
+      mx[j & 3] = fmaxf(mx[j & 3], sv[j]);
+    }
+    // a group without a real key has no finite logit: its weights become 0
+    const float m2 = jhi > jlo ? fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) : 0.f;
+#pragma unroll
+    for (int j = 0; j < NQ; ++j) {
+      const float d2 = sv[j] - m2;  // -inf outside the real keys
+      sv[j] = ex2(d2);
+      zs[j & 3] += sv[j];
+      ts[j & 3] += (j >= jlo && j < jhi) ? sv[j] * d2 : 0.f;
+    }
+  }
+  z = (zs[0] + zs[1]) + (zs[2] + zs[3]);
+  t2 = (ts[0] + ts[1]) + (ts[2] + ts[3]);
+}
 
 template <int D, int NQ>
 struct KRLayout {
@@ -1010,7 +1058,10 @@ __global__ void __launch_bounds__(128)
   const int r = tid;  // row = position i
   const bool row_valid = r < a.b2;
   for (int q = 0; q < a.c2; ++q) {
-    const int nq = group_start(a.b2, a.c2, q + 1) - group_start(a.b2, a.c2, q);
+    const int js = group_start(a.b2, a.c2, q);
+    const int nq = group_start(a.b2, a.c2, q + 1) - js;
+    int jlo, jhi;
+    real_keys(a.real_lo, a.real_hi, a.b2, k, js, nq, &jlo, &jhi);
     bool ok = mbar_wait(s_full, q & 1, abort_flag, a.status);
     ok = __all_sync(0xffffffffu, ok);
     float z = 0.f, t2 = 0.f;
@@ -1026,23 +1077,7 @@ __global__ void __launch_bounds__(128)
       }
       tmem_wait_ld();
       // logits in log2 units; 4 partial maxima and sums break the serial chains
-      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-      for (int j = 0; j < NQ; ++j) {
-        sv[j] = j < nq ? sv[j] * a.sc_log2 : -INFINITY;
-        mx[j & 3] = fmaxf(mx[j & 3], sv[j]);
-      }
-      const float m2 = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-      float zs[4] = {0.f, 0.f, 0.f, 0.f}, ts[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int j = 0; j < NQ; ++j) {
-        const float d2 = sv[j] - m2;  // -inf for j >= nq
-        sv[j] = ex2(d2);
-        zs[j & 3] += sv[j];
-        ts[j & 3] += j < nq ? sv[j] * d2 : 0.f;
-      }
-      z = (zs[0] + zs[1]) + (zs[2] + zs[3]);
-      t2 = (ts[0] + ts[1]) + (ts[2] + ts[3]);
+      r_row_softmax<NQ>(sv, a.sc_log2, jlo, jhi, nq, z, t2);
 #pragma unroll
       for (int u = 0; u < NQ / 8; ++u) {
         uint4 pk;
@@ -1076,7 +1111,7 @@ __global__ void __launch_bounds__(128)
     ok = __all_sync(0xffffffffu, ok);
     if (ok) {
       tc_fence_after();
-      const float inv = 1.f / z;
+      const float inv = z > 0.f ? 1.f / z : 0.f;
       // The b2 rows of this (g, p, k, q) are positions i of the position-major
       // Kt/Y layout: one 3-D TMA box {64 columns, 1, b2 rows}.  Each 64-column
       // block is staged (swizzled) in one of two buffers and handed to a TMA
@@ -1118,7 +1153,7 @@ __global__ void __launch_bounds__(128)
       // entropy of the R row: ln z - sum e (s - m) / z, with s - m in log2 units
       if (row_valid) {
         const long orow = ((((long)g * a.b2 + r) * a.c1 + p) * a.b1 + k) * a.c2 + q;
-        a.hs[orow] = logf(z) - t2 * 0.69314718055994531f * inv;
+        a.hs[orow] = z > 0.f ? logf(z) - t2 * 0.69314718055994531f * inv : -INFINITY;
       }
     }
     tc_fence_before();
@@ -1196,6 +1231,7 @@ struct KR2Args {
   int b1, b2, c1, c2, n_items, write_y;
   float sc_log2;
   int* status;
+  int real_lo, real_hi;  // real tokens (padding): keys outside get zero weight
 };
 
 struct KR2Sub {
@@ -1475,7 +1511,10 @@ __global__ void __launch_bounds__(320, 1)
       const long n = s0 + t * H + h;
       const bool have = n < s1;  // warp-uniform
       const KR2Sub sb = kr2_sub(a, have ? n : s0 + t * H);
-      const int nq = group_start(a.b2, a.c2, sb.q + 1) - group_start(a.b2, a.c2, sb.q);
+      const int js = group_start(a.b2, a.c2, sb.q);
+      const int nq = group_start(a.b2, a.c2, sb.q + 1) - js;
+      int jlo, jhi;
+      real_keys(a.real_lo, a.real_hi, a.b2, sb.k, js, nq, &jlo, &jhi);
       ok = mbar_wait(s_full + w, (t >> 1) & 1, abort_flag, a.status);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
@@ -1489,24 +1528,10 @@ __global__ void __launch_bounds__(320, 1)
         for (int e = 0; e < 16; ++e) sv[c * 16 + e] = tt[e];
       }
       tmem_wait_ld();
-      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-      for (int j = 0; j < NQ; ++j) {
-        sv[j] = j < nq ? sv[j] * a.sc_log2 : -INFINITY;
-        mx[j & 3] = fmaxf(mx[j & 3], sv[j]);
-      }
-      const float m2 = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-      float zs[4] = {0.f, 0.f, 0.f, 0.f}, ts2[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int j = 0; j < NQ; ++j) {
-        const float d2 = sv[j] - m2;
-        sv[j] = ex2(d2);
-        zs[j & 3] += sv[j];
-        ts2[j & 3] += j < nq ? sv[j] * d2 : 0.f;
-      }
-      const float z = (zs[0] + zs[1]) + (zs[2] + zs[3]);
-      const float t2 = (ts2[0] + ts2[1]) + (ts2[2] + ts2[3]);
-      const float inv = have ? 1.f / z : 0.f;  // an absent sub-item contributes P = 0
+      float z, t2;
+      r_row_softmax<NQ>(sv, a.sc_log2, jlo, jhi, nq, z, t2);
+      // an absent sub-item, or a group without a real key, contributes P = 0
+      const float inv = (have && z > 0.f) ? 1.f / z : 0.f;
       uint8_t* pbuf = sP(w);
       if (PAIR) {  // this warp's rows of P were the previous tile's staging: stores must have read them
         if (lane == 0) bulk_wait_read<0>();
@@ -1631,7 +1656,7 @@ __global__ void __launch_bounds__(320, 1)
           }
         }
       }
-      if (row_ok) a.hs[orow_w] = logf(z) - t2 * 0.69314718055994531f / z;
+      if (row_ok) a.hs[orow_w] = z > 0.f ? logf(z) - t2 * 0.69314718055994531f / z : -INFINITY;
     }
     if (PAIR ? lane == 0 : leader) bulk_wait<0>();  // stores done reading shared memory before exit
   }
@@ -1927,6 +1952,8 @@ cudaError_t launch_kr(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, b
   a.write_y = pb.T == 1 ? 1 : 0;
   a.sc_log2 = kLog2e * pb.sc;
   a.status = status;
+  a.real_lo = pb.real_lo;
+  a.real_hi = pb.real_hi;
   const long blocks = (long)pb.G * pb.b1 * pb.c1;
   return timed_launch("tc_r_update", stream, launches, [&] {
     return launch_pdl(kr_kernel<D, NQ>, dim3((unsigned)blocks), dim3(128), L::bytes(pb.c2), stream, tq,
@@ -1992,6 +2019,8 @@ cudaError_t launch_kr2(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, 
   a.write_y = pb.T == 1 ? 1 : 0;
   a.sc_log2 = kLog2e * pb.sc;
   a.status = status;
+  a.real_lo = pb.real_lo;
+  a.real_hi = pb.real_hi;
   const long units = (items * pb.c2 + L::kHalves - 1) / L::kHalves;
   const int grid = (int)std::min<long>(units, num_sms());
   return timed_launch("tc_r_update", stream, launches, [&] {
@@ -2015,7 +2044,7 @@ cudaError_t launch_r_step1(const bf16* q, const bf16* k, const bf16* v, bf16* qt
                            cudaStream_t stream, int* launches) {
   cudaError_t e = timed_launch("tc_init_qt", stream, launches, [&] {
     return launch_pdl(init_qt_bf16_kernel<D>, dim3((unsigned)((long)pb.G * pb.c1 * pb.b2)),
-                      dim3(256), 0, stream, q, qt0, pb.b1, pb.b2, pb.c1);
+                      dim3(256), 0, stream, q, qt0, pb);
   });
   if (e != cudaSuccess) return e;
   switch (kr_group_tile(pb)) {

@@ -118,3 +118,15 @@ def test_noalloc_entry_validates_before_any_launch(lib, d, T, expect):
                                         None) == expect
     assert lib.monarch_attn_fwd_noalloc(None, p, p, p, 1, 1, 4, 4, 64, 1, 1, 1, None) == \
         api.MONARCH_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("dtype,n_real,pad_front,expect", [
+    (api.DTYPE_BF16, 0, 1, api.MONARCH_ERR_INVALID_ARG),     # no real token
+    (api.DTYPE_BF16, 17, 1, api.MONARCH_ERR_INVALID_ARG),    # more than b1*b2 = 16
+    (api.DTYPE_BF16, 10, 2, api.MONARCH_ERR_INVALID_ARG),    # pad_front not 0/1
+    (5, 10, 1, api.MONARCH_ERR_INVALID_ARG),                 # unknown dtype
+])
+def test_padded_entry_validates_before_any_launch(lib, dtype, n_real, pad_front, expect):
+    p = 1 << 20
+    assert lib.monarch_attn_fwd_padded(dtype, p, 2 * p, 3 * p, 4 * p, 1, 1, n_real, 4, 4,
+                                       pad_front, 64, 1, 1, 1, None) == expect
