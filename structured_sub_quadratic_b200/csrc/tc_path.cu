@@ -20,7 +20,10 @@
 // 2^8 (exact result, fewer rescales of the TMEM accumulator).
 //
 // Step one (aggregated queries under the uniform L, R-update) also runs on
-// the tensor cores; later steps of T >= 2 run on the SIMT kernels.
+// the tensor cores, and so do later steps of T >= 2 (non-final L-update with
+// the aggregation L^T Q, R-update from per-sub-item queries) when every L
+// row fits one 128-key tile and every row group one 128-row tile; other
+// shapes run their later steps on the SIMT kernels.
 #include "tc_path.cuh"
 
 #include <cudaTypedefs.h>
@@ -1232,7 +1235,12 @@ struct KR2Args {
   float sc_log2;
   int* status;
   int real_lo, real_hi;  // real tokens (padding): keys outside get zero weight
+  // 0: step one, the aggregated queries Qt0 [G][c1][b2][d] are shared by the
+  // chunks k and groups q of a row group; 1: later steps, every sub-item
+  // (g, p, k, q) has its own rows Qt [G][b1][c1][c2][b2][d]
+  int qt_per_item;
 };
+
 
 struct KR2Sub {
   int g, p, k, q, gp;
@@ -1247,6 +1255,12 @@ __device__ __forceinline__ KR2Sub kr2_sub(const KR2Args& a, long n_sub) {
   s.p = s.gp % a.c1;
   s.g = s.gp / a.c1;
   return s;
+}
+
+// First aggregated-query row of a sub-item.
+__device__ __forceinline__ long kr2_qrow(const KR2Args& a, const KR2Sub& s) {
+  return a.qt_per_item ? ((((long)s.g * a.b1 + s.k) * a.c1 + s.p) * a.c2 + s.q) * a.b2
+                       : (long)s.gp * a.b2;
 }
 
 // Next sub-item in (gp, k, q) order.
@@ -1350,13 +1364,17 @@ __global__ void __launch_bounds__(320, 1)
         mbar_arrive_expect_tx(kv_full + sl, H * 2 * (D / 64) * L::kBox);
         const int gp_a = cur.gp;
         int gp_b = gp_a, krow = 0;
+        long qrow[2] = {0, 0};
         for (int h = 0; h < H; ++h) {
           // An absent second half (odd count, last tile) repeats the first:
           // finite keys that its zero rows of P weigh by zero.
           if (h < nh) {
             krow = (cur.g * a.b1 + cur.k) * a.b2 + group_start(a.b2, a.c2, cur.q);
             gp_b = cur.gp;
+            qrow[h] = kr2_qrow(a, cur);
             kr2_next(a, cur);
+          } else {
+            qrow[h] = qrow[0];
           }
 #pragma unroll
           for (int c = 0; c < D / 64; ++c) {
@@ -1366,22 +1384,24 @@ __global__ void __launch_bounds__(320, 1)
           }
         }
         last_kv = t;
-        const long key = kr2_qkey(gp_a, gp_b);
+        // a new tile needs new query rows when its row groups change (step
+        // one) or always (later steps, one set of rows per sub-item)
+        const long key = a.qt_per_item ? t : kr2_qkey(gp_a, gp_b);
         if (key != cur_key) {
-          if (nq_loads == 0) pdl_wait();  // Qt0 comes from the previous kernel
+          if (nq_loads == 0) pdl_wait();  // the queries come from the previous kernel
           if (ok && nq_loads >= 1) ok = mbar_wait(q_empty, (nq_loads - 1) & 1, abort_flag, a.status);
           if (!ok) break;
           mbar_arrive_expect_tx(q_full, D / 64 * kRows * 128);
           if (PAIR) {
 #pragma unroll
             for (int c = 0; c < D / 64; ++c) {
-              tma_load_2d(sQ + c * kRows * 128, &tm_qt, q_full, c * 64, gp_a * a.b2);
-              tma_load_2d(sQ + c * kRows * 128 + 64 * 128, &tm_qt, q_full, c * 64, gp_b * a.b2);
+              tma_load_2d(sQ + c * kRows * 128, &tm_qt, q_full, c * 64, (int)qrow[0]);
+              tma_load_2d(sQ + c * kRows * 128 + 64 * 128, &tm_qt, q_full, c * 64, (int)qrow[1]);
             }
           } else {
 #pragma unroll
             for (int c = 0; c < D / 64; ++c)
-              tma_load_2d(sQ + c * kRows * 128, &tm_qt, q_full, c * 64, gp_a * a.b2);
+              tma_load_2d(sQ + c * kRows * 128, &tm_qt, q_full, c * 64, (int)qrow[0]);
           }
           cur_key = key;
           ++nq_loads;
@@ -1431,7 +1451,7 @@ __global__ void __launch_bounds__(320, 1)
           gp_b = cur.gp;
           kr2_next(a, cur);
         }
-        return kr2_qkey(gp_a, gp_b);
+        return a.qt_per_item ? t : kr2_qkey(gp_a, gp_b);
       };
       long key = ntiles > 0 ? tile_key(0) : -1;
       unsigned long long idle_since = global_ns();
@@ -1665,6 +1685,225 @@ __global__ void __launch_bounds__(320, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Non-final L-update on the tensor cores, for rows of at most 128 keys
+// (nk = b1 c2) and row groups of at most 128 rows.  One CTA of four warps
+// per (g, i, p):
+//   S = q Kt^T / sqrt(d) + Hs           128 rows x 128 keys in TMEM
+//   L = softmax over the valid keys      exact, thread = row; rows past the
+//                                        group and pad rows get L = 0
+//   [Qt~ | c] = L^T [Q | 1]               128 keys x (d + 64) in TMEM, over the
+//                                        columns S held; c = column sums of L
+//   Qt_{k,p,q,i} = Qt~ / c (0 if c = 0)   thread = key, bf16 rows to global
+// (MonarchAttention OpenReview discussion, the alternating maximisation: the
+// L-update's row softmax, then the aggregated queries of the next
+// R-update.)  L goes to shared memory as bf16 in [row][key] order: with keys
+// as the M dimension that is the MN-major A operand of the second product.
+// Q, staged K-major for the first product, is read again as its MN-major B
+// operand (d contiguous per row), with a constant 64-column block of ones
+// appended, whose products are the column sums.
+// ---------------------------------------------------------------------------
+template <int D>
+struct KLLayout {
+  static constexpr int kChunk = kRows * 128;              // 128 rows x 64 bf16, swizzled
+  static constexpr int kQOff = 0;                          // D / 64 chunks, then the ones
+  static constexpr int kOnesOff = D / 64 * kChunk;
+  static constexpr int kKtOff = kOnesOff + kChunk;         // D / 64 chunks of 128 keys
+  static constexpr int kPOff = kKtOff + D / 64 * kChunk;   // keys 0-63, keys 64-127
+  static constexpr int kBiasOff = kPOff + 2 * kChunk;      // float [128]
+  static constexpr int kBarOff = kBiasOff + 128 * 4;
+  static constexpr int kBytes = kBarOff + 8 * 8;
+  static constexpr uint32_t kTmemCols = 256;
+  static_assert(D == 64 || D == 128, "head dimension");
+};
+
+struct KLArgs {
+  const float* hs;  // [G][b2][c1][nk]
+  bf16* qt;         // [G][b1 k][c1 p][c2 q][b2 i][d]
+  int b1, b2, c1, c2, nk, real_lo, real_hi;
+  float sc;
+  int* status;
+};
+
+template <int D>
+__global__ void __launch_bounds__(128)
+    kl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kt,
+              KLArgs a) {
+  using L = KLLayout<D>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int tid = threadIdx.x, warp = tid >> 5;
+  if (smem_u32(smem) & 1023u) {
+    if (tid == 0) atomicExch(a.status, 2);
+    return;
+  }
+  int bid = blockIdx.x;
+  const int p = bid % a.c1;
+  bid /= a.c1;
+  const int i = bid % a.b2;
+  const int g = bid / a.b2;
+  const int l0 = group_start(a.b1, a.c1, p), l1 = group_start(a.b1, a.c1, p + 1);
+  const long key_row0 = ((long)(g * a.b2 + i) * a.c1 + p) * a.nk;
+  uint8_t* sQ = smem + L::kQOff;
+  uint8_t* sOnes = smem + L::kOnesOff;
+  uint8_t* sKt = smem + L::kKtOff;
+  uint8_t* sP = smem + L::kPOff;
+  float* sBias = reinterpret_cast<float*>(smem + L::kBiasOff);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* load_full = bars + 0;
+  uint64_t* s_full = bars + 1;
+  uint64_t* o_full = bars + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 4);
+  if (tid == 0) {
+    mbar_init(load_full, 1);
+    mbar_init(s_full, 1);
+    mbar_init(o_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  // the ones block: bf16 1.0 in every element
+  for (int x = tid; x < L::kChunk / 16; x += 128)
+    reinterpret_cast<uint4*>(sOnes)[x] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u,
+                                                     0x3F803F80u);
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+  pdl_wait();  // Kt and the entropies come from the previous kernel
+  pdl_launch_dependents();
+  bool issued_s = false, issued_o = false;
+  if (tid == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_kt);
+    mbar_arrive_expect_tx(load_full, 2 * (D / 64) * L::kChunk);
+#pragma unroll
+    for (int c = 0; c < D / 64; ++c) {
+      tma_load_3d(sQ + c * L::kChunk, &tm_q, load_full, c * 64, i, g * a.b1 + l0);
+      tma_load_2d(sKt + c * L::kChunk, &tm_kt, load_full, c * 64, (int)key_row0);
+    }
+  }
+  sBias[tid] = tid < a.nk ? a.hs[key_row0 + tid] : -INFINITY;
+  __syncthreads();
+  if (tid == 0 && mbar_wait(load_full, 0, abort_flag, a.status)) {
+    tc_fence_after();
+    const uint64_t dq = desc_kmajor(smem_u32(sQ)), dk = desc_kmajor(smem_u32(sKt));
+    const uint32_t idesc = idesc_bf16(kRows, 128, false);
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk)
+      mma_bf16_ss(tmem, dq + (((kk >> 2) * L::kChunk + (kk & 3) * 32) >> 4),
+                  dk + (((kk >> 2) * L::kChunk + (kk & 3) * 32) >> 4), idesc, kk > 0 ? 1u : 0u);
+    mma_commit(s_full);
+    issued_s = true;
+  }
+  // ---- softmax, thread = row r of the group ----
+  const int r = tid, l = l0 + r;
+  const bool row_real = l < l1 && l * a.b2 + i >= a.real_lo && l * a.b2 + i < a.real_hi;
+  bool ok = mbar_wait(s_full, 0, abort_flag, a.status);
+  ok = __syncthreads_and(ok);
+  if (ok) {
+    tc_fence_after();
+    float sv[128];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      float t[32];
+      tmem_ld32(tmem + lane_off + c * 32, t);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) sv[c * 32 + e] = t[e];
+    }
+    tmem_wait_ld();
+    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+    for (int c = 0; c < 128; ++c) {
+      sv[c] = fmaf(sv[c], a.sc, sBias[c]);  // -inf past nk and for groups without a real key
+      mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
+    }
+    float m = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+    if (m == -INFINITY) m = 0.f;
+    const float neg_m2 = -m * kLog2e;
+    float zs[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int c = 0; c < 128; ++c) {
+      sv[c] = ex2(fmaf(sv[c], kLog2e, neg_m2));
+      zs[c & 3] += sv[c];
+    }
+    const float z = (zs[0] + zs[1]) + (zs[2] + zs[3]);
+    const float inv = (row_real && z > 0.f) ? 1.f / z : 0.f;
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {  // 16-byte unit u holds keys 8u .. 8u + 7
+      uint4 pk;
+      pk.x = pack_bf16x2(sv[8 * u + 0] * inv, sv[8 * u + 1] * inv);
+      pk.y = pack_bf16x2(sv[8 * u + 2] * inv, sv[8 * u + 3] * inv);
+      pk.z = pack_bf16x2(sv[8 * u + 4] * inv, sv[8 * u + 5] * inv);
+      pk.w = pack_bf16x2(sv[8 * u + 6] * inv, sv[8 * u + 7] * inv);
+      *reinterpret_cast<uint4*>(sP + (u >> 3) * L::kChunk + r * 128 + (((u & 7) ^ (r & 7)) << 4)) =
+          pk;
+    }
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  ok = __syncthreads_and(ok);
+  if (ok && tid == 0) {
+    tc_fence_after();
+    // keys x (d + 64) over the 128 rows, 16 rows per instruction
+    const uint64_t dp = desc_mnmajor(smem_u32(sP), L::kChunk);
+    const uint64_t dq = desc_mnmajor(smem_u32(sQ), L::kChunk);
+    const uint32_t idesc = idesc_bf16(kRows, D + 64, true, true);
+#pragma unroll
+    for (int kk = 0; kk < kRows / 16; ++kk)
+      mma_bf16_ss(tmem, dp + ((kk * 16 * 128) >> 4), dq + ((kk * 16 * 128) >> 4), idesc,
+                  kk > 0 ? 1u : 0u);
+    mma_commit(o_full);
+    issued_o = true;
+  }
+  // ---- epilogue, thread = key m = k c2 + q ----
+  if (ok) ok = mbar_wait(o_full, 0, abort_flag, a.status);
+  ok = __syncthreads_and(ok);
+  if (ok) {
+    tc_fence_after();
+    const int m = tid;
+    float cs[32];
+    tmem_ld32(tmem + lane_off + D, cs);
+    tmem_wait_ld();
+    const float invc = cs[0] > 0.f ? 1.f / cs[0] : 0.f;
+    const int k = m / a.c2, q = m % a.c2;
+    bf16* dst = a.qt + (((((long)g * a.b1 + k) * a.c1 + p) * a.c2 + q) * a.b2 + i) * D;
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      float t[32];
+      tmem_ld32(tmem + lane_off + c * 32, t);
+      tmem_wait_ld();
+      if (m < a.nk) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          uint4 pk;
+          pk.x = pack_bf16x2(t[8 * u + 0] * invc, t[8 * u + 1] * invc);
+          pk.y = pack_bf16x2(t[8 * u + 2] * invc, t[8 * u + 3] * invc);
+          pk.z = pack_bf16x2(t[8 * u + 4] * invc, t[8 * u + 5] * invc);
+          pk.w = pack_bf16x2(t[8 * u + 6] * invc, t[8 * u + 7] * invc);
+          *reinterpret_cast<uint4*>(dst + c * 32 + 8 * u) = pk;
+        }
+      }
+    }
+  }
+  if (tid == 0 && *abort_flag) {  // drain what this CTA issued (bounded)
+    if (!issued_s) drain(load_full, 0);
+    if (issued_s) drain(s_full, 0);
+    if (issued_o) drain(o_full, 0);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
   }
 }
 
@@ -1961,10 +2200,12 @@ cudaError_t launch_kr(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, b
   });
 }
 
+// qt_per_item: the queries are the per-sub-item rows of a later step (else
+// step one's Qt0); write_y: this is the last step (Y is written too).
 template <int D, int NQ, bool PAIR>
 cudaError_t launch_kr2(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, bf16* y,
                        float* hs, const Problem& pb, int* status, cudaStream_t stream,
-                       int* launches) {
+                       int* launches, bool qt_per_item = false, bool write_y = false) {
   using L = KR2Layout<D, NQ, PAIR>;
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
@@ -1976,7 +2217,8 @@ cudaError_t launch_kr2(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, 
   CUtensorMap tq, tk, tv, tkt, tyy;
   {
     // paired tiles load each sub-item's b2 (<= 64) query rows as a 64-row box
-    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)pb.G * pb.c1 * pb.b2};
+    const cuuint64_t rows = (cuuint64_t)pb.G * pb.c1 * pb.b2 * (qt_per_item ? pb.b1 * pb.c2 : 1);
+    const cuuint64_t dims[2] = {(cuuint64_t)D, rows};
     const cuuint64_t str[1] = {(cuuint64_t)D * 2};
     const cuuint32_t box[2] = {64, PAIR ? 64u : (cuuint32_t)kRows};
     if (!make_map(&tq, qt0, 2, dims, str, box)) return cudaErrorInvalidValue;
@@ -2015,8 +2257,10 @@ cudaError_t launch_kr2(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, 
   a.c2 = pb.c2;
   const long items = (long)pb.G * pb.c1 * pb.b1;
   if (items * pb.c2 >= (1L << 31)) return cudaErrorInvalidValue;
+  if ((long)pb.G * pb.c1 * pb.b2 * pb.b1 * pb.c2 >= (1L << 31)) return cudaErrorInvalidValue;
   a.n_items = (int)items;
-  a.write_y = pb.T == 1 ? 1 : 0;
+  a.write_y = (qt_per_item ? write_y : pb.T == 1) ? 1 : 0;
+  a.qt_per_item = qt_per_item ? 1 : 0;
   a.sc_log2 = kLog2e * pb.sc;
   a.status = status;
   a.real_lo = pb.real_lo;
@@ -2033,6 +2277,82 @@ cudaError_t launch_kr2(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, 
 // to 16, the K step of one tcgen05.mma.
 inline int kr_group_tile(const Problem& pb) {
   return ((pb.b2 + pb.c2 - 1) / pb.c2 + 15) / 16 * 16;
+}
+
+template <int D>
+cudaError_t launch_kl(const bf16* q, const bf16* kt, const float* hs, bf16* qt, const Problem& pb,
+                      int* status, cudaStream_t stream, int* launches) {
+  using L = KLLayout<D>;
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err =
+        cudaFuncSetAttribute(kl_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  const int nk = pb.b1 * pb.c2;
+  const long key_rows = (long)pb.G * pb.b2 * pb.c1 * nk;
+  CUtensorMap tq, tk;
+  {
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)pb.b2, (cuuint64_t)pb.G * pb.b1};
+    const cuuint64_t str[2] = {(cuuint64_t)D * 2, (cuuint64_t)pb.b2 * D * 2};
+    const cuuint32_t box[3] = {64, 1, kRows};
+    if (!make_map(&tq, q, 3, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)key_rows};
+    const cuuint64_t str[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64, 128};
+    if (!make_map(&tk, kt, 2, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  KLArgs a;
+  a.hs = hs;
+  a.qt = qt;
+  a.b1 = pb.b1;
+  a.b2 = pb.b2;
+  a.c1 = pb.c1;
+  a.c2 = pb.c2;
+  a.nk = nk;
+  a.real_lo = pb.real_lo;
+  a.real_hi = pb.real_hi;
+  a.sc = pb.sc;
+  a.status = status;
+  const long blocks = (long)pb.G * pb.b2 * pb.c1;
+  return timed_launch("tc_l_update", stream, launches, [&] {
+    return launch_pdl(kl_kernel<D>, dim3((unsigned)blocks), dim3(128), L::kBytes, stream, tq, tk,
+                      a);
+  });
+}
+
+// Steps >= 2 run on the tensor cores when the L-update fits one tile each
+// way (rows of <= 128 keys, row groups of <= 128 rows) and the R-update's
+// column groups take the persistent kernel (<= 64 keys).
+bool tc_later_steps(const Problem& pb) {
+  return pb.b1 * pb.c2 <= 128 && (pb.b1 + pb.c1 - 1) / pb.c1 <= kRows && kr_group_tile(pb) <= 64;
+}
+
+// One later step: the non-final L-update (aggregated queries Qt of every
+// sub-item), then the R-update from them.
+template <int D>
+cudaError_t launch_later_step(const bf16* q, const bf16* k, const bf16* v, bf16* qt, bf16* kt,
+                              bf16* y, float* hs, const Problem& pb, bool last, int* status,
+                              cudaStream_t stream, int* launches) {
+  cudaError_t e = launch_kl<D>(q, kt, hs, qt, pb, status, stream, launches);
+  if (e != cudaSuccess) return e;
+  switch (kr_group_tile(pb)) {
+#define MONARCH_KR2_STEP(NQ)                                                                   \
+  case NQ:                                                                                     \
+    return pb.b2 <= 64 ? launch_kr2<D, NQ, true>(qt, k, v, kt, y, hs, pb, status, stream,     \
+                                                 launches, true, last)                         \
+                       : launch_kr2<D, NQ, false>(qt, k, v, kt, y, hs, pb, status, stream,    \
+                                                  launches, true, last);
+    MONARCH_KR2_STEP(16)
+    MONARCH_KR2_STEP(32)
+    MONARCH_KR2_STEP(48)
+    MONARCH_KR2_STEP(64)
+#undef MONARCH_KR2_STEP
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 // Step one: aggregated queries under the uniform L, then the R-update (the
@@ -2132,7 +2452,17 @@ cudaError_t tc_forward(const bf16* q, const bf16* k, const bf16* v, bf16* out, c
   const QtStrides s1 = {(long)pb.b1 * pb.c1 * pb.c2 * pb.b2 * pb.d,
                         (long)pb.c1 * pb.c2 * pb.b2 * pb.d, (long)pb.c2 * pb.b2 * pb.d,
                         (long)pb.b2 * pb.d, (long)pb.d};
+  const bool tc_steps = tc_later_steps(pb);
+  bf16* qt = reinterpret_cast<bf16*>(ws.qt);  // bf16 rows in the fp32-sized piece
   for (int t = 2; t <= pb.T; ++t) {
+    if (tc_steps) {
+      e = pb.d == 128 ? launch_later_step<128>(q, k, v, qt, kt, y, ws.hs, pb, t == pb.T, status,
+                                               stream, launches)
+                      : launch_later_step<64>(q, k, v, qt, kt, y, ws.hs, pb, t == pb.T, status,
+                                              stream, launches);
+      if (e != cudaSuccess) return e;
+      continue;
+    }
     e = simt_l_update<bf16, bf16>(q, kt, ws.hs, ws.lse, ws.qt, pb, stream, launches);
     if (e != cudaSuccess) return e;
     e = simt_r_update<bf16, bf16>(k, v, ws.qt, s1, kt, y, ws.hs, pb, t == pb.T, stream, launches);

@@ -299,10 +299,14 @@ __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t saddr, uint32_t mn_blo
 }
 
 // Instruction descriptor, kind::f16: bf16 A and B, fp32 accumulator, dense.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major) {
+// A is K-major unless a_mn_major (then its M elements are contiguous, the
+// layout desc_mnmajor describes); likewise B.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major,
+                                                  bool a_mn_major = false) {
   return (1u << 4)                          // D format f32
          | (1u << 7)                        // A format bf16
          | (1u << 10)                       // B format bf16
+         | ((a_mn_major ? 1u : 0u) << 15)   // A major
          | ((b_mn_major ? 1u : 0u) << 16)   // B major
          | ((uint32_t)(N >> 3) << 17)       // N / 8
          | ((uint32_t)(M >> 4) << 24);      // M / 16

@@ -221,3 +221,34 @@ def test_injected_allocation_failure_is_reported_and_recovers(cuda_lib, monkeypa
     monkeypatch.delenv("MONARCH_ATTN_FAIL_ALLOC")
     O = gpu_forward(cuda_lib, q, k, v, 8, 8, 1)
     assert_parity(O, oracle_forward(q, k, v, 8, 8, 1), v, torch.bfloat16)
+
+
+# Later steps (T >= 2) on the tensor cores: the non-final L-update with the
+# aggregation L^T Q, then R-updates from per-sub-item queries.  Each case must
+# match the oracle and must not launch any SIMT kernel.
+LATER_STEPS = [
+    # B, H, b1, b2, d, T, c1, c2, inputs
+    (1, 2, 90, 52, 128, 2, 1, 1, "video"),   # the 480p latent (3, 30, 52), paired R tiles
+    (1, 2, 90, 52, 128, 3, 1, 1, "video"),
+    (1, 3, 64, 64, 64, 2, 1, 1, "iid"),      # sweep 4K shape
+    (1, 2, 60, 80, 128, 2, 1, 2, "iid"),     # unpaired R tiles (80 positions, 40-key groups)
+    (2, 2, 40, 48, 64, 3, 2, 2, "iid"),      # tiled, three steps
+    (1, 2, 45, 20, 128, 2, 3, 2, "iid"),     # tiled with 15-row groups
+]
+
+
+@pytest.mark.parametrize("B,H,b1,b2,d,T,c1,c2,kind", LATER_STEPS)
+def test_later_steps_on_tensor_cores(cuda_lib, B, H, b1, b2, d, T, c1, c2, kind):
+    if kind == "video":
+        q, k, v = video_qkv(B, H, (3, 30, 52), d, torch.bfloat16, seed=3)
+    else:
+        q, k, v = iid_qkv(B, H, b1 * b2, d, torch.bfloat16, seed=b1 + b2 + T)
+    cuda_lib.timing_read()
+    cuda_lib.timing_enable(True)
+    try:
+        O = gpu_forward(cuda_lib, q, k, v, b1, b2, T, c1, c2)
+        names = set(cuda_lib.timing_read())
+    finally:
+        cuda_lib.timing_enable(False)
+    assert "tc_l_update" in names and not any(n.startswith("simt") for n in names), names
+    assert_parity(O, oracle_forward(q, k, v, b1, b2, T, c1, c2), v, torch.bfloat16)
