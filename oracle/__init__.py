@@ -13,6 +13,7 @@ from .monarch_ref import (  # noqa: F401
     groups,
     materialise,
     monarch_attention,
+    monarch_attention_backward,
     objective,
     objective_dense,
     output,

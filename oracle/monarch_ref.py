@@ -405,3 +405,83 @@ def monarch_attention(q, k, v, b1, b2, T, c1=1, c2=1, return_state=False, n_pad=
     if return_state:
         return O, dict(L=L, R=rf, q=qh, k=kh, v=vh, rows=rows, cols=cols, sc=sc, real=real)
     return O
+
+
+# ----------------------------------------------------------------------------
+# the backward pass (T = 1)
+# ----------------------------------------------------------------------------
+def monarch_attention_backward(q, k, v, dO, b1, b2, c1=1, c2=1):
+    """Gradients (dq, dk, dv) of sum(O * dO) for the T = 1 forward pass.
+
+    One refinement step is what the pages finetune with (MonarchRT summary:
+    finetuning collapses the refinement to one iteration; forward and
+    backward kernels).  The chain rule through the steps of the forward pass,
+    in reverse:
+
+      O_(l,i) = sum_{k,q} L Y                  dY  = sum_{l in p} L dO_(l,i)
+                                               dL  = dO_(l,i) . Y
+      L = softmax_{(k,q)}(S_L)                 dS_L = L (dL - sum_{k,q} L dL)
+      S_L = sc q . Kt + Hs                     dq += sc sum_{k,q} dS_L Kt
+                                               dKt = sc sum_{l in p} dS_L q_(l,i)
+                                               dHs = sum_{l in p} dS_L
+      Kt, Y, Hs from R (per (k,p,q,i))         dR_j = dKt . k_j + dY . v_j - dHs (ln R_j + 1)
+      R = softmax_{j in q}(S_R)                dS_R = R (dR - sum_j R dR)
+      S_R = sc Qt0 . k_(k,j)                   dk_j += sum R dKt + sc sum dS_R Qt0
+                                               dv_j += sum R dY
+                                               dQt0 = sc sum_{k,j} dS_R k_j
+      Qt0_{p,i} = mean_{l in p} q_(l,i)        dq_(l,i) += dQt0_{p(l),i} / |p|
+
+    q, k, v, dO: (..., N, d) with N = b1*b2.  Returns float64 arrays of the
+    same shapes.
+    """
+    O, st = monarch_attention(q, k, v, b1, b2, 1, c1, c2, return_state=True)
+    L, rf, qh, kh, vh = st["L"], st["R"], st["q"], st["k"], st["v"]
+    rows, cols, sc = st["rows"], st["cols"], st["sc"]
+    G, _, _, d = qh.shape
+    dOh = np.asarray(dO, dtype=np.float64).reshape(G, b1, b2, -1)
+    Oh = np.asarray(O).reshape(G, b1, b2, -1)
+    nk = b1 * c2
+    dq = np.zeros_like(qh)
+    dKt = np.zeros_like(rf.Kt)                     # (G, k, p, q, i, d)
+    dY = np.zeros_like(rf.Y)
+    dHs = np.zeros_like(rf.Hs)                     # (G, k, p, q, i)
+    # ---- L side, one position i and row group p at a time ----
+    for i in range(b2):
+        Lb = L.block(i)                                          # (G, l, k, q)
+        for pi, (l0, l1) in enumerate(rows):
+            Lp = Lb[:, l0:l1].reshape(G, l1 - l0, nk)            # (G, l, kq)
+            Kt = rf.Kt[:, :, pi, :, i].reshape(G, nk, d)         # (G, kq, d)
+            Yp = rf.Y[:, :, pi, :, i].reshape(G, nk, -1)
+            g = dOh[:, l0:l1, i]                                 # (G, l, dv)
+            dL = g @ np.swapaxes(Yp, -1, -2)                     # (G, l, kq)
+            delta = (g * Oh[:, l0:l1, i]).sum(-1, keepdims=True)  # sum_{kq} L dL = dO . O
+            dS = Lp * (dL - delta)
+            dq[:, l0:l1, i] += sc * (dS @ Kt)
+            dKt[:, :, pi, :, i] = (sc * (np.swapaxes(dS, -1, -2) @ qh[:, l0:l1, i])
+                                   ).reshape(G, b1, c2, d)
+            dHs[:, :, pi, :, i] = dS.sum(axis=1).reshape(G, b1, c2)
+            dY[:, :, pi, :, i] = (np.swapaxes(Lp, -1, -2) @ g).reshape(G, b1, c2, -1)
+    # ---- R side: every (k, p, q, i) row over j in q ----
+    dk = np.zeros_like(kh)
+    dv = np.zeros_like(vh)
+    dQt0 = np.zeros((G, len(rows), b2, d))
+    Qt0 = np.stack([qh[:, l0:l1].mean(axis=1) for l0, l1 in rows], axis=1)  # (G, p, i, d)
+    for pi in range(len(rows)):
+        for qi, (j0, j1) in enumerate(cols):
+            R = rf.R[:, :, pi, :, j0:j1]                         # (G, k, i, j)
+            kq, vq = kh[:, :, j0:j1], vh[:, :, j0:j1]            # (G, k, j, d)
+            a = dKt[:, :, pi, qi]                                # (G, k, i, d)
+            y = dY[:, :, pi, qi]
+            h = dHs[:, :, pi, qi][..., None]                     # (G, k, i, 1)
+            with np.errstate(divide="ignore"):
+                lnR = np.where(R > 0, np.log(np.where(R > 0, R, 1.0)), 0.0)
+            dR = a @ np.swapaxes(kq, -1, -2) + y @ np.swapaxes(vq, -1, -2) - h * (lnR + 1.0)
+            dS = R * (dR - (R * dR).sum(-1, keepdims=True))     # (G, k, i, j)
+            dk[:, :, j0:j1] += np.swapaxes(R, -1, -2) @ a + \
+                sc * (np.swapaxes(dS, -1, -2) @ Qt0[:, None, pi])
+            dv[:, :, j0:j1] += np.swapaxes(R, -1, -2) @ y
+            dQt0[:, pi] += sc * np.einsum("gkij,gkjd->gid", dS, kq)
+    for pi, (l0, l1) in enumerate(rows):
+        dq[:, l0:l1] += dQt0[:, pi][:, None] / (l1 - l0)
+    shape = np.asarray(q).shape
+    return (dq.reshape(shape), dk.reshape(np.asarray(k).shape), dv.reshape(np.asarray(v).shape))
