@@ -196,6 +196,26 @@ MONARCH_API int monarch_attn_fwd_padded(int dtype, const void* q, const void* k,
                                         int pad_front, int d, int T, int c1, int c2,
                                         cudaStream_t stream);
 
+/* Backward pass of the T = 1 forward (one refinement step, the setting the
+ * pages finetune with: MonarchRT summary, "Method" (3), forward and
+ * backward kernels): dq, dk, dv = gradients of sum(O * dout) with respect
+ * to q, k, v, where O = monarch_attn_fwd / _f32(q, k, v, ..., T = 1).
+ *
+ * dtype: MONARCH_DTYPE_BF16 or MONARCH_DTYPE_F32; all seven pointers are
+ * device buffers of that type, (B, H, N, d) contiguous, N = b1*b2,
+ * 16-byte aligned; dq, dk, dv must not overlap each other or any input.
+ * Arithmetic is fp32 throughout (SIMT kernels); the forward intermediates
+ * are recomputed.  The library keeps a cached fp32 workspace per device of
+ * G (c1 b2 d + 5 N c1 c2 d + 2 N c1 c2 + N d + 2 N + 2 b1 c1 b2^2) floats
+ * (G = B*H; allocated on first use, grown on demand, freed by
+ * monarch_attn_release_workspace).  Deterministic (fixed-order reductions,
+ * no atomics).  Asynchronous on `stream`.  Errors as for monarch_attn_fwd;
+ * T other than 1 returns MONARCH_ERR_UNSUPPORTED. */
+MONARCH_API int monarch_attn_bwd(int dtype, const void* q, const void* k, const void* v,
+                                 const void* dout, void* dq, void* dk, void* dv, int B, int H,
+                                 int b1, int b2, int d, int T, int c1, int c2,
+                                 cudaStream_t stream);
+
 /* Bytes of device workspace a call with these arguments uses (0 on invalid
  * arguments).  dtype is MONARCH_DTYPE_BF16 or MONARCH_DTYPE_F32. */
 MONARCH_API size_t monarch_attn_workspace_bytes(int B, int H, int b1, int b2, int d, int T,

@@ -37,6 +37,7 @@ SIGNATURES = {
                                     _I, _P]),
     "monarch_attn_fwd_padded": (_I, [_I, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I,
                                      _I, _P]),
+    "monarch_attn_bwd": (_I, [_I, _P, _P, _P, _P, _P, _P, _P, *_SIZES, _P]),
     "monarch_attn_workspace_bytes": (_Z, [*_SIZES, _I]),
     "monarch_attn_release_workspace": (None, []),
     "monarch_attn_check": (_I, [_P]),
@@ -171,6 +172,24 @@ def monarch_attn_fwd_padded(q, k, v, b1, b2, T, c1=1, c2=1, pad_front=True, out=
                                        out.data_ptr(), B, H, n_real, b1, b2,
                                        1 if pad_front else 0, d, T, c1, c2, _stream_ptr(stream)))
     return out
+
+
+def monarch_attn_bwd(q, k, v, dout, b1, b2, T=1, c1=1, c2=1, stream=None):
+    """Gradients (dq, dk, dv) of sum(O * dout) for the T = 1 forward pass on
+    device tensors (B, H, N, d), N = b1*b2, bf16 or fp32."""
+    lib = load_library()
+    B, H, d = _dims(q, b1, b2)
+    for t in (q, k, v, dout):
+        if t.shape != q.shape or t.dtype != q.dtype or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v, dout must be contiguous CUDA tensors of one shape and dtype")
+    dtype = {torch.bfloat16: DTYPE_BF16, torch.float32: DTYPE_F32}.get(q.dtype)
+    if dtype is None:
+        raise ValueError(f"unsupported dtype {q.dtype}")
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    _check(lib.monarch_attn_bwd(dtype, q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(),
+                                dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, b1, b2, d, T,
+                                c1, c2, _stream_ptr(stream)))
+    return dq, dk, dv
 
 
 def video_blocks(f, h, w, layout):

@@ -1,0 +1,28 @@
+// Host-side interface of the backward-pass kernels (T = 1).
+#pragma once
+
+#include <stddef.h>
+
+#include "common.cuh"
+
+namespace monarch {
+
+// fp32 workspace pieces (element counts); layouts in bwd_kernels.cu.
+struct BwdWorkspaceSizes {
+  size_t qt0, kt, y, hs, lse, delta, dq1, dkt, dy, dhs, rbuf, dsbuf, dqt0_part;
+};
+
+struct BwdWorkspace {
+  float *qt0, *kt, *y, *hs, *lse, *delta, *dq1, *dkt, *dy, *dhs, *rbuf, *dsbuf, *dqt0_part;
+};
+
+BwdWorkspaceSizes bwd_workspace_sizes(const Problem& pb);
+
+// Gradients dq, dk, dv of sum(O * dout) for the forward pass with T = 1
+// (unpadded), on `stream`; adds its launch count to *launches.
+template <typename TIn>
+cudaError_t bwd_forward_t1(const TIn* q, const TIn* k, const TIn* v, const TIn* dout, TIn* dq,
+                           TIn* dk, TIn* dv, const Problem& pb, const BwdWorkspace& ws,
+                           cudaStream_t stream, int* launches);
+
+}  // namespace monarch

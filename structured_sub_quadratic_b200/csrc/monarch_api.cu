@@ -13,6 +13,7 @@
 #include <mutex>
 #include <vector>
 
+#include "bwd_kernels.cuh"
 #include "entry.cuh"
 #include "layout.cuh"
 #include "simt_kernels.cuh"
@@ -45,6 +46,7 @@ DevBuf g_ws[kMaxDevices];      // kernel workspace
 DevBuf g_stage[kMaxDevices];   // staging for the host-buffer entry point
 DevBuf g_layout[kMaxDevices];  // reordered q, k, v and output of the video-layout entry point
 DevBuf g_pad[kMaxDevices];     // padded q, k, v and output of the padded entry point
+DevBuf g_bwd[kMaxDevices];     // workspace of the backward pass
 
 // Raster index tables of the video layouts used so far, per device (uploaded
 // once per (f, h, w, layout); guarded by g_layout_mu).
@@ -487,6 +489,63 @@ int monarch_attn_fwd_padded(int dtype, const void* q, const void* k, const void*
   return MONARCH_OK;
 }
 
+int monarch_attn_bwd(int dtype, const void* q, const void* k, const void* v, const void* dout,
+                     void* dq, void* dk, void* dv, int B, int H, int b1, int b2, int d, int T,
+                     int c1, int c2, cudaStream_t stream) {
+  t_launches = 0;
+  if (dtype != MONARCH_DTYPE_BF16 && dtype != MONARCH_DTYPE_F32) return MONARCH_ERR_INVALID_ARG;
+  int st = monarch::validate_args(B, H, b1, b2, d, T, c1, c2);
+  if (st != MONARCH_OK) return st;
+  if (T != 1) return MONARCH_ERR_UNSUPPORTED;
+  for (const void* ptr : {q, k, v, dout, (const void*)dq, (const void*)dk, (const void*)dv})
+    if (!aligned16(ptr)) return MONARCH_ERR_INVALID_ARG;
+  const Problem pb = monarch::make_problem(B, H, b1, b2, d, T, c1, c2);
+  const size_t bytes_io = (size_t)pb.G * b1 * b2 * d * (dtype == MONARCH_DTYPE_BF16 ? 2 : 4);
+  const void* ins[4] = {q, k, v, dout};
+  const void* outs[3] = {dq, dk, dv};
+  for (const void* o : outs)
+    for (const void* in : ins) {
+      const char *o0 = static_cast<const char*>(o), *i0 = static_cast<const char*>(in);
+      if (o0 < i0 + bytes_io && i0 < o0 + bytes_io) return MONARCH_ERR_INVALID_ARG;
+    }
+  for (int a = 0; a < 3; ++a)
+    for (int b = a + 1; b < 3; ++b) {
+      const char *x = static_cast<const char*>(outs[a]), *y = static_cast<const char*>(outs[b]);
+      if (x < y + bytes_io && y < x + bytes_io) return MONARCH_ERR_INVALID_ARG;
+    }
+  int dev;
+  if ((st = current_device(&dev)) != MONARCH_OK) return st;
+  const monarch::BwdWorkspaceSizes sz = monarch::bwd_workspace_sizes(pb);
+  const size_t* f = &sz.qt0;
+  constexpr int kPieces = sizeof(sz) / sizeof(size_t);
+  size_t total = 0;
+  for (int t = 0; t < kPieces; ++t) total += align_up(f[t] * sizeof(float));
+  std::lock_guard<std::mutex> lock(g_mu);
+  if ((st = ensure(g_bwd[dev], total)) != MONARCH_OK) return st;
+  monarch::BwdWorkspace ws;
+  float** dst = &ws.qt0;
+  char* base = static_cast<char*>(g_bwd[dev].ptr);
+  size_t off = 0;
+  for (int t = 0; t < kPieces; ++t) {
+    dst[t] = reinterpret_cast<float*>(base + off);
+    off += align_up(f[t] * sizeof(float));
+  }
+  using monarch::bf16;
+  const cudaError_t e =
+      dtype == MONARCH_DTYPE_BF16
+          ? monarch::bwd_forward_t1<bf16>(
+                static_cast<const bf16*>(q), static_cast<const bf16*>(k),
+                static_cast<const bf16*>(v), static_cast<const bf16*>(dout),
+                static_cast<bf16*>(dq), static_cast<bf16*>(dk), static_cast<bf16*>(dv), pb, ws,
+                stream, &t_launches)
+          : monarch::bwd_forward_t1<float>(
+                static_cast<const float*>(q), static_cast<const float*>(k),
+                static_cast<const float*>(v), static_cast<const float*>(dout),
+                static_cast<float*>(dq), static_cast<float*>(dk), static_cast<float*>(dv), pb, ws,
+                stream, &t_launches);
+  return e == cudaSuccess ? MONARCH_OK : record_cuda(e);
+}
+
 size_t monarch_attn_workspace_bytes(int B, int H, int b1, int b2, int d, int T, int c1, int c2,
                                     int dtype) {
   if (monarch::validate_args(B, H, b1, b2, d, T, c1, c2) != MONARCH_OK) return 0;
@@ -503,19 +562,21 @@ void monarch_attn_release_workspace(void) {
   cudaGetDevice(&cur);
   for (int dev = 0; dev < kMaxDevices; ++dev) {
     if (!g_ws[dev].ptr && !g_stage[dev].ptr && !g_layout[dev].ptr && !g_pad[dev].ptr &&
-        g_tables[dev].empty())
+        !g_bwd[dev].ptr && g_tables[dev].empty())
       continue;
     cudaSetDevice(dev);
     if (g_ws[dev].ptr) cudaFree(g_ws[dev].ptr);
     if (g_stage[dev].ptr) cudaFree(g_stage[dev].ptr);
     if (g_layout[dev].ptr) cudaFree(g_layout[dev].ptr);
     if (g_pad[dev].ptr) cudaFree(g_pad[dev].ptr);
+    if (g_bwd[dev].ptr) cudaFree(g_bwd[dev].ptr);
     for (PermTable& t : g_tables[dev]) cudaFree(t.dev_table);
     g_tables[dev].clear();
     g_ws[dev] = DevBuf();
     g_stage[dev] = DevBuf();
     g_layout[dev] = DevBuf();
     g_pad[dev] = DevBuf();
+    g_bwd[dev] = DevBuf();
   }
   cudaSetDevice(cur);
 }

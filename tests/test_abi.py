@@ -130,3 +130,18 @@ def test_padded_entry_validates_before_any_launch(lib, dtype, n_real, pad_front,
     p = 1 << 20
     assert lib.monarch_attn_fwd_padded(dtype, p, 2 * p, 3 * p, 4 * p, 1, 1, n_real, 4, 4,
                                        pad_front, 64, 1, 1, 1, None) == expect
+
+
+def test_backward_entry_validates_before_any_launch(lib):
+    p = 1 << 20
+    sizes = (1, 1, 4, 4, 64)
+    # T other than 1
+    assert lib.monarch_attn_bwd(0, p, 2 * p, 3 * p, 4 * p, 5 * p, 6 * p, 7 * p, *sizes, 2, 1, 1,
+                                None) == api.MONARCH_ERR_UNSUPPORTED
+    # dq overlapping q, and dk overlapping dv
+    assert lib.monarch_attn_bwd(0, p, 2 * p, 3 * p, 4 * p, p + 256, 6 * p, 7 * p, *sizes, 1, 1,
+                                1, None) == api.MONARCH_ERR_INVALID_ARG
+    assert lib.monarch_attn_bwd(0, p, 2 * p, 3 * p, 4 * p, 5 * p, 6 * p, 6 * p + 16, *sizes, 1,
+                                1, 1, None) == api.MONARCH_ERR_INVALID_ARG
+    assert lib.monarch_attn_bwd(9, p, 2 * p, 3 * p, 4 * p, 5 * p, 6 * p, 7 * p, *sizes, 1, 1, 1,
+                                None) == api.MONARCH_ERR_INVALID_ARG

@@ -1,0 +1,55 @@
+"""GPU backward pass (T = 1) against the float64 oracle's chain rule.
+
+The oracle's backward is pinned by finite differences and by dense-attention
+gradients (tests/test_oracle_backward.py).  The GPU computes in fp32 from the
+same input values, so the bar is max|g_gpu - g_oracle| <= 1e-4 max|g_oracle|
+for fp32 inputs, and 2e-2 max|g_oracle| for bf16 inputs, where the gradients
+are rounded to bf16 on output (the forward pass's bars, relative to the
+gradient's scale instead of V's).
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import monarch_attention_backward
+from structured_sub_quadratic_b200.inputs import iid_qkv
+
+pytestmark = pytest.mark.gpu
+
+TOL = {torch.float32: 1e-4, torch.bfloat16: 2e-2}
+
+CASES = [
+    # B, H, b1, b2, d, c1, c2
+    (1, 2, 12, 10, 64, 1, 1),
+    (2, 2, 9, 8, 64, 2, 2),
+    (1, 1, 7, 9, 32, 3, 2),
+    (1, 1, 5, 6, 24, 1, 2),
+    (1, 2, 16, 16, 128, 1, 1),
+    (1, 1, 30, 52, 128, 1, 1),
+    (1, 1, 40, 40, 64, 2, 2),
+]
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("B,H,b1,b2,d,c1,c2", CASES)
+def test_backward_parity(cuda_lib, dtype, B, H, b1, b2, d, c1, c2):
+    q, k, v = iid_qkv(B, H, b1 * b2, d, dtype, seed=b1 * 31 + b2)
+    dO = iid_qkv(B, H, b1 * b2, d, dtype, seed=b1 * 31 + b2 + 1)[0]
+    got = cuda_lib.monarch_attn_bwd(q.cuda(), k.cuda(), v.cuda(), dO.cuda(), b1, b2, 1, c1, c2)
+    cuda_lib.check()
+    assert cuda_lib.last_launches() > 0
+    ref = monarch_attention_backward(*(x.double().numpy() for x in (q, k, v, dO)), b1, b2, c1, c2)
+    for name, g, r in zip(("dq", "dk", "dv"), got, ref):
+        g = g.double().cpu().numpy()
+        assert np.isfinite(g).all(), name
+        err, bound = np.abs(g - r).max(), TOL[dtype] * np.abs(r).max()
+        assert err <= bound, f"{name}: max err {err:.3e} > {bound:.3e}"
+
+
+def test_backward_is_deterministic(cuda_lib):
+    q, k, v = (x.cuda() for x in iid_qkv(1, 2, 30 * 52, 128, torch.bfloat16, seed=4))
+    dO = torch.randn_like(q)
+    a = cuda_lib.monarch_attn_bwd(q, k, v, dO, 30, 52, 1)
+    b = cuda_lib.monarch_attn_bwd(q, k, v, dO, 30, 52, 1)
+    torch.cuda.synchronize()
+    assert all(torch.equal(x, y) for x, y in zip(a, b))
