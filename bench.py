@@ -84,6 +84,7 @@ def kernel_work(name: str, wl: Workload):
       kernel          unit (count per launch)   FLOPs per unit          bytes per unit
       init_qt         (g, p, i)  G c1 b2        |p| d                   |p| d e   (Q rows)
       r_update        (g, k)     G b1           6 c1 b2^2 d (last step) 2 b2 d e  (K, V rows)
+      l_update        (g, i, p)  G b2 c1        4 |p| b1 c2 d           |p| d e   (Q rows)
       l_output        (g, i, p)  G b2 c1        4 |p| b1 c2 d           2 |p| d e (Q in, O out)
       small_head      head g     G              the whole forward       4 N d e
     """
@@ -97,6 +98,8 @@ def kernel_work(name: str, wl: Workload):
         return G * b1 * c1 * b2 * b2 * d * 2 * 3, 2 * io
     if name.endswith("l_output"):
         return G * N * b1 * c2 * d * 4, 2 * io
+    if name == "tc_l_update":  # logits + L^T Q of a non-final step
+        return G * N * b1 * c2 * d * 4, io
     if name.endswith("l_stats"):
         return G * N * b1 * c2 * d * 2, io
     if name.endswith("l_aggregate"):
