@@ -1179,7 +1179,8 @@ __global__ void __launch_bounds__(128)
 }
 
 // ---------------------------------------------------------------------------
-// Persistent R-update (step one) for column-group tiles NQ <= 64.  One CTA
+// Persistent R-update for column-group tiles NQ <= 64 (step one, and the
+// later steps with per-sub-item queries).  One CTA
 // per SM walks a contiguous range of sub-items (g, p, k, q): one item (g, p, k)
 // is split into c2 sub-items, one per column group q.  Warp 0 loads (Qt0, and
 // K_q / V_q through a ring of slots), warp 1 issues the MMAs, and two
@@ -1187,7 +1188,9 @@ __global__ void __launch_bounds__(128)
 // normalised before the MMA), then the Kt / Y rows through TMA bulk stores.
 // Each warpgroup owns one 2d-column TMEM slot in which S is later
 // overwritten by [Kt | Y], so tile t+1's S and softmax overlap tile t's
-// stores.
+// stores.  In the epilogue every warp stores its own 32 rows through a 4-D
+// box clipped at b2, staging them in its own rows of P (dead once the
+// [Kt | Y] product has read it), with no barrier across the warpgroup.
 //
 // Paired tiles (PAIR, b2 <= 64): the b2 positions of one sub-item fill only
 // half of the 128 TMEM lanes, so a tile carries two consecutive sub-items A
@@ -1196,9 +1199,7 @@ __global__ void __launch_bounds__(128)
 // is 128 x 2NQ and rows 0-63 use its first NQ columns, rows 64-127 its last
 // NQ.  P is block diagonal ([R_A 0; 0 R_B]), so one product with the stacked
 // [K | V] of both sub-items gives [Kt | Y] of A in rows 0-63 and of B in rows
-// 64-127.  Each warp then stores its own 32 rows with a 4-D TMA box (rows
-// clipped at b2), staging in its own rows of the P buffer, which is dead once
-// the product is done.
+// 64-127.
 //
 // Barriers (tile counter t over the CTA's tiles):
 //   q_full / q_empty       Qt0 tile        kv_full / kv_empty   K/V ring
@@ -1213,15 +1214,14 @@ struct KR2Layout {
   static constexpr int kBlk = kKeys * 128;                 // one 64-column block of K or V
   static constexpr int kKVBytes = 2 * (D / 64) * kBlk;     // K blocks, then V blocks
   static constexpr int kKVSlots = PAIR ? 2 : 3;
-  // P (K-major, 64-key chunks of 128 rows); paired tiles keep two chunks so
-  // that each warp finds two 4 KB staging buffers in its own rows.
-  static constexpr int kPBytes = (PAIR ? 2 : (kKeys + 63) / 64) * kRows * 128;
+  // P (K-major, 64-key chunks of 128 rows): two chunks, so that once the
+  // [Kt | Y] product has read P each warp finds two 4 KB staging buffers in
+  // its own 32 rows for the epilogue's stores.
+  static constexpr int kPBytes = 2 * kRows * 128;
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = D / 64 * kRows * 128;
   static constexpr int kPOff = kKVOff + kKVSlots * kKVBytes;       // [2 wg]
-  static constexpr int kStageOff = kPOff + 2 * kPBytes;            // [2 wg][2] x 16 KB
-  static constexpr int kStageBytes = PAIR ? 0 : 4 * kRows * 128;
-  static constexpr int kBarOff = kStageOff + kStageBytes;
+  static constexpr int kBarOff = kPOff + 2 * kPBytes;
   static constexpr int kBytes = kBarOff + 32 * 8;
   static_assert(NQ % 16 == 0 && NQ <= 64, "group tile");
   static_assert(kBytes <= 227 * 1024, "shared memory");
@@ -1307,7 +1307,6 @@ __global__ void __launch_bounds__(320, 1)
   uint8_t* sQ = smem + L::kQOff;
   auto sKV = [&](int sl) { return smem + L::kKVOff + sl * L::kKVBytes; };
   auto sP = [&](int w) { return smem + L::kPOff + w * L::kPBytes; };
-  auto sStage = [&](int w, int b) { return smem + L::kStageOff + (w * 2 + b) * kRows * 128; };
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
@@ -1521,11 +1520,8 @@ __global__ void __launch_bounds__(320, 1)
     const int r = quad * 32 + lane;           // TMEM lane == tile row
     const int h = PAIR ? (quad >> 1) : 0;     // which sub-item of the tile (warp-uniform)
     const int i = PAIR ? (r & 63) : r;        // position of this row
-    const int wtid = tid - 64 - w * 128;      // 0..127 inside the warpgroup
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t tslot = tmem + w * 256;
-    const bool leader = wtid == 0;
-    int nst = 0;  // unpaired tiles: stores issued by this warpgroup; buffer nst & 1
     bool ok = true;
     for (long t = w; t < ntiles && ok; t += 2) {
       const long n = s0 + t * H + h;
@@ -1553,10 +1549,10 @@ __global__ void __launch_bounds__(320, 1)
       // an absent sub-item, or a group without a real key, contributes P = 0
       const float inv = (have && z > 0.f) ? 1.f / z : 0.f;
       uint8_t* pbuf = sP(w);
-      if (PAIR) {  // this warp's rows of P were the previous tile's staging: stores must have read them
-        if (lane == 0) bulk_wait_read<0>();
-        __syncwarp();
-      }
+      // this warp's rows of P were the previous tile's staging: its stores
+      // must have read them
+      if (lane == 0) bulk_wait_read<0>();
+      __syncwarp();
       // P holds R itself (normalised), so [Kt | Y] comes out of the MMA final.
       // Paired tiles: this row's R in its own half of the columns, zeros in
       // the other half.
@@ -1585,100 +1581,63 @@ __global__ void __launch_bounds__(320, 1)
       const int ycoord = (sb.p * a.b1 + sb.k) * a.c2 + sb.q;
       const bool row_ok = have && i < a.b2;
       const long orow_w = ((((long)sb.g * a.b2 + i) * a.c1 + sb.p) * a.b1 + sb.k) * a.c2 + sb.q;
-      if constexpr (PAIR) {
-        // Each warp stores its own 32 rows (positions i0 .. i0 + 31 of its
-        // sub-item) through a 4-D box clipped at b2, staging in its own rows
-        // of the P buffer (two 4 KB buffers, one per 64-key chunk).
-        const int i0 = (quad & 1) * 32;
-        const bool store = have && i0 < a.b2;  // warp-uniform
-        if (!store) {
-          tc_fence_before();
-          mbar_arrive(tmem_free + w);
-        } else {
-          // TMEM loads run one 32-column unit ahead of the staging: unit
-          // u + 1 is in flight while unit u is packed into its 64-column
-          // block's staging rows; a block goes out once both halves are in.
-          float rs[2][32];
-          tmem_ld32(tslot + lane_off, rs[0]);
+      // Each warp stores its own 32 rows (positions i0 .. i0 + 31 of its
+      // sub-item) through a 4-D box clipped at b2, staging in its own rows
+      // of the P buffer (two 4 KB buffers, one per 64-key chunk); a warp
+      // whose rows all lie past b2 stores nothing.
+      const int i0 = PAIR ? (quad & 1) * 32 : quad * 32;
+      const bool store = have && i0 < a.b2;  // warp-uniform
+      if (!store) {
+        tc_fence_before();
+        mbar_arrive(tmem_free + w);
+      } else {
+        // TMEM loads run one 32-column unit ahead of the staging: unit
+        // u + 1 is in flight while unit u is packed into its 64-column
+        // block's staging rows; a block goes out once both halves are in.
+        float rs[2][32];
+        tmem_ld32(tslot + lane_off, rs[0]);
 #pragma unroll
-          for (int u = 0; u < 4 * (D / 64); ++u) {
-            if (u < 2 * nblk) {
-              const int cb = u >> 1, hf = u & 1;
-              tmem_wait_ld();  // unit u is in registers
-              if (u == 2 * nblk - 1) {  // slot fully read out: the MMA may reuse it
-                tc_fence_before();
-                mbar_arrive(tmem_free + w);
-              } else {
-                tmem_ld32(tslot + lane_off + (u + 1) * 32, rs[(u + 1) & 1]);
-              }
-              uint8_t* buf = pbuf + (cb & 1) * (kRows * 128) + quad * 32 * 128;
-              if (hf == 0) {
-                if (cb >= 2 && lane == 0) bulk_wait_read<1>();  // store of block cb-2 has read buf
-                __syncwarp();
-              }
+        for (int u = 0; u < 4 * (D / 64); ++u) {
+          if (u < 2 * nblk) {
+            const int cb = u >> 1, hf = u & 1;
+            tmem_wait_ld();  // unit u is in registers
+            if (u == 2 * nblk - 1) {  // slot fully read out: the MMA may reuse it
+              tc_fence_before();
+              mbar_arrive(tmem_free + w);
+            } else {
+              tmem_ld32(tslot + lane_off + (u + 1) * 32, rs[(u + 1) & 1]);
+            }
+            uint8_t* buf = pbuf + (cb & 1) * (kRows * 128) + quad * 32 * 128;
+            if (hf == 0) {
+              if (cb >= 2 && lane == 0) bulk_wait_read<1>();  // store of block cb-2 has read buf
+              __syncwarp();
+            }
 #pragma unroll
-              for (int uu = 0; uu < 4; ++uu) {
-                const float* v = rs[u & 1] + 8 * uu;
-                uint4 pk;
-                pk.x = pack_bf16x2(v[0], v[1]);
-                pk.y = pack_bf16x2(v[2], v[3]);
-                pk.z = pack_bf16x2(v[4], v[5]);
-                pk.w = pack_bf16x2(v[6], v[7]);
-                const int chunk = hf * 4 + uu;
-                *reinterpret_cast<uint4*>(buf + lane * 128 + ((chunk ^ (lane & 7)) << 4)) = pk;
-              }
-              if (hf == 1) {
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                  tma_store_4d(cb < D / 64 ? &tm_kt : &tm_y, buf, (cb % (D / 64)) * 64, ycoord,
-                               i0, sb.g);
-                  bulk_commit();
-                }
+            for (int uu = 0; uu < 4; ++uu) {
+              const float* v = rs[u & 1] + 8 * uu;
+              uint4 pk;
+              pk.x = pack_bf16x2(v[0], v[1]);
+              pk.y = pack_bf16x2(v[2], v[3]);
+              pk.z = pack_bf16x2(v[4], v[5]);
+              pk.w = pack_bf16x2(v[6], v[7]);
+              const int chunk = hf * 4 + uu;
+              *reinterpret_cast<uint4*>(buf + lane * 128 + ((chunk ^ (lane & 7)) << 4)) = pk;
+            }
+            if (hf == 1) {
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_4d(cb < D / 64 ? &tm_kt : &tm_y, buf, (cb % (D / 64)) * 64, ycoord,
+                             i0, sb.g);
+                bulk_commit();
               }
             }
-          }
-        }
-      } else {
-        // The b2 rows of this (g, p, k, q) are positions i of the position-major
-        // Kt/Y layout: one 3-D TMA box {64 columns, 1, b2 rows}.  Each 64-column
-        // block is staged (swizzled) in one of two buffers and handed to a TMA
-        // bulk store; a buffer is refilled once its previous store has read it.
-#pragma unroll 1
-        for (int cb = 0; cb < nblk; ++cb, ++nst) {
-          uint8_t* buf = sStage(w, nst & 1);
-          float ta[32], tb[32];
-          tmem_ld32(tslot + lane_off + cb * 64, ta);
-          tmem_ld32(tslot + lane_off + cb * 64 + 32, tb);
-          if (leader) bulk_wait_read<1>();  // the store that last used buf has read it
-          named_barrier(1 + w, 128);
-          tmem_wait_ld();
-          if (cb == nblk - 1) {  // slot fully read out: the MMA may reuse it
-            tc_fence_before();
-            mbar_arrive(tmem_free + w);
-          }
-#pragma unroll
-          for (int uu = 0; uu < 8; ++uu) {
-            const float* v = uu < 4 ? ta + 8 * uu : tb + 8 * (uu - 4);
-            uint4 pk;
-            pk.x = pack_bf16x2(v[0], v[1]);
-            pk.y = pack_bf16x2(v[2], v[3]);
-            pk.z = pack_bf16x2(v[4], v[5]);
-            pk.w = pack_bf16x2(v[6], v[7]);
-            *reinterpret_cast<uint4*>(buf + r * 128 + ((uu ^ (r & 7)) << 4)) = pk;
-          }
-          fence_proxy_async_smem();
-          named_barrier(1 + w, 128);
-          if (leader) {
-            tma_store_3d(cb < D / 64 ? &tm_kt : &tm_y, buf, (cb % (D / 64)) * 64, ycoord,
-                         sb.g * a.b2);
-            bulk_commit();
           }
         }
       }
       if (row_ok) a.hs[orow_w] = z > 0.f ? logf(z) - t2 * 0.69314718055994531f / z : -INFINITY;
     }
-    if (PAIR ? lane == 0 : leader) bulk_wait<0>();  // stores done reading shared memory before exit
+    if (lane == 0) bulk_wait<0>();  // stores done reading shared memory before exit
   }
   tc_fence_before();
   __syncthreads();
@@ -2231,7 +2190,7 @@ cudaError_t launch_kr2(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, 
     if (!make_map(&tv, v, 2, dims, str, box)) return cudaErrorInvalidValue;
   }
   const cuuint64_t ny = (cuuint64_t)pb.c1 * pb.b1 * pb.c2;
-  if (PAIR) {
+  {
     // Kt / Y [G][b2 i][c1 p][b1 k][c2 q][d] viewed as (d, c1*b1*c2, b2, G);
     // one warp's box is {64 columns, 1, 32 positions, 1}, clipped at b2
     const cuuint64_t dims[4] = {(cuuint64_t)D, ny, (cuuint64_t)pb.b2, (cuuint64_t)pb.G};
@@ -2239,13 +2198,6 @@ cudaError_t launch_kr2(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, 
     const cuuint32_t box[4] = {64, 1, 32, 1};
     if (!make_map(&tkt, kt, 4, dims, str, box)) return cudaErrorInvalidValue;
     if (!make_map(&tyy, y, 4, dims, str, box)) return cudaErrorInvalidValue;
-  } else {
-    // Kt / Y viewed as (d, c1*b1*c2, G*b2); one box holds the b2 positions
-    const cuuint64_t dims[3] = {(cuuint64_t)D, ny, (cuuint64_t)pb.G * pb.b2};
-    const cuuint64_t str[2] = {(cuuint64_t)D * 2, ny * D * 2};
-    const cuuint32_t box[3] = {64, 1, (cuuint32_t)pb.b2};
-    if (!make_map(&tkt, kt, 3, dims, str, box)) return cudaErrorInvalidValue;
-    if (!make_map(&tyy, y, 3, dims, str, box)) return cudaErrorInvalidValue;
   }
   KR2Args a;
   a.kt = kt;
