@@ -74,6 +74,8 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
 // holds the normalised weights (all 0 in a row with every column masked);
 // ent gets, per row half h, the entropy ln z - sum_j w_j (s_j - m) / z
 // (-inf for such a row).
+// MASKED (padded problems) also handles rows whose every column is masked.
+template <bool MASKED>
 __device__ __forceinline__ void quad_softmax(float (&s)[2][4], int c_lo, int c_hi, int t,
                                              float (&ent)[2]) {
 #pragma unroll
@@ -89,7 +91,7 @@ __device__ __forceinline__ void quad_softmax(float (&s)[2][4], int c_lo, int c_h
       }
     m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
     m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-    if (m == -INFINITY) m = 0.f;  // every column masked: all weights 0
+    if (MASKED && m == -INFINITY) m = 0.f;  // every column masked: all weights 0
     float z = 0.f, dot = 0.f;
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
@@ -105,12 +107,12 @@ __device__ __forceinline__ void quad_softmax(float (&s)[2][4], int c_lo, int c_h
     z += __shfl_xor_sync(0xffffffffu, z, 2);
     dot += __shfl_xor_sync(0xffffffffu, dot, 1);
     dot += __shfl_xor_sync(0xffffffffu, dot, 2);
-    const float inv = z > 0.f ? 1.f / z : 0.f;
+    const float inv = (!MASKED || z > 0.f) ? 1.f / z : 0.f;
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int e = 0; e < 2; ++e) s[nt][2 * h + e] *= inv;
-    ent[h] = z > 0.f ? __logf(z) - dot * inv : -INFINITY;
+    ent[h] = (!MASKED || z > 0.f) ? __logf(z) - dot * inv : -INFINITY;
   }
 }
 
@@ -126,12 +128,16 @@ __device__ __forceinline__ void acc_to_a(const float (&s)[2][4], uint32_t (&a)[4
 // Padding: the head's real tokens are grid tokens [real_lo, real_hi); q, k, v
 // and out hold only those rows (real_hi - real_lo per head), pad rows are
 // zero in shared memory and are masked in every softmax and aggregation.
+// PADDED selects the masked instantiation; unpadded heads (real_lo = 0,
+// real_hi = N) run the one without masks.
+template <bool PADDED>
 __global__ void __launch_bounds__(kThreads, 1)
     small_head_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
                       const bf16* __restrict__ v, bf16* __restrict__ out, int b1, int b2, int T,
                       float sc, int real_lo, int real_hi) {
   extern __shared__ __align__(16) uint8_t smem[];
   const int N = b1 * b2;
+  auto real_tok = [&](int m) { return !PADDED || (m >= real_lo && m < real_hi); };
   const int n_src = real_hi - real_lo;  // rows per head in q, k, v, out
   bf16* Qs = reinterpret_cast<bf16*>(smem);  // token rows l * b2 + i
   bf16* Ks = Qs + N * kPB;
@@ -155,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int x = tid; x < N * (kD / 8); x += kThreads) {
       const int r = x / (kD / 8), c = x % (kD / 8);
       const int so = r * kPB + c * 8;
-      const bool real = r >= real_lo && r < real_hi;
+      const bool real = real_tok(r);
       const int xs = (r - real_lo) * (kD / 8) + c;
       const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
       *reinterpret_cast<uint4*>(Qs + so) = real ? __ldg(gq + xs) : zero;
@@ -171,14 +177,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     float s0 = 0.f, s1 = 0.f;
     int nl = 0;
     for (int l = 0; l < b1; ++l) {
-      if (l * b2 + i < real_lo || l * b2 + i >= real_hi) continue;
+      if (!real_tok(l * b2 + i)) continue;
       const __nv_bfloat162 p = *reinterpret_cast<const __nv_bfloat162*>(Qs + (l * b2 + i) * kPB + c);
       s0 += __low2float(p);
       s1 += __high2float(p);
       ++nl;
     }
     const float inv_n = nl > 0 ? 1.f / (float)nl : 0.f;
-    const uint32_t m = nl == b1 ? tc::pack_bf16x2(s0 / (float)b1, s1 / (float)b1)
+    const uint32_t m = (!PADDED || nl == b1) ? tc::pack_bf16x2(s0 / (float)b1, s1 / (float)b1)
                                 : tc::pack_bf16x2(s0 * inv_n, s1 * inv_n);
     for (int kk = 0; kk < b1; ++kk) *reinterpret_cast<uint32_t*>(Qt + (kk * b2 + i) * kPB + c) = m;
   }
@@ -211,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int j_lo = min(max(real_lo - kk * b2, 0), b2);
       const int j_hi = max(min(real_hi - kk * b2, b2), j_lo);
       float ent[2];
-      quad_softmax(s, j_lo, j_hi, t, ent);
+      quad_softmax<PADDED>(s, j_lo, j_hi, t, ent);
       if (t == 0) {
         if (g < b2) Hs[g * b1 + kk] = ent[0];
         if (g + 8 < b2) Hs[(g + 8) * b1 + kk] = ent[1];
@@ -279,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           s[nt][e] = fmaf(s[nt][e], sc, Hs[i * b1 + col]);
         }
       float ent[2];
-      quad_softmax(s, 0, b1, t, ent);  // chunks without a real key carry Hs = -inf
+      quad_softmax<PADDED>(s, 0, b1, t, ent);  // chunks without a real key carry Hs = -inf
       if (!last) {
         // L (bf16; rows l >= b1 zeroed) to this position's tile, then
         // Qt = L^T q / column sums of L
@@ -289,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const int row = g + 8 * h, col = nt * 8 + 2 * t;
-            const bool real = row < b1 && row * b2 + i >= real_lo && row * b2 + i < real_hi;
+            const bool real = row < b1 && real_tok(row * b2 + i);
             *reinterpret_cast<uint32_t*>(Lt + row * kPL + col) =
                 real ? tc::pack_bf16x2(s[nt][2 * h], s[nt][2 * h + 1]) : 0u;
           }
@@ -332,8 +338,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bf16* y_src = Ys + (i * b1 + min(lr + (mi & 1) * 8, b1 - 1)) * kPB + (mi >> 1) * 8;
         // only real rows are written, to their row in the unpadded output
         const int m0 = g * b2 + i, m1 = (g + 8) * b2 + i;
-        const bool w0 = g < b1 && m0 >= real_lo && m0 < real_hi;
-        const bool w1 = g + 8 < b1 && m1 >= real_lo && m1 < real_hi;
+        const bool w0 = g < b1 && real_tok(m0);
+        const bool w1 = g + 8 < b1 && real_tok(m1);
         bf16* orow0 = out + (gh * n_src + (m0 - real_lo)) * kD;
         bf16* orow1 = out + (gh * n_src + (m1 - real_lo)) * kD;
 #pragma unroll
@@ -368,15 +374,23 @@ cudaError_t small_head_forward(const bf16* q, const bf16* k, const bf16* v, bf16
   static std::once_flag once;
   static cudaError_t attr = cudaSuccess;
   std::call_once(once, [] {
-    attr = cudaFuncSetAttribute(small_head_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)smem_bytes(kMaxN));
+    attr = cudaFuncSetAttribute(small_head_kernel<false>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes(kMaxN));
+    if (attr == cudaSuccess)
+      attr = cudaFuncSetAttribute(small_head_kernel<true>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)smem_bytes(kMaxN));
   });
   if (attr != cudaSuccess) return attr;
   if (!small_head_supports(pb)) return cudaErrorInvalidValue;
   const size_t smem = smem_bytes(pb.b1 * pb.b2);
   return timed_launch("small_head", stream, launches, [&] {
-    small_head_kernel<<<pb.G, kThreads, smem, stream>>>(q, k, v, out, pb.b1, pb.b2, pb.T, pb.sc,
-                                                         pb.real_lo, pb.real_hi);
+    if (is_padded(pb))
+      small_head_kernel<true><<<pb.G, kThreads, smem, stream>>>(q, k, v, out, pb.b1, pb.b2, pb.T,
+                                                                pb.sc, pb.real_lo, pb.real_hi);
+    else
+      small_head_kernel<false><<<pb.G, kThreads, smem, stream>>>(q, k, v, out, pb.b1, pb.b2, pb.T,
+                                                                 pb.sc, pb.real_lo, pb.real_hi);
   });
 }
 

@@ -885,9 +885,9 @@ __global__ void __launch_bounds__(256)
 }
 
 // ---------------------------------------------------------------------------
-// R-update of step one on the tensor cores.  One CTA per (g, k, p): the b2
-// aggregated queries Qt0_{p,i} (rows, <= 128) against the keys of chunk k,
-// one column group q at a time:
+// R-update of step one on the tensor cores.  One CTA per (g, k, p, position
+// tile): 128 of the b2 aggregated queries Qt0_{p,i} (rows; b2 > 128 takes
+// several tiles) against the keys of chunk k, one column group q at a time:
 //   S_q = Qt0 K_q^T / sqrt(d)            128 x NQ in TMEM (K_q: keys j in q)
 //   R = softmax_j(S_q), Hs = entropy      one TMEM lane (row) per thread
 //   [Kt | Y] = R [K_q | V_q]               one N = 2d MMA chain
@@ -904,6 +904,7 @@ struct KRArgs {
   float sc_log2;
   int* status;
   int real_lo, real_hi;  // real tokens (padding): keys outside get zero weight
+  int n_itiles;          // 128-position tiles per sub-item (b2 > 128 takes several)
 };
 
 // Keys [*j_lo, *j_hi) of the nq keys of column group q (first key js) of
@@ -989,10 +990,13 @@ __global__ void __launch_bounds__(128)
     return;
   }
   int bid = blockIdx.x;
+  const int it = bid % a.n_itiles;  // positions i0 .. i0 + 127 of the sub-item
+  bid /= a.n_itiles;
   const int p = bid % a.c1;
   bid /= a.c1;
   const int k = bid % a.b1;
   const int g = bid / a.b1;
+  const int i0 = it * kRows;
 
   uint8_t* sQ = smem + L::kQOff;
   auto sK = [&](int q) { return smem + L::kKVOff + q * L::kGroupBytes; };
@@ -1052,14 +1056,14 @@ __global__ void __launch_bounds__(128)
       }
     }
     pdl_wait();  // Qt0 comes from the previous kernel
-    const int qrow = (g * a.c1 + p) * a.b2;
+    const int qrow = (g * a.c1 + p) * a.b2 + i0;
 #pragma unroll
     for (int c = 0; c < D / 64; ++c) tma_load_2d(sQ + c * kRows * 128, &tm_qt, load_full, c * 64, qrow);
     load_waited = mbar_wait(load_full, 0, abort_flag, a.status);
     if (load_waited) issue_s(0);
   }
-  const int r = tid;  // row = position i
-  const bool row_valid = r < a.b2;
+  const int r = tid;  // row of the tile = position i0 + r
+  const bool row_valid = i0 + r < a.b2;
   for (int q = 0; q < a.c2; ++q) {
     const int js = group_start(a.b2, a.c2, q);
     const int nq = group_start(a.b2, a.c2, q + 1) - js;
@@ -1115,10 +1119,11 @@ __global__ void __launch_bounds__(128)
     if (ok) {
       tc_fence_after();
       const float inv = z > 0.f ? 1.f / z : 0.f;
-      // The b2 rows of this (g, p, k, q) are positions i of the position-major
-      // Kt/Y layout: one 3-D TMA box {64 columns, 1, b2 rows}.  Each 64-column
-      // block is staged (swizzled) in one of two buffers and handed to a TMA
-      // bulk store; a buffer is refilled once its previous store has read it.
+      // The tile's rows of this (g, p, k, q) are positions i0 + r of the
+      // position-major Kt/Y layout: one 4-D TMA box {64 columns, 1, 128
+      // positions, 1} clipped at b2.  Each 64-column block is staged
+      // (swizzled) in one of two buffers and handed to a TMA bulk store; a
+      // buffer is refilled once its previous store has read it.
       const int nblk = (a.write_y ? 2 : 1) * (D / 64);
       const int ycoord = (p * a.b1 + k) * a.c2 + q;
 #pragma unroll 1
@@ -1147,7 +1152,7 @@ __global__ void __launch_bounds__(128)
         fence_proxy_async_smem();
         __syncthreads();
         if (tid == 0) {
-          tma_store_3d(cb < D / 64 ? &tm_kt : &tm_y, buf, (cb % (D / 64)) * 64, ycoord, g * a.b2);
+          tma_store_4d(cb < D / 64 ? &tm_kt : &tm_y, buf, (cb % (D / 64)) * 64, ycoord, i0, g);
           bulk_commit();
         }
       }
@@ -1155,7 +1160,7 @@ __global__ void __launch_bounds__(128)
       if (tid == 0) bulk_wait_read<0>();
       // entropy of the R row: ln z - sum e (s - m) / z, with s - m in log2 units
       if (row_valid) {
-        const long orow = ((((long)g * a.b2 + r) * a.c1 + p) * a.b1 + k) * a.c2 + q;
+        const long orow = ((((long)g * a.b2 + i0 + r) * a.c1 + p) * a.b1 + k) * a.c2 + q;
         a.hs[orow] = z > 0.f ? logf(z) - t2 * 0.69314718055994531f * inv : -INFINITY;
       }
     }
@@ -2131,13 +2136,14 @@ cudaError_t launch_kr(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, b
   }
   CUtensorMap tkt, tyy;
   {
-    // Kt / Y [G][b2 i][c1 p][b1 k][c2 q][d] viewed as (d, c1*b1*c2, G*b2)
-    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)pb.c1 * pb.b1 * pb.c2,
-                                (cuuint64_t)pb.G * pb.b2};
-    const cuuint64_t str[2] = {(cuuint64_t)D * 2, (cuuint64_t)pb.c1 * pb.b1 * pb.c2 * D * 2};
-    const cuuint32_t box[3] = {64, 1, (cuuint32_t)pb.b2};
-    if (!make_map(&tkt, kt, 3, dims, str, box)) return cudaErrorInvalidValue;
-    if (!make_map(&tyy, y, 3, dims, str, box)) return cudaErrorInvalidValue;
+    // Kt / Y [G][b2 i][c1 p][b1 k][c2 q][d] viewed as (d, c1*b1*c2, b2, G); a
+    // tile's box is {64 columns, 1, 128 positions, 1}, clipped at b2
+    const cuuint64_t ny = (cuuint64_t)pb.c1 * pb.b1 * pb.c2;
+    const cuuint64_t dims[4] = {(cuuint64_t)D, ny, (cuuint64_t)pb.b2, (cuuint64_t)pb.G};
+    const cuuint64_t str[3] = {(cuuint64_t)D * 2, ny * D * 2, ny * pb.b2 * D * 2};
+    const cuuint32_t box[4] = {64, 1, kRows, 1};
+    if (!make_map(&tkt, kt, 4, dims, str, box)) return cudaErrorInvalidValue;
+    if (!make_map(&tyy, y, 4, dims, str, box)) return cudaErrorInvalidValue;
   }
   KRArgs a;
   a.kt = kt;
@@ -2152,7 +2158,9 @@ cudaError_t launch_kr(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, b
   a.status = status;
   a.real_lo = pb.real_lo;
   a.real_hi = pb.real_hi;
-  const long blocks = (long)pb.G * pb.b1 * pb.c1;
+  a.n_itiles = (pb.b2 + kRows - 1) / kRows;
+  const long blocks = (long)pb.G * pb.b1 * pb.c1 * a.n_itiles;
+  if (blocks >= (1L << 31)) return cudaErrorInvalidValue;
   return timed_launch("tc_r_update", stream, launches, [&] {
     return launch_pdl(kr_kernel<D, NQ>, dim3((unsigned)blocks), dim3(128), L::bytes(pb.c2), stream, tq,
                tk, tv, tkt, tyy, a);
@@ -2278,9 +2286,10 @@ cudaError_t launch_kl(const bf16* q, const bf16* kt, const float* hs, bf16* qt, 
 
 // Steps >= 2 run on the tensor cores when the L-update fits one tile each
 // way (rows of <= 128 keys, row groups of <= 128 rows) and the R-update's
-// column groups take the persistent kernel (<= 64 keys).
+// column groups take the persistent kernel (<= 64 keys, <= 128 positions).
 bool tc_later_steps(const Problem& pb) {
-  return pb.b1 * pb.c2 <= 128 && (pb.b1 + pb.c1 - 1) / pb.c1 <= kRows && kr_group_tile(pb) <= 64;
+  return pb.b1 * pb.c2 <= 128 && (pb.b1 + pb.c1 - 1) / pb.c1 <= kRows &&
+         kr_group_tile(pb) <= 64 && pb.b2 <= kRows;
 }
 
 // One later step: the non-final L-update (aggregated queries Qt of every
@@ -2319,6 +2328,22 @@ cudaError_t launch_r_step1(const bf16* q, const bf16* k, const bf16* v, bf16* qt
                       dim3(256), 0, stream, q, qt0, pb);
   });
   if (e != cudaSuccess) return e;
+  if (pb.b2 > kRows) {  // positions in several 128-row tiles: the per-item kernel
+    switch (kr_group_tile(pb)) {
+#define MONARCH_KR_TILED(NQ) \
+  case NQ: return launch_kr<D, NQ>(qt0, k, v, kt, y, hs, pb, status, stream, launches);
+      MONARCH_KR_TILED(16)
+      MONARCH_KR_TILED(32)
+      MONARCH_KR_TILED(48)
+      MONARCH_KR_TILED(64)
+      MONARCH_KR_TILED(80)
+      MONARCH_KR_TILED(96)
+      MONARCH_KR_TILED(112)
+      MONARCH_KR_TILED(128)
+#undef MONARCH_KR_TILED
+      default: return cudaErrorInvalidValue;
+    }
+  }
   switch (kr_group_tile(pb)) {
 #define MONARCH_KR2_CASE(NQ)                                                               \
   case NQ:                                                                                 \
@@ -2376,7 +2401,7 @@ cudaError_t tc_selftest_timeout(int* status, unsigned long long limit_ns, cudaSt
 
 bool tc_supports(const Problem& pb) {
   if (pb.d != 64 && pb.d != 128) return false;
-  if (pb.T < 1 || pb.b2 > 128) return false;  // R-side tile: b2 queries <= 128 rows
+  if (pb.T < 1 || pb.b2 > 1024) return false;  // positions: up to eight 128-row tiles
   const int nq = ((pb.b2 + pb.c2 - 1) / pb.c2 + 15) / 16 * 16;
   if (nq > 2 * pb.d || pb.c2 * nq > 256) return false;  // TMEM columns, shared memory
   const long key_rows = (long)pb.G * pb.b2 * pb.c1 * pb.b1 * pb.c2;

@@ -78,6 +78,9 @@ EDGE = [
     (1, 2, 16, 13, 64, 3, 1, 1),     # largest small-head blocks, three steps
     (1, 1, 1, 9, 64, 2, 1, 1),       # small head, one row block
     (1, 1, 12, 1, 64, 2, 1, 1),      # small head, one position
+    (1, 2, 30, 156, 128, 1, 2, 2),   # b2 > 128: two position tiles, 78-key groups
+    (1, 2, 12, 200, 64, 1, 1, 4),    # two position tiles, 50-key groups
+    (1, 1, 6, 300, 64, 2, 2, 3),     # three position tiles, 100-key groups, two steps
 ]
 
 
@@ -252,3 +255,18 @@ def test_later_steps_on_tensor_cores(cuda_lib, B, H, b1, b2, d, T, c1, c2, kind)
         cuda_lib.timing_enable(False)
     assert "tc_l_update" in names and not any(n.startswith("simt") for n in names), names
     assert_parity(O, oracle_forward(q, k, v, b1, b2, T, c1, c2), v, torch.bfloat16)
+
+
+def test_more_than_128_positions_run_on_tensor_cores(cuda_lib):
+    """The (h,fw) layout of the 480p latent in 2 x 2 tiles: b2 = 156 positions
+    in two 128-row tiles of the R-update, no SIMT kernel."""
+    q, k, v = video_qkv(1, 2, (3, 30, 52), 128, torch.bfloat16, seed=12)
+    cuda_lib.timing_read()
+    cuda_lib.timing_enable(True)
+    try:
+        O = gpu_forward(cuda_lib, q, k, v, 30, 156, 1, 2, 2)
+        names = set(cuda_lib.timing_read())
+    finally:
+        cuda_lib.timing_enable(False)
+    assert "tc_r_update" in names and not any(n.startswith("simt") for n in names), names
+    assert_parity(O, oracle_forward(q, k, v, 30, 156, 1, 2, 2), v, torch.bfloat16)
