@@ -21,8 +21,8 @@
 //
 // Step one (aggregated queries under the uniform L, R-update) also runs on
 // the tensor cores, and so do later steps of T >= 2 (non-final L-update with
-// the aggregation L^T Q, R-update from per-sub-item queries) when every L
-// row fits one 128-key tile and every row group one 128-row tile; other
+// the aggregation L^T Q, R-update from per-sub-item queries) when the
+// R-update's column groups hold <= 64 keys and <= 128 positions; other
 // shapes run their later steps on the SIMT kernels.
 #include "tc_path.cuh"
 
@@ -1872,6 +1872,405 @@ __global__ void __launch_bounds__(128)
 }
 
 // ---------------------------------------------------------------------------
+// Non-final L-update for L rows of more than 128 keys or row groups of more
+// than 128 rows, in two passes.
+//
+// kls_kernel, one CTA per (g, i, p, row tile): the log-sum-exp of every row
+// over all b1 c2 keys, S = q Kt^T / sqrt(d) + Hs a 128-key tile at a time
+// (double-buffered in TMEM), running max and sum in registers, one row per
+// thread of warps 1-4; warp 0 loads (TMA) and issues the MMAs.  No barrier
+// joins the row warps: each reads the biases itself, so a warp whose
+// bounded wait gives up cannot leave the others waiting.
+//
+// klm_kernel, one CTA per (g, i, p, key tile): for every row tile, S again,
+// P = exp(S - lse) (rows past the group and pad rows 0), and
+// [Qt~ | c] += P^T [Q | 1] in TMEM across the row tiles (the product of
+// kl_kernel, accumulated); then thread = key writes Qt = Qt~ / c.  One row
+// tile at a time: load Q, S, softmax, aggregation, each waiting for the last.
+// ---------------------------------------------------------------------------
+template <int D>
+struct KLSLayout {
+  static constexpr int kChunk = kRows * 128;
+  static constexpr int kQOff = 0;                            // D / 64 chunks
+  static constexpr int kKtOff = D / 64 * kChunk;             // 2 slots of D / 64 chunks
+  static constexpr int kBarOff = kKtOff + 2 * (D / 64) * kChunk;
+  static constexpr int kBytes = kBarOff + 16 * 8;
+};
+
+struct KLSArgs {
+  const float* hs;  // [G][b2][c1][nk]
+  float* lse;       // [G][b2][b1]
+  int b1, b2, c1, nk, row_tiles, real_lo, real_hi;
+  float sc;
+  int* status;
+};
+
+template <int D>
+__global__ void __launch_bounds__(160)
+    kls_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kt,
+               KLSArgs a) {
+  using L = KLSLayout<D>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (smem_u32(smem) & 1023u) {
+    if (tid == 0) atomicExch(a.status, 2);
+    return;
+  }
+  int bid = blockIdx.x;
+  const int rt = bid % a.row_tiles;
+  bid /= a.row_tiles;
+  const int p = bid % a.c1;
+  bid /= a.c1;
+  const int i = bid % a.b2;
+  const int g = bid / a.b2;
+  const int l0 = group_start(a.b1, a.c1, p), l1 = group_start(a.b1, a.c1, p + 1);
+  const int row0 = l0 + rt * kRows;
+  const long key_row0 = ((long)(g * a.b2 + i) * a.c1 + p) * a.nk;
+  const int n_kt = (a.nk + 127) / 128;
+  uint8_t* sQ = smem + L::kQOff;
+  auto sKt = [&](int sl) { return smem + L::kKtOff + sl * (D / 64) * L::kChunk; };
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* q_full = bars + 0;
+  uint64_t* kt_full = bars + 1;   // [2]
+  uint64_t* kt_empty = bars + 3;  // [2]
+  uint64_t* s_full = bars + 5;    // [2]
+  uint64_t* s_free = bars + 7;    // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 10);
+  if (tid == 0) {
+    mbar_init(q_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(kt_full + b, 1);
+      mbar_init(kt_empty + b, 1);
+      mbar_init(s_full + b, 1);
+      mbar_init(s_free + b, 128);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // Kt and the entropies come from the previous kernel
+  pdl_launch_dependents();
+  if (warp == 0) {
+    // ---- loads and MMAs, one thread ----
+    if (lane == 0) {
+      bool ok = true;
+      long loaded = 0, issued = 0;
+      mbar_arrive_expect_tx(q_full, (D / 64) * L::kChunk);
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c)
+        tma_load_3d(sQ + c * L::kChunk, &tm_q, q_full, c * 64, i, g * a.b1 + row0);
+      auto load_kt = [&](int kt) {
+        const int sl = kt & 1;
+        mbar_arrive_expect_tx(kt_full + sl, (D / 64) * L::kChunk);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_2d(sKt(sl) + c * L::kChunk, &tm_kt, kt_full + sl, c * 64,
+                      (int)(key_row0 + kt * 128));
+      };
+      for (; loaded < 2 && loaded < n_kt; ++loaded) load_kt((int)loaded);
+      ok = mbar_wait(q_full, 0, abort_flag, a.status);
+      const uint32_t idesc = idesc_bf16(kRows, 128, false);
+      for (int kt = 0; kt < n_kt && ok; ++kt) {
+        const int sl = kt & 1;
+        ok = mbar_wait(kt_full + sl, (kt >> 1) & 1, abort_flag, a.status) &&
+             (kt < 2 || mbar_wait(s_free + sl, ((kt >> 1) - 1) & 1, abort_flag, a.status));
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t dq = desc_kmajor(smem_u32(sQ)), dk = desc_kmajor(smem_u32(sKt(sl)));
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_bf16_ss(tmem + sl * 128, dq + (((kk >> 2) * L::kChunk + (kk & 3) * 32) >> 4),
+                      dk + (((kk >> 2) * L::kChunk + (kk & 3) * 32) >> 4), idesc,
+                      kk > 0 ? 1u : 0u);
+        mma_commit(s_full + sl);
+        mma_commit(kt_empty + sl);
+        issued = kt + 1;
+        if (loaded < n_kt) {
+          ok = mbar_wait(kt_empty + sl, (kt >> 1) & 1, abort_flag, a.status);
+          if (ok) load_kt((int)loaded++);
+        }
+      }
+      if (*abort_flag) {
+        drain(q_full, 0);
+        for (long t = loaded >= 2 ? loaded - 2 : 0; t < loaded; ++t)
+          drain(kt_full + (t & 1), (t >> 1) & 1);
+        if (issued > 0) drain(s_full + ((issued - 1) & 1), ((issued - 1) >> 1) & 1);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---- row statistics, thread = row ----
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const int l = row0 + r;
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    float m_run = -INFINITY, z = 0.f;
+    bool ok = true;
+    for (int kt = 0; kt < n_kt && ok; ++kt) {
+      const int sl = kt & 1;
+      const int col0 = kt * 128;
+      ok = mbar_wait(s_full + sl, (kt >> 1) & 1, abort_flag, a.status);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      float sv[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float t[32];
+        tmem_ld32(tmem + sl * 128 + lane_off + c * 32, t);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) sv[c * 32 + e] = t[e];
+      }
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(s_free + sl);
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      // the tile's entropy biases, read by every thread (L1 broadcasts)
+      const float* hs_t = a.hs + key_row0 + col0;
+#pragma unroll
+      for (int c = 0; c < 128; ++c) {
+        sv[c] = col0 + c < a.nk ? fmaf(sv[c], a.sc, __ldg(hs_t + c)) : -INFINITY;
+        mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
+      }
+      const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      const float mn = fmaxf(m_run, mt);
+      const float base = mn > -INFINITY ? mn : 0.f;
+      float zs[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int c = 0; c < 128; ++c) zs[c & 3] += ex2((sv[c] - base) * kLog2e);
+      z = z * (m_run > -INFINITY ? ex2((m_run - base) * kLog2e) : 0.f) +
+          ((zs[0] + zs[1]) + (zs[2] + zs[3]));
+      m_run = mn;
+    }
+    if (ok && l < l1) a.lse[((long)g * a.b2 + i) * a.b1 + l] = m_run + logf(z);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+template <int D>
+struct KLMLayout {
+  static constexpr int kChunk = kRows * 128;
+  static constexpr int kQOff = 0;                          // D / 64 chunks, then the ones
+  static constexpr int kOnesOff = D / 64 * kChunk;
+  static constexpr int kKtOff = kOnesOff + kChunk;         // D / 64 chunks of 128 keys
+  static constexpr int kPOff = kKtOff + D / 64 * kChunk;   // keys 0-63, keys 64-127
+  static constexpr int kBiasOff = kPOff + 2 * kChunk;      // float [128]
+  static constexpr int kBarOff = kBiasOff + 128 * 4;
+  static constexpr int kBytes = kBarOff + 8 * 8;
+  static constexpr uint32_t kTmemCols = D + 64 + 128 <= 256 ? 256 : 512;
+  static constexpr uint32_t kSCol = kTmemCols - 128;       // S; [Qt~ | c] at [0, D + 64)
+};
+
+struct KLMArgs {
+  const float* hs;   // [G][b2][c1][nk]
+  const float* lse;  // [G][b2][b1]
+  bf16* qt;          // [G][b1 k][c1 p][c2 q][b2 i][d]
+  int b1, b2, c1, c2, nk, key_tiles, real_lo, real_hi;
+  float sc;
+  int* status;
+};
+
+template <int D>
+__global__ void __launch_bounds__(128)
+    klm_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kt,
+               KLMArgs a) {
+  using L = KLMLayout<D>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int tid = threadIdx.x, warp = tid >> 5;
+  if (smem_u32(smem) & 1023u) {
+    if (tid == 0) atomicExch(a.status, 2);
+    return;
+  }
+  int bid = blockIdx.x;
+  const int kt = bid % a.key_tiles;
+  bid /= a.key_tiles;
+  const int p = bid % a.c1;
+  bid /= a.c1;
+  const int i = bid % a.b2;
+  const int g = bid / a.b2;
+  const int l0 = group_start(a.b1, a.c1, p), l1 = group_start(a.b1, a.c1, p + 1);
+  const long key_row0 = ((long)(g * a.b2 + i) * a.c1 + p) * a.nk + kt * 128;
+  const int n_rt = (l1 - l0 + kRows - 1) / kRows;
+  uint8_t* sQ = smem + L::kQOff;
+  uint8_t* sOnes = smem + L::kOnesOff;
+  uint8_t* sKt = smem + L::kKtOff;
+  uint8_t* sP = smem + L::kPOff;
+  float* sBias = reinterpret_cast<float*>(smem + L::kBiasOff);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* kt_full = bars + 0;
+  uint64_t* q_full = bars + 1;
+  uint64_t* s_full = bars + 2;
+  uint64_t* o_full = bars + 3;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 5);
+  if (tid == 0) {
+    mbar_init(kt_full, 1);
+    mbar_init(q_full, 1);
+    mbar_init(s_full, 1);
+    mbar_init(o_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  for (int x = tid; x < L::kChunk / 16; x += 128)
+    reinterpret_cast<uint4*>(sOnes)[x] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u,
+                                                     0x3F803F80u);
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem_s = tmem + L::kSCol;
+  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+  pdl_wait();  // Kt, the entropies and the row statistics come from earlier kernels
+  pdl_launch_dependents();
+  if (tid == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_kt);
+    mbar_arrive_expect_tx(kt_full, (D / 64) * L::kChunk);
+#pragma unroll
+    for (int c = 0; c < D / 64; ++c)
+      tma_load_2d(sKt + c * L::kChunk, &tm_kt, kt_full, c * 64, (int)key_row0);
+  }
+  const int key = kt * 128 + tid;
+  sBias[tid] = key < a.nk ? a.hs[key_row0 + tid] : -INFINITY;
+  __syncthreads();
+  const float* lse_i = a.lse + ((long)g * a.b2 + i) * a.b1;
+  bool ok = true;
+  int issued_s = 0, issued_o = 0, q_loads = 0;
+  for (int rt = 0; rt < n_rt && ok; ++rt) {
+    const int row0 = l0 + rt * kRows;
+    // the previous aggregation has read sQ and sP; load this row tile's Q, then S
+    if (tid == 0) {
+      mbar_arrive_expect_tx(q_full, (D / 64) * L::kChunk);
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c)
+        tma_load_3d(sQ + c * L::kChunk, &tm_q, q_full, c * 64, i, g * a.b1 + row0);
+      ++q_loads;
+      ok = mbar_wait(q_full, rt & 1, abort_flag, a.status) &&
+           (rt > 0 || mbar_wait(kt_full, 0, abort_flag, a.status));
+      if (ok) {
+        tc_fence_after();
+        const uint64_t dq = desc_kmajor(smem_u32(sQ)), dk = desc_kmajor(smem_u32(sKt));
+        const uint32_t idesc = idesc_bf16(kRows, 128, false);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_bf16_ss(tmem_s, dq + (((kk >> 2) * L::kChunk + (kk & 3) * 32) >> 4),
+                      dk + (((kk >> 2) * L::kChunk + (kk & 3) * 32) >> 4), idesc,
+                      kk > 0 ? 1u : 0u);
+        mma_commit(s_full);
+        ++issued_s;
+      }
+    }
+    // ---- P = exp(S - lse), thread = row ----
+    const int r = tid, l = row0 + r;
+    const bool row_real = l < l1 && l * a.b2 + i >= a.real_lo && l * a.b2 + i < a.real_hi;
+    const float lse_row = row_real ? lse_i[l] : 0.f;
+    ok = mbar_wait(s_full, rt & 1, abort_flag, a.status);
+    ok = __syncthreads_and(ok);
+    if (!ok) break;
+    tc_fence_after();
+    float sv[128];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      float t[32];
+      tmem_ld32(tmem_s + lane_off + c * 32, t);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) sv[c * 32 + e] = t[e];
+    }
+    tmem_wait_ld();
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {  // 16-byte unit u holds keys 8u .. 8u + 7
+      float w[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float x = fmaf(sv[8 * u + e], a.sc, sBias[8 * u + e]);
+        w[e] = row_real && x > -INFINITY ? ex2((x - lse_row) * kLog2e) : 0.f;
+      }
+      uint4 pk;
+      pk.x = pack_bf16x2(w[0], w[1]);
+      pk.y = pack_bf16x2(w[2], w[3]);
+      pk.z = pack_bf16x2(w[4], w[5]);
+      pk.w = pack_bf16x2(w[6], w[7]);
+      *reinterpret_cast<uint4*>(sP + (u >> 3) * L::kChunk + r * 128 + (((u & 7) ^ (r & 7)) << 4)) =
+          pk;
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      const uint64_t dp = desc_mnmajor(smem_u32(sP), L::kChunk);
+      const uint64_t dq = desc_mnmajor(smem_u32(sQ), L::kChunk);
+      const uint32_t idesc = idesc_bf16(kRows, D + 64, true, true);
+#pragma unroll
+      for (int kk = 0; kk < kRows / 16; ++kk)
+        mma_bf16_ss(tmem, dp + ((kk * 16 * 128) >> 4), dq + ((kk * 16 * 128) >> 4), idesc,
+                    (rt > 0 || kk > 0) ? 1u : 0u);
+      mma_commit(o_full);
+      ++issued_o;
+      ok = mbar_wait(o_full, rt & 1, abort_flag, a.status);  // sQ and sP free again
+    }
+    ok = __syncthreads_and(ok);
+  }
+  // ---- epilogue, thread = key ----
+  if (ok) {
+    tc_fence_after();
+    float cs[32];
+    tmem_ld32(tmem + lane_off + D, cs);
+    tmem_wait_ld();
+    const float invc = cs[0] > 0.f ? 1.f / cs[0] : 0.f;
+    const int kk_ = key / a.c2, q = key % a.c2;
+    bf16* dst = a.qt + (((((long)g * a.b1 + kk_) * a.c1 + p) * a.c2 + q) * a.b2 + i) * D;
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      float t[32];
+      tmem_ld32(tmem + lane_off + c * 32, t);
+      tmem_wait_ld();
+      if (key < a.nk) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          uint4 pk;
+          pk.x = pack_bf16x2(t[8 * u + 0] * invc, t[8 * u + 1] * invc);
+          pk.y = pack_bf16x2(t[8 * u + 2] * invc, t[8 * u + 3] * invc);
+          pk.z = pack_bf16x2(t[8 * u + 4] * invc, t[8 * u + 5] * invc);
+          pk.w = pack_bf16x2(t[8 * u + 6] * invc, t[8 * u + 7] * invc);
+          *reinterpret_cast<uint4*>(dst + c * 32 + 8 * u) = pk;
+        }
+      }
+    }
+  }
+  if (tid == 0 && *abort_flag) {  // drain what this CTA issued (bounded)
+    drain(kt_full, 0);
+    if (q_loads > 0) drain(q_full, (q_loads - 1) & 1);
+    if (issued_s > 0) drain(s_full, (issued_s - 1) & 1);
+    if (issued_o > 0) drain(o_full, (issued_o - 1) & 1);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Self-test of the bounded-wait path: one CTA waits on an mbarrier that
 // nothing ever arrives on, gives up after limit_ns, records the timeout in
 // the status word and returns normally.
@@ -2284,21 +2683,101 @@ cudaError_t launch_kl(const bf16* q, const bf16* kt, const float* hs, bf16* qt, 
   });
 }
 
-// Steps >= 2 run on the tensor cores when the L-update fits one tile each
-// way (rows of <= 128 keys, row groups of <= 128 rows) and the R-update's
-// column groups take the persistent kernel (<= 64 keys, <= 128 positions).
+// Two-pass non-final L-update (rows of more than 128 keys or row groups of
+// more than 128 rows): row log-sum-exps, then the aggregation per key tile.
+template <int D>
+cudaError_t launch_kl_two_pass(const bf16* q, const bf16* kt, const float* hs, float* lse,
+                               bf16* qt, const Problem& pb, int* status, cudaStream_t stream,
+                               int* launches) {
+  using LS = KLSLayout<D>;
+  using LM = KLMLayout<D>;
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(kls_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    LS::kBytes);
+    if (attr_err == cudaSuccess)
+      attr_err = cudaFuncSetAttribute(klm_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      LM::kBytes);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  const int nk = pb.b1 * pb.c2;
+  const long key_rows = (long)pb.G * pb.b2 * pb.c1 * nk;
+  CUtensorMap tq, tk;
+  {
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)pb.b2, (cuuint64_t)pb.G * pb.b1};
+    const cuuint64_t str[2] = {(cuuint64_t)D * 2, (cuuint64_t)pb.b2 * D * 2};
+    const cuuint32_t box[3] = {64, 1, kRows};
+    if (!make_map(&tq, q, 3, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)key_rows};
+    const cuuint64_t str[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64, 128};
+    if (!make_map(&tk, kt, 2, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  const int gmax = (pb.b1 + pb.c1 - 1) / pb.c1;
+  KLSArgs as;
+  as.hs = hs;
+  as.lse = lse;
+  as.b1 = pb.b1;
+  as.b2 = pb.b2;
+  as.c1 = pb.c1;
+  as.nk = nk;
+  as.row_tiles = (gmax + kRows - 1) / kRows;
+  as.real_lo = pb.real_lo;
+  as.real_hi = pb.real_hi;
+  as.sc = pb.sc;
+  as.status = status;
+  const long units = (long)pb.G * pb.b2 * pb.c1;
+  if (units * as.row_tiles >= (1L << 31) || units * ((nk + 127) / 128) >= (1L << 31))
+    return cudaErrorInvalidValue;
+  cudaError_t e = timed_launch("tc_l_stats", stream, launches, [&] {
+    return launch_pdl(kls_kernel<D>, dim3((unsigned)(units * as.row_tiles)), dim3(160),
+                      LS::kBytes, stream, tq, tk, as);
+  });
+  if (e != cudaSuccess) return e;
+  KLMArgs am;
+  am.hs = hs;
+  am.lse = lse;
+  am.qt = qt;
+  am.b1 = pb.b1;
+  am.b2 = pb.b2;
+  am.c1 = pb.c1;
+  am.c2 = pb.c2;
+  am.nk = nk;
+  am.key_tiles = (nk + 127) / 128;
+  am.real_lo = pb.real_lo;
+  am.real_hi = pb.real_hi;
+  am.sc = pb.sc;
+  am.status = status;
+  return timed_launch("tc_l_update", stream, launches, [&] {
+    return launch_pdl(klm_kernel<D>, dim3((unsigned)(units * am.key_tiles)), dim3(128),
+                      LM::kBytes, stream, tq, tk, am);
+  });
+}
+
+// Steps >= 2 run on the tensor cores when the R-update's column groups take
+// the persistent kernel (<= 64 keys, <= 128 positions); the non-final
+// L-update takes one tile each way (rows of <= 128 keys, row groups of <= 128
+// rows) in one kernel, any other shape in the two-pass pair.
 bool tc_later_steps(const Problem& pb) {
-  return pb.b1 * pb.c2 <= 128 && (pb.b1 + pb.c1 - 1) / pb.c1 <= kRows &&
-         kr_group_tile(pb) <= 64 && pb.b2 <= kRows;
+  return kr_group_tile(pb) <= 64 && pb.b2 <= kRows;
+}
+
+bool kl_single_tile(const Problem& pb) {
+  return pb.b1 * pb.c2 <= 128 && (pb.b1 + pb.c1 - 1) / pb.c1 <= kRows;
 }
 
 // One later step: the non-final L-update (aggregated queries Qt of every
 // sub-item), then the R-update from them.
 template <int D>
 cudaError_t launch_later_step(const bf16* q, const bf16* k, const bf16* v, bf16* qt, bf16* kt,
-                              bf16* y, float* hs, const Problem& pb, bool last, int* status,
-                              cudaStream_t stream, int* launches) {
-  cudaError_t e = launch_kl<D>(q, kt, hs, qt, pb, status, stream, launches);
+                              bf16* y, float* hs, float* lse, const Problem& pb, bool last,
+                              int* status, cudaStream_t stream, int* launches) {
+  cudaError_t e = kl_single_tile(pb)
+                      ? launch_kl<D>(q, kt, hs, qt, pb, status, stream, launches)
+                      : launch_kl_two_pass<D>(q, kt, hs, lse, qt, pb, status, stream, launches);
   if (e != cudaSuccess) return e;
   switch (kr_group_tile(pb)) {
 #define MONARCH_KR2_STEP(NQ)                                                                   \
@@ -2433,10 +2912,10 @@ cudaError_t tc_forward(const bf16* q, const bf16* k, const bf16* v, bf16* out, c
   bf16* qt = reinterpret_cast<bf16*>(ws.qt);  // bf16 rows in the fp32-sized piece
   for (int t = 2; t <= pb.T; ++t) {
     if (tc_steps) {
-      e = pb.d == 128 ? launch_later_step<128>(q, k, v, qt, kt, y, ws.hs, pb, t == pb.T, status,
-                                               stream, launches)
-                      : launch_later_step<64>(q, k, v, qt, kt, y, ws.hs, pb, t == pb.T, status,
-                                              stream, launches);
+      e = pb.d == 128 ? launch_later_step<128>(q, k, v, qt, kt, y, ws.hs, ws.lse, pb, t == pb.T,
+                                               status, stream, launches)
+                      : launch_later_step<64>(q, k, v, qt, kt, y, ws.hs, ws.lse, pb, t == pb.T,
+                                              status, stream, launches);
       if (e != cudaSuccess) return e;
       continue;
     }

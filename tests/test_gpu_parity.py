@@ -237,6 +237,11 @@ LATER_STEPS = [
     (1, 2, 60, 80, 128, 2, 1, 2, "iid"),     # unpaired R tiles (80 positions, 40-key groups)
     (2, 2, 40, 48, 64, 3, 2, 2, "iid"),      # tiled, three steps
     (1, 2, 45, 20, 128, 2, 3, 2, "iid"),     # tiled with 15-row groups
+    # two-pass L-update: rows of more than 128 keys or groups of more than 128 rows
+    (1, 2, 70, 20, 128, 2, 2, 2, "iid"),     # 140 keys per row
+    (1, 1, 200, 8, 64, 2, 1, 1, "iid"),      # 200 keys, 200-row groups (two row tiles)
+    (1, 1, 260, 40, 128, 3, 2, 2, "iid"),    # 520 keys, 130-row groups, paired R tiles
+    (1, 1, 140, 80, 64, 2, 1, 2, "iid"),     # 280 keys, unpaired R tiles
 ]
 
 
@@ -254,6 +259,8 @@ def test_later_steps_on_tensor_cores(cuda_lib, B, H, b1, b2, d, T, c1, c2, kind)
     finally:
         cuda_lib.timing_enable(False)
     assert "tc_l_update" in names and not any(n.startswith("simt") for n in names), names
+    if b1 * c2 > 128 or -(-b1 // c1) > 128:
+        assert "tc_l_stats" in names, names
     assert_parity(O, oracle_forward(q, k, v, b1, b2, T, c1, c2), v, torch.bfloat16)
 
 
