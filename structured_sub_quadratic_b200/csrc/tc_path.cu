@@ -1184,6 +1184,273 @@ __global__ void __launch_bounds__(128)
 }
 
 // ---------------------------------------------------------------------------
+// R-update for column groups of more than 128 keys.  One CTA of four warps
+// per (g, k, p, position tile, group q) streams the group's keys in
+// 128-key sub-tiles with an online softmax (thread = row, log2 units):
+//   S_j = Qt0 K_j^T sc log2(e)       128 x 128 in TMEM, columns [2d, 2d + 128)
+//   m, z, T = sum e (s - m)          running per row; when a sub-tile's max
+//                                    exceeds m by more than 2^8 (lazy), m moves
+//                                    and z, T and the accumulator rows are
+//                                    scaled by 2^(m_old - m_new)
+//   [Kt | Y] += P_j [K_j | V_j]        128 x 2d in TMEM, columns [0, 2d)
+// then [Kt | Y] / z, Hs = ln z - ln 2 T / z, and every warp stores its 32
+// rows through a 4-D box clipped at b2, staged in its rows of P.  Thread 0
+// loads (TMA) and issues the MMAs; one sub-tile at a time.
+// ---------------------------------------------------------------------------
+template <int D>
+struct KRLLayout {
+  static constexpr int kChunk = kRows * 128;                    // 128 rows x 64 bf16
+  static constexpr int kQOff = 0;                               // D / 64 chunks
+  static constexpr int kKVOff = D / 64 * kChunk;                // K chunks, then V chunks
+  static constexpr int kPOff = kKVOff + 2 * (D / 64) * kChunk;  // 2 chunks: 128 keys
+  static constexpr int kBarOff = kPOff + 2 * kChunk;
+  static constexpr int kBytes = kBarOff + 8 * 8;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kSCol = 2 * D;
+};
+
+template <int D>
+__global__ void __launch_bounds__(128)
+    krl_kernel(const __grid_constant__ CUtensorMap tm_qt, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kt,
+               const __grid_constant__ CUtensorMap tm_y, KRArgs a) {
+  using L = KRLLayout<D>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (smem_u32(smem) & 1023u) {
+    if (tid == 0) atomicExch(a.status, 2);
+    return;
+  }
+  int bid = blockIdx.x;
+  const int q = bid % a.c2;
+  bid /= a.c2;
+  const int it = bid % a.n_itiles;
+  bid /= a.n_itiles;
+  const int p = bid % a.c1;
+  bid /= a.c1;
+  const int k = bid % a.b1;
+  const int g = bid / a.b1;
+  const int i0 = it * kRows;
+  const int js = group_start(a.b2, a.c2, q);
+  const int nq = group_start(a.b2, a.c2, q + 1) - js;
+  const int n_sub = (nq + 127) / 128;
+  int jlo, jhi;  // the group's real keys
+  real_keys(a.real_lo, a.real_hi, a.b2, k, js, nq, &jlo, &jhi);
+  uint8_t* sQ = smem + L::kQOff;
+  uint8_t* sKV = smem + L::kKVOff;
+  uint8_t* sP = smem + L::kPOff;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* q_full = bars + 0;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* s_full = bars + 2;
+  uint64_t* o_full = bars + 3;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 5);
+  if (tid == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(kv_full, 1);
+    mbar_init(s_full, 1);
+    mbar_init(o_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem_s = tmem + L::kSCol;
+  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+  pdl_launch_dependents();
+  const int krow0 = (g * a.b1 + k) * a.b2 + js;
+  bool ok = true;
+  int issued_s = 0, issued_o = 0, kv_loads = 0;
+  if (tid == 0) {
+    tma_prefetch_desc(&tm_qt);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    pdl_wait();  // Qt0 comes from the previous kernel
+    mbar_arrive_expect_tx(q_full, (D / 64) * L::kChunk);
+#pragma unroll
+    for (int c = 0; c < D / 64; ++c)
+      tma_load_2d(sQ + c * L::kChunk, &tm_qt, q_full, c * 64, (g * a.c1 + p) * a.b2 + i0);
+  }
+  const int r = tid;  // tile row = position i0 + r
+  float m = -INFINITY, z = 0.f, t2 = 0.f;
+  for (int j = 0; j < n_sub && ok; ++j) {
+    if (tid == 0) {
+      // K_j, V_j into the (single) buffer: the previous product has read it
+      if (j > 0) ok = mbar_wait(o_full, (j - 1) & 1, abort_flag, a.status);
+      if (ok) {
+        mbar_arrive_expect_tx(kv_full, 2 * (D / 64) * L::kChunk);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_2d(sKV + c * L::kChunk, &tm_k, kv_full, c * 64, krow0 + j * 128);
+          tma_load_2d(sKV + (D / 64 + c) * L::kChunk, &tm_v, kv_full, c * 64, krow0 + j * 128);
+        }
+        ++kv_loads;
+        ok = mbar_wait(kv_full, j & 1, abort_flag, a.status) &&
+             (j > 0 || mbar_wait(q_full, 0, abort_flag, a.status));
+      }
+      if (ok) {
+        tc_fence_after();
+        const uint64_t dq = desc_kmajor(smem_u32(sQ)), dk = desc_kmajor(smem_u32(sKV));
+        const uint32_t idesc = idesc_bf16(kRows, 128, false);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_bf16_ss(tmem_s, dq + (((kk >> 2) * L::kChunk + (kk & 3) * 32) >> 4),
+                      dk + (((kk >> 2) * L::kChunk + (kk & 3) * 32) >> 4), idesc,
+                      kk > 0 ? 1u : 0u);
+        mma_commit(s_full);
+        ++issued_s;
+      }
+    }
+    // S_j complete implies the previous [Kt | Y] product complete (in order)
+    ok = mbar_wait(s_full, j & 1, abort_flag, a.status);
+    ok = __syncthreads_and(ok);
+    if (!ok) break;
+    tc_fence_after();
+    float sv[128];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      float t[32];
+      tmem_ld32(tmem_s + lane_off + c * 32, t);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) sv[c * 32 + e] = t[e];
+    }
+    tmem_wait_ld();
+    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+    for (int c = 0; c < 128; ++c) {
+      const int jj = j * 128 + c;
+      sv[c] = (jj >= jlo && jj < jhi) ? sv[c] * a.sc_log2 : -INFINITY;
+      mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
+    }
+    const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+    float alpha = 1.f;
+    bool resc = false;
+    if (mt > m + 8.f) {  // first real keys, or the max grew by more than 2^8
+      alpha = m > -INFINITY ? ex2(m - mt) : 0.f;
+      t2 = m > -INFINITY ? alpha * (t2 + z * (m - mt)) : 0.f;
+      z *= alpha;
+      resc = j > 0;
+      m = mt;
+    }
+    if (__any_sync(0xffffffffu, resc)) {  // scale this warp's accumulator rows
+#pragma unroll 1
+      for (int c = 0; c < 2 * D / 32; ++c) {
+        float t[32];
+        tmem_ld32(tmem + lane_off + c * 32, t);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) t[e] *= alpha;
+        tmem_st32(tmem + lane_off + c * 32, t);
+      }
+      tmem_wait_st();
+    }
+    const float base = m > -INFINITY ? m : 0.f;
+    float zs[4] = {0.f, 0.f, 0.f, 0.f}, ts[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {  // 16-byte unit u holds keys 8u .. 8u + 7
+      float w[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float d2 = sv[8 * u + e] - base;  // -inf outside the real keys
+        w[e] = ex2(d2);
+        zs[e & 3] += w[e];
+        ts[e & 3] += w[e] > 0.f ? w[e] * d2 : 0.f;
+      }
+      uint4 pk;
+      pk.x = pack_bf16x2(w[0], w[1]);
+      pk.y = pack_bf16x2(w[2], w[3]);
+      pk.z = pack_bf16x2(w[4], w[5]);
+      pk.w = pack_bf16x2(w[6], w[7]);
+      *reinterpret_cast<uint4*>(sP + (u >> 3) * L::kChunk + r * 128 + (((u & 7) ^ (r & 7)) << 4)) =
+          pk;
+    }
+    z += (zs[0] + zs[1]) + (zs[2] + zs[3]);
+    t2 += (ts[0] + ts[1]) + (ts[2] + ts[3]);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      const uint64_t dp = desc_kmajor(smem_u32(sP));
+      const uint64_t dkv = desc_mnmajor(smem_u32(sKV), L::kChunk);
+      const uint32_t idesc = idesc_bf16(kRows, 2 * D, true);
+#pragma unroll
+      for (int kk = 0; kk < 128 / 16; ++kk)
+        mma_bf16_ss(tmem, dp + (((kk >> 2) * L::kChunk + (kk & 3) * 32) >> 4),
+                    dkv + ((kk * 16 * 128) >> 4), idesc, (j > 0 || kk > 0) ? 1u : 0u);
+      mma_commit(o_full);
+      ++issued_o;
+    }
+  }
+  // ---- epilogue: [Kt | Y] / z, per-warp stores of this warp's 32 rows ----
+  if (ok) ok = mbar_wait(o_full, (n_sub - 1) & 1, abort_flag, a.status);
+  ok = __syncthreads_and(ok);
+  if (ok) {
+    tc_fence_after();
+    const float inv = z > 0.f ? 1.f / z : 0.f;
+    const int nblk = (a.write_y ? 2 : 1) * (D / 64);
+    const int ycoord = (p * a.b1 + k) * a.c2 + q;
+    const int iw = i0 + warp * 32;  // this warp's first position
+    if (iw < a.b2) {
+#pragma unroll 1
+      for (int cb = 0; cb < nblk; ++cb) {
+        uint8_t* buf = sP + (cb & 1) * L::kChunk + warp * 32 * 128;
+        if (cb >= 2) {
+          if (lane == 0) bulk_wait_read<1>();  // the store of block cb - 2 has read buf
+          __syncwarp();
+        }
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          float t[32];
+          tmem_ld32(tmem + lane_off + cb * 64 + hf * 32, t);
+          tmem_wait_ld();
+#pragma unroll
+          for (int uu = 0; uu < 4; ++uu) {
+            uint4 pk;
+            pk.x = pack_bf16x2(t[8 * uu + 0] * inv, t[8 * uu + 1] * inv);
+            pk.y = pack_bf16x2(t[8 * uu + 2] * inv, t[8 * uu + 3] * inv);
+            pk.z = pack_bf16x2(t[8 * uu + 4] * inv, t[8 * uu + 5] * inv);
+            pk.w = pack_bf16x2(t[8 * uu + 6] * inv, t[8 * uu + 7] * inv);
+            const int chunk = hf * 4 + uu;
+            *reinterpret_cast<uint4*>(buf + lane * 128 + ((chunk ^ (lane & 7)) << 4)) = pk;
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_4d(cb < D / 64 ? &tm_kt : &tm_y, buf, (cb % (D / 64)) * 64, ycoord, iw, g);
+          bulk_commit();
+        }
+      }
+    }
+    if (i0 + r < a.b2) {
+      const long orow = ((((long)g * a.b2 + i0 + r) * a.c1 + p) * a.b1 + k) * a.c2 + q;
+      a.hs[orow] = z > 0.f ? logf(z) - t2 * 0.69314718055994531f / z : -INFINITY;
+    }
+  }
+  if (tid == 0 && *abort_flag) {  // drain what this CTA issued (bounded)
+    drain(q_full, 0);
+    if (kv_loads > 0) drain(kv_full, (kv_loads - 1) & 1);
+    if (issued_s > 0) drain(s_full, (issued_s - 1) & 1);
+    if (issued_o > 0) drain(o_full, (issued_o - 1) & 1);
+  }
+  if (lane == 0) bulk_wait<0>();  // stores done reading shared memory before exit
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Persistent R-update for column-group tiles NQ <= 64 (step one, and the
 // later steps with per-sub-item queries).  One CTA
 // per SM walks a contiguous range of sub-items (g, p, k, q): one item (g, p, k)
@@ -2639,6 +2906,71 @@ inline int kr_group_tile(const Problem& pb) {
 }
 
 template <int D>
+cudaError_t launch_krl(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, bf16* y,
+                       float* hs, const Problem& pb, int* status, cudaStream_t stream,
+                       int* launches) {
+  using L = KRLLayout<D>;
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(krl_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    L::kBytes);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  CUtensorMap tq, tk, tv, tkt, tyy;
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)pb.G * pb.c1 * pb.b2};
+    const cuuint64_t str[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64, kRows};
+    if (!make_map(&tq, qt0, 2, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)pb.G * pb.b1 * pb.b2};
+    const cuuint64_t str[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64, 128};
+    if (!make_map(&tk, k, 2, dims, str, box)) return cudaErrorInvalidValue;
+    if (!make_map(&tv, v, 2, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  {
+    // Kt / Y viewed as (d, c1*b1*c2, b2, G); one warp's box {64, 1, 32, 1}, clipped at b2
+    const cuuint64_t ny = (cuuint64_t)pb.c1 * pb.b1 * pb.c2;
+    const cuuint64_t dims[4] = {(cuuint64_t)D, ny, (cuuint64_t)pb.b2, (cuuint64_t)pb.G};
+    const cuuint64_t str[3] = {(cuuint64_t)D * 2, ny * D * 2, ny * pb.b2 * D * 2};
+    const cuuint32_t box[4] = {64, 1, 32, 1};
+    if (!make_map(&tkt, kt, 4, dims, str, box)) return cudaErrorInvalidValue;
+    if (!make_map(&tyy, y, 4, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  KRArgs a;
+  a.kt = kt;
+  a.y = y;
+  a.hs = hs;
+  a.b1 = pb.b1;
+  a.b2 = pb.b2;
+  a.c1 = pb.c1;
+  a.c2 = pb.c2;
+  a.write_y = pb.T == 1 ? 1 : 0;
+  a.sc_log2 = kLog2e * pb.sc;
+  a.status = status;
+  a.real_lo = pb.real_lo;
+  a.real_hi = pb.real_hi;
+  a.n_itiles = (pb.b2 + kRows - 1) / kRows;
+  const long blocks = (long)pb.G * pb.b1 * pb.c1 * a.n_itiles * pb.c2;
+  if (blocks >= (1L << 31)) return cudaErrorInvalidValue;
+  return timed_launch("tc_r_update", stream, launches, [&] {
+    return launch_pdl(krl_kernel<D>, dim3((unsigned)blocks), dim3(128), L::kBytes, stream, tq, tk,
+                      tv, tkt, tyy, a);
+  });
+}
+
+// The per-item R-update kernel holds every column group of a chunk in
+// shared memory: groups of <= 128 keys (and <= 2d, its TMEM), at most 256
+// keys in all.  Wider groups stream through krl_kernel.
+inline bool kr_holds_groups(const Problem& pb) {
+  const int nq = kr_group_tile(pb);
+  return nq <= 128 && nq <= 2 * pb.d && pb.c2 * nq <= 256;
+}
+
+template <int D>
 cudaError_t launch_kl(const bf16* q, const bf16* kt, const float* hs, bf16* qt, const Problem& pb,
                       int* status, cudaStream_t stream, int* launches) {
   using L = KLLayout<D>;
@@ -2795,9 +3127,10 @@ cudaError_t launch_later_step(const bf16* q, const bf16* k, const bf16* v, bf16*
   }
 }
 
-// Step one: aggregated queries under the uniform L, then the R-update (the
-// persistent kernel for column groups of <= 64 keys, the per-item kernel for
-// wider ones).
+// Step one: aggregated queries under the uniform L, then the R-update: the
+// persistent kernel for column groups of <= 64 keys over <= 128 positions,
+// the per-item kernel for groups it holds in shared memory, the streaming
+// kernel for wider ones.
 template <int D>
 cudaError_t launch_r_step1(const bf16* q, const bf16* k, const bf16* v, bf16* qt0, bf16* kt,
                            bf16* y, float* hs, const Problem& pb, int* status,
@@ -2807,40 +3140,37 @@ cudaError_t launch_r_step1(const bf16* q, const bf16* k, const bf16* v, bf16* qt
                       dim3(256), 0, stream, q, qt0, pb);
   });
   if (e != cudaSuccess) return e;
-  if (pb.b2 > kRows) {  // positions in several 128-row tiles: the per-item kernel
+  // column groups of <= 64 keys over <= 128 positions: the persistent kernel
+  if (kr_group_tile(pb) <= 64 && pb.b2 <= kRows) {
     switch (kr_group_tile(pb)) {
-#define MONARCH_KR_TILED(NQ) \
-  case NQ: return launch_kr<D, NQ>(qt0, k, v, kt, y, hs, pb, status, stream, launches);
-      MONARCH_KR_TILED(16)
-      MONARCH_KR_TILED(32)
-      MONARCH_KR_TILED(48)
-      MONARCH_KR_TILED(64)
-      MONARCH_KR_TILED(80)
-      MONARCH_KR_TILED(96)
-      MONARCH_KR_TILED(112)
-      MONARCH_KR_TILED(128)
-#undef MONARCH_KR_TILED
-      default: return cudaErrorInvalidValue;
-    }
-  }
-  switch (kr_group_tile(pb)) {
 #define MONARCH_KR2_CASE(NQ)                                                               \
   case NQ:                                                                                 \
     return pb.b2 <= 64                                                                     \
                ? launch_kr2<D, NQ, true>(qt0, k, v, kt, y, hs, pb, status, stream, launches) \
                : launch_kr2<D, NQ, false>(qt0, k, v, kt, y, hs, pb, status, stream, launches);
+      MONARCH_KR2_CASE(16)
+      MONARCH_KR2_CASE(32)
+      MONARCH_KR2_CASE(48)
+      MONARCH_KR2_CASE(64)
+#undef MONARCH_KR2_CASE
+      default: return cudaErrorInvalidValue;
+    }
+  }
+  // groups the per-item kernel holds in shared memory (any number of
+  // 128-position tiles), else the streaming kernel
+  if (!kr_holds_groups(pb)) return launch_krl<D>(qt0, k, v, kt, y, hs, pb, status, stream, launches);
+  switch (kr_group_tile(pb)) {
 #define MONARCH_KR_CASE(NQ) \
   case NQ: return launch_kr<D, NQ>(qt0, k, v, kt, y, hs, pb, status, stream, launches);
-    MONARCH_KR2_CASE(16)
-    MONARCH_KR2_CASE(32)
-    MONARCH_KR2_CASE(48)
-    MONARCH_KR2_CASE(64)
+    MONARCH_KR_CASE(16)
+    MONARCH_KR_CASE(32)
+    MONARCH_KR_CASE(48)
+    MONARCH_KR_CASE(64)
     MONARCH_KR_CASE(80)
     MONARCH_KR_CASE(96)
     MONARCH_KR_CASE(112)
     MONARCH_KR_CASE(128)
 #undef MONARCH_KR_CASE
-#undef MONARCH_KR2_CASE
     default: return cudaErrorInvalidValue;
   }
 }
@@ -2881,8 +3211,6 @@ cudaError_t tc_selftest_timeout(int* status, unsigned long long limit_ns, cudaSt
 bool tc_supports(const Problem& pb) {
   if (pb.d != 64 && pb.d != 128) return false;
   if (pb.T < 1 || pb.b2 > 1024) return false;  // positions: up to eight 128-row tiles
-  const int nq = ((pb.b2 + pb.c2 - 1) / pb.c2 + 15) / 16 * 16;
-  if (nq > 2 * pb.d || pb.c2 * nq > 256) return false;  // TMEM columns, shared memory
   const long key_rows = (long)pb.G * pb.b2 * pb.c1 * pb.b1 * pb.c2;
   if (key_rows + 256 >= (1L << 31) || (long)pb.G * pb.b1 >= (1L << 31)) return false;
   return encode_fn() != nullptr;

@@ -45,6 +45,7 @@ CASES = [
     (1, 2, 1, 8, 8, True, 64, 1, 1, 1, torch.bfloat16),
     (1, 2, 30 * 156 - 200, 30, 156, True, 128, 1, 2, 2, torch.bfloat16),  # position tiles
     (1, 2, 200 * 8 - 20, 200, 8, True, 64, 2, 1, 1, torch.bfloat16),  # two-pass L-update
+    (1, 2, 30 * 156 - 100, 30, 156, True, 128, 1, 1, 1, torch.bfloat16),  # streamed groups
 ]
 
 

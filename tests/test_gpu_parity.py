@@ -81,6 +81,10 @@ EDGE = [
     (1, 2, 30, 156, 128, 1, 2, 2),   # b2 > 128: two position tiles, 78-key groups
     (1, 2, 12, 200, 64, 1, 1, 4),    # two position tiles, 50-key groups
     (1, 1, 6, 300, 64, 2, 2, 3),     # three position tiles, 100-key groups, two steps
+    (1, 2, 30, 156, 128, 1, 1, 1),   # 156-key groups: streamed in 128-key sub-tiles
+    (1, 1, 8, 300, 64, 1, 1, 1),     # 300-key groups, three sub-tiles, three position tiles
+    (1, 1, 6, 130, 128, 2, 1, 1),    # 130-key groups, two steps
+    (1, 2, 10, 200, 64, 1, 2, 1),    # 200-key groups in two row groups
 ]
 
 
@@ -277,3 +281,16 @@ def test_more_than_128_positions_run_on_tensor_cores(cuda_lib):
         cuda_lib.timing_enable(False)
     assert "tc_r_update" in names and not any(n.startswith("simt") for n in names), names
     assert_parity(O, oracle_forward(q, k, v, 30, 156, 1, 2, 2), v, torch.bfloat16)
+
+
+def test_streamed_groups_rescale_when_the_max_grows(cuda_lib):
+    """Column groups of 300 keys whose last 128-key sub-tile holds much larger
+    logits, so that it raises the running max by more than 2^8 in most rows
+    and the accumulated [Kt | Y] rows are rescaled."""
+    b1, b2, d = 6, 300, 64
+    q, k, v = iid_qkv(1, 2, b1 * b2, d, torch.float32, seed=31)
+    scale = torch.where(torch.arange(b2) >= 256, 6.0, 1.0)  # the last sub-tile dominates
+    k = (k.view(1, 2, b1, b2, d) * scale.view(1, 1, 1, b2, 1)).view(1, 2, b1 * b2, d)
+    q, k, v = (x.to(torch.bfloat16) for x in (q, k, v))
+    O = gpu_forward(cuda_lib, q, k, v, b1, b2, 1)
+    assert_parity(O, oracle_forward(q, k, v, b1, b2, 1), v, torch.bfloat16)
