@@ -159,9 +159,12 @@ MONARCH_API int monarch_attn_fwd_noalloc(const void* q, const void* k, const voi
  * The result is monarch_attn_fwd / _f32 applied to the tokens reordered
  * into the layout's Monarch order (token l*b2 + i), with the output put back
  * into raster order.  (fh, w) and (f, hw) are already in Monarch order and
- * run directly; the other four layouts gather q, k, v into a cached device
+ * run directly.  (w, fh) and (hw, f) are its transpose (raster token
+ * i*b1 + l), which the bf16 tensor-core kernels read and write in place when
+ * they run every step of the shape.  Otherwise, and for (fw, h) and (h, fw),
+ * the layout gathers q, k, v into a cached device
  * buffer of 4*B*H*N*d elements (allocated on first use, grown on demand,
- * freed by monarch_attn_release_workspace) and scatter the output back: one
+ * freed by monarch_attn_release_workspace) and scatters the output back: one
  * extra read and write of each tensor.  The gather uses a table of N raster
  * indices per (f, h, w, layout) and device, built and uploaded with a
  * synchronous copy on its first use and kept until

@@ -21,11 +21,23 @@ typedef __nv_bfloat16 bf16;
 // weight (its entropy bias is -inf), and pad query rows are left out of the
 // aggregations; unpadded problems have real_lo = 0, real_hi = b1*b2.
 // ---------------------------------------------------------------------------
+//
+// Token order of q, k, v and out: tr = 0 is Monarch order (token l*b2 + i);
+// tr = 1 is the transpose (token i*b1 + l), the raster order of a video
+// latent in the (w,fh) and (hw,f) layouts.  Intermediates are the same
+// either way.
+// ---------------------------------------------------------------------------
 struct Problem {
   int G, b1, b2, d, T, c1, c2;
   float sc;  // 1/sqrt(d)
   int real_lo, real_hi;
+  int tr;
 };
+
+// Row of token (l, i) of head g in q, k, v and out.
+__host__ __device__ __forceinline__ long token_row(const Problem& pb, long g, int l, int i) {
+  return pb.tr ? (g * pb.b2 + i) * pb.b1 + l : (g * pb.b1 + l) * pb.b2 + i;
+}
 
 __host__ __device__ __forceinline__ bool is_real(const Problem& pb, long m) {
   return m >= pb.real_lo && m < pb.real_hi;

@@ -185,7 +185,7 @@ int status_word_locked(int dev, int** out) {
 template <typename TIn>
 int forward_device(const TIn* q, const TIn* k, const TIn* v, TIn* out, int B, int H, int b1,
                    int b2, int d, int T, int c1, int c2, cudaStream_t stream, int dtype,
-                   int real_lo = 0, int real_hi = -1) {
+                   int real_lo = 0, int real_hi = -1, int tr = 0) {
   t_launches = 0;
   int st = monarch::validate_args(B, H, b1, b2, d, T, c1, c2);
   if (st != MONARCH_OK) return st;
@@ -196,6 +196,7 @@ int forward_device(const TIn* q, const TIn* k, const TIn* v, TIn* out, int B, in
     pb.real_lo = real_lo;
     pb.real_hi = real_hi;
   }
+  pb.tr = tr;
   const size_t bytes_io = (size_t)pb.G * b1 * b2 * d * sizeof(TIn);
   const char* o0 = reinterpret_cast<const char*>(out);
   for (const void* in : {(const void*)q, (const void*)k, (const void*)v}) {
@@ -259,6 +260,7 @@ Problem make_problem(int B, int H, int b1, int b2, int d, int T, int c1, int c2)
   pb.sc = 1.0f / sqrtf((float)d);
   pb.real_lo = 0;
   pb.real_hi = b1 * b2;
+  pb.tr = 0;
   return pb;
 }
 
@@ -365,6 +367,20 @@ int monarch_attn_fwd_video(int dtype, const void* q, const void* k, const void* 
                                       rows, cols, d, T, c1, c2, stream);
   };
   if (layout == MONARCH_LAYOUT_FH_W || layout == MONARCH_LAYOUT_F_HW) return fwd(q, k, v, out);
+  // (w,fh) and (hw,f): raster token i*b1 + l is the transpose of Monarch
+  // order, which the tensor-core kernels read and write in place (no
+  // gather, no scatter) when every kernel of the pass is a tensor-core one
+  if (dtype == MONARCH_DTYPE_BF16 &&
+      (layout == MONARCH_LAYOUT_W_FH || layout == MONARCH_LAYOUT_HW_F)) {
+    Problem pt = monarch::make_problem(B, H, rows, cols, d, T, c1, c2);
+    pt.tr = 1;
+    if (monarch::choose_bf16_kernels(pt) == monarch::Bf16Kernels::kTensorCore &&
+        monarch::tc_takes_transposed(pt))
+      return forward_device<monarch::bf16>(
+          static_cast<const monarch::bf16*>(q), static_cast<const monarch::bf16*>(k),
+          static_cast<const monarch::bf16*>(v), static_cast<monarch::bf16*>(out), B, H, rows,
+          cols, d, T, c1, c2, stream, MONARCH_DTYPE_BF16, 0, -1, 1);
+  }
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
     return MONARCH_ERR_INVALID_ARG;
   const int row_bytes = d * (dtype == MONARCH_DTYPE_BF16 ? 2 : 4);

@@ -46,6 +46,18 @@ constexpr float kLog2e = 1.4426950408889634f;
 // Lazy rescale threshold of the output kernel: 8 in log2 units (a factor 2^8).
 constexpr float kRescaleNat = 8.f * 0.69314718055994531f;
 
+// Box coordinates (y, z) in the 3-D tensor maps of q (rows row0.. of
+// position i) and of k, v (keys j0.. of chunk k), for Monarch token order
+// (tr = 0) or its transpose (tr = 1); make_q_slab_map and make_kv_map build
+// the maps.
+__device__ __forceinline__ int2 q_slab_yz(int tr, int g, int b1, int b2, int i, int row0) {
+  return tr ? make_int2(row0, g * b2 + i) : make_int2(i, g * b1 + row0);
+}
+
+__device__ __forceinline__ int2 kv_yz(int tr, int g, int b1, int b2, int k, int j0) {
+  return tr ? make_int2(k, g * b2 + j0) : make_int2(j0, g * b1 + k);
+}
+
 template <int D, int NK>
 struct KOLayout {
   static constexpr int kQBytes = D / 64 * kRows * 128;
@@ -69,7 +81,19 @@ struct KOArgs {
   int b1, b2, c1, nk, row_tiles, n_items;
   float sc;         // 1 / sqrt(d)
   int* status;
+  int tr;           // token order (see Problem)
 };
+
+// First output row of a tile (row0 of position i of head g) and the stride
+// between its rows, in elements.
+__device__ __forceinline__ bf16* out_tile(const KOArgs& a, int g, int i, int row0, int d) {
+  return a.out + (a.tr ? ((long)g * a.b2 + i) * a.b1 + row0 : ((long)g * a.b1 + row0) * a.b2 + i) *
+                     d;
+}
+
+__device__ __forceinline__ long out_stride(const KOArgs& a, int d) {
+  return a.tr ? (long)d : (long)a.b2 * d;
+}
 
 __device__ __forceinline__ void drain(uint64_t* bar, uint32_t parity) {
   const unsigned long long t0 = global_ns();
@@ -263,11 +287,11 @@ __global__ void __launch_bounds__(192, 2)
                               mbar_test(bias_empty + st, ((Tk >> 1) - 1) & 1)));
         if (__shfl_sync(0xffffffffu, ready, 0)) {
           if (lane == 0 && k_j == 0) {
+            const int2 qyz = q_slab_yz(a.tr, kit.g, a.b1, a.b2, kit.i, kit.row0);
             mbar_arrive_expect_tx(q_full, L::kQBytes);
 #pragma unroll
             for (int c = 0; c < D / 64; ++c)
-              tma_load_3d(sQ + c * kRows * 128, &tm_q, q_full, c * 64, kit.i,
-                          kit.g * a.b1 + kit.row0);
+              tma_load_3d(sQ + c * kRows * 128, &tm_q, q_full, c * 64, qyz.x, qyz.y);
           }
           if (!waited) {  // Kt, Y and the bias come from the previous kernel
             pdl_wait();
@@ -539,7 +563,7 @@ __global__ void __launch_bounds__(192, 2)
       if (!ok) break;
       tc_fence_after();
       ko_epilogue<D>(tmem_o, lane_off, row, 1.f / l_run, sP,
-                     a.out + (((long)it.g * a.b1 + it.row0) * a.b2 + it.i) * D, (long)a.b2 * D,
+                     out_tile(a, it.g, it.i, it.row0, D), out_stride(a, D),
                      it.nrows, o_empty);
     }
   }
@@ -655,10 +679,11 @@ __global__ void __launch_bounds__(192, 2)
       if (lane == 0) {
         if (n >= 1) ok = mbar_wait(q_empty, (n - 1) & 1, abort_flag, a.status);
         if (ok) {
+          const int2 qyz = q_slab_yz(a.tr, it.g, a.b1, a.b2, it.i, it.row0);
           mbar_arrive_expect_tx(q_full, L::kQBytes);
 #pragma unroll
           for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(sQ + c * kRows * 128, &tm_q, q_full, c * 64, it.i, it.g * a.b1 + it.row0);
+            tma_load_3d(sQ + c * kRows * 128, &tm_q, q_full, c * 64, qyz.x, qyz.y);
         }
       }
       if (n == 0) pdl_wait();  // Kt, Y and the bias come from the previous kernel
@@ -809,7 +834,7 @@ __global__ void __launch_bounds__(192, 2)
       if (!ok) break;
       tc_fence_after();
       ko_epilogue<D>(tmem_o, lane_off, row, 1.f / l_row, sP,
-                     a.out + (((long)it.g * a.b1 + it.row0) * a.b2 + it.i) * D, (long)a.b2 * D,
+                     out_tile(a, it.g, it.i, it.row0, D), out_stride(a, D),
                      it.nrows, o_empty);
       ++n;
     }
@@ -853,8 +878,8 @@ __global__ void __launch_bounds__(256)
   float acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-  const uint4* base = reinterpret_cast<const uint4*>(q + (g * b1 * b2 + i) * D) + ch;
-  const long row_stride = (long)b2 * D / 8;  // in uint4
+  const uint4* base = reinterpret_cast<const uint4*>(q + token_row(pb, g, 0, i) * D) + ch;
+  const long row_stride = (pb.tr ? (long)D : (long)b2 * D) / 8;  // rows l apart, in uint4
 #pragma unroll 8
   for (int l = l0 + rl; l < l1; l += RL) {
     const uint4 u = __ldg(base + l * row_stride);
@@ -905,6 +930,7 @@ struct KRArgs {
   int* status;
   int real_lo, real_hi;  // real tokens (padding): keys outside get zero weight
   int n_itiles;          // 128-position tiles per sub-item (b2 > 128 takes several)
+  int tr;                // token order of k and v (see Problem)
 };
 
 // Keys [*j_lo, *j_hi) of the nq keys of column group q (first key js) of
@@ -1048,11 +1074,11 @@ __global__ void __launch_bounds__(128)
     tma_prefetch_desc(&tm_v);
     mbar_arrive_expect_tx(load_full, D / 64 * kRows * 128 + a.c2 * L::kGroupBytes);
     for (int q = 0; q < a.c2; ++q) {
-      const int krow = (g * a.b1 + k) * a.b2 + group_start(a.b2, a.c2, q);
+      const int2 kyz = kv_yz(a.tr, g, a.b1, a.b2, k, group_start(a.b2, a.c2, q));
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) {
-        tma_load_2d(sK(q) + c * L::kBox, &tm_k, load_full, c * 64, krow);
-        tma_load_2d(sK(q) + (D / 64 + c) * L::kBox, &tm_v, load_full, c * 64, krow);
+        tma_load_3d(sK(q) + c * L::kBox, &tm_k, load_full, c * 64, kyz.x, kyz.y);
+        tma_load_3d(sK(q) + (D / 64 + c) * L::kBox, &tm_v, load_full, c * 64, kyz.x, kyz.y);
       }
     }
     pdl_wait();  // Qt0 comes from the previous kernel
@@ -1265,7 +1291,6 @@ __global__ void __launch_bounds__(128)
   const uint32_t tmem_s = tmem + L::kSCol;
   const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
   pdl_launch_dependents();
-  const int krow0 = (g * a.b1 + k) * a.b2 + js;
   bool ok = true;
   int issued_s = 0, issued_o = 0, kv_loads = 0;
   if (tid == 0) {
@@ -1286,10 +1311,11 @@ __global__ void __launch_bounds__(128)
       if (j > 0) ok = mbar_wait(o_full, (j - 1) & 1, abort_flag, a.status);
       if (ok) {
         mbar_arrive_expect_tx(kv_full, 2 * (D / 64) * L::kChunk);
+        const int2 kyz = kv_yz(a.tr, g, a.b1, a.b2, k, js + j * 128);
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
-          tma_load_2d(sKV + c * L::kChunk, &tm_k, kv_full, c * 64, krow0 + j * 128);
-          tma_load_2d(sKV + (D / 64 + c) * L::kChunk, &tm_v, kv_full, c * 64, krow0 + j * 128);
+          tma_load_3d(sKV + c * L::kChunk, &tm_k, kv_full, c * 64, kyz.x, kyz.y);
+          tma_load_3d(sKV + (D / 64 + c) * L::kChunk, &tm_v, kv_full, c * 64, kyz.x, kyz.y);
         }
         ++kv_loads;
         ok = mbar_wait(kv_full, j & 1, abort_flag, a.status) &&
@@ -1511,6 +1537,7 @@ struct KR2Args {
   // chunks k and groups q of a row group; 1: later steps, every sub-item
   // (g, p, k, q) has its own rows Qt [G][b1][c1][c2][b2][d]
   int qt_per_item;
+  int tr;  // token order of k and v (see Problem)
 };
 
 
@@ -1634,13 +1661,14 @@ __global__ void __launch_bounds__(320, 1)
         if (!ok) break;
         mbar_arrive_expect_tx(kv_full + sl, H * 2 * (D / 64) * L::kBox);
         const int gp_a = cur.gp;
-        int gp_b = gp_a, krow = 0;
+        int gp_b = gp_a;
+        int2 kyz = make_int2(0, 0);
         long qrow[2] = {0, 0};
         for (int h = 0; h < H; ++h) {
           // An absent second half (odd count, last tile) repeats the first:
           // finite keys that its zero rows of P weigh by zero.
           if (h < nh) {
-            krow = (cur.g * a.b1 + cur.k) * a.b2 + group_start(a.b2, a.c2, cur.q);
+            kyz = kv_yz(a.tr, cur.g, a.b1, a.b2, cur.k, group_start(a.b2, a.c2, cur.q));
             gp_b = cur.gp;
             qrow[h] = kr2_qrow(a, cur);
             kr2_next(a, cur);
@@ -1649,9 +1677,10 @@ __global__ void __launch_bounds__(320, 1)
           }
 #pragma unroll
           for (int c = 0; c < D / 64; ++c) {
-            tma_load_2d(sKV(sl) + c * L::kBlk + h * L::kBox, &tm_k, kv_full + sl, c * 64, krow);
-            tma_load_2d(sKV(sl) + (D / 64 + c) * L::kBlk + h * L::kBox, &tm_v, kv_full + sl, c * 64,
-                        krow);
+            tma_load_3d(sKV(sl) + c * L::kBlk + h * L::kBox, &tm_k, kv_full + sl, c * 64, kyz.x,
+                        kyz.y);
+            tma_load_3d(sKV(sl) + (D / 64 + c) * L::kBlk + h * L::kBox, &tm_v, kv_full + sl,
+                        c * 64, kyz.x, kyz.y);
           }
         }
         last_kv = t;
@@ -1957,6 +1986,7 @@ struct KLArgs {
   int b1, b2, c1, c2, nk, real_lo, real_hi;
   float sc;
   int* status;
+  int tr;  // token order of q (see Problem)
 };
 
 template <int D>
@@ -2016,9 +2046,10 @@ __global__ void __launch_bounds__(128)
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_kt);
     mbar_arrive_expect_tx(load_full, 2 * (D / 64) * L::kChunk);
+    const int2 qyz = q_slab_yz(a.tr, g, a.b1, a.b2, i, l0);
 #pragma unroll
     for (int c = 0; c < D / 64; ++c) {
-      tma_load_3d(sQ + c * L::kChunk, &tm_q, load_full, c * 64, i, g * a.b1 + l0);
+      tma_load_3d(sQ + c * L::kChunk, &tm_q, load_full, c * 64, qyz.x, qyz.y);
       tma_load_2d(sKt + c * L::kChunk, &tm_kt, load_full, c * 64, (int)key_row0);
     }
   }
@@ -2170,6 +2201,7 @@ struct KLSArgs {
   int b1, b2, c1, nk, row_tiles, real_lo, real_hi;
   float sc;
   int* status;
+  int tr;  // token order of q (see Problem)
 };
 
 template <int D>
@@ -2231,9 +2263,10 @@ __global__ void __launch_bounds__(160)
       bool ok = true;
       long loaded = 0, issued = 0;
       mbar_arrive_expect_tx(q_full, (D / 64) * L::kChunk);
+      const int2 qyz = q_slab_yz(a.tr, g, a.b1, a.b2, i, row0);
 #pragma unroll
       for (int c = 0; c < D / 64; ++c)
-        tma_load_3d(sQ + c * L::kChunk, &tm_q, q_full, c * 64, i, g * a.b1 + row0);
+        tma_load_3d(sQ + c * L::kChunk, &tm_q, q_full, c * 64, qyz.x, qyz.y);
       auto load_kt = [&](int kt) {
         const int sl = kt & 1;
         mbar_arrive_expect_tx(kt_full + sl, (D / 64) * L::kChunk);
@@ -2348,6 +2381,7 @@ struct KLMArgs {
   int b1, b2, c1, c2, nk, key_tiles, real_lo, real_hi;
   float sc;
   int* status;
+  int tr;  // token order of q (see Problem)
 };
 
 template <int D>
@@ -2426,9 +2460,10 @@ __global__ void __launch_bounds__(128)
     // the previous aggregation has read sQ and sP; load this row tile's Q, then S
     if (tid == 0) {
       mbar_arrive_expect_tx(q_full, (D / 64) * L::kChunk);
+      const int2 qyz = q_slab_yz(a.tr, g, a.b1, a.b2, i, row0);
 #pragma unroll
       for (int c = 0; c < D / 64; ++c)
-        tma_load_3d(sQ + c * L::kChunk, &tm_q, q_full, c * 64, i, g * a.b1 + row0);
+        tma_load_3d(sQ + c * L::kChunk, &tm_q, q_full, c * 64, qyz.x, qyz.y);
       ++q_loads;
       ok = mbar_wait(q_full, rt & 1, abort_flag, a.status) &&
            (rt > 0 || mbar_wait(kt_full, 0, abort_flag, a.status));
@@ -2628,6 +2663,37 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims
   return true;
 }
 
+// 3-D map of q whose box is the 128 rows l (from row0) of one position i:
+// Monarch order (rows l are b2*d apart) or its transpose (rows l adjacent).
+bool make_q_slab_map(CUtensorMap* m, const bf16* q, const Problem& pb, int D) {
+  if (pb.tr) {
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)pb.b1, (cuuint64_t)pb.G * pb.b2};
+    const cuuint64_t str[2] = {(cuuint64_t)D * 2, (cuuint64_t)pb.b1 * D * 2};
+    const cuuint32_t box[3] = {64, kRows, 1};
+    return make_map(m, q, 3, dims, str, box);
+  }
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)pb.b2, (cuuint64_t)pb.G * pb.b1};
+  const cuuint64_t str[2] = {(cuuint64_t)D * 2, (cuuint64_t)pb.b2 * D * 2};
+  const cuuint32_t box[3] = {64, 1, kRows};
+  return make_map(m, q, 3, dims, str, box);
+}
+
+// 3-D map of k or v whose box is `rows` keys j (from j0) of one chunk k: rows
+// j adjacent (Monarch order) or b1*d apart (transposed); rows past b2 read as
+// zeros.
+bool make_kv_map(CUtensorMap* m, const bf16* x, const Problem& pb, int D, int rows) {
+  if (pb.tr) {
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)pb.b1, (cuuint64_t)pb.G * pb.b2};
+    const cuuint64_t str[2] = {(cuuint64_t)D * 2, (cuuint64_t)pb.b1 * D * 2};
+    const cuuint32_t box[3] = {64, 1, (cuuint32_t)rows};
+    return make_map(m, x, 3, dims, str, box);
+  }
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)pb.b2, (cuuint64_t)pb.G * pb.b1};
+  const cuuint64_t str[2] = {(cuuint64_t)D * 2, (cuuint64_t)pb.b2 * D * 2};
+  const cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
+  return make_map(m, x, 3, dims, str, box);
+}
+
 // Launch with programmatic stream serialisation: the kernel may start while
 // the previous kernel of the stream finishes; it calls pdl_wait() before it
 // reads anything that kernel wrote.
@@ -2677,10 +2743,7 @@ cudaError_t launch_ko(const bf16* q, const bf16* kt, const bf16* y, const float*
   const long key_rows = (long)pb.G * pb.b2 * pb.c1 * nk;
   CUtensorMap tq, tk, tyv;
   {
-    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)pb.b2, (cuuint64_t)pb.G * pb.b1};
-    const cuuint64_t str[2] = {(cuuint64_t)D * 2, (cuuint64_t)pb.b2 * D * 2};
-    const cuuint32_t box[3] = {64, 1, kRows};
-    if (!make_map(&tq, q, 3, dims, str, box)) return cudaErrorInvalidValue;
+    if (!make_q_slab_map(&tq, q, pb, D)) return cudaErrorInvalidValue;
   }
   {
     const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)key_rows};
@@ -2703,6 +2766,7 @@ cudaError_t launch_ko(const bf16* q, const bf16* kt, const bf16* y, const float*
   a.n_items = (int)items;
   a.sc = pb.sc;
   a.status = status;
+  a.tr = pb.tr;
   const int grid = (int)std::min<long>(items, 2L * num_sms());
   return timed_launch("tc_l_output", stream, launches, [&] {
     return launch_pdl(ko_kernel<D, NK>, dim3(grid), dim3(192), L::kAlloc, stream, tq, tk, tyv, a);
@@ -2728,10 +2792,7 @@ cudaError_t launch_ko1(const bf16* q, const bf16* kt, const bf16* y, const float
   const long key_rows = (long)pb.G * pb.b2 * pb.c1 * nk;
   CUtensorMap tq, tk, tyv;
   {
-    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)pb.b2, (cuuint64_t)pb.G * pb.b1};
-    const cuuint64_t str[2] = {(cuuint64_t)D * 2, (cuuint64_t)pb.b2 * D * 2};
-    const cuuint32_t box[3] = {64, 1, kRows};
-    if (!make_map(&tq, q, 3, dims, str, box)) return cudaErrorInvalidValue;
+    if (!make_q_slab_map(&tq, q, pb, D)) return cudaErrorInvalidValue;
   }
   {
     const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)key_rows};
@@ -2754,6 +2815,7 @@ cudaError_t launch_ko1(const bf16* q, const bf16* kt, const bf16* y, const float
   a.n_items = (int)items;
   a.sc = pb.sc;
   a.status = status;
+  a.tr = pb.tr;
   const int grid = (int)std::min<long>(items, 2L * num_sms());
   return timed_launch("tc_l_output", stream, launches, [&] {
     return launch_pdl(ko1_kernel<D, NK>, dim3(grid), dim3(192), L::kAlloc, stream, tq, tk, tyv, a);
@@ -2794,11 +2856,8 @@ cudaError_t launch_kr(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, b
     if (!make_map(&tq, qt0, 2, dims, str, box)) return cudaErrorInvalidValue;
   }
   {
-    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)pb.G * pb.b1 * pb.b2};
-    const cuuint64_t str[1] = {(cuuint64_t)D * 2};
-    const cuuint32_t box[2] = {64, (cuuint32_t)NQ};
-    if (!make_map(&tk, k, 2, dims, str, box)) return cudaErrorInvalidValue;
-    if (!make_map(&tv, v, 2, dims, str, box)) return cudaErrorInvalidValue;
+    if (!make_kv_map(&tk, k, pb, D, NQ) || !make_kv_map(&tv, v, pb, D, NQ))
+      return cudaErrorInvalidValue;
   }
   CUtensorMap tkt, tyy;
   {
@@ -2822,6 +2881,7 @@ cudaError_t launch_kr(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, b
   a.write_y = pb.T == 1 ? 1 : 0;
   a.sc_log2 = kLog2e * pb.sc;
   a.status = status;
+  a.tr = pb.tr;
   a.real_lo = pb.real_lo;
   a.real_hi = pb.real_hi;
   a.n_itiles = (pb.b2 + kRows - 1) / kRows;
@@ -2857,11 +2917,8 @@ cudaError_t launch_kr2(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, 
     if (!make_map(&tq, qt0, 2, dims, str, box)) return cudaErrorInvalidValue;
   }
   {
-    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)pb.G * pb.b1 * pb.b2};
-    const cuuint64_t str[1] = {(cuuint64_t)D * 2};
-    const cuuint32_t box[2] = {64, (cuuint32_t)NQ};
-    if (!make_map(&tk, k, 2, dims, str, box)) return cudaErrorInvalidValue;
-    if (!make_map(&tv, v, 2, dims, str, box)) return cudaErrorInvalidValue;
+    if (!make_kv_map(&tk, k, pb, D, NQ) || !make_kv_map(&tv, v, pb, D, NQ))
+      return cudaErrorInvalidValue;
   }
   const cuuint64_t ny = (cuuint64_t)pb.c1 * pb.b1 * pb.c2;
   {
@@ -2889,6 +2946,7 @@ cudaError_t launch_kr2(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, 
   a.qt_per_item = qt_per_item ? 1 : 0;
   a.sc_log2 = kLog2e * pb.sc;
   a.status = status;
+  a.tr = pb.tr;
   a.real_lo = pb.real_lo;
   a.real_hi = pb.real_hi;
   const long units = (items * pb.c2 + L::kHalves - 1) / L::kHalves;
@@ -2925,11 +2983,8 @@ cudaError_t launch_krl(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, 
     if (!make_map(&tq, qt0, 2, dims, str, box)) return cudaErrorInvalidValue;
   }
   {
-    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)pb.G * pb.b1 * pb.b2};
-    const cuuint64_t str[1] = {(cuuint64_t)D * 2};
-    const cuuint32_t box[2] = {64, 128};
-    if (!make_map(&tk, k, 2, dims, str, box)) return cudaErrorInvalidValue;
-    if (!make_map(&tv, v, 2, dims, str, box)) return cudaErrorInvalidValue;
+    if (!make_kv_map(&tk, k, pb, D, 128) || !make_kv_map(&tv, v, pb, D, 128))
+      return cudaErrorInvalidValue;
   }
   {
     // Kt / Y viewed as (d, c1*b1*c2, b2, G); one warp's box {64, 1, 32, 1}, clipped at b2
@@ -2951,6 +3006,7 @@ cudaError_t launch_krl(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, 
   a.write_y = pb.T == 1 ? 1 : 0;
   a.sc_log2 = kLog2e * pb.sc;
   a.status = status;
+  a.tr = pb.tr;
   a.real_lo = pb.real_lo;
   a.real_hi = pb.real_hi;
   a.n_itiles = (pb.b2 + kRows - 1) / kRows;
@@ -2985,10 +3041,7 @@ cudaError_t launch_kl(const bf16* q, const bf16* kt, const float* hs, bf16* qt, 
   const long key_rows = (long)pb.G * pb.b2 * pb.c1 * nk;
   CUtensorMap tq, tk;
   {
-    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)pb.b2, (cuuint64_t)pb.G * pb.b1};
-    const cuuint64_t str[2] = {(cuuint64_t)D * 2, (cuuint64_t)pb.b2 * D * 2};
-    const cuuint32_t box[3] = {64, 1, kRows};
-    if (!make_map(&tq, q, 3, dims, str, box)) return cudaErrorInvalidValue;
+    if (!make_q_slab_map(&tq, q, pb, D)) return cudaErrorInvalidValue;
   }
   {
     const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)key_rows};
@@ -3008,6 +3061,7 @@ cudaError_t launch_kl(const bf16* q, const bf16* kt, const float* hs, bf16* qt, 
   a.real_hi = pb.real_hi;
   a.sc = pb.sc;
   a.status = status;
+  a.tr = pb.tr;
   const long blocks = (long)pb.G * pb.b2 * pb.c1;
   return timed_launch("tc_l_update", stream, launches, [&] {
     return launch_pdl(kl_kernel<D>, dim3((unsigned)blocks), dim3(128), L::kBytes, stream, tq, tk,
@@ -3037,10 +3091,7 @@ cudaError_t launch_kl_two_pass(const bf16* q, const bf16* kt, const float* hs, f
   const long key_rows = (long)pb.G * pb.b2 * pb.c1 * nk;
   CUtensorMap tq, tk;
   {
-    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)pb.b2, (cuuint64_t)pb.G * pb.b1};
-    const cuuint64_t str[2] = {(cuuint64_t)D * 2, (cuuint64_t)pb.b2 * D * 2};
-    const cuuint32_t box[3] = {64, 1, kRows};
-    if (!make_map(&tq, q, 3, dims, str, box)) return cudaErrorInvalidValue;
+    if (!make_q_slab_map(&tq, q, pb, D)) return cudaErrorInvalidValue;
   }
   {
     const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)key_rows};
@@ -3061,6 +3112,7 @@ cudaError_t launch_kl_two_pass(const bf16* q, const bf16* kt, const float* hs, f
   as.real_hi = pb.real_hi;
   as.sc = pb.sc;
   as.status = status;
+  as.tr = pb.tr;
   const long units = (long)pb.G * pb.b2 * pb.c1;
   if (units * as.row_tiles >= (1L << 31) || units * ((nk + 127) / 128) >= (1L << 31))
     return cudaErrorInvalidValue;
@@ -3083,6 +3135,7 @@ cudaError_t launch_kl_two_pass(const bf16* q, const bf16* kt, const float* hs, f
   am.real_hi = pb.real_hi;
   am.sc = pb.sc;
   am.status = status;
+  am.tr = pb.tr;
   return timed_launch("tc_l_update", stream, launches, [&] {
     return launch_pdl(klm_kernel<D>, dim3((unsigned)(units * am.key_tiles)), dim3(128),
                       LM::kBytes, stream, tq, tk, am);
@@ -3210,10 +3263,14 @@ cudaError_t tc_selftest_timeout(int* status, unsigned long long limit_ns, cudaSt
 
 bool tc_supports(const Problem& pb) {
   if (pb.d != 64 && pb.d != 128) return false;
-  if (pb.T < 1 || pb.b2 > 1024) return false;  // positions: up to eight 128-row tiles
+  if (pb.T < 1) return false;
   const long key_rows = (long)pb.G * pb.b2 * pb.c1 * pb.b1 * pb.c2;
   if (key_rows + 256 >= (1L << 31) || (long)pb.G * pb.b1 >= (1L << 31)) return false;
   return encode_fn() != nullptr;
+}
+
+bool tc_takes_transposed(const Problem& pb) {
+  return tc_supports(pb) && (pb.T == 1 || tc_later_steps(pb));
 }
 
 size_t tc_workspace_bytes(const Problem& pb) {

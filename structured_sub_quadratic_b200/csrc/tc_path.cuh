@@ -10,6 +10,11 @@ namespace monarch {
 // True when the tensor-core kernels take this shape.
 bool tc_supports(const Problem& pb);
 
+// True when every tensor-core kernel of this shape's forward pass takes q,
+// k, v and out in transposed token order (Problem::tr; the later steps of
+// some shapes run on SIMT kernels, which do not).
+bool tc_takes_transposed(const Problem& pb);
+
 // Workspace bytes the tensor-core path needs for this shape.
 size_t tc_workspace_bytes(const Problem& pb);
 

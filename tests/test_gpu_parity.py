@@ -85,6 +85,7 @@ EDGE = [
     (1, 1, 8, 300, 64, 1, 1, 1),     # 300-key groups, three sub-tiles, three position tiles
     (1, 1, 6, 130, 128, 2, 1, 1),    # 130-key groups, two steps
     (1, 2, 10, 200, 64, 1, 2, 1),    # 200-key groups in two row groups
+    (1, 1, 3, 1560, 128, 1, 1, 1),   # the (f,hw) blocks of the 480p latent: 13 position tiles
 ]
 
 
@@ -294,3 +295,26 @@ def test_streamed_groups_rescale_when_the_max_grows(cuda_lib):
     q, k, v = (x.to(torch.bfloat16) for x in (q, k, v))
     O = gpu_forward(cuda_lib, q, k, v, b1, b2, 1)
     assert_parity(O, oracle_forward(q, k, v, b1, b2, 1), v, torch.bfloat16)
+
+
+@pytest.mark.parametrize("layout,latent,T,c", [("w,fh", (2, 6, 8), 1, 1), ("w,fh", (2, 6, 8), 2, 2),
+                                               ("hw,f", (2, 6, 8), 2, 1),
+                                               ("w,fh", (3, 30, 52), 1, 1),
+                                               ("hw,f", (3, 30, 52), 1, 1)])
+def test_transposed_layouts_run_in_place(cuda_lib, layout, latent, T, c):
+    """(w,fh) and (hw,f) are the transpose of Monarch order: the tensor-core
+    kernels read q, k, v and write out in raster order, with no permute
+    launch, and match the oracle on the permuted tokens."""
+    d = 64 if latent[0] == 2 else 128
+    q, k, v = video_qkv(1, 2, latent, d, torch.bfloat16, seed=13)
+    cuda_lib.timing_read()
+    cuda_lib.timing_enable(True)
+    try:
+        O = cuda_lib.monarch_attn_fwd_video(q.cuda(), k.cuda(), v.cuda(), *latent, layout, T, c, c)
+        cuda_lib.check()
+        names = set(cuda_lib.timing_read())
+    finally:
+        cuda_lib.timing_enable(False)
+    assert "permute_rows" not in names and not any(n.startswith("simt") for n in names), names
+    assert_parity(O.double().cpu().numpy(), layout_oracle(q, k, v, latent, layout, T, c, c), v,
+                  torch.bfloat16)
