@@ -490,10 +490,21 @@ __global__ void __launch_bounds__(192, 2)
         // the serial chains
         float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         if (valid >= NK) {
+          // packed pairs: the same roundings as the scalar forms, half the
+          // instructions (the softmax warps share their schedulers)
+          const float2 sc2 = make_float2(a.sc, a.sc);
 #pragma unroll
-          for (int c = 0; c < NK; ++c) {
-            sv[c] = fmaf(sv[c], a.sc, bias[c]);
-            mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
+          for (int c = 0; c < NK; c += 4) {
+            const float4 b4 = *reinterpret_cast<const float4*>(bias + c);
+            const float2 lo = fma2(make_float2(sv[c], sv[c + 1]), sc2, make_float2(b4.x, b4.y));
+            const float2 hi = fma2(make_float2(sv[c + 2], sv[c + 3]), sc2, make_float2(b4.z, b4.w));
+            sv[c] = lo.x;
+            sv[c + 1] = lo.y;
+            sv[c + 2] = hi.x;
+            sv[c + 3] = hi.y;
+            const int m = (c >> 2) & 1;
+            mx[m] = max3(mx[m], lo.x, lo.y);
+            mx[2 + m] = max3(mx[2 + m], hi.x, hi.y);
           }
         } else {
 #pragma unroll
@@ -515,15 +526,23 @@ __global__ void __launch_bounds__(192, 2)
         }
         // every key seen so far masked (groups without a real key): weights 0
         const float neg_m2 = m_run > -INFINITY ? -m_run * kLog2e : 0.f;
-        float ls[4] = {0.f, 0.f, 0.f, 0.f};
+        // four partial sums (columns c mod 4), as packed pairs
+        const float2 l2e = make_float2(kLog2e, kLog2e), nm2 = make_float2(neg_m2, neg_m2);
+        float2 ls01 = make_float2(0.f, 0.f), ls23 = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int c = 0; c < NK; ++c) {
+        for (int c = 0; c < NK; c += 4) {
           if (c < NK / 2 || !half) {
-            sv[c] = ex2(fmaf(sv[c], kLog2e, neg_m2));
-            ls[c & 3] += sv[c];
+            const float2 x0 = fma2(make_float2(sv[c], sv[c + 1]), l2e, nm2);
+            const float2 x1 = fma2(make_float2(sv[c + 2], sv[c + 3]), l2e, nm2);
+            sv[c] = ex2(x0.x);
+            sv[c + 1] = ex2(x0.y);
+            sv[c + 2] = ex2(x1.x);
+            sv[c + 3] = ex2(x1.y);
+            ls01 = add2(ls01, make_float2(sv[c], sv[c + 1]));
+            ls23 = add2(ls23, make_float2(sv[c + 2], sv[c + 3]));
           }
         }
-        l_run = l_run * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
+        l_run = l_run * alpha + ((ls01.x + ls01.y) + (ls23.x + ls23.y));
         if (__any_sync(0xffffffffu, resc)) {
           // O is stable once the previous tile's P Y is done
           ok = mbar_wait(pv_done + ((T - 1) & 1), ((T - 1) >> 1) & 1, abort_flag, a.status);
@@ -954,19 +973,43 @@ __device__ __forceinline__ void r_row_softmax(float (&sv)[NQ], float sc_log2, in
   float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
   float zs[4] = {0.f, 0.f, 0.f, 0.f}, ts[4] = {0.f, 0.f, 0.f, 0.f};
   if (jlo == 0 && jhi == nq) {
+    // packed pairs (the scalar roundings, half the instructions); the sums
+    // over columns j mod 4 are the pairs (0, 1) and (2, 3)
+    static_assert(NQ % 4 == 0, "group tile");
+    const float2 s2 = make_float2(sc_log2, sc_log2);
 #pragma unroll
-    for (int j = 0; j < NQ; ++j) {
-      sv[j] = j < nq ? sv[j] * sc_log2 : -INFINITY;
-      mx[j & 3] = fmaxf(mx[j & 3], sv[j]);
+    for (int j = 0; j < NQ; j += 4) {
+      const float2 a = mul2(make_float2(sv[j], sv[j + 1]), s2);
+      const float2 b = mul2(make_float2(sv[j + 2], sv[j + 3]), s2);
+      sv[j] = j < nq ? a.x : -INFINITY;
+      sv[j + 1] = j + 1 < nq ? a.y : -INFINITY;
+      sv[j + 2] = j + 2 < nq ? b.x : -INFINITY;
+      sv[j + 3] = j + 3 < nq ? b.y : -INFINITY;
+      const int m = (j >> 2) & 1;
+      mx[m] = max3(mx[m], sv[j], sv[j + 1]);
+      mx[2 + m] = max3(mx[2 + m], sv[j + 2], sv[j + 3]);
     }
     const float m2 = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+    const float2 nm = make_float2(-m2, -m2);
+    float2 z01 = make_float2(0.f, 0.f), z23 = z01, t01 = z01, t23 = z01;
 #pragma unroll
-    for (int j = 0; j < NQ; ++j) {
-      const float d2 = sv[j] - m2;  // -inf for j >= nq
-      sv[j] = ex2(d2);
-      zs[j & 3] += sv[j];
-      ts[j & 3] += j < nq ? sv[j] * d2 : 0.f;
+    for (int j = 0; j < NQ; j += 4) {
+      const float2 d0 = add2(make_float2(sv[j], sv[j + 1]), nm);  // -inf for j >= nq
+      const float2 d1 = add2(make_float2(sv[j + 2], sv[j + 3]), nm);
+      sv[j] = ex2(d0.x);
+      sv[j + 1] = ex2(d0.y);
+      sv[j + 2] = ex2(d1.x);
+      sv[j + 3] = ex2(d1.y);
+      const float2 e0 = make_float2(sv[j], sv[j + 1]), e1 = make_float2(sv[j + 2], sv[j + 3]);
+      z01 = add2(z01, e0);
+      z23 = add2(z23, e1);
+      const float2 p0 = mul2(e0, d0), p1 = mul2(e1, d1);
+      t01 = add2(t01, make_float2(j < nq ? p0.x : 0.f, j + 1 < nq ? p0.y : 0.f));
+      t23 = add2(t23, make_float2(j + 2 < nq ? p1.x : 0.f, j + 3 < nq ? p1.y : 0.f));
     }
+    z = (z01.x + z01.y) + (z23.x + z23.y);
+    t2 = (t01.x + t01.y) + (t23.x + t23.y);
+    return;
   } else {
 #pragma unroll
     for (int j = 0; j < NQ; ++j) {

@@ -86,6 +86,12 @@ EDGE = [
     (1, 1, 6, 130, 128, 2, 1, 1),    # 130-key groups, two steps
     (1, 2, 10, 200, 64, 1, 2, 1),    # 200-key groups in two row groups
     (1, 1, 3, 1560, 128, 1, 1, 1),   # the (f,hw) blocks of the 480p latent: 13 position tiles
+    # unpaired R tiles (64 < b2 <= 128) with d = 128
+    (1, 2, 33, 128, 128, 1, 1, 2),   # 128 positions, 64-key groups
+    (1, 1, 21, 100, 128, 1, 2, 2),   # 50-key groups in a 64-key tile, uneven row groups
+    (2, 1, 17, 96, 128, 2, 1, 3),    # 32-key groups, two steps (Kt-only first R-update)
+    (1, 1, 9, 80, 128, 1, 1, 5),     # 16-key groups
+    (1, 1, 400, 72, 128, 1, 1, 2),   # 800 sub-items over the SMs: several tiles per warpgroup
 ]
 
 
