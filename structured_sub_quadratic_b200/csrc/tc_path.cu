@@ -870,19 +870,22 @@ __global__ void __launch_bounds__(192, 2)
 // Step-one aggregated queries under the uniform initial L (bf16):
 // Qt0[g][p][i][:] = mean_{l in p} q_(l,i).  One block per (g, p, i): 16-byte
 // column chunks x row lanes, every row load of a thread in flight at once;
-// the row lanes are summed in a fixed order (warp shuffles, then the 8 warps
-// through shared memory).  Launched with programmatic stream serialisation:
+// the row lanes are summed in a fixed order (warp shuffles, then the NT / 32
+// warps through shared memory).  NT = 256 threads while the blocks fit one
+// wave (5 per SM), else 128: more, smaller blocks resident at once (measured:
+// the 16K-token sweep's 1536 blocks 17.6 -> 13.1 us, the 480p latent's 624
+// blocks 0.9 us slower at 128).  Launched with programmatic stream serialisation:
 // its blocks may be scheduled while the previous kernel of the stream
 // finishes, but they wait for it before reading q (which may be that
 // kernel's output) and only then let the next kernel launch, so every later
 // kernel of the call (which reads K and V early) runs after all earlier work.
 // ---------------------------------------------------------------------------
-template <int D>
-__global__ void __launch_bounds__(256)
+template <int D, int NT>
+__global__ void __launch_bounds__(NT)
     init_qt_bf16_kernel(const bf16* __restrict__ q, bf16* __restrict__ qt0, Problem pb) {
   constexpr int CH = D / 8;        // 16-byte chunks per row
-  constexpr int RL = 256 / CH;     // row lanes
-  __shared__ float red[8][D];
+  constexpr int RL = NT / CH;      // row lanes
+  __shared__ float red[NT / 32][D];
   const int b1 = pb.b1, b2 = pb.b2, c1 = pb.c1;
   int bid = blockIdx.x;
   const int i = bid % b2;
@@ -922,7 +925,7 @@ __global__ void __launch_bounds__(256)
   if (threadIdx.x < D) {
     float sum = 0.f;
 #pragma unroll
-    for (int w8 = 0; w8 < 8; ++w8) sum += red[w8][threadIdx.x];
+    for (int w8 = 0; w8 < NT / 32; ++w8) sum += red[w8][threadIdx.x];
     qt0[((g * c1 + p) * b2 + i) * D + threadIdx.x] =
         __float2bfloat16_rn(l1 > l0 ? sum / (float)(l1 - l0) : 0.f);
   }
@@ -3232,8 +3235,12 @@ cudaError_t launch_r_step1(const bf16* q, const bf16* k, const bf16* v, bf16* qt
                            bf16* y, float* hs, const Problem& pb, int* status,
                            cudaStream_t stream, int* launches) {
   cudaError_t e = timed_launch("tc_init_qt", stream, launches, [&] {
-    return launch_pdl(init_qt_bf16_kernel<D>, dim3((unsigned)((long)pb.G * pb.c1 * pb.b2)),
-                      dim3(256), 0, stream, q, qt0, pb);
+    const long units = (long)pb.G * pb.c1 * pb.b2;
+    return units <= 5L * num_sms()
+               ? launch_pdl(init_qt_bf16_kernel<D, 256>, dim3((unsigned)units), dim3(256), 0,
+                            stream, q, qt0, pb)
+               : launch_pdl(init_qt_bf16_kernel<D, 128>, dim3((unsigned)units), dim3(128), 0,
+                            stream, q, qt0, pb);
   });
   if (e != cudaSuccess) return e;
   // column groups of <= 64 keys over <= 128 positions: the persistent kernel
