@@ -75,9 +75,8 @@ bool mul_ok(size_t a, size_t b, size_t* out) {
 bool aligned16(const void* p) { return p != nullptr && ((uintptr_t)p & 15u) == 0; }
 
 // Workspace of one call: none for the one-CTA-per-head kernel (small untiled
-// heads with T >= 2, whose later steps would otherwise run on the SIMT
-// kernels), the tensor-core path's if it takes the shape, else the SIMT
-// path's (fp32 pieces, each 256-byte aligned).
+// heads with T >= 2, every step kept on chip), the tensor-core path's if it
+// takes the shape, else the SIMT path's (fp32 pieces, each 256-byte aligned).
 struct Plan {
   bool small = false;
   bool tc = false;

@@ -953,7 +953,16 @@ struct KRArgs {
   int real_lo, real_hi;  // real tokens (padding): keys outside get zero weight
   int n_itiles;          // 128-position tiles per sub-item (b2 > 128 takes several)
   int tr;                // token order of k and v (see Problem)
+  // 0: step one, the aggregated queries Qt0 [G][c1][b2][d] of a row group;
+  // 1: later steps, every sub-item (g, p, k, q) has its own rows
+  // Qt [G][b1][c1][c2][b2][d]
+  int qt_per_item;
 };
+
+// First query row (in the tensor map of Qt0 or Qt) of sub-item (g, p, k, q).
+__device__ __forceinline__ int kr_qrow(const KRArgs& a, int g, int p, int k, int q) {
+  return a.qt_per_item ? (((g * a.b1 + k) * a.c1 + p) * a.c2 + q) * a.b2 : (g * a.c1 + p) * a.b2;
+}
 
 // Keys [*j_lo, *j_hi) of the nq keys of column group q (first key js) of
 // chunk k are real; an empty range marks a group without a real key.
@@ -1080,11 +1089,13 @@ __global__ void __launch_bounds__(128)
   uint64_t* o_full = bars + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 4);
+  uint64_t* q_full = bars + 5;  // later steps: the next group's query rows
 
   if (tid == 0) {
     mbar_init(load_full, 1);
     mbar_init(s_full, 1);
     mbar_init(o_full, 1);
+    mbar_init(q_full, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -1100,7 +1111,7 @@ __global__ void __launch_bounds__(128)
 
   pdl_launch_dependents();
   bool load_waited = false;
-  int s_issued = 0, o_issued = 0;
+  int s_issued = 0, o_issued = 0, q_loads = 0, q_waited = 0;
   auto issue_s = [&](int q) {
     tc_fence_after();
     const uint32_t qb = smem_u32(sQ), kb = smem_u32(sK(q));
@@ -1127,8 +1138,8 @@ __global__ void __launch_bounds__(128)
         tma_load_3d(sK(q) + (D / 64 + c) * L::kBox, &tm_v, load_full, c * 64, kyz.x, kyz.y);
       }
     }
-    pdl_wait();  // Qt0 comes from the previous kernel
-    const int qrow = (g * a.c1 + p) * a.b2 + i0;
+    pdl_wait();  // the queries come from the previous kernel
+    const int qrow = kr_qrow(a, g, p, k, 0) + i0;
 #pragma unroll
     for (int c = 0; c < D / 64; ++c) tma_load_2d(sQ + c * kRows * 128, &tm_qt, load_full, c * 64, qrow);
     load_waited = mbar_wait(load_full, 0, abort_flag, a.status);
@@ -1143,6 +1154,15 @@ __global__ void __launch_bounds__(128)
     real_keys(a.real_lo, a.real_hi, a.b2, k, js, nq, &jlo, &jhi);
     bool ok = mbar_wait(s_full, q & 1, abort_flag, a.status);
     ok = __all_sync(0xffffffffu, ok);
+    if (ok && a.qt_per_item && q + 1 < a.c2 && tid == 0) {
+      // S_q has read this group's rows: the next group's come in meanwhile
+      mbar_arrive_expect_tx(q_full, D / 64 * kRows * 128);
+      const int qrow = kr_qrow(a, g, p, k, q + 1) + i0;
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c)
+        tma_load_2d(sQ + c * kRows * 128, &tm_qt, q_full, c * 64, qrow);
+      ++q_loads;
+    }
     float z = 0.f, t2 = 0.f;
     if (ok) {
       tc_fence_after();
@@ -1239,10 +1259,18 @@ __global__ void __launch_bounds__(128)
     tc_fence_before();
     __syncthreads();
     if (*abort_flag) break;
-    if (tid == 0 && q + 1 < a.c2) issue_s(q + 1);
+    if (tid == 0 && q + 1 < a.c2) {
+      bool qok = true;
+      if (a.qt_per_item) {
+        qok = mbar_wait(q_full, q_waited & 1, abort_flag, a.status);
+        if (qok) ++q_waited;
+      }
+      if (qok) issue_s(q + 1);
+    }
   }
   if (tid == 0 && *abort_flag) {
     if (!load_waited) drain(load_full, 0);
+    if (q_loads > q_waited) drain(q_full, q_waited & 1);
     if (s_issued > 0) drain(s_full, (s_issued - 1) & 1);
     if (o_issued > 0) drain(o_full, (o_issued - 1) & 1);
   }
@@ -1343,11 +1371,11 @@ __global__ void __launch_bounds__(128)
     tma_prefetch_desc(&tm_qt);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
-    pdl_wait();  // Qt0 comes from the previous kernel
+    pdl_wait();  // the queries come from the previous kernel
     mbar_arrive_expect_tx(q_full, (D / 64) * L::kChunk);
 #pragma unroll
     for (int c = 0; c < D / 64; ++c)
-      tma_load_2d(sQ + c * L::kChunk, &tm_qt, q_full, c * 64, (g * a.c1 + p) * a.b2 + i0);
+      tma_load_2d(sQ + c * L::kChunk, &tm_qt, q_full, c * 64, kr_qrow(a, g, p, k, q) + i0);
   }
   const int r = tid;  // tile row = position i0 + r
   float m = -INFINITY, z = 0.f, t2 = 0.f;
@@ -2880,7 +2908,8 @@ cudaError_t dispatch_ko(const bf16* q, const bf16* kt, const bf16* y, const floa
 
 template <int D, int NQ>
 cudaError_t launch_kr(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, bf16* y, float* hs,
-                      const Problem& pb, int* status, cudaStream_t stream, int* launches) {
+                      const Problem& pb, int* status, cudaStream_t stream, int* launches,
+                      bool qt_per_item = false, bool write_y = false) {
   using L = KRLayout<D, NQ>;
   constexpr int kMaxBytes = L::bytes(256 / NQ);
   static std::once_flag attr_once;
@@ -2896,7 +2925,8 @@ cudaError_t launch_kr(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, b
   if (L::bytes(pb.c2) > kMaxBytes) return cudaErrorInvalidValue;
   CUtensorMap tq, tk, tv;
   {
-    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)pb.G * pb.c1 * pb.b2};
+    const cuuint64_t rows = (cuuint64_t)pb.G * pb.c1 * pb.b2 * (qt_per_item ? pb.b1 * pb.c2 : 1);
+    const cuuint64_t dims[2] = {(cuuint64_t)D, rows};
     const cuuint64_t str[1] = {(cuuint64_t)D * 2};
     const cuuint32_t box[2] = {64, kRows};
     if (!make_map(&tq, qt0, 2, dims, str, box)) return cudaErrorInvalidValue;
@@ -2924,7 +2954,8 @@ cudaError_t launch_kr(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, b
   a.b2 = pb.b2;
   a.c1 = pb.c1;
   a.c2 = pb.c2;
-  a.write_y = pb.T == 1 ? 1 : 0;
+  a.write_y = (qt_per_item ? write_y : pb.T == 1) ? 1 : 0;
+  a.qt_per_item = qt_per_item ? 1 : 0;
   a.sc_log2 = kLog2e * pb.sc;
   a.status = status;
   a.tr = pb.tr;
@@ -3012,7 +3043,8 @@ inline int kr_group_tile(const Problem& pb) {
 template <int D>
 cudaError_t launch_krl(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, bf16* y,
                        float* hs, const Problem& pb, int* status, cudaStream_t stream,
-                       int* launches) {
+                       int* launches,
+                       bool qt_per_item = false, bool write_y = false) {
   using L = KRLLayout<D>;
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
@@ -3023,7 +3055,8 @@ cudaError_t launch_krl(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, 
   if (attr_err != cudaSuccess) return attr_err;
   CUtensorMap tq, tk, tv, tkt, tyy;
   {
-    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)pb.G * pb.c1 * pb.b2};
+    const cuuint64_t rows = (cuuint64_t)pb.G * pb.c1 * pb.b2 * (qt_per_item ? pb.b1 * pb.c2 : 1);
+    const cuuint64_t dims[2] = {(cuuint64_t)D, rows};
     const cuuint64_t str[1] = {(cuuint64_t)D * 2};
     const cuuint32_t box[2] = {64, kRows};
     if (!make_map(&tq, qt0, 2, dims, str, box)) return cudaErrorInvalidValue;
@@ -3049,7 +3082,8 @@ cudaError_t launch_krl(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, 
   a.b2 = pb.b2;
   a.c1 = pb.c1;
   a.c2 = pb.c2;
-  a.write_y = pb.T == 1 ? 1 : 0;
+  a.write_y = (qt_per_item ? write_y : pb.T == 1) ? 1 : 0;
+  a.qt_per_item = qt_per_item ? 1 : 0;
   a.sc_log2 = kLog2e * pb.sc;
   a.status = status;
   a.tr = pb.tr;
@@ -3188,20 +3222,15 @@ cudaError_t launch_kl_two_pass(const bf16* q, const bf16* kt, const float* hs, f
   });
 }
 
-// Steps >= 2 run on the tensor cores when the R-update's column groups take
-// the persistent kernel (<= 64 keys, <= 128 positions); the non-final
-// L-update takes one tile each way (rows of <= 128 keys, row groups of <= 128
-// rows) in one kernel, any other shape in the two-pass pair.
-bool tc_later_steps(const Problem& pb) {
-  return kr_group_tile(pb) <= 64 && pb.b2 <= kRows;
-}
-
 bool kl_single_tile(const Problem& pb) {
   return pb.b1 * pb.c2 <= 128 && (pb.b1 + pb.c1 - 1) / pb.c1 <= kRows;
 }
 
 // One later step: the non-final L-update (aggregated queries Qt of every
-// sub-item), then the R-update from them.
+// sub-item), then the R-update from them.  The L-update takes one tile each
+// way (rows of <= 128 keys, row groups of <= 128 rows) in one kernel, any
+// other shape in the two-pass pair; the R-update takes the kernel step one
+// takes for the same groups, reading each sub-item's own query rows.
 template <int D>
 cudaError_t launch_later_step(const bf16* q, const bf16* k, const bf16* v, bf16* qt, bf16* kt,
                               bf16* y, float* hs, float* lse, const Problem& pb, bool last,
@@ -3210,18 +3239,37 @@ cudaError_t launch_later_step(const bf16* q, const bf16* k, const bf16* v, bf16*
                       ? launch_kl<D>(q, kt, hs, qt, pb, status, stream, launches)
                       : launch_kl_two_pass<D>(q, kt, hs, lse, qt, pb, status, stream, launches);
   if (e != cudaSuccess) return e;
-  switch (kr_group_tile(pb)) {
+  if (kr_group_tile(pb) <= 64 && pb.b2 <= kRows) {
+    switch (kr_group_tile(pb)) {
 #define MONARCH_KR2_STEP(NQ)                                                                   \
   case NQ:                                                                                     \
     return pb.b2 <= 64 ? launch_kr2<D, NQ, true>(qt, k, v, kt, y, hs, pb, status, stream,     \
                                                  launches, true, last)                         \
                        : launch_kr2<D, NQ, false>(qt, k, v, kt, y, hs, pb, status, stream,    \
                                                   launches, true, last);
-    MONARCH_KR2_STEP(16)
-    MONARCH_KR2_STEP(32)
-    MONARCH_KR2_STEP(48)
-    MONARCH_KR2_STEP(64)
+      MONARCH_KR2_STEP(16)
+      MONARCH_KR2_STEP(32)
+      MONARCH_KR2_STEP(48)
+      MONARCH_KR2_STEP(64)
 #undef MONARCH_KR2_STEP
+      default: return cudaErrorInvalidValue;
+    }
+  }
+  if (!kr_holds_groups(pb))
+    return launch_krl<D>(qt, k, v, kt, y, hs, pb, status, stream, launches, true, last);
+  switch (kr_group_tile(pb)) {
+#define MONARCH_KR_STEP(NQ)                                                                   \
+  case NQ:                                                                                    \
+    return launch_kr<D, NQ>(qt, k, v, kt, y, hs, pb, status, stream, launches, true, last);
+    MONARCH_KR_STEP(16)
+    MONARCH_KR_STEP(32)
+    MONARCH_KR_STEP(48)
+    MONARCH_KR_STEP(64)
+    MONARCH_KR_STEP(80)
+    MONARCH_KR_STEP(96)
+    MONARCH_KR_STEP(112)
+    MONARCH_KR_STEP(128)
+#undef MONARCH_KR_STEP
     default: return cudaErrorInvalidValue;
   }
 }
@@ -3319,9 +3367,7 @@ bool tc_supports(const Problem& pb) {
   return encode_fn() != nullptr;
 }
 
-bool tc_takes_transposed(const Problem& pb) {
-  return tc_supports(pb) && (pb.T == 1 || tc_later_steps(pb));
-}
+bool tc_takes_transposed(const Problem& pb) { return tc_supports(pb); }
 
 size_t tc_workspace_bytes(const Problem& pb) {
   size_t total = 0;
@@ -3340,23 +3386,12 @@ cudaError_t tc_forward(const bf16* q, const bf16* k, const bf16* v, bf16* out, c
                               : launch_r_step1<64>(q, k, v, qt0, kt, y, ws.hs, pb, status, stream,
                                                    launches);
   if (e != cudaSuccess) return e;
-  const QtStrides s1 = {(long)pb.b1 * pb.c1 * pb.c2 * pb.b2 * pb.d,
-                        (long)pb.c1 * pb.c2 * pb.b2 * pb.d, (long)pb.c2 * pb.b2 * pb.d,
-                        (long)pb.b2 * pb.d, (long)pb.d};
-  const bool tc_steps = tc_later_steps(pb);
   bf16* qt = reinterpret_cast<bf16*>(ws.qt);  // bf16 rows in the fp32-sized piece
   for (int t = 2; t <= pb.T; ++t) {
-    if (tc_steps) {
-      e = pb.d == 128 ? launch_later_step<128>(q, k, v, qt, kt, y, ws.hs, ws.lse, pb, t == pb.T,
-                                               status, stream, launches)
-                      : launch_later_step<64>(q, k, v, qt, kt, y, ws.hs, ws.lse, pb, t == pb.T,
-                                              status, stream, launches);
-      if (e != cudaSuccess) return e;
-      continue;
-    }
-    e = simt_l_update<bf16, bf16>(q, kt, ws.hs, ws.lse, ws.qt, pb, stream, launches);
-    if (e != cudaSuccess) return e;
-    e = simt_r_update<bf16, bf16>(k, v, ws.qt, s1, kt, y, ws.hs, pb, t == pb.T, stream, launches);
+    e = pb.d == 128 ? launch_later_step<128>(q, k, v, qt, kt, y, ws.hs, ws.lse, pb, t == pb.T,
+                                             status, stream, launches)
+                    : launch_later_step<64>(q, k, v, qt, kt, y, ws.hs, ws.lse, pb, t == pb.T,
+                                            status, stream, launches);
     if (e != cudaSuccess) return e;
   }
   if (pb.d == 128) return dispatch_ko<128>(q, kt, y, ws.hs, out, pb, status, stream, launches);
