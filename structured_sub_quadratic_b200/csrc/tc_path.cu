@@ -2251,21 +2251,24 @@ __global__ void __launch_bounds__(128)
 // over all b1 c2 keys, S = q Kt^T / sqrt(d) + Hs a 128-key tile at a time
 // (double-buffered in TMEM), running max and sum in registers, one row per
 // thread of warps 1-4; warp 0 loads (TMA) and issues the MMAs.  No barrier
-// joins the row warps: each reads the biases itself, so a warp whose
-// bounded wait gives up cannot leave the others waiting.
+// joins the row warps: each stages the tile's biases in its own shared
+// copy (coalesced loads issued before it waits for S, then broadcasts), so
+// a warp whose bounded wait gives up cannot leave the others waiting.
 //
 // klm_kernel, one CTA per (g, i, p, key tile): for every row tile, S again,
 // P = exp(S - lse) (rows past the group and pad rows 0), and
 // [Qt~ | c] += P^T [Q | 1] in TMEM across the row tiles (the product of
-// kl_kernel, accumulated); then thread = key writes Qt = Qt~ / c.  One row
-// tile at a time: load Q, S, softmax, aggregation, each waiting for the last.
+// kl_kernel, accumulated); then thread = key writes Qt = Qt~ / c.  Queries
+// and P are double-buffered: the next row tile's queries load, and the
+// aggregation of this one runs, while the next S and softmax proceed.
 // ---------------------------------------------------------------------------
 template <int D>
 struct KLSLayout {
   static constexpr int kChunk = kRows * 128;
   static constexpr int kQOff = 0;                            // D / 64 chunks
   static constexpr int kKtOff = D / 64 * kChunk;             // 2 slots of D / 64 chunks
-  static constexpr int kBarOff = kKtOff + 2 * (D / 64) * kChunk;
+  static constexpr int kBiasOff = kKtOff + 2 * (D / 64) * kChunk;  // float [4 row warps][128]
+  static constexpr int kBarOff = kBiasOff + 4 * 128 * 4;
   static constexpr int kBytes = kBarOff + 16 * 8;
 };
 
@@ -2387,10 +2390,24 @@ __global__ void __launch_bounds__(160)
     const int l = row0 + r;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     float m_run = -INFINITY, z = 0.f;
+    float* wbias = reinterpret_cast<float*>(smem + L::kBiasOff) + (warp - 1) * 128;
     bool ok = true;
     for (int kt = 0; kt < n_kt && ok; ++kt) {
       const int sl = kt & 1;
       const int col0 = kt * 128;
+      // this tile's entropy biases, -inf past the row's keys (which also
+      // masks the zero-filled Kt rows there)
+      {
+        const float* hs_t = a.hs + key_row0 + col0;
+        float b[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          b[e] = col0 + e * 32 + lane < a.nk ? __ldg(hs_t + e * 32 + lane) : -INFINITY;
+        __syncwarp();  // the previous tile's reads of wbias are done
+#pragma unroll
+        for (int e = 0; e < 4; ++e) wbias[e * 32 + lane] = b[e];
+        __syncwarp();
+      }
       ok = mbar_wait(s_full + sl, (kt >> 1) & 1, abort_flag, a.status);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
@@ -2406,22 +2423,37 @@ __global__ void __launch_bounds__(160)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(s_free + sl);
+      // logits, maxima and sums on packed pairs (scalar roundings); the
+      // partial sums over columns c mod 4 are the pairs (0, 1) and (2, 3)
       float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      // the tile's entropy biases, read by every thread (L1 broadcasts)
-      const float* hs_t = a.hs + key_row0 + col0;
+      const float2 sc2 = make_float2(a.sc, a.sc);
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        sv[c] = col0 + c < a.nk ? fmaf(sv[c], a.sc, __ldg(hs_t + c)) : -INFINITY;
-        mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
+      for (int c = 0; c < 128; c += 4) {
+        const float4 b4 = *reinterpret_cast<const float4*>(wbias + c);
+        const float2 lo = fma2(make_float2(sv[c], sv[c + 1]), sc2, make_float2(b4.x, b4.y));
+        const float2 hi = fma2(make_float2(sv[c + 2], sv[c + 3]), sc2, make_float2(b4.z, b4.w));
+        sv[c] = lo.x;
+        sv[c + 1] = lo.y;
+        sv[c + 2] = hi.x;
+        sv[c + 3] = hi.y;
+        const int m = (c >> 2) & 1;
+        mx[m] = max3(mx[m], lo.x, lo.y);
+        mx[2 + m] = max3(mx[2 + m], hi.x, hi.y);
       }
       const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
       const float mn = fmaxf(m_run, mt);
       const float base = mn > -INFINITY ? mn : 0.f;
-      float zs[4] = {0.f, 0.f, 0.f, 0.f};
+      const float2 nb = make_float2(-base, -base), l2e = make_float2(kLog2e, kLog2e);
+      float2 z01 = make_float2(0.f, 0.f), z23 = z01;
 #pragma unroll
-      for (int c = 0; c < 128; ++c) zs[c & 3] += ex2((sv[c] - base) * kLog2e);
+      for (int c = 0; c < 128; c += 4) {
+        const float2 x0 = mul2(add2(make_float2(sv[c], sv[c + 1]), nb), l2e);
+        const float2 x1 = mul2(add2(make_float2(sv[c + 2], sv[c + 3]), nb), l2e);
+        z01 = add2(z01, make_float2(ex2(x0.x), ex2(x0.y)));
+        z23 = add2(z23, make_float2(ex2(x1.x), ex2(x1.y)));
+      }
       z = z * (m_run > -INFINITY ? ex2((m_run - base) * kLog2e) : 0.f) +
-          ((zs[0] + zs[1]) + (zs[2] + zs[3]));
+          ((z01.x + z01.y) + (z23.x + z23.y));
       m_run = mn;
     }
     if (ok && l < l1) a.lse[((long)g * a.b2 + i) * a.b1 + l] = m_run + logf(z);
@@ -2437,15 +2469,18 @@ __global__ void __launch_bounds__(160)
 template <int D>
 struct KLMLayout {
   static constexpr int kChunk = kRows * 128;
-  static constexpr int kQOff = 0;                          // D / 64 chunks, then the ones
-  static constexpr int kOnesOff = D / 64 * kChunk;
-  static constexpr int kKtOff = kOnesOff + kChunk;         // D / 64 chunks of 128 keys
-  static constexpr int kPOff = kKtOff + D / 64 * kChunk;   // keys 0-63, keys 64-127
-  static constexpr int kBiasOff = kPOff + 2 * kChunk;      // float [128]
+  // two query buffers, each D / 64 chunks and then a chunk of ones (the
+  // [Q | 1] operand), so that the next row tile's queries load during this one
+  static constexpr int kQBufBytes = (D / 64 + 1) * kChunk;
+  static constexpr int kQOff = 0;
+  static constexpr int kKtOff = 2 * kQBufBytes;            // D / 64 chunks of 128 keys
+  static constexpr int kPOff = kKtOff + D / 64 * kChunk;   // 2 buffers: keys 0-63, 64-127
+  static constexpr int kBiasOff = kPOff + 4 * kChunk;      // float [128]
   static constexpr int kBarOff = kBiasOff + 128 * 4;
-  static constexpr int kBytes = kBarOff + 8 * 8;
+  static constexpr int kBytes = kBarOff + 10 * 8;
   static constexpr uint32_t kTmemCols = D + 64 + 128 <= 256 ? 256 : 512;
   static constexpr uint32_t kSCol = kTmemCols - 128;       // S; [Qt~ | c] at [0, D + 64)
+  static_assert(kBytes <= 227 * 1024, "shared memory");
 };
 
 struct KLMArgs {
@@ -2459,7 +2494,7 @@ struct KLMArgs {
 };
 
 template <int D>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(256)
     klm_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kt,
                KLMArgs a) {
   using L = KLMLayout<D>;
@@ -2479,21 +2514,21 @@ __global__ void __launch_bounds__(128)
   const int l0 = group_start(a.b1, a.c1, p), l1 = group_start(a.b1, a.c1, p + 1);
   const long key_row0 = ((long)(g * a.b2 + i) * a.c1 + p) * a.nk + kt * 128;
   const int n_rt = (l1 - l0 + kRows - 1) / kRows;
-  uint8_t* sQ = smem + L::kQOff;
-  uint8_t* sOnes = smem + L::kOnesOff;
+  auto sQ = [&](int b) { return smem + L::kQOff + b * L::kQBufBytes; };
   uint8_t* sKt = smem + L::kKtOff;
-  uint8_t* sP = smem + L::kPOff;
+  auto sP = [&](int b) { return smem + L::kPOff + b * 2 * L::kChunk; };
   float* sBias = reinterpret_cast<float*>(smem + L::kBiasOff);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
   uint64_t* kt_full = bars + 0;
-  uint64_t* q_full = bars + 1;
-  uint64_t* s_full = bars + 2;
-  uint64_t* o_full = bars + 3;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 5);
+  uint64_t* q_full = bars + 1;  // [2], one per query buffer
+  uint64_t* s_full = bars + 3;
+  uint64_t* o_full = bars + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 6);
   if (tid == 0) {
     mbar_init(kt_full, 1);
     mbar_init(q_full, 1);
+    mbar_init(q_full + 1, 1);
     mbar_init(s_full, 1);
     mbar_init(o_full, 1);
     *abort_flag = 0;
@@ -2503,18 +2538,29 @@ __global__ void __launch_bounds__(128)
     tmem_alloc(tmem_slot, L::kTmemCols);
     tmem_relinquish();
   }
-  for (int x = tid; x < L::kChunk / 16; x += 128)
-    reinterpret_cast<uint4*>(sOnes)[x] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u,
-                                                     0x3F803F80u);
+  for (int b = 0; b < 2; ++b) {
+    uint4* ones = reinterpret_cast<uint4*>(sQ(b) + D / 64 * L::kChunk);
+    for (int x = tid; x < L::kChunk / 16; x += 256)
+      ones[x] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+  }
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tmem_s = tmem + L::kSCol;
-  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;  // warp w: lanes of w % 4
   pdl_wait();  // Kt, the entropies and the row statistics come from earlier kernels
   pdl_launch_dependents();
+  auto load_q = [&](int rt) {  // row tile rt's queries into buffer rt & 1 (one thread)
+    const int b = rt & 1;
+    mbar_arrive_expect_tx(q_full + b, (D / 64) * L::kChunk);
+    const int2 qyz = q_slab_yz(a.tr, g, a.b1, a.b2, i, l0 + rt * kRows);
+#pragma unroll
+    for (int c = 0; c < D / 64; ++c)
+      tma_load_3d(sQ(b) + c * L::kChunk, &tm_q, q_full + b, c * 64, qyz.x, qyz.y);
+  };
+  int q_loads = 0;
   if (tid == 0) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_kt);
@@ -2522,28 +2568,33 @@ __global__ void __launch_bounds__(128)
 #pragma unroll
     for (int c = 0; c < D / 64; ++c)
       tma_load_2d(sKt + c * L::kChunk, &tm_kt, kt_full, c * 64, (int)key_row0);
+    load_q(0);
+    q_loads = 1;
   }
-  const int key = kt * 128 + tid;
-  sBias[tid] = key < a.nk ? a.hs[key_row0 + tid] : -INFINITY;
+  const int key = kt * 128 + (tid & 127);
+  if (tid < 128) sBias[tid] = key < a.nk ? a.hs[key_row0 + tid] : -INFINITY;
   __syncthreads();
   const float* lse_i = a.lse + ((long)g * a.b2 + i) * a.b1;
   bool ok = true;
-  int issued_s = 0, issued_o = 0, q_loads = 0;
+  int issued_s = 0, issued_o = 0;
   for (int rt = 0; rt < n_rt && ok; ++rt) {
     const int row0 = l0 + rt * kRows;
-    // the previous aggregation has read sQ and sP; load this row tile's Q, then S
+    const int qb = rt & 1;
     if (tid == 0) {
-      mbar_arrive_expect_tx(q_full, (D / 64) * L::kChunk);
-      const int2 qyz = q_slab_yz(a.tr, g, a.b1, a.b2, i, row0);
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c)
-        tma_load_3d(sQ + c * L::kChunk, &tm_q, q_full, c * 64, qyz.x, qyz.y);
-      ++q_loads;
-      ok = mbar_wait(q_full, rt & 1, abort_flag, a.status) &&
+      // the next row tile's queries go to the other buffer once the
+      // aggregation that read it (row tile rt - 1) is done
+      if (rt + 1 < n_rt) {
+        if (rt >= 1) ok = mbar_wait(o_full, (rt - 1) & 1, abort_flag, a.status);
+        if (ok) {
+          load_q(rt + 1);
+          ++q_loads;
+        }
+      }
+      ok = ok && mbar_wait(q_full + qb, (rt >> 1) & 1, abort_flag, a.status) &&
            (rt > 0 || mbar_wait(kt_full, 0, abort_flag, a.status));
       if (ok) {
         tc_fence_after();
-        const uint64_t dq = desc_kmajor(smem_u32(sQ)), dk = desc_kmajor(smem_u32(sKt));
+        const uint64_t dq = desc_kmajor(smem_u32(sQ(qb))), dk = desc_kmajor(smem_u32(sKt));
         const uint32_t idesc = idesc_bf16(kRows, 128, false);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
@@ -2554,29 +2605,34 @@ __global__ void __launch_bounds__(128)
         ++issued_s;
       }
     }
-    // ---- P = exp(S - lse), thread = row ----
-    const int r = tid, l = row0 + r;
+    // ---- P = exp(S - lse): two threads per row (warps w and w + 4 share the
+    // TMEM lanes), each over 64 of the tile's keys ----
+    const int r = tid & 127, half = tid >> 7, l = row0 + r;
     const bool row_real = l < l1 && l * a.b2 + i >= a.real_lo && l * a.b2 + i < a.real_hi;
     const float lse_row = row_real ? lse_i[l] : 0.f;
-    ok = mbar_wait(s_full, rt & 1, abort_flag, a.status);
+    ok = ok && mbar_wait(s_full, rt & 1, abort_flag, a.status);
     ok = __syncthreads_and(ok);
     if (!ok) break;
     tc_fence_after();
-    float sv[128];
+    float sv[64];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < 2; ++c) {
       float t[32];
-      tmem_ld32(tmem_s + lane_off + c * 32, t);
+      tmem_ld32(tmem_s + lane_off + half * 64 + c * 32, t);
 #pragma unroll
       for (int e = 0; e < 32; ++e) sv[c * 32 + e] = t[e];
     }
     tmem_wait_ld();
+    // P of this row tile into buffer rt & 1, last read by the aggregation of
+    // row tile rt - 2 (complete: its successor's was waited for above)
+    uint8_t* pbuf = sP(rt & 1);
 #pragma unroll
-    for (int u = 0; u < 16; ++u) {  // 16-byte unit u holds keys 8u .. 8u + 7
+    for (int uu = 0; uu < 8; ++uu) {  // 16-byte unit u holds keys 8u .. 8u + 7
+      const int u = half * 8 + uu;
       float w[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        const float x = fmaf(sv[8 * u + e], a.sc, sBias[8 * u + e]);
+        const float x = fmaf(sv[8 * uu + e], a.sc, sBias[8 * u + e]);
         w[e] = row_real && x > -INFINITY ? ex2((x - lse_row) * kLog2e) : 0.f;
       }
       uint4 pk;
@@ -2584,16 +2640,15 @@ __global__ void __launch_bounds__(128)
       pk.y = pack_bf16x2(w[2], w[3]);
       pk.z = pack_bf16x2(w[4], w[5]);
       pk.w = pack_bf16x2(w[6], w[7]);
-      *reinterpret_cast<uint4*>(sP + (u >> 3) * L::kChunk + r * 128 + (((u & 7) ^ (r & 7)) << 4)) =
-          pk;
+      *reinterpret_cast<uint4*>(pbuf + half * L::kChunk + r * 128 + ((uu ^ (r & 7)) << 4)) = pk;
     }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     if (tid == 0) {
       tc_fence_after();
-      const uint64_t dp = desc_mnmajor(smem_u32(sP), L::kChunk);
-      const uint64_t dq = desc_mnmajor(smem_u32(sQ), L::kChunk);
+      const uint64_t dp = desc_mnmajor(smem_u32(pbuf), L::kChunk);
+      const uint64_t dq = desc_mnmajor(smem_u32(sQ(qb)), L::kChunk);
       const uint32_t idesc = idesc_bf16(kRows, D + 64, true, true);
 #pragma unroll
       for (int kk = 0; kk < kRows / 16; ++kk)
@@ -2601,12 +2656,14 @@ __global__ void __launch_bounds__(128)
                     (rt > 0 || kk > 0) ? 1u : 0u);
       mma_commit(o_full);
       ++issued_o;
-      ok = mbar_wait(o_full, rt & 1, abort_flag, a.status);  // sQ and sP free again
     }
-    ok = __syncthreads_and(ok);
   }
-  // ---- epilogue, thread = key ----
-  if (ok) {
+  // the last aggregation complete: [Qt~ | c] final
+  if (tid == 0 && ok && issued_o > 0)
+    ok = mbar_wait(o_full, (issued_o - 1) & 1, abort_flag, a.status);
+  ok = __syncthreads_and(ok);
+  // ---- epilogue, thread = key (warps 0-3) ----
+  if (ok && warp < 4) {
     tc_fence_after();
     float cs[32];
     tmem_ld32(tmem + lane_off + D, cs);
@@ -2634,7 +2691,7 @@ __global__ void __launch_bounds__(128)
   }
   if (tid == 0 && *abort_flag) {  // drain what this CTA issued (bounded)
     drain(kt_full, 0);
-    if (q_loads > 0) drain(q_full, (q_loads - 1) & 1);
+    for (int t = q_loads >= 2 ? q_loads - 2 : 0; t < q_loads; ++t) drain(q_full + (t & 1), (t >> 1) & 1);
     if (issued_s > 0) drain(s_full, (issued_s - 1) & 1);
     if (issued_o > 0) drain(o_full, (issued_o - 1) & 1);
   }
@@ -3217,7 +3274,7 @@ cudaError_t launch_kl_two_pass(const bf16* q, const bf16* kt, const float* hs, f
   am.status = status;
   am.tr = pb.tr;
   return timed_launch("tc_l_update", stream, launches, [&] {
-    return launch_pdl(klm_kernel<D>, dim3((unsigned)(units * am.key_tiles)), dim3(128),
+    return launch_pdl(klm_kernel<D>, dim3((unsigned)(units * am.key_tiles)), dim3(256),
                       LM::kBytes, stream, tq, tk, am);
   });
 }
