@@ -802,48 +802,66 @@ __global__ void __launch_bounds__(192, 2)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      // pass 1: row max of sc q.Kt + Hs over the valid keys
-      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      // logits sc q.Kt + Hs over the valid keys (one TMEM read, packed pairs
+      // with the scalar roundings), then the row max
+      float sv[NK];
 #pragma unroll
       for (int c = 0; c < NK / 32; ++c) {
         if (c < nch) {
           float t[32];
           tmem_ld32(tmem_s + lane_off + c * 32, t);
-          tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int col = c * 32 + e;
-            const float v = col < a.nk ? fmaf(t[e], sc, sBias[col]) : -INFINITY;
-            mx[e & 3] = fmaxf(mx[e & 3], v);
-          }
+          for (int e = 0; e < 32; ++e) sv[c * 32 + e] = t[e];
+        }
+      }
+      tmem_wait_ld();
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      const float2 sc2 = make_float2(sc, sc);
+#pragma unroll
+      for (int c = 0; c < NK; c += 4) {
+        if (c < nch * 32) {
+          const float4 b4 = *reinterpret_cast<const float4*>(sBias + c);
+          float2 lo = fma2(make_float2(sv[c], sv[c + 1]), sc2, make_float2(b4.x, b4.y));
+          float2 hi = fma2(make_float2(sv[c + 2], sv[c + 3]), sc2, make_float2(b4.z, b4.w));
+          sv[c] = c < a.nk ? lo.x : -INFINITY;
+          sv[c + 1] = c + 1 < a.nk ? lo.y : -INFINITY;
+          sv[c + 2] = c + 2 < a.nk ? hi.x : -INFINITY;
+          sv[c + 3] = c + 3 < a.nk ? hi.y : -INFINITY;
+          const int mm = (c >> 2) & 1;
+          mx[mm] = max3(mx[mm], sv[c], sv[c + 1]);
+          mx[2 + mm] = max3(mx[2 + mm], sv[c + 2], sv[c + 3]);
         }
       }
       const float m = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
       const float neg_m2 = -m * kLog2e;
-      // pass 2: P = exp(S - m) as bf16 pairs over the first columns of S (a
-      // chunk's P lands in columns already read), and the row sum
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      // P = exp(S - m) as bf16 pairs over the first columns of S (already
+      // read), and the row sum (partial sums over columns c mod 4)
+      const float2 l2e = make_float2(kLog2e, kLog2e), nm2 = make_float2(neg_m2, neg_m2);
+      float2 ls01 = make_float2(0.f, 0.f), ls23 = ls01;
+#pragma unroll
+      for (int c = 0; c < NK; c += 4) {
+        if (c < nch * 32) {
+          const float2 x0 = fma2(make_float2(sv[c], sv[c + 1]), l2e, nm2);
+          const float2 x1 = fma2(make_float2(sv[c + 2], sv[c + 3]), l2e, nm2);
+          sv[c] = ex2(x0.x);
+          sv[c + 1] = ex2(x0.y);
+          sv[c + 2] = ex2(x1.x);
+          sv[c + 3] = ex2(x1.y);
+          ls01 = add2(ls01, make_float2(sv[c], sv[c + 1]));
+          ls23 = add2(ls23, make_float2(sv[c + 2], sv[c + 3]));
+        }
+      }
 #pragma unroll
       for (int c = 0; c < NK / 32; ++c) {
         if (c < nch) {
-          float t[32];
-          tmem_ld32(tmem_s + lane_off + c * 32, t);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int col = c * 32 + e;
-            const float v = col < a.nk ? fmaf(t[e], sc, sBias[col]) : -INFINITY;
-            t[e] = ex2(fmaf(v, kLog2e, neg_m2));
-            ls[e & 3] += t[e];
-          }
           uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(t[2 * e], t[2 * e + 1]);
+          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(sv[c * 32 + 2 * e], sv[c * 32 + 2 * e + 1]);
           tmem_st16(tmem_s + lane_off + c * 16, pk);
         }
       }
       mbar_arrive(bias_empty);
-      const float l_row = (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      const float l_row = (ls01.x + ls01.y) + (ls23.x + ls23.y);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(p_full);
@@ -2024,14 +2042,16 @@ __global__ void __launch_bounds__(320, 1)
 
 // ---------------------------------------------------------------------------
 // Non-final L-update on the tensor cores, for rows of at most 128 keys
-// (nk = b1 c2) and row groups of at most 128 rows.  One CTA of four warps
+// (nk = b1 c2) and row groups of at most 128 rows.  One CTA of eight warps
 // per (g, i, p):
 //   S = q Kt^T / sqrt(d) + Hs           128 rows x 128 keys in TMEM
-//   L = softmax over the valid keys      exact, thread = row; rows past the
-//                                        group and pad rows get L = 0
+//   L = softmax over the valid keys      exact, two threads per row (64 keys
+//                                        each; maximum and sum combined in
+//                                        shared memory); rows past the group
+//                                        and pad rows get L = 0
 //   [Qt~ | c] = L^T [Q | 1]               128 keys x (d + 64) in TMEM, over the
 //                                        columns S held; c = column sums of L
-//   Qt_{k,p,q,i} = Qt~ / c (0 if c = 0)   thread = key, bf16 rows to global
+//   Qt_{k,p,q,i} = Qt~ / c (0 if c = 0)   thread = key (warps 0-3), bf16 rows
 // (MonarchAttention OpenReview discussion, the alternating maximisation: the
 // L-update's row softmax, then the aggregated queries of the next
 // R-update.)  L goes to shared memory as bf16 in [row][key] order: with keys
@@ -2064,7 +2084,7 @@ struct KLArgs {
 };
 
 template <int D>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(256)
     kl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kt,
               KLArgs a) {
   using L = KLLayout<D>;
@@ -2104,7 +2124,7 @@ __global__ void __launch_bounds__(128)
     tmem_relinquish();
   }
   // the ones block: bf16 1.0 in every element
-  for (int x = tid; x < L::kChunk / 16; x += 128)
+  for (int x = tid; x < L::kChunk / 16; x += 256)
     reinterpret_cast<uint4*>(sOnes)[x] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u,
                                                      0x3F803F80u);
   fence_proxy_async_smem();
@@ -2112,7 +2132,7 @@ __global__ void __launch_bounds__(128)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;  // warp w: lanes of w % 4
   pdl_wait();  // Kt and the entropies come from the previous kernel
   pdl_launch_dependents();
   bool issued_s = false, issued_o = false;
@@ -2127,7 +2147,7 @@ __global__ void __launch_bounds__(128)
       tma_load_2d(sKt + c * L::kChunk, &tm_kt, load_full, c * 64, (int)key_row0);
     }
   }
-  sBias[tid] = tid < a.nk ? a.hs[key_row0 + tid] : -INFINITY;
+  if (tid < 128) sBias[tid] = tid < a.nk ? a.hs[key_row0 + tid] : -INFINITY;
   __syncthreads();
   if (tid == 0 && mbar_wait(load_full, 0, abort_flag, a.status)) {
     tc_fence_after();
@@ -2140,48 +2160,75 @@ __global__ void __launch_bounds__(128)
     mma_commit(s_full);
     issued_s = true;
   }
-  // ---- softmax, thread = row r of the group ----
-  const int r = tid, l = l0 + r;
+  // ---- softmax: two threads per row r of the group (warps w and w + 4
+  // share the TMEM lanes), each over 64 keys; the row's maximum and sum are
+  // combined through the Kt buffer, dead once S is complete ----
+  const int r = tid & 127, half = tid >> 7, l = l0 + r;
   const bool row_real = l < l1 && l * a.b2 + i >= a.real_lo && l * a.b2 + i < a.real_hi;
+  float* red = reinterpret_cast<float*>(sKt);  // [max: 2][128], [sum: 2][128]
   bool ok = mbar_wait(s_full, 0, abort_flag, a.status);
   ok = __syncthreads_and(ok);
+  float sv[64];
   if (ok) {
     tc_fence_after();
-    float sv[128];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < 2; ++c) {
       float t[32];
-      tmem_ld32(tmem + lane_off + c * 32, t);
+      tmem_ld32(tmem + lane_off + half * 64 + c * 32, t);
 #pragma unroll
       for (int e = 0; e < 32; ++e) sv[c * 32 + e] = t[e];
     }
     tmem_wait_ld();
+    // logits (-inf past nk and for groups without a real key) and maxima
     float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+    const float2 sc2 = make_float2(a.sc, a.sc);
 #pragma unroll
-    for (int c = 0; c < 128; ++c) {
-      sv[c] = fmaf(sv[c], a.sc, sBias[c]);  // -inf past nk and for groups without a real key
-      mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
+    for (int c = 0; c < 64; c += 4) {
+      const float4 b4 = *reinterpret_cast<const float4*>(sBias + half * 64 + c);
+      const float2 lo = fma2(make_float2(sv[c], sv[c + 1]), sc2, make_float2(b4.x, b4.y));
+      const float2 hi = fma2(make_float2(sv[c + 2], sv[c + 3]), sc2, make_float2(b4.z, b4.w));
+      sv[c] = lo.x;
+      sv[c + 1] = lo.y;
+      sv[c + 2] = hi.x;
+      sv[c + 3] = hi.y;
+      const int mm = (c >> 2) & 1;
+      mx[mm] = max3(mx[mm], lo.x, lo.y);
+      mx[2 + mm] = max3(mx[2 + mm], hi.x, hi.y);
     }
-    float m = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+    red[half * 128 + r] = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+  }
+  ok = __syncthreads_and(ok);
+  float m = 0.f;
+  if (ok) {
+    m = fmaxf(red[r], red[128 + r]);
     if (m == -INFINITY) m = 0.f;
-    const float neg_m2 = -m * kLog2e;
-    float zs[4] = {0.f, 0.f, 0.f, 0.f};
+    const float2 l2e = make_float2(kLog2e, kLog2e), nm2 = make_float2(-m * kLog2e, -m * kLog2e);
+    float2 z01 = make_float2(0.f, 0.f), z23 = z01;
 #pragma unroll
-    for (int c = 0; c < 128; ++c) {
-      sv[c] = ex2(fmaf(sv[c], kLog2e, neg_m2));
-      zs[c & 3] += sv[c];
+    for (int c = 0; c < 64; c += 4) {
+      const float2 x0 = fma2(make_float2(sv[c], sv[c + 1]), l2e, nm2);
+      const float2 x1 = fma2(make_float2(sv[c + 2], sv[c + 3]), l2e, nm2);
+      sv[c] = ex2(x0.x);
+      sv[c + 1] = ex2(x0.y);
+      sv[c + 2] = ex2(x1.x);
+      sv[c + 3] = ex2(x1.y);
+      z01 = add2(z01, make_float2(sv[c], sv[c + 1]));
+      z23 = add2(z23, make_float2(sv[c + 2], sv[c + 3]));
     }
-    const float z = (zs[0] + zs[1]) + (zs[2] + zs[3]);
+    red[256 + half * 128 + r] = (z01.x + z01.y) + (z23.x + z23.y);
+  }
+  ok = __syncthreads_and(ok);
+  if (ok) {
+    const float z = red[256 + r] + red[384 + r];
     const float inv = (row_real && z > 0.f) ? 1.f / z : 0.f;
 #pragma unroll
-    for (int u = 0; u < 16; ++u) {  // 16-byte unit u holds keys 8u .. 8u + 7
+    for (int uu = 0; uu < 8; ++uu) {  // this half's 16-byte units (keys 8u .. 8u + 7)
       uint4 pk;
-      pk.x = pack_bf16x2(sv[8 * u + 0] * inv, sv[8 * u + 1] * inv);
-      pk.y = pack_bf16x2(sv[8 * u + 2] * inv, sv[8 * u + 3] * inv);
-      pk.z = pack_bf16x2(sv[8 * u + 4] * inv, sv[8 * u + 5] * inv);
-      pk.w = pack_bf16x2(sv[8 * u + 6] * inv, sv[8 * u + 7] * inv);
-      *reinterpret_cast<uint4*>(sP + (u >> 3) * L::kChunk + r * 128 + (((u & 7) ^ (r & 7)) << 4)) =
-          pk;
+      pk.x = pack_bf16x2(sv[8 * uu + 0] * inv, sv[8 * uu + 1] * inv);
+      pk.y = pack_bf16x2(sv[8 * uu + 2] * inv, sv[8 * uu + 3] * inv);
+      pk.z = pack_bf16x2(sv[8 * uu + 4] * inv, sv[8 * uu + 5] * inv);
+      pk.w = pack_bf16x2(sv[8 * uu + 6] * inv, sv[8 * uu + 7] * inv);
+      *reinterpret_cast<uint4*>(sP + half * L::kChunk + r * 128 + ((uu ^ (r & 7)) << 4)) = pk;
     }
     fence_proxy_async_smem();
   }
@@ -2203,7 +2250,7 @@ __global__ void __launch_bounds__(128)
   // ---- epilogue, thread = key m = k c2 + q ----
   if (ok) ok = mbar_wait(o_full, 0, abort_flag, a.status);
   ok = __syncthreads_and(ok);
-  if (ok) {
+  if (ok && warp < 4) {
     tc_fence_after();
     const int m = tid;
     float cs[32];
@@ -3201,7 +3248,7 @@ cudaError_t launch_kl(const bf16* q, const bf16* kt, const float* hs, bf16* qt, 
   a.tr = pb.tr;
   const long blocks = (long)pb.G * pb.b2 * pb.c1;
   return timed_launch("tc_l_update", stream, launches, [&] {
-    return launch_pdl(kl_kernel<D>, dim3((unsigned)blocks), dim3(128), L::kBytes, stream, tq, tk,
+    return launch_pdl(kl_kernel<D>, dim3((unsigned)blocks), dim3(256), L::kBytes, stream, tq, tk,
                       a);
   });
 }
