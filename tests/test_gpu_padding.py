@@ -38,6 +38,11 @@ CASES = [
     (1, 2, 400 - 68, 100, 4, True, 64, 1, 1, 4, torch.bfloat16),
     (1, 2, 20 * 24 - 30, 20, 24, True, 64, 2, 2, 2, torch.bfloat16),
     (1, 2, 20 * 24 - 30, 20, 24, False, 64, 2, 2, 2, torch.float32),
+    # later steps through the two-pass L-update and the per-item / streaming R-updates
+    (1, 2, 140 * 80 - 100, 140, 80, True, 64, 2, 1, 2, torch.bfloat16),
+    (1, 1, 200 * 8 - 11, 200, 8, True, 64, 2, 1, 1, torch.bfloat16),
+    (1, 1, 52 * 90 - 40, 52, 90, True, 128, 2, 1, 1, torch.bfloat16),
+    (1, 1, 30 * 156 - 70, 30, 156, False, 128, 2, 1, 1, torch.bfloat16),
     (1, 2, 6 * 7 - 10, 6, 7, True, 64, 0, 1, 3, torch.float32),
     (1, 2, 6 * 7 - 10, 6, 7, False, 64, 0, 1, 3, torch.bfloat16),
     (1, 1, 5 * 6 - 4, 5, 6, True, 7, 2, 1, 2, torch.bfloat16),
