@@ -23,6 +23,9 @@
 
 #include <math.h>
 
+#include <type_traits>
+
+#include "bwd_tc.cuh"
 #include "simt_kernels.cuh"
 #include "timing.cuh"
 
@@ -379,8 +382,8 @@ inline unsigned ceil_div(long n, long m) { return (unsigned)((n + m - 1) / m); }
 
 template <typename TIn, int DV>
 cudaError_t run_bwd(const TIn* q, const TIn* k, const TIn* v, const TIn* dout, TIn* dq, TIn* dk,
-                    TIn* dv, const Problem& pb, const BwdWorkspace& ws, cudaStream_t stream,
-                    int* launches) {
+                    TIn* dv, const Problem& pb, const BwdWorkspace& ws, int* status,
+                    cudaStream_t stream, int* launches) {
   const int G = pb.G, b1 = pb.b1, b2 = pb.b2, c1 = pb.c1, c2 = pb.c2, d = pb.d;
   // forward intermediates: Qt0, Kt, Y, Hs (fp32)
   SimtWorkspace fw{};
@@ -393,13 +396,23 @@ cudaError_t run_bwd(const TIn* q, const TIn* k, const TIn* v, const TIn* dout, T
   if (e != cudaSuccess) return e;
   const size_t shm2 = (size_t)kWarps * 2 * d * sizeof(float);
   const size_t shm3 = (size_t)kWarps * 3 * d * sizeof(float);
-  e = timed_launch("bwd_l_rows", stream, launches, [&] {
+  bool l_side_done = false;
+  if constexpr (std::is_same<TIn, bf16>::value) {
+    if (bwd_tc_l_side_supports(pb)) {
+      e = bwd_tc_l_side(q, dout, ws.kt, ws.y, ws.hs, reinterpret_cast<bf16*>(ws.kt16),
+                        reinterpret_cast<bf16*>(ws.y16), ws.dq1, ws.dkt, ws.dy, ws.dhs, pb,
+                        status, stream, launches);
+      if (e != cudaSuccess) return e;
+      l_side_done = true;
+    }
+  }
+  if (!l_side_done) e = timed_launch("bwd_l_rows", stream, launches, [&] {
     l_bwd_rows_kernel<TIn, DV><<<ceil_div((long)G * b2 * ceil_div(b1, kWarps), 1), kThreads,
                                  shm2, stream>>>(q, dout, ws.kt, ws.y, ws.hs, ws.dq1, ws.lse,
                                                  ws.delta, pb);
   });
   if (e != cudaSuccess) return e;
-  e = timed_launch("bwd_l_keys", stream, launches, [&] {
+  if (!l_side_done) e = timed_launch("bwd_l_keys", stream, launches, [&] {
     l_bwd_keys_kernel<TIn, DV><<<(unsigned)((long)G * b2 * c1 * ceil_div((long)b1 * c2, kWarps)),
                                  kThreads, shm2, stream>>>(q, dout, ws.kt, ws.y, ws.hs, ws.lse,
                                                            ws.delta, ws.dkt, ws.dy, ws.dhs, pb);
@@ -440,25 +453,30 @@ BwdWorkspaceSizes bwd_workspace_sizes(const Problem& pb) {
   s.rbuf = G * b1 * c1 * b2 * b2;
   s.dsbuf = s.rbuf;
   s.dqt0_part = G * c1 * b2 * b1 * c2 * d;
+  s.kt16 = (s.kt + 1) / 2;
+  s.y16 = s.kt16;
   return s;
 }
 
 template <typename TIn>
 cudaError_t bwd_forward_t1(const TIn* q, const TIn* k, const TIn* v, const TIn* dout, TIn* dq,
                            TIn* dk, TIn* dv, const Problem& pb, const BwdWorkspace& ws,
-                           cudaStream_t stream, int* launches) {
+                           int* status, cudaStream_t stream, int* launches) {
   if (pb.T != 1 || is_padded(pb)) return cudaErrorInvalidValue;
-  if (pb.d <= 32) return run_bwd<TIn, 1>(q, k, v, dout, dq, dk, dv, pb, ws, stream, launches);
-  if (pb.d <= 64) return run_bwd<TIn, 2>(q, k, v, dout, dq, dk, dv, pb, ws, stream, launches);
-  if (pb.d <= 128) return run_bwd<TIn, 4>(q, k, v, dout, dq, dk, dv, pb, ws, stream, launches);
-  return run_bwd<TIn, 8>(q, k, v, dout, dq, dk, dv, pb, ws, stream, launches);
+  if (pb.d <= 32)
+    return run_bwd<TIn, 1>(q, k, v, dout, dq, dk, dv, pb, ws, status, stream, launches);
+  if (pb.d <= 64)
+    return run_bwd<TIn, 2>(q, k, v, dout, dq, dk, dv, pb, ws, status, stream, launches);
+  if (pb.d <= 128)
+    return run_bwd<TIn, 4>(q, k, v, dout, dq, dk, dv, pb, ws, status, stream, launches);
+  return run_bwd<TIn, 8>(q, k, v, dout, dq, dk, dv, pb, ws, status, stream, launches);
 }
 
 template cudaError_t bwd_forward_t1<float>(const float*, const float*, const float*, const float*,
                                            float*, float*, float*, const Problem&,
-                                           const BwdWorkspace&, cudaStream_t, int*);
+                                           const BwdWorkspace&, int*, cudaStream_t, int*);
 template cudaError_t bwd_forward_t1<bf16>(const bf16*, const bf16*, const bf16*, const bf16*,
                                           bf16*, bf16*, bf16*, const Problem&,
-                                          const BwdWorkspace&, cudaStream_t, int*);
+                                          const BwdWorkspace&, int*, cudaStream_t, int*);
 
 }  // namespace monarch

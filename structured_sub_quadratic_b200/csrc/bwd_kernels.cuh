@@ -8,21 +8,26 @@
 namespace monarch {
 
 // fp32 workspace pieces (element counts); layouts in bwd_kernels.cu.
+// (kt16, y16: bf16 copies of Kt and Y for the tensor-core L side, counted in
+// floats.)
 struct BwdWorkspaceSizes {
-  size_t qt0, kt, y, hs, lse, delta, dq1, dkt, dy, dhs, rbuf, dsbuf, dqt0_part;
+  size_t qt0, kt, y, hs, lse, delta, dq1, dkt, dy, dhs, rbuf, dsbuf, dqt0_part, kt16, y16;
 };
 
 struct BwdWorkspace {
-  float *qt0, *kt, *y, *hs, *lse, *delta, *dq1, *dkt, *dy, *dhs, *rbuf, *dsbuf, *dqt0_part;
+  float *qt0, *kt, *y, *hs, *lse, *delta, *dq1, *dkt, *dy, *dhs, *rbuf, *dsbuf, *dqt0_part,
+      *kt16, *y16;
 };
 
 BwdWorkspaceSizes bwd_workspace_sizes(const Problem& pb);
 
 // Gradients dq, dk, dv of sum(O * dout) for the forward pass with T = 1
-// (unpadded), on `stream`; adds its launch count to *launches.
+// (unpadded), on `stream`; adds its launch count to *launches.  bf16 shapes
+// the tensor-core L side takes (bwd_tc.cuh) run it there; `status` is the
+// device status word its bounded waits set on timeout.
 template <typename TIn>
 cudaError_t bwd_forward_t1(const TIn* q, const TIn* k, const TIn* v, const TIn* dout, TIn* dq,
                            TIn* dk, TIn* dv, const Problem& pb, const BwdWorkspace& ws,
-                           cudaStream_t stream, int* launches);
+                           int* status, cudaStream_t stream, int* launches);
 
 }  // namespace monarch

@@ -1,0 +1,29 @@
+// Host-side interface of the tensor-core (tcgen05) L side of the backward
+// pass (bf16, T = 1).
+#pragma once
+
+#include "common.cuh"
+
+namespace monarch {
+
+// True when the tensor-core L side takes this backward shape: d in {64, 128},
+// rows of at most 128 keys (b1 c2 <= 128), row groups of at most 128 rows,
+// Monarch token order, no padding.
+bool bwd_tc_l_side_supports(const Problem& pb);
+
+// The L side of the backward pass on the tensor cores.  Inputs: q and dO
+// (bf16, (G, N, d)), the recomputed fp32 Kt, Y [G][b2][c1][b1][c2][d] and Hs;
+// kt16 and y16 are bf16 scratch of Kt's size that receive their bf16
+// copies.  Outputs, fp32, in the layouts the R side reads:
+//   dq1 [G][N][d]   the L side's part of dq: sc sum_{k,q} dS_L Kt
+//   dkt, dy         [G][b2][c1][b1][c2][d]: sc sum_l dS_L q, sum_l L dO
+//   dhs             [G][b2][c1][b1][c2]: sum_l dS_L
+// with L the final L-update's weights, dS_L = L (dO . Y - delta) and
+// delta = dO . O = sum_{k,q} L (dO . Y).  `status` is the device status word
+// that the bounded waits set on timeout.  Adds its launches to *launches.
+cudaError_t bwd_tc_l_side(const bf16* q, const bf16* dout, const float* kt, const float* y,
+                          const float* hs, bf16* kt16, bf16* y16, float* dq1, float* dkt,
+                          float* dy, float* dhs, const Problem& pb, int* status,
+                          cudaStream_t stream, int* launches);
+
+}  // namespace monarch

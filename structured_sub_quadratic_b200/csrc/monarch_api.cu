@@ -537,6 +537,8 @@ int monarch_attn_bwd(int dtype, const void* q, const void* k, const void* v, con
   for (int t = 0; t < kPieces; ++t) total += align_up(f[t] * sizeof(float));
   std::lock_guard<std::mutex> lock(g_mu);
   if ((st = ensure(g_bwd[dev], total)) != MONARCH_OK) return st;
+  int* status = nullptr;
+  if ((st = status_word_locked(dev, &status)) != MONARCH_OK) return st;
   monarch::BwdWorkspace ws;
   float** dst = &ws.qt0;
   char* base = static_cast<char*>(g_bwd[dev].ptr);
@@ -552,12 +554,12 @@ int monarch_attn_bwd(int dtype, const void* q, const void* k, const void* v, con
                 static_cast<const bf16*>(q), static_cast<const bf16*>(k),
                 static_cast<const bf16*>(v), static_cast<const bf16*>(dout),
                 static_cast<bf16*>(dq), static_cast<bf16*>(dk), static_cast<bf16*>(dv), pb, ws,
-                stream, &t_launches)
+                status, stream, &t_launches)
           : monarch::bwd_forward_t1<float>(
                 static_cast<const float*>(q), static_cast<const float*>(k),
                 static_cast<const float*>(v), static_cast<const float*>(dout),
                 static_cast<float*>(dq), static_cast<float*>(dk), static_cast<float*>(dv), pb, ws,
-                stream, &t_launches);
+                status, stream, &t_launches);
   return e == cudaSuccess ? MONARCH_OK : record_cuda(e);
 }
 

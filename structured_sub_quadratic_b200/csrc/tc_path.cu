@@ -3473,6 +3473,15 @@ bool tc_supports(const Problem& pb) {
 
 bool tc_takes_transposed(const Problem& pb) { return tc_supports(pb); }
 
+bool tc_make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
+                 const cuuint64_t* strides, const cuuint32_t* box) {
+  return make_map(m, base, rank, dims, strides, box);
+}
+
+bool tc_make_q_slab_map(CUtensorMap* m, const bf16* q, const Problem& pb, int D) {
+  return make_q_slab_map(m, q, pb, D);
+}
+
 size_t tc_workspace_bytes(const Problem& pb) {
   size_t total = 0;
   carve(pb, nullptr, &total);

@@ -1,6 +1,7 @@
 // Host-side interface of the tcgen05 tensor-core MonarchAttention path (bf16).
 #pragma once
 
+#include <cuda.h>
 #include <stddef.h>
 
 #include "common.cuh"
@@ -10,10 +11,20 @@ namespace monarch {
 // True when the tensor-core kernels take this shape.
 bool tc_supports(const Problem& pb);
 
-// True when every tensor-core kernel of this shape's forward pass takes q,
-// k, v and out in transposed token order (Problem::tr; the later steps of
-// some shapes run on SIMT kernels, which do not).
+// True when the tensor-core kernels of this shape's forward pass take q, k,
+// v and out in transposed token order (Problem::tr): every shape they take.
 bool tc_takes_transposed(const Problem& pb);
+
+// bf16 TMA tensor map with 128-byte swizzle (dims and box innermost first,
+// strides in bytes for dims 1..); encoded maps are cached.  False when the
+// driver rejects it.
+bool tc_make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
+                 const cuuint64_t* strides, const cuuint32_t* box);
+
+// 3-D map of q (or of any (G, N, d) bf16 tensor in q's layout) whose box is
+// the 128 rows l of one position i, from the coordinates (column, i,
+// g b1 + l0) in Monarch order.
+bool tc_make_q_slab_map(CUtensorMap* m, const bf16* q, const Problem& pb, int D);
 
 // Workspace bytes the tensor-core path needs for this shape.
 size_t tc_workspace_bytes(const Problem& pb);

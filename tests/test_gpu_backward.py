@@ -1,11 +1,12 @@
 """GPU backward pass (T = 1) against the float64 oracle's chain rule.
 
 The oracle's backward is pinned by finite differences and by dense-attention
-gradients (tests/test_oracle_backward.py).  The GPU computes in fp32 from the
-same input values, so the bar is max|g_gpu - g_oracle| <= 1e-4 max|g_oracle|
-for fp32 inputs, and 2e-2 max|g_oracle| for bf16 inputs, where the gradients
-are rounded to bf16 on output (the forward pass's bars, relative to the
-gradient's scale instead of V's).
+gradients (tests/test_oracle_backward.py).  The SIMT kernels compute in fp32
+from the same input values; the tensor-core L side (bf16 rows of <= 128 keys)
+multiplies bf16 operands into fp32.  The bar is max|g_gpu - g_oracle| <=
+1e-4 max|g_oracle| for fp32 inputs, and 2e-2 max|g_oracle| for bf16 inputs,
+where the gradients are rounded to bf16 on output (the forward pass's bars,
+relative to the gradient's scale instead of V's).
 """
 import numpy as np
 import pytest
@@ -53,3 +54,33 @@ def test_backward_is_deterministic(cuda_lib):
     b = cuda_lib.monarch_attn_bwd(q, k, v, dO, 30, 52, 1)
     torch.cuda.synchronize()
     assert all(torch.equal(x, y) for x, y in zip(a, b))
+
+
+TC_L_SIDE = [
+    # B, H, b1, b2, d, c1, c2: bf16 rows of <= 128 keys, groups of <= 128 rows
+    (1, 2, 90, 52, 128, 1, 1),   # the 480p latent's blocks
+    (1, 1, 64, 20, 64, 1, 2),    # 128 keys per row, 64-key groups
+    (1, 2, 100, 12, 128, 2, 1),  # 50-row groups
+    (2, 1, 13, 11, 64, 3, 5),    # tiled, ragged groups
+]
+
+
+@pytest.mark.parametrize("B,H,b1,b2,d,c1,c2", TC_L_SIDE)
+def test_backward_l_side_on_tensor_cores(cuda_lib, B, H, b1, b2, d, c1, c2):
+    q, k, v = iid_qkv(B, H, b1 * b2, d, torch.bfloat16, seed=b1 * 7 + b2)
+    dO = iid_qkv(B, H, b1 * b2, d, torch.bfloat16, seed=b1 * 7 + b2 + 1)[0]
+    cuda_lib.timing_read()
+    cuda_lib.timing_enable(True)
+    try:
+        got = cuda_lib.monarch_attn_bwd(q.cuda(), k.cuda(), v.cuda(), dO.cuda(), b1, b2, 1, c1, c2)
+        names = set(cuda_lib.timing_read())
+    finally:
+        cuda_lib.timing_enable(False)
+    cuda_lib.check()
+    assert "bwd_tc_l_side" in names and "bwd_l_rows" not in names, names
+    ref = monarch_attention_backward(*(x.double().numpy() for x in (q, k, v, dO)), b1, b2, c1, c2)
+    for name, g, r in zip(("dq", "dk", "dv"), got, ref):
+        g = g.double().cpu().numpy()
+        assert np.isfinite(g).all(), name
+        err, bound = np.abs(g - r).max(), TOL[torch.bfloat16] * np.abs(r).max()
+        assert err <= bound, f"{name}: max err {err:.3e} > {bound:.3e}"
