@@ -385,26 +385,34 @@ cudaError_t run_bwd(const TIn* q, const TIn* k, const TIn* v, const TIn* dout, T
                     TIn* dv, const Problem& pb, const BwdWorkspace& ws, int* status,
                     cudaStream_t stream, int* launches) {
   const int G = pb.G, b1 = pb.b1, b2 = pb.b2, c1 = pb.c1, c2 = pb.c2, d = pb.d;
-  // forward intermediates: Qt0, Kt, Y, Hs (fp32)
-  SimtWorkspace fw{};
-  fw.qt0 = ws.qt0;
-  fw.kt = ws.kt;
-  fw.y = ws.y;
-  fw.hs = ws.hs;
-  cudaError_t e = simt_forward<TIn, float>(q, k, v, (TIn*)nullptr, pb, fw, stream, launches,
-                                           false);
-  if (e != cudaSuccess) return e;
   const size_t shm2 = (size_t)kWarps * 2 * d * sizeof(float);
   const size_t shm3 = (size_t)kWarps * 3 * d * sizeof(float);
+  cudaError_t e = cudaSuccess;
   bool l_side_done = false;
   if constexpr (std::is_same<TIn, bf16>::value) {
+    // bf16 rows of <= 128 keys: the tensor-core step one recomputes the
+    // forward quantities and the tensor-core L side takes them
     if (bwd_tc_l_side_supports(pb)) {
-      e = bwd_tc_l_side(q, dout, ws.kt, ws.y, ws.hs, reinterpret_cast<bf16*>(ws.kt16),
-                        reinterpret_cast<bf16*>(ws.y16), ws.dq1, ws.dkt, ws.dy, ws.dhs, pb,
-                        status, stream, launches);
+      bf16* kt16 = reinterpret_cast<bf16*>(ws.kt16);
+      bf16* y16 = reinterpret_cast<bf16*>(ws.y16);
+      e = bwd_tc_recompute(q, k, v, reinterpret_cast<bf16*>(ws.qt016), kt16, y16, ws.hs, ws.qt0,
+                           pb, status, stream, launches);
+      if (e != cudaSuccess) return e;
+      e = bwd_tc_l_side(q, dout, kt16, y16, ws.hs, ws.dq1, ws.dkt, ws.dy, ws.dhs, pb, status,
+                        stream, launches);
       if (e != cudaSuccess) return e;
       l_side_done = true;
     }
+  }
+  if (!l_side_done) {
+    // forward intermediates: Qt0, Kt, Y, Hs (fp32)
+    SimtWorkspace fw{};
+    fw.qt0 = ws.qt0;
+    fw.kt = ws.kt;
+    fw.y = ws.y;
+    fw.hs = ws.hs;
+    e = simt_forward<TIn, float>(q, k, v, (TIn*)nullptr, pb, fw, stream, launches, false);
+    if (e != cudaSuccess) return e;
   }
   if (!l_side_done) e = timed_launch("bwd_l_rows", stream, launches, [&] {
     l_bwd_rows_kernel<TIn, DV><<<ceil_div((long)G * b2 * ceil_div(b1, kWarps), 1), kThreads,
@@ -453,6 +461,7 @@ BwdWorkspaceSizes bwd_workspace_sizes(const Problem& pb) {
   s.rbuf = G * b1 * c1 * b2 * b2;
   s.dsbuf = s.rbuf;
   s.dqt0_part = G * c1 * b2 * b1 * c2 * d;
+  s.qt016 = (s.qt0 + 1) / 2;
   s.kt16 = (s.kt + 1) / 2;
   s.y16 = s.kt16;
   return s;

@@ -8,15 +8,15 @@
 namespace monarch {
 
 // fp32 workspace pieces (element counts); layouts in bwd_kernels.cu.
-// (kt16, y16: bf16 copies of Kt and Y for the tensor-core L side, counted in
-// floats.)
+// (qt016, kt16, y16: the bf16 Qt0, Kt and Y of the tensor-core recompute,
+// counted in floats.)
 struct BwdWorkspaceSizes {
-  size_t qt0, kt, y, hs, lse, delta, dq1, dkt, dy, dhs, rbuf, dsbuf, dqt0_part, kt16, y16;
+  size_t qt0, kt, y, hs, lse, delta, dq1, dkt, dy, dhs, rbuf, dsbuf, dqt0_part, qt016, kt16, y16;
 };
 
 struct BwdWorkspace {
   float *qt0, *kt, *y, *hs, *lse, *delta, *dq1, *dkt, *dy, *dhs, *rbuf, *dsbuf, *dqt0_part,
-      *kt16, *y16;
+      *qt016, *kt16, *y16;
 };
 
 BwdWorkspaceSizes bwd_workspace_sizes(const Problem& pb);

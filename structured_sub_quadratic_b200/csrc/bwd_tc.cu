@@ -335,16 +335,11 @@ __global__ void __launch_bounds__(128, 1)
   }
 }
 
-// fp32 -> bf16 (round to nearest even) of two arrays of n elements each.
-__global__ void to_bf16_kernel(const float* __restrict__ a, const float* __restrict__ b,
-                               bf16* __restrict__ a16, bf16* __restrict__ b16, long n2) {
-  for (long x = blockIdx.x * (long)blockDim.x + threadIdx.x; x < n2;
-       x += (long)gridDim.x * blockDim.x) {
-    const float2 va = reinterpret_cast<const float2*>(a)[x];
-    const float2 vb = reinterpret_cast<const float2*>(b)[x];
-    reinterpret_cast<uint32_t*>(a16)[x] = pack_bf16x2(va.x, va.y);
-    reinterpret_cast<uint32_t*>(b16)[x] = pack_bf16x2(vb.x, vb.y);
-  }
+// bf16 -> fp32 of n elements.
+__global__ void to_f32_kernel(const bf16* __restrict__ a, float* __restrict__ out, long n) {
+  for (long x = blockIdx.x * (long)blockDim.x + threadIdx.x; x < n;
+       x += (long)gridDim.x * blockDim.x)
+    out[x] = __bfloat162float(a[x]);
 }
 
 template <int D>
@@ -393,23 +388,29 @@ cudaError_t launch_lbw(const bf16* q, const bf16* dout, const bf16* kt16, const 
 
 bool bwd_tc_l_side_supports(const Problem& pb) {
   if (pb.d != 64 && pb.d != 128) return false;
-  if (pb.tr || is_padded(pb) || pb.T != 1) return false;
+  if (pb.tr || is_padded(pb) || pb.T != 1 || !tc_supports(pb)) return false;
   if (pb.b1 * pb.c2 > kTile || (pb.b1 + pb.c1 - 1) / pb.c1 > kTile) return false;
   const long key_rows = (long)pb.G * pb.b2 * pb.c1 * pb.b1 * pb.c2;
   return key_rows + kTile < (1L << 31) && (long)pb.G * pb.b1 < (1L << 31);
 }
 
-cudaError_t bwd_tc_l_side(const bf16* q, const bf16* dout, const float* kt, const float* y,
-                          const float* hs, bf16* kt16, bf16* y16, float* dq1, float* dkt,
-                          float* dy, float* dhs, const Problem& pb, int* status,
-                          cudaStream_t stream, int* launches) {
+cudaError_t bwd_tc_recompute(const bf16* q, const bf16* k, const bf16* v, bf16* qt0_16,
+                             bf16* kt16, bf16* y16, float* hs, float* qt0, const Problem& pb,
+                             int* status, cudaStream_t stream, int* launches) {
   if (!bwd_tc_l_side_supports(pb)) return cudaErrorInvalidValue;
-  const long n2 = (long)pb.G * pb.b1 * pb.b2 * pb.c1 * pb.c2 * pb.d / 2;
-  cudaError_t e = timed_launch("bwd_tc_to_bf16", stream, launches, [&] {
-    to_bf16_kernel<<<(unsigned)std::min<long>((n2 + 255) / 256, 148L * 16), 256, 0, stream>>>(
-        kt, y, kt16, y16, n2);
-  });
+  cudaError_t e = tc_step_one(q, k, v, qt0_16, kt16, y16, hs, pb, status, stream, launches);
   if (e != cudaSuccess) return e;
+  const long n = (long)pb.G * pb.c1 * pb.b2 * pb.d;
+  return timed_launch("bwd_tc_qt0_f32", stream, launches, [&] {
+    to_f32_kernel<<<(unsigned)std::min<long>((n + 255) / 256, 148L * 8), 256, 0, stream>>>(
+        qt0_16, qt0, n);
+  });
+}
+
+cudaError_t bwd_tc_l_side(const bf16* q, const bf16* dout, const bf16* kt16, const bf16* y16,
+                          const float* hs, float* dq1, float* dkt, float* dy, float* dhs,
+                          const Problem& pb, int* status, cudaStream_t stream, int* launches) {
+  if (!bwd_tc_l_side_supports(pb)) return cudaErrorInvalidValue;
   return pb.d == 128 ? launch_lbw<128>(q, dout, kt16, y16, hs, dq1, dkt, dy, dhs, pb, status,
                                        stream, launches)
                      : launch_lbw<64>(q, dout, kt16, y16, hs, dq1, dkt, dy, dhs, pb, status,

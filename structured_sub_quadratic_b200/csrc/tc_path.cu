@@ -3482,6 +3482,15 @@ bool tc_make_q_slab_map(CUtensorMap* m, const bf16* q, const Problem& pb, int D)
   return make_q_slab_map(m, q, pb, D);
 }
 
+cudaError_t tc_step_one(const bf16* q, const bf16* k, const bf16* v, bf16* qt0, bf16* kt, bf16* y,
+                        float* hs, const Problem& pb, int* status, cudaStream_t stream,
+                        int* launches) {
+  if (!tc_supports(pb)) return cudaErrorInvalidValue;
+  return pb.d == 128
+             ? launch_r_step1<128>(q, k, v, qt0, kt, y, hs, pb, status, stream, launches)
+             : launch_r_step1<64>(q, k, v, qt0, kt, y, hs, pb, status, stream, launches);
+}
+
 size_t tc_workspace_bytes(const Problem& pb) {
   size_t total = 0;
   carve(pb, nullptr, &total);

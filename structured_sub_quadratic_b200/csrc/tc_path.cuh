@@ -26,6 +26,13 @@ bool tc_make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* d
 // g b1 + l0) in Monarch order.
 bool tc_make_q_slab_map(CUtensorMap* m, const bf16* q, const Problem& pb, int D);
 
+// Step one of the forward pass alone (the step-one aggregation, then the
+// R-update): bf16 Qt0 [G][c1][b2][d], Kt and Y [G][b2][c1][b1][c2][d] (Y
+// when pb.T == 1), fp32 Hs.  For shapes tc_supports() takes.
+cudaError_t tc_step_one(const bf16* q, const bf16* k, const bf16* v, bf16* qt0, bf16* kt, bf16* y,
+                        float* hs, const Problem& pb, int* status, cudaStream_t stream,
+                        int* launches);
+
 // Workspace bytes the tensor-core path needs for this shape.
 size_t tc_workspace_bytes(const Problem& pb);
 
