@@ -388,20 +388,31 @@ cudaError_t run_bwd(const TIn* q, const TIn* k, const TIn* v, const TIn* dout, T
   const size_t shm2 = (size_t)kWarps * 2 * d * sizeof(float);
   const size_t shm3 = (size_t)kWarps * 3 * d * sizeof(float);
   cudaError_t e = cudaSuccess;
-  bool l_side_done = false;
+  bool l_side_done = false, r_side_done = false;
   if constexpr (std::is_same<TIn, bf16>::value) {
     // bf16 rows of <= 128 keys: the tensor-core step one recomputes the
-    // forward quantities and the tensor-core L side takes them
+    // forward quantities and the tensor-core L side takes them; untiled
+    // chunks of <= 128 positions take the tensor-core R side too
     if (bwd_tc_l_side_supports(pb)) {
+      bf16* qt016 = reinterpret_cast<bf16*>(ws.qt016);
       bf16* kt16 = reinterpret_cast<bf16*>(ws.kt16);
       bf16* y16 = reinterpret_cast<bf16*>(ws.y16);
-      e = bwd_tc_recompute(q, k, v, reinterpret_cast<bf16*>(ws.qt016), kt16, y16, ws.hs, ws.qt0,
-                           pb, status, stream, launches);
+      const bool tc_r = bwd_tc_r_side_supports(pb);
+      bf16* dkt16 = tc_r ? reinterpret_cast<bf16*>(ws.dkt16) : nullptr;
+      bf16* dy16 = tc_r ? reinterpret_cast<bf16*>(ws.dy16) : nullptr;
+      e = bwd_tc_recompute(q, k, v, qt016, kt16, y16, ws.hs, ws.qt0, pb, status, stream,
+                           launches);
       if (e != cudaSuccess) return e;
-      e = bwd_tc_l_side(q, dout, kt16, y16, ws.hs, ws.dq1, ws.dkt, ws.dy, ws.dhs, pb, status,
-                        stream, launches);
+      e = bwd_tc_l_side(q, dout, kt16, y16, ws.hs, ws.dq1, ws.dkt, ws.dy, ws.dhs, dkt16, dy16, pb,
+                        status, stream, launches);
       if (e != cudaSuccess) return e;
       l_side_done = true;
+      if (tc_r) {
+        e = bwd_tc_r_side(qt016, k, v, dkt16, dy16, ws.dhs, ws.dqt0_part, dk, dv, pb, status,
+                          stream, launches);
+        if (e != cudaSuccess) return e;
+        r_side_done = true;
+      }
     }
   }
   if (!l_side_done) {
@@ -426,12 +437,12 @@ cudaError_t run_bwd(const TIn* q, const TIn* k, const TIn* v, const TIn* dout, T
                                                            ws.delta, ws.dkt, ws.dy, ws.dhs, pb);
   });
   if (e != cudaSuccess) return e;
-  e = timed_launch("bwd_r_rows", stream, launches, [&] {
+  if (!r_side_done) e = timed_launch("bwd_r_rows", stream, launches, [&] {
     r_bwd_rows_kernel<TIn, DV><<<(unsigned)((long)G * b1), kThreads, shm3, stream>>>(
         k, v, ws.qt0, ws.dkt, ws.dy, ws.dhs, ws.rbuf, ws.dsbuf, ws.dqt0_part, pb);
   });
   if (e != cudaSuccess) return e;
-  e = timed_launch("bwd_r_keys", stream, launches, [&] {
+  if (!r_side_done) e = timed_launch("bwd_r_keys", stream, launches, [&] {
     r_bwd_keys_kernel<TIn, DV><<<(unsigned)((long)G * b1 * ceil_div(b2, kWarps)), kThreads, 0,
                                  stream>>>(ws.qt0, ws.dkt, ws.dy, ws.rbuf, ws.dsbuf, dk, dv, pb);
   });
@@ -464,6 +475,8 @@ BwdWorkspaceSizes bwd_workspace_sizes(const Problem& pb) {
   s.qt016 = (s.qt0 + 1) / 2;
   s.kt16 = (s.kt + 1) / 2;
   s.y16 = s.kt16;
+  s.dkt16 = s.kt16;
+  s.dy16 = s.kt16;
   return s;
 }
 

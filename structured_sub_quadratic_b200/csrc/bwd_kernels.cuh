@@ -8,15 +8,16 @@
 namespace monarch {
 
 // fp32 workspace pieces (element counts); layouts in bwd_kernels.cu.
-// (qt016, kt16, y16: the bf16 Qt0, Kt and Y of the tensor-core recompute,
-// counted in floats.)
+// (qt016, kt16, y16: the bf16 Qt0, Kt and Y of the tensor-core recompute;
+// dkt16, dy16: bf16 dKt and dY for the tensor-core R side; counted in floats.)
 struct BwdWorkspaceSizes {
-  size_t qt0, kt, y, hs, lse, delta, dq1, dkt, dy, dhs, rbuf, dsbuf, dqt0_part, qt016, kt16, y16;
+  size_t qt0, kt, y, hs, lse, delta, dq1, dkt, dy, dhs, rbuf, dsbuf, dqt0_part, qt016, kt16, y16,
+      dkt16, dy16;
 };
 
 struct BwdWorkspace {
   float *qt0, *kt, *y, *hs, *lse, *delta, *dq1, *dkt, *dy, *dhs, *rbuf, *dsbuf, *dqt0_part,
-      *qt016, *kt16, *y16;
+      *qt016, *kt16, *y16, *dkt16, *dy16;
 };
 
 BwdWorkspaceSizes bwd_workspace_sizes(const Problem& pb);

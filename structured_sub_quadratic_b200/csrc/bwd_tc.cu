@@ -58,6 +58,8 @@ struct LBArgs {
   float* dkt;       // [G][b2][c1][nk][d]
   float* dy;
   float* dhs;       // [G][b2][c1][nk]
+  bf16* dkt16;      // optional bf16 copies, [G][c1][nk][b2][d] (chunk-major)
+  bf16* dy16;
   int b1, b2, c1, nk;
   float sc;
   int* status;
@@ -315,6 +317,23 @@ __global__ void __launch_bounds__(128, 1)
           *reinterpret_cast<float4*>(dyrow + c * 32 + e) =
               make_float4(u[e], u[e + 1], u[e + 2], u[e + 3]);
         }
+        if (a.dkt16 != nullptr) {
+          const long crow = (((long)g * a.c1 + p) * a.nk + m) * a.b2 + i;
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            uint4 pk, pv;
+            pk.x = pack_bf16x2(t[e] * a.sc, t[e + 1] * a.sc);
+            pk.y = pack_bf16x2(t[e + 2] * a.sc, t[e + 3] * a.sc);
+            pk.z = pack_bf16x2(t[e + 4] * a.sc, t[e + 5] * a.sc);
+            pk.w = pack_bf16x2(t[e + 6] * a.sc, t[e + 7] * a.sc);
+            pv.x = pack_bf16x2(u[e], u[e + 1]);
+            pv.y = pack_bf16x2(u[e + 2], u[e + 3]);
+            pv.z = pack_bf16x2(u[e + 4], u[e + 5]);
+            pv.w = pack_bf16x2(u[e + 6], u[e + 7]);
+            *reinterpret_cast<uint4*>(a.dkt16 + crow * D + c * 32 + e) = pk;
+            *reinterpret_cast<uint4*>(a.dy16 + crow * D + c * 32 + e) = pv;
+          }
+        }
       }
     }
     float cs[32];
@@ -335,6 +354,360 @@ __global__ void __launch_bounds__(128, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// R side of the backward, untiled (c1 = c2 = 1, b2 <= 128): one CTA of four
+// warps per chunk (g, k), rows i = the b2 positions, keys j = the chunk's b2
+// keys.  With the L side's dKt, dY (bf16, chunk-major) and dHs:
+//   S_R = sc Qt0 K^T,  R = softmax_j S_R,
+//   dR = dKt K^T + dY V^T - dHs (ln R + 1),  dS_R = R (dR - sum_j R dR),
+//   partial dQt0 = sc dS_R K,  dk = R^T dKt + sc dS_R^T Qt0,  dv = R^T dY
+// (the chain rule through Kt = R K, Y = R V and Hs = the entropy of R).  S_R
+// and dR are products into TMEM; one thread per row forms R and sc dS_R
+// (bf16, [row][key]); the three gradients are products with R^T and dS_R^T
+// as MN-major A operands.
+// ---------------------------------------------------------------------------
+template <int D>
+struct RBLayout {
+  static constexpr int kChunk = kTile * 128;
+  static constexpr int kQOff = 0;                          // Qt0 rows i
+  static constexpr int kKOff = kQOff + D / 64 * kChunk;    // K rows j
+  static constexpr int kVOff = kKOff + D / 64 * kChunk;    // V rows j
+  static constexpr int kDKOff = kVOff + D / 64 * kChunk;   // dKt rows i
+  static constexpr int kDYOff = kDKOff + D / 64 * kChunk;  // dY rows i
+  static constexpr int kROff = kDYOff + D / 64 * kChunk;   // R [i][j]: keys 0-63, 64-127
+  static constexpr int kDSOff = kROff + 2 * kChunk;        // sc dS_R [i][j]
+  static constexpr int kBarOff = kDSOff + 2 * kChunk;
+  static constexpr int kBytes = kBarOff + 8 * 8;
+  // TMEM: S_R [0, 128), dR [128, 256); then partial dQt0 over S_R, dv over
+  // dR, dk at [256, 256 + D)
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kDRCol = 128, kDKCol = 256;
+  static_assert(D == 64 || D == 128, "head dimension");
+  static_assert(kBytes <= 227 * 1024, "shared memory");
+};
+
+struct RBArgs {
+  const float* dhs;  // [G][b2 i][b1 k]
+  float* dqt0_part;  // [G][b2 i][b1 k][d]
+  bf16* dk;          // (G, N, d)
+  bf16* dv;
+  int b1, b2;
+  float sc;
+  int* status;
+};
+
+template <int D>
+__global__ void __launch_bounds__(128, 1)
+    rbw_kernel(const __grid_constant__ CUtensorMap tm_qt0, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_dk,
+               const __grid_constant__ CUtensorMap tm_dy, RBArgs a) {
+  using L = RBLayout<D>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int tid = threadIdx.x, warp = tid >> 5;
+  if (smem_u32(smem) & 1023u) {
+    if (tid == 0) atomicExch(a.status, 2);
+    return;
+  }
+  const int k = blockIdx.x % a.b1;
+  const int g = blockIdx.x / a.b1;
+  const int chunk_row0 = (g * a.b1 + k) * a.b2;  // keys j of chunk k; dKt, dY rows i of (g, k)
+  uint8_t* sQ = smem + L::kQOff;
+  uint8_t* sK = smem + L::kKOff;
+  uint8_t* sV = smem + L::kVOff;
+  uint8_t* sDK = smem + L::kDKOff;
+  uint8_t* sDY = smem + L::kDYOff;
+  uint8_t* sR = smem + L::kROff;
+  uint8_t* sDS = smem + L::kDSOff;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* load_full = bars + 0;
+  uint64_t* s_full = bars + 1;
+  uint64_t* o_full = bars + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 4);
+  if (tid == 0) {
+    mbar_init(load_full, 1);
+    mbar_init(s_full, 1);
+    mbar_init(o_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+  bool issued_s = false, issued_o = false;
+  if (tid == 0) {
+    tma_prefetch_desc(&tm_qt0);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_dk);
+    tma_prefetch_desc(&tm_dy);
+    mbar_arrive_expect_tx(load_full, 5 * (D / 64) * L::kChunk);
+#pragma unroll
+    for (int c = 0; c < D / 64; ++c) {
+      tma_load_2d(sQ + c * L::kChunk, &tm_qt0, load_full, c * 64, g * a.b2);
+      tma_load_2d(sK + c * L::kChunk, &tm_k, load_full, c * 64, chunk_row0);
+      tma_load_2d(sV + c * L::kChunk, &tm_v, load_full, c * 64, chunk_row0);
+      tma_load_2d(sDK + c * L::kChunk, &tm_dk, load_full, c * 64, chunk_row0);
+      tma_load_2d(sDY + c * L::kChunk, &tm_dy, load_full, c * 64, chunk_row0);
+    }
+    if (mbar_wait(load_full, 0, abort_flag, a.status)) {
+      tc_fence_after();
+      const uint32_t idesc = idesc_bf16(kTile, kTile, false);
+      const uint64_t dq = desc_kmajor(smem_u32(sQ)), dkk = desc_kmajor(smem_u32(sK));
+      const uint64_t dvv = desc_kmajor(smem_u32(sV)), ddk = desc_kmajor(smem_u32(sDK));
+      const uint64_t ddy = desc_kmajor(smem_u32(sDY));
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {  // S_R / sc = Qt0 K^T
+        const uint32_t off = ((kk >> 2) * L::kChunk + (kk & 3) * 32) >> 4;
+        mma_bf16_ss(tmem, dq + off, dkk + off, idesc, kk > 0 ? 1u : 0u);
+      }
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {  // dKt K^T
+        const uint32_t off = ((kk >> 2) * L::kChunk + (kk & 3) * 32) >> 4;
+        mma_bf16_ss(tmem + L::kDRCol, ddk + off, dkk + off, idesc, kk > 0 ? 1u : 0u);
+      }
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {  // + dY V^T
+        const uint32_t off = ((kk >> 2) * L::kChunk + (kk & 3) * 32) >> 4;
+        mma_bf16_ss(tmem + L::kDRCol, ddy + off, dvv + off, idesc, 1u);
+      }
+      mma_commit(s_full);
+      issued_s = true;
+    }
+  }
+  // ---- thread = row i: R, dR, sc dS_R ----
+  const int r = tid;
+  const bool row_ok = r < a.b2;
+  bool ok = mbar_wait(s_full, 0, abort_flag, a.status);
+  ok = __syncthreads_and(ok);
+  if (ok) {
+    tc_fence_after();
+    const float s2 = a.sc * kLog2e;  // logits in log2 units
+    float m = -INFINITY;
+#pragma unroll 1
+    for (int c = 0; c < kTile / 32; ++c) {
+      float t[32];
+      tmem_ld32(tmem + lane_off + c * 32, t);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        if (c * 32 + e < a.b2) m = fmaxf(m, t[e] * s2);
+    }
+    float z = 0.f;
+#pragma unroll 1
+    for (int c = 0; c < kTile / 32; ++c) {
+      float t[32];
+      tmem_ld32(tmem + lane_off + c * 32, t);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        if (c * 32 + e < a.b2) z += ex2(fmaf(t[e], s2, -m));
+    }
+    const float lz = m + log2f(z);  // log2 of the row's normaliser
+    const float dh = row_ok ? a.dhs[((long)g * a.b2 + r) * a.b1 + k] : 0.f;
+    // rho = sum_j R dR, with dR including the entropy term; R to its tile
+    float rho = 0.f;
+#pragma unroll 1
+    for (int c = 0; c < kTile / 32; ++c) {
+      float t[32], dr[32];
+      tmem_ld32(tmem + lane_off + c * 32, t);
+      tmem_ld32(tmem + lane_off + L::kDRCol + c * 32, dr);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float x2 = fmaf(t[e], s2, -lz);  // log2 R
+        const bool live = row_ok && c * 32 + e < a.b2;
+        const float w = live ? ex2(x2) : 0.f;
+        const float d_r = dr[e] - dh * (x2 * 0.69314718055994531f + 1.f);
+        rho = fmaf(w, live ? d_r : 0.f, rho);
+        t[e] = w;
+      }
+#pragma unroll
+      for (int uu = 0; uu < 4; ++uu) {
+        const float* w = t + 8 * uu;
+        uint4 pk;
+        pk.x = pack_bf16x2(w[0], w[1]);
+        pk.y = pack_bf16x2(w[2], w[3]);
+        pk.z = pack_bf16x2(w[4], w[5]);
+        pk.w = pack_bf16x2(w[6], w[7]);
+        *rk_unit(sR, r, c * 4 + uu) = pk;
+      }
+    }
+#pragma unroll 1
+    for (int c = 0; c < kTile / 32; ++c) {
+      float t[32], dr[32];
+      tmem_ld32(tmem + lane_off + c * 32, t);
+      tmem_ld32(tmem + lane_off + L::kDRCol + c * 32, dr);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float x2 = fmaf(t[e], s2, -lz);
+        const bool live = row_ok && c * 32 + e < a.b2;
+        const float w = live ? ex2(x2) : 0.f;
+        const float d_r = dr[e] - dh * (x2 * 0.69314718055994531f + 1.f);
+        t[e] = live ? a.sc * w * (d_r - rho) : 0.f;
+      }
+#pragma unroll
+      for (int uu = 0; uu < 4; ++uu) {
+        const float* w = t + 8 * uu;
+        uint4 pk;
+        pk.x = pack_bf16x2(w[0], w[1]);
+        pk.y = pack_bf16x2(w[2], w[3]);
+        pk.z = pack_bf16x2(w[4], w[5]);
+        pk.w = pack_bf16x2(w[6], w[7]);
+        *rk_unit(sDS, r, c * 4 + uu) = pk;
+      }
+    }
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  ok = __syncthreads_and(ok);
+  if (ok && tid == 0) {
+    tc_fence_after();
+    // partial dQt0 = (sc dS_R) K: A K-major (rows x keys), B = K MN-major
+    {
+      const uint32_t idesc = idesc_bf16(kTile, D, true);
+      const uint64_t da = desc_kmajor(smem_u32(sDS));
+      const uint64_t db = desc_mnmajor(smem_u32(sK), L::kChunk);
+#pragma unroll
+      for (int kk = 0; kk < kTile / 16; ++kk)
+        mma_bf16_ss(tmem, da + (((kk >> 2) * L::kChunk + (kk & 3) * 32) >> 4),
+                    db + ((kk * 16 * 128) >> 4), idesc, kk > 0 ? 1u : 0u);
+    }
+    // dk = R^T dKt + (sc dS_R)^T Qt0 and dv = R^T dY: A MN-major (keys
+    // contiguous in each row), B MN-major (d contiguous in each row)
+    {
+      const uint32_t idesc = idesc_bf16(kTile, D, true, true);
+      const uint64_t rw = desc_mnmajor(smem_u32(sR), L::kChunk);
+      const uint64_t ds = desc_mnmajor(smem_u32(sDS), L::kChunk);
+      const uint64_t bdk = desc_mnmajor(smem_u32(sDK), L::kChunk);
+      const uint64_t bq = desc_mnmajor(smem_u32(sQ), L::kChunk);
+      const uint64_t bdy = desc_mnmajor(smem_u32(sDY), L::kChunk);
+#pragma unroll
+      for (int kk = 0; kk < kTile / 16; ++kk) {
+        const uint32_t off = (kk * 16 * 128) >> 4;
+        mma_bf16_ss(tmem + L::kDKCol, rw + off, bdk + off, idesc, kk > 0 ? 1u : 0u);
+      }
+#pragma unroll
+      for (int kk = 0; kk < kTile / 16; ++kk) {
+        const uint32_t off = (kk * 16 * 128) >> 4;
+        mma_bf16_ss(tmem + L::kDKCol, ds + off, bq + off, idesc, 1u);
+      }
+#pragma unroll
+      for (int kk = 0; kk < kTile / 16; ++kk) {
+        const uint32_t off = (kk * 16 * 128) >> 4;
+        mma_bf16_ss(tmem + L::kDRCol, rw + off, bdy + off, idesc, kk > 0 ? 1u : 0u);
+      }
+    }
+    mma_commit(o_full);
+    issued_o = true;
+  }
+  if (ok) ok = mbar_wait(o_full, 0, abort_flag, a.status);
+  ok = __syncthreads_and(ok);
+  if (ok) {
+    tc_fence_after();
+    // thread = row i: the partial dQt0 of (g, i, k)
+    float* prow = a.dqt0_part + (((long)g * a.b2 + r) * a.b1 + k) * D;
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      float t[32];
+      tmem_ld32(tmem + lane_off + c * 32, t);
+      tmem_wait_ld();
+      if (row_ok) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(prow + c * 32 + e) =
+              make_float4(t[e], t[e + 1], t[e + 2], t[e + 3]);
+      }
+    }
+    // thread = key j: dk and dv of token k b2 + j
+    const bool key_ok = tid < a.b2;
+    bf16* dkrow = a.dk + ((long)chunk_row0 + tid) * D;
+    bf16* dvrow = a.dv + ((long)chunk_row0 + tid) * D;
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      float t[32], u[32];
+      tmem_ld32(tmem + lane_off + L::kDKCol + c * 32, t);
+      tmem_ld32(tmem + lane_off + L::kDRCol + c * 32, u);
+      tmem_wait_ld();
+      if (key_ok) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 8) {
+          uint4 pk, pv;
+          pk.x = pack_bf16x2(t[e], t[e + 1]);
+          pk.y = pack_bf16x2(t[e + 2], t[e + 3]);
+          pk.z = pack_bf16x2(t[e + 4], t[e + 5]);
+          pk.w = pack_bf16x2(t[e + 6], t[e + 7]);
+          pv.x = pack_bf16x2(u[e], u[e + 1]);
+          pv.y = pack_bf16x2(u[e + 2], u[e + 3]);
+          pv.z = pack_bf16x2(u[e + 4], u[e + 5]);
+          pv.w = pack_bf16x2(u[e + 6], u[e + 7]);
+          *reinterpret_cast<uint4*>(dkrow + c * 32 + e) = pk;
+          *reinterpret_cast<uint4*>(dvrow + c * 32 + e) = pv;
+        }
+      }
+    }
+  }
+  if (tid == 0 && *abort_flag) {  // drain what this CTA issued (bounded)
+    if (!issued_s) drain_bar(load_full, 0);
+    if (issued_s) drain_bar(s_full, 0);
+    if (issued_o) drain_bar(o_full, 0);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+template <int D>
+cudaError_t launch_rbw(const bf16* qt0_16, const bf16* k, const bf16* v, const bf16* dkt16,
+                       const bf16* dy16, const float* dhs, float* dqt0_part, bf16* dk, bf16* dv,
+                       const Problem& pb, int* status, cudaStream_t stream, int* launches) {
+  using L = RBLayout<D>;
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(rbw_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    L::kBytes);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  const long n_rows = (long)pb.G * pb.b1 * pb.b2;  // tokens, and rows of dKt / dY per head
+  CUtensorMap tq, tk, tv, tdk, tdy;
+  const cuuint64_t str[1] = {(cuuint64_t)D * 2};
+  const cuuint32_t box[2] = {64, kTile};
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)pb.G * pb.b2};
+    if (!tc_make_map(&tq, qt0_16, 2, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)n_rows};
+    if (!tc_make_map(&tk, k, 2, dims, str, box) || !tc_make_map(&tv, v, 2, dims, str, box) ||
+        !tc_make_map(&tdk, dkt16, 2, dims, str, box) || !tc_make_map(&tdy, dy16, 2, dims, str, box))
+      return cudaErrorInvalidValue;
+  }
+  RBArgs a;
+  a.dhs = dhs;
+  a.dqt0_part = dqt0_part;
+  a.dk = dk;
+  a.dv = dv;
+  a.b1 = pb.b1;
+  a.b2 = pb.b2;
+  a.sc = pb.sc;
+  a.status = status;
+  return timed_launch("bwd_tc_r_side", stream, launches, [&] {
+    rbw_kernel<D><<<(unsigned)((long)pb.G * pb.b1), 128, L::kBytes, stream>>>(tq, tk, tv, tdk,
+                                                                               tdy, a);
+  });
+}
+
 // bf16 -> fp32 of n elements.
 __global__ void to_f32_kernel(const bf16* __restrict__ a, float* __restrict__ out, long n) {
   for (long x = blockIdx.x * (long)blockDim.x + threadIdx.x; x < n;
@@ -345,7 +718,8 @@ __global__ void to_f32_kernel(const bf16* __restrict__ a, float* __restrict__ ou
 template <int D>
 cudaError_t launch_lbw(const bf16* q, const bf16* dout, const bf16* kt16, const bf16* y16,
                        const float* hs, float* dq1, float* dkt, float* dy, float* dhs,
-                       const Problem& pb, int* status, cudaStream_t stream, int* launches) {
+                       bf16* dkt16, bf16* dy16, const Problem& pb, int* status,
+                       cudaStream_t stream, int* launches) {
   using L = LBLayout<D>;
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
@@ -372,6 +746,8 @@ cudaError_t launch_lbw(const bf16* q, const bf16* dout, const bf16* kt16, const 
   a.dkt = dkt;
   a.dy = dy;
   a.dhs = dhs;
+  a.dkt16 = dkt16;
+  a.dy16 = dy16;
   a.b1 = pb.b1;
   a.b2 = pb.b2;
   a.c1 = pb.c1;
@@ -409,12 +785,28 @@ cudaError_t bwd_tc_recompute(const bf16* q, const bf16* k, const bf16* v, bf16* 
 
 cudaError_t bwd_tc_l_side(const bf16* q, const bf16* dout, const bf16* kt16, const bf16* y16,
                           const float* hs, float* dq1, float* dkt, float* dy, float* dhs,
-                          const Problem& pb, int* status, cudaStream_t stream, int* launches) {
+                          bf16* dkt16, bf16* dy16, const Problem& pb, int* status,
+                          cudaStream_t stream, int* launches) {
   if (!bwd_tc_l_side_supports(pb)) return cudaErrorInvalidValue;
-  return pb.d == 128 ? launch_lbw<128>(q, dout, kt16, y16, hs, dq1, dkt, dy, dhs, pb, status,
-                                       stream, launches)
-                     : launch_lbw<64>(q, dout, kt16, y16, hs, dq1, dkt, dy, dhs, pb, status,
-                                      stream, launches);
+  return pb.d == 128 ? launch_lbw<128>(q, dout, kt16, y16, hs, dq1, dkt, dy, dhs, dkt16, dy16, pb,
+                                       status, stream, launches)
+                     : launch_lbw<64>(q, dout, kt16, y16, hs, dq1, dkt, dy, dhs, dkt16, dy16, pb,
+                                      status, stream, launches);
+}
+
+bool bwd_tc_r_side_supports(const Problem& pb) {
+  return bwd_tc_l_side_supports(pb) && pb.c1 == 1 && pb.c2 == 1 && pb.b2 <= kTile;
+}
+
+cudaError_t bwd_tc_r_side(const bf16* qt0_16, const bf16* k, const bf16* v, const bf16* dkt16,
+                          const bf16* dy16, const float* dhs, float* dqt0_part, bf16* dk,
+                          bf16* dv, const Problem& pb, int* status, cudaStream_t stream,
+                          int* launches) {
+  if (!bwd_tc_r_side_supports(pb)) return cudaErrorInvalidValue;
+  return pb.d == 128 ? launch_rbw<128>(qt0_16, k, v, dkt16, dy16, dhs, dqt0_part, dk, dv, pb,
+                                       status, stream, launches)
+                     : launch_rbw<64>(qt0_16, k, v, dkt16, dy16, dhs, dqt0_part, dk, dv, pb,
+                                      status, stream, launches);
 }
 
 }  // namespace monarch

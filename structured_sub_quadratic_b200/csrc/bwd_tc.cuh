@@ -29,8 +29,23 @@ cudaError_t bwd_tc_recompute(const bf16* q, const bf16* k, const bf16* v, bf16* 
 // with L the final L-update's weights, dS_L = L (dO . Y - delta) and
 // delta = dO . O = sum_{k,q} L (dO . Y).  `status` is the device status word
 // that the bounded waits set on timeout.  Adds its launches to *launches.
+// dkt16 and dy16, when not null, receive bf16 copies of dKt and dY in
+// chunk-major order [G][c1][b1 k][c2 q][b2 i][d], the R side's operands.
 cudaError_t bwd_tc_l_side(const bf16* q, const bf16* dout, const bf16* kt16, const bf16* y16,
                           const float* hs, float* dq1, float* dkt, float* dy, float* dhs,
-                          const Problem& pb, int* status, cudaStream_t stream, int* launches);
+                          bf16* dkt16, bf16* dy16, const Problem& pb, int* status,
+                          cudaStream_t stream, int* launches);
+
+// True when the tensor-core R side also takes the shape: untiled
+// (c1 = c2 = 1) with b2 <= 128 positions.
+bool bwd_tc_r_side_supports(const Problem& pb);
+
+// The R side on the tensor cores: from bf16 Qt0 [G][b2][d], k, v and the L
+// side's bf16 dKt, dY (chunk-major) and fp32 dHs, writes the partial dQt0
+// [G][b2 i][b1 k][d] (fp32) and the final dk, dv (bf16, (G, N, d)).
+cudaError_t bwd_tc_r_side(const bf16* qt0_16, const bf16* k, const bf16* v, const bf16* dkt16,
+                          const bf16* dy16, const float* dhs, float* dqt0_part, bf16* dk,
+                          bf16* dv, const Problem& pb, int* status, cudaStream_t stream,
+                          int* launches);
 
 }  // namespace monarch

@@ -57,8 +57,11 @@ def test_backward_is_deterministic(cuda_lib):
 
 
 TC_L_SIDE = [
-    # B, H, b1, b2, d, c1, c2: bf16 rows of <= 128 keys, groups of <= 128 rows
+    # B, H, b1, b2, d, c1, c2: bf16 rows of <= 128 keys, groups of <= 128 rows;
+    # the untiled ones (c1 = c2 = 1, b2 <= 128) take the tensor-core R side too
     (1, 2, 90, 52, 128, 1, 1),   # the 480p latent's blocks
+    (1, 2, 64, 64, 64, 1, 1),    # the 4K sweep's blocks
+    (1, 1, 20, 128, 64, 1, 1),   # 128 positions per chunk
     (1, 1, 64, 20, 64, 1, 2),    # 128 keys per row, 64-key groups
     (1, 2, 100, 12, 128, 2, 1),  # 50-row groups
     (2, 1, 13, 11, 64, 3, 5),    # tiled, ragged groups
@@ -66,7 +69,7 @@ TC_L_SIDE = [
 
 
 @pytest.mark.parametrize("B,H,b1,b2,d,c1,c2", TC_L_SIDE)
-def test_backward_l_side_on_tensor_cores(cuda_lib, B, H, b1, b2, d, c1, c2):
+def test_backward_on_tensor_cores(cuda_lib, B, H, b1, b2, d, c1, c2):
     q, k, v = iid_qkv(B, H, b1 * b2, d, torch.bfloat16, seed=b1 * 7 + b2)
     dO = iid_qkv(B, H, b1 * b2, d, torch.bfloat16, seed=b1 * 7 + b2 + 1)[0]
     cuda_lib.timing_read()
@@ -78,6 +81,8 @@ def test_backward_l_side_on_tensor_cores(cuda_lib, B, H, b1, b2, d, c1, c2):
         cuda_lib.timing_enable(False)
     cuda_lib.check()
     assert "bwd_tc_l_side" in names and "bwd_l_rows" not in names, names
+    if c1 == 1 and c2 == 1:
+        assert "bwd_tc_r_side" in names and "bwd_r_rows" not in names, names
     ref = monarch_attention_backward(*(x.double().numpy() for x in (q, k, v, dO)), b1, b2, c1, c2)
     for name, g, r in zip(("dq", "dk", "dv"), got, ref):
         g = g.double().cpu().numpy()
