@@ -207,13 +207,18 @@ MONARCH_API int monarch_attn_fwd_padded(int dtype, const void* q, const void* k,
  * dtype: MONARCH_DTYPE_BF16 or MONARCH_DTYPE_F32; all seven pointers are
  * device buffers of that type, (B, H, N, d) contiguous, N = b1*b2,
  * 16-byte aligned; dq, dk, dv must not overlap each other or any input.
- * Arithmetic is fp32 throughout (SIMT kernels); the forward intermediates
- * are recomputed.  The library keeps a cached fp32 workspace per device of
- * G (c1 b2 d + 5 N c1 c2 d + 2 N c1 c2 + N d + 2 N + 2 b1 c1 b2^2) floats
- * (G = B*H; allocated on first use, grown on demand, freed by
- * monarch_attn_release_workspace).  Deterministic (fixed-order reductions,
- * no atomics).  Asynchronous on `stream`.  Errors as for monarch_attn_fwd;
- * T other than 1 returns MONARCH_ERR_UNSUPPORTED. */
+ * The forward intermediates are recomputed.  bf16 calls with d in {64, 128},
+ * b1 c2 <= 128 and row groups of <= 128 rows run the L side on the tensor
+ * cores (bf16 operands, fp32 accumulation), and with c1 = c2 = 1 and
+ * b2 <= 128 the R side too; every other case, and the final sum of dq,
+ * runs in fp32 on SIMT kernels.  The library keeps a cached workspace per
+ * device of about G (1.5 c1 b2 d + 7 N c1 c2 d + 2 N c1 c2 + N d + 2 N +
+ * 2 b1 c1 b2^2) floats (G = B*H; allocated on first use, grown on demand,
+ * freed by monarch_attn_release_workspace).  Deterministic (fixed-order
+ * reductions, no atomics).  Asynchronous on `stream`.  Errors as for
+ * monarch_attn_fwd, plus MONARCH_ERR_DEVICE_TIMEOUT from monarch_attn_check
+ * if a tensor-core kernel's bounded wait expired; T other than 1 returns
+ * MONARCH_ERR_UNSUPPORTED. */
 MONARCH_API int monarch_attn_bwd(int dtype, const void* q, const void* k, const void* v,
                                  const void* dout, void* dq, void* dk, void* dv, int B, int H,
                                  int b1, int b2, int d, int T, int c1, int c2,
