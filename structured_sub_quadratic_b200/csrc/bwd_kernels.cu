@@ -1,8 +1,9 @@
 // Backward pass of the T = 1 forward (MonarchRT summary, "Method" (3):
 // forward and backward kernels for finetuning with one refinement step).
 // SIMT kernels in fp32 arithmetic for fp32 or bf16 inputs; every reduction
-// is a fixed-order loop in one warp (no atomics), so results are
-// deterministic.
+// runs in a fixed order (no atomics), so results are deterministic.  bf16
+// shapes the tensor-core kernels take (bwd_tc.cu) run their recompute, L side
+// and (untiled) R side there; the final dq sum always runs here.
 //
 // Forward quantities are recomputed: Qt0, Kt, Y, Hs by the SIMT forward
 // kernels, the L rows' log-sum-exps and O here.  With G = dO:
@@ -348,10 +349,13 @@ template <typename TIn, int DV>
 __global__ void __launch_bounds__(kThreads)
     q_bwd_kernel(const float* __restrict__ dq1, const float* __restrict__ dqt0_part,
                  TIn* __restrict__ dQ, Problem pb) {
+  // one block per (g, p, i): warp w sums the partials kq = w, w + 8, ...;
+  // the eight warp sums are added in a fixed order, so the result is
+  // deterministic; then the warps share the group's rows l
+  __shared__ float red[kWarps][DV * 32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int d = pb.d, b1 = pb.b1, b2 = pb.b2, c1 = pb.c1, c2 = pb.c2;
-  const long unit = (long)blockIdx.x * kWarps + warp;
-  if (unit >= (long)pb.G * c1 * b2) return;
+  const long unit = blockIdx.x;
   const int i = (int)(unit % b2);
   const int p = (int)((unit / b2) % c1);
   const long g = unit / ((long)b2 * c1);
@@ -359,16 +363,26 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
   for (int u = 0; u < DV; ++u) a[u] = 0.f;
   const float* part = dqt0_part + ((g * c1 + p) * b2 + i) * (long)b1 * c2 * d;
-  for (int kq = 0; kq < b1 * c2; ++kq) {
+  for (int kq = warp; kq < b1 * c2; kq += kWarps) {
 #pragma unroll
     for (int u = 0; u < DV; ++u) {
       const int x = lane + 32 * u;
       if (x < d) a[u] += part[(long)kq * d + x];
     }
   }
+#pragma unroll
+  for (int u = 0; u < DV; ++u) red[warp][lane + 32 * u] = a[u];
+  __syncthreads();
+#pragma unroll
+  for (int u = 0; u < DV; ++u) {
+    float t = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) t += red[w][lane + 32 * u];
+    a[u] = t;
+  }
   const int l0 = group_start(b1, c1, p), l1 = group_start(b1, c1, p + 1);
   const float inv = 1.f / (float)(l1 - l0);
-  for (int l = l0; l < l1; ++l) {
+  for (int l = l0 + warp; l < l1; l += kWarps) {
     const long row = (g * b1 + l) * b2 + i;
 #pragma unroll
     for (int u = 0; u < DV; ++u) {
@@ -448,7 +462,7 @@ cudaError_t run_bwd(const TIn* q, const TIn* k, const TIn* v, const TIn* dout, T
   });
   if (e != cudaSuccess) return e;
   return timed_launch("bwd_q", stream, launches, [&] {
-    q_bwd_kernel<TIn, DV><<<ceil_div((long)G * c1 * b2, kWarps), kThreads, 0, stream>>>(
+    q_bwd_kernel<TIn, DV><<<(unsigned)((long)G * c1 * b2), kThreads, 0, stream>>>(
         ws.dq1, ws.dqt0_part, dq, pb);
   });
 }
