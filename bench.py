@@ -112,7 +112,9 @@ def kernel_work(name: str, wl: Workload):
 
 
 def kernel_bound(name: str):
-    return "alu" if name.startswith("simt") else None
+    # SIMT fp32 kernels, and the CUDA-core kernels of groups too small for the
+    # tensor-core tiles (cc_*), against the FP32 lane rate
+    return "alu" if name.startswith(("simt", "cc_")) else None
 
 
 def roofline_for(name, tot_ms, launches, wl, peaks, peak_src, traffic):

@@ -31,7 +31,9 @@
 #include <mutex>
 #include <utility>
 
+#include "launch.cuh"
 #include "simt_kernels.cuh"
+#include "small_dim.cuh"
 #include "tc_ptx.cuh"
 #include "timing.cuh"
 
@@ -2872,37 +2874,6 @@ bool make_kv_map(CUtensorMap* m, const bf16* x, const Problem& pb, int D, int ro
   return make_map(m, x, 3, dims, str, box);
 }
 
-// Launch with programmatic stream serialisation: the kernel may start while
-// the previous kernel of the stream finishes; it calls pdl_wait() before it
-// reads anything that kernel wrote.
-template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                       cudaStream_t stream, Args&&... args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
-}
-
-int num_sms() {
-  static int n = 0;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
-      n = 148;
-  });
-  return n;
-}
-
 template <int D, int NK>
 cudaError_t launch_ko(const bf16* q, const bf16* kt, const bf16* y, const float* hs, bf16* out,
                       const Problem& pb, int* status, cudaStream_t stream, int* launches) {
@@ -3000,12 +2971,14 @@ cudaError_t launch_ko1(const bf16* q, const bf16* kt, const bf16* y, const float
   });
 }
 
-// Output kernel by key count: one key tile per row when b1*c2 <= 64, else
-// the online-softmax kernel over 64-key tiles.
+// Output kernel by key count: one warp per (g, i, p) on the CUDA cores for
+// rows of <= 8 keys, one key tile per row when b1*c2 <= 64, else the
+// online-softmax kernel over 64-key tiles.
 template <int D>
 cudaError_t dispatch_ko(const bf16* q, const bf16* kt, const bf16* y, const float* hs, bf16* out,
                         const Problem& pb, int* status, cudaStream_t stream, int* launches) {
   const int nk = pb.b1 * pb.c2;
+  if (small_out_fits(pb)) return launch_small_out(q, kt, y, hs, out, pb, stream, launches);
   if (nk <= 64) return launch_ko1<D, 64>(q, kt, y, hs, out, pb, status, stream, launches);
   return launch_ko<D, 64>(q, kt, y, hs, out, pb, status, stream, launches);
 }
@@ -3343,6 +3316,7 @@ cudaError_t launch_later_step(const bf16* q, const bf16* k, const bf16* v, bf16*
                       ? launch_kl<D>(q, kt, hs, qt, pb, status, stream, launches)
                       : launch_kl_two_pass<D>(q, kt, hs, lse, qt, pb, status, stream, launches);
   if (e != cudaSuccess) return e;
+  if (small_r_fits(pb)) return launch_small_r(qt, k, v, kt, y, hs, pb, true, last, stream, launches);
   if (kr_group_tile(pb) <= 64 && pb.b2 <= kRows) {
     switch (kr_group_tile(pb)) {
 #define MONARCH_KR2_STEP(NQ)                                                                   \
@@ -3386,15 +3360,25 @@ template <int D>
 cudaError_t launch_r_step1(const bf16* q, const bf16* k, const bf16* v, bf16* qt0, bf16* kt,
                            bf16* y, float* hs, const Problem& pb, int* status,
                            cudaStream_t stream, int* launches) {
-  cudaError_t e = timed_launch("tc_init_qt", stream, launches, [&] {
-    const long units = (long)pb.G * pb.c1 * pb.b2;
-    return units <= 5L * num_sms()
-               ? launch_pdl(init_qt_bf16_kernel<D, 256>, dim3((unsigned)units), dim3(256), 0,
-                            stream, q, qt0, pb)
-               : launch_pdl(init_qt_bf16_kernel<D, 128>, dim3((unsigned)units), dim3(128), 0,
-                            stream, q, qt0, pb);
-  });
+  cudaError_t e =
+      small_init_fits(pb)
+          ? launch_small_init(q, qt0, pb, stream, launches)
+          : timed_launch("tc_init_qt", stream, launches, [&] {
+              // fewer units than SMs (a few long row groups): 32 warps per unit
+              const long units = (long)pb.G * pb.c1 * pb.b2;
+              if (units < num_sms())
+                return launch_pdl(init_qt_bf16_kernel<D, 1024>, dim3((unsigned)units),
+                                  dim3(1024), 0, stream, q, qt0, pb);
+              return units <= 5L * num_sms()
+                         ? launch_pdl(init_qt_bf16_kernel<D, 256>, dim3((unsigned)units),
+                                      dim3(256), 0, stream, q, qt0, pb)
+                         : launch_pdl(init_qt_bf16_kernel<D, 128>, dim3((unsigned)units),
+                                      dim3(128), 0, stream, q, qt0, pb);
+            });
   if (e != cudaSuccess) return e;
+  // column groups of <= 8 keys over <= 32 positions: one warp per group
+  if (small_r_fits(pb))
+    return launch_small_r(qt0, k, v, kt, y, hs, pb, false, pb.T == 1, stream, launches);
   // column groups of <= 64 keys over <= 128 positions: the persistent kernel
   if (kr_group_tile(pb) <= 64 && pb.b2 <= kRows) {
     switch (kr_group_tile(pb)) {

@@ -330,3 +330,33 @@ def test_transposed_layouts_run_in_place(cuda_lib, layout, latent, T, c):
     assert "permute_rows" not in names and not any(n.startswith("simt") for n in names), names
     assert_parity(O.double().cpu().numpy(), layout_oracle(q, k, v, latent, layout, T, c, c), v,
                   torch.bfloat16)
+
+
+# Groups too small for the tensor-core tiles run on the CUDA cores (one warp
+# per group): the step-one aggregation for row groups of <= 16 rows, the
+# R-update for column groups of <= 8 keys over <= 32 positions, the output
+# for rows of <= 8 keys.  Each case names the cc_* kernels it must launch.
+SMALL_GROUPS = [
+    # B, H, b1, b2, d, T, c1, c2, expected CUDA-core kernels
+    (1, 2, 60, 3, 128, 1, 1, 1, {"cc_r_update"}),                # (hw,f)-like: 3-key groups
+    (1, 2, 3, 40, 128, 1, 1, 1, {"cc_init_qt", "cc_l_output"}),  # (f,hw)-like: 3-key rows
+    (2, 1, 4, 6, 64, 1, 2, 2, {"cc_init_qt", "cc_r_update", "cc_l_output"}),  # tiled, 8-key rows
+    (1, 2, 5, 4, 128, 2, 1, 1, {"cc_init_qt", "cc_r_update", "cc_l_output"}),  # two steps
+    (1, 1, 20, 32, 64, 3, 2, 4, {"cc_init_qt", "cc_r_update"}),  # 8-key groups, 32 positions
+    (1, 1, 7, 5, 128, 1, 7, 1, {"cc_init_qt", "cc_r_update", "cc_l_output"}),  # 1-row groups
+]
+
+
+@pytest.mark.parametrize("B,H,b1,b2,d,T,c1,c2,cc", SMALL_GROUPS)
+def test_small_groups_run_on_cuda_cores(cuda_lib, B, H, b1, b2, d, T, c1, c2, cc):
+    q, k, v = iid_qkv(B, H, b1 * b2, d, torch.bfloat16, seed=7 * b1 + b2 + T)
+    cuda_lib.timing_read()
+    cuda_lib.timing_enable(True)
+    try:
+        O = gpu_forward(cuda_lib, q, k, v, b1, b2, T, c1, c2)
+        names = set(cuda_lib.timing_read())
+    finally:
+        cuda_lib.timing_enable(False)
+    assert {n for n in names if n.startswith("cc_")} == cc, names
+    assert not any(n.startswith("simt") for n in names), names
+    assert_parity(O, oracle_forward(q, k, v, b1, b2, T, c1, c2), v, torch.bfloat16)
