@@ -1304,36 +1304,77 @@ __global__ void __launch_bounds__(128)
 }
 
 // ---------------------------------------------------------------------------
-// R-update for column groups of more than 128 keys.  One CTA of four warps
-// per (g, k, p, position tile, group q) streams the group's keys in
-// 128-key sub-tiles with an online softmax (thread = row, log2 units):
-//   S_j = Qt0 K_j^T sc log2(e)       128 x 128 in TMEM, columns [2d, 2d + 128)
-//   m, z, T = sum e (s - m)          running per row; when a sub-tile's max
-//                                    exceeds m by more than 2^8 (lazy), m moves
-//                                    and z, T and the accumulator rows are
-//                                    scaled by 2^(m_old - m_new)
-//   [Kt | Y] += P_j [K_j | V_j]        128 x 2d in TMEM, columns [0, 2d)
-// then [Kt | Y] / z, Hs = ln z - ln 2 T / z, and every warp stores its 32
-// rows through a 4-D box clipped at b2, staged in its rows of P.  Thread 0
-// loads (TMA) and issues the MMAs; one sub-tile at a time.
+// R-update for column groups of more than 128 keys, persistent and
+// warp-specialised.  A work item is (g, k, p, position tile, group q): 128
+// aggregated queries against the group's keys, streamed in 128-key tiles
+// with an online softmax (thread = row, log2 units):
+//   S_j = Qt K_j^T                     128 x 128 in TMEM, two buffers
+//   m, z, T = sum e (s - m)            running per row; when a tile's max
+//                                      exceeds m by more than 2^8 (lazy), m
+//                                      moves and z, T and the accumulator
+//                                      rows are scaled by 2^(m_old - m_new)
+//   P_j = 2^(s sc log2(e) - m)         bf16 pairs written over S_j in TMEM
+//   [Kt | Y] += P_j [K_j | V_j]          128 x 2d in TMEM, A = P_j from TMEM
+// then [Kt | Y] / z and Hs = ln z - ln 2 T / z.  Warp 0 loads the query
+// tile and the K_j | V_j tiles (TMA, a two-slot ring), warp 1 issues the
+// MMAs from one thread (event-driven, as the output kernel), warps 2-5 run
+// the softmax and the epilogue, in which each warp stores its 32 rows
+// through a 4-D box clipped at b2.  S_{j+1} is computed while the softmax
+// works on S_j, and the next item's first tiles while the epilogue stores
+// this one's rows.  Barriers (tile counter T over the CTA's items):
+//   q_full / q_empty         query tile of an item
+//   kv_full / kv_empty [2]   K_j | V_j ring (free once P_j [K_j | V_j] is done)
+//   s_full [2]               S_j in its TMEM buffer
+//   p_full [2]               P_j written over S_j
+//   pv_done [2]              the product of tile j complete (its buffer free)
+//   o_empty                  the epilogue has read the accumulator
 // ---------------------------------------------------------------------------
 template <int D>
 struct KRLLayout {
-  static constexpr int kChunk = kRows * 128;                    // 128 rows x 64 bf16
-  static constexpr int kQOff = 0;                               // D / 64 chunks
-  static constexpr int kKVOff = D / 64 * kChunk;                // K chunks, then V chunks
-  static constexpr int kPOff = kKVOff + 2 * (D / 64) * kChunk;  // 2 chunks: 128 keys
-  static constexpr int kBarOff = kPOff + 2 * kChunk;
-  static constexpr int kBytes = kBarOff + 8 * 8;
+  static constexpr int kChunk = kRows * 128;                  // 128 rows x 64 bf16
+  static constexpr int kQOff = 0;                             // D / 64 chunks
+  static constexpr int kSlotBytes = 2 * (D / 64) * kChunk;    // K chunks, then V chunks
+  static constexpr int kKVOff = D / 64 * kChunk;              // two slots
+  static constexpr int kStageOff = kKVOff + 2 * kSlotBytes;   // two chunks: 64 columns each
+  static constexpr int kBarOff = kStageOff + 2 * kChunk;
+  static constexpr int kBytes = kBarOff + 16 * 8;
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kSCol = 2 * D;
+  static constexpr uint32_t kSCol = 2 * D;  // S buffers at [2d, 2d + 128), [2d + 128, 2d + 256)
+  static_assert(2 * D + 256 <= 512 && kBytes <= 227 * 1024, "TMEM and shared memory");
 };
 
+struct KRLItem {
+  int g, k, p, q, i0, js, nq, n_sub, jlo, jhi;
+};
+
+// Item order: group q fastest, then position tile, row group, chunk, head.
+__device__ __forceinline__ void krl_decode(const KRArgs& a, int item, KRLItem& t) {
+  int bid = item;
+  t.q = bid % a.c2;
+  bid /= a.c2;
+  const int it = bid % a.n_itiles;
+  bid /= a.n_itiles;
+  t.p = bid % a.c1;
+  bid /= a.c1;
+  t.k = bid % a.b1;
+  t.g = bid / a.b1;
+  t.i0 = it * kRows;
+  t.js = group_start(a.b2, a.c2, t.q);
+  t.nq = group_start(a.b2, a.c2, t.q + 1) - t.js;
+  t.n_sub = (t.nq + 127) / 128;
+  real_keys(a.real_lo, a.real_hi, a.b2, t.k, t.js, t.nq, &t.jlo, &t.jhi);
+}
+
+__device__ __forceinline__ int krl_nsub(const KRArgs& a, int item) {
+  const int q = item % a.c2;
+  return (group_start(a.b2, a.c2, q + 1) - group_start(a.b2, a.c2, q) + 127) / 128;
+}
+
 template <int D>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(192, 1)
     krl_kernel(const __grid_constant__ CUtensorMap tm_qt, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kt,
-               const __grid_constant__ CUtensorMap tm_y, KRArgs a) {
+               const __grid_constant__ CUtensorMap tm_y, KRArgs a, int n_items) {
   using L = KRLLayout<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1341,230 +1382,332 @@ __global__ void __launch_bounds__(128)
     if (tid == 0) atomicExch(a.status, 2);
     return;
   }
-  int bid = blockIdx.x;
-  const int q = bid % a.c2;
-  bid /= a.c2;
-  const int it = bid % a.n_itiles;
-  bid /= a.n_itiles;
-  const int p = bid % a.c1;
-  bid /= a.c1;
-  const int k = bid % a.b1;
-  const int g = bid / a.b1;
-  const int i0 = it * kRows;
-  const int js = group_start(a.b2, a.c2, q);
-  const int nq = group_start(a.b2, a.c2, q + 1) - js;
-  const int n_sub = (nq + 127) / 128;
-  int jlo, jhi;  // the group's real keys
-  real_keys(a.real_lo, a.real_hi, a.b2, k, js, nq, &jlo, &jhi);
+  pdl_launch_dependents();
   uint8_t* sQ = smem + L::kQOff;
-  uint8_t* sKV = smem + L::kKVOff;
-  uint8_t* sP = smem + L::kPOff;
+  auto sKV = [&](int sl) { return smem + L::kKVOff + sl * L::kSlotBytes; };
+  uint8_t* sStage = smem + L::kStageOff;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
   uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;
-  uint64_t* s_full = bars + 2;
-  uint64_t* o_full = bars + 3;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 5);
+  uint64_t* q_empty = bars + 1;
+  uint64_t* kv_full = bars + 2;   // [2]
+  uint64_t* kv_empty = bars + 4;  // [2]
+  uint64_t* s_full = bars + 6;    // [2]
+  uint64_t* p_full = bars + 8;    // [2]
+  uint64_t* pv_done = bars + 10;  // [2]
+  uint64_t* o_empty = bars + 12;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 14);
   if (tid == 0) {
     mbar_init(q_full, 1);
-    mbar_init(kv_full, 1);
-    mbar_init(s_full, 1);
-    mbar_init(o_full, 1);
+    mbar_init(q_empty, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(kv_full + s, 1);
+      mbar_init(kv_empty + s, 1);
+      mbar_init(s_full + s, 1);
+      mbar_init(p_full + s, 128);
+      mbar_init(pv_done + s, 1);
+    }
+    mbar_init(o_empty, 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0) {
+  if (warp == 1) {
     tmem_alloc(tmem_slot, L::kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const uint32_t tmem_s = tmem + L::kSCol;
-  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-  pdl_launch_dependents();
-  bool ok = true;
-  int issued_s = 0, issued_o = 0, kv_loads = 0;
-  if (tid == 0) {
-    tma_prefetch_desc(&tm_qt);
-    tma_prefetch_desc(&tm_k);
-    tma_prefetch_desc(&tm_v);
-    pdl_wait();  // the queries come from the previous kernel
-    mbar_arrive_expect_tx(q_full, (D / 64) * L::kChunk);
+  const uint32_t tmem = *tmem_slot;  // accumulator [Kt | Y] in columns [0, 2d)
+  auto tmem_s = [&](int sb) { return tmem + L::kSCol + sb * 128; };
+
+  if (warp == 0) {
+    // ---------------------------- producer ----------------------------
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_qt);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      pdl_wait();  // the queries come from the previous kernel
+      long T = 0, last_kv = -1;
+      int q_loads = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+        KRLItem t;
+        krl_decode(a, item, t);
+        if (q_loads >= 1) ok = mbar_wait(q_empty, (q_loads - 1) & 1, abort_flag, a.status);
+        if (!ok) break;
+        mbar_arrive_expect_tx(q_full, (D / 64) * L::kChunk);
 #pragma unroll
-    for (int c = 0; c < D / 64; ++c)
-      tma_load_2d(sQ + c * L::kChunk, &tm_qt, q_full, c * 64, kr_qrow(a, g, p, k, q) + i0);
-  }
-  const int r = tid;  // tile row = position i0 + r
-  float m = -INFINITY, z = 0.f, t2 = 0.f;
-  for (int j = 0; j < n_sub && ok; ++j) {
-    if (tid == 0) {
-      // K_j, V_j into the (single) buffer: the previous product has read it
-      if (j > 0) ok = mbar_wait(o_full, (j - 1) & 1, abort_flag, a.status);
-      if (ok) {
-        mbar_arrive_expect_tx(kv_full, 2 * (D / 64) * L::kChunk);
-        const int2 kyz = kv_yz(a.tr, g, a.b1, a.b2, k, js + j * 128);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_2d(sQ + c * L::kChunk, &tm_qt, q_full, c * 64,
+                      kr_qrow(a, t.g, t.p, t.k, t.q) + t.i0);
+        ++q_loads;
+        for (int j = 0; j < t.n_sub && ok; ++j, ++T) {
+          const int sl = (int)(T & 1);
+          if (T >= 2) ok = mbar_wait(kv_empty + sl, ((T >> 1) - 1) & 1, abort_flag, a.status);
+          if (!ok) break;
+          mbar_arrive_expect_tx(kv_full + sl, L::kSlotBytes);
+          const int2 kyz = kv_yz(a.tr, t.g, a.b1, a.b2, t.k, t.js + j * 128);
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d(sKV + c * L::kChunk, &tm_k, kv_full, c * 64, kyz.x, kyz.y);
-          tma_load_3d(sKV + (D / 64 + c) * L::kChunk, &tm_v, kv_full, c * 64, kyz.x, kyz.y);
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_3d(sKV(sl) + c * L::kChunk, &tm_k, kv_full + sl, c * 64, kyz.x, kyz.y);
+            tma_load_3d(sKV(sl) + (D / 64 + c) * L::kChunk, &tm_v, kv_full + sl, c * 64, kyz.x,
+                        kyz.y);
+          }
+          last_kv = T;
         }
-        ++kv_loads;
-        ok = mbar_wait(kv_full, j & 1, abort_flag, a.status) &&
-             (j > 0 || mbar_wait(q_full, 0, abort_flag, a.status));
       }
-      if (ok) {
+      if (*abort_flag) {  // drain the loads this thread issued (bounded)
+        if (q_loads >= 1) drain(q_full, (q_loads - 1) & 1);
+        for (long t = (last_kv >= 1 ? last_kv - 1 : 0); t <= last_kv; ++t)
+          drain(kv_full + (t & 1), (t >> 1) & 1);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------- MMA --------------------------------
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_bf16(kRows, 128, false);
+      const uint32_t idesc_o = idesc_bf16(kRows, 2 * D, true);
+      const uint64_t dq = desc_kmajor(smem_u32(sQ));
+      const uint64_t dk0 = desc_kmajor(smem_u32(sKV(0))), dk1 = desc_kmajor(smem_u32(sKV(1)));
+      const uint64_t dkv0 = desc_mnmajor(smem_u32(sKV(0)), L::kChunk),
+                     dkv1 = desc_mnmajor(smem_u32(sKV(1)), L::kChunk);
+      int s_item = blockIdx.x, p_item = blockIdx.x;
+      int s_nsub = s_item < n_items ? krl_nsub(a, s_item) : 0;
+      int p_nsub = s_nsub;
+      int s_j = 0, s_n = 0, p_j = 0, p_n = 0;
+      long Ts = 0, Tp = 0, last_s = -1, last_pv = -1;
+      bool ok = true;
+      unsigned long long idle_since = global_ns();
+      while (p_item < n_items && ok) {
+        bool progressed = false;
+        if (s_item < n_items) {
+          const int st = (int)(Ts & 1);
+          if ((s_j > 0 || mbar_test(q_full, s_n & 1)) && mbar_test(kv_full + st, (Ts >> 1) & 1) &&
+              (Ts < 2 || mbar_test(pv_done + st, ((Ts >> 1) - 1) & 1))) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+              mma_bf16_ss(tmem_s(st), dq + (((kk >> 2) * L::kChunk + (kk & 3) * 32) >> 4),
+                          (st ? dk1 : dk0) + (((kk >> 2) * L::kChunk + (kk & 3) * 32) >> 4),
+                          idesc_s, kk > 0 ? 1u : 0u);
+            mma_commit(s_full + st);
+            last_s = Ts;
+            ++Ts;
+            if (++s_j == s_nsub) {
+              mma_commit(q_empty);  // the item's query tile is no longer needed
+              s_j = 0;
+              ++s_n;
+              s_item += gridDim.x;
+              s_nsub = s_item < n_items ? krl_nsub(a, s_item) : 0;
+            }
+            progressed = true;
+          }
+        }
+        if (Tp < Ts) {
+          const int st = (int)(Tp & 1);
+          if (mbar_test(p_full + st, (Tp >> 1) & 1) &&
+              (p_j > 0 || p_n == 0 || mbar_test(o_empty, (p_n - 1) & 1))) {
+            tc_fence_after();
+            // A = P_j from TMEM (8 columns per 16 keys), B = [K_j | V_j] MN-major
+#pragma unroll
+            for (int kk = 0; kk < 128 / 16; ++kk)
+              mma_bf16_ts(tmem, tmem_s(st) + kk * 8, (st ? dkv1 : dkv0) + ((kk * 16 * 128) >> 4),
+                          idesc_o, (p_j > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(kv_empty + st);
+            mma_commit(pv_done + st);
+            last_pv = Tp;
+            ++Tp;
+            if (++p_j == p_nsub) {
+              p_j = 0;
+              ++p_n;
+              p_item += gridDim.x;
+              p_nsub = p_item < n_items ? krl_nsub(a, p_item) : 0;
+            }
+            progressed = true;
+          }
+        }
+        if (progressed) {
+          idle_since = global_ns();
+        } else if ((__nanosleep(20), *abort_flag)) {
+          ok = false;
+        } else if (global_ns() - idle_since > kWaitLimitNs) {
+          *abort_flag = 1;
+          atomicExch(a.status, 1);
+          ok = false;
+        }
+      }
+      if (*abort_flag) {  // drain this thread's MMAs (bounded)
+        if (last_s >= 0) drain(s_full + (last_s & 1), (last_s >> 1) & 1);
+        if (last_pv >= 0) drain(pv_done + (last_pv & 1), (last_pv >> 1) & 1);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ----------------------- softmax + epilogue ------------------------
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;  // TMEM lane == tile row == position i0 + r
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    long T = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+      KRLItem t;
+      krl_decode(a, item, t);
+      float m = -INFINITY, z = 0.f, t2 = 0.f;
+      for (int j = 0; j < t.n_sub; ++j, ++T) {
+        const int sb = (int)(T & 1);
+        ok = mbar_wait(s_full + sb, (T >> 1) & 1, abort_flag, a.status);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
         tc_fence_after();
-        const uint64_t dq = desc_kmajor(smem_u32(sQ)), dk = desc_kmajor(smem_u32(sKV));
-        const uint32_t idesc = idesc_bf16(kRows, 128, false);
+        float sv[128];
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_bf16_ss(tmem_s, dq + (((kk >> 2) * L::kChunk + (kk & 3) * 32) >> 4),
-                      dk + (((kk >> 2) * L::kChunk + (kk & 3) * 32) >> 4), idesc,
-                      kk > 0 ? 1u : 0u);
-        mma_commit(s_full);
-        ++issued_s;
-      }
-    }
-    // S_j complete implies the previous [Kt | Y] product complete (in order)
-    ok = mbar_wait(s_full, j & 1, abort_flag, a.status);
-    ok = __syncthreads_and(ok);
-    if (!ok) break;
-    tc_fence_after();
-    float sv[128];
+        for (int c = 0; c < 4; ++c) {
+          float tt[32];
+          tmem_ld32(tmem_s(sb) + lane_off + c * 32, tt);
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      float t[32];
-      tmem_ld32(tmem_s + lane_off + c * 32, t);
-#pragma unroll
-      for (int e = 0; e < 32; ++e) sv[c * 32 + e] = t[e];
-    }
-    tmem_wait_ld();
-    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-    for (int c = 0; c < 128; ++c) {
-      const int jj = j * 128 + c;
-      sv[c] = (jj >= jlo && jj < jhi) ? sv[c] * a.sc_log2 : -INFINITY;
-      mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
-    }
-    const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-    float alpha = 1.f;
-    bool resc = false;
-    if (mt > m + 8.f) {  // first real keys, or the max grew by more than 2^8
-      alpha = m > -INFINITY ? ex2(m - mt) : 0.f;
-      t2 = m > -INFINITY ? alpha * (t2 + z * (m - mt)) : 0.f;
-      z *= alpha;
-      resc = j > 0;
-      m = mt;
-    }
-    if (__any_sync(0xffffffffu, resc)) {  // scale this warp's accumulator rows
-#pragma unroll 1
-      for (int c = 0; c < 2 * D / 32; ++c) {
-        float t[32];
-        tmem_ld32(tmem + lane_off + c * 32, t);
+          for (int e = 0; e < 32; ++e) sv[c * 32 + e] = tt[e];
+        }
         tmem_wait_ld();
+        // logits in log2 units over the group's real keys; 4 partial maxima
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        const bool full = t.jlo <= j * 128 && (j + 1) * 128 <= t.jhi;  // warp-uniform
+        if (full) {
+          const float2 s2 = make_float2(a.sc_log2, a.sc_log2);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) t[e] *= alpha;
-        tmem_st32(tmem + lane_off + c * 32, t);
+          for (int c = 0; c < 128; c += 4) {
+            const float2 lo = mul2(make_float2(sv[c], sv[c + 1]), s2);
+            const float2 hi = mul2(make_float2(sv[c + 2], sv[c + 3]), s2);
+            sv[c] = lo.x;
+            sv[c + 1] = lo.y;
+            sv[c + 2] = hi.x;
+            sv[c + 3] = hi.y;
+            const int mm = (c >> 2) & 1;
+            mx[mm] = max3(mx[mm], lo.x, lo.y);
+            mx[2 + mm] = max3(mx[2 + mm], hi.x, hi.y);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 128; ++c) {
+            const int jj = j * 128 + c;
+            sv[c] = (jj >= t.jlo && jj < t.jhi) ? sv[c] * a.sc_log2 : -INFINITY;
+            mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
+          }
+        }
+        const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        float alpha = 1.f;
+        bool resc = false;
+        if (mt > m + 8.f) {  // first real keys, or the max grew by more than 2^8
+          alpha = m > -INFINITY ? ex2(m - mt) : 0.f;
+          t2 = m > -INFINITY ? alpha * (t2 + z * (m - mt)) : 0.f;
+          z *= alpha;
+          resc = j > 0;
+          m = mt;
+        }
+        if (__any_sync(0xffffffffu, resc)) {
+          // the accumulator is stable once the previous tile's product is done
+          ok = mbar_wait(pv_done + ((T - 1) & 1), ((T - 1) >> 1) & 1, abort_flag, a.status);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < 2 * D / 32; ++c) {
+            float tt[32];
+            tmem_ld32(tmem + lane_off + c * 32, tt);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) tt[e] *= alpha;
+            tmem_st32(tmem + lane_off + c * 32, tt);
+          }
+          tmem_wait_st();
+        }
+        const float base = m > -INFINITY ? m : 0.f;
+        float zs[4] = {0.f, 0.f, 0.f, 0.f}, ts[4] = {0.f, 0.f, 0.f, 0.f};
+        // exponentials 32 keys at a time, each group's P (bf16 pairs) stored
+        // at once over the first 64 columns of this tile's S buffer
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float d2 = sv[c * 32 + e] - base;  // -inf outside the real keys
+            const float w = ex2(d2);
+            zs[e & 3] += w;
+            ts[e & 3] += full ? w * d2 : (w > 0.f ? w * d2 : 0.f);
+            if (e & 1)
+              pk[e >> 1] = pack_bf16x2(sv[c * 32 + e - 1], w);
+            else
+              sv[c * 32 + e] = w;
+          }
+          tmem_st16(tmem_s(sb) + lane_off + c * 16, pk);
+        }
+        z += (zs[0] + zs[1]) + (zs[2] + zs[3]);
+        t2 += (ts[0] + ts[1]) + (ts[2] + ts[3]);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(p_full + sb);
       }
-      tmem_wait_st();
-    }
-    const float base = m > -INFINITY ? m : 0.f;
-    float zs[4] = {0.f, 0.f, 0.f, 0.f}, ts[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int u = 0; u < 16; ++u) {  // 16-byte unit u holds keys 8u .. 8u + 7
-      float w[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float d2 = sv[8 * u + e] - base;  // -inf outside the real keys
-        w[e] = ex2(d2);
-        zs[e & 3] += w[e];
-        ts[e & 3] += w[e] > 0.f ? w[e] * d2 : 0.f;
-      }
-      uint4 pk;
-      pk.x = pack_bf16x2(w[0], w[1]);
-      pk.y = pack_bf16x2(w[2], w[3]);
-      pk.z = pack_bf16x2(w[4], w[5]);
-      pk.w = pack_bf16x2(w[6], w[7]);
-      *reinterpret_cast<uint4*>(sP + (u >> 3) * L::kChunk + r * 128 + (((u & 7) ^ (r & 7)) << 4)) =
-          pk;
-    }
-    z += (zs[0] + zs[1]) + (zs[2] + zs[3]);
-    t2 += (ts[0] + ts[1]) + (ts[2] + ts[3]);
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
+      if (!ok) break;
+      // ---- epilogue: [Kt | Y] / z, per-warp stores of this warp's 32 rows ----
+      ok = mbar_wait(pv_done + ((T - 1) & 1), ((T - 1) >> 1) & 1, abort_flag, a.status);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
       tc_fence_after();
-      const uint64_t dp = desc_kmajor(smem_u32(sP));
-      const uint64_t dkv = desc_mnmajor(smem_u32(sKV), L::kChunk);
-      const uint32_t idesc = idesc_bf16(kRows, 2 * D, true);
-#pragma unroll
-      for (int kk = 0; kk < 128 / 16; ++kk)
-        mma_bf16_ss(tmem, dp + (((kk >> 2) * L::kChunk + (kk & 3) * 32) >> 4),
-                    dkv + ((kk * 16 * 128) >> 4), idesc, (j > 0 || kk > 0) ? 1u : 0u);
-      mma_commit(o_full);
-      ++issued_o;
-    }
-  }
-  // ---- epilogue: [Kt | Y] / z, per-warp stores of this warp's 32 rows ----
-  if (ok) ok = mbar_wait(o_full, (n_sub - 1) & 1, abort_flag, a.status);
-  ok = __syncthreads_and(ok);
-  if (ok) {
-    tc_fence_after();
-    const float inv = z > 0.f ? 1.f / z : 0.f;
-    const int nblk = (a.write_y ? 2 : 1) * (D / 64);
-    const int ycoord = (p * a.b1 + k) * a.c2 + q;
-    const int iw = i0 + warp * 32;  // this warp's first position
-    if (iw < a.b2) {
+      const float inv = z > 0.f ? 1.f / z : 0.f;
+      const int nblk = (a.write_y ? 2 : 1) * (D / 64);
+      const int ycoord = (t.p * a.b1 + t.k) * a.c2 + t.q;
+      const int iw = t.i0 + quad * 32;  // this warp's first position
+      const bool store = iw < a.b2;     // warp-uniform
+      if (lane == 0) bulk_wait_read<0>();  // the previous item's stores have read the staging
+      __syncwarp();
 #pragma unroll 1
       for (int cb = 0; cb < nblk; ++cb) {
-        uint8_t* buf = sP + (cb & 1) * L::kChunk + warp * 32 * 128;
-        if (cb >= 2) {
+        uint8_t* buf = sStage + (cb & 1) * L::kChunk + quad * 32 * 128;
+        if (cb >= 2 && store) {
           if (lane == 0) bulk_wait_read<1>();  // the store of block cb - 2 has read buf
           __syncwarp();
         }
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
-          float t[32];
-          tmem_ld32(tmem + lane_off + cb * 64 + hf * 32, t);
+          float tt[32];
+          tmem_ld32(tmem + lane_off + cb * 64 + hf * 32, tt);
           tmem_wait_ld();
+          if (store) {
 #pragma unroll
-          for (int uu = 0; uu < 4; ++uu) {
-            uint4 pk;
-            pk.x = pack_bf16x2(t[8 * uu + 0] * inv, t[8 * uu + 1] * inv);
-            pk.y = pack_bf16x2(t[8 * uu + 2] * inv, t[8 * uu + 3] * inv);
-            pk.z = pack_bf16x2(t[8 * uu + 4] * inv, t[8 * uu + 5] * inv);
-            pk.w = pack_bf16x2(t[8 * uu + 6] * inv, t[8 * uu + 7] * inv);
-            const int chunk = hf * 4 + uu;
-            *reinterpret_cast<uint4*>(buf + lane * 128 + ((chunk ^ (lane & 7)) << 4)) = pk;
+            for (int uu = 0; uu < 4; ++uu) {
+              uint4 pk;
+              pk.x = pack_bf16x2(tt[8 * uu + 0] * inv, tt[8 * uu + 1] * inv);
+              pk.y = pack_bf16x2(tt[8 * uu + 2] * inv, tt[8 * uu + 3] * inv);
+              pk.z = pack_bf16x2(tt[8 * uu + 4] * inv, tt[8 * uu + 5] * inv);
+              pk.w = pack_bf16x2(tt[8 * uu + 6] * inv, tt[8 * uu + 7] * inv);
+              const int chunk = hf * 4 + uu;
+              *reinterpret_cast<uint4*>(buf + lane * 128 + ((chunk ^ (lane & 7)) << 4)) = pk;
+            }
           }
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_4d(cb < D / 64 ? &tm_kt : &tm_y, buf, (cb % (D / 64)) * 64, ycoord, iw, g);
-          bulk_commit();
+        if (store) {
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_4d(cb < D / 64 ? &tm_kt : &tm_y, buf, (cb % (D / 64)) * 64, ycoord, iw, t.g);
+            bulk_commit();
+          }
         }
       }
+      // the accumulator is read out: the next item's first product may overwrite it
+      tc_fence_before();
+      mbar_arrive(o_empty);
+      if (t.i0 + r < a.b2) {
+        const long orow = ((((long)t.g * a.b2 + t.i0 + r) * a.c1 + t.p) * a.b1 + t.k) * a.c2 + t.q;
+        a.hs[orow] = z > 0.f ? logf(z) - t2 * 0.69314718055994531f / z : -INFINITY;
+      }
     }
-    if (i0 + r < a.b2) {
-      const long orow = ((((long)g * a.b2 + i0 + r) * a.c1 + p) * a.b1 + k) * a.c2 + q;
-      a.hs[orow] = z > 0.f ? logf(z) - t2 * 0.69314718055994531f / z : -INFINITY;
-    }
+    if (lane == 0) bulk_wait<0>();  // stores done reading shared memory before exit
   }
-  if (tid == 0 && *abort_flag) {  // drain what this CTA issued (bounded)
-    drain(q_full, 0);
-    if (kv_loads > 0) drain(kv_full, (kv_loads - 1) & 1);
-    if (issued_s > 0) drain(s_full, (issued_s - 1) & 1);
-    if (issued_o > 0) drain(o_full, (issued_o - 1) & 1);
-  }
-  if (lane == 0) bulk_wait<0>();  // stores done reading shared memory before exit
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, L::kTmemCols);
   }
@@ -3167,11 +3310,12 @@ cudaError_t launch_krl(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, 
   a.real_lo = pb.real_lo;
   a.real_hi = pb.real_hi;
   a.n_itiles = (pb.b2 + kRows - 1) / kRows;
-  const long blocks = (long)pb.G * pb.b1 * pb.c1 * a.n_itiles * pb.c2;
-  if (blocks >= (1L << 31)) return cudaErrorInvalidValue;
+  const long items = (long)pb.G * pb.b1 * pb.c1 * a.n_itiles * pb.c2;
+  if (items >= (1L << 31)) return cudaErrorInvalidValue;
+  const int grid = (int)std::min<long>(items, num_sms());  // persistent: one CTA per SM
   return timed_launch("tc_r_update", stream, launches, [&] {
-    return launch_pdl(krl_kernel<D>, dim3((unsigned)blocks), dim3(128), L::kBytes, stream, tq, tk,
-                      tv, tkt, tyy, a);
+    return launch_pdl(krl_kernel<D>, dim3(grid), dim3(192), L::kBytes, stream, tq, tk, tv, tkt,
+                      tyy, a, (int)items);
   });
 }
 
