@@ -1317,17 +1317,24 @@ __global__ void __launch_bounds__(128)
 //   [Kt | Y] += P_j [K_j | V_j]          128 x 2d in TMEM, A = P_j from TMEM
 // then [Kt | Y] / z and Hs = ln z - ln 2 T / z.  Warp 0 loads the query
 // tile and the K_j | V_j tiles (TMA, a two-slot ring), warp 1 issues the
-// MMAs from one thread (event-driven, as the output kernel), warps 2-5 run
-// the softmax and the epilogue, in which each warp stores its 32 rows
-// through a 4-D box clipped at b2.  S_{j+1} is computed while the softmax
-// works on S_j, and the next item's first tiles while the epilogue stores
-// this one's rows.  Barriers (tile counter T over the CTA's items):
+// MMAs from one thread (event-driven, as the output kernel), and warps 2-9
+// run the softmax and the epilogue, two warps per row: warps 2-5 take keys
+// 0-63 of every tile, warps 6-9 keys 64-127.  The two halves exchange each
+// tile's row maxima through shared memory, so both hold the same running
+// maximum and take the same rescaling decisions; each keeps its own z and T
+// (added once per item) and rescales its half of the accumulator columns.
+// In the epilogue each warp stores its 32 rows of every other 64-column
+// block through a 4-D box clipped at b2.  S_{j+1} is computed while the
+// softmax works on S_j, and the next item's first tiles while the epilogue
+// stores this one's rows.  Barriers (tile counter T over the CTA's items):
 //   q_full / q_empty         query tile of an item
 //   kv_full / kv_empty [2]   K_j | V_j ring (free once P_j [K_j | V_j] is done)
 //   s_full [2]               S_j in its TMEM buffer
 //   p_full [2]               P_j written over S_j
 //   pv_done [2]              the product of tile j complete (its buffer free)
 //   o_empty                  the epilogue has read the accumulator
+//   xchg [2]                 both halves' tile maxima are in shared memory
+//   zx                       both halves' z (and T) of an item are in shared memory
 // ---------------------------------------------------------------------------
 template <int D>
 struct KRLLayout {
@@ -1336,8 +1343,10 @@ struct KRLLayout {
   static constexpr int kSlotBytes = 2 * (D / 64) * kChunk;    // K chunks, then V chunks
   static constexpr int kKVOff = D / 64 * kChunk;              // two slots
   static constexpr int kStageOff = kKVOff + 2 * kSlotBytes;   // two chunks: 64 columns each
-  static constexpr int kBarOff = kStageOff + 2 * kChunk;
-  static constexpr int kBytes = kBarOff + 16 * 8;
+  static constexpr int kXchgOff = kStageOff + 2 * kChunk;     // float [2][2][kRows] maxima
+  static constexpr int kZOff = kXchgOff + 4 * kRows * 4;      // float [2][3][kRows]: z, z, T
+  static constexpr int kBarOff = kZOff + 6 * kRows * 4;
+  static constexpr int kBytes = kBarOff + 20 * 8;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kSCol = 2 * D;  // S buffers at [2d, 2d + 128), [2d + 128, 2d + 256)
   static_assert(2 * D + 256 <= 512 && kBytes <= 227 * 1024, "TMEM and shared memory");
@@ -1371,7 +1380,7 @@ __device__ __forceinline__ int krl_nsub(const KRArgs& a, int item) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     krl_kernel(const __grid_constant__ CUtensorMap tm_qt, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kt,
                const __grid_constant__ CUtensorMap tm_y, KRArgs a, int n_items) {
@@ -1386,6 +1395,8 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* sQ = smem + L::kQOff;
   auto sKV = [&](int sl) { return smem + L::kKVOff + sl * L::kSlotBytes; };
   uint8_t* sStage = smem + L::kStageOff;
+  float* sXchg = reinterpret_cast<float*>(smem + L::kXchgOff);
+  float* sZ = reinterpret_cast<float*>(smem + L::kZOff);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
@@ -1397,6 +1408,8 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* o_empty = bars + 12;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 14);
+  uint64_t* xchg = bars + 15;     // [2]
+  uint64_t* zx = bars + 17;
   if (tid == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
@@ -1404,10 +1417,12 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(kv_full + s, 1);
       mbar_init(kv_empty + s, 1);
       mbar_init(s_full + s, 1);
-      mbar_init(p_full + s, 128);
+      mbar_init(p_full + s, 256);
       mbar_init(pv_done + s, 1);
+      mbar_init(xchg + s, 256);
     }
-    mbar_init(o_empty, 128);
+    mbar_init(o_empty, 256);
+    mbar_init(zx, 256);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -1545,38 +1560,41 @@ __global__ void __launch_bounds__(192, 1)
     }
     __syncwarp();
   } else {
-    // ----------------------- softmax + epilogue ------------------------
+    // -------------- softmax (two warps per row) + epilogue --------------
+    const int half = (warp - 2) >> 2;  // 0: keys 0-63 of a tile (warps 2-5), 1: keys 64-127
     const int quad = warp & 3;
     const int r = quad * 32 + lane;  // TMEM lane == tile row == position i0 + r
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     long T = 0;
+    int n_done = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
       KRLItem t;
       krl_decode(a, item, t);
-      float m = -INFINITY, z = 0.f, t2 = 0.f;
+      float m = -INFINITY, z = 0.f, t2 = 0.f;  // m shared by both halves; z, t2 this half's
       for (int j = 0; j < t.n_sub; ++j, ++T) {
         const int sb = (int)(T & 1);
         ok = mbar_wait(s_full + sb, (T >> 1) & 1, abort_flag, a.status);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
-        float sv[128];
+        const int k0 = j * 128 + half * 64;  // this half's first key of the group
+        float sv[64];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           float tt[32];
-          tmem_ld32(tmem_s(sb) + lane_off + c * 32, tt);
+          tmem_ld32(tmem_s(sb) + lane_off + half * 64 + c * 32, tt);
 #pragma unroll
           for (int e = 0; e < 32; ++e) sv[c * 32 + e] = tt[e];
         }
         tmem_wait_ld();
         // logits in log2 units over the group's real keys; 4 partial maxima
         float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        const bool full = t.jlo <= j * 128 && (j + 1) * 128 <= t.jhi;  // warp-uniform
+        const bool full = t.jlo <= k0 && k0 + 64 <= t.jhi;  // warp-uniform
         if (full) {
           const float2 s2 = make_float2(a.sc_log2, a.sc_log2);
 #pragma unroll
-          for (int c = 0; c < 128; c += 4) {
+          for (int c = 0; c < 64; c += 4) {
             const float2 lo = mul2(make_float2(sv[c], sv[c + 1]), s2);
             const float2 hi = mul2(make_float2(sv[c + 2], sv[c + 3]), s2);
             sv[c] = lo.x;
@@ -1589,13 +1607,25 @@ __global__ void __launch_bounds__(192, 1)
           }
         } else {
 #pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            const int jj = j * 128 + c;
+          for (int c = 0; c < 64; ++c) {
+            const int jj = k0 + c;
             sv[c] = (jj >= t.jlo && jj < t.jhi) ? sv[c] * a.sc_log2 : -INFINITY;
             mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
           }
         }
-        const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        // the tile maximum of the row: this half's, then the other half's
+        // (buffer sb is written again two tiles on, after the other half
+        // has passed the next exchange)
+        const float mh = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        float* xb = sXchg + sb * 2 * kRows;
+        xb[half * kRows + r] = mh;
+        tc_fence_before();  // this half's S loads are done before the other half writes P
+        mbar_arrive(xchg + sb);
+        ok = mbar_wait(xchg + sb, (T >> 1) & 1, abort_flag, a.status);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        const float mt = fmaxf(mh, xb[(1 - half) * kRows + r]);
         float alpha = 1.f;
         bool resc = false;
         if (mt > m + 8.f) {  // first real keys, or the max grew by more than 2^8
@@ -1606,13 +1636,14 @@ __global__ void __launch_bounds__(192, 1)
           m = mt;
         }
         if (__any_sync(0xffffffffu, resc)) {
-          // the accumulator is stable once the previous tile's product is done
+          // the accumulator is stable once the previous tile's product is
+          // done; each half scales its d columns of [Kt | Y]
           ok = mbar_wait(pv_done + ((T - 1) & 1), ((T - 1) >> 1) & 1, abort_flag, a.status);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll 1
-          for (int c = 0; c < 2 * D / 32; ++c) {
+          for (int c = half * (D / 32); c < (half + 1) * (D / 32); ++c) {
             float tt[32];
             tmem_ld32(tmem + lane_off + c * 32, tt);
             tmem_wait_ld();
@@ -1625,9 +1656,9 @@ __global__ void __launch_bounds__(192, 1)
         const float base = m > -INFINITY ? m : 0.f;
         float zs[4] = {0.f, 0.f, 0.f, 0.f}, ts[4] = {0.f, 0.f, 0.f, 0.f};
         // exponentials 32 keys at a time, each group's P (bf16 pairs) stored
-        // at once over the first 64 columns of this tile's S buffer
+        // at once: this half's 32 columns of the first 64 of the S buffer
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
@@ -1640,7 +1671,7 @@ __global__ void __launch_bounds__(192, 1)
             else
               sv[c * 32 + e] = w;
           }
-          tmem_st16(tmem_s(sb) + lane_off + c * 16, pk);
+          tmem_st16(tmem_s(sb) + lane_off + half * 32 + c * 16, pk);
         }
         z += (zs[0] + zs[1]) + (zs[2] + zs[3]);
         t2 += (ts[0] + ts[1]) + (ts[2] + ts[3]);
@@ -1649,23 +1680,30 @@ __global__ void __launch_bounds__(192, 1)
         mbar_arrive(p_full + sb);
       }
       if (!ok) break;
-      // ---- epilogue: [Kt | Y] / z, per-warp stores of this warp's 32 rows ----
-      ok = mbar_wait(pv_done + ((T - 1) & 1), ((T - 1) >> 1) & 1, abort_flag, a.status);
+      // ---- epilogue: [Kt | Y] / z; this warp stores its 32 rows of the
+      // 64-column blocks cb = half, half + 2, ... ----
+      // both halves' z and the second half's T through shared memory (a
+      // buffer per item parity, written again after the next exchange)
+      float* zb = sZ + (n_done & 1) * 3 * kRows;
+      zb[half * kRows + r] = z;
+      if (half == 1) zb[2 * kRows + r] = t2;
+      mbar_arrive(zx);
+      ok = mbar_wait(zx, n_done & 1, abort_flag, a.status);
+      if (ok) ok = mbar_wait(pv_done + ((T - 1) & 1), ((T - 1) >> 1) & 1, abort_flag, a.status);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const float inv = z > 0.f ? 1.f / z : 0.f;
+      const float zt = zb[r] + zb[kRows + r];  // the same sum in both halves
+      const float inv = zt > 0.f ? 1.f / zt : 0.f;
       const int nblk = (a.write_y ? 2 : 1) * (D / 64);
       const int ycoord = (t.p * a.b1 + t.k) * a.c2 + t.q;
       const int iw = t.i0 + quad * 32;  // this warp's first position
       const bool store = iw < a.b2;     // warp-uniform
-      if (lane == 0) bulk_wait_read<0>();  // the previous item's stores have read the staging
-      __syncwarp();
+      uint8_t* buf = sStage + half * L::kChunk + quad * 32 * 128;
 #pragma unroll 1
-      for (int cb = 0; cb < nblk; ++cb) {
-        uint8_t* buf = sStage + (cb & 1) * L::kChunk + quad * 32 * 128;
-        if (cb >= 2 && store) {
-          if (lane == 0) bulk_wait_read<1>();  // the store of block cb - 2 has read buf
+      for (int cb = half; cb < nblk; cb += 2) {
+        if (store) {  // the previous store from buf has read it
+          if (lane == 0) bulk_wait_read<0>();
           __syncwarp();
         }
 #pragma unroll
@@ -1698,10 +1736,12 @@ __global__ void __launch_bounds__(192, 1)
       // the accumulator is read out: the next item's first product may overwrite it
       tc_fence_before();
       mbar_arrive(o_empty);
-      if (t.i0 + r < a.b2) {
+      if (half == 0 && t.i0 + r < a.b2) {
+        const float tt2 = t2 + zb[2 * kRows + r];
         const long orow = ((((long)t.g * a.b2 + t.i0 + r) * a.c1 + t.p) * a.b1 + t.k) * a.c2 + t.q;
-        a.hs[orow] = z > 0.f ? logf(z) - t2 * 0.69314718055994531f / z : -INFINITY;
+        a.hs[orow] = zt > 0.f ? logf(zt) - tt2 * 0.69314718055994531f / zt : -INFINITY;
       }
+      ++n_done;
     }
     if (lane == 0) bulk_wait<0>();  // stores done reading shared memory before exit
   }
@@ -3314,7 +3354,7 @@ cudaError_t launch_krl(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, 
   if (items >= (1L << 31)) return cudaErrorInvalidValue;
   const int grid = (int)std::min<long>(items, num_sms());  // persistent: one CTA per SM
   return timed_launch("tc_r_update", stream, launches, [&] {
-    return launch_pdl(krl_kernel<D>, dim3(grid), dim3(192), L::kBytes, stream, tq, tk, tv, tkt,
+    return launch_pdl(krl_kernel<D>, dim3(grid), dim3(320), L::kBytes, stream, tq, tk, tv, tkt,
                       tyy, a, (int)items);
   });
 }
