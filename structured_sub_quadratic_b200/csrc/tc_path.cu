@@ -20,10 +20,10 @@
 // 2^8 (exact result, fewer rescales of the TMEM accumulator).
 //
 // Step one (aggregated queries under the uniform L, R-update) also runs on
-// the tensor cores, and so do later steps of T >= 2 (non-final L-update with
-// the aggregation L^T Q, R-update from per-sub-item queries) when the
-// R-update's column groups hold <= 64 keys and <= 128 positions; other
-// shapes run their later steps on the SIMT kernels.
+// the tensor cores, and so do the later steps of T >= 2 (non-final L-update
+// with the aggregation L^T Q, R-update from per-sub-item queries).  Groups
+// too small for a 128-row tile (a few keys or rows) take the CUDA-core
+// kernels of small_dim.cu instead.
 #include "tc_path.cuh"
 
 #include <cudaTypedefs.h>
@@ -952,16 +952,13 @@ __global__ void __launch_bounds__(NT)
 }
 
 // ---------------------------------------------------------------------------
-// R-update of step one on the tensor cores.  One CTA per (g, k, p, position
-// tile): 128 of the b2 aggregated queries Qt0_{p,i} (rows; b2 > 128 takes
-// several tiles) against the keys of chunk k, one column group q at a time:
-//   S_q = Qt0 K_q^T / sqrt(d)            128 x NQ in TMEM (K_q: keys j in q)
+// Arguments of the streaming R-update (krl_kernel, below): for every
+// sub-item (g, p, k, q) and tile of 128 positions,
+//   S_q = Qt K_q^T / sqrt(d)            K_q: the keys j of column group q of chunk k
 //   R = softmax_j(S_q), Hs = entropy      one TMEM lane (row) per thread
-//   [Kt | Y] = R [K_q | V_q]               one N = 2d MMA chain
-// K_q and V_q of every group are separate TMA boxes (any start row), laid
-// side by side so that [K_q | V_q] is one MN-major operand; K_q alone is the
-// K-major operand of S_q.  The output accumulator reuses the TMEM columns of
-// S_q (S_q is in registers by then), so a CTA holds 2d columns.
+//   [Kt | Y] = R [K_q | V_q]
+// with Qt the step-one aggregated queries Qt0 (shared by the chunks of a row
+// group) or a later step's per-sub-item rows.
 // ---------------------------------------------------------------------------
 struct KRArgs {
   bf16* kt;   // [G][b2][c1][b1][c2][d]
@@ -1060,247 +1057,6 @@ __device__ __forceinline__ void r_row_softmax(float (&sv)[NQ], float sc_log2, in
   }
   z = (zs[0] + zs[1]) + (zs[2] + zs[3]);
   t2 = (ts[0] + ts[1]) + (ts[2] + ts[3]);
-}
-
-template <int D, int NQ>
-struct KRLayout {
-  static constexpr int kBox = NQ * 128;                    // one 64-column box of NQ rows
-  static constexpr int kGroupBytes = 2 * (D / 64) * kBox;  // K_q then V_q
-  static constexpr int kQOff = 0;
-  static constexpr int kKVOff = D / 64 * kRows * 128;
-  static constexpr int kPBytes = (NQ + 63) / 64 * kRows * 128;
-  static constexpr int kStageBytes = kRows * 128;  // one 64-column staging block
-  __host__ __device__ static constexpr int p_off(int c2) { return kKVOff + c2 * kGroupBytes; }
-  __host__ __device__ static constexpr int stage_off(int c2) { return p_off(c2) + kPBytes; }
-  __host__ __device__ static constexpr int bar_off(int c2) { return stage_off(c2) + kStageBytes; }
-  __host__ __device__ static constexpr int bytes(int c2) { return bar_off(c2) + 64; }
-  static constexpr uint32_t kTmemCols = 2 * D;  // O (2d columns); S_q uses the first NQ
-  static_assert(NQ % 16 == 0 && NQ <= 128 && NQ <= 2 * D, "group tile");
-};
-
-template <int D, int NQ>
-__global__ void __launch_bounds__(128)
-    kr_kernel(const __grid_constant__ CUtensorMap tm_qt, const __grid_constant__ CUtensorMap tm_k,
-              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kt,
-              const __grid_constant__ CUtensorMap tm_y, KRArgs a) {
-  using L = KRLayout<D, NQ>;
-  extern __shared__ __align__(1024) uint8_t smem[];
-  const int tid = threadIdx.x, warp = tid >> 5;
-  if (smem_u32(smem) & 1023u) {
-    if (tid == 0) atomicExch(a.status, 2);
-    return;
-  }
-  int bid = blockIdx.x;
-  const int it = bid % a.n_itiles;  // positions i0 .. i0 + 127 of the sub-item
-  bid /= a.n_itiles;
-  const int p = bid % a.c1;
-  bid /= a.c1;
-  const int k = bid % a.b1;
-  const int g = bid / a.b1;
-  const int i0 = it * kRows;
-
-  uint8_t* sQ = smem + L::kQOff;
-  auto sK = [&](int q) { return smem + L::kKVOff + q * L::kGroupBytes; };
-  uint8_t* sP = smem + L::p_off(a.c2);
-  uint8_t* sStage[2] = {sP, smem + L::stage_off(a.c2)};  // P is free once [Kt | Y] is done
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::bar_off(a.c2));
-  uint64_t* load_full = bars + 0;
-  uint64_t* s_full = bars + 1;
-  uint64_t* o_full = bars + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 4);
-  uint64_t* q_full = bars + 5;  // later steps: the next group's query rows
-
-  if (tid == 0) {
-    mbar_init(load_full, 1);
-    mbar_init(s_full, 1);
-    mbar_init(o_full, 1);
-    mbar_init(q_full, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 0) {
-    tmem_alloc(tmem_slot, L::kTmemCols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-
-  pdl_launch_dependents();
-  bool load_waited = false;
-  int s_issued = 0, o_issued = 0, q_loads = 0, q_waited = 0;
-  auto issue_s = [&](int q) {
-    tc_fence_after();
-    const uint32_t qb = smem_u32(sQ), kb = smem_u32(sK(q));
-    const uint32_t idesc = idesc_bf16(kRows, NQ, false);
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const uint64_t ad = desc_kmajor(qb + (kk >> 2) * (kRows * 128) + (kk & 3) * 32);
-      const uint64_t bd = desc_kmajor(kb + (kk >> 2) * L::kBox + (kk & 3) * 32);
-      mma_bf16_ss(tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
-    }
-    mma_commit(s_full);
-    ++s_issued;
-  };
-  if (tid == 0) {
-    tma_prefetch_desc(&tm_qt);
-    tma_prefetch_desc(&tm_k);
-    tma_prefetch_desc(&tm_v);
-    mbar_arrive_expect_tx(load_full, D / 64 * kRows * 128 + a.c2 * L::kGroupBytes);
-    for (int q = 0; q < a.c2; ++q) {
-      const int2 kyz = kv_yz(a.tr, g, a.b1, a.b2, k, group_start(a.b2, a.c2, q));
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        tma_load_3d(sK(q) + c * L::kBox, &tm_k, load_full, c * 64, kyz.x, kyz.y);
-        tma_load_3d(sK(q) + (D / 64 + c) * L::kBox, &tm_v, load_full, c * 64, kyz.x, kyz.y);
-      }
-    }
-    pdl_wait();  // the queries come from the previous kernel
-    const int qrow = kr_qrow(a, g, p, k, 0) + i0;
-#pragma unroll
-    for (int c = 0; c < D / 64; ++c) tma_load_2d(sQ + c * kRows * 128, &tm_qt, load_full, c * 64, qrow);
-    load_waited = mbar_wait(load_full, 0, abort_flag, a.status);
-    if (load_waited) issue_s(0);
-  }
-  const int r = tid;  // row of the tile = position i0 + r
-  const bool row_valid = i0 + r < a.b2;
-  for (int q = 0; q < a.c2; ++q) {
-    const int js = group_start(a.b2, a.c2, q);
-    const int nq = group_start(a.b2, a.c2, q + 1) - js;
-    int jlo, jhi;
-    real_keys(a.real_lo, a.real_hi, a.b2, k, js, nq, &jlo, &jhi);
-    bool ok = mbar_wait(s_full, q & 1, abort_flag, a.status);
-    ok = __all_sync(0xffffffffu, ok);
-    if (ok && a.qt_per_item && q + 1 < a.c2 && tid == 0) {
-      // S_q has read this group's rows: the next group's come in meanwhile
-      mbar_arrive_expect_tx(q_full, D / 64 * kRows * 128);
-      const int qrow = kr_qrow(a, g, p, k, q + 1) + i0;
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c)
-        tma_load_2d(sQ + c * kRows * 128, &tm_qt, q_full, c * 64, qrow);
-      ++q_loads;
-    }
-    float z = 0.f, t2 = 0.f;
-    if (ok) {
-      tc_fence_after();
-      float sv[NQ];
-#pragma unroll
-      for (int c = 0; c < NQ / 16; ++c) {
-        float t[16];
-        tmem_ld16(tmem + lane_off + c * 16, t);
-#pragma unroll
-        for (int e = 0; e < 16; ++e) sv[c * 16 + e] = t[e];
-      }
-      tmem_wait_ld();
-      // logits in log2 units; 4 partial maxima and sums break the serial chains
-      r_row_softmax<NQ>(sv, a.sc_log2, jlo, jhi, nq, z, t2);
-#pragma unroll
-      for (int u = 0; u < NQ / 8; ++u) {
-        uint4 pk;
-        pk.x = pack_bf16x2(sv[8 * u + 0], sv[8 * u + 1]);
-        pk.y = pack_bf16x2(sv[8 * u + 2], sv[8 * u + 3]);
-        pk.z = pack_bf16x2(sv[8 * u + 4], sv[8 * u + 5]);
-        pk.w = pack_bf16x2(sv[8 * u + 6], sv[8 * u + 7]);
-        const int chunk = u >> 3, unit = u & 7;
-        *reinterpret_cast<uint4*>(sP + chunk * (kRows * 128) + r * 128 +
-                                  ((unit ^ (r & 7)) << 4)) = pk;
-      }
-      fence_proxy_async_smem();
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (*abort_flag) break;
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t pb = smem_u32(sP), kb = smem_u32(sK(q));
-      const uint32_t idesc = idesc_bf16(kRows, 2 * D, true);
-#pragma unroll
-      for (int kk = 0; kk < NQ / 16; ++kk) {
-        const uint64_t ad = desc_kmajor(pb + (kk >> 2) * (kRows * 128) + (kk & 3) * 32);
-        const uint64_t bd = desc_mnmajor(kb + kk * 16 * 128, L::kBox);
-        mma_bf16_ss(tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
-      }
-      mma_commit(o_full);
-      ++o_issued;
-    }
-    ok = mbar_wait(o_full, q & 1, abort_flag, a.status);
-    ok = __all_sync(0xffffffffu, ok);
-    if (ok) {
-      tc_fence_after();
-      const float inv = z > 0.f ? 1.f / z : 0.f;
-      // The tile's rows of this (g, p, k, q) are positions i0 + r of the
-      // position-major Kt/Y layout: one 4-D TMA box {64 columns, 1, 128
-      // positions, 1} clipped at b2.  Each 64-column block is staged
-      // (swizzled) in one of two buffers and handed to a TMA bulk store; a
-      // buffer is refilled once its previous store has read it.
-      const int nblk = (a.write_y ? 2 : 1) * (D / 64);
-      const int ycoord = (p * a.b1 + k) * a.c2 + q;
-#pragma unroll 1
-      for (int cb = 0; cb < nblk; ++cb) {
-        uint8_t* buf = sStage[cb & 1];
-        if (cb >= 2) {
-          if (tid == 0) bulk_wait_read<1>();
-          __syncthreads();
-        }
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          float t[32];
-          tmem_ld32(tmem + lane_off + cb * 64 + c * 32, t);
-          tmem_wait_ld();
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            uint4 pk;
-            pk.x = pack_bf16x2(t[8 * u + 0] * inv, t[8 * u + 1] * inv);
-            pk.y = pack_bf16x2(t[8 * u + 2] * inv, t[8 * u + 3] * inv);
-            pk.z = pack_bf16x2(t[8 * u + 4] * inv, t[8 * u + 5] * inv);
-            pk.w = pack_bf16x2(t[8 * u + 6] * inv, t[8 * u + 7] * inv);
-            const int unit = c * 4 + u;
-            *reinterpret_cast<uint4*>(buf + r * 128 + ((unit ^ (r & 7)) << 4)) = pk;
-          }
-        }
-        fence_proxy_async_smem();
-        __syncthreads();
-        if (tid == 0) {
-          tma_store_4d(cb < D / 64 ? &tm_kt : &tm_y, buf, (cb % (D / 64)) * 64, ycoord, i0, g);
-          bulk_commit();
-        }
-      }
-      // the staging buffers (P among them) are reused by the next group
-      if (tid == 0) bulk_wait_read<0>();
-      // entropy of the R row: ln z - sum e (s - m) / z, with s - m in log2 units
-      if (row_valid) {
-        const long orow = ((((long)g * a.b2 + i0 + r) * a.c1 + p) * a.b1 + k) * a.c2 + q;
-        a.hs[orow] = z > 0.f ? logf(z) - t2 * 0.69314718055994531f * inv : -INFINITY;
-      }
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (*abort_flag) break;
-    if (tid == 0 && q + 1 < a.c2) {
-      bool qok = true;
-      if (a.qt_per_item) {
-        qok = mbar_wait(q_full, q_waited & 1, abort_flag, a.status);
-        if (qok) ++q_waited;
-      }
-      if (qok) issue_s(q + 1);
-    }
-  }
-  if (tid == 0 && *abort_flag) {
-    if (!load_waited) drain(load_full, 0);
-    if (q_loads > q_waited) drain(q_full, q_waited & 1);
-    if (s_issued > 0) drain(s_full, (s_issued - 1) & 1);
-    if (o_issued > 0) drain(o_full, (o_issued - 1) & 1);
-  }
-  if (tid == 0) bulk_wait<0>();  // stores done reading shared memory before the CTA exits
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) {
-    tc_fence_after();
-    tmem_dealloc(tmem, L::kTmemCols);
-  }
 }
 
 // ---------------------------------------------------------------------------
@@ -3166,70 +2922,6 @@ cudaError_t dispatch_ko(const bf16* q, const bf16* kt, const bf16* y, const floa
   return launch_ko<D, 64>(q, kt, y, hs, out, pb, status, stream, launches);
 }
 
-template <int D, int NQ>
-cudaError_t launch_kr(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, bf16* y, float* hs,
-                      const Problem& pb, int* status, cudaStream_t stream, int* launches,
-                      bool qt_per_item = false, bool write_y = false) {
-  using L = KRLayout<D, NQ>;
-  constexpr int kMaxBytes = L::bytes(256 / NQ);
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(kr_kernel<D, NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    kMaxBytes);
-    if (attr_err == cudaSuccess)
-      attr_err = cudaFuncSetAttribute(kr_kernel<D, NQ>,
-                                      cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-  });
-  if (attr_err != cudaSuccess) return attr_err;
-  if (L::bytes(pb.c2) > kMaxBytes) return cudaErrorInvalidValue;
-  CUtensorMap tq, tk, tv;
-  {
-    const cuuint64_t rows = (cuuint64_t)pb.G * pb.c1 * pb.b2 * (qt_per_item ? pb.b1 * pb.c2 : 1);
-    const cuuint64_t dims[2] = {(cuuint64_t)D, rows};
-    const cuuint64_t str[1] = {(cuuint64_t)D * 2};
-    const cuuint32_t box[2] = {64, kRows};
-    if (!make_map(&tq, qt0, 2, dims, str, box)) return cudaErrorInvalidValue;
-  }
-  {
-    if (!make_kv_map(&tk, k, pb, D, NQ) || !make_kv_map(&tv, v, pb, D, NQ))
-      return cudaErrorInvalidValue;
-  }
-  CUtensorMap tkt, tyy;
-  {
-    // Kt / Y [G][b2 i][c1 p][b1 k][c2 q][d] viewed as (d, c1*b1*c2, b2, G); a
-    // tile's box is {64 columns, 1, 128 positions, 1}, clipped at b2
-    const cuuint64_t ny = (cuuint64_t)pb.c1 * pb.b1 * pb.c2;
-    const cuuint64_t dims[4] = {(cuuint64_t)D, ny, (cuuint64_t)pb.b2, (cuuint64_t)pb.G};
-    const cuuint64_t str[3] = {(cuuint64_t)D * 2, ny * D * 2, ny * pb.b2 * D * 2};
-    const cuuint32_t box[4] = {64, 1, kRows, 1};
-    if (!make_map(&tkt, kt, 4, dims, str, box)) return cudaErrorInvalidValue;
-    if (!make_map(&tyy, y, 4, dims, str, box)) return cudaErrorInvalidValue;
-  }
-  KRArgs a;
-  a.kt = kt;
-  a.y = y;
-  a.hs = hs;
-  a.b1 = pb.b1;
-  a.b2 = pb.b2;
-  a.c1 = pb.c1;
-  a.c2 = pb.c2;
-  a.write_y = (qt_per_item ? write_y : pb.T == 1) ? 1 : 0;
-  a.qt_per_item = qt_per_item ? 1 : 0;
-  a.sc_log2 = kLog2e * pb.sc;
-  a.status = status;
-  a.tr = pb.tr;
-  a.real_lo = pb.real_lo;
-  a.real_hi = pb.real_hi;
-  a.n_itiles = (pb.b2 + kRows - 1) / kRows;
-  const long blocks = (long)pb.G * pb.b1 * pb.c1 * a.n_itiles;
-  if (blocks >= (1L << 31)) return cudaErrorInvalidValue;
-  return timed_launch("tc_r_update", stream, launches, [&] {
-    return launch_pdl(kr_kernel<D, NQ>, dim3((unsigned)blocks), dim3(128), L::bytes(pb.c2), stream, tq,
-               tk, tv, tkt, tyy, a);
-  });
-}
-
 // qt_per_item: the queries are the per-sub-item rows of a later step (else
 // step one's Qt0); write_y: this is the last step (Y is written too).
 template <int D, int NQ, bool PAIR>
@@ -3357,14 +3049,6 @@ cudaError_t launch_krl(const bf16* qt0, const bf16* k, const bf16* v, bf16* kt, 
     return launch_pdl(krl_kernel<D>, dim3(grid), dim3(320), L::kBytes, stream, tq, tk, tv, tkt,
                       tyy, a, (int)items);
   });
-}
-
-// The per-item R-update kernel holds every column group of a chunk in
-// shared memory: groups of <= 128 keys (and <= 2d, its TMEM), at most 256
-// keys in all.  Wider groups stream through krl_kernel.
-inline bool kr_holds_groups(const Problem& pb) {
-  const int nq = kr_group_tile(pb);
-  return nq <= 128 && nq <= 2 * pb.d && pb.c2 * nq <= 256;
 }
 
 template <int D>
@@ -3517,29 +3201,13 @@ cudaError_t launch_later_step(const bf16* q, const bf16* k, const bf16* v, bf16*
       default: return cudaErrorInvalidValue;
     }
   }
-  if (!kr_holds_groups(pb))
-    return launch_krl<D>(qt, k, v, kt, y, hs, pb, status, stream, launches, true, last);
-  switch (kr_group_tile(pb)) {
-#define MONARCH_KR_STEP(NQ)                                                                   \
-  case NQ:                                                                                    \
-    return launch_kr<D, NQ>(qt, k, v, kt, y, hs, pb, status, stream, launches, true, last);
-    MONARCH_KR_STEP(16)
-    MONARCH_KR_STEP(32)
-    MONARCH_KR_STEP(48)
-    MONARCH_KR_STEP(64)
-    MONARCH_KR_STEP(80)
-    MONARCH_KR_STEP(96)
-    MONARCH_KR_STEP(112)
-    MONARCH_KR_STEP(128)
-#undef MONARCH_KR_STEP
-    default: return cudaErrorInvalidValue;
-  }
+  return launch_krl<D>(qt, k, v, kt, y, hs, pb, status, stream, launches, true, last);
 }
 
-// Step one: aggregated queries under the uniform L, then the R-update: the
-// persistent kernel for column groups of <= 64 keys over <= 128 positions,
-// the per-item kernel for groups it holds in shared memory, the streaming
-// kernel for wider ones.
+// Step one: aggregated queries under the uniform L, then the R-update: one
+// warp per group on the CUDA cores for groups of <= 8 keys over <= 32
+// positions, the paired-tile kernel for column groups of <= 64 keys over
+// <= 128 positions, the streaming kernel for wider groups or more positions.
 template <int D>
 cudaError_t launch_r_step1(const bf16* q, const bf16* k, const bf16* v, bf16* qt0, bf16* kt,
                            bf16* y, float* hs, const Problem& pb, int* status,
@@ -3579,23 +3247,8 @@ cudaError_t launch_r_step1(const bf16* q, const bf16* k, const bf16* v, bf16* qt
       default: return cudaErrorInvalidValue;
     }
   }
-  // groups the per-item kernel holds in shared memory (any number of
-  // 128-position tiles), else the streaming kernel
-  if (!kr_holds_groups(pb)) return launch_krl<D>(qt0, k, v, kt, y, hs, pb, status, stream, launches);
-  switch (kr_group_tile(pb)) {
-#define MONARCH_KR_CASE(NQ) \
-  case NQ: return launch_kr<D, NQ>(qt0, k, v, kt, y, hs, pb, status, stream, launches);
-    MONARCH_KR_CASE(16)
-    MONARCH_KR_CASE(32)
-    MONARCH_KR_CASE(48)
-    MONARCH_KR_CASE(64)
-    MONARCH_KR_CASE(80)
-    MONARCH_KR_CASE(96)
-    MONARCH_KR_CASE(112)
-    MONARCH_KR_CASE(128)
-#undef MONARCH_KR_CASE
-    default: return cudaErrorInvalidValue;
-  }
+  // wider groups, or more than 128 positions: the streaming kernel
+  return launch_krl<D>(qt0, k, v, kt, y, hs, pb, status, stream, launches);
 }
 
 constexpr size_t kAlign = 256;
