@@ -88,15 +88,16 @@ __global__ void __launch_bounds__(kWarps * 32)
     small_init_kernel(const bf16* __restrict__ q, bf16* __restrict__ qt0, Problem pb) {
   constexpr int E = D / 32;
   const int lane = threadIdx.x & 31;
-  const long unit = (long)blockIdx.x * kWarps + (threadIdx.x >> 5);
+  // 32-bit index arithmetic (the launch checks that every index fits)
+  const int unit = (int)blockIdx.x * kWarps + (int)(threadIdx.x >> 5);
   // qt0 may still be read by the previous call's R-update
   pdl_wait();
   pdl_launch_dependents();
-  if (unit >= (long)pb.G * pb.c1 * pb.b2) return;
-  const int i = (int)(unit % pb.b2);
-  const long gp = unit / pb.b2;
-  const int p = (int)(gp % pb.c1);
-  const long g = gp / pb.c1;
+  if (unit >= pb.G * pb.c1 * pb.b2) return;
+  const int i = unit % pb.b2;
+  const int gp = unit / pb.b2;
+  const int p = gp % pb.c1;
+  const int g = gp / pb.c1;
   const int l0 = group_start(pb.b1, pb.c1, p), l1 = group_start(pb.b1, pb.c1, p + 1);
   float acc[E];
 #pragma unroll
@@ -110,7 +111,7 @@ __global__ void __launch_bounds__(kWarps * 32)
   const float n = (float)(l1 - l0);
 #pragma unroll
   for (int e = 0; e < E; ++e) acc[e] /= n;
-  store_row<E>(qt0 + unit * D + lane * E, acc);
+  store_row<E>(qt0 + (long)unit * D + lane * E, acc);
 }
 
 // Sub-item (g, p, k, q) of the R-update, in the tensor-core kernels' order;
@@ -122,16 +123,17 @@ __global__ void __launch_bounds__(kWarps * 32)
                    float* __restrict__ hs, Problem pb, int qt_per_item, int write_y) {
   constexpr int E = D / 32;
   const int lane = threadIdx.x & 31;
-  const long sub = (long)blockIdx.x * kWarps + (threadIdx.x >> 5);
+  // 32-bit index arithmetic (the launch checks that every index fits)
+  const int sub = (int)blockIdx.x * kWarps + (int)(threadIdx.x >> 5);
   pdl_wait();  // the query rows come from the previous kernel
   pdl_launch_dependents();
-  if (sub >= (long)pb.G * pb.c1 * pb.b1 * pb.c2) return;
-  const int q = (int)(sub % pb.c2);
-  const long item = sub / pb.c2;
-  const int kc = (int)(item % pb.b1);
-  const long gp = item / pb.b1;
-  const int p = (int)(gp % pb.c1);
-  const long g = gp / pb.c1;
+  if (sub >= pb.G * pb.c1 * pb.b1 * pb.c2) return;
+  const int q = sub % pb.c2;
+  const int item = sub / pb.c2;
+  const int kc = item % pb.b1;
+  const int gp = item / pb.b1;
+  const int p = gp % pb.c1;
+  const int g = gp / pb.c1;
   const int js = group_start(pb.b2, pb.c2, q), nq = group_start(pb.b2, pb.c2, q + 1) - js;
   // the group's keys and values, row j of chunk kc
   float kr[NK][E], vr[NK][E];
@@ -144,8 +146,9 @@ __global__ void __launch_bounds__(kWarps * 32)
     }
   }
   const float sc_log2 = pb.sc * kLog2e;
-  const bf16* qrows = qt + (qt_per_item ? (((g * pb.b1 + kc) * pb.c1 + p) * pb.c2 + q) * pb.b2
-                                        : (g * pb.c1 + p) * pb.b2) * D + lane * E;
+  // Qt0 [G][c1][b2][d] (step one) or a later step's Qt [G][b1][c1][c2][b2][d]
+  const int qset = qt_per_item ? ((g * pb.b1 + kc) * pb.c1 + p) * pb.c2 + q : gp;
+  const bf16* qrows = qt + (long)qset * pb.b2 * D + lane * E;
   float qn[E];
   load_row<E>(qrows, qn);
   for (int i = 0; i < pb.b2; ++i) {
@@ -190,7 +193,7 @@ __global__ void __launch_bounds__(kWarps * 32)
       }
     }
     // [G][b2][c1][b1][c2] row of (g, i, p, kc, q)
-    const long orow = (((g * pb.b2 + i) * pb.c1 + p) * pb.b1 + kc) * pb.c2 + q;
+    const long orow = (long)(((g * pb.b2 + i) * pb.c1 + p) * pb.b1 + kc) * pb.c2 + q;
     store_row<E>(kt + orow * D + lane * E, ko);
     if (write_y) store_row<E>(y + orow * D + lane * E, yo);
     // entropy -sum R ln R = ln z - sum_j e_j (x_j - max) ln 2 / z
@@ -207,16 +210,17 @@ __global__ void __launch_bounds__(kWarps * 32)
                      bf16* __restrict__ out, Problem pb) {
   constexpr int E = D / 32;
   const int lane = threadIdx.x & 31;
-  const long item = (long)blockIdx.x * kWarps + (threadIdx.x >> 5);
+  // 32-bit index arithmetic (the launch checks that every index fits)
+  const int item = (int)blockIdx.x * kWarps + (int)(threadIdx.x >> 5);
   pdl_wait();  // Kt, Y and Hs come from the previous kernel
   pdl_launch_dependents();
-  if (item >= (long)pb.G * pb.b2 * pb.c1) return;
-  const int p = (int)(item % pb.c1);
-  const long gi = item / pb.c1;
-  const int i = (int)(gi % pb.b2);
-  const long g = gi / pb.b2;
+  if (item >= pb.G * pb.b2 * pb.c1) return;
+  const int p = item % pb.c1;
+  const int gi = item / pb.c1;
+  const int i = gi % pb.b2;
+  const int g = gi / pb.b2;
   const int nk = pb.b1 * pb.c2;
-  const long key0 = item * nk;  // row ((g b2 + i) c1 + p) nk of Kt, Y and Hs
+  const long key0 = (long)item * nk;  // row ((g b2 + i) c1 + p) nk of Kt, Y and Hs
   float kr[NK][E], yr[NK][E], bias[NK];
 #pragma unroll
   for (int j = 0; j < NK; ++j) {
@@ -272,20 +276,27 @@ unsigned blocks_for(long warps) { return (unsigned)((warps + kWarps - 1) / kWarp
 
 }  // namespace
 
+// The kernels index units, sub-items, items and the rows of Qt and of Kt / Y
+// / Hs ([G][b2][c1][b1][c2]) in 32-bit arithmetic: every such count must be
+// below 2^31.
+static bool small_indices_fit(const Problem& pb) {
+  return (long)pb.G * pb.b2 * pb.c1 * pb.b1 * pb.c2 < (1L << 31) &&
+         (long)pb.G * pb.c1 * pb.b2 * (pb.b1 * pb.c2) < (1L << 31);
+}
+
 bool small_init_fits(const Problem& pb) {
   return (pb.d == 64 || pb.d == 128) && !is_padded(pb) &&
-         (pb.b1 + pb.c1 - 1) / pb.c1 <= kMaxRows && (long)pb.G * pb.c1 * pb.b2 < (1L << 31);
+         (pb.b1 + pb.c1 - 1) / pb.c1 <= kMaxRows && small_indices_fit(pb);
 }
 
 bool small_r_fits(const Problem& pb) {
   return (pb.d == 64 || pb.d == 128) && !is_padded(pb) &&
-         (pb.b2 + pb.c2 - 1) / pb.c2 <= kMaxKeys && pb.b2 <= kMaxPos &&
-         (long)pb.G * pb.c1 * pb.b1 * pb.c2 < (1L << 31) * kWarps;
+         (pb.b2 + pb.c2 - 1) / pb.c2 <= kMaxKeys && pb.b2 <= kMaxPos && small_indices_fit(pb);
 }
 
 bool small_out_fits(const Problem& pb) {
   return (pb.d == 64 || pb.d == 128) && !is_padded(pb) && pb.b1 * pb.c2 <= kMaxKeys &&
-         (long)pb.G * pb.b2 * pb.c1 < (1L << 31) * kWarps;
+         small_indices_fit(pb);
 }
 
 cudaError_t launch_small_init(const bf16* q, bf16* qt0, const Problem& pb, cudaStream_t stream,
