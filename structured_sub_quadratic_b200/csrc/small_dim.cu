@@ -276,12 +276,11 @@ unsigned blocks_for(long warps) { return (unsigned)((warps + kWarps - 1) / kWarp
 
 }  // namespace
 
-// The kernels index units, sub-items, items and the rows of Qt and of Kt / Y
-// / Hs ([G][b2][c1][b1][c2]) in 32-bit arithmetic: every such count must be
-// below 2^31.
+// The kernels index units, sub-items, items, the query sets of Qt and the
+// rows of Kt / Y / Hs ([G][b2][c1][b1][c2]) in 32-bit arithmetic; the largest
+// of these counts is G b2 c1 b1 c2.
 static bool small_indices_fit(const Problem& pb) {
-  return (long)pb.G * pb.b2 * pb.c1 * pb.b1 * pb.c2 < (1L << 31) &&
-         (long)pb.G * pb.c1 * pb.b2 * (pb.b1 * pb.c2) < (1L << 31);
+  return (long)pb.G * pb.b2 * pb.c1 * pb.b1 * pb.c2 < (1L << 31);
 }
 
 bool small_init_fits(const Problem& pb) {
