@@ -92,10 +92,16 @@ MONARCH_API int monarch_attn_fwd_f32(const float* q, const float* k, const float
                          cudaStream_t stream);
 
 /* Same computation on HOST buffers (dtype MONARCH_DTYPE_BF16 or _F32).
- * Copies q, k, v to cached device staging buffers on `stream`, runs the
- * forward pass, copies the result into out_host and synchronises `stream`
- * before returning.  Pinned host memory gives full PCIe/C2C bandwidth;
- * pageable memory works but is slower. */
+ * Copies q, k, v to cached device staging buffers, runs the forward pass and
+ * copies the result into out_host, in up to 12 groups of heads: a group's
+ * copy-in (on a copy stream of the library's own), its forward pass (on
+ * `stream`) and its copy-out (on a second copy stream) overlap the
+ * neighbouring groups', ordered by events after the work already on
+ * `stream`.  The output is bit-identical to monarch_attn_fwd's (every group
+ * runs the kernels of the whole call).  Synchronises `stream` and both copy
+ * streams before returning, on success and on error.  Pinned host memory
+ * gives full PCIe/C2C bandwidth and the overlap; pageable memory works but
+ * is slower. */
 MONARCH_API int monarch_attn_fwd_host(int dtype, const void* q_host, const void* k_host,
                           const void* v_host, void* out_host,
                           int B, int H, int b1, int b2, int d, int T, int c1, int c2,

@@ -32,6 +32,11 @@ struct Problem {
   float sc;  // 1/sqrt(d)
   int real_lo, real_hi;
   int tr;
+  // Launch-shape hint: when a call is split into groups of heads, the
+  // (g, p, i) unit count of the whole call, which the bf16 step-one
+  // aggregation's thread count follows (its row sums' order depends on it),
+  // so that the split call gives bit-identical results; 0 means G c1 b2.
+  long init_units;
 };
 
 // Row of token (l, i) of head g in q, k, v and out.

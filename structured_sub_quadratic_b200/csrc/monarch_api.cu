@@ -7,6 +7,7 @@
 // else.  The video-layout entry point reorders tokens around a forward call.
 #include "monarch_attn.h"
 
+#include <algorithm>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -44,6 +45,19 @@ std::mutex g_layout_mu;         // held for a whole video-layout call
 std::mutex g_pad_mu;            // held for a whole padded call
 DevBuf g_ws[kMaxDevices];      // kernel workspace
 DevBuf g_stage[kMaxDevices];   // staging for the host-buffer entry point
+
+// Copy pipeline of the host-buffer entry point, per device (guarded by
+// g_stage_mu; created on first use, kept until the process exits): a
+// host-to-device and a device-to-host copy stream, and the events that order
+// them with the caller's stream, one pair per group of heads.
+constexpr int kHostChunks = 12;
+struct HostPipe {
+  bool ready = false;
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t start = nullptr, done = nullptr;
+  cudaEvent_t in[kHostChunks] = {}, comp[kHostChunks] = {};
+};
+HostPipe g_pipe[kMaxDevices];
 DevBuf g_layout[kMaxDevices];  // reordered q, k, v and output of the video-layout entry point
 DevBuf g_pad[kMaxDevices];     // padded q, k, v and output of the padded entry point
 DevBuf g_bwd[kMaxDevices];     // workspace of the backward pass
@@ -181,10 +195,12 @@ int status_word_locked(int dev, int** out) {
 
 // real_lo, real_hi: the real tokens of the b1*b2 grid (padding; the default
 // is every token).  q, k, v, out always hold whole grids here.
+// init_units: the launch-shape hint of Problem (a call split into groups of
+// heads passes the whole call's unit count).
 template <typename TIn>
 int forward_device(const TIn* q, const TIn* k, const TIn* v, TIn* out, int B, int H, int b1,
                    int b2, int d, int T, int c1, int c2, cudaStream_t stream, int dtype,
-                   int real_lo = 0, int real_hi = -1, int tr = 0) {
+                   int real_lo = 0, int real_hi = -1, int tr = 0, long init_units = 0) {
   t_launches = 0;
   int st = monarch::validate_args(B, H, b1, b2, d, T, c1, c2);
   if (st != MONARCH_OK) return st;
@@ -196,6 +212,7 @@ int forward_device(const TIn* q, const TIn* k, const TIn* v, TIn* out, int B, in
     pb.real_hi = real_hi;
   }
   pb.tr = tr;
+  pb.init_units = init_units;
   const size_t bytes_io = (size_t)pb.G * b1 * b2 * d * sizeof(TIn);
   const char* o0 = reinterpret_cast<const char*>(out);
   for (const void* in : {(const void*)q, (const void*)k, (const void*)v}) {
@@ -260,6 +277,7 @@ Problem make_problem(int B, int H, int b1, int b2, int d, int T, int c1, int c2)
   pb.real_lo = 0;
   pb.real_hi = b1 * b2;
   pb.tr = 0;
+  pb.init_units = 0;
   return pb;
 }
 
@@ -304,7 +322,9 @@ int monarch_attn_fwd_host(int dtype, const void* q_host, const void* k_host, con
   int st = monarch::validate_args(B, H, b1, b2, d, T, c1, c2);
   if (st != MONARCH_OK) return st;
   const size_t elt = dtype == MONARCH_DTYPE_BF16 ? 2 : 4;
-  const size_t n = (size_t)B * H * b1 * b2 * d * elt;
+  const size_t head_bytes = (size_t)b1 * b2 * d * elt;
+  const long G = (long)B * H;
+  const size_t n = (size_t)G * head_bytes;
   const size_t slot = align_up(n);
   int dev;
   if ((st = current_device(&dev)) != MONARCH_OK) return st;
@@ -313,21 +333,83 @@ int monarch_attn_fwd_host(int dtype, const void* q_host, const void* k_host, con
     std::lock_guard<std::mutex> lock(g_mu);
     if ((st = ensure(g_stage[dev], 4 * slot)) != MONARCH_OK) return st;
   }
+  HostPipe& pp = g_pipe[dev];
+  cudaError_t e = cudaSuccess;
+  if (!pp.ready) {
+    if ((e = cudaStreamCreateWithFlags(&pp.h2d, cudaStreamNonBlocking)) != cudaSuccess ||
+        (e = cudaStreamCreateWithFlags(&pp.d2h, cudaStreamNonBlocking)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&pp.start, cudaEventDisableTiming)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&pp.done, cudaEventDisableTiming)) != cudaSuccess)
+      return record_cuda(e);
+    for (int c = 0; c < kHostChunks; ++c)
+      if ((e = cudaEventCreateWithFlags(&pp.in[c], cudaEventDisableTiming)) != cudaSuccess ||
+          (e = cudaEventCreateWithFlags(&pp.comp[c], cudaEventDisableTiming)) != cudaSuccess)
+        return record_cuda(e);
+    pp.ready = true;
+  }
   char* base = static_cast<char*>(g_stage[dev].ptr);
   char *dq = base, *dk = base + slot, *dv = base + 2 * slot, *dout = base + 3 * slot;
-  cudaError_t e;
-  if ((e = cudaMemcpyAsync(dq, q_host, n, cudaMemcpyHostToDevice, stream)) != cudaSuccess ||
-      (e = cudaMemcpyAsync(dk, k_host, n, cudaMemcpyHostToDevice, stream)) != cudaSuccess ||
-      (e = cudaMemcpyAsync(dv, v_host, n, cudaMemcpyHostToDevice, stream)) != cudaSuccess)
+  // Heads are independent: groups of heads are copied in on pp.h2d, computed
+  // on `stream` and copied out on pp.d2h, so that group c + 1's copy-in and
+  // group c - 1's copy-out overlap group c's forward pass.  Each group runs
+  // the kernels of the whole call (the launch-shape hint), so the output is
+  // bit-identical to monarch_attn_fwd's.
+  const long hc = (G + kHostChunks - 1) / kHostChunks;  // heads per group
+  const int nc = (int)((G + hc - 1) / hc);
+  const long init_units = G * c1 * b2;
+  const auto* qh = static_cast<const char*>(q_host);
+  const auto* kh = static_cast<const char*>(k_host);
+  const auto* vh = static_cast<const char*>(v_host);
+  auto* oh = static_cast<char*>(out_host);
+  int launches = 0;
+  // the copies start after the work already on `stream`
+  if ((e = cudaEventRecord(pp.start, stream)) != cudaSuccess ||
+      (e = cudaStreamWaitEvent(pp.h2d, pp.start, 0)) != cudaSuccess)
     return record_cuda(e);
-  st = dtype == MONARCH_DTYPE_BF16
-           ? monarch_attn_fwd(dq, dk, dv, dout, B, H, b1, b2, d, T, c1, c2, stream)
-           : monarch_attn_fwd_f32(reinterpret_cast<float*>(dq), reinterpret_cast<float*>(dk),
-                                  reinterpret_cast<float*>(dv), reinterpret_cast<float*>(dout), B,
-                                  H, b1, b2, d, T, c1, c2, stream);
-  if (st != MONARCH_OK) return st;
-  if ((e = cudaMemcpyAsync(out_host, dout, n, cudaMemcpyDeviceToHost, stream)) != cudaSuccess)
-    return record_cuda(e);
+  for (int c = 0; c < nc && st == MONARCH_OK && e == cudaSuccess; ++c) {
+    const long h0 = c * hc, hn = std::min(hc, G - h0);
+    const size_t off = (size_t)h0 * head_bytes, bytes = (size_t)hn * head_bytes;
+    if ((e = cudaMemcpyAsync(dq + off, qh + off, bytes, cudaMemcpyHostToDevice, pp.h2d)) !=
+            cudaSuccess ||
+        (e = cudaMemcpyAsync(dk + off, kh + off, bytes, cudaMemcpyHostToDevice, pp.h2d)) !=
+            cudaSuccess ||
+        (e = cudaMemcpyAsync(dv + off, vh + off, bytes, cudaMemcpyHostToDevice, pp.h2d)) !=
+            cudaSuccess ||
+        (e = cudaEventRecord(pp.in[c], pp.h2d)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(stream, pp.in[c], 0)) != cudaSuccess)
+      break;
+    st = dtype == MONARCH_DTYPE_BF16
+             ? forward_device<monarch::bf16>(
+                   reinterpret_cast<const monarch::bf16*>(dq + off),
+                   reinterpret_cast<const monarch::bf16*>(dk + off),
+                   reinterpret_cast<const monarch::bf16*>(dv + off),
+                   reinterpret_cast<monarch::bf16*>(dout + off), 1, (int)hn, b1, b2, d, T, c1, c2,
+                   stream, MONARCH_DTYPE_BF16, 0, -1, 0, init_units)
+             : forward_device<float>(reinterpret_cast<const float*>(dq + off),
+                                     reinterpret_cast<const float*>(dk + off),
+                                     reinterpret_cast<const float*>(dv + off),
+                                     reinterpret_cast<float*>(dout + off), 1, (int)hn, b1, b2, d,
+                                     T, c1, c2, stream, MONARCH_DTYPE_F32, 0, -1, 0, init_units);
+    launches += t_launches;
+    if (st != MONARCH_OK) break;
+    if ((e = cudaEventRecord(pp.comp[c], stream)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(pp.d2h, pp.comp[c], 0)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(oh + off, dout + off, bytes, cudaMemcpyDeviceToHost, pp.d2h)) !=
+            cudaSuccess)
+      break;
+  }
+  if (e == cudaSuccess && st == MONARCH_OK) {
+    if ((e = cudaEventRecord(pp.done, pp.d2h)) == cudaSuccess)
+      e = cudaStreamWaitEvent(stream, pp.done, 0);
+  }
+  t_launches = launches;
+  if (e != cudaSuccess || st != MONARCH_OK) {
+    // nothing may still read or write the caller's buffers after the return
+    cudaStreamSynchronize(pp.h2d);
+    cudaStreamSynchronize(pp.d2h);
+    cudaStreamSynchronize(stream);
+    return e != cudaSuccess ? record_cuda(e) : st;
+  }
   return monarch_attn_check(stream);
 }
 

@@ -3216,12 +3216,14 @@ cudaError_t launch_r_step1(const bf16* q, const bf16* k, const bf16* v, bf16* qt
       small_init_fits(pb)
           ? launch_small_init(q, qt0, pb, stream, launches)
           : timed_launch("tc_init_qt", stream, launches, [&] {
-              // fewer units than SMs (a few long row groups): 32 warps per unit
+              // fewer units than SMs (a few long row groups): 32 warps per unit.
+              // The thread count follows the whole call's units (see Problem).
               const long units = (long)pb.G * pb.c1 * pb.b2;
-              if (units < num_sms())
+              const long shape_units = pb.init_units > 0 ? pb.init_units : units;
+              if (shape_units < num_sms())
                 return launch_pdl(init_qt_bf16_kernel<D, 1024>, dim3((unsigned)units),
                                   dim3(1024), 0, stream, q, qt0, pb);
-              return units <= 5L * num_sms()
+              return shape_units <= 5L * num_sms()
                          ? launch_pdl(init_qt_bf16_kernel<D, 256>, dim3((unsigned)units),
                                       dim3(256), 0, stream, q, qt0, pb)
                          : launch_pdl(init_qt_bf16_kernel<D, 128>, dim3((unsigned)units),

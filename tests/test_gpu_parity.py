@@ -126,6 +126,22 @@ def test_host_buffer_entry_matches_device_entry(cuda_lib):
     np.testing.assert_array_equal(out.double().numpy(), O)
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_host_buffer_entry_pipelines_head_groups(cuda_lib, dtype):
+    """The host-buffer entry copies and computes in groups of heads on three
+    streams: with 26 heads (groups of 3, the last of 2) and two different
+    input sets back to back, each result equals the device entry's bit for
+    bit."""
+    B, H, b1, b2, d, T = 2, 13, 12, 20, 64, 1
+    for seed in (21, 22):
+        q, k, v = iid_qkv(B, H, b1 * b2, d, dtype, seed=seed)
+        qh, kh, vh = (x.pin_memory() for x in (q, k, v))
+        out = torch.empty_like(qh).pin_memory()
+        cuda_lib.monarch_attn_fwd_host(qh, kh, vh, out, b1, b2, T)
+        O = gpu_forward(cuda_lib, q, k, v, b1, b2, T)
+        np.testing.assert_array_equal(out.double().numpy(), O)
+
+
 def test_repeat_calls_are_deterministic(cuda_lib):
     wl = WORKLOADS["480p"]
     q, k, v = (x.cuda() for x in make_inputs(wl))
