@@ -93,7 +93,8 @@ MONARCH_API int monarch_attn_fwd_f32(const float* q, const float* k, const float
 
 /* Same computation on HOST buffers (dtype MONARCH_DTYPE_BF16 or _F32).
  * Copies q, k, v to cached device staging buffers, runs the forward pass and
- * copies the result into out_host, in up to 12 groups of heads: a group's
+ * copies the result into out_host, in groups of heads (up to 12, each with
+ * at least 32 MiB of q, k and v; smaller calls take one group): a group's
  * copy-in (on a copy stream of the library's own), its forward pass (on
  * `stream`) and its copy-out (on a second copy stream) overlap the
  * neighbouring groups', ordered by events after the work already on

@@ -51,6 +51,7 @@ DevBuf g_stage[kMaxDevices];   // staging for the host-buffer entry point
 // host-to-device and a device-to-host copy stream, and the events that order
 // them with the caller's stream, one pair per group of heads.
 constexpr int kHostChunks = 12;
+constexpr size_t kHostGroupBytes = (size_t)32 << 20;
 struct HostPipe {
   bool ready = false;
   cudaStream_t h2d = nullptr, d2h = nullptr;
@@ -354,7 +355,11 @@ int monarch_attn_fwd_host(int dtype, const void* q_host, const void* k_host, con
   // group c - 1's copy-out overlap group c's forward pass.  Each group runs
   // the kernels of the whole call (the launch-shape hint), so the output is
   // bit-identical to monarch_attn_fwd's.
-  const long hc = (G + kHostChunks - 1) / kHostChunks;  // heads per group
+  // groups of at least kHostGroupBytes of input (a smaller call's forward
+  // pass is too short to hide copies behind, and each group adds copy and
+  // launch overhead), at most kHostChunks
+  const long groups = std::max(1L, std::min((long)kHostChunks, (long)(3 * n / kHostGroupBytes)));
+  const long hc = (G + groups - 1) / groups;  // heads per group
   const int nc = (int)((G + hc - 1) / hc);
   const long init_units = G * c1 * b2;
   const auto* qh = static_cast<const char*>(q_host);

@@ -128,11 +128,12 @@ def test_host_buffer_entry_matches_device_entry(cuda_lib):
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_host_buffer_entry_pipelines_head_groups(cuda_lib, dtype):
-    """The host-buffer entry copies and computes in groups of heads on three
-    streams: with 26 heads (groups of 3, the last of 2) and two different
+    """The host-buffer entry copies and computes in groups of heads (at least
+    32 MiB of input each) on three streams: with 26 heads of 16 K tokens (9
+    groups of up to 3 heads in fp32, 4 of up to 7 in bf16) and two different
     input sets back to back, each result equals the device entry's bit for
     bit."""
-    B, H, b1, b2, d, T = 2, 13, 12, 20, 64, 1
+    B, H, b1, b2, d, T = 2, 13, 128, 128, 64, 1
     for seed in (21, 22):
         q, k, v = iid_qkv(B, H, b1 * b2, d, dtype, seed=seed)
         qh, kh, vh = (x.pin_memory() for x in (q, k, v))
