@@ -17,21 +17,23 @@ struct RowPairs {
   void* dst[3];
 };
 
-template <typename U, int UNITS>
+// I: the index type, int when every unit index fits (a 32-bit division per
+// unit instead of a 64-bit one), else long.
+template <typename U, int UNITS, typename I>
 __global__ void __launch_bounds__(256)
-    permute_rows_kernel(RowPairs pairs, const int* __restrict__ table, long total, int N,
+    permute_rows_kernel(RowPairs pairs, const int* __restrict__ table, I total, int N,
                         int units_rt, bool to_monarch) {
   const int units = UNITS > 0 ? UNITS : units_rt;
   const U* __restrict__ src = static_cast<const U*>(pairs.src[blockIdx.y]);
   U* __restrict__ dst = static_cast<U*>(pairs.dst[blockIdx.y]);
-  for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
-       idx += (long)gridDim.x * blockDim.x) {
-    const long row = idx / units;
+  for (I idx = (I)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (I)gridDim.x * blockDim.x) {
+    const I row = idx / units;
     const int c = (int)(idx - row * units);
-    const long g = row / N;
+    const I g = row / N;
     const int m = (int)(row - g * N);
-    const long n = __ldg(table + m);
-    const long mi = (g * N + m) * units + c, ni = (g * N + n) * units + c;
+    const I n = __ldg(table + m);
+    const I mi = (g * N + m) * units + c, ni = (g * N + n) * units + c;
     if (to_monarch)
       dst[mi] = src[ni];
     else
@@ -50,8 +52,12 @@ cudaError_t launch(const RowPairs& pairs, int npairs, const int* table, long G, 
   const long want = (total + 255) / 256;
   const int grid = (int)(want < 16L * sms ? want : 16L * sms);
   return timed_launch("permute_rows", stream, launches, [&] {
-    permute_rows_kernel<U, UNITS><<<dim3(grid, npairs), 256, 0, stream>>>(pairs, table, total, N,
-                                                                          units, to_monarch);
+    if (total < (1L << 31) - 256L * grid)  // idx never overflows int
+      permute_rows_kernel<U, UNITS, int><<<dim3(grid, npairs), 256, 0, stream>>>(
+          pairs, table, (int)total, N, units, to_monarch);
+    else
+      permute_rows_kernel<U, UNITS, long><<<dim3(grid, npairs), 256, 0, stream>>>(
+          pairs, table, total, N, units, to_monarch);
   });
 }
 
