@@ -17,6 +17,8 @@ struct RowPairs {
   void* dst[3];
 };
 
+constexpr int kPermDepth = 4;
+
 // I: the index type, int when every unit index fits (a 32-bit division per
 // unit instead of a 64-bit one), else long.
 template <typename U, int UNITS, typename I>
@@ -26,18 +28,30 @@ __global__ void __launch_bounds__(256)
   const int units = UNITS > 0 ? UNITS : units_rt;
   const U* __restrict__ src = static_cast<const U*>(pairs.src[blockIdx.y]);
   U* __restrict__ dst = static_cast<U*>(pairs.dst[blockIdx.y]);
-  for (I idx = (I)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
-       idx += (I)gridDim.x * blockDim.x) {
-    const I row = idx / units;
-    const int c = (int)(idx - row * units);
-    const I g = row / N;
-    const int m = (int)(row - g * N);
-    const I n = __ldg(table + m);
-    const I mi = (g * N + m) * units + c, ni = (g * N + n) * units + c;
-    if (to_monarch)
-      dst[mi] = src[ni];
-    else
-      dst[ni] = src[mi];
+  // kPermDepth units per thread and pass, every load issued before the stores
+  const I stride = (I)gridDim.x * blockDim.x;
+  for (I base = (I)blockIdx.x * blockDim.x + threadIdx.x; base < total;
+       base += stride * kPermDepth) {
+    I from[kPermDepth], to[kPermDepth];
+    U val[kPermDepth];
+#pragma unroll
+    for (int r = 0; r < kPermDepth; ++r) {
+      const I idx = base + r * stride;
+      if (idx < total) {
+        const I row = idx / units;
+        const int c = (int)(idx - row * units);
+        const I g = row / N;
+        const int m = (int)(row - g * N);
+        const I n = __ldg(table + m);
+        const I mi = (g * N + m) * units + c, ni = (g * N + n) * units + c;
+        from[r] = to_monarch ? ni : mi;
+        to[r] = to_monarch ? mi : ni;
+        val[r] = src[from[r]];
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kPermDepth; ++r)
+      if (base + r * stride < total) dst[to[r]] = val[r];
   }
 }
 
@@ -49,10 +63,10 @@ cudaError_t launch(const RowPairs& pairs, int npairs, const int* table, long G, 
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const long want = (total + 255) / 256;
+  const long want = (total + 256L * kPermDepth - 1) / (256L * kPermDepth);
   const int grid = (int)(want < 16L * sms ? want : 16L * sms);
   return timed_launch("permute_rows", stream, launches, [&] {
-    if (total < (1L << 31) - 256L * grid)  // idx never overflows int
+    if (total < (1L << 31) - 256L * grid * kPermDepth)  // no index overflows int
       permute_rows_kernel<U, UNITS, int><<<dim3(grid, npairs), 256, 0, stream>>>(
           pairs, table, (int)total, N, units, to_monarch);
     else
