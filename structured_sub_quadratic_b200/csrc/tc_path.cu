@@ -1510,8 +1510,8 @@ __global__ void __launch_bounds__(320, 1)
 }
 
 // ---------------------------------------------------------------------------
-// Persistent R-update for column-group tiles NQ <= 64 (step one, and the
-// later steps with per-sub-item queries).  One CTA
+// Persistent R-update for column-group tiles NQ <= 96 (paired tiles: NQ <=
+// 64) (step one, and the later steps with per-sub-item queries).  One CTA
 // per SM walks a contiguous range of sub-items (g, p, k, q): one item (g, p, k)
 // is split into c2 sub-items, one per column group q.  Warp 0 loads (Qt0, and
 // K_q / V_q through a ring of slots), warp 1 issues the MMAs, and two
@@ -1544,7 +1544,9 @@ struct KR2Layout {
   static constexpr int kBox = NQ * 128;                    // one TMA box: NQ keys x 64 columns
   static constexpr int kBlk = kKeys * 128;                 // one 64-column block of K or V
   static constexpr int kKVBytes = 2 * (D / 64) * kBlk;     // K blocks, then V blocks
-  static constexpr int kKVSlots = PAIR ? 2 : 3;
+  // three ring slots when they fit beside Q and P, else two
+  static constexpr int kKVSlots =
+      PAIR ? 2 : (D / 64 * kRows * 128 + 3 * kKVBytes + 4 * kRows * 128 + 256 <= 227 * 1024 ? 3 : 2);
   // P (K-major, 64-key chunks of 128 rows): two chunks, so that once the
   // [Kt | Y] product has read P each warp finds two 4 KB staging buffers in
   // its own 32 rows for the epilogue's stores.
@@ -1554,7 +1556,7 @@ struct KR2Layout {
   static constexpr int kPOff = kKVOff + kKVSlots * kKVBytes;       // [2 wg]
   static constexpr int kBarOff = kPOff + 2 * kPBytes;
   static constexpr int kBytes = kBarOff + 32 * 8;
-  static_assert(NQ % 16 == 0 && NQ <= 64, "group tile");
+  static_assert(NQ % 16 == 0 && NQ <= (PAIR ? 64 : 96), "group tile");
   static_assert(kBytes <= 227 * 1024, "shared memory");
 };
 
@@ -3185,7 +3187,7 @@ cudaError_t launch_later_step(const bf16* q, const bf16* k, const bf16* v, bf16*
                       : launch_kl_two_pass<D>(q, kt, hs, lse, qt, pb, status, stream, launches);
   if (e != cudaSuccess) return e;
   if (small_r_fits(pb)) return launch_small_r(qt, k, v, kt, y, hs, pb, true, last, stream, launches);
-  if (kr_group_tile(pb) <= 64 && pb.b2 <= kRows) {
+  if (kr_group_tile(pb) <= 96 && pb.b2 <= kRows) {
     switch (kr_group_tile(pb)) {
 #define MONARCH_KR2_STEP(NQ)                                                                   \
   case NQ:                                                                                     \
@@ -3197,6 +3199,12 @@ cudaError_t launch_later_step(const bf16* q, const bf16* k, const bf16* v, bf16*
       MONARCH_KR2_STEP(32)
       MONARCH_KR2_STEP(48)
       MONARCH_KR2_STEP(64)
+#define MONARCH_KR2_WIDE(NQ)                                                                    \
+  case NQ:                                                                                      \
+    return launch_kr2<D, NQ, false>(qt, k, v, kt, y, hs, pb, status, stream, launches, true, last);
+      MONARCH_KR2_WIDE(80)
+      MONARCH_KR2_WIDE(96)
+#undef MONARCH_KR2_WIDE
 #undef MONARCH_KR2_STEP
       default: return cudaErrorInvalidValue;
     }
@@ -3206,8 +3214,9 @@ cudaError_t launch_later_step(const bf16* q, const bf16* k, const bf16* v, bf16*
 
 // Step one: aggregated queries under the uniform L, then the R-update: one
 // warp per group on the CUDA cores for groups of <= 8 keys over <= 32
-// positions, the paired-tile kernel for column groups of <= 64 keys over
-// <= 128 positions, the streaming kernel for wider groups or more positions.
+// positions, the paired-tile kernel for column groups of <= 96 keys over
+// <= 128 positions (two groups per tile when b2 <= 64 and the groups hold
+// <= 64 keys), the streaming kernel for wider groups or more positions.
 template <int D>
 cudaError_t launch_r_step1(const bf16* q, const bf16* k, const bf16* v, bf16* qt0, bf16* kt,
                            bf16* y, float* hs, const Problem& pb, int* status,
@@ -3234,7 +3243,7 @@ cudaError_t launch_r_step1(const bf16* q, const bf16* k, const bf16* v, bf16* qt
   if (small_r_fits(pb))
     return launch_small_r(qt0, k, v, kt, y, hs, pb, false, pb.T == 1, stream, launches);
   // column groups of <= 64 keys over <= 128 positions: the persistent kernel
-  if (kr_group_tile(pb) <= 64 && pb.b2 <= kRows) {
+  if (kr_group_tile(pb) <= 96 && pb.b2 <= kRows) {
     switch (kr_group_tile(pb)) {
 #define MONARCH_KR2_CASE(NQ)                                                               \
   case NQ:                                                                                 \
@@ -3245,6 +3254,11 @@ cudaError_t launch_r_step1(const bf16* q, const bf16* k, const bf16* v, bf16* qt
       MONARCH_KR2_CASE(32)
       MONARCH_KR2_CASE(48)
       MONARCH_KR2_CASE(64)
+#define MONARCH_KR2_WIDE(NQ) \
+  case NQ: return launch_kr2<D, NQ, false>(qt0, k, v, kt, y, hs, pb, status, stream, launches);
+      MONARCH_KR2_WIDE(80)
+      MONARCH_KR2_WIDE(96)
+#undef MONARCH_KR2_WIDE
 #undef MONARCH_KR2_CASE
       default: return cudaErrorInvalidValue;
     }

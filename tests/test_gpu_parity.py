@@ -92,6 +92,10 @@ EDGE = [
     (2, 1, 17, 96, 128, 2, 1, 3),    # 32-key groups, two steps (Kt-only first R-update)
     (1, 1, 9, 80, 128, 1, 1, 5),     # 16-key groups
     (1, 1, 400, 72, 128, 1, 1, 2),   # 800 sub-items over the SMs: several tiles per warpgroup
+    # unpaired R tiles of 65-96 keys (two K|V slots at d = 128)
+    (1, 2, 20, 90, 64, 2, 1, 1),     # 90-key groups in 96-key tiles, two steps
+    (1, 1, 16, 75, 128, 1, 1, 1),    # 75-key groups in 80-key tiles
+    (2, 1, 24, 96, 128, 2, 1, 1),    # 96-key groups, full tiles, two steps
 ]
 
 
