@@ -21,6 +21,7 @@
 //                O = L Y
 #include "small_dim.cuh"
 
+#include <cooperative_groups.h>
 #include <math.h>
 
 #include "launch.cuh"
@@ -112,6 +113,77 @@ __global__ void __launch_bounds__(kWarps * 32)
 #pragma unroll
   for (int e = 0; e < E; ++e) acc[e] /= n;
   store_row<E>(qt0 + (long)unit * D + lane * E, acc);
+}
+
+// Aggregation of a few long row groups (fewer (g, p, i) units than a
+// quarter of the SMs, each of >= kSplitMinRows rows): a cluster of kSplit
+// CTAs per unit, CTA r summing the r-th slice of the group's rows (16-byte
+// column chunks x row lanes, warp shuffles, then the warps in shared
+// memory); CTA 0 adds the kSplit slice sums in rank order through
+// distributed shared memory, so the result does not depend on scheduling.
+constexpr int kSplit = 8;
+constexpr int kSplitMinRows = 256;
+
+template <int D>
+__global__ void __launch_bounds__(256)
+    split_init_kernel(const bf16* __restrict__ q, bf16* __restrict__ qt0, Problem pb) {
+  namespace cg = cooperative_groups;
+  constexpr int CH = D / 8;     // 16-byte chunks per row
+  constexpr int RL = 256 / CH;  // row lanes
+  __shared__ float red[8][D];
+  __shared__ float part[D];     // this CTA's slice sum, read by CTA 0 of the cluster
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
+  const int unit = (int)blockIdx.x / kSplit;  // (g c1 + p) b2 + i
+  const int i = unit % pb.b2;
+  const int gp = unit / pb.b2;
+  const int p = gp % pb.c1;
+  const int g = gp / pb.c1;
+  const int l0 = group_start(pb.b1, pb.c1, p), l1 = group_start(pb.b1, pb.c1, p + 1);
+  const int n = l1 - l0;
+  const int s0 = l0 + (int)((long)n * rank / kSplit), s1 = l0 + (int)((long)n * (rank + 1) / kSplit);
+  pdl_wait();  // qt0 may still be read by the previous call's R-update
+  pdl_launch_dependents();
+  const int ch = threadIdx.x % CH, rl = threadIdx.x / CH, lane = threadIdx.x & 31;
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  const uint4* base = reinterpret_cast<const uint4*>(q + token_row(pb, g, 0, i) * D) + ch;
+  const long row_stride = (pb.tr ? (long)D : (long)pb.b2 * D) / 8;  // rows l apart, in uint4
+#pragma unroll 4
+  for (int l = s0 + rl; l < s1; l += RL) {
+    const uint4 u = __ldg(base + l * row_stride);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      acc[2 * e] += __uint_as_float(w[e] << 16);
+      acc[2 * e + 1] += __uint_as_float(w[e] & 0xffff0000u);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+#pragma unroll
+    for (int o = CH; o < 32; o <<= 1) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
+  }
+  if (lane < CH) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) red[threadIdx.x >> 5][ch * 8 + e] = acc[e];
+  }
+  __syncthreads();
+  if (threadIdx.x < D) {
+    float sum = 0.f;
+#pragma unroll
+    for (int w8 = 0; w8 < 8; ++w8) sum += red[w8][threadIdx.x];
+    part[threadIdx.x] = sum;
+  }
+  cluster.sync();  // every slice sum is in its CTA's shared memory
+  if (rank == 0 && threadIdx.x < D) {
+    float sum = 0.f;
+#pragma unroll
+    for (int r = 0; r < kSplit; ++r) sum += cluster.map_shared_rank(part, r)[threadIdx.x];
+    qt0[(long)unit * D + threadIdx.x] = __float2bfloat16_rn(sum / (float)n);
+  }
+  cluster.sync();  // CTA 0 has read every slice sum before any CTA exits
 }
 
 // Sub-item (g, p, k, q) of the R-update, in the tensor-core kernels' order;
@@ -283,9 +355,17 @@ static bool small_indices_fit(const Problem& pb) {
   return (long)pb.G * pb.b2 * pb.c1 * pb.b1 * pb.c2 < (1L << 31);
 }
 
+// A few long row groups: the clustered aggregation (every group of
+// >= kSplitMinRows rows, fewer units than a quarter of the SMs).
+static bool split_init_fits(const Problem& pb) {
+  return (pb.d == 64 || pb.d == 128) && !is_padded(pb) && pb.b1 / pb.c1 >= kSplitMinRows &&
+         (long)pb.G * pb.c1 * pb.b2 * 4 < num_sms() && small_indices_fit(pb);
+}
+
 bool small_init_fits(const Problem& pb) {
-  return (pb.d == 64 || pb.d == 128) && !is_padded(pb) &&
-         (pb.b1 + pb.c1 - 1) / pb.c1 <= kMaxRows && small_indices_fit(pb);
+  return ((pb.d == 64 || pb.d == 128) && !is_padded(pb) &&
+          (pb.b1 + pb.c1 - 1) / pb.c1 <= kMaxRows && small_indices_fit(pb)) ||
+         split_init_fits(pb);
 }
 
 bool small_r_fits(const Problem& pb) {
@@ -301,6 +381,26 @@ bool small_out_fits(const Problem& pb) {
 cudaError_t launch_small_init(const bf16* q, bf16* qt0, const Problem& pb, cudaStream_t stream,
                               int* launches) {
   if (!small_init_fits(pb)) return cudaErrorInvalidValue;
+  if (split_init_fits(pb)) {
+    const unsigned units = (unsigned)((long)pb.G * pb.c1 * pb.b2);
+    return timed_launch("cc_init_qt", stream, launches, [&] {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(units * kSplit);
+      cfg.blockDim = dim3(256);
+      cfg.stream = stream;
+      cudaLaunchAttribute attr[2];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = kSplit;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[1].val.programmaticStreamSerializationAllowed = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 2;
+      return pb.d == 128 ? cudaLaunchKernelEx(&cfg, split_init_kernel<128>, q, qt0, pb)
+                         : cudaLaunchKernelEx(&cfg, split_init_kernel<64>, q, qt0, pb);
+    });
+  }
   const unsigned grid = blocks_for((long)pb.G * pb.c1 * pb.b2);
   return timed_launch("cc_init_qt", stream, launches, [&] {
     return pb.d == 128 ? launch_pdl(small_init_kernel<128>, dim3(grid), dim3(kWarps * 32), 0,

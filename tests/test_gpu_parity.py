@@ -365,6 +365,8 @@ SMALL_GROUPS = [
     (1, 2, 5, 4, 128, 2, 1, 1, {"cc_init_qt", "cc_r_update", "cc_l_output"}),  # two steps
     (1, 1, 20, 32, 64, 3, 2, 4, {"cc_init_qt", "cc_r_update"}),  # 8-key groups, 32 positions
     (1, 1, 7, 5, 128, 1, 7, 1, {"cc_init_qt", "cc_r_update", "cc_l_output"}),  # 1-row groups
+    (1, 2, 600, 3, 128, 1, 1, 1, {"cc_init_qt", "cc_r_update"}),  # 6 long row groups: clusters
+    (2, 1, 520, 4, 64, 2, 2, 1, {"cc_init_qt", "cc_r_update"}),   # the same, d = 64, tiled, T = 2
 ]
 
 
