@@ -118,9 +118,9 @@ MONARCH_API int monarch_attn_fwd_host(int dtype, const void* q_host, const void*
  * Arguments, layout and result are those of monarch_attn_fwd, and it runs
  * the same kernels, so the output is bit-identical to monarch_attn_fwd's on
  * the same inputs.  Only the shapes those kernels take run here (d = 64 or
- * 128, T >= 1, b2 <= 128 and column groups of <= 128 keys; small untiled
- * heads with T >= 2 need no scratch at all); any other shape returns
- * MONARCH_ERR_UNSUPPORTED.  The caller still passes q, k, v and out.
+ * 128 and T >= 1; small untiled heads with T >= 2 need no scratch at all);
+ * any other shape returns MONARCH_ERR_UNSUPPORTED.  The caller still passes
+ * q, k, v and out.
  *
  * Scratch: one static device array of 64 MiB (67108864 bytes) on every
  * device that loads this library, held until the process exits.  A shape
