@@ -9,7 +9,7 @@ Each case below drives one kernel path through its masks:
   * a post-padded 480p-like head: paired tcgen05 R tiles;
   * 80-position chunks in two column groups, 45 pad tokens first (chunk 0's
     first group holds no real key): unpaired tcgen05 R tiles;
-  * 100-key column groups with a whole pad chunk: the per-item R kernel;
+  * 100-key column groups with a whole pad chunk: the streaming R kernel;
   * 400 keys per L row whose first 68 are masked: the online output kernel
     starting on a key tile with no real key;
   * T = 2 (later steps on the SIMT kernels), T = 0, odd d, one real token.
@@ -38,7 +38,7 @@ CASES = [
     (1, 2, 400 - 68, 100, 4, True, 64, 1, 1, 4, torch.bfloat16),
     (1, 2, 20 * 24 - 30, 20, 24, True, 64, 2, 2, 2, torch.bfloat16),
     (1, 2, 20 * 24 - 30, 20, 24, False, 64, 2, 2, 2, torch.float32),
-    # later steps through the two-pass L-update and the per-item / streaming R-updates
+    # later steps through the two-pass L-update and the paired-tile / streaming R-updates
     (1, 2, 140 * 80 - 100, 140, 80, True, 64, 2, 1, 2, torch.bfloat16),
     (1, 1, 200 * 8 - 11, 200, 8, True, 64, 2, 1, 1, torch.bfloat16),
     (1, 1, 52 * 90 - 40, 52, 90, True, 128, 2, 1, 1, torch.bfloat16),

@@ -274,7 +274,7 @@ LATER_STEPS = [
     (1, 1, 200, 8, 64, 2, 1, 1, "iid"),      # 200 keys, 200-row groups (two row tiles)
     (1, 1, 260, 40, 128, 3, 2, 2, "iid"),    # 520 keys, 130-row groups, paired R tiles
     (1, 1, 140, 80, 64, 2, 1, 2, "iid"),     # 280 keys, unpaired R tiles
-    # R-update of the later steps in the per-item and streaming kernels
+    # R-update of the later steps in the paired-tile (<= 96 keys) and streaming kernels
     (1, 2, 64, 128, 64, 2, 1, 1, "iid"),     # 128-key groups (the 16K sweep's shape, 64 chunks)
     (1, 2, 52, 90, 128, 2, 1, 1, "iid"),     # 90-key groups (the (w,fh) blocks of the 480p latent)
     (1, 1, 30, 156, 128, 3, 2, 2, "iid"),    # 78-key groups over two position tiles, three steps
